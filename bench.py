@@ -1,0 +1,385 @@
+"""Benchmark of the paged-KV decode step on B200.
+
+One step = the whole hot path on one batch: copy-on-write block copies (when
+the workload has them), slot of every appended token, scatter of the new K/V
+rows, decode attention (plus the log-sum-exp reduce when a context spans
+several partitions). The step is captured once in a CUDA graph (the launch
+path of a serving decode loop) and replayed; every replay is bracketed by
+timing events recorded inside the graph. Before every timed step a 512 MiB
+buffer is written to evict the 126 MB L2, so the KV bytes come from HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 1..5] [--impl ours|reference]
+
+Under torchrun each rank runs its own independently seeded batch of the same
+shape (sequences are independent; there is no exchange step), and rank 0
+prints one JSON line with the slowest rank's times.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = ("paged decode attention KV GB/s (% of B200 HBM peak) and decode tokens/s, 1 GPU")
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+FLUSH_BYTES = 512 << 20
+
+
+def hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "pagedattention_paged_kv_decode_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was
+    taken on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "decode_dram_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    ent = rec.get(workload)
+    if not ent or ent.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples (200 ms) while the timed region runs."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: str):
+        self.gpu = gpu_index
+        self.rows = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        rows = [r for t, r in self.rows if t0 - 0.25 <= t <= t1 + 0.25] or [r for _, r in self.rows]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        mx = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if len(r) > 6 + i and r[6 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import pagedattention_paged_kv_decode_b200 as pk
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    w = W.named(args.workload, seed=W.rank_seed(1000 + args.workload, rank))
+    dw = W.to_device(w, dev, encode=pk.load_cache)
+    S = w.num_seqs
+    bound = w.max_blocks_per_seq * w.block_size  # host-side bound: table capacity, no sync
+    cfg = pk.choose_config(dw.key_cache, S, bound)
+    parts = -(-bound // cfg["partition_size"])
+    launches_per_step = 3 + (1 if w.cow_pairs.size else 0) + (1 if parts > 1 else 0)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    stream = torch.cuda.Stream(dev)
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
+
+    def step():
+        ev[0].record()
+        if w.cow_pairs.size:
+            pk.copy_blocks(dw.key_cache, dw.value_cache, dw.cow_pairs)
+        pk.slot_mapping(dw.block_tables, dw.context_lens, dw.key_cache, out=dw.slots)
+        pk.kv_cache_write(dw.new_key, dw.new_value, dw.key_cache, dw.value_cache, dw.slots,
+                          w.k_scale, w.v_scale)
+        ev[1].record()
+        pk.paged_attention_decode(dw.out, dw.query, dw.key_cache, dw.value_cache,
+                                  dw.block_tables, dw.context_lens, w.scale, w.k_scale,
+                                  w.v_scale, max_context_len=bound)
+        ev[2].record()
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):          # un-captured warm-up: sizes the split workspace, sets attributes
+            step()
+        stream.synchronize()
+        assert pk.check_status(stream) == 0
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            step()
+        stream.synchronize()
+
+        def timed_step():
+            flush.fill_(1)
+            graph.replay()
+            stream.synchronize()
+            return ev[0].elapsed_time(ev[2]), ev[1].elapsed_time(ev[2])
+
+        for _ in range(max(3, args.warmup)):
+            timed_step()
+
+        visible = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
+        sampler = ClockSampler(visible[local_rank] if len(visible) > local_rank and visible[local_rank]
+                               else str(local_rank))
+        sampler.start()
+        time.sleep(0.3)
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0 = time.time()
+        step_ms, dec_ms = [], []
+        for _ in range(args.steps):
+            a, b = timed_step()
+            step_ms.append(a)
+            dec_ms.append(b)
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        t1 = time.time()
+        sampler.stop()
+        assert pk.check_status(stream) == 0
+
+        # ------------------------------------------------ end to end (host buffers)
+        host_in = {k: getattr(dw, k).cpu().pin_memory()
+                   for k in ("query", "new_key", "new_value", "block_tables", "context_lens", "cow_pairs")}
+        host_out = torch.empty(dw.out.shape, dtype=dw.out.dtype).pin_memory()
+        e2e_start = torch.cuda.Event(enable_timing=True)
+        e2e_end = torch.cuda.Event(enable_timing=True)
+        h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+        d2h = host_out.numel() * host_out.element_size()
+        e2e_ms = []
+        for i in range(max(3, args.warmup) + args.steps):
+            flush.fill_(1)
+            e2e_start.record()
+            for k, t in host_in.items():
+                getattr(dw, k).copy_(t, non_blocking=True)
+            graph.replay()
+            host_out.copy_(dw.out, non_blocking=True)
+            e2e_end.record()
+            stream.synchronize()
+            if i >= max(3, args.warmup):
+                e2e_ms.append(e2e_start.elapsed_time(e2e_end))
+
+    stats = torch.tensor([statistics.mean(step_ms), statistics.mean(dec_ms), statistics.mean(e2e_ms)],
+                         dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(stats, op=dist.ReduceOp.MAX)
+    step_t, dec_t, e2e_t = (float(x) for x in stats.cpu())
+    clocks = sampler.summary(t0, t1)
+    del graph
+    if dist:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    kv = w.kv_bytes()
+    peak, peak_kind = hbm_peak()
+    dec_bytes = w.decode_bytes()
+    achieved = dec_bytes / (dec_t * 1e-3) / 1e9
+    value = world * kv / (step_t * 1e-3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(step_t, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "kv_dtype": w.kv_dtype,
+        "data": "synthetic (seeded numpy PCG64; no dataset)",
+        "config": {
+            "workload": w.name, "num_seqs": S, "num_heads": w.num_heads,
+            "head_size": w.head_size, "block_size": w.block_size, "kv_dtype": w.kv_dtype,
+            "num_blocks": w.num_blocks, "mean_context": round(float(w.context_lens.mean()), 1),
+            "max_context": w.max_context_len, "kv_bytes_per_step": kv,
+            "launch": cfg, "parallelism": f"replicas x{world} (independent batches, no collective)",
+            "l2": "512 MiB buffer written before every timed step (L2 is 126 MB)",
+            "step": "CUDA graph: " + ("copy_blocks, " if w.cow_pairs.size else "")
+                    + "slot_mapping, kv_cache_write, paged_attention_decode"
+                    + (" (+lse reduce)" if parts > 1 else ""),
+        },
+        "tokens_per_s": round(world * S / (step_t * 1e-3), 1),
+        "hbm_pct_of_nominal_8tbs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
+        "hbm_pct_of_measured": round(100 * value / world / peak, 2),
+        "decode_ms": round(dec_t, 5),
+        "decode_kv_gbs": round(kv / (dec_t * 1e-3) / 1e9, 2),
+        "roofline": {
+            "bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} copy bandwidth",
+            "traffic": recorded_traffic(w.name),
+            "kernel": "paged_decode_kernel" + (" + lse_reduce_kernel" if parts > 1 else ""),
+            "algorithmic_bytes_per_launch": dec_bytes,
+        },
+        "e2e": {"value": round(world * kv / (e2e_t * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "ms_per_step": round(e2e_t, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "path": "pinned host inputs -> device copies -> graph replay -> output to pinned host"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------- CPU oracle
+
+def cpu_baseline(w, seconds: float):
+    """The oracle, single-threaded, on this host: whole decode steps of one
+    sequence at a time (all heads) over a bounded, seeded sample of the
+    workload's sequences. Building the host pools (and, for E4M3, encoding
+    the sampled sequences' blocks) happens outside the timed region. Returns
+    the same GB/s metric."""
+    import oracle
+    order = np.random.default_rng(0).permutation(w.num_seqs)
+    pk_, pv_ = w.pool_host()
+    if w.kv_dtype == "e4m3":
+        kc = np.zeros(pk_.shape, np.uint8)
+        vc = np.zeros(pv_.shape, np.uint8)
+        encoded = np.zeros(w.num_blocks, bool)
+    else:
+        kc, vc = pk_, pv_
+    ctx = w.context_lens
+    done_bytes, elapsed, n = 0, 0.0, 0
+    while elapsed < seconds and n < 100000:
+        s = int(order[n % w.num_seqs])
+        if w.kv_dtype == "e4m3":
+            bt = w.block_tables[s]
+            blocks = np.array([b for b in bt[bt >= 0] if not encoded[b]], np.int64)
+            if blocks.size:
+                slots = (blocks[:, None] * w.block_size + np.arange(w.block_size)).reshape(-1).astype(np.int32)
+                oracle.kv_cache_write(pk_[blocks].reshape(-1, w.num_heads, w.head_size),
+                                      pv_[blocks].reshape(-1, w.num_heads, w.head_size), kc, vc,
+                                      slots, w.k_scale, w.v_scale)
+                encoded[blocks] = True
+        t = time.perf_counter()
+        if w.cow_pairs.size:
+            oracle.copy_blocks(kc, vc, w.cow_pairs[s:s + 1])
+        slot = oracle.slot_mapping(w.block_tables[s:s + 1], ctx[s:s + 1], w.block_size)
+        oracle.kv_cache_write(w.new_key[s:s + 1], w.new_value[s:s + 1], kc, vc, slot,
+                              w.k_scale, w.v_scale)
+        oracle.paged_attention(w.query[s:s + 1], kc, vc, w.block_tables[s:s + 1], ctx[s:s + 1],
+                               w.scale, w.k_scale, w.v_scale)
+        elapsed += time.perf_counter() - t
+        done_bytes += int(ctx[s]) * w.num_heads * w.head_size * w.elem_bytes * 2
+        n += 1
+    return {"value": round(done_bytes / elapsed / 1e9, 4), "unit": "GB/s", "cores": 1,
+            "kind": "oracle",
+            "sample": f"{n} sequences (all {w.num_heads} heads each) of {w.name}, one decode step "
+                      f"each (copy-on-write, slot, cache write, attention): {elapsed:.1f} s, "
+                      f"single-thread fp64"}
+
+
+def run_reference(args, rank, world):
+    """The CPU oracle as the reference arm: rank 0 only, same metric and unit."""
+    if rank != 0:
+        return
+    w = W.named(args.workload)
+    per_step = max(0.5, args.cpu_seconds / max(1, args.steps + args.warmup))
+    vals = []
+    for i in range(args.warmup + args.steps):
+        r = cpu_baseline(w, per_step)
+        if i >= args.warmup:
+            vals.append(r["value"])
+    v = statistics.mean(vals)
+    kv = w.kv_bytes()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(kv / (v * 1e9) * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded numpy PCG64; no dataset)",
+        "config": {"workload": w.name, "num_seqs": w.num_seqs, "num_heads": w.num_heads,
+                   "head_size": w.head_size, "block_size": w.block_size, "kv_dtype": w.kv_dtype},
+        "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"each step: {per_step:.1f} s of whole-sequence oracle steps"},
+        "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"note: --gpus {args.gpus} but WORLD_SIZE {world}; using WORLD_SIZE", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,200 @@
+/*
+ * pagedkv.h -- C ABI of libpagedkv.so: paged-KV decode attention for NVIDIA
+ * B200 (sm_100a), with the cache-write scatter, the slot derivation and the
+ * block copy that surround it.
+ *
+ * Sources (each page is cited by its title and section):
+ *   [P1] "vLLM-v0.17.1技术解析：PagedAttention内存管理与显存优化技巧",
+ *        §2.2 PagedAttention的创新设计 (block table, physical block pool),
+ *        §3.2 高效CUDA内核优化 (fused kernels, coalesced access), §3.3 量化支持 (FP8).
+ *   [P2] "在A10G上榨干LLaMA-7B：vLLM与PagedAttention实战",
+ *        §2.1 从逻辑块到物理块 (logical/physical blocks, growth on append),
+ *        §2.2 内存共享与写时复制 (prefix sharing, copy-on-write).
+ *   [P3] KV-cache / PagedAttention article at l189.com/news/180929,
+ *        §2.1 块状存储结构 (16-token blocks, per-block byte size),
+ *        §2.2 槽位映射机制 (slot mapping: one int32 per token),
+ *        §4 (FP8 KV cache, block size 32 for long texts).
+ *
+ * Conventions shared by every call
+ *   - All data pointers are DEVICE pointers owned by the caller, on the
+ *     current CUDA device. The library never frees or retains them.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Every call
+ *     only enqueues work on that stream and returns; none synchronises,
+ *     except pa_check_status.
+ *   - Return value: PA_OK (0) or a negative PA_ERR_* code. On an error no
+ *     kernel has been launched, and pa_last_error() returns a message
+ *     (thread-local, valid until the next call on the same thread).
+ *   - Index contents that only the device can see (slots, block ids,
+ *     context lengths, copy pairs) are bounds-checked in the kernels: an
+ *     offending item is skipped or clamped, never dereferenced, and a bit is
+ *     set in a per-device error word that pa_check_status reads and clears.
+ *   - KV cache layout (both K and V): contiguous
+ *     [num_blocks][block_size][num_heads][head_size] of fp16 or of E4M3 codes
+ *     ([P1] §2.2 physical block pool; [P3] §2.1 block of block_size tokens x
+ *     num_heads x head_size). Logical token t of a sequence lives in physical
+ *     block block_tables[s][t / block_size], row t % block_size.
+ *   - Supported shapes: head_size 64 or 128; block_size 16 or 32;
+ *     num_heads >= 1; num_blocks * block_size < 2^31.
+ *   - Query, output, new K/V rows and caches must be 16-byte aligned.
+ */
+#ifndef PAGEDKV_H
+#define PAGEDKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PA_OK 0
+#define PA_ERR_INVALID (-1)   /* null pointer, bad size, shape or alignment */
+#define PA_ERR_DTYPE (-2)     /* unsupported cache dtype */
+#define PA_ERR_OVERFLOW (-3)  /* num_blocks * block_size >= 2^31 */
+#define PA_ERR_CUDA (-4)      /* a CUDA runtime or driver call failed */
+#define PA_ERR_WORKSPACE (-5) /* caller workspace missing, too small or misaligned */
+
+/* Bits of the device error word (pa_check_status). */
+#define PA_DEV_BAD_SLOT 1u        /* slot >= num_blocks*block_size: token skipped */
+#define PA_DEV_BAD_BLOCK 2u       /* table entry outside [0, num_blocks): rows read as zeros */
+#define PA_DEV_CTX_OVER_TABLE 4u  /* context_len > max_blocks_per_seq*block_size: clamped */
+#define PA_DEV_CTX_OVER_BOUND 8u  /* context_len > max_context_len given to the call: clamped */
+#define PA_DEV_BAD_PAIR 16u       /* copy pair index outside [0, num_blocks): pair skipped */
+#define PA_DEV_WAIT_TIMEOUT 32u   /* an on-chip pipeline wait ran out (never expected) */
+
+/* KV cache element type: fp16, or OCP FP8 E4M3 ("fn" variant: no infinities,
+ * max 448) with one fp32 scale per cache tensor ([P1] §3.3, [P3] §4). */
+#define PA_F16 0
+#define PA_E4M3 1
+
+typedef struct {
+    int32_t num_blocks;   /* physical blocks in the pool */
+    int32_t block_size;   /* tokens per block: 16 or 32 */
+    int32_t num_heads;    /* KV heads (= query heads) */
+    int32_t head_size;    /* 64 or 128 */
+    int32_t dtype;        /* PA_F16 or PA_E4M3 */
+} pa_cache_desc;
+
+/* Launch shape of the decode. Any field 0 = library choice.
+ *   partition_size: tokens per split-context partition, a multiple of
+ *       block_size. Sequences longer than one partition are computed as
+ *       partial results plus a log-sum-exp reduction.
+ *   heads_per_cta:  1, 2, 4 or 8 and a divisor of num_heads.
+ *   warps_per_head: 1, 2 or 4 warps sharing one head's tokens in a CTA.
+ *   stages:         2..8 K/V tiles in flight per CTA. */
+typedef struct {
+    int32_t partition_size;
+    int32_t heads_per_cta;
+    int32_t warps_per_head;
+    int32_t stages;
+} pa_decode_config;
+
+/* Library version, e.g. 100 for 0.1.0. */
+int pa_version(void);
+
+/* Message for the last nonzero status returned on this thread ("" if none). */
+const char *pa_last_error(void);
+
+/* Synchronise `stream`, then read and clear the device error word of the
+ * current device into *code (0 = no device-side error since the last read).
+ * Returns PA_OK or PA_ERR_CUDA. */
+int pa_check_status(void *stream, uint32_t *code);
+
+/* ---------------------------------------------------------------- a1
+ * Slot of the token each sequence appends in a decode step ([P3] §2.2 slot
+ * mapping; [P2] §2.1 growth on append). With L = context_lens[s] (which
+ * includes the appended token) and pos = L-1:
+ *     slot_mapping[s] = block_tables[s][pos / block_size] * block_size
+ *                       + pos % block_size
+ * and -1 when L <= 0. block_tables: int32 [num_seqs][max_blocks_per_seq].
+ * Device checks: L beyond the table row sets PA_DEV_CTX_OVER_TABLE, a block
+ * id outside the pool sets PA_DEV_BAD_BLOCK; both give slot -1. */
+int pa_slot_mapping(int32_t *slot_mapping, const int32_t *block_tables,
+                    int max_blocks_per_seq, const int32_t *context_lens,
+                    int num_seqs, pa_cache_desc cache, void *stream);
+
+/* ---------------------------------------------------------------- a2
+ * Store each new token's K and V rows (all heads) into the cache slot that
+ * slot_mapping gives ([P2] §2.1: the new token's KV goes into the mapped
+ * block; [P3] §2.2 slot mapping). key/value: fp16 [n_tokens][num_heads]
+ * [head_size], row i at key + i*key_stride elements (stride a multiple of 8).
+ * slot s -> block s / block_size, row s % block_size. Negative slots are
+ * padding and are skipped. fp16 caches receive the bits unchanged; E4M3
+ * caches receive e4m3_rn_satfinite(fp32(x) / scale) with an IEEE fp32 divide
+ * (k_scale for K, v_scale for V; both ignored for fp16). Slots beyond the
+ * pool set PA_DEV_BAD_SLOT and are skipped. Two tokens with the same slot in
+ * one call: undefined which one lands. */
+int pa_kv_cache_write(const void *key, const void *value, int64_t key_stride,
+                      int64_t value_stride, void *key_cache, void *value_cache,
+                      pa_cache_desc cache, const int32_t *slot_mapping,
+                      int n_tokens, float k_scale, float v_scale, void *stream);
+
+/* ---------------------------------------------------------------- a3
+ * Copy-on-write block copy ([P2] §2.2): for each pair (src, dst) of
+ * src_dst_pairs (int32 [n_pairs][2]), physical block dst of both caches
+ * becomes a copy of block src (block_size*num_heads*head_size elements).
+ * Pairs run concurrently: a dst that is also some pair's src, or that
+ * appears twice, is undefined. Indices outside the pool set PA_DEV_BAD_PAIR
+ * and the pair is skipped. */
+int pa_copy_blocks(void *key_cache, void *value_cache, pa_cache_desc cache,
+                   const int32_t *src_dst_pairs, int n_pairs, void *stream);
+
+/* ---------------------------------------------------------------- a4..a9
+ * Decode attention of one query token per sequence over its cached K/V,
+ * read through its block table ([P1] §2.2; [P2] §2.1). For each sequence s
+ * and head h, with L = context_lens[s] and token t in physical block
+ * block_tables[s][t / block_size], row t % block_size:
+ *     z_t = scale * k_scale * sum_d q[s,h,d] * K_t[h,d]
+ *     out[s,h,:] = v_scale * sum_t softmax(z)_t * V_t[h,:]       (t < L)
+ * (k_scale, v_scale only for E4M3 caches, which hold K/k_scale, V/v_scale).
+ * L = 0 gives zeros. query, out: fp16 [num_seqs][num_heads][head_size].
+ * max_context_len: a host-known upper bound on every context length (e.g.
+ * max_blocks_per_seq*block_size); it sizes the split-context grid. Contexts
+ * above it or above the table row are clamped and flagged.
+ * Sequences longer than the partition size are split: each partition writes
+ * a normalised partial output and its log-sum-exp, and a second kernel
+ * combines them. The workspace for those partials is owned by the library:
+ * one buffer per (device, stream), grown with cudaMallocAsync on `stream`
+ * and never shrunk. It is not allocated when no sequence can span more than
+ * one partition. Issue a first call with the largest shapes before
+ * capturing a CUDA graph so that capture does not need to grow it. */
+int pa_paged_attention_decode(void *out, const void *query,
+                              const void *key_cache, const void *value_cache,
+                              pa_cache_desc cache, const int32_t *block_tables,
+                              int max_blocks_per_seq, const int32_t *context_lens,
+                              int num_seqs, int max_context_len, float scale,
+                              float k_scale, float v_scale, void *stream);
+
+/* Fill *cfg with the launch shape the library would use (fields given as
+ * nonzero are kept and validated). Returns PA_OK or PA_ERR_INVALID. */
+int pa_decode_choose_config(pa_cache_desc cache, int num_seqs, int max_context_len,
+                            pa_decode_config *cfg);
+
+/* Bytes of workspace a pa_paged_attention_decode_ws call with this shape
+ * and config needs (0 when no split is possible). cfg may be NULL (library
+ * choice). Layout, when nonzero: float lse[num_seqs][num_heads][P] (base-2
+ * log-sum-exp of each partition's logits, in units of z*log2(e)), then at
+ * the next 256-byte boundary float o[num_seqs][num_heads][P][head_size]
+ * (each partition's softmax-normalised output, before v_scale), with
+ * P = ceil(max_context_len / partition_size). Entries of partitions that a
+ * sequence does not have are left untouched. */
+size_t pa_decode_workspace_size(pa_cache_desc cache, int num_seqs, int max_context_len,
+                                const pa_decode_config *cfg);
+
+/* pa_paged_attention_decode with an explicit launch shape (cfg may be NULL)
+ * and a caller-owned workspace of at least pa_decode_workspace_size bytes,
+ * 256-byte aligned (may be NULL when that size is 0). Allocates nothing. */
+int pa_paged_attention_decode_ws(void *out, const void *query,
+                                 const void *key_cache, const void *value_cache,
+                                 pa_cache_desc cache, const int32_t *block_tables,
+                                 int max_blocks_per_seq, const int32_t *context_lens,
+                                 int num_seqs, int max_context_len, float scale,
+                                 float k_scale, float v_scale,
+                                 const pa_decode_config *cfg, void *workspace,
+                                 size_t workspace_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H */

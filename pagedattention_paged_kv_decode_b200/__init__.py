@@ -1,0 +1,21 @@
+"""Paged-KV decode attention for NVIDIA B200 (sm_100a).
+
+The calls below marshal torch tensors into the C ABI of ``libpagedkv.so``
+(``include/pagedkv.h``); every step runs in that library's CUDA kernels.
+Importing this package does not touch the GPU; the first call loads the
+library and fails loudly if it has not been built.
+"""
+from .capi import PagedKVError  # noqa: F401
+from .ops import (  # noqa: F401
+    cache_desc,
+    check_status,
+    choose_config,
+    copy_blocks,
+    decode_step,
+    decode_workspace_size,
+    kv_cache_write,
+    load_cache,
+    paged_attention_decode,
+    slot_mapping,
+    version,
+)

@@ -1,0 +1,532 @@
+// pa_api.cu -- the C ABI of libpagedkv.so (declared in include/pagedkv.h):
+// argument validation, launch-shape choice, TMA descriptors, the split
+// workspace and kernel launches. Every compute step runs in the kernels of
+// pa_decode.cuh and pa_cache_ops.cuh; nothing here touches KV data.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "pa_cache_ops.cuh"
+#include "pa_decode.cuh"
+#include "pagedkv.h"
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+int fail(int code, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int ok() {
+    g_msg[0] = '\0';
+    return PA_OK;
+}
+
+int cuda_fail(cudaError_t e, const char *what) {
+    return fail(PA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_cache(const pa_cache_desc &c) {
+    if (c.dtype != PA_F16 && c.dtype != PA_E4M3)
+        return fail(PA_ERR_DTYPE, "cache dtype %d is neither PA_F16 nor PA_E4M3", c.dtype);
+    if (c.num_blocks < 1 || c.num_heads < 1)
+        return fail(PA_ERR_INVALID, "num_blocks (%d) and num_heads (%d) must be >= 1",
+                    c.num_blocks, c.num_heads);
+    if (c.block_size != 16 && c.block_size != 32)
+        return fail(PA_ERR_INVALID, "block_size %d: supported are 16 and 32", c.block_size);
+    if (c.head_size != 64 && c.head_size != 128)
+        return fail(PA_ERR_INVALID, "head_size %d: supported are 64 and 128", c.head_size);
+    if ((int64_t)c.num_blocks * c.block_size >= (int64_t(1) << 31))
+        return fail(PA_ERR_OVERFLOW, "num_blocks * block_size = %lld does not fit int32 slots",
+                    (long long)c.num_blocks * c.block_size);
+    return PA_OK;
+}
+
+int elem_bytes(const pa_cache_desc &c) { return c.dtype == PA_F16 ? 2 : 1; }
+
+// ------------------------------------------------------------ TMA maps
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+struct MapKey {
+    const void *ptr;
+    int nb, bs, nh, hd, dtype, g;
+    bool operator==(const MapKey &o) const {
+        return ptr == o.ptr && nb == o.nb && bs == o.bs && nh == o.nh && hd == o.hd &&
+               dtype == o.dtype && g == o.g;
+    }
+};
+
+std::mutex g_map_mu;
+std::vector<std::pair<MapKey, CUtensorMap>> g_maps;  // small FIFO cache
+
+// 4-D view of a cache, innermost first: {head_size, num_heads, block_size,
+// num_blocks}; box {head_size, G, block_size, 1} = one physical block's rows
+// for G heads. Zero fill outside the pool.
+int cache_tensor_map(const void *cache, const pa_cache_desc &c, int G, CUtensorMap *out) {
+    const MapKey key{cache, c.num_blocks, c.block_size, c.num_heads, c.head_size, c.dtype, G};
+    {
+        std::lock_guard<std::mutex> lk(g_map_mu);
+        for (auto &e : g_maps)
+            if (e.first == key) {
+                *out = e.second;
+                return PA_OK;
+            }
+    }
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    const cuuint64_t eb = (cuuint64_t)elem_bytes(c);
+    const cuuint64_t dims[4] = {(cuuint64_t)c.head_size, (cuuint64_t)c.num_heads,
+                                (cuuint64_t)c.block_size, (cuuint64_t)c.num_blocks};
+    const cuuint64_t strides[3] = {(cuuint64_t)c.head_size * eb,
+                                   (cuuint64_t)c.head_size * c.num_heads * eb,
+                                   (cuuint64_t)c.head_size * c.num_heads * c.block_size * eb};
+    const cuuint32_t box[4] = {(cuuint32_t)c.head_size, (cuuint32_t)G, (cuuint32_t)c.block_size, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUtensorMap m;
+    const CUresult r = enc(&m,
+                           c.dtype == PA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                             : CU_TENSOR_MAP_DATA_TYPE_UINT8,
+                           4, const_cast<void *>(cache), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    {
+        std::lock_guard<std::mutex> lk(g_map_mu);
+        if (g_maps.size() >= 64) g_maps.erase(g_maps.begin());
+        g_maps.emplace_back(key, m);
+    }
+    *out = m;
+    return PA_OK;
+}
+
+// ----------------------------------------------------- launch shape
+
+constexpr int kNumSMs = 148;
+constexpr size_t kMaxSmem = 227 * 1024;
+
+int fill_config(const pa_cache_desc &c, int num_seqs, int max_ctx, pa_decode_config *cfg) {
+    const int H = c.num_heads, B = c.block_size;
+    pa_decode_config r = *cfg;
+    auto stage_bytes = [&](int G) {
+        return pa::SmemLayout(B, G, c.head_size, elem_bytes(c), 1, 1).stage_bytes;
+    };
+    if (r.heads_per_cta == 0) {
+        int G = 4;
+        while (G > 1 && (H % G || stage_bytes(G) * 4 > 160 * 1024)) G >>= 1;
+        const int P0 = r.partition_size ? r.partition_size : 512;
+        const int parts = std::max(1, (max_ctx + P0 - 1) / P0);
+        while (G > 1 && (int64_t)num_seqs * (H / G) * parts < 3 * kNumSMs) G >>= 1;
+        r.heads_per_cta = G;
+    }
+    if (r.partition_size == 0) {
+        int P = 512;
+        const int64_t units0 = (int64_t)num_seqs * (H / r.heads_per_cta);
+        while (P > 4 * B && units0 * std::max(1, (max_ctx + P - 1) / P) < 3 * kNumSMs) P >>= 1;
+        r.partition_size = P;
+    }
+    if (r.warps_per_head == 0) r.warps_per_head = std::min(4, std::max(1, 8 / r.heads_per_cta));
+    if (r.stages == 0) {
+        const size_t sb = stage_bytes(r.heads_per_cta);
+        r.stages = (int)std::max<size_t>(2, std::min<size_t>(8, (128 * 1024) / sb));
+    }
+    if (r.partition_size < B || r.partition_size % B)
+        return fail(PA_ERR_INVALID, "partition_size %d must be a positive multiple of block_size %d",
+                    r.partition_size, B);
+    const int G = r.heads_per_cta;
+    if (!(G == 1 || G == 2 || G == 4 || G == 8) || H % G)
+        return fail(PA_ERR_INVALID, "heads_per_cta %d must be 1, 2, 4 or 8 and divide num_heads %d",
+                    G, H);
+    const int W = r.warps_per_head;
+    if (!(W == 1 || W == 2 || W == 4) || G * W > pa::kMaxConsumerWarps)
+        return fail(PA_ERR_INVALID, "warps_per_head %d must be 1, 2 or 4 with heads*warps <= %d", W,
+                    pa::kMaxConsumerWarps);
+    if (r.stages < 2 || r.stages > 8)
+        return fail(PA_ERR_INVALID, "stages %d must be in [2, 8]", r.stages);
+    const pa::SmemLayout lay(B, G, c.head_size, elem_bytes(c), W, r.stages);
+    if (lay.total > kMaxSmem)
+        return fail(PA_ERR_INVALID, "launch shape needs %zu bytes of shared memory (max %zu)",
+                    lay.total, kMaxSmem);
+    *cfg = r;
+    return PA_OK;
+}
+
+int max_parts_of(int max_ctx, int P) { return std::max(1, (max_ctx + P - 1) / P); }
+
+size_t ws_lse_bytes(const pa_cache_desc &c, int S, int parts) {
+    return ((size_t)S * c.num_heads * parts * sizeof(float) + 255) / 256 * 256;
+}
+
+size_t ws_bytes(const pa_cache_desc &c, int S, int max_ctx, const pa_decode_config &cfg) {
+    const int parts = max_parts_of(max_ctx, cfg.partition_size);
+    if (parts <= 1) return 0;
+    return ws_lse_bytes(c, S, parts) + (size_t)S * c.num_heads * parts * c.head_size * sizeof(float);
+}
+
+// ----------------------------------------------------- kernel tables
+
+using DecodeKernel = void (*)(const CUtensorMap, const CUtensorMap, const pa::DecodeParams);
+using ReduceKernel = void (*)(const pa::DecodeParams);
+
+DecodeKernel pick_decode(int D, int B, bool fp8) {
+#define PA_PICK(d, b, f) \
+    if (D == d && B == b && fp8 == f) return pa::paged_decode_kernel<d, b, f>;
+    PA_PICK(64, 16, false) PA_PICK(64, 32, false) PA_PICK(128, 16, false) PA_PICK(128, 32, false)
+    PA_PICK(64, 16, true) PA_PICK(64, 32, true) PA_PICK(128, 16, true) PA_PICK(128, 32, true)
+#undef PA_PICK
+    return nullptr;
+}
+
+ReduceKernel pick_reduce(int D) {
+    return D == 64 ? pa::lse_reduce_kernel<64> : pa::lse_reduce_kernel<128>;
+}
+
+std::mutex g_attr_mu;
+std::vector<std::pair<const void *, int>> g_attr_done;  // (kernel, device) with max smem set
+
+int ensure_smem_attr(const void *fn, int device) {
+    std::lock_guard<std::mutex> lk(g_attr_mu);
+    for (auto &e : g_attr_done)
+        if (e.first == fn && e.second == device) return PA_OK;
+    const cudaError_t e =
+        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxSmem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    g_attr_done.emplace_back(fn, device);
+    return PA_OK;
+}
+
+// ---------------------------------------------- internal split workspace
+
+struct WsEntry {
+    int device;
+    cudaStream_t stream;
+    void *ptr;
+    size_t bytes;
+};
+std::mutex g_ws_mu;
+std::vector<WsEntry> g_ws;
+
+int internal_workspace(size_t need, cudaStream_t st, int device, void **out) {
+    std::lock_guard<std::mutex> lk(g_ws_mu);
+    WsEntry *ent = nullptr;
+    for (auto &e : g_ws)
+        if (e.device == device && e.stream == st) ent = &e;
+    if (ent && ent->bytes >= need) {
+        *out = ent->ptr;
+        return PA_OK;
+    }
+    const size_t bytes = std::max<size_t>(need + need / 4, 1 << 20);
+    void *p = nullptr;
+    cudaError_t e = cudaMallocAsync(&p, bytes, st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync (split workspace)");
+    if (ent) {
+        e = cudaFreeAsync(ent->ptr, st);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync (split workspace)");
+        ent->ptr = p;
+        ent->bytes = bytes;
+    } else {
+        g_ws.push_back(WsEntry{device, st, p, bytes});
+    }
+    *out = p;
+    return PA_OK;
+}
+
+int check_decode_args(void *out, const void *query, const void *kc, const void *vc,
+                      const pa_cache_desc &c, const int32_t *bt, int maxblk, const int32_t *ctx,
+                      int S, int max_ctx, float scale, float k_scale, float v_scale) {
+    int rc = check_cache(c);
+    if (rc) return rc;
+    if (S < 0) return fail(PA_ERR_INVALID, "num_seqs %d < 0", S);
+    if (S > 65535) return fail(PA_ERR_INVALID, "num_seqs %d > 65535", S);
+    if (S == 0) return PA_OK;
+    if (!out || !query || !kc || !vc || !bt || !ctx)
+        return fail(PA_ERR_INVALID, "null pointer argument");
+    if (!aligned16(out) || !aligned16(query) || !aligned16(kc) || !aligned16(vc))
+        return fail(PA_ERR_INVALID, "out, query and caches must be 16-byte aligned");
+    if (maxblk < 1) return fail(PA_ERR_INVALID, "max_blocks_per_seq %d < 1", maxblk);
+    if ((int64_t)maxblk * c.block_size >= (int64_t(1) << 31))
+        return fail(PA_ERR_OVERFLOW, "max_blocks_per_seq * block_size overflows int32");
+    if (max_ctx < 0) return fail(PA_ERR_INVALID, "max_context_len %d < 0", max_ctx);
+    if (!std::isfinite(scale)) return fail(PA_ERR_INVALID, "scale is not finite");
+    if (c.dtype == PA_E4M3 &&
+        !(std::isfinite(k_scale) && std::isfinite(v_scale) && k_scale > 0 && v_scale > 0))
+        return fail(PA_ERR_INVALID, "k_scale and v_scale must be finite and > 0");
+    return PA_OK;
+}
+
+int launch_decode(void *out, const void *query, const void *kc, const void *vc,
+                  const pa_cache_desc &c, const int32_t *bt, int maxblk, const int32_t *ctx, int S,
+                  int max_ctx, float scale, float k_scale, float v_scale,
+                  const pa_decode_config &cfg, void *ws, cudaStream_t st, int device) {
+    const int B = c.block_size, D = c.head_size;
+    const bool fp8 = c.dtype == PA_E4M3;
+    max_ctx = std::min<int64_t>(max_ctx, (int64_t)maxblk * B);
+    const int parts = max_parts_of(max_ctx, cfg.partition_size);
+    const int G = cfg.heads_per_cta, W = cfg.warps_per_head;
+
+    CUtensorMap mk, mv;
+    int rc = cache_tensor_map(kc, c, G, &mk);
+    if (rc) return rc;
+    rc = cache_tensor_map(vc, c, G, &mv);
+    if (rc) return rc;
+
+    pa::DecodeParams p{};
+    p.out = static_cast<__half *>(out);
+    p.query = static_cast<const __half *>(query);
+    p.block_tables = bt;
+    p.context_lens = ctx;
+    if (parts > 1) {
+        p.ws_lse = static_cast<float *>(ws);
+        p.ws_o = reinterpret_cast<float *>(static_cast<char *>(ws) + ws_lse_bytes(c, S, parts));
+    }
+    p.num_seqs = S;
+    p.num_heads = c.num_heads;
+    p.num_blocks = c.num_blocks;
+    p.block_size = B;
+    p.max_blocks_per_seq = maxblk;
+    p.max_context_len = max_ctx;
+    p.partition_size = cfg.partition_size;
+    p.max_parts = parts;
+    p.heads_per_cta = G;
+    p.warps_per_head = W;
+    p.stages = cfg.stages;
+    p.qk_scale_log2 = scale * (fp8 ? k_scale : 1.0f) * pa::kLog2e;
+    p.out_scale = fp8 ? v_scale : 1.0f;
+
+    DecodeKernel kern = pick_decode(D, B, fp8);
+    if (!kern) return fail(PA_ERR_INVALID, "no kernel for head_size %d block_size %d", D, B);
+    rc = ensure_smem_attr(reinterpret_cast<const void *>(kern), device);
+    if (rc) return rc;
+    const pa::SmemLayout lay(B, G, D, elem_bytes(c), W, cfg.stages);
+    const dim3 grid(parts, c.num_heads / G, S);
+    const dim3 block(32 * (G * W + 1));
+    kern<<<grid, block, lay.total, st>>>(mk, mv, p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "paged_decode_kernel launch");
+    if (parts > 1) {
+        pick_reduce(D)<<<dim3((c.num_heads + 3) / 4, S), 128, 0, st>>>(p);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "lse_reduce_kernel launch");
+    }
+    return ok();
+}
+
+int current_device(int *dev) {
+    const cudaError_t e = cudaGetDevice(dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    return PA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int pa_version(void) { return 100; }
+
+const char *pa_last_error(void) { return g_msg; }
+
+int pa_check_status(void *stream, uint32_t *code) {
+    if (!code) return fail(PA_ERR_INVALID, "code is null");
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    unsigned int v = 0, zero = 0;
+    e = cudaMemcpyFromSymbol(&v, pa::g_error_word, sizeof(v));
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+    e = cudaMemcpyToSymbol(pa::g_error_word, &zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+    *code = v;
+    return ok();
+}
+
+int pa_slot_mapping(int32_t *slot_mapping, const int32_t *block_tables, int max_blocks_per_seq,
+                    const int32_t *context_lens, int num_seqs, pa_cache_desc cache, void *stream) {
+    int rc = check_cache(cache);
+    if (rc) return rc;
+    if (num_seqs < 0) return fail(PA_ERR_INVALID, "num_seqs %d < 0", num_seqs);
+    if (num_seqs == 0) return ok();
+    if (!slot_mapping || !block_tables || !context_lens)
+        return fail(PA_ERR_INVALID, "null pointer argument");
+    if (max_blocks_per_seq < 1) return fail(PA_ERR_INVALID, "max_blocks_per_seq < 1");
+    const int threads = 128;
+    pa::slot_mapping_kernel<<<(num_seqs + threads - 1) / threads, threads, 0,
+                              static_cast<cudaStream_t>(stream)>>>(
+        slot_mapping, block_tables, max_blocks_per_seq, context_lens, num_seqs, cache.block_size,
+        cache.num_blocks);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "slot_mapping_kernel launch");
+    return ok();
+}
+
+int pa_kv_cache_write(const void *key, const void *value, int64_t key_stride, int64_t value_stride,
+                      void *key_cache, void *value_cache, pa_cache_desc cache,
+                      const int32_t *slot_mapping, int n_tokens, float k_scale, float v_scale,
+                      void *stream) {
+    int rc = check_cache(cache);
+    if (rc) return rc;
+    if (n_tokens < 0) return fail(PA_ERR_INVALID, "n_tokens %d < 0", n_tokens);
+    if (n_tokens == 0) return ok();
+    if (n_tokens > 65535) return fail(PA_ERR_INVALID, "n_tokens %d > 65535 per call", n_tokens);
+    if (!key || !value || !key_cache || !value_cache || !slot_mapping)
+        return fail(PA_ERR_INVALID, "null pointer argument");
+    if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache))
+        return fail(PA_ERR_INVALID, "key, value and caches must be 16-byte aligned");
+    const int row = cache.num_heads * cache.head_size;
+    if (key_stride < row || value_stride < row || key_stride % 8 || value_stride % 8)
+        return fail(PA_ERR_INVALID,
+                    "key_stride/value_stride (%lld/%lld) must be >= %d and multiples of 8",
+                    (long long)key_stride, (long long)value_stride, row);
+    if (cache.dtype == PA_E4M3 &&
+        !(std::isfinite(k_scale) && std::isfinite(v_scale) && k_scale > 0 && v_scale > 0))
+        return fail(PA_ERR_INVALID, "k_scale and v_scale must be finite and > 0");
+    const int chunks = row / 8;
+    const dim3 grid((chunks + 127) / 128, n_tokens);
+    const int64_t pool_slots = (int64_t)cache.num_blocks * cache.block_size;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const __half *k = static_cast<const __half *>(key);
+    const __half *v = static_cast<const __half *>(value);
+    if (cache.dtype == PA_F16)
+        pa::kv_cache_write_kernel<false><<<grid, 128, 0, st>>>(
+            k, v, key_stride, value_stride, key_cache, value_cache, slot_mapping, row, pool_slots,
+            1.0f, 1.0f);
+    else
+        pa::kv_cache_write_kernel<true><<<grid, 128, 0, st>>>(
+            k, v, key_stride, value_stride, key_cache, value_cache, slot_mapping, row, pool_slots,
+            k_scale, v_scale);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "kv_cache_write_kernel launch");
+    return ok();
+}
+
+int pa_copy_blocks(void *key_cache, void *value_cache, pa_cache_desc cache,
+                   const int32_t *src_dst_pairs, int n_pairs, void *stream) {
+    int rc = check_cache(cache);
+    if (rc) return rc;
+    if (n_pairs < 0) return fail(PA_ERR_INVALID, "n_pairs %d < 0", n_pairs);
+    if (n_pairs == 0) return ok();
+    if (n_pairs > 65535) return fail(PA_ERR_INVALID, "n_pairs %d > 65535 per call", n_pairs);
+    if (!key_cache || !value_cache || !src_dst_pairs)
+        return fail(PA_ERR_INVALID, "null pointer argument");
+    if (!aligned16(key_cache) || !aligned16(value_cache))
+        return fail(PA_ERR_INVALID, "caches must be 16-byte aligned");
+    const int64_t block_vecs =
+        (int64_t)cache.block_size * cache.num_heads * cache.head_size * elem_bytes(cache) / 16;
+    const int64_t per_cta = (int64_t)pa::kCopyThreads * pa::kCopyVecs;
+    const dim3 grid((unsigned)((block_vecs + per_cta - 1) / per_cta), n_pairs, 2);
+    pa::copy_blocks_kernel<<<grid, pa::kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+        key_cache, value_cache, src_dst_pairs, block_vecs, cache.num_blocks);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "copy_blocks_kernel launch");
+    return ok();
+}
+
+int pa_decode_choose_config(pa_cache_desc cache, int num_seqs, int max_context_len,
+                            pa_decode_config *cfg) {
+    int rc = check_cache(cache);
+    if (rc) return rc;
+    if (!cfg) return fail(PA_ERR_INVALID, "cfg is null");
+    if (num_seqs < 0 || max_context_len < 0)
+        return fail(PA_ERR_INVALID, "num_seqs and max_context_len must be >= 0");
+    rc = fill_config(cache, num_seqs, max_context_len, cfg);
+    if (rc) return rc;
+    return ok();
+}
+
+size_t pa_decode_workspace_size(pa_cache_desc cache, int num_seqs, int max_context_len,
+                                const pa_decode_config *cfg) {
+    if (check_cache(cache) || num_seqs <= 0 || max_context_len < 0) return 0;
+    pa_decode_config r = cfg ? *cfg : pa_decode_config{0, 0, 0, 0};
+    if (fill_config(cache, num_seqs, max_context_len, &r)) return 0;
+    return ws_bytes(cache, num_seqs, max_context_len, r);
+}
+
+int pa_paged_attention_decode(void *out, const void *query, const void *key_cache,
+                              const void *value_cache, pa_cache_desc cache,
+                              const int32_t *block_tables, int max_blocks_per_seq,
+                              const int32_t *context_lens, int num_seqs, int max_context_len,
+                              float scale, float k_scale, float v_scale, void *stream) {
+    int rc = check_decode_args(out, query, key_cache, value_cache, cache, block_tables,
+                               max_blocks_per_seq, context_lens, num_seqs, max_context_len, scale,
+                               k_scale, v_scale);
+    if (rc) return rc;
+    if (num_seqs == 0) return ok();
+    const int bound = (int)std::min<int64_t>(max_context_len, (int64_t)max_blocks_per_seq * cache.block_size);
+    pa_decode_config cfg{0, 0, 0, 0};
+    rc = fill_config(cache, num_seqs, bound, &cfg);
+    if (rc) return rc;
+    int dev = 0;
+    rc = current_device(&dev);
+    if (rc) return rc;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    void *ws = nullptr;
+    const size_t need = ws_bytes(cache, num_seqs, bound, cfg);
+    if (need) {
+        rc = internal_workspace(need, st, dev, &ws);
+        if (rc) return rc;
+    }
+    return launch_decode(out, query, key_cache, value_cache, cache, block_tables,
+                         max_blocks_per_seq, context_lens, num_seqs, bound, scale, k_scale,
+                         v_scale, cfg, ws, st, dev);
+}
+
+int pa_paged_attention_decode_ws(void *out, const void *query, const void *key_cache,
+                                 const void *value_cache, pa_cache_desc cache,
+                                 const int32_t *block_tables, int max_blocks_per_seq,
+                                 const int32_t *context_lens, int num_seqs, int max_context_len,
+                                 float scale, float k_scale, float v_scale,
+                                 const pa_decode_config *cfg, void *workspace,
+                                 size_t workspace_bytes, void *stream) {
+    int rc = check_decode_args(out, query, key_cache, value_cache, cache, block_tables,
+                               max_blocks_per_seq, context_lens, num_seqs, max_context_len, scale,
+                               k_scale, v_scale);
+    if (rc) return rc;
+    if (num_seqs == 0) return ok();
+    const int bound = (int)std::min<int64_t>(max_context_len, (int64_t)max_blocks_per_seq * cache.block_size);
+    pa_decode_config r = cfg ? *cfg : pa_decode_config{0, 0, 0, 0};
+    rc = fill_config(cache, num_seqs, bound, &r);
+    if (rc) return rc;
+    const size_t need = ws_bytes(cache, num_seqs, bound, r);
+    if (need && (!workspace || workspace_bytes < need ||
+                 (reinterpret_cast<uintptr_t>(workspace) & 255u)))
+        return fail(PA_ERR_WORKSPACE,
+                    "workspace of %zu bytes at %p: need %zu bytes, 256-byte aligned",
+                    workspace_bytes, workspace, need);
+    int dev = 0;
+    rc = current_device(&dev);
+    if (rc) return rc;
+    return launch_decode(out, query, key_cache, value_cache, cache, block_tables,
+                         max_blocks_per_seq, context_lens, num_seqs, bound, scale, k_scale,
+                         v_scale, r, workspace, static_cast<cudaStream_t>(stream), dev);
+}
+
+}  // extern "C"

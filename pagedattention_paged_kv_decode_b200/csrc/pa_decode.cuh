@@ -1,0 +1,449 @@
+// pa_decode.cuh -- paged decode attention kernels for sm_100a.
+//
+// What is computed (the plain definition of single-query softmax attention
+// over the tokens a block table addresses; the pages fix the block table and
+// the physical block pool -- "vLLM-v0.17.1技术解析" §2.2, "在A10G上榨干LLaMA-7B"
+// §2.1 -- but print no kernel):
+//   z_t = scale * k_scale * q . K_t,   out = v_scale * sum_t softmax(z)_t V_t
+//
+// Design (one CTA = one sequence x a group of G heads x one partition of the
+// context):
+//   * a producer warp reads the block-table entries of the partition and
+//     issues, per physical block, two TMA tiled loads -- the K and V tiles
+//     [block_size][G][head_size] of the 4-D cache view [NB][B][H][D] -- into a
+//     ring of shared-memory stages guarded by full/empty mbarriers;
+//   * G x W consumer warps: warp (g, w) owns head g and every W-th block of
+//     the partition. Per block it forms the logits with 16-byte shared loads
+//     and fp32 FMAs, reduces them with a transposing butterfly (one shuffle
+//     per token per lane), runs the online-softmax update and accumulates
+//     P.V in fp32 registers;
+//   * the W warps of a head merge (m, l, acc) through shared memory; a
+//     sequence that fits one partition writes fp16 output directly, longer
+//     ones write (lse, normalised o) for the log-sum-exp reduce kernel.
+// Nothing here is a dense contraction (one query row per head), so the
+// kernel runs on the CUDA cores and is bound by HBM bandwidth.
+#pragma once
+
+#include "pa_device.cuh"
+
+namespace pa {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kMaxConsumerWarps = 16;                       // heads_per_cta * warps_per_head
+constexpr int kMaxDecodeThreads = 32 * (kMaxConsumerWarps + 1);
+
+struct DecodeParams {
+    __half *out;                 // [S][H][D]
+    const __half *query;         // [S][H][D]
+    const int32_t *block_tables; // [S][max_blocks_per_seq]
+    const int32_t *context_lens; // [S]
+    float *ws_lse;               // [S][H][max_parts] (split only)
+    float *ws_o;                 // [S][H][max_parts][D] (split only)
+    int num_seqs;
+    int num_heads;
+    int num_blocks;
+    int block_size;
+    int max_blocks_per_seq;
+    int max_context_len;
+    int partition_size;          // tokens, multiple of block_size
+    int max_parts;               // ceil(max_context_len / partition_size)
+    int heads_per_cta;           // G
+    int warps_per_head;          // W
+    int stages;
+    float qk_scale_log2;         // scale * k_scale * log2(e)
+    float out_scale;             // v_scale (1 for fp16 caches)
+};
+
+// Lane geometry of a consumer warp. Each lane holds EPL consecutive elements
+// of a K/V row (16 bytes), LPR lanes cover one row of head_size elements,
+// and the warp's NGRP lane groups take different tokens of a block.
+template <int D, int B, bool kFp8>
+struct Geometry {
+    static constexpr int kElemBytes = kFp8 ? 1 : 2;
+    static constexpr int EPL = 16 / kElemBytes;
+    static constexpr int LPR = D / EPL;
+    static constexpr int NGRP = 32 / LPR;
+    static constexpr int TPG = B / NGRP;          // tokens of a block per lane group
+    static constexpr int DUP = LPR / TPG;         // lanes holding the same logit after the butterfly
+    static constexpr int kRowBytes = D * kElemBytes;
+    static_assert(LPR >= 1 && LPR <= 32 && 32 % LPR == 0, "head_size / lane mapping");
+    static_assert(TPG >= 1 && TPG <= LPR && LPR % TPG == 0, "block_size / lane mapping");
+};
+
+// Transposing butterfly: on entry part[j] is this lane's partial dot product
+// for token j of its group (over its EPL dims). After the log2(LPR) rounds,
+// part[0] is the full dot product of token (sub / DUP), where sub is the
+// lane's index inside its group. Each split round hands half of the values
+// to the partner lane and keeps the other half, so a group of LPR lanes
+// reduces TPG dot products with TPG-1 (+ log2 DUP) shuffles per lane.
+template <int TPG, int LPR>
+__device__ __forceinline__ float butterfly_reduce(float (&part)[TPG], int lane) {
+    int n = TPG;
+#pragma unroll
+    for (int mask = LPR / 2; mask >= 1; mask >>= 1) {
+        if (n > 1) {
+            const int half = n / 2;
+            const bool upper = (lane & mask) != 0;
+#pragma unroll
+            for (int k = 0; k < TPG / 2; ++k) {
+                if (k < half) {
+                    const float send = upper ? part[k] : part[k + half];
+                    const float keep = upper ? part[k + half] : part[k];
+                    part[k] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
+                }
+            }
+            n = half;
+        } else {
+            part[0] += __shfl_xor_sync(0xffffffffu, part[0], mask);
+        }
+    }
+    return part[0];
+}
+
+// 16 bytes of a K/V row -> EPL floats.
+template <bool kFp8>
+__device__ __forceinline__ void unpack16(const uint4 &raw, float *f);
+
+template <>
+__device__ __forceinline__ void unpack16<false>(const uint4 &raw, float *f) {
+    const __half2 *h = reinterpret_cast<const __half2 *>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 x = __half22float2(h[i]);
+        f[2 * i] = x.x;
+        f[2 * i + 1] = x.y;
+    }
+}
+
+template <>
+__device__ __forceinline__ void unpack16<true>(const uint4 &raw, float *f) {
+    const uint16_t *c = reinterpret_cast<const uint16_t *>(&raw);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float2 x = __half22float2(e4m3x2_to_half2(c[i]));
+        f[2 * i] = x.x;
+        f[2 * i + 1] = x.y;
+    }
+}
+
+__device__ __forceinline__ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Shared-memory carve-up, identical on host and device.
+struct SmemLayout {
+    size_t tile_bytes;   // one K (or V) tile: B * G * D * elem
+    size_t stage_bytes;  // K tile + V tile
+    size_t bars_off;     // full[stages], empty[stages]
+    size_t merge_off;    // W * G * (D + 2) floats
+    size_t total;
+    __host__ __device__ SmemLayout(int B, int G, int D, int elem, int W, int stages) {
+        tile_bytes = (size_t)B * G * D * elem;
+        stage_bytes = 2 * tile_bytes;
+        bars_off = stage_bytes * stages;
+        merge_off = bars_off + 2 * 8 * (size_t)stages;
+        merge_off = (merge_off + 15) / 16 * 16;
+        total = merge_off + sizeof(float) * (size_t)W * G * (D + 2);
+    }
+};
+
+template <int D, int B, bool kFp8>
+__global__ void __launch_bounds__(kMaxDecodeThreads, 1)
+paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                    const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
+    using Geo = Geometry<D, B, kFp8>;
+    constexpr int EPL = Geo::EPL, LPR = Geo::LPR, TPG = Geo::TPG, DUP = Geo::DUP;
+
+    extern __shared__ __align__(1024) unsigned char smem[];
+    const int G = p.heads_per_cta, W = p.warps_per_head, stages = p.stages;
+    const SmemLayout lay(B, G, D, Geo::kElemBytes, W, stages);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + lay.bars_off);
+    uint64_t *empty = full + stages;
+    float *merge = reinterpret_cast<float *>(smem + lay.merge_off);
+
+    const int part = blockIdx.x;
+    const int h0 = blockIdx.y * G;
+    const int s = blockIdx.z;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int n_consumers = G * W;
+
+    // Context length, clamped to what the table and the grid can address.
+    int L = __ldg(p.context_lens + s);
+    const int cap = p.max_blocks_per_seq * B;
+    if (L > cap) {
+        if (threadIdx.x == 0 && part == 0 && blockIdx.y == 0) flag_error(PA_DEV_CTX_OVER_TABLE);
+        L = cap;
+    }
+    if (L > p.max_context_len) {
+        if (threadIdx.x == 0 && part == 0 && blockIdx.y == 0) flag_error(PA_DEV_CTX_OVER_BOUND);
+        L = p.max_context_len;
+    }
+    if (L < 0) L = 0;
+    const int n_parts = (L + p.partition_size - 1) / p.partition_size;
+    if (part >= n_parts) {
+        if (L == 0 && part == 0) {  // empty context: zeros
+            for (int i = threadIdx.x; i < G * D / 8; i += blockDim.x) {
+                const int g = i / (D / 8), c = i % (D / 8);
+                reinterpret_cast<uint4 *>(p.out + ((size_t)s * p.num_heads + h0 + g) * D)[c] =
+                    make_uint4(0, 0, 0, 0);
+            }
+        }
+        return;
+    }
+    const int t0 = part * p.partition_size;
+    const int t1 = min(L, t0 + p.partition_size);
+    const int blk0 = t0 / B;
+    const int nblk = (t1 - t0 + B - 1) / B;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < stages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], G);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp == n_consumers) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            prefetch_tensor_map(&tmap_k);
+            prefetch_tensor_map(&tmap_v);
+        }
+        const int32_t *row = p.block_tables + (size_t)s * p.max_blocks_per_seq + blk0;
+        const uint64_t policy = l2_policy_evict_first();
+        const uint32_t tx_bytes = (uint32_t)lay.stage_bytes;
+        bool ok = true;
+        int stage = 0, use = 0;
+        for (int base = 0; base < nblk && ok; base += 32) {
+            int my_blk = 0;
+            if (base + lane < nblk) my_blk = __ldg(row + base + lane);
+            const int cnt = min(32, nblk - base);
+            for (int j = 0; j < cnt; ++j) {
+                int blk = __shfl_sync(0xffffffffu, my_blk, j);
+                if (lane == 0) {
+                    if (blk < 0 || blk >= p.num_blocks) {
+                        flag_error(PA_DEV_BAD_BLOCK);
+                        blk = p.num_blocks;  // out of range: the TMA zero-fills the tile
+                    }
+                    if (use > 0) ok = mbar_wait(&empty[stage], (use - 1) & 1);
+                    if (ok) {
+                        unsigned char *kdst = smem + (size_t)stage * lay.stage_bytes;
+                        mbar_arrive_expect_tx(&full[stage], tx_bytes);
+                        tma_load_4d(kdst, &tmap_k, &full[stage], 0, h0, 0, blk, policy);
+                        tma_load_4d(kdst + lay.tile_bytes, &tmap_v, &full[stage], 0, h0, 0, blk,
+                                    policy);
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                if (++stage == stages) {
+                    stage = 0;
+                    ++use;
+                }
+            }
+        }
+        return;
+    }
+
+    // --------------------------------------------------------------- consumers
+    const int g = warp % G;
+    const int w = warp / G;
+    const int h = h0 + g;
+    const int grp = lane / LPR;
+    const int sub = lane % LPR;
+
+    float q[EPL];
+    {
+        const __half *qp = p.query + ((size_t)s * p.num_heads + h) * D;
+        if constexpr (kFp8) {
+            // EPL = 16 elements: two 16-byte fp16 chunks
+            const uint4 a = __ldg(reinterpret_cast<const uint4 *>(qp) + 2 * sub);
+            const uint4 b = __ldg(reinterpret_cast<const uint4 *>(qp) + 2 * sub + 1);
+            unpack16<false>(a, q);
+            unpack16<false>(b, q + 8);
+        } else {
+            const uint4 a = __ldg(reinterpret_cast<const uint4 *>(qp) + sub);
+            unpack16<false>(a, q);
+        }
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) q[e] *= p.qk_scale_log2;
+    }
+
+    float m = -INFINITY, l = 0.f;
+    float acc[EPL];
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
+
+    const size_t row_stride = (size_t)G * D * Geo::kElemBytes;  // bytes between tokens in a tile
+    const size_t head_off = (size_t)g * D * Geo::kElemBytes + (size_t)sub * 16;
+    bool ok = true;
+    int stage = w % stages, use = w / stages;
+    for (int i = w; i < nblk; i += W) {
+        if (!mbar_wait(&full[stage], use & 1)) {
+            ok = false;
+            break;
+        }
+        const unsigned char *ktile = smem + (size_t)stage * lay.stage_bytes;
+        const unsigned char *vtile = ktile + lay.tile_bytes;
+        const int valid = min(B, t1 - (t0 + i * B));  // tokens of this block inside the context
+
+        // ---- logits of this lane group's TPG tokens
+        float part_dot[TPG];
+#pragma unroll
+        for (int j = 0; j < TPG; ++j) {
+            const int t = grp * TPG + j;
+            const uint4 raw = *reinterpret_cast<const uint4 *>(ktile + t * row_stride + head_off);
+            float k[EPL];
+            unpack16<kFp8>(raw, k);
+            float d = 0.f;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) d = fmaf(q[e], k[e], d);
+            part_dot[j] = d;
+        }
+        const int my_t = grp * TPG + sub / DUP;
+        float z = butterfly_reduce<TPG, LPR>(part_dot, lane);
+        z = (my_t < valid) ? z : -INFINITY;
+
+        // ---- online softmax (base 2)
+        const float m_new = fmaxf(m, warp_max(z));
+        const float alpha = fast_exp2(m - m_new);
+        const float pz = fast_exp2(z - m_new);
+        l = l * alpha + pz;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) acc[e] *= alpha;
+        m = m_new;
+
+        // ---- P.V for this lane group's tokens
+#pragma unroll
+        for (int j = 0; j < TPG; ++j) {
+            const int t = grp * TPG + j;
+            const float pj = __shfl_sync(0xffffffffu, pz, grp * LPR + j * DUP);
+            if (t < valid) {
+                const uint4 raw = *reinterpret_cast<const uint4 *>(vtile + t * row_stride + head_off);
+                float v[EPL];
+                unpack16<kFp8>(raw, v);
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) acc[e] = fmaf(pj, v[e], acc[e]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[stage]);
+        stage += W;
+        while (stage >= stages) {
+            stage -= stages;
+            ++use;
+        }
+    }
+    (void)ok;
+
+    // ---- reduce this warp's state: l over all lanes, acc over lane groups
+    l = warp_sum(l) * (1.0f / DUP);
+#pragma unroll
+    for (int mask = LPR; mask < 32; mask <<= 1) {
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], mask);
+    }
+
+    // ---- merge the W warps of each head through shared memory
+    if (W > 1) {
+        float *slot = merge + (size_t)(w * G + g) * (D + 2);
+        if (grp == 0) {
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) slot[sub * EPL + e] = acc[e];
+        }
+        if (lane == 0) {
+            slot[D] = m;
+            slot[D + 1] = l;
+        }
+        asm volatile("bar.sync 1, %0;" ::"r"(n_consumers * 32) : "memory");
+        if (w != 0) return;
+        float M = -INFINITY;
+        for (int k = 0; k < W; ++k) M = fmaxf(M, merge[(size_t)(k * G + g) * (D + 2) + D]);
+        float Lsum = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
+        for (int k = 0; k < W; ++k) {
+            const float *o = merge + (size_t)(k * G + g) * (D + 2);
+            const float f = fast_exp2(o[D] - M);  // warps without tokens: m = -inf -> 0
+            Lsum += o[D + 1] * f;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) acc[e] += o[sub * EPL + e] * f;
+        }
+        m = M;
+        l = Lsum;
+    }
+
+    if (grp != 0) return;
+    const float inv_l = 1.0f / l;
+    if (n_parts == 1) {
+        __half *op = p.out + ((size_t)s * p.num_heads + h) * D + sub * EPL;
+#pragma unroll
+        for (int c = 0; c < EPL / 8; ++c) {
+            uint4 pk;
+            __half2 *hp = reinterpret_cast<__half2 *>(&pk);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                hp[i] = __floats2half2_rn(acc[c * 8 + 2 * i] * inv_l * p.out_scale,
+                                          acc[c * 8 + 2 * i + 1] * inv_l * p.out_scale);
+            reinterpret_cast<uint4 *>(op)[c] = pk;
+        }
+    } else {
+        const size_t idx = ((size_t)s * p.num_heads + h) * p.max_parts + part;
+        float *op = p.ws_o + idx * D + sub * EPL;
+#pragma unroll
+        for (int c = 0; c < EPL / 4; ++c)
+            reinterpret_cast<float4 *>(op)[c] =
+                make_float4(acc[4 * c] * inv_l, acc[4 * c + 1] * inv_l, acc[4 * c + 2] * inv_l,
+                            acc[4 * c + 3] * inv_l);
+        if (sub == 0) p.ws_lse[idx] = m + fast_log2(l);
+    }
+}
+
+// Log-sum-exp reduction of the partitions of each (sequence, head) whose
+// context spans more than one partition. One warp per (sequence, head):
+//   M = max_p lse_p,  w_p = 2^(lse_p - M),  out = v_scale * sum_p w_p o_p / sum_p w_p
+template <int D>
+__global__ void __launch_bounds__(128)
+lse_reduce_kernel(const DecodeParams p) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = blockIdx.x * 4 + warp;
+    const int s = blockIdx.y;
+    if (h >= p.num_heads) return;
+    int L = __ldg(p.context_lens + s);
+    L = min(L, p.max_blocks_per_seq * p.block_size);   // same clamps as the partition kernel
+    L = min(L, p.max_context_len);
+    const int n_parts = L > 0 ? (L + p.partition_size - 1) / p.partition_size : 0;
+    if (n_parts <= 1) return;
+    const size_t base = ((size_t)s * p.num_heads + h) * p.max_parts;
+    float M = -INFINITY;
+    for (int i = lane; i < n_parts; i += 32) M = fmaxf(M, p.ws_lse[base + i]);
+    M = warp_max(M);
+    constexpr int DPL = D / 32;  // dims per lane
+    float acc[DPL];
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+    float wsum = 0.f;
+    for (int i = 0; i < n_parts; ++i) {
+        const float wgt = fast_exp2(p.ws_lse[base + i] - M);
+        wsum += wgt;
+        const float *o = p.ws_o + (base + i) * D + lane * DPL;
+        if constexpr (DPL == 4) {
+            const float4 v = *reinterpret_cast<const float4 *>(o);
+            acc[0] = fmaf(wgt, v.x, acc[0]);
+            acc[1] = fmaf(wgt, v.y, acc[1]);
+            acc[2] = fmaf(wgt, v.z, acc[2]);
+            acc[3] = fmaf(wgt, v.w, acc[3]);
+        } else {
+            const float2 v = *reinterpret_cast<const float2 *>(o);
+            acc[0] = fmaf(wgt, v.x, acc[0]);
+            acc[1] = fmaf(wgt, v.y, acc[1]);
+        }
+    }
+    const float f = p.out_scale / wsum;
+    __half *op = p.out + ((size_t)s * p.num_heads + h) * D + lane * DPL;
+#pragma unroll
+    for (int e = 0; e < DPL; e += 2)
+        *reinterpret_cast<__half2 *>(op + e) = __floats2half2_rn(acc[e] * f, acc[e + 1] * f);
+}
+
+}  // namespace pa

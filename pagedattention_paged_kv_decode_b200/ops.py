@@ -1,0 +1,210 @@
+"""Torch-tensor binding of the C ABI: the same calls, argument marshalling only.
+
+Every function validates dtype/device/shape of the tensors it is given, then
+passes raw device pointers, sizes and the current CUDA stream to the
+library; all work runs in the library's CUDA kernels.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import capi
+from .capi import CacheDesc, DecodeConfig, check, lib
+
+_E4M3_DTYPES = (torch.uint8, torch.float8_e4m3fn)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def cache_desc(key_cache: torch.Tensor) -> CacheDesc:
+    if key_cache.dim() != 4:
+        raise ValueError("caches are [num_blocks, block_size, num_heads, head_size]")
+    if key_cache.dtype == torch.float16:
+        dt = capi.PA_F16
+    elif key_cache.dtype in _E4M3_DTYPES:
+        dt = capi.PA_E4M3
+    else:
+        raise TypeError(f"cache dtype {key_cache.dtype}: use float16, or uint8/float8_e4m3fn for E4M3")
+    nb, bs, nh, hd = key_cache.shape
+    return CacheDesc(nb, bs, nh, hd, dt)
+
+
+def _check_pair(key_cache, value_cache):
+    if key_cache.shape != value_cache.shape or key_cache.dtype != value_cache.dtype:
+        raise ValueError("key_cache and value_cache differ in shape or dtype")
+    for t in (key_cache, value_cache):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("caches must be contiguous CUDA tensors")
+
+
+def _i32(t: torch.Tensor, name: str) -> torch.Tensor:
+    if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous int32 CUDA tensor")
+    return t
+
+
+def slot_mapping(block_tables: torch.Tensor, context_lens: torch.Tensor, key_cache: torch.Tensor,
+                 out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Slot of each sequence's appended token (position context_len - 1)."""
+    _i32(block_tables, "block_tables")
+    _i32(context_lens, "context_lens")
+    S = context_lens.shape[0]
+    if out is None:
+        out = torch.empty(S, dtype=torch.int32, device=context_lens.device)
+    _i32(out, "out")
+    check(lib().pa_slot_mapping(out.data_ptr(), block_tables.data_ptr(), block_tables.shape[1],
+                                context_lens.data_ptr(), S, cache_desc(key_cache), _stream(stream)))
+    return out
+
+
+def kv_cache_write(key: torch.Tensor, value: torch.Tensor, key_cache: torch.Tensor,
+                   value_cache: torch.Tensor, slot_mapping: torch.Tensor,
+                   k_scale: float = 1.0, v_scale: float = 1.0, stream=None) -> None:
+    """Scatter new K/V rows ([n, H, D] fp16, row stride free) into their slots."""
+    _check_pair(key_cache, value_cache)
+    _i32(slot_mapping, "slot_mapping")
+    n = slot_mapping.shape[0]
+    for t in (key, value):
+        if t.dtype != torch.float16 or not t.is_cuda or t.dim() != 3 or t.shape[0] != n:
+            raise ValueError("key/value must be float16 CUDA tensors [n_tokens, H, D]")
+        if t.stride(2) != 1 or t.stride(1) != t.shape[2]:
+            raise ValueError("key/value rows must be contiguous within a token")
+    check(lib().pa_kv_cache_write(key.data_ptr(), value.data_ptr(), key.stride(0), value.stride(0),
+                                  key_cache.data_ptr(), value_cache.data_ptr(), cache_desc(key_cache),
+                                  slot_mapping.data_ptr(), n, float(k_scale), float(v_scale),
+                                  _stream(stream)))
+
+
+def copy_blocks(key_cache: torch.Tensor, value_cache: torch.Tensor, src_dst_pairs: torch.Tensor,
+                stream=None) -> None:
+    """Copy whole physical blocks (both caches) for each (src, dst) pair."""
+    _check_pair(key_cache, value_cache)
+    _i32(src_dst_pairs, "src_dst_pairs")
+    n = src_dst_pairs.numel() // 2
+    check(lib().pa_copy_blocks(key_cache.data_ptr(), value_cache.data_ptr(), cache_desc(key_cache),
+                               src_dst_pairs.data_ptr(), n, _stream(stream)))
+
+
+def _config(config) -> DecodeConfig | None:
+    if config is None:
+        return None
+    if isinstance(config, DecodeConfig):
+        return config
+    return DecodeConfig(**{k: int(config.get(k, 0)) for k, _ in DecodeConfig._fields_})
+
+
+def choose_config(key_cache: torch.Tensor, num_seqs: int, max_context_len: int, config=None) -> dict:
+    cfg = _config(config) or DecodeConfig(0, 0, 0, 0)
+    check(lib().pa_decode_choose_config(cache_desc(key_cache), num_seqs, max_context_len,
+                                        ctypes.byref(cfg)))
+    return cfg.as_dict()
+
+
+def decode_workspace_size(key_cache: torch.Tensor, num_seqs: int, max_context_len: int,
+                          config=None) -> int:
+    cfg = _config(config)
+    return int(lib().pa_decode_workspace_size(cache_desc(key_cache), num_seqs, max_context_len,
+                                              ctypes.byref(cfg) if cfg is not None else None))
+
+
+def paged_attention_decode(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
+                           value_cache: torch.Tensor, block_tables: torch.Tensor,
+                           context_lens: torch.Tensor, scale: float, k_scale: float = 1.0,
+                           v_scale: float = 1.0, max_context_len: int | None = None,
+                           config=None, workspace: torch.Tensor | None = None, stream=None) -> None:
+    """Decode attention into ``out`` ([S, H, D] fp16).
+
+    ``max_context_len`` is a host-side bound on every context length; by
+    default the table capacity ``block_tables.shape[1] * block_size`` (no
+    device sync). With ``config`` or ``workspace`` given, the caller-workspace
+    entry point is used (``workspace`` a uint8 CUDA tensor of at least
+    ``decode_workspace_size`` bytes).
+    """
+    _check_pair(key_cache, value_cache)
+    _i32(block_tables, "block_tables")
+    _i32(context_lens, "context_lens")
+    for t in (out, query):
+        if t.dtype != torch.float16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("out and query must be contiguous float16 CUDA tensors")
+    S, H, D = query.shape
+    if out.shape != query.shape or context_lens.shape[0] != S or block_tables.shape[0] != S:
+        raise ValueError("shape mismatch between out, query, block_tables and context_lens")
+    desc = cache_desc(key_cache)
+    if desc.num_heads != H or desc.head_size != D:
+        raise ValueError("query heads/head_size differ from the cache's")
+    if max_context_len is None:
+        max_context_len = block_tables.shape[1] * desc.block_size
+    args = (out.data_ptr(), query.data_ptr(), key_cache.data_ptr(), value_cache.data_ptr(), desc,
+            block_tables.data_ptr(), block_tables.shape[1], context_lens.data_ptr(), S,
+            int(max_context_len), float(scale), float(k_scale), float(v_scale))
+    if config is None and workspace is None:
+        check(lib().pa_paged_attention_decode(*args, _stream(stream)))
+        return
+    cfg = _config(config)
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        if not workspace.is_cuda or not workspace.is_contiguous():
+            raise ValueError("workspace must be a contiguous CUDA tensor")
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    check(lib().pa_paged_attention_decode_ws(*args, ctypes.byref(cfg) if cfg is not None else None,
+                                             ws_ptr, ws_bytes, _stream(stream)))
+
+
+def check_status(stream=None) -> int:
+    """Synchronise the stream; return and clear the device error bits (PA_DEV_*)."""
+    code = ctypes.c_uint32(0)
+    check(lib().pa_check_status(_stream(stream), ctypes.byref(code)))
+    return int(code.value)
+
+
+def version() -> int:
+    return int(lib().pa_version())
+
+
+def load_cache(key_cache: torch.Tensor, value_cache: torch.Tensor, key_src: torch.Tensor,
+               value_src: torch.Tensor, k_scale: float = 1.0, v_scale: float = 1.0,
+               stream=None) -> None:
+    """Write whole fp16 pools [NB, B, H, D] into the caches, slot by slot.
+
+    This is ``kv_cache_write`` with the identity slot list, in calls of at
+    most 65535 tokens; for E4M3 caches it quantises with the given scales.
+    """
+    _check_pair(key_cache, value_cache)
+    nb, bs, nh, hd = key_cache.shape
+    if key_src.shape != key_cache.shape or value_src.shape != key_cache.shape:
+        raise ValueError("source pools must have the cache's shape")
+    n = nb * bs
+    ks = key_src.reshape(n, nh, hd)
+    vs = value_src.reshape(n, nh, hd)
+    chunk = 65535
+    slots = torch.arange(min(n, chunk), dtype=torch.int32, device=key_cache.device)
+    for i in range(0, n, chunk):
+        m = min(chunk, n - i)
+        kv_cache_write(ks[i:i + m], vs[i:i + m], key_cache, value_cache, slots[:m] + i,
+                       k_scale, v_scale, stream)
+
+
+def decode_step(out: torch.Tensor, query: torch.Tensor, new_key: torch.Tensor,
+                new_value: torch.Tensor, key_cache: torch.Tensor, value_cache: torch.Tensor,
+                block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
+                k_scale: float = 1.0, v_scale: float = 1.0, cow_pairs: torch.Tensor | None = None,
+                slots: torch.Tensor | None = None, max_context_len: int | None = None,
+                config=None, workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """One decode step of the whole path, all on the device, in order:
+    copy-on-write block copies (if any pairs), slot of each appended token,
+    scatter of the new K/V rows into those slots, decode attention.
+    ``block_tables`` are the tables after any copy-on-write repoint.
+    Returns the slot tensor."""
+    if cow_pairs is not None and cow_pairs.numel():
+        copy_blocks(key_cache, value_cache, cow_pairs, stream)
+    slots = slot_mapping(block_tables, context_lens, key_cache, out=slots, stream=stream)
+    kv_cache_write(new_key, new_value, key_cache, value_cache, slots, k_scale, v_scale, stream)
+    paged_attention_decode(out, query, key_cache, value_cache, block_tables, context_lens, scale,
+                           k_scale, v_scale, max_context_len, config, workspace, stream)
+    return slots

@@ -1,0 +1,132 @@
+"""Host-side checks of the C ABI (no GPU): the library loads, exports every
+symbol that include/pagedkv.h declares, and rejects bad arguments before any
+CUDA call (so these run on a machine without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from pagedattention_paged_kv_decode_b200 import capi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pagedkv.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_path_calls():
+    names = declared_functions()
+    for n in ("pa_kv_cache_write", "pa_paged_attention_decode", "pa_copy_blocks", "pa_slot_mapping",
+              "pa_paged_attention_decode_ws", "pa_check_status", "pa_last_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(capi.LIB)
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+    assert set(declared_functions()) == set(capi.SIGNATURES)
+
+
+def test_version_and_empty_error():
+    assert capi.lib().pa_version() == 100
+
+
+F = capi.CacheDesc(64, 16, 8, 128, capi.PA_F16)
+P = 0x10000  # fake, 16-byte aligned "device" address: validation fails before any use
+
+
+def _last():
+    return capi.lib().pa_last_error().decode()
+
+
+@pytest.mark.parametrize("desc,code", [
+    (capi.CacheDesc(64, 16, 8, 128, 7), capi.PA_ERR_DTYPE),
+    (capi.CacheDesc(64, 8, 8, 128, 0), capi.PA_ERR_INVALID),
+    (capi.CacheDesc(64, 16, 8, 96, 0), capi.PA_ERR_INVALID),
+    (capi.CacheDesc(0, 16, 8, 128, 0), capi.PA_ERR_INVALID),
+    (capi.CacheDesc(1 << 27, 16, 8, 128, 0), capi.PA_ERR_OVERFLOW),
+])
+def test_bad_cache_descriptors(desc, code):
+    L = capi.lib()
+    assert L.pa_kv_cache_write(P, P, 1024, 1024, P, P, desc, P, 4, 1.0, 1.0, None) == code
+    assert _last()
+    assert L.pa_copy_blocks(P, P, desc, P, 4, None) == code
+    assert L.pa_slot_mapping(P, P, 4, P, 4, desc, None) == code
+    assert L.pa_paged_attention_decode(P, P, P, P, desc, P, 4, P, 4, 64, 0.1, 1.0, 1.0, None) == code
+
+
+def test_null_and_misaligned_pointers():
+    L = capi.lib()
+    assert L.pa_kv_cache_write(None, P, 1024, 1024, P, P, F, P, 4, 1.0, 1.0, None) == capi.PA_ERR_INVALID
+    assert L.pa_kv_cache_write(P + 2, P, 1024, 1024, P, P, F, P, 4, 1.0, 1.0, None) == capi.PA_ERR_INVALID
+    assert "aligned" in _last()
+    assert L.pa_kv_cache_write(P, P, 1020, 1024, P, P, F, P, 4, 1.0, 1.0, None) == capi.PA_ERR_INVALID
+    assert L.pa_copy_blocks(P, None, F, P, 4, None) == capi.PA_ERR_INVALID
+    assert L.pa_paged_attention_decode(P, P + 8, P, P, F, P, 4, P, 4, 64, 0.1, 1.0, 1.0, None) == capi.PA_ERR_INVALID
+    assert L.pa_paged_attention_decode(P, P, P, P, F, None, 4, P, 4, 64, 0.1, 1.0, 1.0, None) == capi.PA_ERR_INVALID
+
+
+def test_bad_scales_and_counts():
+    L = capi.lib()
+    E = capi.CacheDesc(64, 16, 8, 128, capi.PA_E4M3)
+    assert L.pa_kv_cache_write(P, P, 1024, 1024, P, P, E, P, 4, 0.0, 1.0, None) == capi.PA_ERR_INVALID
+    assert L.pa_paged_attention_decode(P, P, P, P, E, P, 4, P, 4, 64, 0.1, 1.0, float("nan"), None) == capi.PA_ERR_INVALID
+    assert L.pa_paged_attention_decode(P, P, P, P, F, P, 4, P, 4, 64, float("inf"), 1.0, 1.0, None) == capi.PA_ERR_INVALID
+    assert L.pa_paged_attention_decode(P, P, P, P, F, P, 0, P, 4, 64, 0.1, 1.0, 1.0, None) == capi.PA_ERR_INVALID
+    assert L.pa_paged_attention_decode(P, P, P, P, F, P, 4, P, -1, 64, 0.1, 1.0, 1.0, None) == capi.PA_ERR_INVALID
+    assert L.pa_kv_cache_write(P, P, 1024, 1024, P, P, F, P, -3, 1.0, 1.0, None) == capi.PA_ERR_INVALID
+    # zero-sized work is a no-op that launches nothing
+    assert L.pa_kv_cache_write(P, P, 1024, 1024, P, P, F, P, 0, 1.0, 1.0, None) == capi.PA_OK
+    assert L.pa_copy_blocks(P, P, F, P, 0, None) == capi.PA_OK
+    assert L.pa_slot_mapping(P, P, 4, P, 0, F, None) == capi.PA_OK
+    assert L.pa_paged_attention_decode(P, P, P, P, F, P, 4, P, 0, 64, 0.1, 1.0, 1.0, None) == capi.PA_OK
+
+
+def _choose(desc, S, maxL, **kw):
+    cfg = capi.DecodeConfig(kw.get("partition_size", 0), kw.get("heads_per_cta", 0),
+                            kw.get("warps_per_head", 0), kw.get("stages", 0))
+    rc = capi.lib().pa_decode_choose_config(desc, S, maxL, ctypes.byref(cfg))
+    return rc, cfg
+
+
+def test_config_choice_is_valid_and_fills_the_gpu():
+    for desc, S, maxL in [(capi.CacheDesc(2048, 16, 32, 128, 0), 16, 192),
+                          (capi.CacheDesc(16384, 16, 40, 128, 0), 64, 2048),
+                          (capi.CacheDesc(700, 32, 32, 128, 0), 32, 4096),
+                          (capi.CacheDesc(13600, 16, 32, 128, 1), 256, 4096),
+                          (capi.CacheDesc(32, 16, 4, 64, 0), 4, 64)]:
+        rc, cfg = _choose(desc, S, maxL)
+        assert rc == capi.PA_OK, _last()
+        assert cfg.partition_size % desc.block_size == 0
+        assert desc.num_heads % cfg.heads_per_cta == 0
+        units = S * (desc.num_heads // cfg.heads_per_cta) * -(-maxL // cfg.partition_size)
+        assert units >= 3 * 148 or cfg.heads_per_cta == 1
+
+
+def test_config_validation_and_workspace_size():
+    desc = capi.CacheDesc(2048, 16, 32, 128, 0)
+    assert _choose(desc, 16, 512, partition_size=24)[0] == capi.PA_ERR_INVALID
+    assert _choose(desc, 16, 512, heads_per_cta=3)[0] == capi.PA_ERR_INVALID
+    assert _choose(desc, 16, 512, heads_per_cta=8, warps_per_head=4)[0] == capi.PA_ERR_INVALID  # 32 warps
+    assert _choose(desc, 16, 512, stages=9)[0] == capi.PA_ERR_INVALID
+    assert _choose(desc, 16, 512, heads_per_cta=8, stages=8)[0] == capi.PA_ERR_INVALID  # smem > 227 KB
+    rc, cfg = _choose(desc, 16, 512, partition_size=128, heads_per_cta=2, warps_per_head=2, stages=4)
+    assert rc == 0
+    L = capi.lib()
+    ws = L.pa_decode_workspace_size(desc, 16, 512, ctypes.byref(cfg))
+    lse = -(-(16 * 32 * 4 * 4) // 256) * 256
+    assert ws == lse + 16 * 32 * 4 * 128 * 4
+    one = capi.DecodeConfig(512, 2, 2, 4)
+    assert L.pa_decode_workspace_size(desc, 16, 512, ctypes.byref(one)) == 0
+    small = L.pa_paged_attention_decode_ws(P, P, P, P, desc, P, 32, P, 16, 512, 0.1, 1.0, 1.0,
+                                           ctypes.byref(cfg), P, ws - 1, None)
+    assert small == capi.PA_ERR_WORKSPACE
+    unaligned = L.pa_paged_attention_decode_ws(P, P, P, P, desc, P, 32, P, 16, 512, 0.1, 1.0, 1.0,
+                                               ctypes.byref(cfg), P + 16, ws, None)
+    assert unaligned == capi.PA_ERR_WORKSPACE

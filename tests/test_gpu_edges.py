@@ -1,0 +1,135 @@
+"""GPU edge cases: device-side bounds checks (error word, no fault), copy-on-write
+semantics, strided new-token rows, empty batches."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import pagedattention_paged_kv_decode_b200 as pk
+from pagedattention_paged_kv_decode_b200 import capi
+import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+def small(dev, kv="f16", ctx=(5, 40, 17), B=16, H=2, D=128, seed=1):
+    w = W.build("edge", H, D, B, kv, list(ctx), 20, 4, seed, q_std=1.0, kv_std=1.0)
+    return w, W.to_device(w, dev, encode=pk.load_cache)
+
+
+def test_slot_beyond_pool_is_skipped_and_flagged(cuda_device):
+    w, dw = small(cuda_device)
+    before = dw.key_cache.clone()
+    slots = torch.tensor([3, 20 * 16, 7], dtype=torch.int32, device=cuda_device)
+    pk.kv_cache_write(dw.new_key, dw.new_value, dw.key_cache, dw.value_cache, slots)
+    assert pk.check_status() == capi.PA_DEV_BAD_SLOT
+    assert pk.check_status() == 0                       # read clears
+    after = dw.key_cache
+    assert torch.equal(after[0, 3], dw.new_key[0]) and torch.equal(after[0, 7], dw.new_key[2])
+    mask = torch.ones(20, 16, dtype=torch.bool)
+    mask[0, 3] = mask[0, 7] = False
+    assert torch.equal(after.cpu()[mask], before.cpu()[mask])
+
+
+def test_bad_block_ids_read_as_zero_rows_and_flag(cuda_device):
+    w, dw = small(cuda_device)
+    bt = dw.block_tables.clone()
+    bt[1, 1] = 20 + 5
+    bt[2, 0] = -3
+    pk.paged_attention_decode(dw.out, dw.query, dw.key_cache, dw.value_cache, bt, dw.context_lens,
+                              w.scale, max_context_len=64)
+    assert pk.check_status() == capi.PA_DEV_BAD_BLOCK
+    assert torch.isfinite(dw.out.float()).all()
+    assert pk.check_status() == 0
+    pk.slot_mapping(bt, dw.context_lens, dw.key_cache, out=dw.slots)
+    assert pk.check_status() == capi.PA_DEV_BAD_BLOCK   # seq 1 appends into logical block 2: fine; seq 2 -> -3
+    assert dw.slots.cpu().tolist()[2] == -1
+
+
+def test_context_beyond_table_and_bound_are_clamped_and_flagged(cuda_device):
+    w, dw = small(cuda_device)
+    ctx = dw.context_lens.clone()
+    ctx[0] = 4 * 16 + 9                                  # table holds 4 blocks
+    pk.paged_attention_decode(dw.out, dw.query, dw.key_cache, dw.value_cache, dw.block_tables, ctx,
+                              w.scale)
+    assert pk.check_status() & capi.PA_DEV_CTX_OVER_TABLE
+    pk.slot_mapping(dw.block_tables, ctx, dw.key_cache, out=dw.slots)
+    assert pk.check_status() == capi.PA_DEV_CTX_OVER_TABLE
+    pk.paged_attention_decode(dw.out, dw.query, dw.key_cache, dw.value_cache, dw.block_tables,
+                              dw.context_lens, w.scale, max_context_len=20)
+    assert pk.check_status() == capi.PA_DEV_CTX_OVER_BOUND
+
+
+def test_bad_copy_pair_is_skipped_and_flagged(cuda_device):
+    w, dw = small(cuda_device)
+    before = dw.key_cache.clone()
+    pairs = torch.tensor([[2, 19], [1, 99]], dtype=torch.int32, device=cuda_device)
+    pk.copy_blocks(dw.key_cache, dw.value_cache, pairs)
+    assert pk.check_status() == capi.PA_DEV_BAD_PAIR
+    assert torch.equal(dw.key_cache[19], before[2])
+    before[19] = before[2]
+    assert torch.equal(dw.key_cache, before)
+
+
+def test_copy_on_write_keeps_sharers_independent(cuda_device):
+    """Two sequences share a prefix block; the first one appends into it after
+    a copy ("在A10G上榨干LLaMA-7B" §2.2): the sharer's output and the shared
+    block must not change, and the writer must see its new token. The
+    expected pools and outputs come from the oracle's own steps on the host."""
+    B, H, D = 16, 2, 64
+    w = W.build("cow", H, D, B, "f16", [12, 12], 8, 2, 3, q_std=1.0, kv_std=1.0,
+                deal_order="identity")
+    dw = W.to_device(w, cuda_device)
+    kc, vc = w.pool_host()
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(cuda_device)
+    # both sequences read block 0 (tokens 0..10 present); seq 1's own block 1 is unused
+    bt = np.array([[0, -1], [0, -1]], np.int32)
+    ctx = np.array([11, 11], np.int32)
+    out0 = torch.empty_like(dw.query)
+    pk.paged_attention_decode(out0, dw.query, dw.key_cache, dw.value_cache, dev(bt), dev(ctx), w.scale)
+    # seq 0 appends token 11: copy block 0 -> 5, repoint its table, write into block 5
+    pairs = np.array([[0, 5]], np.int32)
+    bt2 = np.array([[5, -1], [0, -1]], np.int32)
+    ctx2 = np.array([12, 11], np.int32)
+    pk.copy_blocks(dw.key_cache, dw.value_cache, dev(pairs))
+    slots = pk.slot_mapping(dev(bt2), dev(ctx2), dw.key_cache)
+    pk.kv_cache_write(dw.new_key[:1], dw.new_value[:1], dw.key_cache, dw.value_cache, slots[:1])
+    out1 = torch.empty_like(dw.query)
+    pk.paged_attention_decode(out1, dw.query, dw.key_cache, dw.value_cache, dev(bt2), dev(ctx2), w.scale)
+    assert pk.check_status() == 0
+    ref_slots = oracle.slot_mapping(bt2, ctx2, B)
+    assert slots.cpu().tolist() == ref_slots.tolist() == [5 * 16 + 11, 0 * 16 + 10]
+    shared = kc[0].copy()
+    oracle.copy_blocks(kc, vc, pairs)
+    oracle.kv_cache_write(w.new_key[:1], w.new_value[:1], kc, vc, ref_slots[:1])
+    assert np.array_equal(kc[0], shared)
+    assert np.array_equal(dw.key_cache.cpu().numpy().view(np.uint16), kc.view(np.uint16))
+    assert np.array_equal(dw.value_cache.cpu().numpy().view(np.uint16), vc.view(np.uint16))
+    assert torch.equal(out1[1], out0[1])
+    ref = oracle.paged_attention(w.query, kc, vc, bt2, ctx2, w.scale)
+    assert np.abs(out1.cpu().numpy().astype(np.float64) - ref).max() <= 2e-3
+    assert not torch.equal(out1[0], out0[0])
+
+
+def test_strided_rows_from_a_fused_qkv_buffer(cuda_device):
+    S, H, D, B = 5, 4, 64, 16
+    h = np.random.default_rng(4).standard_normal((S, 3, H, D)).astype(np.float16)
+    qkv = torch.from_numpy(h).to(cuda_device)
+    kc = torch.zeros(4, B, H, D, dtype=torch.float16, device=cuda_device)
+    vc = torch.zeros_like(kc)
+    slots = torch.tensor([0, 17, -1, 33, 63], dtype=torch.int32, device=cuda_device)
+    pk.kv_cache_write(qkv[:, 1], qkv[:, 2], kc, vc, slots)
+    rk = np.zeros((4, B, H, D), np.float16)
+    rv = np.zeros_like(rk)
+    oracle.kv_cache_write(h[:, 1], h[:, 2], rk, rv, slots.cpu().numpy())
+    assert np.array_equal(kc.cpu().numpy().view(np.uint16), rk.view(np.uint16))
+    assert np.array_equal(vc.cpu().numpy().view(np.uint16), rv.view(np.uint16))
+
+
+def test_empty_batch_is_a_no_op(cuda_device):
+    kc = torch.zeros(4, 16, 2, 64, dtype=torch.float16, device=cuda_device)
+    e = torch.empty(0, 2, 64, dtype=torch.float16, device=cuda_device)
+    pk.paged_attention_decode(e, e, kc, kc.clone(), torch.empty(0, 1, dtype=torch.int32, device=cuda_device),
+                              torch.empty(0, dtype=torch.int32, device=cuda_device), 0.125)
+    pk.kv_cache_write(e, e, kc, kc.clone(), torch.empty(0, dtype=torch.int32, device=cuda_device))
+    assert pk.check_status() == 0

@@ -284,3 +284,47 @@ def named(config_id: int, seed: int | None = None, poison: str = POISON_HUGE) ->
 def rank_seed(seed: int, rank: int) -> int:
     """Seed of rank ``rank``'s independent batch in a multi-GPU run."""
     return seed + 7919 * rank
+
+
+@dataclass
+class DeviceWorkload:
+    """A workload's tensors on a CUDA device (torch), ready for one decode step."""
+    w: Workload
+    query: object
+    new_key: object
+    new_value: object
+    block_tables: object
+    context_lens: object
+    cow_pairs: object
+    key_cache: object
+    value_cache: object
+    out: object
+    slots: object
+
+
+def to_device(w: Workload, device, encode=None) -> DeviceWorkload:
+    """Upload a workload. fp16 caches are the pools as drawn; E4M3 caches are
+    produced by ``encode(key_cache, value_cache, key_src, value_src, k_scale,
+    v_scale)``, which the caller supplies (the library's bulk cache write)."""
+    import torch
+
+    def up(a):
+        return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+    pk, pv = w.pool_device(device)
+    if w.kv_dtype == "e4m3":
+        if encode is None:
+            raise ValueError("E4M3 workloads need an encode callable")
+        kc = torch.empty(pk.shape, dtype=torch.uint8, device=device)
+        vc = torch.empty(pv.shape, dtype=torch.uint8, device=device)
+        encode(kc, vc, pk, pv, w.k_scale, w.v_scale)
+        del pk, pv
+    else:
+        kc, vc = pk, pv
+    S, H, D = w.query.shape
+    return DeviceWorkload(
+        w=w, query=up(w.query), new_key=up(w.new_key), new_value=up(w.new_value),
+        block_tables=up(w.block_tables), context_lens=up(w.context_lens),
+        cow_pairs=up(w.cow_pairs.astype(np.int32)), key_cache=kc, value_cache=vc,
+        out=torch.empty((S, H, D), dtype=torch.float16, device=device),
+        slots=torch.empty(S, dtype=torch.int32, device=device))
