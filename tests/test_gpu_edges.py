@@ -34,15 +34,15 @@ def test_slot_beyond_pool_is_skipped_and_flagged(cuda_device):
 def test_bad_block_ids_read_as_zero_rows_and_flag(cuda_device):
     w, dw = small(cuda_device)
     bt = dw.block_tables.clone()
-    bt[1, 1] = 20 + 5
-    bt[2, 0] = -3
+    bt[1, 1] = 20 + 5            # seq 1 (L=40) reads logical blocks 0..2
+    bt[2, 1] = -3                # seq 2 (L=17) reads logical blocks 0..1 and appends into block 1
     pk.paged_attention_decode(dw.out, dw.query, dw.key_cache, dw.value_cache, bt, dw.context_lens,
                               w.scale, max_context_len=64)
     assert pk.check_status() == capi.PA_DEV_BAD_BLOCK
     assert torch.isfinite(dw.out.float()).all()
     assert pk.check_status() == 0
     pk.slot_mapping(bt, dw.context_lens, dw.key_cache, out=dw.slots)
-    assert pk.check_status() == capi.PA_DEV_BAD_BLOCK   # seq 1 appends into logical block 2: fine; seq 2 -> -3
+    assert pk.check_status() == capi.PA_DEV_BAD_BLOCK   # seq 2 appends into logical block 1 (-3)
     assert dw.slots.cpu().tolist()[2] == -1
 
 
