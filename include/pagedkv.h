@@ -193,6 +193,30 @@ int pa_paged_attention_decode_ws(void *out, const void *query,
                                  const pa_decode_config *cfg, void *workspace,
                                  size_t workspace_bytes, void *stream);
 
+/* pa_paged_attention_decode for callers that cannot allocate device memory.
+ * The paper has no counterpart to this call: it exists for callers such as
+ * engine plugins whose host framework owns all device memory, code running
+ * under CUDA stream capture, or loops with a fixed memory plan, none of which
+ * may call cudaMalloc or an allocating library on this path. Arguments,
+ * results and errors are those of pa_paged_attention_decode (library-chosen
+ * launch shape); the split partials go to a static device array of 16 MiB
+ * inside the library instead of a workspace, and the call allocates nothing.
+ *   - Limit: a decode whose partials exceed 16 MiB (pa_decode_workspace_size
+ *     with cfg NULL) returns PA_ERR_WORKSPACE before launching anything.
+ *   - The array is held by every GPU that loads the library until exit.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents; nothing in it has to start at zero (each partial is written
+ *     before it is read). Calls whose kernels may overlap on the GPU (other
+ *     streams, other threads) race on it: serialise them. */
+int pa_paged_attention_decode_noalloc(void *out, const void *query,
+                                      const void *key_cache, const void *value_cache,
+                                      pa_cache_desc cache, const int32_t *block_tables,
+                                      int max_blocks_per_seq, const int32_t *context_lens,
+                                      int num_seqs, int max_context_len, float scale,
+                                      float k_scale, float v_scale, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -530,3 +530,78 @@ int pa_paged_attention_decode_ws(void *out, const void *query, const void *key_c
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode for callers that may not allocate device memory at all.
+//
+// Some callers cannot call cudaMalloc (or any allocator) on the path that
+// runs the decode: engine plugins whose host framework owns every device
+// buffer and forbids allocation during execution, code that runs while a
+// CUDA graph is being captured (an allocation there becomes part of the
+// graph), and real-time loops with a fixed, pre-planned memory budget. The
+// split-context partials of such a call live in the file-scope array below
+// instead of a workspace. The array is part of the library's device image:
+// every GPU that loads the library holds its kDecodeScratchBytes until the
+// process exits.
+namespace {
+
+constexpr size_t kDecodeScratchBytes = size_t(16) << 20;  // 16 MiB per device
+
+static __device__ __align__(256) unsigned char g_decode_scratch[kDecodeScratchBytes];
+
+std::mutex g_scratch_mu;
+constexpr int kMaxDevices = 128;
+void *g_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_decode_scratch on the current device. In host code the
+// array's name is only a host-side stand-in, so its address is looked up once
+// per device with cudaGetSymbolAddress and cached.
+int scratch_address(int device, void **out) {
+    if (device < 0 || device >= kMaxDevices)
+        return fail(PA_ERR_INVALID, "device ordinal %d out of range", device);
+    std::lock_guard<std::mutex> lk(g_scratch_mu);
+    if (!g_scratch_addr[device]) {
+        void *p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress (static decode scratch)");
+        g_scratch_addr[device] = p;
+    }
+    *out = g_scratch_addr[device];
+    return PA_OK;
+}
+
+}  // namespace
+
+extern "C" int pa_paged_attention_decode_noalloc(
+    void *out, const void *query, const void *key_cache, const void *value_cache,
+    pa_cache_desc cache, const int32_t *block_tables, int max_blocks_per_seq,
+    const int32_t *context_lens, int num_seqs, int max_context_len, float scale, float k_scale,
+    float v_scale, void *stream) {
+    int rc = check_decode_args(out, query, key_cache, value_cache, cache, block_tables,
+                               max_blocks_per_seq, context_lens, num_seqs, max_context_len, scale,
+                               k_scale, v_scale);
+    if (rc) return rc;
+    if (num_seqs == 0) return ok();
+    const int bound =
+        (int)std::min<int64_t>(max_context_len, (int64_t)max_blocks_per_seq * cache.block_size);
+    pa_decode_config cfg{0, 0, 0, 0};
+    rc = fill_config(cache, num_seqs, bound, &cfg);
+    if (rc) return rc;
+    const size_t need = ws_bytes(cache, num_seqs, bound, cfg);
+    if (need > kDecodeScratchBytes)
+        return fail(PA_ERR_WORKSPACE,
+                    "this decode needs %zu bytes of split scratch but the static scratch of "
+                    "pa_paged_attention_decode_noalloc holds %zu; lower num_seqs or "
+                    "max_context_len, or call pa_paged_attention_decode_ws",
+                    need, kDecodeScratchBytes);
+    int dev = 0;
+    rc = current_device(&dev);
+    if (rc) return rc;
+    void *scratch = nullptr;
+    rc = scratch_address(dev, &scratch);  // first call on a device: symbol lookup
+    if (rc) return rc;
+    return launch_decode(out, query, key_cache, value_cache, cache, block_tables,
+                         max_blocks_per_seq, context_lens, num_seqs, bound, scale, k_scale,
+                         v_scale, cfg, need ? scratch : nullptr, static_cast<cudaStream_t>(stream),
+                         dev);
+}
