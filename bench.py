@@ -152,9 +152,14 @@ def run_ours(args, rank, world, local_rank):
     dw = W.to_device(w, dev, encode=pk.load_cache)
     S = w.num_seqs
     bound = w.max_blocks_per_seq * w.block_size  # host-side bound: table capacity, no sync
-    cfg = pk.choose_config(dw.key_cache, S, bound)
+    launch = None
+    if args.launch:
+        launch = dict(zip(("partition_size", "heads_per_cta", "warps_per_head", "stages"),
+                          (int(x) for x in args.launch.split(","))))
+    cfg = pk.choose_config(dw.key_cache, S, bound, launch)
     parts = -(-bound // cfg["partition_size"])
-    launches_per_step = 3 + (1 if w.cow_pairs.size else 0) + (1 if parts > 1 else 0)
+    launches_per_step = ((3 if args.unfused else 1) + (1 if w.cow_pairs.size else 0)
+                         + (1 if parts > 1 else 0))
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     stream = torch.cuda.Stream(dev)
@@ -164,13 +169,21 @@ def run_ours(args, rank, world, local_rank):
         ev[0].record()
         if w.cow_pairs.size:
             pk.copy_blocks(dw.key_cache, dw.value_cache, dw.cow_pairs)
-        pk.slot_mapping(dw.block_tables, dw.context_lens, dw.key_cache, out=dw.slots)
-        pk.kv_cache_write(dw.new_key, dw.new_value, dw.key_cache, dw.value_cache, dw.slots,
-                          w.k_scale, w.v_scale)
-        ev[1].record()
-        pk.paged_attention_decode(dw.out, dw.query, dw.key_cache, dw.value_cache,
-                                  dw.block_tables, dw.context_lens, w.scale, w.k_scale,
-                                  w.v_scale, max_context_len=bound)
+        if args.unfused:
+            pk.slot_mapping(dw.block_tables, dw.context_lens, dw.key_cache, out=dw.slots)
+            pk.kv_cache_write(dw.new_key, dw.new_value, dw.key_cache, dw.value_cache, dw.slots,
+                              w.k_scale, w.v_scale)
+            ev[1].record()
+            pk.paged_attention_decode(dw.out, dw.query, dw.key_cache, dw.value_cache,
+                                      dw.block_tables, dw.context_lens, w.scale, w.k_scale,
+                                      w.v_scale, max_context_len=bound)
+        else:
+            ev[1].record()
+            pk.paged_attention_decode_append(dw.out, dw.query, dw.new_key, dw.new_value,
+                                             dw.key_cache, dw.value_cache, dw.block_tables,
+                                             dw.context_lens, w.scale, w.k_scale, w.v_scale,
+                                             max_context_len=bound, slot_mapping=dw.slots,
+                                             config=launch)
         ev[2].record()
 
     with torch.cuda.stream(stream):
@@ -245,7 +258,7 @@ def run_ours(args, rank, world, local_rank):
 
     kv = w.kv_bytes()
     peak, peak_kind = hbm_peak()
-    dec_bytes = w.decode_bytes()
+    dec_bytes = w.decode_bytes() if args.unfused else W.fused_step_bytes(w)
     achieved = dec_bytes / (dec_t * 1e-3) / 1e9
     value = aggregate_gbs(world, kv, step_t)
     line = {
@@ -270,7 +283,8 @@ def run_ours(args, rank, world, local_rank):
             "launch": cfg, "parallelism": f"replicas x{world} (independent batches, no collective)",
             "l2": "512 MiB buffer written before every timed step (L2 is 126 MB)",
             "step": "CUDA graph: " + ("copy_blocks, " if w.cow_pairs.size else "")
-                    + "slot_mapping, kv_cache_write, paged_attention_decode"
+                    + ("slot_mapping, kv_cache_write, paged_attention_decode" if args.unfused
+                       else "paged_attention_decode_append (slot + K/V store + decode in one launch)")
                     + (" (+lse reduce)" if parts > 1 else ""),
         },
         "tokens_per_s": round(world * S / (step_t * 1e-3), 1),
@@ -282,7 +296,8 @@ def run_ours(args, rank, world, local_rank):
             "bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} copy bandwidth",
             "traffic": recorded_traffic(w.name),
-            "kernel": "paged_decode_kernel" + (" + lse_reduce_kernel" if parts > 1 else ""),
+            "kernel": "paged_decode_kernel" + ("" if args.unfused else " (fused append)")
+                      + (" + lse_reduce_kernel" if parts > 1 else ""),
             "algorithmic_bytes_per_launch": dec_bytes,
         },
         "e2e": {"value": round(aggregate_gbs(world, kv, e2e_t), 2), "unit": "GB/s",
@@ -380,6 +395,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--unfused", action="store_true",
+                    help="slot mapping, cache write and decode as three launches")
+    ap.add_argument("--launch", default="",
+                    help="decode launch shape partition_size,heads_per_cta,warps_per_head,stages")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -193,6 +193,31 @@ int pa_paged_attention_decode_ws(void *out, const void *query,
                                  const pa_decode_config *cfg, void *workspace,
                                  size_t workspace_bytes, void *stream);
 
+/* Fused append + decode ([P1] §3.2 fused kernels): one launch (plus the
+ * log-sum-exp reduce when a context is split) performs, for every sequence,
+ * the slot derivation of pa_slot_mapping, the store of pa_kv_cache_write for
+ * its new token (fp16 copy or E4M3 encode with k_scale/v_scale), and the
+ * decode of pa_paged_attention_decode over all L tokens including the new
+ * one. The CTA that owns a sequence's last partition stores the new rows of
+ * its heads before it loads the block holding them.
+ *   new_key/new_value: fp16 [num_seqs][num_heads][head_size], row stride
+ *       key_stride/value_stride elements (multiples of 8), 16-byte aligned.
+ *   slot_mapping_out: int32 [num_seqs] receiving each sequence's slot (-1
+ *       when L <= 0, the context is clamped, or the block id is invalid), or
+ *       NULL. Sequences with L <= 0 write nothing.
+ *   cfg / workspace: as in pa_paged_attention_decode_ws; workspace NULL =
+ *       the library-owned workspace of pa_paged_attention_decode.
+ * Results equal pa_slot_mapping + pa_kv_cache_write + the decode, in order. */
+int pa_paged_attention_decode_append(void *out, const void *query, const void *new_key,
+                                     const void *new_value, int64_t key_stride,
+                                     int64_t value_stride, void *key_cache, void *value_cache,
+                                     pa_cache_desc cache, const int32_t *block_tables,
+                                     int max_blocks_per_seq, const int32_t *context_lens,
+                                     int num_seqs, int max_context_len, float scale,
+                                     float k_scale, float v_scale, int32_t *slot_mapping_out,
+                                     const pa_decode_config *cfg, void *workspace,
+                                     size_t workspace_bytes, void *stream);
+
 /* pa_paged_attention_decode for callers that cannot allocate device memory.
  * The paper has no counterpart to this call: it exists for callers such as
  * engine plugins whose host framework owns all device memory, code running

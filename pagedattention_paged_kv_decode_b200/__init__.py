@@ -16,6 +16,7 @@ from .ops import (  # noqa: F401
     kv_cache_write,
     load_cache,
     paged_attention_decode,
+    paged_attention_decode_append,
     slot_mapping,
     version,
 )

@@ -59,6 +59,9 @@ SIGNATURES = {
     "pa_decode_workspace_size": (ctypes.c_size_t, [CacheDesc, _I, _I, ctypes.POINTER(DecodeConfig)]),
     "pa_paged_attention_decode_ws": (_I, [_P, _P, _P, _P, CacheDesc, _P, _I, _P, _I, _I, _F, _F, _F,
                                           ctypes.POINTER(DecodeConfig), _P, ctypes.c_size_t, _P]),
+    "pa_paged_attention_decode_append": (_I, [_P, _P, _P, _P, _I64, _I64, _P, _P, CacheDesc, _P, _I, _P,
+                                              _I, _I, _F, _F, _F, _P, ctypes.POINTER(DecodeConfig),
+                                              _P, ctypes.c_size_t, _P]),
     "pa_paged_attention_decode_noalloc": (_I, [_P, _P, _P, _P, CacheDesc, _P, _I, _P, _I, _I, _F, _F,
                                                _F, _P]),
 }

@@ -285,10 +285,19 @@ int check_decode_args(void *out, const void *query, const void *kc, const void *
     return PA_OK;
 }
 
+struct AppendArgs {
+    const void *new_key;
+    const void *new_value;
+    int64_t key_stride;
+    int64_t value_stride;
+    int32_t *slot_out;
+};
+
 int launch_decode(void *out, const void *query, const void *kc, const void *vc,
                   const pa_cache_desc &c, const int32_t *bt, int maxblk, const int32_t *ctx, int S,
                   int max_ctx, float scale, float k_scale, float v_scale,
-                  const pa_decode_config &cfg, void *ws, cudaStream_t st, int device) {
+                  const pa_decode_config &cfg, void *ws, cudaStream_t st, int device,
+                  const AppendArgs *app = nullptr) {
     const int B = c.block_size, D = c.head_size;
     const bool fp8 = c.dtype == PA_E4M3;
     max_ctx = std::min<int64_t>(max_ctx, (int64_t)maxblk * B);
@@ -323,6 +332,17 @@ int launch_decode(void *out, const void *query, const void *kc, const void *vc,
     p.stages = cfg.stages;
     p.qk_scale_log2 = scale * (fp8 ? k_scale : 1.0f) * pa::kLog2e;
     p.out_scale = fp8 ? v_scale : 1.0f;
+    if (app) {
+        p.new_key = static_cast<const __half *>(app->new_key);
+        p.new_value = static_cast<const __half *>(app->new_value);
+        p.new_key_stride = app->key_stride;
+        p.new_value_stride = app->value_stride;
+        p.key_cache = const_cast<void *>(kc);
+        p.value_cache = const_cast<void *>(vc);
+        p.slot_out = app->slot_out;
+        p.k_scale = fp8 ? k_scale : 1.0f;
+        p.v_scale = fp8 ? v_scale : 1.0f;
+    }
 
     DecodeKernel kern = pick_decode(D, B, fp8);
     if (!kern) return fail(PA_ERR_INVALID, "no kernel for head_size %d block_size %d", D, B);
@@ -530,6 +550,52 @@ int pa_paged_attention_decode_ws(void *out, const void *query, const void *key_c
 }
 
 }  // extern "C"
+
+extern "C" int pa_paged_attention_decode_append(
+    void *out, const void *query, const void *new_key, const void *new_value, int64_t key_stride,
+    int64_t value_stride, void *key_cache, void *value_cache, pa_cache_desc cache,
+    const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+    int num_seqs, int max_context_len, float scale, float k_scale, float v_scale,
+    int32_t *slot_mapping_out, const pa_decode_config *cfg, void *workspace,
+    size_t workspace_bytes, void *stream) {
+    int rc = check_decode_args(out, query, key_cache, value_cache, cache, block_tables,
+                               max_blocks_per_seq, context_lens, num_seqs, max_context_len, scale,
+                               k_scale, v_scale);
+    if (rc) return rc;
+    if (num_seqs == 0) return ok();
+    if (!new_key || !new_value) return fail(PA_ERR_INVALID, "null new_key/new_value");
+    if (!aligned16(new_key) || !aligned16(new_value))
+        return fail(PA_ERR_INVALID, "new_key and new_value must be 16-byte aligned");
+    const int row = cache.num_heads * cache.head_size;
+    if (key_stride < row || value_stride < row || key_stride % 8 || value_stride % 8)
+        return fail(PA_ERR_INVALID,
+                    "key_stride/value_stride (%lld/%lld) must be >= %d and multiples of 8",
+                    (long long)key_stride, (long long)value_stride, row);
+    const int bound =
+        (int)std::min<int64_t>(max_context_len, (int64_t)max_blocks_per_seq * cache.block_size);
+    pa_decode_config r = cfg ? *cfg : pa_decode_config{0, 0, 0, 0};
+    rc = fill_config(cache, num_seqs, bound, &r);
+    if (rc) return rc;
+    const size_t need = ws_bytes(cache, num_seqs, bound, r);
+    int dev = 0;
+    rc = current_device(&dev);
+    if (rc) return rc;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    void *ws = workspace;
+    if (need && workspace) {
+        if (workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+            return fail(PA_ERR_WORKSPACE,
+                        "workspace of %zu bytes at %p: need %zu bytes, 256-byte aligned",
+                        workspace_bytes, workspace, need);
+    } else if (need) {
+        rc = internal_workspace(need, st, dev, &ws);
+        if (rc) return rc;
+    }
+    const AppendArgs app{new_key, new_value, key_stride, value_stride, slot_mapping_out};
+    return launch_decode(out, query, key_cache, value_cache, cache, block_tables,
+                         max_blocks_per_seq, context_lens, num_seqs, bound, scale, k_scale,
+                         v_scale, r, ws, st, dev, &app);
+}
 
 // ---------------------------------------------------------------------------
 // Decode for callers that may not allocate device memory at all.

@@ -63,18 +63,8 @@ kv_cache_write_kernel(const __half *__restrict__ key, const __half *__restrict__
         reinterpret_cast<uint4 *>(static_cast<__half *>(key_cache) + dst)[0] = kraw;
         reinterpret_cast<uint4 *>(static_cast<__half *>(value_cache) + dst)[0] = vraw;
     } else {
-        const __half2 *kh = reinterpret_cast<const __half2 *>(&kraw);
-        const __half2 *vh = reinterpret_cast<const __half2 *>(&vraw);
-        uint2 kq, vq;
-        uint16_t *kc = reinterpret_cast<uint16_t *>(&kq);
-        uint16_t *vc = reinterpret_cast<uint16_t *>(&vq);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float2 kf = __half22float2(kh[j]);
-            const float2 vf = __half22float2(vh[j]);
-            kc[j] = float2_to_e4m3x2(__fdiv_rn(kf.x, k_scale), __fdiv_rn(kf.y, k_scale));
-            vc[j] = float2_to_e4m3x2(__fdiv_rn(vf.x, v_scale), __fdiv_rn(vf.y, v_scale));
-        }
+        const uint2 kq = encode8_e4m3(kraw, k_scale);
+        const uint2 vq = encode8_e4m3(vraw, v_scale);
         reinterpret_cast<uint2 *>(static_cast<uint8_t *>(key_cache) + dst)[0] = kq;
         reinterpret_cast<uint2 *>(static_cast<uint8_t *>(value_cache) + dst)[0] = vq;
     }

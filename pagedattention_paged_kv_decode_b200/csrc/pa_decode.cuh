@@ -52,7 +52,21 @@ struct DecodeParams {
     int stages;
     float qk_scale_log2;         // scale * k_scale * log2(e)
     float out_scale;             // v_scale (1 for fp16 caches)
+    // Fused append (all null/0 for a plain decode): each sequence's new token
+    // at position L-1 is stored into its slot before the block holding it is
+    // loaded; slot_out[s] receives that slot (-1 if none).
+    const __half *new_key;       // [S][H][D], row stride new_key_stride elements
+    const __half *new_value;
+    int64_t new_key_stride;
+    int64_t new_value_stride;
+    void *key_cache;             // same pools the tensor maps describe
+    void *value_cache;
+    int32_t *slot_out;
+    float k_scale;               // E4M3 encode scales (1 for fp16 caches)
+    float v_scale;
 };
+
+constexpr int kMaxAppendChunks = 4;  // 16-byte chunks per lane: G*D/8 <= 128
 
 // Lane geometry of a consumer warp. Each lane holds EPL consecutive elements
 // of a K/V row (16 bytes), LPR lanes cover one row of head_size elements,
@@ -126,8 +140,6 @@ __device__ __forceinline__ void unpack16<true>(const uint4 &raw, float *f) {
     }
 }
 
-__device__ __forceinline__ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
-
 // Shared-memory carve-up, identical on host and device.
 struct SmemLayout {
     size_t tile_bytes;   // one K (or V) tile: B * G * D * elem
@@ -167,7 +179,8 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int n_consumers = G * W;
 
     // Context length, clamped to what the table and the grid can address.
-    int L = __ldg(p.context_lens + s);
+    const int L_in = __ldg(p.context_lens + s);
+    int L = L_in;
     const int cap = p.max_blocks_per_seq * B;
     if (L > cap) {
         if (threadIdx.x == 0 && part == 0 && blockIdx.y == 0) flag_error(PA_DEV_CTX_OVER_TABLE);
@@ -180,7 +193,8 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
     if (L < 0) L = 0;
     const int n_parts = (L + p.partition_size - 1) / p.partition_size;
     if (part >= n_parts) {
-        if (L == 0 && part == 0) {  // empty context: zeros
+        if (L == 0 && part == 0) {  // empty context: zeros (and no appended token)
+            if (p.slot_out && blockIdx.y == 0 && threadIdx.x == 0) p.slot_out[s] = -1;
             for (int i = threadIdx.x; i < G * D / 8; i += blockDim.x) {
                 const int g = i / (D / 8), c = i % (D / 8);
                 reinterpret_cast<uint4 *>(p.out + ((size_t)s * p.num_heads + h0 + g) * D)[c] =
@@ -212,6 +226,29 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const int32_t *row = p.block_tables + (size_t)s * p.max_blocks_per_seq + blk0;
         const uint64_t policy = l2_policy_evict_first();
         const uint32_t tx_bytes = (uint32_t)lay.stage_bytes;
+
+        // Fused append: the CTA owning the sequence's last partition stores the
+        // new token's rows for its G heads. Its source rows are fetched now so
+        // the loads overlap the table read and the first tile loads.
+        // (A clamped context has no valid position for its new token: no append.)
+        const bool last = p.new_key != nullptr && part == n_parts - 1;
+        const bool append = last && L == L_in;
+        if (last && !append && p.slot_out && blockIdx.y == 0 && lane == 0) p.slot_out[s] = -1;
+        const int n_chunks = G * D / 8;  // 16-byte fp16 chunks of G heads
+        uint4 nk[kMaxAppendChunks], nv[kMaxAppendChunks];
+        if (append) {
+            const uint4 *ks = reinterpret_cast<const uint4 *>(p.new_key + (size_t)s * p.new_key_stride + (size_t)h0 * D);
+            const uint4 *vs = reinterpret_cast<const uint4 *>(p.new_value + (size_t)s * p.new_value_stride + (size_t)h0 * D);
+#pragma unroll
+            for (int k = 0; k < kMaxAppendChunks; ++k) {
+                const int c = lane + 32 * k;
+                if (c < n_chunks) {
+                    nk[k] = __ldg(ks + c);
+                    nv[k] = __ldg(vs + c);
+                }
+            }
+        }
+
         bool ok = true;
         int stage = 0, use = 0;
         for (int base = 0; base < nblk && ok; base += 32) {
@@ -220,11 +257,36 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
             const int cnt = min(32, nblk - base);
             for (int j = 0; j < cnt; ++j) {
                 int blk = __shfl_sync(0xffffffffu, my_blk, j);
-                if (lane == 0) {
-                    if (blk < 0 || blk >= p.num_blocks) {
-                        flag_error(PA_DEV_BAD_BLOCK);
-                        blk = p.num_blocks;  // out of range: the TMA zero-fills the tile
+                const bool bad = blk < 0 || blk >= p.num_blocks;
+                if (bad) blk = p.num_blocks;  // out of range: the TMA zero-fills the tile
+                if (append && base + j == nblk - 1) {
+                    // a1 + a2 for this sequence and these heads, before the tile that holds them
+                    const int pos = L - 1;
+                    const int slot = bad ? -1 : blk * B + pos % B;
+                    if (!bad) {
+                        const size_t dst = ((size_t)blk * B + pos % B) * p.num_heads * D + (size_t)h0 * D;
+#pragma unroll
+                        for (int k = 0; k < kMaxAppendChunks; ++k) {
+                            const int c = lane + 32 * k;
+                            if (c < n_chunks) {
+                                if constexpr (!kFp8) {
+                                    reinterpret_cast<uint4 *>(static_cast<__half *>(p.key_cache) + dst)[c] = nk[k];
+                                    reinterpret_cast<uint4 *>(static_cast<__half *>(p.value_cache) + dst)[c] = nv[k];
+                                } else {
+                                    reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.key_cache) + dst)[c] =
+                                        encode8_e4m3(nk[k], p.k_scale);
+                                    reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.value_cache) + dst)[c] =
+                                        encode8_e4m3(nv[k], p.v_scale);
+                                }
+                            }
+                        }
+                        fence_proxy_async_global();
                     }
+                    if (p.slot_out && blockIdx.y == 0 && lane == 0) p.slot_out[s] = slot;
+                    __syncwarp();
+                }
+                if (lane == 0) {
+                    if (bad) flag_error(PA_DEV_BAD_BLOCK);
                     if (use > 0) ok = mbar_wait(&empty[stage], (use - 1) & 1);
                     if (ok) {
                         unsigned char *kdst = smem + (size_t)stage * lay.stage_bytes;

@@ -100,6 +100,12 @@ __device__ __forceinline__ void tma_load_4d(void *smem_dst, const CUtensorMap *m
         : "memory");
 }
 
+// Orders this thread's earlier generic-proxy global stores before later
+// async-proxy (TMA) accesses of the same memory.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
@@ -150,6 +156,20 @@ __device__ __forceinline__ __half2 e4m3x2_to_half2(uint16_t codes) {
 __device__ __forceinline__ uint16_t float2_to_e4m3x2(float lo, float hi) {
     uint16_t r;
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// 8 fp16 values -> 8 E4M3 codes of x / scale (IEEE divide, RNE, saturate):
+// the same conversion as the cache-write kernel.
+__device__ __forceinline__ uint2 encode8_e4m3(const uint4 &raw, float scale) {
+    const __half2 *h = reinterpret_cast<const __half2 *>(&raw);
+    uint2 r;
+    uint16_t *c = reinterpret_cast<uint16_t *>(&r);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float2 f = __half22float2(h[j]);
+        c[j] = float2_to_e4m3x2(__fdiv_rn(f.x, scale), __fdiv_rn(f.y, scale));
+    }
     return r;
 }
 

@@ -156,6 +156,50 @@ def paged_attention_decode(out: torch.Tensor, query: torch.Tensor, key_cache: to
                                              ws_ptr, ws_bytes, _stream(stream)))
 
 
+def paged_attention_decode_append(out: torch.Tensor, query: torch.Tensor, new_key: torch.Tensor,
+                                  new_value: torch.Tensor, key_cache: torch.Tensor,
+                                  value_cache: torch.Tensor, block_tables: torch.Tensor,
+                                  context_lens: torch.Tensor, scale: float, k_scale: float = 1.0,
+                                  v_scale: float = 1.0, max_context_len: int | None = None,
+                                  slot_mapping: torch.Tensor | None = None, config=None,
+                                  workspace: torch.Tensor | None = None, stream=None) -> None:
+    """Fused step: slot of each appended token, its K/V store, and the decode.
+
+    ``slot_mapping`` (int32 [S], optional) receives the slots."""
+    _check_pair(key_cache, value_cache)
+    _i32(block_tables, "block_tables")
+    _i32(context_lens, "context_lens")
+    for t in (out, query):
+        if t.dtype != torch.float16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("out and query must be contiguous float16 CUDA tensors")
+    S, H, D = query.shape
+    for t in (new_key, new_value):
+        if t.dtype != torch.float16 or not t.is_cuda or tuple(t.shape) != (S, H, D):
+            raise ValueError("new_key/new_value must be float16 CUDA tensors [S, H, D]")
+        if t.stride(2) != 1 or t.stride(1) != D:
+            raise ValueError("new_key/new_value rows must be contiguous within a token")
+    if out.shape != query.shape or context_lens.shape[0] != S or block_tables.shape[0] != S:
+        raise ValueError("shape mismatch between out, query, block_tables and context_lens")
+    desc = cache_desc(key_cache)
+    if desc.num_heads != H or desc.head_size != D:
+        raise ValueError("query heads/head_size differ from the cache's")
+    if max_context_len is None:
+        max_context_len = block_tables.shape[1] * desc.block_size
+    if slot_mapping is not None:
+        _i32(slot_mapping, "slot_mapping")
+    cfg = _config(config)
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    check(lib().pa_paged_attention_decode_append(
+        out.data_ptr(), query.data_ptr(), new_key.data_ptr(), new_value.data_ptr(),
+        new_key.stride(0), new_value.stride(0), key_cache.data_ptr(), value_cache.data_ptr(), desc,
+        block_tables.data_ptr(), block_tables.shape[1], context_lens.data_ptr(), S,
+        int(max_context_len), float(scale), float(k_scale), float(v_scale),
+        slot_mapping.data_ptr() if slot_mapping is not None else None,
+        ctypes.byref(cfg) if cfg is not None else None, ws_ptr, ws_bytes, _stream(stream)))
+
+
 def check_status(stream=None) -> int:
     """Synchronise the stream; return and clear the device error bits (PA_DEV_*)."""
     code = ctypes.c_uint32(0)
@@ -195,14 +239,23 @@ def decode_step(out: torch.Tensor, query: torch.Tensor, new_key: torch.Tensor,
                 block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
                 k_scale: float = 1.0, v_scale: float = 1.0, cow_pairs: torch.Tensor | None = None,
                 slots: torch.Tensor | None = None, max_context_len: int | None = None,
-                config=None, workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+                config=None, workspace: torch.Tensor | None = None, stream=None,
+                fused: bool = True) -> torch.Tensor:
     """One decode step of the whole path, all on the device, in order:
     copy-on-write block copies (if any pairs), slot of each appended token,
     scatter of the new K/V rows into those slots, decode attention.
-    ``block_tables`` are the tables after any copy-on-write repoint.
-    Returns the slot tensor."""
+    ``block_tables`` are the tables after any copy-on-write repoint. With
+    ``fused`` the last three run as one launch (paged_attention_decode_append);
+    otherwise as three separate calls. Returns the slot tensor."""
     if cow_pairs is not None and cow_pairs.numel():
         copy_blocks(key_cache, value_cache, cow_pairs, stream)
+    if fused:
+        if slots is None:
+            slots = torch.empty(query.shape[0], dtype=torch.int32, device=query.device)
+        paged_attention_decode_append(out, query, new_key, new_value, key_cache, value_cache,
+                                      block_tables, context_lens, scale, k_scale, v_scale,
+                                      max_context_len, slots, config, workspace, stream)
+        return slots
     slots = slot_mapping(block_tables, context_lens, key_cache, out=slots, stream=stream)
     kv_cache_write(new_key, new_value, key_cache, value_cache, slots, k_scale, v_scale, stream)
     paged_attention_decode(out, query, key_cache, value_cache, block_tables, context_lens, scale,

@@ -133,3 +133,25 @@ def test_empty_batch_is_a_no_op(cuda_device):
                               torch.empty(0, dtype=torch.int32, device=cuda_device), 0.125)
     pk.kv_cache_write(e, e, kc, kc.clone(), torch.empty(0, dtype=torch.int32, device=cuda_device))
     assert pk.check_status() == 0
+
+
+def test_fused_append_skips_bad_blocks_and_clamped_contexts(cuda_device):
+    """The fused step derives the same slots as pa_slot_mapping: -1 (and no
+    store) for an invalid block id or a context beyond the table."""
+    w, dw = small(cuda_device)
+    bt = dw.block_tables.clone()
+    bt[2, 1] = -3                       # seq 2 (L=17) appends into logical block 1
+    ctx = dw.context_lens.clone()
+    ctx[0] = 4 * 16 + 9                 # beyond the 4-block table
+    before = dw.key_cache.clone()
+    pk.paged_attention_decode_append(dw.out, dw.query, dw.new_key, dw.new_value, dw.key_cache,
+                                     dw.value_cache, bt, ctx, w.scale, slot_mapping=dw.slots)
+    code = pk.check_status()
+    assert code == capi.PA_DEV_BAD_BLOCK | capi.PA_DEV_CTX_OVER_TABLE
+    slots = dw.slots.cpu().tolist()
+    assert slots[0] == -1 and slots[2] == -1
+    ref = oracle.slot_mapping(w.block_tables, w.context_lens, 16)
+    assert slots[1] == ref[1]
+    changed = (dw.key_cache != before).reshape(20 * 16, -1).any(dim=1).nonzero().flatten().tolist()
+    assert changed == [int(ref[1])]      # only seq 1's new row was stored
+    assert torch.isfinite(dw.out.float()).all()

@@ -18,17 +18,18 @@ pytestmark = pytest.mark.gpu
 TOL = {"f16": 2e-3, "e4m3": 1e-2}
 
 
-def run_step(w, dev, config=None, max_context_len=None):
+def run_step(w, dev, config=None, max_context_len=None, fused=True):
     dw = W.to_device(w, dev, encode=pk.load_cache)
     ws = None
-    if config is not None:
+    if config is not None and not fused:
         nbytes = pk.decode_workspace_size(dw.key_cache, w.num_seqs,
                                           max_context_len or w.max_context_len, config)
         ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
     pk.decode_step(dw.out, dw.query, dw.new_key, dw.new_value, dw.key_cache, dw.value_cache,
                    dw.block_tables, dw.context_lens, w.scale, w.k_scale, w.v_scale,
                    cow_pairs=dw.cow_pairs, slots=dw.slots,
-                   max_context_len=max_context_len or w.max_context_len, config=config, workspace=ws)
+                   max_context_len=max_context_len or w.max_context_len, config=config, workspace=ws,
+                   fused=fused)
     assert pk.check_status() == 0
     return dw
 
@@ -61,10 +62,11 @@ def compare_step(w, dw, seqs, check_all_blocks):
     return err
 
 
+@pytest.mark.parametrize("fused", [True, False], ids=["fused", "separate"])
 @pytest.mark.parametrize("cfg", [1, 2, 3, 4, 5])
-def test_named_workload_step(cuda_device, cfg):
+def test_named_workload_step(cuda_device, cfg, fused):
     w = W.named(cfg)
-    dw = run_step(w, cuda_device)
+    dw = run_step(w, cuda_device, fused=fused)
     seqs = list(range(w.num_seqs)) if cfg <= 2 else sample_seqs(w, 8, seed=cfg)
     compare_step(w, dw, seqs, check_all_blocks=cfg <= 2)
 
@@ -80,10 +82,11 @@ def ragged_case(D, B, kv, seed, ctx=None, poison=W.POISON_HUGE, H=4):
 SHAPES = [(D, B, kv) for kv in ("f16", "e4m3") for D in (64, 128) for B in (16, 32)]
 
 
+@pytest.mark.parametrize("fused", [True, False], ids=["fused", "separate"])
 @pytest.mark.parametrize("D,B,kv", SHAPES)
-def test_all_kernel_variants_default_config(cuda_device, D, B, kv):
+def test_all_kernel_variants_default_config(cuda_device, D, B, kv, fused):
     w = ragged_case(D, B, kv, seed=D + B)
-    dw = run_step(w, cuda_device)
+    dw = run_step(w, cuda_device, fused=fused)
     compare_step(w, dw, list(range(w.num_seqs)), check_all_blocks=True)
 
 
@@ -117,8 +120,9 @@ def test_launch_shapes(cuda_device, launch, D, B, kv):
 def test_nan_poison_is_never_touched(cuda_device, kv):
     w = ragged_case(128, 16, kv, seed=3, poison=W.POISON_NAN)
     for launch in (None, dict(partition_size=32, heads_per_cta=2, warps_per_head=2, stages=3)):
-        dw = run_step(w, cuda_device, config=launch)
-        compare_step(w, dw, list(range(w.num_seqs)), check_all_blocks=False)
+        for fused in (True, False):
+            dw = run_step(w, cuda_device, config=launch, fused=fused)
+            compare_step(w, dw, list(range(w.num_seqs)), check_all_blocks=False)
 
 
 def test_split_partials_match_oracle_partitions(cuda_device):

@@ -111,6 +111,13 @@ _HUGE_PAIR = np.array([60000.0, -60000.0], np.float16)
 _HUGE_PAIR_I32 = int(_HUGE_PAIR.view(np.int32)[0])
 
 
+def fused_step_bytes(w: "Workload") -> int:
+    """Algorithmic bytes of one fused append+decode launch: the decode's bytes
+    plus the new K/V rows read (fp16) and stored (cache dtype) and the slots."""
+    S, H, D = w.num_seqs, w.num_heads, w.head_size
+    return w.decode_bytes() + S * H * D * 2 * 2 + S * H * D * w.elem_bytes * 2 + 4 * S
+
+
 def _poison_fill(shape, poison: str) -> np.ndarray:
     if poison == POISON_NAN:
         return np.full(shape, np.nan, np.float16)
