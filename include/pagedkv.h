@@ -81,7 +81,8 @@ typedef struct {
  *       partial results plus a log-sum-exp reduction.
  *   heads_per_cta:  1, 2, 4 or 8 and a divisor of num_heads.
  *   warps_per_head: 1, 2 or 4 warps sharing one head's tokens in a CTA.
- *   stages:         2..8 K/V tiles in flight per CTA. */
+ *   stages:         2..8 K/V tiles in flight per CTA, a multiple of
+ *                   warps_per_head. */
 typedef struct {
     int32_t partition_size;
     int32_t heads_per_cta;

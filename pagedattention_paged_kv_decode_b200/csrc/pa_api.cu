@@ -156,10 +156,17 @@ int fill_config(const pa_cache_desc &c, int num_seqs, int max_ctx, pa_decode_con
         while (P > 4 * B && units0 * std::max(1, (max_ctx + P - 1) / P) < 3 * kNumSMs) P >>= 1;
         r.partition_size = P;
     }
-    if (r.warps_per_head == 0) r.warps_per_head = std::min(4, std::max(1, 8 / r.heads_per_cta));
+    // stages must be a multiple of warps_per_head (see the check below).
+    if (r.warps_per_head == 0) {
+        int W = std::min(4, std::max(1, 8 / r.heads_per_cta));
+        while (W > 1 && r.stages != 0 && r.stages % W) W >>= 1;
+        r.warps_per_head = W;
+    }
     if (r.stages == 0) {
         const size_t sb = stage_bytes(r.heads_per_cta);
-        r.stages = (int)std::max<size_t>(2, std::min<size_t>(8, (128 * 1024) / sb));
+        int st = (int)std::max<size_t>(2, std::min<size_t>(8, (128 * 1024) / sb));
+        st = std::max(r.warps_per_head, st / r.warps_per_head * r.warps_per_head);
+        r.stages = std::max(2, st);
     }
     if (r.partition_size < B || r.partition_size % B)
         return fail(PA_ERR_INVALID, "partition_size %d must be a positive multiple of block_size %d",
@@ -174,6 +181,13 @@ int fill_config(const pa_cache_desc &c, int num_seqs, int max_ctx, pa_decode_con
                     pa::kMaxConsumerWarps);
     if (r.stages < 2 || r.stages > 8)
         return fail(PA_ERR_INVALID, "stages %d must be in [2, 8]", r.stages);
+    // Warp w of a head consumes blocks w, w+W, ... from stage i % stages and
+    // waits on that stage's full barrier by phase parity. A parity wait is
+    // only meaningful for the current or the immediately preceding phase, so
+    // the previous use of the stage must be one the same warp has already
+    // consumed: with stages % W == 0 every stage belongs to exactly one warp.
+    if (r.stages % W)
+        return fail(PA_ERR_INVALID, "stages %d must be a multiple of warps_per_head %d", r.stages, W);
     const pa::SmemLayout lay(B, G, c.head_size, elem_bytes(c), W, r.stages);
     if (lay.total > kMaxSmem)
         return fail(PA_ERR_INVALID, "launch shape needs %zu bytes of shared memory (max %zu)",

@@ -115,6 +115,13 @@ def test_config_validation_and_workspace_size():
     assert _choose(desc, 16, 512, heads_per_cta=3)[0] == capi.PA_ERR_INVALID
     assert _choose(desc, 16, 512, heads_per_cta=8, warps_per_head=4)[0] == capi.PA_ERR_INVALID  # 32 warps
     assert _choose(desc, 16, 512, stages=9)[0] == capi.PA_ERR_INVALID
+    # a warp waits on a stage's barrier by phase parity: stages must be a multiple of warps
+    assert _choose(desc, 16, 512, heads_per_cta=1, warps_per_head=4, stages=2)[0] == capi.PA_ERR_INVALID
+    assert _choose(desc, 16, 512, heads_per_cta=2, warps_per_head=2, stages=3)[0] == capi.PA_ERR_INVALID
+    rc, c = _choose(desc, 16, 512, stages=6)
+    assert rc == 0 and c.stages % c.warps_per_head == 0
+    rc, c = _choose(desc, 16, 512, heads_per_cta=1, warps_per_head=4)
+    assert rc == 0 and c.stages % 4 == 0
     assert _choose(desc, 16, 512, heads_per_cta=8, stages=8)[0] == capi.PA_ERR_INVALID  # smem > 227 KB
     rc, cfg = _choose(desc, 16, 512, partition_size=128, heads_per_cta=2, warps_per_head=2, stages=4)
     assert rc == 0
