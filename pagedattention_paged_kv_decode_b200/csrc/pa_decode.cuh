@@ -178,6 +178,21 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int lane = threadIdx.x & 31;
     const int n_consumers = G * W;
 
+    // Loads whose addresses do not depend on the context length are issued
+    // before it arrives: the producer's first 32 table entries of this
+    // partition (entries past the row are not read), the consumers' query rows.
+    const int blk0_pre = part * (p.partition_size / B);
+    int pre_blk = 0;
+    if (warp == n_consumers && blk0_pre + lane < p.max_blocks_per_seq)
+        pre_blk = __ldg(p.block_tables + (size_t)s * p.max_blocks_per_seq + blk0_pre + lane);
+    uint4 q_raw[EPL / 8];
+    if (warp < n_consumers) {
+        const uint4 *qp = reinterpret_cast<const uint4 *>(
+            p.query + ((size_t)s * p.num_heads + h0 + warp % G) * D);
+#pragma unroll
+        for (int c = 0; c < EPL / 8; ++c) q_raw[c] = __ldg(qp + (lane % LPR) * (EPL / 8) + c);
+    }
+
     // Context length, clamped to what the table and the grid can address.
     const int L_in = __ldg(p.context_lens + s);
     int L = L_in;
@@ -252,8 +267,8 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
         bool ok = true;
         int stage = 0, use = 0;
         for (int base = 0; base < nblk && ok; base += 32) {
-            int my_blk = 0;
-            if (base + lane < nblk) my_blk = __ldg(row + base + lane);
+            int my_blk = pre_blk;  // entries 0..31 were prefetched above
+            if (base > 0 && base + lane < nblk) my_blk = __ldg(row + base + lane);
             const int cnt = min(32, nblk - base);
             for (int j = 0; j < cnt; ++j) {
                 int blk = __shfl_sync(0xffffffffu, my_blk, j);
@@ -316,17 +331,8 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
 
     float q[EPL];
     {
-        const __half *qp = p.query + ((size_t)s * p.num_heads + h) * D;
-        if constexpr (kFp8) {
-            // EPL = 16 elements: two 16-byte fp16 chunks
-            const uint4 a = __ldg(reinterpret_cast<const uint4 *>(qp) + 2 * sub);
-            const uint4 b = __ldg(reinterpret_cast<const uint4 *>(qp) + 2 * sub + 1);
-            unpack16<false>(a, q);
-            unpack16<false>(b, q + 8);
-        } else {
-            const uint4 a = __ldg(reinterpret_cast<const uint4 *>(qp) + sub);
-            unpack16<false>(a, q);
-        }
+#pragma unroll
+        for (int c = 0; c < EPL / 8; ++c) unpack16<false>(q_raw[c], q + 8 * c);  // fp16 query
 #pragma unroll
         for (int e = 0; e < EPL; ++e) q[e] *= p.qk_scale_log2;
     }
