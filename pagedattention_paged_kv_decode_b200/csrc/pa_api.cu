@@ -142,30 +142,43 @@ int fill_config(const pa_cache_desc &c, int num_seqs, int max_ctx, pa_decode_con
     auto stage_bytes = [&](int G) {
         return pa::SmemLayout(B, G, c.head_size, elem_bytes(c), 1, 1).stage_bytes;
     };
+    auto units = [&](int G, int P) {  // CTAs of the grid, from the host-side length bound
+        return (int64_t)num_seqs * (H / G) * std::max(1, (max_ctx + P - 1) / P);
+    };
+    // Defaults, fitted by launch-shape sweeps on B200 (sequences x heads x
+    // contexts of 16x32x<=178, 64x40x<=2048, 32x32x<=4096, 256x32x<=4096):
+    // about four consumer warps per CTA, a ring of about 64 KiB so that three
+    // or more CTAs share an SM, enough CTAs for every SM, and long partitions
+    // only when the grid stays large with them.
     if (r.heads_per_cta == 0) {
         int G = 4;
-        while (G > 1 && (H % G || stage_bytes(G) * 4 > 160 * 1024)) G >>= 1;
+        while (G > 1 && (H % G || stage_bytes(G) * 2 > 96 * 1024)) G >>= 1;
         const int P0 = r.partition_size ? r.partition_size : 512;
-        const int parts = std::max(1, (max_ctx + P0 - 1) / P0);
-        while (G > 1 && (int64_t)num_seqs * (H / G) * parts < 3 * kNumSMs) G >>= 1;
+        while (G > 1 && units(G, P0) < 3 * kNumSMs) G >>= 1;
         r.heads_per_cta = G;
     }
+    const int G0 = r.heads_per_cta;
     if (r.partition_size == 0) {
-        int P = 512;
-        const int64_t units0 = (int64_t)num_seqs * (H / r.heads_per_cta);
-        while (P > 4 * B && units0 * std::max(1, (max_ctx + P - 1) / P) < 3 * kNumSMs) P >>= 1;
+        int P = units(G0, 1024) >= 12 * kNumSMs ? 1024 : 512;
+        while (P > 4 * B && units(G0, P) < 3 * kNumSMs) P >>= 1;
         r.partition_size = P;
     }
     // stages must be a multiple of warps_per_head (see the check below).
     if (r.warps_per_head == 0) {
-        int W = std::min(4, std::max(1, 8 / r.heads_per_cta));
+        int W = std::min(4, std::max(1, 4 / G0));
         while (W > 1 && r.stages != 0 && r.stages % W) W >>= 1;
         r.warps_per_head = W;
     }
     if (r.stages == 0) {
-        const size_t sb = stage_bytes(r.heads_per_cta);
-        int st = (int)std::max<size_t>(2, std::min<size_t>(8, (128 * 1024) / sb));
-        st = std::max(r.warps_per_head, st / r.warps_per_head * r.warps_per_head);
+        const int W = r.warps_per_head;
+        size_t ring = 64 * 1024;
+        const int64_t n = units(G0, r.partition_size);
+        if (n < 4 * kNumSMs) {  // small grid: keep every CTA resident at once
+            const int64_t per_sm = std::max<int64_t>(1, (n + kNumSMs - 1) / kNumSMs);
+            ring = std::min<size_t>(ring, (200 * 1024) / per_sm);
+        }
+        int st = (int)std::min<size_t>(8, std::max<size_t>(2, ring / stage_bytes(G0)));
+        st = std::max(W, st / W * W);
         r.stages = std::max(2, st);
     }
     if (r.partition_size < B || r.partition_size % B)

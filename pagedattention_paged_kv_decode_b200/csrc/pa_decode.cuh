@@ -144,15 +144,16 @@ __device__ __forceinline__ void unpack16<true>(const uint4 &raw, float *f) {
 struct SmemLayout {
     size_t tile_bytes;   // one K (or V) tile: B * G * D * elem
     size_t stage_bytes;  // K tile + V tile
-    size_t bars_off;     // full[stages], empty[stages]
+    size_t bars_off;     // full[stages], empty[stages], newrow
+    size_t newrow_off;   // appended token's K row then V row: 2 * G * D * elem
     size_t merge_off;    // W * G * (D + 2) floats
     size_t total;
     __host__ __device__ SmemLayout(int B, int G, int D, int elem, int W, int stages) {
         tile_bytes = (size_t)B * G * D * elem;
         stage_bytes = 2 * tile_bytes;
         bars_off = stage_bytes * stages;
-        merge_off = bars_off + 2 * 8 * (size_t)stages;
-        merge_off = (merge_off + 15) / 16 * 16;
+        newrow_off = (bars_off + 8 * (2 * (size_t)stages + 1) + 15) / 16 * 16;
+        merge_off = newrow_off + 2 * (size_t)G * D * elem;
         total = merge_off + sizeof(float) * (size_t)W * G * (D + 2);
     }
 };
@@ -169,6 +170,8 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const SmemLayout lay(B, G, D, Geo::kElemBytes, W, stages);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + lay.bars_off);
     uint64_t *empty = full + stages;
+    uint64_t *newrow_bar = empty + stages;  // the appended rows are in shared memory
+    unsigned char *newrow = smem + lay.newrow_off;
     float *merge = reinterpret_cast<float *>(smem + lay.merge_off);
 
     const int part = blockIdx.x;
@@ -228,6 +231,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], G);
         }
+        mbar_init(newrow_bar, 1);
         fence_mbar_init();
     }
     __syncthreads();
@@ -243,17 +247,20 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const uint32_t tx_bytes = (uint32_t)lay.stage_bytes;
 
         // Fused append: the CTA owning the sequence's last partition stores the
-        // new token's rows for its G heads. Its source rows are fetched now so
-        // the loads overlap the table read and the first tile loads.
-        // (A clamped context has no valid position for its new token: no append.)
+        // new token's rows for its G heads. (A clamped context has no valid
+        // position for its new token: no append.)
         const bool last = p.new_key != nullptr && part == n_parts - 1;
         const bool append = last && L == L_in;
         if (last && !append && p.slot_out && blockIdx.y == 0 && lane == 0) p.slot_out[s] = -1;
         const int n_chunks = G * D / 8;  // 16-byte fp16 chunks of G heads
+        // The appended rows' loads are issued now; they are stored after the
+        // tile loads have been issued (no tile load waits for them).
         uint4 nk[kMaxAppendChunks], nv[kMaxAppendChunks];
+        int app_blk = 0;
         if (append) {
             const uint4 *ks = reinterpret_cast<const uint4 *>(p.new_key + (size_t)s * p.new_key_stride + (size_t)h0 * D);
             const uint4 *vs = reinterpret_cast<const uint4 *>(p.new_value + (size_t)s * p.new_value_stride + (size_t)h0 * D);
+            app_blk = __ldg(p.block_tables + (size_t)s * p.max_blocks_per_seq + (L - 1) / B);  // L <= cap
 #pragma unroll
             for (int k = 0; k < kMaxAppendChunks; ++k) {
                 const int c = lane + 32 * k;
@@ -274,32 +281,6 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 int blk = __shfl_sync(0xffffffffu, my_blk, j);
                 const bool bad = blk < 0 || blk >= p.num_blocks;
                 if (bad) blk = p.num_blocks;  // out of range: the TMA zero-fills the tile
-                if (append && base + j == nblk - 1) {
-                    // a1 + a2 for this sequence and these heads, before the tile that holds them
-                    const int pos = L - 1;
-                    const int slot = bad ? -1 : blk * B + pos % B;
-                    if (!bad) {
-                        const size_t dst = ((size_t)blk * B + pos % B) * p.num_heads * D + (size_t)h0 * D;
-#pragma unroll
-                        for (int k = 0; k < kMaxAppendChunks; ++k) {
-                            const int c = lane + 32 * k;
-                            if (c < n_chunks) {
-                                if constexpr (!kFp8) {
-                                    reinterpret_cast<uint4 *>(static_cast<__half *>(p.key_cache) + dst)[c] = nk[k];
-                                    reinterpret_cast<uint4 *>(static_cast<__half *>(p.value_cache) + dst)[c] = nv[k];
-                                } else {
-                                    reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.key_cache) + dst)[c] =
-                                        encode8_e4m3(nk[k], p.k_scale);
-                                    reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.value_cache) + dst)[c] =
-                                        encode8_e4m3(nv[k], p.v_scale);
-                                }
-                            }
-                        }
-                        fence_proxy_async_global();
-                    }
-                    if (p.slot_out && blockIdx.y == 0 && lane == 0) p.slot_out[s] = slot;
-                    __syncwarp();
-                }
                 if (lane == 0) {
                     if (bad) flag_error(PA_DEV_BAD_BLOCK);
                     if (use > 0) ok = mbar_wait(&empty[stage], (use - 1) & 1);
@@ -318,6 +299,41 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     ++use;
                 }
             }
+        }
+        if (append) {
+            // a1 + a2 for this sequence and these heads. The rows go to the
+            // cache for later steps and, in cache format, to shared memory,
+            // from which the consumers take the appended token (that row of
+            // its tile is never used, so the tile load did not wait for this).
+            const int pos = L - 1;
+            const bool bad = app_blk < 0 || app_blk >= p.num_blocks;
+            const size_t dst = ((size_t)(bad ? 0 : app_blk) * B + pos % B) * p.num_heads * D + (size_t)h0 * D;
+#pragma unroll
+            for (int k = 0; k < kMaxAppendChunks; ++k) {
+                const int c = lane + 32 * k;
+                if (c < n_chunks) {
+                    if constexpr (!kFp8) {
+                        reinterpret_cast<uint4 *>(newrow)[c] = nk[k];
+                        reinterpret_cast<uint4 *>(newrow + (size_t)G * D * 2)[c] = nv[k];
+                        if (!bad) {
+                            reinterpret_cast<uint4 *>(static_cast<__half *>(p.key_cache) + dst)[c] = nk[k];
+                            reinterpret_cast<uint4 *>(static_cast<__half *>(p.value_cache) + dst)[c] = nv[k];
+                        }
+                    } else {
+                        const uint2 ek = encode8_e4m3(nk[k], p.k_scale);
+                        const uint2 ev = encode8_e4m3(nv[k], p.v_scale);
+                        reinterpret_cast<uint2 *>(newrow)[c] = ek;
+                        reinterpret_cast<uint2 *>(newrow + (size_t)G * D)[c] = ev;
+                        if (!bad) {
+                            reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.key_cache) + dst)[c] = ek;
+                            reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.value_cache) + dst)[c] = ev;
+                        }
+                    }
+                }
+            }
+            if (p.slot_out && blockIdx.y == 0 && lane == 0) p.slot_out[s] = bad ? -1 : app_blk * B + pos % B;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(newrow_bar);  // release: the rows are in shared memory
         }
         return;
     }
@@ -344,6 +360,10 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
 
     const size_t row_stride = (size_t)G * D * Geo::kElemBytes;  // bytes between tokens in a tile
     const size_t head_off = (size_t)g * D * Geo::kElemBytes + (size_t)sub * 16;
+    // The appended token (fused append only) is read from shared memory.
+    const bool appended = p.new_key != nullptr && part == n_parts - 1 && L == L_in;
+    const int t_new_block = appended ? (L - 1 - t0) / B : -1;  // block index within the partition
+    const int t_new_row = appended ? (L - 1) % B : -1;
     bool ok = true;
     int stage = w % stages, use = w / stages;
     for (int i = w; i < nblk; i += W) {
@@ -354,13 +374,24 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const unsigned char *ktile = smem + (size_t)stage * lay.stage_bytes;
         const unsigned char *vtile = ktile + lay.tile_bytes;
         const int valid = min(B, t1 - (t0 + i * B));  // tokens of this block inside the context
+        int t_new = -1;
+        if (i == t_new_block) {
+            if (!mbar_wait(newrow_bar, 0)) {
+                ok = false;
+                break;
+            }
+            t_new = t_new_row;
+        }
+        const unsigned char *knew = newrow;
+        const unsigned char *vnew = newrow + (size_t)G * D * Geo::kElemBytes;
 
         // ---- logits of this lane group's TPG tokens
         float part_dot[TPG];
 #pragma unroll
         for (int j = 0; j < TPG; ++j) {
             const int t = grp * TPG + j;
-            const uint4 raw = *reinterpret_cast<const uint4 *>(ktile + t * row_stride + head_off);
+            const unsigned char *krow = (t == t_new) ? knew : ktile + t * row_stride;
+            const uint4 raw = *reinterpret_cast<const uint4 *>(krow + head_off);
             float k[EPL];
             unpack16<kFp8>(raw, k);
             float d = 0.f;
@@ -387,7 +418,8 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
             const int t = grp * TPG + j;
             const float pj = __shfl_sync(0xffffffffu, pz, grp * LPR + j * DUP);
             if (t < valid) {
-                const uint4 raw = *reinterpret_cast<const uint4 *>(vtile + t * row_stride + head_off);
+                const unsigned char *vrow = (t == t_new) ? vnew : vtile + t * row_stride;
+                const uint4 raw = *reinterpret_cast<const uint4 *>(vrow + head_off);
                 float v[EPL];
                 unpack16<kFp8>(raw, v);
 #pragma unroll
