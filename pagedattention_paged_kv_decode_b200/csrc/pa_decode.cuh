@@ -188,6 +188,24 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
     int pre_blk = 0;
     if (warp == n_consumers && blk0_pre + lane < p.max_blocks_per_seq)
         pre_blk = __ldg(p.block_tables + (size_t)s * p.max_blocks_per_seq + blk0_pre + lane);
+    // Fused append: partition 0 is the last partition of every context of up
+    // to one partition, so its producer fetches the appended rows before the
+    // context length is known (other partitions fetch them once it is).
+    const int n_chunks = G * D / 8;  // 16-byte fp16 chunks of G heads
+    uint4 nk[kMaxAppendChunks], nv[kMaxAppendChunks];
+    const bool pre_append = p.new_key != nullptr && part == 0 && warp == n_consumers;
+    if (pre_append) {
+        const uint4 *ks = reinterpret_cast<const uint4 *>(p.new_key + (size_t)s * p.new_key_stride + (size_t)h0 * D);
+        const uint4 *vs = reinterpret_cast<const uint4 *>(p.new_value + (size_t)s * p.new_value_stride + (size_t)h0 * D);
+#pragma unroll
+        for (int k = 0; k < kMaxAppendChunks; ++k) {
+            const int c = lane + 32 * k;
+            if (c < n_chunks) {
+                nk[k] = __ldg(ks + c);
+                nv[k] = __ldg(vs + c);
+            }
+        }
+    }
     uint4 q_raw[EPL / 8];
     if (warp < n_consumers) {
         const uint4 *qp = reinterpret_cast<const uint4 *>(
@@ -252,21 +270,24 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const bool last = p.new_key != nullptr && part == n_parts - 1;
         const bool append = last && L == L_in;
         if (last && !append && p.slot_out && blockIdx.y == 0 && lane == 0) p.slot_out[s] = -1;
-        const int n_chunks = G * D / 8;  // 16-byte fp16 chunks of G heads
-        // The appended rows' loads are issued now; they are stored after the
-        // tile loads have been issued (no tile load waits for them).
-        uint4 nk[kMaxAppendChunks], nv[kMaxAppendChunks];
+        // The appended rows are stored after the tile loads have been issued
+        // (no tile load waits for them). The new token's block id is the
+        // partition's last table entry.
         int app_blk = 0;
         if (append) {
-            const uint4 *ks = reinterpret_cast<const uint4 *>(p.new_key + (size_t)s * p.new_key_stride + (size_t)h0 * D);
-            const uint4 *vs = reinterpret_cast<const uint4 *>(p.new_value + (size_t)s * p.new_value_stride + (size_t)h0 * D);
-            app_blk = __ldg(p.block_tables + (size_t)s * p.max_blocks_per_seq + (L - 1) / B);  // L <= cap
+            const int last_entry = nblk - 1;
+            const int from_pre = __shfl_sync(0xffffffffu, pre_blk, last_entry & 31);
+            app_blk = last_entry < 32 ? from_pre : __ldg(row + last_entry);
+            if (!pre_append) {
+                const uint4 *ks = reinterpret_cast<const uint4 *>(p.new_key + (size_t)s * p.new_key_stride + (size_t)h0 * D);
+                const uint4 *vs = reinterpret_cast<const uint4 *>(p.new_value + (size_t)s * p.new_value_stride + (size_t)h0 * D);
 #pragma unroll
-            for (int k = 0; k < kMaxAppendChunks; ++k) {
-                const int c = lane + 32 * k;
-                if (c < n_chunks) {
-                    nk[k] = __ldg(ks + c);
-                    nv[k] = __ldg(vs + c);
+                for (int k = 0; k < kMaxAppendChunks; ++k) {
+                    const int c = lane + 32 * k;
+                    if (c < n_chunks) {
+                        nk[k] = __ldg(ks + c);
+                        nv[k] = __ldg(vs + c);
+                    }
                 }
             }
         }
