@@ -81,13 +81,17 @@ typedef struct {
  *       partial results plus a log-sum-exp reduction.
  *   heads_per_cta:  1, 2, 4 or 8 and a divisor of num_heads.
  *   warps_per_head: 1, 2 or 4 warps sharing one head's tokens in a CTA.
- *   stages:         2..8 K/V tiles in flight per CTA, a multiple of
- *                   warps_per_head. */
+ *   stages:         2..8 K/V tiles in flight per work unit, a multiple of
+ *                   warps_per_head.
+ *   units_per_cta:  1..4 work units (sequence x head group x partition) that
+ *                   one CTA serves, each with its own ring of stages;
+ *                   units_per_cta * heads_per_cta * warps_per_head <= 16. */
 typedef struct {
     int32_t partition_size;
     int32_t heads_per_cta;
     int32_t warps_per_head;
     int32_t stages;
+    int32_t units_per_cta;
 } pa_decode_config;
 
 /* Library version, e.g. 100 for 0.1.0. */

@@ -36,7 +36,8 @@ class CacheDesc(ctypes.Structure):
 
 class DecodeConfig(ctypes.Structure):
     _fields_ = [("partition_size", ctypes.c_int32), ("heads_per_cta", ctypes.c_int32),
-                ("warps_per_head", ctypes.c_int32), ("stages", ctypes.c_int32)]
+                ("warps_per_head", ctypes.c_int32), ("stages", ctypes.c_int32),
+                ("units_per_cta", ctypes.c_int32)]
 
     def as_dict(self):
         return {k: getattr(self, k) for k, _ in self._fields_}

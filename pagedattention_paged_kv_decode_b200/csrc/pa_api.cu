@@ -140,7 +140,7 @@ int fill_config(const pa_cache_desc &c, int num_seqs, int max_ctx, pa_decode_con
     const int H = c.num_heads, B = c.block_size;
     pa_decode_config r = *cfg;
     auto stage_bytes = [&](int G) {
-        return pa::SmemLayout(B, G, c.head_size, elem_bytes(c), 1, 1).stage_bytes;
+        return pa::SmemLayout(B, G, c.head_size, elem_bytes(c), 1, 1, 1).stage_bytes;
     };
     auto units = [&](int G, int P) {  // CTAs of the grid, from the host-side length bound
         return (int64_t)num_seqs * (H / G) * std::max(1, (max_ctx + P - 1) / P);
@@ -163,17 +163,29 @@ int fill_config(const pa_cache_desc &c, int num_seqs, int max_ctx, pa_decode_con
         while (P > 4 * B && units(G0, P) < 3 * kNumSMs) P >>= 1;
         r.partition_size = P;
     }
+    // A small grid (fewer units than four per SM) packs several units into
+    // each CTA, each with its own ring, so that one CTA per SM keeps nearly
+    // all of its units' blocks in flight at once.
+    if (r.units_per_cta == 0) {
+        const int64_t n = units(G0, r.partition_size);
+        int C = 1;
+        if (n < 4 * kNumSMs) C = (int)std::min<int64_t>(pa::kMaxUnitsPerCta, (n + kNumSMs - 1) / kNumSMs);
+        while (C > 1 && C * G0 > pa::kMaxConsumerWarps) --C;
+        r.units_per_cta = C;
+    }
+    const int C0 = r.units_per_cta;
     // stages must be a multiple of warps_per_head (see the check below).
     if (r.warps_per_head == 0) {
-        int W = std::min(4, std::max(1, 4 / G0));
-        while (W > 1 && r.stages != 0 && r.stages % W) W >>= 1;
+        int W = C0 > 1 ? 2 : std::min(4, std::max(1, 4 / G0));
+        while (W > 1 && (r.stages != 0 && r.stages % W)) W >>= 1;
+        while (W > 1 && C0 * G0 * W > pa::kMaxConsumerWarps) W >>= 1;
         r.warps_per_head = W;
     }
     if (r.stages == 0) {
         const int W = r.warps_per_head;
-        size_t ring = 64 * 1024;
+        size_t ring = C0 > 1 ? (200 * 1024) / C0 : 64 * 1024;
         const int64_t n = units(G0, r.partition_size);
-        if (n < 4 * kNumSMs) {  // small grid: keep every CTA resident at once
+        if (C0 == 1 && n < 4 * kNumSMs) {  // small grid: keep every CTA resident at once
             const int64_t per_sm = std::max<int64_t>(1, (n + kNumSMs - 1) / kNumSMs);
             ring = std::min<size_t>(ring, (200 * 1024) / per_sm);
         }
@@ -189,8 +201,12 @@ int fill_config(const pa_cache_desc &c, int num_seqs, int max_ctx, pa_decode_con
         return fail(PA_ERR_INVALID, "heads_per_cta %d must be 1, 2, 4 or 8 and divide num_heads %d",
                     G, H);
     const int W = r.warps_per_head;
-    if (!(W == 1 || W == 2 || W == 4) || G * W > pa::kMaxConsumerWarps)
-        return fail(PA_ERR_INVALID, "warps_per_head %d must be 1, 2 or 4 with heads*warps <= %d", W,
+    const int C = r.units_per_cta;
+    if (C < 1 || C > pa::kMaxUnitsPerCta)
+        return fail(PA_ERR_INVALID, "units_per_cta %d must be in [1, %d]", C, pa::kMaxUnitsPerCta);
+    if (!(W == 1 || W == 2 || W == 4) || C * G * W > pa::kMaxConsumerWarps)
+        return fail(PA_ERR_INVALID,
+                    "warps_per_head %d must be 1, 2 or 4 with units*heads*warps <= %d", W,
                     pa::kMaxConsumerWarps);
     if (r.stages < 2 || r.stages > 8)
         return fail(PA_ERR_INVALID, "stages %d must be in [2, 8]", r.stages);
@@ -201,7 +217,7 @@ int fill_config(const pa_cache_desc &c, int num_seqs, int max_ctx, pa_decode_con
     // consumed: with stages % W == 0 every stage belongs to exactly one warp.
     if (r.stages % W)
         return fail(PA_ERR_INVALID, "stages %d must be a multiple of warps_per_head %d", r.stages, W);
-    const pa::SmemLayout lay(B, G, c.head_size, elem_bytes(c), W, r.stages);
+    const pa::SmemLayout lay(B, G, c.head_size, elem_bytes(c), W, r.stages, C);
     if (lay.total > kMaxSmem)
         return fail(PA_ERR_INVALID, "launch shape needs %zu bytes of shared memory (max %zu)",
                     lay.total, kMaxSmem);
@@ -357,6 +373,8 @@ int launch_decode(void *out, const void *query, const void *kc, const void *vc,
     p.heads_per_cta = G;
     p.warps_per_head = W;
     p.stages = cfg.stages;
+    p.units_per_cta = cfg.units_per_cta;
+    p.num_units = (int64_t)S * (c.num_heads / G) * parts;
     p.qk_scale_log2 = scale * (fp8 ? k_scale : 1.0f) * pa::kLog2e;
     p.out_scale = fp8 ? v_scale : 1.0f;
     if (app) {
@@ -375,9 +393,15 @@ int launch_decode(void *out, const void *query, const void *kc, const void *vc,
     if (!kern) return fail(PA_ERR_INVALID, "no kernel for head_size %d block_size %d", D, B);
     rc = ensure_smem_attr(reinterpret_cast<const void *>(kern), device);
     if (rc) return rc;
-    const pa::SmemLayout lay(B, G, D, elem_bytes(c), W, cfg.stages);
-    const dim3 grid(parts, c.num_heads / G, S);
-    const dim3 block(32 * (G * W + 1));
+    const int C = cfg.units_per_cta;
+    const pa::SmemLayout lay(B, G, D, elem_bytes(c), W, cfg.stages, C);
+    // Every unit u is served by CTA u % grid, slot u / grid: grid * C >= units.
+    // Packed CTAs are spread over all SMs (some slots of the last ones idle).
+    const int64_t n_ctas = std::max<int64_t>((p.num_units + C - 1) / C,
+                                             std::min<int64_t>(p.num_units, kNumSMs));
+    if (n_ctas > 0x7fffffff) return fail(PA_ERR_INVALID, "too many work units (%lld)", (long long)p.num_units);
+    const dim3 grid((unsigned)n_ctas);
+    const dim3 block(32 * (C * G * W + 1));
     kern<<<grid, block, lay.total, st>>>(mk, mv, p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "paged_decode_kernel launch");
@@ -512,7 +536,7 @@ int pa_decode_choose_config(pa_cache_desc cache, int num_seqs, int max_context_l
 size_t pa_decode_workspace_size(pa_cache_desc cache, int num_seqs, int max_context_len,
                                 const pa_decode_config *cfg) {
     if (check_cache(cache) || num_seqs <= 0 || max_context_len < 0) return 0;
-    pa_decode_config r = cfg ? *cfg : pa_decode_config{0, 0, 0, 0};
+    pa_decode_config r = cfg ? *cfg : pa_decode_config{0, 0, 0, 0, 0};
     if (fill_config(cache, num_seqs, max_context_len, &r)) return 0;
     return ws_bytes(cache, num_seqs, max_context_len, r);
 }
@@ -559,7 +583,7 @@ int pa_paged_attention_decode_ws(void *out, const void *query, const void *key_c
     if (rc) return rc;
     if (num_seqs == 0) return ok();
     const int bound = (int)std::min<int64_t>(max_context_len, (int64_t)max_blocks_per_seq * cache.block_size);
-    pa_decode_config r = cfg ? *cfg : pa_decode_config{0, 0, 0, 0};
+    pa_decode_config r = cfg ? *cfg : pa_decode_config{0, 0, 0, 0, 0};
     rc = fill_config(cache, num_seqs, bound, &r);
     if (rc) return rc;
     const size_t need = ws_bytes(cache, num_seqs, bound, r);
@@ -600,7 +624,7 @@ extern "C" int pa_paged_attention_decode_append(
                     (long long)key_stride, (long long)value_stride, row);
     const int bound =
         (int)std::min<int64_t>(max_context_len, (int64_t)max_blocks_per_seq * cache.block_size);
-    pa_decode_config r = cfg ? *cfg : pa_decode_config{0, 0, 0, 0};
+    pa_decode_config r = cfg ? *cfg : pa_decode_config{0, 0, 0, 0, 0};
     rc = fill_config(cache, num_seqs, bound, &r);
     if (rc) return rc;
     const size_t need = ws_bytes(cache, num_seqs, bound, r);

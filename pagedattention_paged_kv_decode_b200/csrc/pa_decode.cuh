@@ -6,12 +6,13 @@
 // §2.1 -- but print no kernel):
 //   z_t = scale * k_scale * q . K_t,   out = v_scale * sum_t softmax(z)_t V_t
 //
-// Design (one CTA = one sequence x a group of G heads x one partition of the
-// context):
-//   * a producer warp reads the block-table entries of the partition and
-//     issues, per physical block, two TMA tiled loads -- the K and V tiles
-//     [block_size][G][head_size] of the 4-D cache view [NB][B][H][D] -- into a
-//     ring of shared-memory stages guarded by full/empty mbarriers;
+// Design (one work unit = one sequence x a group of G heads x one partition
+// of the context; a CTA serves C units, each in its own slot):
+//   * a producer warp reads the block-table entries of every slot's
+//     partition and issues, per physical block, two TMA tiled loads -- the K
+//     and V tiles [block_size][G][head_size] of the 4-D cache view
+//     [NB][B][H][D] -- into the slot's ring of shared-memory stages guarded by
+//     full/empty mbarriers, a ring-full per slot first, then in turn;
 //   * G x W consumer warps: warp (g, w) owns head g and every W-th block of
 //     the partition. Per block it forms the logits with 16-byte shared loads
 //     and fp32 FMAs, reduces them with a transposing butterfly (one shuffle
@@ -29,7 +30,8 @@
 namespace pa {
 
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kMaxConsumerWarps = 16;                       // heads_per_cta * warps_per_head
+constexpr int kMaxConsumerWarps = 16;  // units_per_cta * heads_per_cta * warps_per_head
+constexpr int kMaxUnitsPerCta = 4;
 constexpr int kMaxDecodeThreads = 32 * (kMaxConsumerWarps + 1);
 
 struct DecodeParams {
@@ -50,6 +52,8 @@ struct DecodeParams {
     int heads_per_cta;           // G
     int warps_per_head;          // W
     int stages;
+    int units_per_cta;           // C work units (slots) per CTA
+    int64_t num_units;           // num_seqs * (num_heads / G) * max_parts
     float qk_scale_log2;         // scale * k_scale * log2(e)
     float out_scale;             // v_scale (1 for fp16 caches)
     // Fused append (all null/0 for a plain decode): each sequence's new token
@@ -140,23 +144,66 @@ __device__ __forceinline__ void unpack16<true>(const uint4 &raw, float *f) {
     }
 }
 
-// Shared-memory carve-up, identical on host and device.
+// Shared-memory carve-up, identical on host and device. A CTA serves C work
+// units ("slots"); slot j owns a ring of `stages` K/V stages, the appended
+// token's rows and a merge area. The mbarriers of all slots follow the slots:
+// full[C][stages], empty[C][stages], newrow[C].
 struct SmemLayout {
     size_t tile_bytes;   // one K (or V) tile: B * G * D * elem
     size_t stage_bytes;  // K tile + V tile
-    size_t bars_off;     // full[stages], empty[stages], newrow
-    size_t newrow_off;   // appended token's K row then V row: 2 * G * D * elem
-    size_t merge_off;    // W * G * (D + 2) floats
+    size_t newrow_off;   // within a slot: appended K row then V row, 2 * G * D * elem
+    size_t merge_off;    // within a slot: W * G * (D + 2) floats
+    size_t slot_bytes;   // multiple of 128 (TMA destinations stay 128-byte aligned)
+    size_t bars_off;
     size_t total;
-    __host__ __device__ SmemLayout(int B, int G, int D, int elem, int W, int stages) {
+    __host__ __device__ SmemLayout(int B, int G, int D, int elem, int W, int stages, int C) {
         tile_bytes = (size_t)B * G * D * elem;
         stage_bytes = 2 * tile_bytes;
-        bars_off = stage_bytes * stages;
-        newrow_off = (bars_off + 8 * (2 * (size_t)stages + 1) + 15) / 16 * 16;
-        merge_off = newrow_off + 2 * (size_t)G * D * elem;
-        total = merge_off + sizeof(float) * (size_t)W * G * (D + 2);
+        newrow_off = stage_bytes * stages;
+        merge_off = newrow_off + (2 * (size_t)G * D * elem + 15) / 16 * 16;
+        slot_bytes = (merge_off + sizeof(float) * (size_t)W * G * (D + 2) + 127) / 128 * 128;
+        bars_off = slot_bytes * C;
+        total = bars_off + 8 * (size_t)C * (2 * stages + 1);
     }
 };
+
+// One work unit: sequence s, heads h0 .. h0+G-1, partition `part` of the
+// context (tokens t0 .. t1-1 in physical blocks blk0 .. blk0+nblk-1 of the
+// table row). Units are numbered with the partition fastest, then the head
+// group, then the sequence; CTA c serves units c, c + gridDim.x, ... (one per
+// slot), so neighbouring units land on different CTAs.
+struct Unit {
+    int s, h0, part;
+    int L_in, L;       // context length as given and as clamped to the table and bound
+    int n_parts;       // partitions of this context
+    int t0, t1, blk0, nblk;
+    bool live;         // part < n_parts
+    bool append;       // fused append happens in this unit
+};
+
+__device__ __forceinline__ Unit unit_of(const DecodeParams &p, int B, int j) {
+    Unit u;
+    const int64_t id = (int64_t)blockIdx.x + (int64_t)j * gridDim.x;
+    const int HG = p.num_heads / p.heads_per_cta;
+    const bool exists = id < p.num_units;
+    const int64_t idc = exists ? id : 0;
+    u.part = (int)(idc % p.max_parts);
+    const int64_t rest = idc / p.max_parts;
+    u.h0 = (int)(rest % HG) * p.heads_per_cta;
+    u.s = (int)(rest / HG);
+    u.L_in = exists ? __ldg(p.context_lens + u.s) : 0;
+    int L = min(u.L_in, p.max_blocks_per_seq * B);
+    L = min(L, p.max_context_len);
+    u.L = max(L, 0);
+    u.n_parts = (u.L + p.partition_size - 1) / p.partition_size;
+    u.live = exists && u.part < u.n_parts;
+    u.t0 = u.part * p.partition_size;
+    u.t1 = min(u.L, u.t0 + p.partition_size);
+    u.blk0 = u.t0 / B;
+    u.nblk = u.live ? (u.t1 - u.t0 + B - 1) / B : 0;
+    u.append = u.live && p.new_key != nullptr && u.part == u.n_parts - 1 && u.L == u.L_in;
+    return u;
+}
 
 template <int D, int B, bool kFp8>
 __global__ void __launch_bounds__(kMaxDecodeThreads, 1)
@@ -164,247 +211,238 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
     using Geo = Geometry<D, B, kFp8>;
     constexpr int EPL = Geo::EPL, LPR = Geo::LPR, TPG = Geo::TPG, DUP = Geo::DUP;
+    constexpr int EB = Geo::kElemBytes;
 
     extern __shared__ __align__(1024) unsigned char smem[];
-    const int G = p.heads_per_cta, W = p.warps_per_head, stages = p.stages;
-    const SmemLayout lay(B, G, D, Geo::kElemBytes, W, stages);
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + lay.bars_off);
-    uint64_t *empty = full + stages;
-    uint64_t *newrow_bar = empty + stages;  // the appended rows are in shared memory
-    unsigned char *newrow = smem + lay.newrow_off;
-    float *merge = reinterpret_cast<float *>(smem + lay.merge_off);
+    const int G = p.heads_per_cta, W = p.warps_per_head, stages = p.stages, C = p.units_per_cta;
+    const SmemLayout lay(B, G, D, EB, W, stages, C);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + lay.bars_off);
+    uint64_t *full_all = bars;                           // [C][stages]
+    uint64_t *empty_all = bars + (size_t)C * stages;     // [C][stages]
+    uint64_t *newrow_all = bars + 2 * (size_t)C * stages;  // [C]
 
-    const int part = blockIdx.x;
-    const int h0 = blockIdx.y * G;
-    const int s = blockIdx.z;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int n_consumers = G * W;
-
-    // Loads whose addresses do not depend on the context length are issued
-    // before it arrives: the producer's first 32 table entries of this
-    // partition (entries past the row are not read), the consumers' query rows.
-    const int blk0_pre = part * (p.partition_size / B);
-    int pre_blk = 0;
-    if (warp == n_consumers && blk0_pre + lane < p.max_blocks_per_seq)
-        pre_blk = __ldg(p.block_tables + (size_t)s * p.max_blocks_per_seq + blk0_pre + lane);
-    // Fused append: partition 0 is the last partition of every context of up
-    // to one partition, so its producer fetches the appended rows before the
-    // context length is known (other partitions fetch them once it is).
-    const int n_chunks = G * D / 8;  // 16-byte fp16 chunks of G heads
-    uint4 nk[kMaxAppendChunks], nv[kMaxAppendChunks];
-    const bool pre_append = p.new_key != nullptr && part == 0 && warp == n_consumers;
-    if (pre_append) {
-        const uint4 *ks = reinterpret_cast<const uint4 *>(p.new_key + (size_t)s * p.new_key_stride + (size_t)h0 * D);
-        const uint4 *vs = reinterpret_cast<const uint4 *>(p.new_value + (size_t)s * p.new_value_stride + (size_t)h0 * D);
-#pragma unroll
-        for (int k = 0; k < kMaxAppendChunks; ++k) {
-            const int c = lane + 32 * k;
-            if (c < n_chunks) {
-                nk[k] = __ldg(ks + c);
-                nv[k] = __ldg(vs + c);
-            }
-        }
-    }
-    uint4 q_raw[EPL / 8];
-    if (warp < n_consumers) {
-        const uint4 *qp = reinterpret_cast<const uint4 *>(
-            p.query + ((size_t)s * p.num_heads + h0 + warp % G) * D);
-#pragma unroll
-        for (int c = 0; c < EPL / 8; ++c) q_raw[c] = __ldg(qp + (lane % LPR) * (EPL / 8) + c);
-    }
-
-    // Context length, clamped to what the table and the grid can address.
-    const int L_in = __ldg(p.context_lens + s);
-    int L = L_in;
-    const int cap = p.max_blocks_per_seq * B;
-    if (L > cap) {
-        if (threadIdx.x == 0 && part == 0 && blockIdx.y == 0) flag_error(PA_DEV_CTX_OVER_TABLE);
-        L = cap;
-    }
-    if (L > p.max_context_len) {
-        if (threadIdx.x == 0 && part == 0 && blockIdx.y == 0) flag_error(PA_DEV_CTX_OVER_BOUND);
-        L = p.max_context_len;
-    }
-    if (L < 0) L = 0;
-    const int n_parts = (L + p.partition_size - 1) / p.partition_size;
-    if (part >= n_parts) {
-        if (L == 0 && part == 0) {  // empty context: zeros (and no appended token)
-            if (p.slot_out && blockIdx.y == 0 && threadIdx.x == 0) p.slot_out[s] = -1;
-            for (int i = threadIdx.x; i < G * D / 8; i += blockDim.x) {
-                const int g = i / (D / 8), c = i % (D / 8);
-                reinterpret_cast<uint4 *>(p.out + ((size_t)s * p.num_heads + h0 + g) * D)[c] =
-                    make_uint4(0, 0, 0, 0);
-            }
-        }
-        return;
-    }
-    const int t0 = part * p.partition_size;
-    const int t1 = min(L, t0 + p.partition_size);
-    const int blk0 = t0 / B;
-    const int nblk = (t1 - t0 + B - 1) / B;
-
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < stages; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], G);
-        }
-        mbar_init(newrow_bar, 1);
-        fence_mbar_init();
-    }
-    __syncthreads();
+    const int per_slot = G * W;
+    const int n_consumers = C * per_slot;
+    const int n_chunks = G * D / 8;  // 16-byte fp16 chunks of G heads' rows
 
     if (warp == n_consumers) {
-        // ------------------------------------------------------------ producer
+        // ================================================================ producer
+        // Loads whose addresses do not depend on context lengths go first:
+        // the first 32 table entries of every slot's partition.
+        int pre_blk[kMaxUnitsPerCta];
+#pragma unroll
+        for (int j = 0; j < kMaxUnitsPerCta; ++j) {
+            pre_blk[j] = 0;
+            if (j < C) {
+                const int64_t id = (int64_t)blockIdx.x + (int64_t)j * gridDim.x;
+                if (id < p.num_units) {
+                    const int part = (int)(id % p.max_parts);
+                    const int s = (int)(id / p.max_parts / (p.num_heads / G));
+                    const int e = part * (p.partition_size / B) + lane;
+                    if (e < p.max_blocks_per_seq)
+                        pre_blk[j] = __ldg(p.block_tables + (size_t)s * p.max_blocks_per_seq + e);
+                }
+            }
+        }
         if (lane == 0) {
             prefetch_tensor_map(&tmap_k);
             prefetch_tensor_map(&tmap_v);
+            for (int i = 0; i < C * stages; ++i) {
+                mbar_init(&full_all[i], 1);
+                mbar_init(&empty_all[i], G);
+            }
+            for (int j = 0; j < C; ++j) mbar_init(&newrow_all[j], 1);
+            fence_mbar_init();
         }
-        const int32_t *row = p.block_tables + (size_t)s * p.max_blocks_per_seq + blk0;
+        __syncwarp();
+        asm volatile("bar.arrive 1, %0;" ::"r"((n_consumers + 1) * 32) : "memory");  // barriers ready
+
+        Unit u[kMaxUnitsPerCta];
+        int issued[kMaxUnitsPerCta];
+        int cur_blk[kMaxUnitsPerCta];  // 32 table entries of the chunk being issued
+#pragma unroll
+        for (int j = 0; j < kMaxUnitsPerCta; ++j) {
+            if (j < C) u[j] = unit_of(p, B, j);
+            else u[j].live = u[j].append = false, u[j].nblk = 0;
+            issued[j] = 0;
+            cur_blk[j] = pre_blk[j];
+            if (j < C && lane == 0 && u[j].part == 0 && u[j].h0 == 0 &&
+                (int64_t)blockIdx.x + (int64_t)j * gridDim.x < p.num_units) {
+                if (u[j].L_in > p.max_blocks_per_seq * B) flag_error(PA_DEV_CTX_OVER_TABLE);
+                else if (u[j].L_in > p.max_context_len) flag_error(PA_DEV_CTX_OVER_BOUND);
+                // sequences with nothing to append report slot -1
+                if (p.slot_out && !(p.new_key != nullptr && u[j].L == u[j].L_in && u[j].L > 0))
+                    p.slot_out[u[j].s] = -1;
+            }
+        }
         const uint64_t policy = l2_policy_evict_first();
         const uint32_t tx_bytes = (uint32_t)lay.stage_bytes;
+        bool ok = true;
 
-        // Fused append: the CTA owning the sequence's last partition stores the
-        // new token's rows for its G heads. (A clamped context has no valid
-        // position for its new token: no append.)
-        const bool last = p.new_key != nullptr && part == n_parts - 1;
-        const bool append = last && L == L_in;
-        if (last && !append && p.slot_out && blockIdx.y == 0 && lane == 0) p.slot_out[s] = -1;
-        // The appended rows are stored after the tile loads have been issued
-        // (no tile load waits for them). The new token's block id is the
-        // partition's last table entry.
-        int app_blk = 0;
-        if (append) {
-            const int last_entry = nblk - 1;
-            const int from_pre = __shfl_sync(0xffffffffu, pre_blk, last_entry & 31);
-            app_blk = last_entry < 32 ? from_pre : __ldg(row + last_entry);
-            if (!pre_append) {
-                const uint4 *ks = reinterpret_cast<const uint4 *>(p.new_key + (size_t)s * p.new_key_stride + (size_t)h0 * D);
-                const uint4 *vs = reinterpret_cast<const uint4 *>(p.new_value + (size_t)s * p.new_value_stride + (size_t)h0 * D);
+        // Issues the next block of slot j (waiting for its stage to drain).
+        auto issue = [&](int j) {
+            const Unit &x = u[j];
+            const int i = issued[j];
+            if ((i & 31) == 0 && i > 0) {
+                cur_blk[j] = 0;
+                if (i + lane < x.nblk)
+                    cur_blk[j] = __ldg(p.block_tables + (size_t)x.s * p.max_blocks_per_seq + x.blk0 + i + lane);
+            }
+            int blk = __shfl_sync(0xffffffffu, cur_blk[j], i & 31);
+            const bool bad = blk < 0 || blk >= p.num_blocks;
+            if (bad) blk = p.num_blocks;  // out of range: the TMA zero-fills the tile
+            const int st = i % stages, use = i / stages;
+            if (lane == 0) {
+                if (bad) flag_error(PA_DEV_BAD_BLOCK);
+                if (use > 0) ok = mbar_wait(&empty_all[j * stages + st], (use - 1) & 1);
+                if (ok) {
+                    unsigned char *kdst = smem + (size_t)j * lay.slot_bytes + (size_t)st * lay.stage_bytes;
+                    uint64_t *fb = &full_all[j * stages + st];
+                    mbar_arrive_expect_tx(fb, tx_bytes);
+                    tma_load_4d(kdst, &tmap_k, fb, 0, x.h0, 0, blk, policy);
+                    tma_load_4d(kdst + lay.tile_bytes, &tmap_v, fb, 0, x.h0, 0, blk, policy);
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            issued[j] = i + 1;
+        };
+
+        // 1) the first ring-full of every slot (no waits)
+#pragma unroll
+        for (int j = 0; j < kMaxUnitsPerCta; ++j)
+            if (j < C)
+                while (ok && issued[j] < min(u[j].nblk, stages)) issue(j);
+
+        // 2) fused append (a1 + a2): the new token's rows go to the cache for
+        //    later steps and, in cache format, to the slot's shared memory, from
+        //    which the consumers take the appended token (that row of its tile
+        //    is never used, so no tile load waited for this)
+#pragma unroll
+        for (int j = 0; j < kMaxUnitsPerCta; ++j) {
+            if (j < C && u[j].append) {
+                const Unit &x = u[j];
+                const int pos = x.L - 1;
+                const int last = x.nblk - 1;
+                int app_blk = __shfl_sync(0xffffffffu, pre_blk[j], last & 31);
+                if (last >= 32) app_blk = __ldg(p.block_tables + (size_t)x.s * p.max_blocks_per_seq + x.blk0 + last);
+                const bool bad = app_blk < 0 || app_blk >= p.num_blocks;
+                const uint4 *ks = reinterpret_cast<const uint4 *>(p.new_key + (size_t)x.s * p.new_key_stride + (size_t)x.h0 * D);
+                const uint4 *vs = reinterpret_cast<const uint4 *>(p.new_value + (size_t)x.s * p.new_value_stride + (size_t)x.h0 * D);
+                const size_t dst = ((size_t)(bad ? 0 : app_blk) * B + pos % B) * p.num_heads * D + (size_t)x.h0 * D;
+                unsigned char *nrow = smem + (size_t)j * lay.slot_bytes + lay.newrow_off;
 #pragma unroll
                 for (int k = 0; k < kMaxAppendChunks; ++k) {
                     const int c = lane + 32 * k;
                     if (c < n_chunks) {
-                        nk[k] = __ldg(ks + c);
-                        nv[k] = __ldg(vs + c);
+                        const uint4 nk = __ldg(ks + c);
+                        const uint4 nv = __ldg(vs + c);
+                        if constexpr (!kFp8) {
+                            reinterpret_cast<uint4 *>(nrow)[c] = nk;
+                            reinterpret_cast<uint4 *>(nrow + (size_t)G * D * 2)[c] = nv;
+                            if (!bad) {
+                                reinterpret_cast<uint4 *>(static_cast<__half *>(p.key_cache) + dst)[c] = nk;
+                                reinterpret_cast<uint4 *>(static_cast<__half *>(p.value_cache) + dst)[c] = nv;
+                            }
+                        } else {
+                            const uint2 ek = encode8_e4m3(nk, p.k_scale);
+                            const uint2 ev = encode8_e4m3(nv, p.v_scale);
+                            reinterpret_cast<uint2 *>(nrow)[c] = ek;
+                            reinterpret_cast<uint2 *>(nrow + (size_t)G * D)[c] = ev;
+                            if (!bad) {
+                                reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.key_cache) + dst)[c] = ek;
+                                reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.value_cache) + dst)[c] = ev;
+                            }
+                        }
                     }
                 }
+                if (p.slot_out && x.h0 == 0 && lane == 0) p.slot_out[x.s] = bad ? -1 : app_blk * B + pos % B;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&newrow_all[j]);  // release: the rows are in shared memory
             }
         }
 
-        bool ok = true;
-        int stage = 0, use = 0;
-        for (int base = 0; base < nblk && ok; base += 32) {
-            int my_blk = pre_blk;  // entries 0..31 were prefetched above
-            if (base > 0 && base + lane < nblk) my_blk = __ldg(row + base + lane);
-            const int cnt = min(32, nblk - base);
-            for (int j = 0; j < cnt; ++j) {
-                int blk = __shfl_sync(0xffffffffu, my_blk, j);
-                const bool bad = blk < 0 || blk >= p.num_blocks;
-                if (bad) blk = p.num_blocks;  // out of range: the TMA zero-fills the tile
-                if (lane == 0) {
-                    if (bad) flag_error(PA_DEV_BAD_BLOCK);
-                    if (use > 0) ok = mbar_wait(&empty[stage], (use - 1) & 1);
-                    if (ok) {
-                        unsigned char *kdst = smem + (size_t)stage * lay.stage_bytes;
-                        mbar_arrive_expect_tx(&full[stage], tx_bytes);
-                        tma_load_4d(kdst, &tmap_k, &full[stage], 0, h0, 0, blk, policy);
-                        tma_load_4d(kdst + lay.tile_bytes, &tmap_v, &full[stage], 0, h0, 0, blk,
-                                    policy);
-                    }
-                }
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) break;
-                if (++stage == stages) {
-                    stage = 0;
-                    ++use;
-                }
-            }
-        }
-        if (append) {
-            // a1 + a2 for this sequence and these heads. The rows go to the
-            // cache for later steps and, in cache format, to shared memory,
-            // from which the consumers take the appended token (that row of
-            // its tile is never used, so the tile load did not wait for this).
-            const int pos = L - 1;
-            const bool bad = app_blk < 0 || app_blk >= p.num_blocks;
-            const size_t dst = ((size_t)(bad ? 0 : app_blk) * B + pos % B) * p.num_heads * D + (size_t)h0 * D;
+        // 3) the rest, one block per slot in turn
+        bool more = true;
+        while (ok && more) {
+            more = false;
 #pragma unroll
-            for (int k = 0; k < kMaxAppendChunks; ++k) {
-                const int c = lane + 32 * k;
-                if (c < n_chunks) {
-                    if constexpr (!kFp8) {
-                        reinterpret_cast<uint4 *>(newrow)[c] = nk[k];
-                        reinterpret_cast<uint4 *>(newrow + (size_t)G * D * 2)[c] = nv[k];
-                        if (!bad) {
-                            reinterpret_cast<uint4 *>(static_cast<__half *>(p.key_cache) + dst)[c] = nk[k];
-                            reinterpret_cast<uint4 *>(static_cast<__half *>(p.value_cache) + dst)[c] = nv[k];
-                        }
-                    } else {
-                        const uint2 ek = encode8_e4m3(nk[k], p.k_scale);
-                        const uint2 ev = encode8_e4m3(nv[k], p.v_scale);
-                        reinterpret_cast<uint2 *>(newrow)[c] = ek;
-                        reinterpret_cast<uint2 *>(newrow + (size_t)G * D)[c] = ev;
-                        if (!bad) {
-                            reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.key_cache) + dst)[c] = ek;
-                            reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.value_cache) + dst)[c] = ev;
-                        }
-                    }
+            for (int j = 0; j < kMaxUnitsPerCta; ++j) {
+                if (j < C && ok && issued[j] < u[j].nblk) {
+                    issue(j);
+                    more = true;
                 }
             }
-            if (p.slot_out && blockIdx.y == 0 && lane == 0) p.slot_out[s] = bad ? -1 : app_blk * B + pos % B;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(newrow_bar);  // release: the rows are in shared memory
         }
         return;
     }
 
-    // --------------------------------------------------------------- consumers
-    const int g = warp % G;
-    const int w = warp / G;
-    const int h = h0 + g;
+    // ================================================================ consumers
+    const int slot = warp / per_slot;
+    const int gw = warp % per_slot;
+    const int g = gw % G;
+    const int w = gw / G;
     const int grp = lane / LPR;
     const int sub = lane % LPR;
 
-    float q[EPL];
+    // Query row: its address depends on the unit id only.
+    uint4 q_raw[EPL / 8];
     {
+        const int64_t id = (int64_t)blockIdx.x + (int64_t)slot * gridDim.x;
+        const int64_t idc = id < p.num_units ? id : 0;
+        const int64_t rest = idc / p.max_parts;
+        const int hq = (int)(rest % (p.num_heads / G)) * G + g;
+        const int sq = (int)(rest / (p.num_heads / G));
+        const uint4 *qp = reinterpret_cast<const uint4 *>(p.query + ((size_t)sq * p.num_heads + hq) * D);
 #pragma unroll
-        for (int c = 0; c < EPL / 8; ++c) unpack16<false>(q_raw[c], q + 8 * c);  // fp16 query
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) q[e] *= p.qk_scale_log2;
+        for (int c = 0; c < EPL / 8; ++c) q_raw[c] = __ldg(qp + sub * (EPL / 8) + c);
     }
+    const Unit x = unit_of(p, B, slot);
+    const int h = x.h0 + g;
+    unsigned char *slot_base = smem + (size_t)slot * lay.slot_bytes;
+    uint64_t *full = full_all + slot * stages;
+    uint64_t *empty = empty_all + slot * stages;
+    float *merge = reinterpret_cast<float *>(slot_base + lay.merge_off);
+    asm volatile("bar.sync 1, %0;" ::"r"((n_consumers + 1) * 32) : "memory");  // barriers ready
+
+    if (!x.live) {
+        // empty context: zeros (partition 0 of a context of length 0)
+        const int64_t id = (int64_t)blockIdx.x + (int64_t)slot * gridDim.x;
+        if (id < p.num_units && x.L == 0 && x.part == 0 && w == 0 && lane < D / 8)
+            reinterpret_cast<uint4 *>(p.out + ((size_t)x.s * p.num_heads + h) * D)[lane] = make_uint4(0, 0, 0, 0);
+        return;  // (all warps of this slot leave together: no merge barrier to meet)
+    }
+
+    float q[EPL];
+#pragma unroll
+    for (int c = 0; c < EPL / 8; ++c) unpack16<false>(q_raw[c], q + 8 * c);  // fp16 query
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) q[e] *= p.qk_scale_log2;
 
     float m = -INFINITY, l = 0.f;
     float acc[EPL];
 #pragma unroll
     for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
 
-    const size_t row_stride = (size_t)G * D * Geo::kElemBytes;  // bytes between tokens in a tile
-    const size_t head_off = (size_t)g * D * Geo::kElemBytes + (size_t)sub * 16;
+    const size_t row_stride = (size_t)G * D * EB;  // bytes between tokens in a tile
+    const size_t head_off = (size_t)g * D * EB + (size_t)sub * 16;
     // The appended token (fused append only) is read from shared memory.
-    const bool appended = p.new_key != nullptr && part == n_parts - 1 && L == L_in;
-    const int t_new_block = appended ? (L - 1 - t0) / B : -1;  // block index within the partition
-    const int t_new_row = appended ? (L - 1) % B : -1;
-    bool ok = true;
+    const int t_new_block = x.append ? (x.L - 1 - x.t0) / B : -1;
+    const int t_new_row = x.append ? (x.L - 1) % B : -1;
+    const unsigned char *knew = slot_base + lay.newrow_off;
+    const unsigned char *vnew = knew + (size_t)G * D * EB;
     int stage = w % stages, use = w / stages;
-    for (int i = w; i < nblk; i += W) {
-        if (!mbar_wait(&full[stage], use & 1)) {
-            ok = false;
-            break;
-        }
-        const unsigned char *ktile = smem + (size_t)stage * lay.stage_bytes;
+    for (int i = w; i < x.nblk; i += W) {
+        if (!mbar_wait(&full[stage], use & 1)) break;
+        const unsigned char *ktile = slot_base + (size_t)stage * lay.stage_bytes;
         const unsigned char *vtile = ktile + lay.tile_bytes;
-        const int valid = min(B, t1 - (t0 + i * B));  // tokens of this block inside the context
+        const int valid = min(B, x.t1 - (x.t0 + i * B));  // tokens of this block inside the context
         int t_new = -1;
         if (i == t_new_block) {
-            if (!mbar_wait(newrow_bar, 0)) {
-                ok = false;
-                break;
-            }
+            if (!mbar_wait(&newrow_all[slot], 0)) break;
             t_new = t_new_row;
         }
-        const unsigned char *knew = newrow;
-        const unsigned char *vnew = newrow + (size_t)G * D * Geo::kElemBytes;
 
         // ---- logits of this lane group's TPG tokens
         float part_dot[TPG];
@@ -455,7 +493,6 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
             ++use;
         }
     }
-    (void)ok;
 
     // ---- reduce this warp's state: l over all lanes, acc over lane groups
     l = warp_sum(l) * (1.0f / DUP);
@@ -465,18 +502,18 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
         for (int e = 0; e < EPL; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], mask);
     }
 
-    // ---- merge the W warps of each head through shared memory
+    // ---- merge the W warps of each head through the slot's shared memory
     if (W > 1) {
-        float *slot = merge + (size_t)(w * G + g) * (D + 2);
+        float *mine = merge + (size_t)(w * G + g) * (D + 2);
         if (grp == 0) {
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) slot[sub * EPL + e] = acc[e];
+            for (int e = 0; e < EPL; ++e) mine[sub * EPL + e] = acc[e];
         }
         if (lane == 0) {
-            slot[D] = m;
-            slot[D + 1] = l;
+            mine[D] = m;
+            mine[D + 1] = l;
         }
-        asm volatile("bar.sync 1, %0;" ::"r"(n_consumers * 32) : "memory");
+        asm volatile("bar.sync %0, %1;" ::"r"(2 + slot), "r"(per_slot * 32) : "memory");
         if (w != 0) return;
         float M = -INFINITY;
         for (int k = 0; k < W; ++k) M = fmaxf(M, merge[(size_t)(k * G + g) * (D + 2) + D]);
@@ -496,8 +533,8 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
 
     if (grp != 0) return;
     const float inv_l = 1.0f / l;
-    if (n_parts == 1) {
-        __half *op = p.out + ((size_t)s * p.num_heads + h) * D + sub * EPL;
+    if (x.n_parts == 1) {
+        __half *op = p.out + ((size_t)x.s * p.num_heads + h) * D + sub * EPL;
 #pragma unroll
         for (int c = 0; c < EPL / 8; ++c) {
             uint4 pk;
@@ -509,7 +546,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
             reinterpret_cast<uint4 *>(op)[c] = pk;
         }
     } else {
-        const size_t idx = ((size_t)s * p.num_heads + h) * p.max_parts + part;
+        const size_t idx = ((size_t)x.s * p.num_heads + h) * p.max_parts + x.part;
         float *op = p.ws_o + idx * D + sub * EPL;
 #pragma unroll
         for (int c = 0; c < EPL / 4; ++c)

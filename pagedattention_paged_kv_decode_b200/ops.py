@@ -100,7 +100,7 @@ def _config(config) -> DecodeConfig | None:
 
 
 def choose_config(key_cache: torch.Tensor, num_seqs: int, max_context_len: int, config=None) -> dict:
-    cfg = _config(config) or DecodeConfig(0, 0, 0, 0)
+    cfg = _config(config) or DecodeConfig(0, 0, 0, 0, 0)
     check(lib().pa_decode_choose_config(cache_desc(key_cache), num_seqs, max_context_len,
                                         ctypes.byref(cfg)))
     return cfg.as_dict()

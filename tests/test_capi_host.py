@@ -90,7 +90,8 @@ def test_bad_scales_and_counts():
 
 def _choose(desc, S, maxL, **kw):
     cfg = capi.DecodeConfig(kw.get("partition_size", 0), kw.get("heads_per_cta", 0),
-                            kw.get("warps_per_head", 0), kw.get("stages", 0))
+                            kw.get("warps_per_head", 0), kw.get("stages", 0),
+                            kw.get("units_per_cta", 0))
     rc = capi.lib().pa_decode_choose_config(desc, S, maxL, ctypes.byref(cfg))
     return rc, cfg
 
@@ -107,6 +108,10 @@ def test_config_choice_is_valid_and_fills_the_gpu():
         assert desc.num_heads % cfg.heads_per_cta == 0
         units = S * (desc.num_heads // cfg.heads_per_cta) * -(-maxL // cfg.partition_size)
         assert units >= 3 * 148 or cfg.heads_per_cta == 1
+        assert cfg.stages % cfg.warps_per_head == 0
+        assert cfg.units_per_cta * cfg.heads_per_cta * cfg.warps_per_head <= 16
+        ctas = max(-(-units // cfg.units_per_cta), min(units, 148))   # the library's grid
+        assert ctas * cfg.units_per_cta >= units and ctas >= min(units, 148)
 
 
 def test_config_validation_and_workspace_size():
@@ -115,6 +120,8 @@ def test_config_validation_and_workspace_size():
     assert _choose(desc, 16, 512, heads_per_cta=3)[0] == capi.PA_ERR_INVALID
     assert _choose(desc, 16, 512, heads_per_cta=8, warps_per_head=4)[0] == capi.PA_ERR_INVALID  # 32 warps
     assert _choose(desc, 16, 512, stages=9)[0] == capi.PA_ERR_INVALID
+    assert _choose(desc, 16, 512, units_per_cta=5)[0] == capi.PA_ERR_INVALID
+    assert _choose(desc, 16, 512, units_per_cta=4, heads_per_cta=2, warps_per_head=4)[0] == capi.PA_ERR_INVALID
     # a warp waits on a stage's barrier by phase parity: stages must be a multiple of warps
     assert _choose(desc, 16, 512, heads_per_cta=1, warps_per_head=4, stages=2)[0] == capi.PA_ERR_INVALID
     assert _choose(desc, 16, 512, heads_per_cta=2, warps_per_head=2, stages=3)[0] == capi.PA_ERR_INVALID
@@ -129,7 +136,7 @@ def test_config_validation_and_workspace_size():
     ws = L.pa_decode_workspace_size(desc, 16, 512, ctypes.byref(cfg))
     lse = -(-(16 * 32 * 4 * 4) // 256) * 256
     assert ws == lse + 16 * 32 * 4 * 128 * 4
-    one = capi.DecodeConfig(512, 2, 2, 4)
+    one = capi.DecodeConfig(512, 2, 2, 4, 1)
     assert L.pa_decode_workspace_size(desc, 16, 512, ctypes.byref(one)) == 0
     small = L.pa_paged_attention_decode_ws(P, P, P, P, desc, P, 32, P, 16, 512, 0.1, 1.0, 1.0,
                                            ctypes.byref(cfg), P, ws - 1, None)

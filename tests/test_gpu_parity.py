@@ -98,10 +98,14 @@ LAUNCH = [
     dict(partition_size=512, heads_per_cta=2, warps_per_head=4, stages=8),
     dict(partition_size=2048, heads_per_cta=1, warps_per_head=2, stages=2),
     dict(partition_size=128, heads_per_cta=1, warps_per_head=1, stages=3),
+    dict(partition_size=64, heads_per_cta=1, warps_per_head=2, stages=4, units_per_cta=4),
+    dict(partition_size=32, heads_per_cta=2, warps_per_head=1, stages=3, units_per_cta=3),
+    dict(partition_size=512, heads_per_cta=1, warps_per_head=1, stages=2, units_per_cta=2),
+    dict(partition_size=128, heads_per_cta=4, warps_per_head=2, stages=2, units_per_cta=2),
 ]
 
 
-@pytest.mark.parametrize("launch", LAUNCH, ids=lambda d: "p{partition_size}_g{heads_per_cta}_w{warps_per_head}_s{stages}".format(**d))
+@pytest.mark.parametrize("launch", LAUNCH, ids=lambda d: "p{partition_size}_g{heads_per_cta}_w{warps_per_head}_s{stages}_c{}".format(d.get("units_per_cta", 1), **d))
 @pytest.mark.parametrize("D,B,kv", [(128, 16, "f16"), (128, 32, "f16"), (128, 16, "e4m3"), (64, 32, "e4m3")])
 def test_launch_shapes(cuda_device, launch, D, B, kv):
     if launch["partition_size"] % B:
@@ -120,7 +124,8 @@ def test_launch_shapes(cuda_device, launch, D, B, kv):
 @pytest.mark.parametrize("kv", ["f16", "e4m3"])
 def test_nan_poison_is_never_touched(cuda_device, kv):
     w = ragged_case(128, 16, kv, seed=3, poison=W.POISON_NAN)
-    for launch in (None, dict(partition_size=32, heads_per_cta=2, warps_per_head=2, stages=4)):
+    for launch in (None, dict(partition_size=32, heads_per_cta=2, warps_per_head=2, stages=4),
+                   dict(partition_size=64, heads_per_cta=1, warps_per_head=2, stages=2, units_per_cta=3)):
         for fused in (True, False):
             dw = run_step(w, cuda_device, config=launch, fused=fused)
             compare_step(w, dw, list(range(w.num_seqs)), check_all_blocks=False)
