@@ -170,7 +170,8 @@ int fill_config(const pa_cache_desc &c, int num_seqs, int max_ctx, pa_decode_con
         const int64_t n = units(G0, r.partition_size);
         int C = 1;
         if (n < 4 * kNumSMs) C = (int)std::min<int64_t>(pa::kMaxUnitsPerCta, (n + kNumSMs - 1) / kNumSMs);
-        while (C > 1 && C * G0 > pa::kMaxConsumerWarps) --C;
+        const int Wgiven = std::max(1, r.warps_per_head);
+        while (C > 1 && C * G0 * Wgiven > pa::kMaxConsumerWarps) --C;
         r.units_per_cta = C;
     }
     const int C0 = r.units_per_cta;

@@ -121,6 +121,10 @@ def test_config_validation_and_workspace_size():
     assert _choose(desc, 16, 512, heads_per_cta=8, warps_per_head=4)[0] == capi.PA_ERR_INVALID  # 32 warps
     assert _choose(desc, 16, 512, stages=9)[0] == capi.PA_ERR_INVALID
     assert _choose(desc, 16, 512, units_per_cta=5)[0] == capi.PA_ERR_INVALID
+    # a given warps_per_head bounds the default number of units per CTA
+    small = capi.CacheDesc(100, 16, 4, 128, 0)
+    rc, c = _choose(small, 12, 1100, partition_size=64, heads_per_cta=4, warps_per_head=4, stages=4)
+    assert rc == 0 and c.units_per_cta * 4 * 4 <= 16
     assert _choose(desc, 16, 512, units_per_cta=4, heads_per_cta=2, warps_per_head=4)[0] == capi.PA_ERR_INVALID
     # a warp waits on a stage's barrier by phase parity: stages must be a multiple of warps
     assert _choose(desc, 16, 512, heads_per_cta=1, warps_per_head=4, stages=2)[0] == capi.PA_ERR_INVALID
