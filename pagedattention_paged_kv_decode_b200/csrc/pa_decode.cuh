@@ -70,7 +70,6 @@ struct DecodeParams {
     float v_scale;
 };
 
-constexpr int kMaxAppendChunks = 4;  // 16-byte chunks per lane: G*D/8 <= 128
 
 // Lane geometry of a consumer warp. Each lane holds EPL consecutive elements
 // of a K/V row (16 bytes), LPR lanes cover one row of head_size elements,
@@ -145,13 +144,12 @@ __device__ __forceinline__ void unpack16<true>(const uint4 &raw, float *f) {
 }
 
 // Shared-memory carve-up, identical on host and device. A CTA serves C work
-// units ("slots"); slot j owns a ring of `stages` K/V stages, the appended
-// token's rows and a merge area. The mbarriers of all slots follow the slots:
-// full[C][stages], empty[C][stages], newrow[C].
+// units ("slots"); slot j owns a ring of `stages` K/V stages and a merge
+// area. The mbarriers of all slots follow the slots: full[C][stages],
+// empty[C][stages].
 struct SmemLayout {
     size_t tile_bytes;   // one K (or V) tile: B * G * D * elem
     size_t stage_bytes;  // K tile + V tile
-    size_t newrow_off;   // within a slot: appended K row then V row, 2 * G * D * elem
     size_t merge_off;    // within a slot: W * G * (D + 2) floats
     size_t slot_bytes;   // multiple of 128 (TMA destinations stay 128-byte aligned)
     size_t bars_off;
@@ -159,11 +157,10 @@ struct SmemLayout {
     __host__ __device__ SmemLayout(int B, int G, int D, int elem, int W, int stages, int C) {
         tile_bytes = (size_t)B * G * D * elem;
         stage_bytes = 2 * tile_bytes;
-        newrow_off = stage_bytes * stages;
-        merge_off = newrow_off + (2 * (size_t)G * D * elem + 15) / 16 * 16;
+        merge_off = stage_bytes * stages;
         slot_bytes = (merge_off + sizeof(float) * (size_t)W * G * (D + 2) + 127) / 128 * 128;
         bars_off = slot_bytes * C;
-        total = bars_off + 8 * (size_t)C * (2 * stages + 1);
+        total = bars_off + 8 * (size_t)C * 2 * stages;
     }
 };
 
@@ -219,13 +216,11 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + lay.bars_off);
     uint64_t *full_all = bars;                           // [C][stages]
     uint64_t *empty_all = bars + (size_t)C * stages;     // [C][stages]
-    uint64_t *newrow_all = bars + 2 * (size_t)C * stages;  // [C]
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int per_slot = G * W;
     const int n_consumers = C * per_slot;
-    const int n_chunks = G * D / 8;  // 16-byte fp16 chunks of G heads' rows
 
     if (warp == n_consumers) {
         // ================================================================ producer
@@ -253,7 +248,6 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 mbar_init(&full_all[i], 1);
                 mbar_init(&empty_all[i], G);
             }
-            for (int j = 0; j < C; ++j) mbar_init(&newrow_all[j], 1);
             fence_mbar_init();
         }
         __syncwarp();
@@ -263,11 +257,14 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
         int issued[kMaxUnitsPerCta];
         int cur_blk[kMaxUnitsPerCta];  // 32 table entries of the chunk being issued
 #pragma unroll
-        for (int j = 0; j < kMaxUnitsPerCta; ++j) {
+        for (int j = 0; j < kMaxUnitsPerCta; ++j) {  // independent loads: all in flight together
             if (j < C) u[j] = unit_of(p, B, j);
             else u[j].live = u[j].append = false, u[j].nblk = 0;
             issued[j] = 0;
             cur_blk[j] = pre_blk[j];
+        }
+#pragma unroll
+        for (int j = 0; j < kMaxUnitsPerCta; ++j) {
             if (j < C && lane == 0 && u[j].part == 0 && u[j].h0 == 0 &&
                 (int64_t)blockIdx.x + (int64_t)j * gridDim.x < p.num_units) {
                 if (u[j].L_in > p.max_blocks_per_seq * B) flag_error(PA_DEV_CTX_OVER_TABLE);
@@ -315,55 +312,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
             if (j < C)
                 while (ok && issued[j] < min(u[j].nblk, stages)) issue(j);
 
-        // 2) fused append (a1 + a2): the new token's rows go to the cache for
-        //    later steps and, in cache format, to the slot's shared memory, from
-        //    which the consumers take the appended token (that row of its tile
-        //    is never used, so no tile load waited for this)
-#pragma unroll
-        for (int j = 0; j < kMaxUnitsPerCta; ++j) {
-            if (j < C && u[j].append) {
-                const Unit &x = u[j];
-                const int pos = x.L - 1;
-                const int last = x.nblk - 1;
-                int app_blk = __shfl_sync(0xffffffffu, pre_blk[j], last & 31);
-                if (last >= 32) app_blk = __ldg(p.block_tables + (size_t)x.s * p.max_blocks_per_seq + x.blk0 + last);
-                const bool bad = app_blk < 0 || app_blk >= p.num_blocks;
-                const uint4 *ks = reinterpret_cast<const uint4 *>(p.new_key + (size_t)x.s * p.new_key_stride + (size_t)x.h0 * D);
-                const uint4 *vs = reinterpret_cast<const uint4 *>(p.new_value + (size_t)x.s * p.new_value_stride + (size_t)x.h0 * D);
-                const size_t dst = ((size_t)(bad ? 0 : app_blk) * B + pos % B) * p.num_heads * D + (size_t)x.h0 * D;
-                unsigned char *nrow = smem + (size_t)j * lay.slot_bytes + lay.newrow_off;
-#pragma unroll
-                for (int k = 0; k < kMaxAppendChunks; ++k) {
-                    const int c = lane + 32 * k;
-                    if (c < n_chunks) {
-                        const uint4 nk = __ldg(ks + c);
-                        const uint4 nv = __ldg(vs + c);
-                        if constexpr (!kFp8) {
-                            reinterpret_cast<uint4 *>(nrow)[c] = nk;
-                            reinterpret_cast<uint4 *>(nrow + (size_t)G * D * 2)[c] = nv;
-                            if (!bad) {
-                                reinterpret_cast<uint4 *>(static_cast<__half *>(p.key_cache) + dst)[c] = nk;
-                                reinterpret_cast<uint4 *>(static_cast<__half *>(p.value_cache) + dst)[c] = nv;
-                            }
-                        } else {
-                            const uint2 ek = encode8_e4m3(nk, p.k_scale);
-                            const uint2 ev = encode8_e4m3(nv, p.v_scale);
-                            reinterpret_cast<uint2 *>(nrow)[c] = ek;
-                            reinterpret_cast<uint2 *>(nrow + (size_t)G * D)[c] = ev;
-                            if (!bad) {
-                                reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.key_cache) + dst)[c] = ek;
-                                reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.value_cache) + dst)[c] = ev;
-                            }
-                        }
-                    }
-                }
-                if (p.slot_out && x.h0 == 0 && lane == 0) p.slot_out[x.s] = bad ? -1 : app_blk * B + pos % B;
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&newrow_all[j]);  // release: the rows are in shared memory
-            }
-        }
-
-        // 3) the rest, one block per slot in turn
+        // 2) the rest, one block per slot in turn
         bool more = true;
         while (ok && more) {
             more = false;
@@ -387,7 +336,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int sub = lane % LPR;
 
     // Query row: its address depends on the unit id only.
-    uint4 q_raw[EPL / 8];
+    uint4 q_raw[EPL / 8], nk_raw[EPL / 8], nv_raw[EPL / 8];
     {
         const int64_t id = (int64_t)blockIdx.x + (int64_t)slot * gridDim.x;
         const int64_t idc = id < p.num_units ? id : 0;
@@ -397,6 +346,17 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const uint4 *qp = reinterpret_cast<const uint4 *>(p.query + ((size_t)sq * p.num_heads + hq) * D);
 #pragma unroll
         for (int c = 0; c < EPL / 8; ++c) q_raw[c] = __ldg(qp + sub * (EPL / 8) + c);
+        // Fused append: this lane's dims of the head's new K/V row, fetched
+        // with the query (used only if this unit turns out to hold the token).
+        if (p.new_key != nullptr) {
+            const uint4 *kp = reinterpret_cast<const uint4 *>(p.new_key + (size_t)sq * p.new_key_stride + (size_t)hq * D);
+            const uint4 *vp = reinterpret_cast<const uint4 *>(p.new_value + (size_t)sq * p.new_value_stride + (size_t)hq * D);
+#pragma unroll
+            for (int c = 0; c < EPL / 8; ++c) {
+                nk_raw[c] = __ldg(kp + sub * (EPL / 8) + c);
+                nv_raw[c] = __ldg(vp + sub * (EPL / 8) + c);
+            }
+        }
     }
     const Unit x = unit_of(p, B, slot);
     const int h = x.h0 + g;
@@ -427,30 +387,53 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
 
     const size_t row_stride = (size_t)G * D * EB;  // bytes between tokens in a tile
     const size_t head_off = (size_t)g * D * EB + (size_t)sub * 16;
-    // The appended token (fused append only) is read from shared memory.
-    const int t_new_block = x.append ? (x.L - 1 - x.t0) / B : -1;
-    const int t_new_row = x.append ? (x.L - 1) % B : -1;
-    const unsigned char *knew = slot_base + lay.newrow_off;
-    const unsigned char *vnew = knew + (size_t)G * D * EB;
+    // Fused append (a1 + a2): the unit holding position L-1 takes the new
+    // token from registers, in cache format (E4M3 codes for an fp8 cache, so
+    // that it is used exactly as a later step will read it back), and the
+    // first warp of each head stores the head's row into the token's slot.
+    // That row of the tile is never read, so no tile load waits for the store.
+    int t_new_block = -1, t_new_row = -1;
+    uint4 k_new = make_uint4(0, 0, 0, 0), v_new = make_uint4(0, 0, 0, 0);
+    if (x.append) {
+        const int pos = x.L - 1;
+        t_new_block = (pos - x.t0) / B;
+        t_new_row = pos % B;
+        if constexpr (!kFp8) {
+            k_new = nk_raw[0];
+            v_new = nv_raw[0];
+        } else {
+            const uint2 k0 = encode8_e4m3(nk_raw[0], p.k_scale), k1 = encode8_e4m3(nk_raw[1], p.k_scale);
+            const uint2 v0 = encode8_e4m3(nv_raw[0], p.v_scale), v1 = encode8_e4m3(nv_raw[1], p.v_scale);
+            k_new = make_uint4(k0.x, k0.y, k1.x, k1.y);
+            v_new = make_uint4(v0.x, v0.y, v1.x, v1.y);
+        }
+        if (w == 0 && grp == 0) {
+            const int blk = __ldg(p.block_tables + (size_t)x.s * p.max_blocks_per_seq + pos / B);
+            const bool bad = blk < 0 || blk >= p.num_blocks;  // flagged where its tile is loaded
+            if (!bad) {
+                const size_t dst = (((size_t)blk * B + pos % B) * p.num_heads + h) * D * EB + (size_t)sub * 16;
+                *reinterpret_cast<uint4 *>(static_cast<unsigned char *>(p.key_cache) + dst) = k_new;
+                *reinterpret_cast<uint4 *>(static_cast<unsigned char *>(p.value_cache) + dst) = v_new;
+            }
+            if (p.slot_out && h == 0 && sub == 0) p.slot_out[x.s] = bad ? -1 : blk * B + pos % B;
+        }
+    }
     int stage = w % stages, use = w / stages;
     for (int i = w; i < x.nblk; i += W) {
         if (!mbar_wait(&full[stage], use & 1)) break;
         const unsigned char *ktile = slot_base + (size_t)stage * lay.stage_bytes;
         const unsigned char *vtile = ktile + lay.tile_bytes;
         const int valid = min(B, x.t1 - (x.t0 + i * B));  // tokens of this block inside the context
-        int t_new = -1;
-        if (i == t_new_block) {
-            if (!mbar_wait(&newrow_all[slot], 0)) break;
-            t_new = t_new_row;
-        }
+        const int t_new = (i == t_new_block) ? t_new_row : -1;
 
         // ---- logits of this lane group's TPG tokens
         float part_dot[TPG];
 #pragma unroll
         for (int j = 0; j < TPG; ++j) {
             const int t = grp * TPG + j;
-            const unsigned char *krow = (t == t_new) ? knew : ktile + t * row_stride;
-            const uint4 raw = *reinterpret_cast<const uint4 *>(krow + head_off);
+            uint4 raw;
+            if (t == t_new) raw = k_new;
+            else raw = *reinterpret_cast<const uint4 *>(ktile + t * row_stride + head_off);
             float k[EPL];
             unpack16<kFp8>(raw, k);
             float d = 0.f;
@@ -477,8 +460,9 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
             const int t = grp * TPG + j;
             const float pj = __shfl_sync(0xffffffffu, pz, grp * LPR + j * DUP);
             if (t < valid) {
-                const unsigned char *vrow = (t == t_new) ? vnew : vtile + t * row_stride;
-                const uint4 raw = *reinterpret_cast<const uint4 *>(vrow + head_off);
+                uint4 raw;
+                if (t == t_new) raw = v_new;
+                else raw = *reinterpret_cast<const uint4 *>(vtile + t * row_stride + head_off);
                 float v[EPL];
                 unpack16<kFp8>(raw, v);
 #pragma unroll
