@@ -163,17 +163,10 @@ int fill_config(const pa_cache_desc &c, int num_seqs, int max_ctx, pa_decode_con
         while (P > 4 * B && units(G0, P) < 3 * kNumSMs) P >>= 1;
         r.partition_size = P;
     }
-    // A small grid (fewer units than four per SM) packs several units into
-    // each CTA, each with its own ring, so that one CTA per SM keeps nearly
-    // all of its units' blocks in flight at once.
-    if (r.units_per_cta == 0) {
-        const int64_t n = units(G0, r.partition_size);
-        int C = 1;
-        if (n < 4 * kNumSMs) C = (int)std::min<int64_t>(pa::kMaxUnitsPerCta, (n + kNumSMs - 1) / kNumSMs);
-        const int Wgiven = std::max(1, r.warps_per_head);
-        while (C > 1 && C * G0 * Wgiven > pa::kMaxConsumerWarps) --C;
-        r.units_per_cta = C;
-    }
+    // One unit per CTA by default: measured on B200, packing 2-4 units of a
+    // small batch into one CTA (one producer thread issuing every slot's tile
+    // loads) was slower than one CTA per unit with several CTAs per SM.
+    if (r.units_per_cta == 0) r.units_per_cta = 1;
     const int C0 = r.units_per_cta;
     // stages must be a multiple of warps_per_head (see the check below).
     if (r.warps_per_head == 0) {
@@ -376,7 +369,8 @@ int launch_decode(void *out, const void *query, const void *kc, const void *vc,
     p.stages = cfg.stages;
     p.units_per_cta = cfg.units_per_cta;
     p.num_units = (int64_t)S * (c.num_heads / G) * parts;
-    p.qk_scale_log2 = scale * (fp8 ? k_scale : 1.0f) * pa::kLog2e;
+    p.qk_scale_log2 = scale * pa::kLog2e;
+    p.logit_k_scale = fp8 ? k_scale : 1.0f;
     p.out_scale = fp8 ? v_scale : 1.0f;
     if (app) {
         p.new_key = static_cast<const __half *>(app->new_key);

@@ -54,7 +54,8 @@ struct DecodeParams {
     int stages;
     int units_per_cta;           // C work units (slots) per CTA
     int64_t num_units;           // num_seqs * (num_heads / G) * max_parts
-    float qk_scale_log2;         // scale * k_scale * log2(e)
+    float qk_scale_log2;         // scale * log2(e)
+    float logit_k_scale;         // k_scale, applied to each E4M3 logit (1 for fp16 caches)
     float out_scale;             // v_scale (1 for fp16 caches)
     // Fused append (all null/0 for a plain decode): each sequence's new token
     // at position L-1 is stored into its slot before the block holding it is
@@ -374,11 +375,26 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
         return;  // (all warps of this slot leave together: no merge barrier to meet)
     }
 
-    float q[EPL];
+    // fp16 caches: query in fp32, pre-scaled by scale*log2(e). E4M3 caches:
+    // the pre-scaled query rounded to f16 pairs, multiplied exactly against
+    // the decoded f16 keys by mixed-precision FMAs (k_scale goes on the logit).
+    float q[kFp8 ? 1 : EPL];
+    uint32_t q2[kFp8 ? EPL / 2 : 1];
+    {
+        float qf[EPL];
 #pragma unroll
-    for (int c = 0; c < EPL / 8; ++c) unpack16<false>(q_raw[c], q + 8 * c);  // fp16 query
+        for (int c = 0; c < EPL / 8; ++c) unpack16<false>(q_raw[c], qf + 8 * c);
+        if constexpr (kFp8) {
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) q[e] *= p.qk_scale_log2;
+            for (int e = 0; e < EPL / 2; ++e) {
+                const __half2 h = __floats2half2_rn(qf[2 * e] * p.qk_scale_log2, qf[2 * e + 1] * p.qk_scale_log2);
+                q2[e] = *reinterpret_cast<const uint32_t *>(&h);
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) q[e] = qf[e] * p.qk_scale_log2;
+        }
+    }
 
     float m = -INFINITY, l = 0.f;
     float acc[EPL];
@@ -434,15 +450,22 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
             uint4 raw;
             if (t == t_new) raw = k_new;
             else raw = *reinterpret_cast<const uint4 *>(ktile + t * row_stride + head_off);
-            float k[EPL];
-            unpack16<kFp8>(raw, k);
             float d = 0.f;
+            if constexpr (kFp8) {
+                const uint16_t *c = reinterpret_cast<const uint16_t *>(&raw);
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) d = fmaf(q[e], k[e], d);
+                for (int e = 0; e < EPL / 2; ++e) d = fma2_f16_f32(q2[e], e4m3x2_to_f16x2_bits(c[e]), d);
+            } else {
+                float k[EPL];
+                unpack16<false>(raw, k);
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) d = fmaf(q[e], k[e], d);
+            }
             part_dot[j] = d;
         }
         const int my_t = grp * TPG + sub / DUP;
         float z = butterfly_reduce<TPG, LPR>(part_dot, lane);
+        if constexpr (kFp8) z *= p.logit_k_scale;
         z = (my_t < valid) ? z : -INFINITY;
 
         // ---- online softmax (base 2)
@@ -463,10 +486,20 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 uint4 raw;
                 if (t == t_new) raw = v_new;
                 else raw = *reinterpret_cast<const uint4 *>(vtile + t * row_stride + head_off);
-                float v[EPL];
-                unpack16<kFp8>(raw, v);
+                if constexpr (kFp8) {
+                    // weight rounded to f16 (relative error <= 2^-11), exact products
+                    const __half ph = __float2half_rn(pj);
+                    const uint16_t pb = *reinterpret_cast<const uint16_t *>(&ph);
+                    const uint16_t *c = reinterpret_cast<const uint16_t *>(&raw);
 #pragma unroll
-                for (int e = 0; e < EPL; ++e) acc[e] = fmaf(pj, v[e], acc[e]);
+                    for (int e = 0; e < EPL / 2; ++e)
+                        fma_pair_f16_f32(pb, e4m3x2_to_f16x2_bits(c[e]), acc[2 * e], acc[2 * e + 1]);
+                } else {
+                    float v[EPL];
+                    unpack16<false>(raw, v);
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) acc[e] = fmaf(pj, v[e], acc[e]);
+                }
             }
         }
         __syncwarp();

@@ -326,6 +326,8 @@ def to_device(w: Workload, device, encode=None) -> DeviceWorkload:
         vc = torch.empty(pv.shape, dtype=torch.uint8, device=device)
         encode(kc, vc, pk, pv, w.k_scale, w.v_scale)
         del pk, pv
+        torch.cuda.synchronize(device)
+        torch.cuda.empty_cache()    # release the fp16 source pools
     else:
         kc, vc = pk, pv
     S, H, D = w.query.shape
