@@ -452,9 +452,15 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
             else raw = *reinterpret_cast<const uint4 *>(ktile + t * row_stride + head_off);
             float d = 0.f;
             if constexpr (kFp8) {
+                // packed f16x2 products of the f16 query and the decoded keys,
+                // summed in f16x2 over this lane's 16 elements, then in fp32
                 const uint16_t *c = reinterpret_cast<const uint16_t *>(&raw);
+                __half2 s2 = __float2half2_rn(0.f);
 #pragma unroll
-                for (int e = 0; e < EPL / 2; ++e) d = fma2_f16_f32(q2[e], e4m3x2_to_f16x2_bits(c[e]), d);
+                for (int e = 0; e < EPL / 2; ++e)
+                    s2 = __hfma2(*reinterpret_cast<const __half2 *>(&q2[e]), e4m3x2_to_half2(c[e]), s2);
+                const float2 sf = __half22float2(s2);
+                d = sf.x + sf.y;
             } else {
                 float k[EPL];
                 unpack16<false>(raw, k);
@@ -477,7 +483,13 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
         for (int e = 0; e < EPL; ++e) acc[e] *= alpha;
         m = m_new;
 
-        // ---- P.V for this lane group's tokens
+        // ---- P.V for this lane group's tokens (E4M3: the block's tokens are
+        //      accumulated in f16x2, then added to the fp32 accumulators)
+        __half2 pv2[kFp8 ? EPL / 2 : 1];
+        if constexpr (kFp8) {
+#pragma unroll
+            for (int e = 0; e < EPL / 2; ++e) pv2[e] = __float2half2_rn(0.f);
+        }
 #pragma unroll
         for (int j = 0; j < TPG; ++j) {
             const int t = grp * TPG + j;
@@ -487,19 +499,24 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 if (t == t_new) raw = v_new;
                 else raw = *reinterpret_cast<const uint4 *>(vtile + t * row_stride + head_off);
                 if constexpr (kFp8) {
-                    // weight rounded to f16 (relative error <= 2^-11), exact products
-                    const __half ph = __float2half_rn(pj);
-                    const uint16_t pb = *reinterpret_cast<const uint16_t *>(&ph);
+                    const __half2 p2 = __float2half2_rn(pj);  // weight <= 1 in f16
                     const uint16_t *c = reinterpret_cast<const uint16_t *>(&raw);
 #pragma unroll
-                    for (int e = 0; e < EPL / 2; ++e)
-                        fma_pair_f16_f32(pb, e4m3x2_to_f16x2_bits(c[e]), acc[2 * e], acc[2 * e + 1]);
+                    for (int e = 0; e < EPL / 2; ++e) pv2[e] = __hfma2(p2, e4m3x2_to_half2(c[e]), pv2[e]);
                 } else {
                     float v[EPL];
                     unpack16<false>(raw, v);
 #pragma unroll
                     for (int e = 0; e < EPL; ++e) acc[e] = fmaf(pj, v[e], acc[e]);
                 }
+            }
+        }
+        if constexpr (kFp8) {
+#pragma unroll
+            for (int e = 0; e < EPL / 2; ++e) {
+                const float2 f = __half22float2(pv2[e]);
+                acc[2 * e] += f.x;
+                acc[2 * e + 1] += f.y;
             }
         }
         __syncwarp();

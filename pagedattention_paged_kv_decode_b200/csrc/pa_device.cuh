@@ -140,29 +140,6 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-// acc + lo(a)*lo(b) + hi(a)*hi(b) for f16x2 operands: each product of two
-// halves is formed exactly and added in fp32 (mixed-precision FMA).
-__device__ __forceinline__ float fma2_f16_f32(uint32_t a2, uint32_t b2, float acc) {
-    asm("{\n\t.reg .f16 al, ah, bl, bh;\n\t"
-        "mov.b32 {al, ah}, %1;\n\t"
-        "mov.b32 {bl, bh}, %2;\n\t"
-        "fma.rn.f32.f16 %0, al, bl, %0;\n\t"
-        "fma.rn.f32.f16 %0, ah, bh, %0;\n\t}"
-        : "+f"(acc)
-        : "r"(a2), "r"(b2));
-    return acc;
-}
-
-// a0 += x*lo(v2), a1 += x*hi(v2): f16 x f16 products, fp32 accumulators.
-__device__ __forceinline__ void fma_pair_f16_f32(uint16_t x, uint32_t v2, float &a0, float &a1) {
-    asm("{\n\t.reg .f16 vl, vh;\n\t"
-        "mov.b32 {vl, vh}, %3;\n\t"
-        "fma.rn.f32.f16 %0, %2, vl, %0;\n\t"
-        "fma.rn.f32.f16 %1, %2, vh, %1;\n\t}"
-        : "+f"(a0), "+f"(a1)
-        : "h"(x), "r"(v2));
-}
-
 // Two E4M3 codes (low byte = first element) -> two halves, exact.
 __device__ __forceinline__ __half2 e4m3x2_to_half2(uint16_t codes) {
     uint32_t h2;
@@ -170,11 +147,6 @@ __device__ __forceinline__ __half2 e4m3x2_to_half2(uint16_t codes) {
     return *reinterpret_cast<__half2 *>(&h2);
 }
 
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2_bits(uint16_t codes) {
-    uint32_t h2;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(codes));
-    return h2;
-}
 
 // Two floats -> two E4M3 codes, round to nearest even, saturate to +/-448
 // (NaN stays NaN). Low byte = lo.
