@@ -257,6 +257,9 @@ def run_ours(args, rank, world, local_rank):
             if i >= max(3, args.warmup):
                 e2e_ms.append(e2e_start.elapsed_time(e2e_end))
 
+        # ------------------------------------------------ swap to/from pinned host memory
+        swap = measure_swap(pk, dw, stream, torch)
+
     step_t, dec_t, e2e_t = slowest_rank([statistics.mean(step_ms), statistics.mean(dec_ms),
                                          statistics.mean(e2e_ms)], dist, dev)
     clocks = sampler.summary(t0, t1)
@@ -315,11 +318,42 @@ def run_ours(args, rank, world, local_rank):
                 "ms_per_step": round(e2e_t, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "path": "pinned host inputs -> device copies -> graph replay -> output to pinned host"},
         "gpu_launches": launches_per_step * args.steps,
+        "swap_blocks": swap,
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     print(json.dumps(line), flush=True)
+
+
+def measure_swap(pk, dw, stream, torch, n_blocks: int = 256, reps: int = 5):
+    """Block swap between the device pool and a pinned host pool (the pages'
+    --swap-space), outside the timed decode steps: GB/s of K+V moved out
+    (device -> host) and in (host -> device), n_blocks blocks per call."""
+    kc, vc = dw.key_cache, dw.value_cache
+    n = min(n_blocks, kc.shape[0])
+    hk = torch.empty((n,) + tuple(kc.shape[1:]), dtype=kc.dtype).pin_memory()
+    hv = torch.empty_like(hk).pin_memory()
+    pairs_out = torch.stack([torch.arange(n), torch.arange(n)], 1).to(torch.int32).to(kc.device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    res = {}
+    for name, call in (("out", lambda: pk.swap_blocks(hk, hv, kc, vc, pairs_out)),
+                       ("in", lambda: pk.swap_blocks(kc, vc, hk, hv, pairs_out))):
+        call()
+        ts = []
+        for _ in range(reps):
+            e0.record()
+            call()
+            e1.record()
+            stream.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        nbytes = 2 * n * kc[0].numel() * kc.element_size()
+        res[f"{name}_gbs"] = round(nbytes / (statistics.mean(ts) * 1e-3) / 1e9, 2)
+    assert pk.check_status(stream) == 0
+    res.update(blocks=n, bytes_per_call=2 * n * kc[0].numel() * kc.element_size(),
+               host="pinned host pool read/written by the swap kernel over the host link")
+    return res
 
 
 # ------------------------------------------------------------- CPU oracle

@@ -144,6 +144,22 @@ int pa_kv_cache_write(const void *key, const void *value, int64_t key_stride,
 int pa_copy_blocks(void *key_cache, void *value_cache, pa_cache_desc cache,
                    const int32_t *src_dst_pairs, int n_pairs, void *stream);
 
+/* ---------------------------------------------------------------- swap
+ * Block swap between two pools of the same block shape ([P1] §4.1 and
+ * [P2] §5.2: --swap-space, KV blocks spilled to CPU memory and brought
+ * back): for each pair (src, dst) of src_dst_pairs (int32 [n_pairs][2],
+ * device memory), block dst of the destination caches becomes a copy of
+ * block src of the source caches (K and V). Either pool may be device memory
+ * or pinned host memory accessible from the device (cudaHostAlloc / torch
+ * pin_memory under unified addressing); the kernel reaches host memory over
+ * the host link. cache gives the block shape and dtype (its num_blocks is
+ * not used); src_num_blocks and dst_num_blocks bound the indices (outside:
+ * PA_DEV_BAD_PAIR, pair skipped). Pairs run concurrently; repeated dst
+ * blocks are undefined. */
+int pa_swap_blocks(void *dst_key_cache, void *dst_value_cache, int dst_num_blocks,
+                   const void *src_key_cache, const void *src_value_cache, int src_num_blocks,
+                   pa_cache_desc cache, const int32_t *src_dst_pairs, int n_pairs, void *stream);
+
 /* ---------------------------------------------------------------- a4..a9
  * Decode attention of one query token per sequence over its cached K/V,
  * read through its block table ([P1] §2.2; [P2] §2.1). For each sequence s

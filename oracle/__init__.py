@@ -59,6 +59,8 @@ def _load():
         _lib.oracle_kv_cache_write.argtypes = [P, P, I64, I64, P, P, I, I, I, I, I, P, I, F, F]
         _lib.oracle_copy_blocks.restype = I
         _lib.oracle_copy_blocks.argtypes = [P, P, I64, I, P, I]
+        _lib.oracle_swap_blocks.restype = I
+        _lib.oracle_swap_blocks.argtypes = [P, P, I, P, P, I, I64, P, I]
         _lib.oracle_paged_attention.restype = I
         _lib.oracle_paged_attention.argtypes = [P, P, P, P, I, I, I, I, I, P, I, P, I, F, F, F, P, I]
         _lib.oracle_attention_partials.restype = I
@@ -153,6 +155,16 @@ def copy_blocks(key_cache: np.ndarray, value_cache: np.ndarray, src_dst_pairs: n
     block_bytes = key_cache[0].nbytes
     _check(_load().oracle_copy_blocks(_ptr(key_cache), _ptr(value_cache), block_bytes, nb,
                                       _ptr(pairs), pairs.shape[0]), "copy_blocks")
+
+
+def swap_blocks(dst_key: np.ndarray, dst_value: np.ndarray, src_key: np.ndarray,
+                src_value: np.ndarray, src_dst_pairs: np.ndarray) -> None:
+    """In place on dst_key/dst_value ([NB', B, H, D]); blocks copied from the source pools."""
+    assert dst_key.shape[1:] == src_key.shape[1:] and dst_key.dtype == src_key.dtype
+    pairs = np.ascontiguousarray(src_dst_pairs, dtype=np.int32).reshape(-1, 2)
+    _check(_load().oracle_swap_blocks(_ptr(dst_key), _ptr(dst_value), dst_key.shape[0],
+                                      _ptr(src_key), _ptr(src_value), src_key.shape[0],
+                                      src_key[0].nbytes, _ptr(pairs), pairs.shape[0]), "swap_blocks")
 
 
 def paged_attention(query: np.ndarray, key_cache: np.ndarray, value_cache: np.ndarray,

@@ -211,6 +211,27 @@ int oracle_copy_blocks(void *key_cache, void *value_cache, int64_t block_bytes,
     return 0;
 }
 
+/* Swap ([P1] §4.1 and [P2] §5.2, --swap-space: KV blocks moved to CPU
+ * memory and back): for each (src, dst) pair in order, block dst of the
+ * destination pools becomes a copy of block src of the source pools.
+ * Returns 0, or -1 on an index outside its pool (nothing after it is copied). */
+int oracle_swap_blocks(void *dst_key, void *dst_value, int dst_num_blocks,
+                       const void *src_key, const void *src_value, int src_num_blocks,
+                       int64_t block_bytes, const int32_t *src_dst_pairs, int n_pairs)
+{
+    for (int i = 0; i < n_pairs; ++i) {
+        int32_t src = src_dst_pairs[2 * i];
+        int32_t dst = src_dst_pairs[2 * i + 1];
+        if (src < 0 || src >= src_num_blocks || dst < 0 || dst >= dst_num_blocks)
+            return -1;
+        memcpy((char *)dst_key + dst * block_bytes, (const char *)src_key + src * block_bytes,
+               (size_t)block_bytes);
+        memcpy((char *)dst_value + dst * block_bytes, (const char *)src_value + src * block_bytes,
+               (size_t)block_bytes);
+    }
+    return 0;
+}
+
 /* ----------------------------------------------------- decode attention */
 
 static double cache_value(const void *cache, int kv_dtype, int64_t idx, double scale)

@@ -18,5 +18,6 @@ from .ops import (  # noqa: F401
     paged_attention_decode,
     paged_attention_decode_append,
     slot_mapping,
+    swap_blocks,
     version,
 )

@@ -55,6 +55,7 @@ SIGNATURES = {
     "pa_slot_mapping": (_I, [_P, _P, _I, _P, _I, CacheDesc, _P]),
     "pa_kv_cache_write": (_I, [_P, _P, _I64, _I64, _P, _P, CacheDesc, _P, _I, _F, _F, _P]),
     "pa_copy_blocks": (_I, [_P, _P, CacheDesc, _P, _I, _P]),
+    "pa_swap_blocks": (_I, [_P, _P, _I, _P, _P, _I, CacheDesc, _P, _I, _P]),
     "pa_paged_attention_decode": (_I, [_P, _P, _P, _P, CacheDesc, _P, _I, _P, _I, _I, _F, _F, _F, _P]),
     "pa_decode_choose_config": (_I, [CacheDesc, _I, _I, ctypes.POINTER(DecodeConfig)]),
     "pa_decode_workspace_size": (ctypes.c_size_t, [CacheDesc, _I, _I, ctypes.POINTER(DecodeConfig)]),

@@ -516,6 +516,36 @@ int pa_copy_blocks(void *key_cache, void *value_cache, pa_cache_desc cache,
     return ok();
 }
 
+int pa_swap_blocks(void *dst_key_cache, void *dst_value_cache, int dst_num_blocks,
+                   const void *src_key_cache, const void *src_value_cache, int src_num_blocks,
+                   pa_cache_desc cache, const int32_t *src_dst_pairs, int n_pairs, void *stream) {
+    pa_cache_desc c = cache;
+    c.num_blocks = std::max(1, std::max(dst_num_blocks, src_num_blocks));
+    int rc = check_cache(c);
+    if (rc) return rc;
+    if (dst_num_blocks < 1 || src_num_blocks < 1)
+        return fail(PA_ERR_INVALID, "dst_num_blocks (%d) and src_num_blocks (%d) must be >= 1",
+                    dst_num_blocks, src_num_blocks);
+    if (n_pairs < 0) return fail(PA_ERR_INVALID, "n_pairs %d < 0", n_pairs);
+    if (n_pairs == 0) return ok();
+    if (n_pairs > 65535) return fail(PA_ERR_INVALID, "n_pairs %d > 65535 per call", n_pairs);
+    if (!dst_key_cache || !dst_value_cache || !src_key_cache || !src_value_cache || !src_dst_pairs)
+        return fail(PA_ERR_INVALID, "null pointer argument");
+    if (!aligned16(dst_key_cache) || !aligned16(dst_value_cache) || !aligned16(src_key_cache) ||
+        !aligned16(src_value_cache))
+        return fail(PA_ERR_INVALID, "caches must be 16-byte aligned");
+    const int64_t block_vecs =
+        (int64_t)c.block_size * c.num_heads * c.head_size * elem_bytes(c) / 16;
+    const int64_t per_cta = (int64_t)pa::kCopyThreads * pa::kCopyVecs;
+    const dim3 grid((unsigned)((block_vecs + per_cta - 1) / per_cta), n_pairs, 2);
+    pa::swap_blocks_kernel<<<grid, pa::kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+        dst_key_cache, dst_value_cache, src_key_cache, src_value_cache, src_dst_pairs, block_vecs,
+        src_num_blocks, dst_num_blocks);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "swap_blocks_kernel launch");
+    return ok();
+}
+
 int pa_decode_choose_config(pa_cache_desc cache, int num_seqs, int max_context_len,
                             pa_decode_config *cfg) {
     int rc = check_cache(cache);

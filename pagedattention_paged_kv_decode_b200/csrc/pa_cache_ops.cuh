@@ -102,4 +102,38 @@ copy_blocks_kernel(void *__restrict__ key_cache, void *__restrict__ value_cache,
     }
 }
 
+// Swap (the pages' --swap-space: KV blocks spilled to and restored from CPU
+// memory): grid (chunks of a block, pairs, 2 caches). Block dst of the
+// destination pool becomes a copy of block src of the source pool; either
+// pool may be device memory or pinned host memory mapped into the device's
+// address space, which the loads or stores then reach over the host link.
+__global__ void __launch_bounds__(kCopyThreads)
+swap_blocks_kernel(void *__restrict__ dst_key, void *__restrict__ dst_value,
+                   const void *__restrict__ src_key, const void *__restrict__ src_value,
+                   const int32_t *__restrict__ pairs, int64_t block_vecs, int src_blocks,
+                   int dst_blocks) {
+    const int pr = blockIdx.y;
+    const int32_t src = pairs[2 * pr];
+    const int32_t dst = pairs[2 * pr + 1];
+    if (src < 0 || src >= src_blocks || dst < 0 || dst >= dst_blocks) {
+        if (blockIdx.x == 0 && blockIdx.z == 0 && threadIdx.x == 0) flag_error(PA_DEV_BAD_PAIR);
+        return;
+    }
+    const uint4 *from = static_cast<const uint4 *>(blockIdx.z == 0 ? src_key : src_value) +
+                        (size_t)src * block_vecs;
+    uint4 *to = static_cast<uint4 *>(blockIdx.z == 0 ? dst_key : dst_value) + (size_t)dst * block_vecs;
+    const int64_t v0 = (int64_t)blockIdx.x * kCopyThreads * kCopyVecs + threadIdx.x;
+    uint4 r[kCopyVecs];
+#pragma unroll
+    for (int k = 0; k < kCopyVecs; ++k) {
+        const int64_t v = v0 + (int64_t)k * kCopyThreads;
+        if (v < block_vecs) r[k] = from[v];
+    }
+#pragma unroll
+    for (int k = 0; k < kCopyVecs; ++k) {
+        const int64_t v = v0 + (int64_t)k * kCopyThreads;
+        if (v < block_vecs) to[v] = r[k];
+    }
+}
+
 }  // namespace pa

@@ -91,6 +91,30 @@ def copy_blocks(key_cache: torch.Tensor, value_cache: torch.Tensor, src_dst_pair
                                src_dst_pairs.data_ptr(), n, _stream(stream)))
 
 
+def swap_blocks(dst_key_cache: torch.Tensor, dst_value_cache: torch.Tensor,
+                src_key_cache: torch.Tensor, src_value_cache: torch.Tensor,
+                src_dst_pairs: torch.Tensor, stream=None) -> None:
+    """Copy whole blocks from the source pools into the destination pools.
+
+    One side may be a pinned CPU tensor (``pin_memory()``), which the kernel
+    reads or writes over the host link; ``src_dst_pairs`` is int32 [n, 2] on
+    the device."""
+    for a, b in ((dst_key_cache, dst_value_cache), (src_key_cache, src_value_cache)):
+        if a.shape != b.shape or a.dtype != b.dtype or not a.is_contiguous() or not b.is_contiguous():
+            raise ValueError("key/value pools of one side differ or are not contiguous")
+        if not a.is_cuda and not a.is_pinned():
+            raise ValueError("a CPU pool must be pinned (pin_memory())")
+    if dst_key_cache.shape[1:] != src_key_cache.shape[1:] or dst_key_cache.dtype != src_key_cache.dtype:
+        raise ValueError("source and destination block shapes differ")
+    _i32(src_dst_pairs, "src_dst_pairs")
+    n = src_dst_pairs.numel() // 2
+    check(lib().pa_swap_blocks(dst_key_cache.data_ptr(), dst_value_cache.data_ptr(),
+                               dst_key_cache.shape[0], src_key_cache.data_ptr(),
+                               src_value_cache.data_ptr(), src_key_cache.shape[0],
+                               cache_desc(src_key_cache), src_dst_pairs.data_ptr(), n,
+                               _stream(stream)))
+
+
 def _config(config) -> DecodeConfig | None:
     if config is None:
         return None

@@ -155,3 +155,37 @@ def test_fused_append_skips_bad_blocks_and_clamped_contexts(cuda_device):
     changed = (dw.key_cache != before).reshape(20 * 16, -1).any(dim=1).nonzero().flatten().tolist()
     assert changed == [int(ref[1])]      # only seq 1's new row was stored
     assert torch.isfinite(dw.out.float()).all()
+
+
+@pytest.mark.parametrize("kv", ["f16", "e4m3"])
+def test_swap_blocks_device_and_pinned_host(cuda_device, kv):
+    """Swap out to a pinned CPU pool and back in, against the oracle's copies."""
+    dt = torch.float16 if kv == "f16" else torch.uint8
+    rng = np.random.default_rng(9)
+    shape = (12, 16, 4, 128)
+    if kv == "f16":
+        hk = rng.standard_normal(shape).astype(np.float16)
+        hv = rng.standard_normal(shape).astype(np.float16)
+    else:
+        hk = rng.integers(0, 256, shape, dtype=np.uint8)
+        hv = rng.integers(0, 256, shape, dtype=np.uint8)
+    gk = torch.from_numpy(hk).to(cuda_device)
+    gv = torch.from_numpy(hv).to(cuda_device)
+    ck = torch.zeros((5,) + shape[1:], dtype=dt).pin_memory()
+    cv = torch.zeros((5,) + shape[1:], dtype=dt).pin_memory()
+    out_pairs = np.array([[3, 0], [11, 4], [7, 2]], np.int32)
+    pk.swap_blocks(ck, cv, gk, gv, torch.from_numpy(out_pairs).to(cuda_device))
+    assert pk.check_status() == 0
+    rk = np.zeros((5,) + shape[1:], hk.dtype)
+    rv = np.zeros_like(rk)
+    oracle.swap_blocks(rk, rv, hk, hv, out_pairs)
+    assert np.array_equal(ck.numpy().view(np.uint8), rk.view(np.uint8))
+    assert np.array_equal(cv.numpy().view(np.uint8), rv.view(np.uint8))
+    in_pairs = np.array([[0, 1], [4, 5], [2, 9]], np.int32)
+    pk.swap_blocks(gk, gv, ck, cv, torch.from_numpy(in_pairs).to(cuda_device))
+    bad = torch.tensor([[0, 12]], dtype=torch.int32, device=cuda_device)
+    pk.swap_blocks(gk, gv, ck, cv, bad)
+    assert pk.check_status() == capi.PA_DEV_BAD_PAIR
+    oracle.swap_blocks(hk, hv, rk, rv, in_pairs)
+    assert np.array_equal(gk.cpu().numpy().view(np.uint8), hk.view(np.uint8))
+    assert np.array_equal(gv.cpu().numpy().view(np.uint8), hv.view(np.uint8))

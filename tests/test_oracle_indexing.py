@@ -161,3 +161,22 @@ def test_named_workload_laws(cfg):
     live = np.zeros(pk.shape[:2], bool)
     live[w.live_blocks, w.live_offsets] = True
     assert (np.abs(pk[~live].astype(np.float32)) == 60000).all()
+
+
+def test_swap_blocks_between_pools():
+    rng = np.random.default_rng(8)
+    gk = rng.standard_normal((6, 4, 2, 8)).astype(np.float16)
+    gv = rng.standard_normal((6, 4, 2, 8)).astype(np.float16)
+    ck = np.zeros((3, 4, 2, 8), np.float16)
+    cv = np.zeros((3, 4, 2, 8), np.float16)
+    oracle.swap_blocks(ck, cv, gk, gv, np.array([[5, 0], [2, 2]], np.int32))   # out: device -> host pool
+    assert np.array_equal(ck[0], gk[5]) and np.array_equal(cv[2], gv[2]) and not ck[1].any()
+    g0 = gk.copy()
+    oracle.swap_blocks(gk, gv, ck, cv, np.array([[0, 1]], np.int32))           # in: host -> device pool
+    assert np.array_equal(gk[1], g0[5])
+    for b in (0, 2, 3, 4, 5):
+        assert np.array_equal(gk[b], g0[b])
+    with pytest.raises(ValueError):
+        oracle.swap_blocks(ck, cv, gk, gv, np.array([[6, 0]], np.int32))
+    with pytest.raises(ValueError):
+        oracle.swap_blocks(ck, cv, gk, gv, np.array([[0, 3]], np.int32))
