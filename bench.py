@@ -163,7 +163,7 @@ def run_ours(args, rank, world, local_rank):
     launches_per_step = ((3 if args.unfused else 1) + (1 if w.cow_pairs.size else 0)
                          + (1 if parts > 1 else 0))
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    flush_sink = torch.zeros((), dtype=torch.int32, device=dev)
+    flush_sink = torch.zeros((), dtype=torch.int64, device=dev)
 
     stream = torch.cuda.Stream(dev)
     ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
@@ -204,7 +204,7 @@ def run_ours(args, rank, world, local_rank):
             # the written lines (their write-back happens here, outside the timed
             # step) and leaves L2 holding clean lines of the flush buffer only.
             flush.fill_(1)
-            flush_sink.copy_(flush.sum(dtype=torch.int32))
+            flush_sink.copy_(flush.view(torch.int64).sum())
 
         def timed_step():
             evict_l2()
