@@ -158,10 +158,13 @@ def run_ours(args, rank, world, local_rank):
     if args.launch:
         launch = dict(zip(("partition_size", "heads_per_cta", "warps_per_head", "stages"),
                           (int(x) for x in args.launch.split(","))))
+    shared = bool(w.shared_blocks) and not args.no_shared_prefix and not args.unfused
     cfg = pk.choose_config(dw.key_cache, S, bound, launch)
     parts = -(-bound // cfg["partition_size"])
     launches_per_step = ((3 if args.unfused else 1) + (1 if w.cow_pairs.size else 0)
                          + (1 if parts > 1 else 0))
+    if shared:   # prefix kernel + decode of the private parts + reduce
+        launches_per_step = 3 + (1 if w.cow_pairs.size else 0)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_sink = torch.zeros((), dtype=torch.int64, device=dev)
 
@@ -180,6 +183,14 @@ def run_ours(args, rank, world, local_rank):
             pk.paged_attention_decode(dw.out, dw.query, dw.key_cache, dw.value_cache,
                                       dw.block_tables, dw.context_lens, w.scale, w.k_scale,
                                       w.v_scale, max_context_len=bound)
+        elif shared:
+            ev[1].record()
+            pk.paged_attention_decode_shared_prefix(dw.out, dw.query, dw.key_cache, dw.value_cache,
+                                                    dw.block_tables, dw.context_lens,
+                                                    w.shared_blocks, w.scale, w.k_scale, w.v_scale,
+                                                    new_key=dw.new_key, new_value=dw.new_value,
+                                                    max_context_len=bound, slot_mapping=dw.slots,
+                                                    config=launch)
         else:
             ev[1].record()
             pk.paged_attention_decode_append(dw.out, dw.query, dw.new_key, dw.new_value,
@@ -298,8 +309,11 @@ def run_ours(args, rank, world, local_rank):
                   "no step data and no dirty lines left in L2",
             "step": "CUDA graph: " + ("copy_blocks, " if w.cow_pairs.size else "")
                     + ("slot_mapping, kv_cache_write, paged_attention_decode" if args.unfused
+                       else ("paged_attention_decode_shared_prefix (prefix kernel over the "
+                             f"{w.shared_blocks} shared blocks + fused append/decode of the rest "
+                             "+ lse reduce)") if shared
                        else "paged_attention_decode_append (slot + K/V store + decode in one launch)")
-                    + (" (+lse reduce)" if parts > 1 else ""),
+                    + (" (+lse reduce)" if parts > 1 and not shared else ""),
         },
         "tokens_per_s": round(world * S / (step_t * 1e-3), 1),
         "hbm_pct_of_nominal_8tbs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
@@ -310,8 +324,9 @@ def run_ours(args, rank, world, local_rank):
             "bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} copy bandwidth",
             "traffic": recorded_traffic(w.name),
-            "kernel": "paged_decode_kernel" + ("" if args.unfused else " (fused append)")
-                      + (" + lse_reduce_kernel" if parts > 1 else ""),
+            "kernel": ("paged_prefix_kernel + paged_decode_kernel (fused append) + lse_reduce_kernel"
+                       if shared else "paged_decode_kernel" + ("" if args.unfused else " (fused append)")
+                       + (" + lse_reduce_kernel" if parts > 1 else "")),
             "algorithmic_bytes_per_launch": dec_bytes,
         },
         "e2e": {"value": round(aggregate_gbs(world, kv, e2e_t), 2), "unit": "GB/s",
@@ -440,6 +455,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-shared-prefix", action="store_true",
+                    help="decode a shared-prefix workload without the prefix kernel")
     ap.add_argument("--unfused", action="store_true",
                     help="slot mapping, cache write and decode as three launches")
     ap.add_argument("--launch", default="",

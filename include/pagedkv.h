@@ -61,6 +61,7 @@ extern "C" {
 #define PA_DEV_CTX_OVER_BOUND 8u  /* context_len > max_context_len given to the call: clamped */
 #define PA_DEV_BAD_PAIR 16u       /* copy pair index outside [0, num_blocks): pair skipped */
 #define PA_DEV_WAIT_TIMEOUT 32u   /* an on-chip pipeline wait ran out (never expected) */
+#define PA_DEV_PREFIX 64u         /* shared-prefix contract broken (see ..._shared_prefix) */
 
 /* KV cache element type: fp16, or OCP FP8 E4M3 ("fn" variant: no infinities,
  * max 448) with one fp32 scale per cache tensor ([P1] §3.3, [P3] §4). */
@@ -238,6 +239,37 @@ int pa_paged_attention_decode_append(void *out, const void *query, const void *n
                                      float k_scale, float v_scale, int32_t *slot_mapping_out,
                                      const pa_decode_config *cfg, void *workspace,
                                      size_t workspace_bytes, void *stream);
+
+/* Decode (optionally with the fused append) for a batch whose sequences all
+ * start with the same shared_prefix_blocks physical blocks ([P2] §2.2:
+ * requests with the same prompt map its logical blocks to the same physical
+ * blocks). Contract: for every row s, block_tables[s][0 .. n-1] equals
+ * block_tables[0][0 .. n-1] (n = shared_prefix_blocks, whole blocks); a row
+ * that differs sets PA_DEV_PREFIX. Each shared tile is read once per head
+ * and applied to up to 16 sequences' queries; the private rest of every
+ * context is decoded as in pa_paged_attention_decode; a log-sum-exp
+ * reduction merges both (three launches). Results equal
+ * pa_paged_attention_decode (or _append when new_key is given) on the same
+ * tables. With new_key/new_value (both or neither), each sequence's new
+ * token must lie after the prefix (L > n * block_size), else it is not
+ * stored, its slot is -1 and PA_DEV_PREFIX is set. cfg shapes the decode of
+ * the private part (NULL = library choice); workspace NULL = the library's
+ * own, else at least pa_shared_prefix_workspace_size bytes, 256-aligned. */
+int pa_paged_attention_decode_shared_prefix(void *out, const void *query, const void *new_key,
+                                            const void *new_value, int64_t key_stride,
+                                            int64_t value_stride, void *key_cache,
+                                            void *value_cache, pa_cache_desc cache,
+                                            const int32_t *block_tables, int max_blocks_per_seq,
+                                            const int32_t *context_lens, int num_seqs,
+                                            int max_context_len, int shared_prefix_blocks,
+                                            float scale, float k_scale, float v_scale,
+                                            int32_t *slot_mapping_out, const pa_decode_config *cfg,
+                                            void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace bytes of a pa_paged_attention_decode_shared_prefix call (0 on
+ * invalid arguments). */
+size_t pa_shared_prefix_workspace_size(pa_cache_desc cache, int num_seqs, int max_context_len,
+                                       int shared_prefix_blocks, const pa_decode_config *cfg);
 
 /* pa_paged_attention_decode for callers that cannot allocate device memory.
  * The paper has no counterpart to this call: it exists for callers such as

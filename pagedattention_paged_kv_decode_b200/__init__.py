@@ -17,6 +17,7 @@ from .ops import (  # noqa: F401
     load_cache,
     paged_attention_decode,
     paged_attention_decode_append,
+    paged_attention_decode_shared_prefix,
     slot_mapping,
     swap_blocks,
     version,

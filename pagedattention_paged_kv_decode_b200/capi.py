@@ -23,6 +23,7 @@ PA_DEV_CTX_OVER_TABLE = 4
 PA_DEV_CTX_OVER_BOUND = 8
 PA_DEV_BAD_PAIR = 16
 PA_DEV_WAIT_TIMEOUT = 32
+PA_DEV_PREFIX = 64
 
 PA_F16 = 0
 PA_E4M3 = 1
@@ -64,6 +65,10 @@ SIGNATURES = {
     "pa_paged_attention_decode_append": (_I, [_P, _P, _P, _P, _I64, _I64, _P, _P, CacheDesc, _P, _I, _P,
                                               _I, _I, _F, _F, _F, _P, ctypes.POINTER(DecodeConfig),
                                               _P, ctypes.c_size_t, _P]),
+    "pa_paged_attention_decode_shared_prefix": (_I, [_P, _P, _P, _P, _I64, _I64, _P, _P, CacheDesc, _P, _I,
+                                                     _P, _I, _I, _I, _F, _F, _F, _P,
+                                                     ctypes.POINTER(DecodeConfig), _P, ctypes.c_size_t, _P]),
+    "pa_shared_prefix_workspace_size": (ctypes.c_size_t, [CacheDesc, _I, _I, _I, ctypes.POINTER(DecodeConfig)]),
     "pa_paged_attention_decode_noalloc": (_I, [_P, _P, _P, _P, CacheDesc, _P, _I, _P, _I, _I, _F, _F,
                                                _F, _P]),
 }

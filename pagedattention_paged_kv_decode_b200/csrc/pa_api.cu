@@ -245,6 +245,15 @@ DecodeKernel pick_decode(int D, int B, bool fp8) {
     return nullptr;
 }
 
+DecodeKernel pick_prefix(int D, int B, bool fp8) {
+#define PA_PICK(d, b, f) \
+    if (D == d && B == b && fp8 == f) return pa::paged_prefix_kernel<d, b, f>;
+    PA_PICK(64, 16, false) PA_PICK(64, 32, false) PA_PICK(128, 16, false) PA_PICK(128, 32, false)
+    PA_PICK(64, 16, true) PA_PICK(64, 32, true) PA_PICK(128, 16, true) PA_PICK(128, 32, true)
+#undef PA_PICK
+    return nullptr;
+}
+
 ReduceKernel pick_reduce(int D) {
     return D == 64 ? pa::lse_reduce_kernel<64> : pa::lse_reduce_kernel<128>;
 }
@@ -330,15 +339,29 @@ struct AppendArgs {
     int32_t *slot_out;
 };
 
+// Launch shape of the shared-prefix kernel (see pa_paged_attention_decode_shared_prefix).
+struct PrefixPlan {
+    int prefix_tokens;  // shared tokens (whole blocks)
+    int partition;      // tokens per prefix partition
+    int parts;          // prefix partitions
+    int heads;          // heads per CTA
+    int queries;        // sequences per CTA
+    int stages;
+};
+
 int launch_decode(void *out, const void *query, const void *kc, const void *vc,
                   const pa_cache_desc &c, const int32_t *bt, int maxblk, const int32_t *ctx, int S,
                   int max_ctx, float scale, float k_scale, float v_scale,
                   const pa_decode_config &cfg, void *ws, cudaStream_t st, int device,
-                  const AppendArgs *app = nullptr) {
+                  const AppendArgs *app = nullptr, const PrefixPlan *pre = nullptr) {
     const int B = c.block_size, D = c.head_size;
     const bool fp8 = c.dtype == PA_E4M3;
     max_ctx = std::min<int64_t>(max_ctx, (int64_t)maxblk * B);
-    const int parts = max_parts_of(max_ctx, cfg.partition_size);
+    const int prefix_tokens = pre ? pre->prefix_tokens : 0;
+    // suffix partitions (all partitions without a shared prefix); at least one
+    // unit per sequence so that every sequence's slot and flags are handled
+    const int parts = max_parts_of(std::max(max_ctx - prefix_tokens, 0), cfg.partition_size);
+    const int ws_parts = parts + (pre ? pre->parts : 0);
     const int G = cfg.heads_per_cta, W = cfg.warps_per_head;
 
     CUtensorMap mk, mv;
@@ -352,9 +375,16 @@ int launch_decode(void *out, const void *query, const void *kc, const void *vc,
     p.query = static_cast<const __half *>(query);
     p.block_tables = bt;
     p.context_lens = ctx;
-    if (parts > 1) {
+    if (ws_parts > 1 || pre) {
         p.ws_lse = static_cast<float *>(ws);
-        p.ws_o = reinterpret_cast<float *>(static_cast<char *>(ws) + ws_lse_bytes(c, S, parts));
+        p.ws_o = reinterpret_cast<float *>(static_cast<char *>(ws) + ws_lse_bytes(c, S, ws_parts));
+    }
+    p.ws_parts = ws_parts;
+    if (pre) {
+        p.prefix_tokens = pre->prefix_tokens;
+        p.prefix_parts = pre->parts;
+        p.prefix_partition = pre->partition;
+        p.queries_per_cta = pre->queries;
     }
     p.num_seqs = S;
     p.num_heads = c.num_heads;
@@ -388,6 +418,26 @@ int launch_decode(void *out, const void *query, const void *kc, const void *vc,
     if (!kern) return fail(PA_ERR_INVALID, "no kernel for head_size %d block_size %d", D, B);
     rc = ensure_smem_attr(reinterpret_cast<const void *>(kern), device);
     if (rc) return rc;
+    cudaError_t e;
+    if (pre) {
+        DecodeKernel pkern = pick_prefix(D, B, fp8);
+        rc = ensure_smem_attr(reinterpret_cast<const void *>(pkern), device);
+        if (rc) return rc;
+        CUtensorMap pk_, pv_;
+        rc = cache_tensor_map(kc, c, pre->heads, &pk_);
+        if (rc) return rc;
+        rc = cache_tensor_map(vc, c, pre->heads, &pv_);
+        if (rc) return rc;
+        pa::DecodeParams pp = p;
+        pp.heads_per_cta = pre->heads;
+        pp.stages = pre->stages;
+        const pa::SmemLayout play(B, pre->heads, D, elem_bytes(c), 1, pre->stages, 1);
+        const int64_t n_qb = (S + pre->queries - 1) / pre->queries;
+        const int64_t n = (int64_t)(c.num_heads / pre->heads) * pre->parts * n_qb;
+        pkern<<<dim3((unsigned)n), dim3(32 * (pre->heads * pre->queries + 1)), play.total, st>>>(pk_, pv_, pp);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "paged_prefix_kernel launch");
+    }
     const int C = cfg.units_per_cta;
     const pa::SmemLayout lay(B, G, D, elem_bytes(c), W, cfg.stages, C);
     // Every unit u is served by CTA u % grid, slot u / grid: grid * C >= units.
@@ -398,9 +448,9 @@ int launch_decode(void *out, const void *query, const void *kc, const void *vc,
     const dim3 grid((unsigned)n_ctas);
     const dim3 block(32 * (C * G * W + 1));
     kern<<<grid, block, lay.total, st>>>(mk, mv, p);
-    cudaError_t e = cudaGetLastError();
+    e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "paged_decode_kernel launch");
-    if (parts > 1) {
+    if (ws_parts > 1 || pre) {
         pick_reduce(D)<<<dim3((c.num_heads + 3) / 4, S), 128, 0, st>>>(p);
         e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "lse_reduce_kernel launch");
@@ -671,6 +721,101 @@ extern "C" int pa_paged_attention_decode_append(
     return launch_decode(out, query, key_cache, value_cache, cache, block_tables,
                          max_blocks_per_seq, context_lens, num_seqs, bound, scale, k_scale,
                          v_scale, r, ws, st, dev, &app);
+}
+
+namespace {
+
+// Shared-prefix plan and the suffix config; returns the workspace bytes.
+int plan_shared_prefix(const pa_cache_desc &c, int S, int bound, int prefix_blocks,
+                       const pa_decode_config *cfg, pa_decode_config *suffix, PrefixPlan *pre,
+                       size_t *ws) {
+    const int B = c.block_size;
+    if (prefix_blocks < 1) return fail(PA_ERR_INVALID, "shared_prefix_blocks %d < 1", prefix_blocks);
+    pre->prefix_tokens = prefix_blocks * B;
+    if (pre->prefix_tokens > bound)
+        return fail(PA_ERR_INVALID, "shared prefix (%d tokens) beyond the context bound %d",
+                    pre->prefix_tokens, bound);
+    pre->partition = std::max(B, 512 / B * B);
+    pre->parts = (pre->prefix_tokens + pre->partition - 1) / pre->partition;
+    pre->heads = 1;
+    pre->queries = std::min(S, pa::kMaxConsumerWarps);
+    const size_t sb = pa::SmemLayout(B, 1, c.head_size, elem_bytes(c), 1, 1, 1).stage_bytes;
+    pre->stages = (int)std::max<size_t>(2, std::min<size_t>(8, (96 * 1024) / sb));
+    pa_decode_config r = cfg ? *cfg : pa_decode_config{0, 0, 0, 0, 0};
+    const int suffix_bound = std::max(bound - pre->prefix_tokens, B);
+    int rc = fill_config(c, S, suffix_bound, &r);
+    if (rc) return rc;
+    *suffix = r;
+    const int ws_parts = max_parts_of(suffix_bound, r.partition_size) + pre->parts;
+    *ws = ws_lse_bytes(c, S, ws_parts) + (size_t)S * c.num_heads * ws_parts * c.head_size * sizeof(float);
+    return PA_OK;
+}
+
+}  // namespace
+
+extern "C" size_t pa_shared_prefix_workspace_size(pa_cache_desc cache, int num_seqs,
+                                                  int max_context_len, int shared_prefix_blocks,
+                                                  const pa_decode_config *cfg) {
+    if (check_cache(cache) || num_seqs <= 0 || max_context_len < 0) return 0;
+    pa_decode_config r;
+    PrefixPlan pre;
+    size_t ws = 0;
+    if (plan_shared_prefix(cache, num_seqs, max_context_len, shared_prefix_blocks, cfg, &r, &pre, &ws))
+        return 0;
+    return ws;
+}
+
+extern "C" int pa_paged_attention_decode_shared_prefix(
+    void *out, const void *query, const void *new_key, const void *new_value, int64_t key_stride,
+    int64_t value_stride, void *key_cache, void *value_cache, pa_cache_desc cache,
+    const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+    int num_seqs, int max_context_len, int shared_prefix_blocks, float scale, float k_scale,
+    float v_scale, int32_t *slot_mapping_out, const pa_decode_config *cfg, void *workspace,
+    size_t workspace_bytes, void *stream) {
+    int rc = check_decode_args(out, query, key_cache, value_cache, cache, block_tables,
+                               max_blocks_per_seq, context_lens, num_seqs, max_context_len, scale,
+                               k_scale, v_scale);
+    if (rc) return rc;
+    if (num_seqs == 0) return ok();
+    if ((new_key == nullptr) != (new_value == nullptr))
+        return fail(PA_ERR_INVALID, "new_key and new_value must both be given or both be NULL");
+    if (new_key) {
+        if (!aligned16(new_key) || !aligned16(new_value))
+            return fail(PA_ERR_INVALID, "new_key and new_value must be 16-byte aligned");
+        const int row = cache.num_heads * cache.head_size;
+        if (key_stride < row || value_stride < row || key_stride % 8 || value_stride % 8)
+            return fail(PA_ERR_INVALID,
+                        "key_stride/value_stride (%lld/%lld) must be >= %d and multiples of 8",
+                        (long long)key_stride, (long long)value_stride, row);
+    }
+    if (shared_prefix_blocks > max_blocks_per_seq)
+        return fail(PA_ERR_INVALID, "shared_prefix_blocks %d > max_blocks_per_seq %d",
+                    shared_prefix_blocks, max_blocks_per_seq);
+    const int bound =
+        (int)std::min<int64_t>(max_context_len, (int64_t)max_blocks_per_seq * cache.block_size);
+    pa_decode_config r;
+    PrefixPlan pre;
+    size_t need = 0;
+    rc = plan_shared_prefix(cache, num_seqs, bound, shared_prefix_blocks, cfg, &r, &pre, &need);
+    if (rc) return rc;
+    int dev = 0;
+    rc = current_device(&dev);
+    if (rc) return rc;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    void *ws = workspace;
+    if (workspace) {
+        if (workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+            return fail(PA_ERR_WORKSPACE,
+                        "workspace of %zu bytes at %p: need %zu bytes, 256-byte aligned",
+                        workspace_bytes, workspace, need);
+    } else {
+        rc = internal_workspace(need, st, dev, &ws);
+        if (rc) return rc;
+    }
+    const AppendArgs app{new_key, new_value, key_stride, value_stride, slot_mapping_out};
+    return launch_decode(out, query, key_cache, value_cache, cache, block_tables,
+                         max_blocks_per_seq, context_lens, num_seqs, bound, scale, k_scale,
+                         v_scale, r, ws, st, dev, new_key ? &app : nullptr, &pre);
 }
 
 // ---------------------------------------------------------------------------

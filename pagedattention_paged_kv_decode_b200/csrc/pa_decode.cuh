@@ -54,6 +54,16 @@ struct DecodeParams {
     int stages;
     int units_per_cta;           // C work units (slots) per CTA
     int64_t num_units;           // num_seqs * (num_heads / G) * max_parts
+    // Shared prefix (all 0 for a plain decode): the first prefix_tokens
+    // tokens of every sequence live in the same physical blocks (those of
+    // table row 0). The decode kernel then covers tokens prefix_tokens.. only
+    // and always writes partials, at index prefix_parts + part of each
+    // (sequence, head); the prefix kernel fills indices 0..prefix_parts-1.
+    int prefix_tokens;
+    int prefix_parts;
+    int prefix_partition;        // tokens per prefix partition (multiple of block_size)
+    int queries_per_cta;         // prefix kernel: sequences sharing one CTA's tiles
+    int ws_parts;                // partial slots per (sequence, head) in the workspace
     float qk_scale_log2;         // scale * log2(e)
     float logit_k_scale;         // k_scale, applied to each E4M3 logit (1 for fp16 caches)
     float out_scale;             // v_scale (1 for fp16 caches)
@@ -144,6 +154,142 @@ __device__ __forceinline__ void unpack16<true>(const uint4 &raw, float *f) {
     }
 }
 
+// Online-softmax attention state of one warp for one (query, head): the
+// per-tile arithmetic shared by the decode and the shared-prefix kernels.
+// Lane layout (Geometry): lane group `grp` takes TPG tokens of each tile,
+// lane `sub` of the group holds EPL elements of the query, K/V rows and
+// output accumulator.
+template <int D, int B, bool kFp8>
+struct HeadAttn {
+    using Geo = Geometry<D, B, kFp8>;
+    static constexpr int EPL = Geo::EPL, LPR = Geo::LPR, TPG = Geo::TPG, DUP = Geo::DUP;
+    // fp16 caches: query in fp32, pre-scaled by scale*log2(e). E4M3 caches:
+    // the pre-scaled query rounded to f16 pairs for packed f16x2 products
+    // with the decoded keys (k_scale goes on each logit).
+    float q[kFp8 ? 1 : EPL];
+    uint32_t q2[kFp8 ? EPL / 2 : 1];
+    float m, l;
+    float acc[EPL];
+
+    __device__ __forceinline__ void init(const uint4 (&q_raw)[EPL / 8], float qk_scale_log2) {
+        float qf[EPL];
+#pragma unroll
+        for (int c = 0; c < EPL / 8; ++c) unpack16<false>(q_raw[c], qf + 8 * c);
+        if constexpr (kFp8) {
+#pragma unroll
+            for (int e = 0; e < EPL / 2; ++e) {
+                const __half2 h = __floats2half2_rn(qf[2 * e] * qk_scale_log2, qf[2 * e + 1] * qk_scale_log2);
+                q2[e] = *reinterpret_cast<const uint32_t *>(&h);
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) q[e] = qf[e] * qk_scale_log2;
+        }
+        m = -INFINITY;
+        l = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
+    }
+
+    // One tile: rows t < valid of the tile (row t at `ktile + t*row_stride +
+    // head_off`, V likewise) take part; row t_new (if >= 0) is taken from
+    // k_new/v_new instead (the appended token, already in cache format).
+    __device__ __forceinline__ void consume(const unsigned char *ktile, const unsigned char *vtile,
+                                            size_t row_stride, size_t head_off, int valid, int t_new,
+                                            const uint4 &k_new, const uint4 &v_new,
+                                            float logit_k_scale, int lane) {
+        const int grp = lane / LPR, sub = lane % LPR;
+        // ---- logits of this lane group's TPG tokens
+        float part_dot[TPG];
+#pragma unroll
+        for (int j = 0; j < TPG; ++j) {
+            const int t = grp * TPG + j;
+            uint4 raw;
+            if (t == t_new) raw = k_new;
+            else raw = *reinterpret_cast<const uint4 *>(ktile + t * row_stride + head_off);
+            float d = 0.f;
+            if constexpr (kFp8) {
+                // packed f16x2 products of the f16 query and the decoded keys,
+                // summed in f16x2 over this lane's 16 elements, then in fp32
+                const uint16_t *c = reinterpret_cast<const uint16_t *>(&raw);
+                __half2 s2 = __float2half2_rn(0.f);
+#pragma unroll
+                for (int e = 0; e < EPL / 2; ++e)
+                    s2 = __hfma2(*reinterpret_cast<const __half2 *>(&q2[e]), e4m3x2_to_half2(c[e]), s2);
+                const float2 sf = __half22float2(s2);
+                d = sf.x + sf.y;
+            } else {
+                float k[EPL];
+                unpack16<false>(raw, k);
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) d = fmaf(q[e], k[e], d);
+            }
+            part_dot[j] = d;
+        }
+        const int my_t = grp * TPG + sub / DUP;
+        float z = butterfly_reduce<TPG, LPR>(part_dot, lane);
+        if constexpr (kFp8) z *= logit_k_scale;
+        z = (my_t < valid) ? z : -INFINITY;
+
+        // ---- online softmax (base 2)
+        const float m_new = fmaxf(m, warp_max(z));
+        const float alpha = fast_exp2(m - m_new);
+        const float pz = fast_exp2(z - m_new);
+        l = l * alpha + pz;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) acc[e] *= alpha;
+        m = m_new;
+
+        // ---- P.V for this lane group's tokens (E4M3: the tile's tokens are
+        //      accumulated in f16x2, then added to the fp32 accumulators)
+        __half2 pv2[kFp8 ? EPL / 2 : 1];
+        if constexpr (kFp8) {
+#pragma unroll
+            for (int e = 0; e < EPL / 2; ++e) pv2[e] = __float2half2_rn(0.f);
+        }
+#pragma unroll
+        for (int j = 0; j < TPG; ++j) {
+            const int t = grp * TPG + j;
+            const float pj = __shfl_sync(0xffffffffu, pz, grp * LPR + j * DUP);
+            if (t < valid) {
+                uint4 raw;
+                if (t == t_new) raw = v_new;
+                else raw = *reinterpret_cast<const uint4 *>(vtile + t * row_stride + head_off);
+                if constexpr (kFp8) {
+                    const __half2 p2 = __float2half2_rn(pj);  // weight <= 1 in f16
+                    const uint16_t *c = reinterpret_cast<const uint16_t *>(&raw);
+#pragma unroll
+                    for (int e = 0; e < EPL / 2; ++e) pv2[e] = __hfma2(p2, e4m3x2_to_half2(c[e]), pv2[e]);
+                } else {
+                    float v[EPL];
+                    unpack16<false>(raw, v);
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) acc[e] = fmaf(pj, v[e], acc[e]);
+                }
+            }
+        }
+        if constexpr (kFp8) {
+#pragma unroll
+            for (int e = 0; e < EPL / 2; ++e) {
+                const float2 f = __half22float2(pv2[e]);
+                acc[2 * e] += f.x;
+                acc[2 * e + 1] += f.y;
+            }
+        }
+    }
+
+    // Sums l over all lanes and acc over the lane groups (group 0 then holds
+    // the warp's whole accumulator).
+    __device__ __forceinline__ void finish() {
+        l = warp_sum(l) * (1.0f / DUP);
+#pragma unroll
+        for (int mask = LPR; mask < 32; mask <<= 1) {
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], mask);
+        }
+    }
+};
+
 // Shared-memory carve-up, identical on host and device. A CTA serves C work
 // units ("slots"); slot j owns a ring of `stages` K/V stages and a merge
 // area. The mbarriers of all slots follow the slots: full[C][stages],
@@ -193,13 +339,15 @@ __device__ __forceinline__ Unit unit_of(const DecodeParams &p, int B, int j) {
     int L = min(u.L_in, p.max_blocks_per_seq * B);
     L = min(L, p.max_context_len);
     u.L = max(L, 0);
-    u.n_parts = (u.L + p.partition_size - 1) / p.partition_size;
+    const int rem = max(u.L - p.prefix_tokens, 0);  // tokens after the shared prefix
+    u.n_parts = (rem + p.partition_size - 1) / p.partition_size;
     u.live = exists && u.part < u.n_parts;
-    u.t0 = u.part * p.partition_size;
+    u.t0 = p.prefix_tokens + u.part * p.partition_size;
     u.t1 = min(u.L, u.t0 + p.partition_size);
     u.blk0 = u.t0 / B;
     u.nblk = u.live ? (u.t1 - u.t0 + B - 1) / B : 0;
-    u.append = u.live && p.new_key != nullptr && u.part == u.n_parts - 1 && u.L == u.L_in;
+    u.append = u.live && p.new_key != nullptr && u.part == u.n_parts - 1 && u.L == u.L_in &&
+               u.L > p.prefix_tokens;
     return u;
 }
 
@@ -208,7 +356,7 @@ __global__ void __launch_bounds__(kMaxDecodeThreads, 1)
 paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
     using Geo = Geometry<D, B, kFp8>;
-    constexpr int EPL = Geo::EPL, LPR = Geo::LPR, TPG = Geo::TPG, DUP = Geo::DUP;
+    constexpr int EPL = Geo::EPL, LPR = Geo::LPR;
     constexpr int EB = Geo::kElemBytes;
 
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -236,7 +384,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 if (id < p.num_units) {
                     const int part = (int)(id % p.max_parts);
                     const int s = (int)(id / p.max_parts / (p.num_heads / G));
-                    const int e = part * (p.partition_size / B) + lane;
+                    const int e = (p.prefix_tokens + part * p.partition_size) / B + lane;
                     if (e < p.max_blocks_per_seq)
                         pre_blk[j] = __ldg(p.block_tables + (size_t)s * p.max_blocks_per_seq + e);
                 }
@@ -271,8 +419,25 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 if (u[j].L_in > p.max_blocks_per_seq * B) flag_error(PA_DEV_CTX_OVER_TABLE);
                 else if (u[j].L_in > p.max_context_len) flag_error(PA_DEV_CTX_OVER_BOUND);
                 // sequences with nothing to append report slot -1
-                if (p.slot_out && !(p.new_key != nullptr && u[j].L == u[j].L_in && u[j].L > 0))
+                if (p.slot_out && !(p.new_key != nullptr && u[j].L == u[j].L_in && u[j].L > p.prefix_tokens))
                     p.slot_out[u[j].s] = -1;
+                // shared prefix: appending inside the shared blocks breaks copy-on-write
+                if (p.prefix_tokens > 0 && p.new_key != nullptr && u[j].L > 0 && u[j].L <= p.prefix_tokens)
+                    flag_error(PA_DEV_PREFIX);
+            }
+        }
+        // shared prefix: this sequence's first table entries must be row 0's
+        if (p.prefix_tokens > 0) {
+#pragma unroll
+            for (int j = 0; j < kMaxUnitsPerCta; ++j) {
+                const int64_t id = (int64_t)blockIdx.x + (int64_t)j * gridDim.x;
+                if (j < C && id < p.num_units && u[j].part == 0 && u[j].h0 == 0 && u[j].s > 0) {
+                    bool same = true;
+                    for (int e = lane; e < p.prefix_tokens / B; e += 32)
+                        same &= __ldg(p.block_tables + (size_t)u[j].s * p.max_blocks_per_seq + e) ==
+                                __ldg(p.block_tables + e);
+                    if (!__all_sync(0xffffffffu, same) && lane == 0) flag_error(PA_DEV_PREFIX);
+                }
             }
         }
         const uint64_t policy = l2_policy_evict_first();
@@ -370,36 +535,13 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
     if (!x.live) {
         // empty context: zeros (partition 0 of a context of length 0)
         const int64_t id = (int64_t)blockIdx.x + (int64_t)slot * gridDim.x;
-        if (id < p.num_units && x.L == 0 && x.part == 0 && w == 0 && lane < D / 8)
+        if (id < p.num_units && x.L == 0 && x.part == 0 && p.prefix_tokens == 0 && w == 0 && lane < D / 8)
             reinterpret_cast<uint4 *>(p.out + ((size_t)x.s * p.num_heads + h) * D)[lane] = make_uint4(0, 0, 0, 0);
         return;  // (all warps of this slot leave together: no merge barrier to meet)
     }
 
-    // fp16 caches: query in fp32, pre-scaled by scale*log2(e). E4M3 caches:
-    // the pre-scaled query rounded to f16 pairs, multiplied exactly against
-    // the decoded f16 keys by mixed-precision FMAs (k_scale goes on the logit).
-    float q[kFp8 ? 1 : EPL];
-    uint32_t q2[kFp8 ? EPL / 2 : 1];
-    {
-        float qf[EPL];
-#pragma unroll
-        for (int c = 0; c < EPL / 8; ++c) unpack16<false>(q_raw[c], qf + 8 * c);
-        if constexpr (kFp8) {
-#pragma unroll
-            for (int e = 0; e < EPL / 2; ++e) {
-                const __half2 h = __floats2half2_rn(qf[2 * e] * p.qk_scale_log2, qf[2 * e + 1] * p.qk_scale_log2);
-                q2[e] = *reinterpret_cast<const uint32_t *>(&h);
-            }
-        } else {
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) q[e] = qf[e] * p.qk_scale_log2;
-        }
-    }
-
-    float m = -INFINITY, l = 0.f;
-    float acc[EPL];
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
+    HeadAttn<D, B, kFp8> st;
+    st.init(q_raw, p.qk_scale_log2);
 
     const size_t row_stride = (size_t)G * D * EB;  // bytes between tokens in a tile
     const size_t head_off = (size_t)g * D * EB + (size_t)sub * 16;
@@ -441,84 +583,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const unsigned char *vtile = ktile + lay.tile_bytes;
         const int valid = min(B, x.t1 - (x.t0 + i * B));  // tokens of this block inside the context
         const int t_new = (i == t_new_block) ? t_new_row : -1;
-
-        // ---- logits of this lane group's TPG tokens
-        float part_dot[TPG];
-#pragma unroll
-        for (int j = 0; j < TPG; ++j) {
-            const int t = grp * TPG + j;
-            uint4 raw;
-            if (t == t_new) raw = k_new;
-            else raw = *reinterpret_cast<const uint4 *>(ktile + t * row_stride + head_off);
-            float d = 0.f;
-            if constexpr (kFp8) {
-                // packed f16x2 products of the f16 query and the decoded keys,
-                // summed in f16x2 over this lane's 16 elements, then in fp32
-                const uint16_t *c = reinterpret_cast<const uint16_t *>(&raw);
-                __half2 s2 = __float2half2_rn(0.f);
-#pragma unroll
-                for (int e = 0; e < EPL / 2; ++e)
-                    s2 = __hfma2(*reinterpret_cast<const __half2 *>(&q2[e]), e4m3x2_to_half2(c[e]), s2);
-                const float2 sf = __half22float2(s2);
-                d = sf.x + sf.y;
-            } else {
-                float k[EPL];
-                unpack16<false>(raw, k);
-#pragma unroll
-                for (int e = 0; e < EPL; ++e) d = fmaf(q[e], k[e], d);
-            }
-            part_dot[j] = d;
-        }
-        const int my_t = grp * TPG + sub / DUP;
-        float z = butterfly_reduce<TPG, LPR>(part_dot, lane);
-        if constexpr (kFp8) z *= p.logit_k_scale;
-        z = (my_t < valid) ? z : -INFINITY;
-
-        // ---- online softmax (base 2)
-        const float m_new = fmaxf(m, warp_max(z));
-        const float alpha = fast_exp2(m - m_new);
-        const float pz = fast_exp2(z - m_new);
-        l = l * alpha + pz;
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) acc[e] *= alpha;
-        m = m_new;
-
-        // ---- P.V for this lane group's tokens (E4M3: the block's tokens are
-        //      accumulated in f16x2, then added to the fp32 accumulators)
-        __half2 pv2[kFp8 ? EPL / 2 : 1];
-        if constexpr (kFp8) {
-#pragma unroll
-            for (int e = 0; e < EPL / 2; ++e) pv2[e] = __float2half2_rn(0.f);
-        }
-#pragma unroll
-        for (int j = 0; j < TPG; ++j) {
-            const int t = grp * TPG + j;
-            const float pj = __shfl_sync(0xffffffffu, pz, grp * LPR + j * DUP);
-            if (t < valid) {
-                uint4 raw;
-                if (t == t_new) raw = v_new;
-                else raw = *reinterpret_cast<const uint4 *>(vtile + t * row_stride + head_off);
-                if constexpr (kFp8) {
-                    const __half2 p2 = __float2half2_rn(pj);  // weight <= 1 in f16
-                    const uint16_t *c = reinterpret_cast<const uint16_t *>(&raw);
-#pragma unroll
-                    for (int e = 0; e < EPL / 2; ++e) pv2[e] = __hfma2(p2, e4m3x2_to_half2(c[e]), pv2[e]);
-                } else {
-                    float v[EPL];
-                    unpack16<false>(raw, v);
-#pragma unroll
-                    for (int e = 0; e < EPL; ++e) acc[e] = fmaf(pj, v[e], acc[e]);
-                }
-            }
-        }
-        if constexpr (kFp8) {
-#pragma unroll
-            for (int e = 0; e < EPL / 2; ++e) {
-                const float2 f = __half22float2(pv2[e]);
-                acc[2 * e] += f.x;
-                acc[2 * e + 1] += f.y;
-            }
-        }
+        st.consume(ktile, vtile, row_stride, head_off, valid, t_new, k_new, v_new, p.logit_k_scale, lane);
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[stage]);
         stage += W;
@@ -529,12 +594,9 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
     }
 
     // ---- reduce this warp's state: l over all lanes, acc over lane groups
-    l = warp_sum(l) * (1.0f / DUP);
-#pragma unroll
-    for (int mask = LPR; mask < 32; mask <<= 1) {
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], mask);
-    }
+    st.finish();
+    float m = st.m, l = st.l;
+    float (&acc)[EPL] = st.acc;
 
     // ---- merge the W warps of each head through the slot's shared memory
     if (W > 1) {
@@ -567,7 +629,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
 
     if (grp != 0) return;
     const float inv_l = 1.0f / l;
-    if (x.n_parts == 1) {
+    if (x.n_parts == 1 && p.prefix_tokens == 0) {
         __half *op = p.out + ((size_t)x.s * p.num_heads + h) * D + sub * EPL;
 #pragma unroll
         for (int c = 0; c < EPL / 8; ++c) {
@@ -580,7 +642,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
             reinterpret_cast<uint4 *>(op)[c] = pk;
         }
     } else {
-        const size_t idx = ((size_t)x.s * p.num_heads + h) * p.max_parts + x.part;
+        const size_t idx = ((size_t)x.s * p.num_heads + h) * p.ws_parts + p.prefix_parts + x.part;
         float *op = p.ws_o + idx * D + sub * EPL;
 #pragma unroll
         for (int c = 0; c < EPL / 4; ++c)
@@ -591,9 +653,12 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
     }
 }
 
-// Log-sum-exp reduction of the partitions of each (sequence, head) whose
-// context spans more than one partition. One warp per (sequence, head):
+// Log-sum-exp reduction of the partial results of each (sequence, head):
+// the partitions of a context longer than one partition, and with a shared
+// prefix, the prefix partitions followed by the suffix partitions. One warp
+// per (sequence, head):
 //   M = max_p lse_p,  w_p = 2^(lse_p - M),  out = v_scale * sum_p w_p o_p / sum_p w_p
+// Partials without tokens carry lse = -inf and o = 0 (weight 0).
 template <int D>
 __global__ void __launch_bounds__(128)
 lse_reduce_kernel(const DecodeParams p) {
@@ -602,15 +667,24 @@ lse_reduce_kernel(const DecodeParams p) {
     const int s = blockIdx.y;
     if (h >= p.num_heads) return;
     int L = __ldg(p.context_lens + s);
-    L = min(L, p.max_blocks_per_seq * p.block_size);   // same clamps as the partition kernel
+    L = min(L, p.max_blocks_per_seq * p.block_size);   // same clamps as the partition kernels
     L = min(L, p.max_context_len);
-    const int n_parts = L > 0 ? (L + p.partition_size - 1) / p.partition_size : 0;
-    if (n_parts <= 1) return;
-    const size_t base = ((size_t)s * p.num_heads + h) * p.max_parts;
+    L = max(L, 0);
+    const int rem = max(L - p.prefix_tokens, 0);
+    const int n_suffix = (rem + p.partition_size - 1) / p.partition_size;
+    const int n_parts = p.prefix_parts + n_suffix;
+    constexpr int DPL = D / 32;  // dims per lane
+    __half *op = p.out + ((size_t)s * p.num_heads + h) * D + lane * DPL;
+    if (p.prefix_tokens == 0 && n_parts <= 1) return;  // written by the partition kernel
+    if (L == 0) {
+#pragma unroll
+        for (int e = 0; e < DPL; e += 2) *reinterpret_cast<__half2 *>(op + e) = __floats2half2_rn(0.f, 0.f);
+        return;
+    }
+    const size_t base = ((size_t)s * p.num_heads + h) * p.ws_parts;
     float M = -INFINITY;
     for (int i = lane; i < n_parts; i += 32) M = fmaxf(M, p.ws_lse[base + i]);
     M = warp_max(M);
-    constexpr int DPL = D / 32;  // dims per lane
     float acc[DPL];
 #pragma unroll
     for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
@@ -632,10 +706,136 @@ lse_reduce_kernel(const DecodeParams p) {
         }
     }
     const float f = p.out_scale / wsum;
-    __half *op = p.out + ((size_t)s * p.num_heads + h) * D + lane * DPL;
 #pragma unroll
     for (int e = 0; e < DPL; e += 2)
         *reinterpret_cast<__half2 *>(op + e) = __floats2half2_rn(acc[e] * f, acc[e + 1] * f);
+}
+
+// Shared-prefix attention ("在A10G上榨干LLaMA-7B" §2.2: requests sharing a
+// prompt map its logical blocks to the same physical blocks). The prefix
+// blocks -- the first prefix_tokens tokens of table row 0, which every row
+// shares -- are read once per CTA and applied to the queries of up to
+// queries_per_cta sequences: one CTA = G heads x one prefix partition x a
+// block of sequences; consumer warp (g, i) computes head g of sequence
+// qb * queries_per_cta + i over every tile (masked to that sequence's own
+// length) with the same per-tile arithmetic as the decode, and writes the
+// partition's partial (lse, o) at index pp of the sequence's partials.
+template <int D, int B, bool kFp8>
+__global__ void __launch_bounds__(kMaxDecodeThreads, 1)
+paged_prefix_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                    const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
+    using Geo = Geometry<D, B, kFp8>;
+    constexpr int EPL = Geo::EPL, LPR = Geo::LPR;
+    constexpr int EB = Geo::kElemBytes;
+    extern __shared__ __align__(1024) unsigned char smem[];
+    const int G = p.heads_per_cta, QC = p.queries_per_cta, stages = p.stages;
+    const SmemLayout lay(B, G, D, EB, 1, stages, 1);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + lay.bars_off);
+    uint64_t *empty = full + stages;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_consumers = G * QC;
+
+    const int n_qb = (p.num_seqs + QC - 1) / QC;
+    const int qb = blockIdx.x % n_qb;
+    const int rest = blockIdx.x / n_qb;
+    const int pp = rest % p.prefix_parts;
+    const int h0 = (rest / p.prefix_parts) * G;
+    const int t0 = pp * p.prefix_partition;
+    const int t1 = min(p.prefix_tokens, t0 + p.prefix_partition);
+    const int blk0 = t0 / B;
+    const int nblk = (t1 - t0 + B - 1) / B;
+
+    if (warp == n_consumers) {
+        // ---------------------------------------------------------- producer
+        int pre = 0;
+        if (lane < nblk) pre = __ldg(p.block_tables + blk0 + lane);  // row 0 holds the shared blocks
+        if (lane == 0) {
+            prefetch_tensor_map(&tmap_k);
+            prefetch_tensor_map(&tmap_v);
+            for (int i = 0; i < stages; ++i) {
+                mbar_init(&full[i], 1);
+                mbar_init(&empty[i], n_consumers);
+            }
+            fence_mbar_init();
+        }
+        __syncwarp();
+        asm volatile("bar.arrive 1, %0;" ::"r"((n_consumers + 1) * 32) : "memory");
+        const uint64_t policy = l2_policy_evict_first();
+        bool ok = true;
+        for (int i = 0; i < nblk && ok; ++i) {
+            if (i > 0 && (i & 31) == 0) {
+                pre = 0;
+                if (i + lane < nblk) pre = __ldg(p.block_tables + blk0 + i + lane);
+            }
+            int blk = __shfl_sync(0xffffffffu, pre, i & 31);
+            const bool bad = blk < 0 || blk >= p.num_blocks;
+            if (bad) blk = p.num_blocks;
+            const int st = i % stages, use = i / stages;
+            if (lane == 0) {
+                if (bad) flag_error(PA_DEV_BAD_BLOCK);
+                if (use > 0) ok = mbar_wait(&empty[st], (use - 1) & 1);
+                if (ok) {
+                    unsigned char *kdst = smem + (size_t)st * lay.stage_bytes;
+                    mbar_arrive_expect_tx(&full[st], (uint32_t)lay.stage_bytes);
+                    tma_load_4d(kdst, &tmap_k, &full[st], 0, h0, 0, blk, policy);
+                    tma_load_4d(kdst + lay.tile_bytes, &tmap_v, &full[st], 0, h0, 0, blk, policy);
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+        }
+        return;
+    }
+
+    // -------------------------------------------------------------- consumers
+    const int g = warp % G;
+    const int s = qb * QC + warp / G;
+    const int h = h0 + g;
+    const bool active = s < p.num_seqs;
+    const int sub = lane % LPR, grp = lane / LPR;
+    uint4 q_raw[EPL / 8];
+    int L = 0;
+    if (active) {
+        const uint4 *qp = reinterpret_cast<const uint4 *>(p.query + ((size_t)s * p.num_heads + h) * D);
+#pragma unroll
+        for (int c = 0; c < EPL / 8; ++c) q_raw[c] = __ldg(qp + sub * (EPL / 8) + c);
+        L = __ldg(p.context_lens + s);
+        L = min(L, p.max_blocks_per_seq * B);
+        L = max(min(L, p.max_context_len), 0);
+    } else {
+#pragma unroll
+        for (int c = 0; c < EPL / 8; ++c) q_raw[c] = make_uint4(0, 0, 0, 0);
+    }
+    asm volatile("bar.sync 1, %0;" ::"r"((n_consumers + 1) * 32) : "memory");
+    HeadAttn<D, B, kFp8> st;
+    st.init(q_raw, p.qk_scale_log2);
+    const int end = min(t1, L);  // this sequence's tokens in the partition
+    const size_t row_stride = (size_t)G * D * EB;
+    const size_t head_off = (size_t)g * D * EB + (size_t)sub * 16;
+    const uint4 none = make_uint4(0, 0, 0, 0);
+    for (int i = 0; i < nblk; ++i) {
+        const int stg = i % stages, use = i / stages;
+        if (!mbar_wait(&full[stg], use & 1)) break;
+        const int valid = min(B, end - (t0 + i * B));
+        if (valid > 0) {
+            const unsigned char *ktile = smem + (size_t)stg * lay.stage_bytes;
+            st.consume(ktile, ktile + lay.tile_bytes, row_stride, head_off, valid, -1, none, none,
+                       p.logit_k_scale, lane);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[stg]);
+    }
+    if (!active) return;
+    st.finish();
+    if (grp != 0) return;
+    const size_t idx = ((size_t)s * p.num_heads + h) * p.ws_parts + pp;
+    float *op = p.ws_o + idx * D + sub * EPL;
+    const bool any = st.l > 0.f;
+    const float inv_l = any ? 1.0f / st.l : 0.f;
+#pragma unroll
+    for (int c = 0; c < EPL / 4; ++c)
+        reinterpret_cast<float4 *>(op)[c] = make_float4(st.acc[4 * c] * inv_l, st.acc[4 * c + 1] * inv_l,
+                                                        st.acc[4 * c + 2] * inv_l, st.acc[4 * c + 3] * inv_l);
+    if (sub == 0) p.ws_lse[idx] = any ? st.m + fast_log2(st.l) : -INFINITY;
 }
 
 }  // namespace pa

@@ -224,6 +224,53 @@ def paged_attention_decode_append(out: torch.Tensor, query: torch.Tensor, new_ke
         ctypes.byref(cfg) if cfg is not None else None, ws_ptr, ws_bytes, _stream(stream)))
 
 
+def paged_attention_decode_shared_prefix(out: torch.Tensor, query: torch.Tensor,
+                                         key_cache: torch.Tensor, value_cache: torch.Tensor,
+                                         block_tables: torch.Tensor, context_lens: torch.Tensor,
+                                         shared_prefix_blocks: int, scale: float,
+                                         k_scale: float = 1.0, v_scale: float = 1.0,
+                                         new_key: torch.Tensor | None = None,
+                                         new_value: torch.Tensor | None = None,
+                                         max_context_len: int | None = None,
+                                         slot_mapping: torch.Tensor | None = None, config=None,
+                                         workspace: torch.Tensor | None = None, stream=None) -> None:
+    """Decode (with the fused append when new_key/new_value are given) for a
+    batch whose tables all start with the same ``shared_prefix_blocks`` blocks."""
+    _check_pair(key_cache, value_cache)
+    _i32(block_tables, "block_tables")
+    _i32(context_lens, "context_lens")
+    for t in (out, query):
+        if t.dtype != torch.float16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("out and query must be contiguous float16 CUDA tensors")
+    S, H, D = query.shape
+    if (new_key is None) != (new_value is None):
+        raise ValueError("give both new_key and new_value, or neither")
+    for t in (new_key, new_value):
+        if t is not None and (t.dtype != torch.float16 or not t.is_cuda or tuple(t.shape) != (S, H, D)
+                              or t.stride(2) != 1 or t.stride(1) != D):
+            raise ValueError("new_key/new_value must be float16 CUDA tensors [S, H, D] with contiguous rows")
+    desc = cache_desc(key_cache)
+    if max_context_len is None:
+        max_context_len = block_tables.shape[1] * desc.block_size
+    if slot_mapping is not None:
+        _i32(slot_mapping, "slot_mapping")
+    cfg = _config(config)
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    check(lib().pa_paged_attention_decode_shared_prefix(
+        out.data_ptr(), query.data_ptr(),
+        new_key.data_ptr() if new_key is not None else None,
+        new_value.data_ptr() if new_value is not None else None,
+        new_key.stride(0) if new_key is not None else H * D,
+        new_value.stride(0) if new_value is not None else H * D,
+        key_cache.data_ptr(), value_cache.data_ptr(), desc, block_tables.data_ptr(),
+        block_tables.shape[1], context_lens.data_ptr(), S, int(max_context_len),
+        int(shared_prefix_blocks), float(scale), float(k_scale), float(v_scale),
+        slot_mapping.data_ptr() if slot_mapping is not None else None,
+        ctypes.byref(cfg) if cfg is not None else None, ws_ptr, ws_bytes, _stream(stream)))
+
+
 def check_status(stream=None) -> int:
     """Synchronise the stream; return and clear the device error bits (PA_DEV_*)."""
     code = ctypes.c_uint32(0)
@@ -264,15 +311,25 @@ def decode_step(out: torch.Tensor, query: torch.Tensor, new_key: torch.Tensor,
                 k_scale: float = 1.0, v_scale: float = 1.0, cow_pairs: torch.Tensor | None = None,
                 slots: torch.Tensor | None = None, max_context_len: int | None = None,
                 config=None, workspace: torch.Tensor | None = None, stream=None,
-                fused: bool = True) -> torch.Tensor:
+                fused: bool = True, shared_prefix_blocks: int = 0) -> torch.Tensor:
     """One decode step of the whole path, all on the device, in order:
     copy-on-write block copies (if any pairs), slot of each appended token,
     scatter of the new K/V rows into those slots, decode attention.
     ``block_tables`` are the tables after any copy-on-write repoint. With
     ``fused`` the last three run as one launch (paged_attention_decode_append);
-    otherwise as three separate calls. Returns the slot tensor."""
+    otherwise as three separate calls. With ``shared_prefix_blocks`` > 0 the
+    decode reads the shared prefix once per head (paged_attention_decode_shared_prefix).
+    Returns the slot tensor."""
     if cow_pairs is not None and cow_pairs.numel():
         copy_blocks(key_cache, value_cache, cow_pairs, stream)
+    if shared_prefix_blocks:
+        if slots is None:
+            slots = torch.empty(query.shape[0], dtype=torch.int32, device=query.device)
+        paged_attention_decode_shared_prefix(out, query, key_cache, value_cache, block_tables,
+                                             context_lens, shared_prefix_blocks, scale, k_scale,
+                                             v_scale, new_key, new_value, max_context_len, slots,
+                                             config, workspace, stream)
+        return slots
     if fused:
         if slots is None:
             slots = torch.empty(query.shape[0], dtype=torch.int32, device=query.device)

@@ -10,6 +10,7 @@ import torch
 
 import oracle
 import pagedattention_paged_kv_decode_b200 as pk
+from pagedattention_paged_kv_decode_b200 import capi
 import workloads as W
 from _oracle_step import oracle_step, sample_seqs
 
@@ -18,7 +19,7 @@ pytestmark = pytest.mark.gpu
 TOL = {"f16": 2e-3, "e4m3": 1e-2}
 
 
-def run_step(w, dev, config=None, max_context_len=None, fused=True):
+def run_step(w, dev, config=None, max_context_len=None, fused=True, shared=False):
     dw = W.to_device(w, dev, encode=pk.load_cache)
     ws = None
     if config is not None and not fused:
@@ -29,7 +30,7 @@ def run_step(w, dev, config=None, max_context_len=None, fused=True):
                    dw.block_tables, dw.context_lens, w.scale, w.k_scale, w.v_scale,
                    cow_pairs=dw.cow_pairs, slots=dw.slots,
                    max_context_len=max_context_len or w.max_context_len, config=config, workspace=ws,
-                   fused=fused)
+                   fused=fused, shared_prefix_blocks=w.shared_blocks if shared else 0)
     assert pk.check_status() == 0
     return dw
 
@@ -189,3 +190,69 @@ def test_determinism(cuda_device):
     a = host(run_step(w, cuda_device).out)
     b = host(run_step(w, cuda_device).out)
     assert np.array_equal(a.view(np.uint16), b.view(np.uint16))
+
+
+# ------------------------------------------------------------ shared prefix
+
+def test_shared_prefix_named_workload_4(cuda_device):
+    w = W.named(4)
+    assert w.shared_blocks == 95
+    dw = run_step(w, cuda_device, shared=True)
+    compare_step(w, dw, sample_seqs(w, 8, seed=4), check_all_blocks=False)
+
+
+def prefix_case(D, B, kv, prefix_blocks, suffixes, seed, cow=False, H=4):
+    prefix = prefix_blocks * B
+    ctx = [prefix + x for x in suffixes]
+    need = prefix_blocks + sum(-(-max(0, L - prefix) // B) for L in ctx) + (len(ctx) if cow else 0)
+    width = max(-(-L // B) for L in ctx)
+    return W.build(f"prefix_{kv}_d{D}_b{B}", H, D, B, kv, ctx, need + 5, width, seed,
+                   q_std=1.0, kv_std=1.0, shared_prefix=prefix, cow=cow)
+
+
+@pytest.mark.parametrize("cow", [False, True], ids=["shared", "cow"])
+@pytest.mark.parametrize("D,B,kv", [(128, 16, "f16"), (128, 32, "f16"), (64, 16, "e4m3"), (128, 32, "e4m3")])
+def test_shared_prefix_matches_oracle(cuda_device, D, B, kv, cow):
+    suffixes = [1, B, B + 3, 700, 1300, 40, 2 * B - 1]
+    w = prefix_case(D, B, kv, 40 if B == 16 else 20, suffixes, seed=D + B + cow, cow=cow)
+    assert w.shared_blocks == (39 if B == 16 else 19) if cow else (40 if B == 16 else 20)
+    dw = run_step(w, cuda_device, shared=True)
+    compare_step(w, dw, list(range(w.num_seqs)), check_all_blocks=True)
+
+
+def test_shared_prefix_plain_decode_with_short_contexts(cuda_device):
+    """Without an append, contexts may end inside the shared prefix; the
+    prefix kernel masks each sequence to its own length."""
+    B, prefix_blocks = 16, 12
+    w = prefix_case(128, B, "f16", prefix_blocks, [5, 300, 17, 1], seed=31)
+    ctx = w.context_lens.copy()
+    ctx[1] = 100       # ends inside the prefix
+    ctx[3] = 1
+    dw = W.to_device(w, cuda_device)
+    pk.paged_attention_decode_shared_prefix(dw.out, dw.query, dw.key_cache, dw.value_cache,
+                                            dw.block_tables, torch.from_numpy(ctx).to(cuda_device),
+                                            prefix_blocks, w.scale)
+    assert pk.check_status() == 0
+    kc, vc = w.pool_host()
+    ref = oracle.paged_attention(w.query, kc, vc, w.block_tables, ctx, w.scale)
+    got = host(dw.out).astype(np.float64)
+    assert np.abs(got - ref).max() <= 2e-3
+
+
+def test_shared_prefix_contract_is_checked(cuda_device):
+    B, prefix_blocks = 16, 8
+    w = prefix_case(128, B, "f16", prefix_blocks, [5, 20, 33], seed=32)
+    dw = W.to_device(w, cuda_device)
+    bt = dw.block_tables.clone()
+    bt[2, 3] = bt[1, prefix_blocks]      # row 2 no longer shares logical block 3
+    pk.paged_attention_decode_shared_prefix(dw.out, dw.query, dw.key_cache, dw.value_cache, bt,
+                                            dw.context_lens, prefix_blocks, w.scale)
+    assert pk.check_status() == capi.PA_DEV_PREFIX
+    ctx = dw.context_lens.clone()
+    ctx[0] = prefix_blocks * B           # the appended token would land in a shared block
+    pk.paged_attention_decode_shared_prefix(dw.out, dw.query, dw.key_cache, dw.value_cache,
+                                            dw.block_tables, ctx, prefix_blocks, w.scale,
+                                            new_key=dw.new_key, new_value=dw.new_value,
+                                            slot_mapping=dw.slots)
+    assert pk.check_status() == capi.PA_DEV_PREFIX
+    assert dw.slots.cpu().tolist()[0] == -1

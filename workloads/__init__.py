@@ -56,6 +56,7 @@ class Workload:
     poison: str = POISON_HUGE
     cow_pairs: np.ndarray = field(default_factory=lambda: np.zeros((0, 2), np.int32))
     block_tables_shared: np.ndarray | None = None   # tables before the copy-on-write repoint
+    shared_blocks: int = 0         # leading table entries identical in every row of block_tables
     seed: int = 0
 
     @property
@@ -246,7 +247,9 @@ def build(name: str, num_heads: int, head_size: int, block_size: int, kv_dtype: 
                     new_value=new_value, block_tables=tables, context_lens=ctx,
                     live_blocks=blk.astype(np.int32), live_offsets=off.astype(np.int32),
                     live_key=live_k, live_value=live_v, poison=poison, cow_pairs=cow_pairs,
-                    block_tables_shared=shared_tables, seed=seed)
+                    block_tables_shared=shared_tables,
+                    shared_blocks=(n_shared - 1 if cow else n_shared) if (S > 1 and min(need, default=0) >= n_shared) else 0,
+                    seed=seed)
 
 
 # --------------------------------------------------------- named workloads
