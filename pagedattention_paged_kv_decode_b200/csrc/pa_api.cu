@@ -81,10 +81,10 @@ EncodeTiledFn encode_fn() {
 
 struct MapKey {
     const void *ptr;
-    int nb, bs, nh, hd, dtype, g;
+    int nb, bs, nh, hd, dtype, g, swz;
     bool operator==(const MapKey &o) const {
         return ptr == o.ptr && nb == o.nb && bs == o.bs && nh == o.nh && hd == o.hd &&
-               dtype == o.dtype && g == o.g;
+               dtype == o.dtype && g == o.g && swz == o.swz;
     }
 };
 
@@ -94,8 +94,10 @@ std::vector<std::pair<MapKey, CUtensorMap>> g_maps;  // small FIFO cache
 // 4-D view of a cache, innermost first: {head_size, num_heads, block_size,
 // num_blocks}; box {head_size, G, block_size, 1} = one physical block's rows
 // for G heads. Zero fill outside the pool.
-int cache_tensor_map(const void *cache, const pa_cache_desc &c, int G, CUtensorMap *out) {
-    const MapKey key{cache, c.num_blocks, c.block_size, c.num_heads, c.head_size, c.dtype, G};
+// swz = 1: box {64, 1, block_size, 1} (a 64-dim half of one head's rows)
+// with 128-byte swizzle, for the tensor-core shared-prefix kernel.
+int cache_tensor_map(const void *cache, const pa_cache_desc &c, int G, CUtensorMap *out, int swz = 0) {
+    const MapKey key{cache, c.num_blocks, c.block_size, c.num_heads, c.head_size, c.dtype, G, swz};
     {
         std::lock_guard<std::mutex> lk(g_map_mu);
         for (auto &e : g_maps)
@@ -112,14 +114,16 @@ int cache_tensor_map(const void *cache, const pa_cache_desc &c, int G, CUtensorM
     const cuuint64_t strides[3] = {(cuuint64_t)c.head_size * eb,
                                    (cuuint64_t)c.head_size * c.num_heads * eb,
                                    (cuuint64_t)c.head_size * c.num_heads * c.block_size * eb};
-    const cuuint32_t box[4] = {(cuuint32_t)c.head_size, (cuuint32_t)G, (cuuint32_t)c.block_size, 1};
+    const cuuint32_t box[4] = {swz ? 64u : (cuuint32_t)c.head_size, swz ? 1u : (cuuint32_t)G,
+                               (cuuint32_t)c.block_size, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     CUtensorMap m;
     const CUresult r = enc(&m,
                            c.dtype == PA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                              : CU_TENSOR_MAP_DATA_TYPE_UINT8,
                            4, const_cast<void *>(cache), dims, strides, box, estr,
-                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           swz ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
     {
@@ -256,6 +260,14 @@ DecodeKernel pick_prefix(int D, int B, bool fp8) {
     return nullptr;
 }
 
+DecodeKernel pick_prefix_mma(int D, int B) {
+    if (D == 64 && B == 16) return pa::paged_prefix_mma_kernel<64, 16>;
+    if (D == 64 && B == 32) return pa::paged_prefix_mma_kernel<64, 32>;
+    if (D == 128 && B == 16) return pa::paged_prefix_mma_kernel<128, 16>;
+    if (D == 128 && B == 32) return pa::paged_prefix_mma_kernel<128, 32>;
+    return nullptr;
+}
+
 ReduceKernel pick_reduce(int D) {
     return D == 64 ? pa::lse_reduce_kernel<64> : pa::lse_reduce_kernel<128>;
 }
@@ -349,6 +361,7 @@ struct PrefixPlan {
     int heads;          // heads per CTA
     int queries;        // sequences per CTA
     int stages;
+    bool mma;           // fp16 caches: the tensor-core kernel
 };
 
 int launch_decode(void *out, const void *query, const void *kc, const void *vc,
@@ -422,21 +435,27 @@ int launch_decode(void *out, const void *query, const void *kc, const void *vc,
     if (rc) return rc;
     cudaError_t e;
     if (pre) {
-        DecodeKernel pkern = pick_prefix(D, B, fp8);
+        DecodeKernel pkern = pre->mma ? pick_prefix_mma(D, B) : pick_prefix(D, B, fp8);
         rc = ensure_smem_attr(reinterpret_cast<const void *>(pkern), device);
         if (rc) return rc;
         CUtensorMap pk_, pv_;
-        rc = cache_tensor_map(kc, c, pre->heads, &pk_);
+        rc = cache_tensor_map(kc, c, pre->heads, &pk_, pre->mma ? 1 : 0);
         if (rc) return rc;
-        rc = cache_tensor_map(vc, c, pre->heads, &pv_);
+        rc = cache_tensor_map(vc, c, pre->heads, &pv_, pre->mma ? 1 : 0);
         if (rc) return rc;
         pa::DecodeParams pp = p;
         pp.heads_per_cta = pre->heads;
         pp.stages = pre->stages;
-        const pa::SmemLayout play(B, pre->heads, D, elem_bytes(c), 1, pre->stages, 1);
         const int64_t n_qb = (S + pre->queries - 1) / pre->queries;
         const int64_t n = (int64_t)(c.num_heads / pre->heads) * pre->parts * n_qb;
-        pkern<<<dim3((unsigned)n), dim3(32 * (pre->heads * pre->queries + 1)), play.total, st>>>(pk_, pv_, pp);
+        if (pre->mma) {
+            // ring + barriers + 1 KiB to align the ring to 1024 bytes in the kernel
+            const size_t smem_bytes = (size_t)pre->stages * 4 * B * D + 16 * (size_t)pre->stages + 1024;
+            pkern<<<dim3((unsigned)n), dim3(32 * 5), smem_bytes, st>>>(pk_, pv_, pp);
+        } else {
+            const pa::SmemLayout play(B, pre->heads, D, elem_bytes(c), 1, pre->stages, 1);
+            pkern<<<dim3((unsigned)n), dim3(32 * (pre->heads * pre->queries + 1)), play.total, st>>>(pk_, pv_, pp);
+        }
         e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "paged_prefix_kernel launch");
     }
@@ -740,7 +759,8 @@ int plan_shared_prefix(const pa_cache_desc &c, int S, int bound, int prefix_bloc
     pre->partition = std::max(B, 512 / B * B);
     pre->parts = (pre->prefix_tokens + pre->partition - 1) / pre->partition;
     pre->heads = 1;
-    pre->queries = std::min(S, pa::kMaxConsumerWarps);
+    pre->mma = c.dtype == PA_F16;
+    pre->queries = pre->mma ? pa::kPrefixMmaQueries : std::min(S, pa::kMaxConsumerWarps);
     const size_t sb = pa::SmemLayout(B, 1, c.head_size, elem_bytes(c), 1, 1, 1).stage_bytes;
     pre->stages = (int)std::max<size_t>(2, std::min<size_t>(8, (96 * 1024) / sb));
     pa_decode_config r = cfg ? *cfg : pa_decode_config{0, 0, 0, 0, 0};

@@ -838,4 +838,257 @@ paged_prefix_kernel(const __grid_constant__ CUtensorMap tmap_k,
     if (sub == 0) p.ws_lse[idx] = any ? st.m + fast_log2(st.l) : -INFINITY;
 }
 
+// Shared-prefix attention on tensor cores (fp16 caches). One CTA = one head
+// x one prefix partition x up to 64 sequences; consumer warp w takes the 16
+// sequences 16w .. 16w+15 of the CTA's block. The producer streams the
+// shared blocks' K and V tiles (64-dim halves, 128-byte swizzle) through a
+// ring. Per tile and warp:
+//   S (16 x B)  = Q (16 x D) . K^T        mma.m16n8k16, K fragments by ldmatrix
+//   online softmax per row on the S fragments (masked to each row's length)
+//   O (16 x D) += P (16 x B) . V          P reused from the S registers as the
+//                                         A operand, V fragments by ldmatrix.trans
+// then the partition's partial (lse, o) of each sequence is written. Q and P
+// are f16 (P <= 1: relative rounding <= 2^-11); S and O accumulate in fp32.
+constexpr int kPrefixMmaQueries = 64;  // sequences per CTA (4 warps x 16)
+
+template <int D, int B>
+struct PrefixMmaLayout {
+    static constexpr int kHalves = D / 64;              // 64-dim half tiles per row
+    static constexpr int kHalfTile = B * 128;            // bytes of one half tile
+    static constexpr int kTile = kHalves * kHalfTile;    // one K (or V) tile
+    static constexpr int kStage = 2 * kTile;
+};
+
+template <int D, int B>
+__global__ void __launch_bounds__(32 * 5, 1)
+paged_prefix_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                        const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
+    using Lay = PrefixMmaLayout<D, B>;
+    constexpr int KS = D / 16;   // k-steps over dims
+    constexpr int NT = B / 8;    // score n-tiles (8 tokens each)
+    constexpr int ON = D / 8;    // output n-tiles (8 dims each)
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    // 128-byte-swizzled TMA destinations must be 1024-byte aligned: align the
+    // ring explicitly (the launch adds 1 KiB of slack).
+    unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const int stages = p.stages;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)stages * Lay::kStage);
+    uint64_t *empty = full + stages;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int S = p.num_seqs;
+    const int n_qb = (S + kPrefixMmaQueries - 1) / kPrefixMmaQueries;
+    const int qb = blockIdx.x % n_qb;
+    const int rest = blockIdx.x / n_qb;
+    const int pp = rest % p.prefix_parts;
+    const int h = rest / p.prefix_parts;
+    const int q_base = qb * kPrefixMmaQueries;
+    const int n_consumers = min(4, (S - q_base + 15) / 16);
+    const int t0 = pp * p.prefix_partition;
+    const int t1 = min(p.prefix_tokens, t0 + p.prefix_partition);
+    const int blk0 = t0 / B;
+    const int nblk = (t1 - t0 + B - 1) / B;
+
+    if (warp == n_consumers) {
+        // ---------------------------------------------------------- producer
+        int pre = 0;
+        if (lane < nblk) pre = __ldg(p.block_tables + blk0 + lane);  // row 0 holds the shared blocks
+        if (lane == 0) {
+            prefetch_tensor_map(&tmap_k);
+            prefetch_tensor_map(&tmap_v);
+            for (int i = 0; i < stages; ++i) {
+                mbar_init(&full[i], 1);
+                mbar_init(&empty[i], n_consumers);
+            }
+            fence_mbar_init();
+        }
+        __syncwarp();
+        asm volatile("bar.arrive 1, %0;" ::"r"((n_consumers + 1) * 32) : "memory");
+        const uint64_t policy = l2_policy_evict_first();
+        bool ok = true;
+        for (int i = 0; i < nblk && ok; ++i) {
+            if (i > 0 && (i & 31) == 0) {
+                pre = 0;
+                if (i + lane < nblk) pre = __ldg(p.block_tables + blk0 + i + lane);
+            }
+            int blk = __shfl_sync(0xffffffffu, pre, i & 31);
+            const bool bad = blk < 0 || blk >= p.num_blocks;
+            if (bad) blk = p.num_blocks;
+            const int st = i % stages, use = i / stages;
+            if (lane == 0) {
+                if (bad) flag_error(PA_DEV_BAD_BLOCK);
+                if (use > 0) ok = mbar_wait(&empty[st], (use - 1) & 1);
+                if (ok) {
+                    unsigned char *kdst = smem + (size_t)st * Lay::kStage;
+                    mbar_arrive_expect_tx(&full[st], (uint32_t)Lay::kStage);
+#pragma unroll
+                    for (int hf = 0; hf < Lay::kHalves; ++hf) {
+                        tma_load_4d(kdst + hf * Lay::kHalfTile, &tmap_k, &full[st], 64 * hf, h, 0, blk, policy);
+                        tma_load_4d(kdst + Lay::kTile + hf * Lay::kHalfTile, &tmap_v, &full[st], 64 * hf, h, 0,
+                                    blk, policy);
+                    }
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+        }
+        return;
+    }
+    if (warp > n_consumers) return;
+
+    // -------------------------------------------------------------- consumers
+    const int g = lane >> 2;          // fragment row (and row + 8)
+    const int c = (lane & 3) * 2;     // fragment column pair
+    const int q0 = q_base + warp * 16;
+    const int rows[2] = {q0 + g, q0 + g + 8};
+    int Lr[2];
+    uint32_t qa[KS][4];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        int L = 0;
+        if (rows[r] < S) {
+            L = __ldg(p.context_lens + rows[r]);
+            L = min(L, p.max_blocks_per_seq * B);
+            L = max(min(L, p.max_context_len), 0);
+        }
+        Lr[r] = min(L, t1);  // this row's tokens end here (within the partition)
+    }
+    {
+        const float sc = p.qk_scale_log2;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+#pragma unroll
+                for (int hi = 0; hi < 2; ++hi) {
+                    uint32_t v = 0;
+                    if (rows[r] < S) {
+                        const __half2 x = *reinterpret_cast<const __half2 *>(
+                            p.query + ((size_t)rows[r] * p.num_heads + h) * D + ks * 16 + c + 8 * hi);
+                        const float2 f = __half22float2(x);
+                        v = pack_half2(f.x * sc, f.y * sc);
+                    }
+                    qa[ks][r + 2 * hi] = v;  // a0 (row g), a1 (row g+8), a2/a3: +8 columns
+                }
+            }
+        }
+    }
+    asm volatile("bar.sync 1, %0;" ::"r"((n_consumers + 1) * 32) : "memory");
+
+    float o[ON][4];
+#pragma unroll
+    for (int j = 0; j < ON; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+
+    for (int i = 0; i < nblk; ++i) {
+        const int st = i % stages, use = i / stages;
+        if (!mbar_wait(&full[st], use & 1)) break;
+        const unsigned char *kt = smem + (size_t)st * Lay::kStage;
+        const unsigned char *vt = kt + Lay::kTile;
+        const int tb = t0 + i * B;  // first token of the tile
+
+        // ---- S = Q K^T
+        float sacc[NT][4];
+#pragma unroll
+        for (int n = 0; n < NT; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
+#pragma unroll
+        for (int np = 0; np < NT / 2; ++np) {
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+                // matrices: (tokens +0..7, dims +0..7), (+0..7, +8..15), (+8..15, +0..7), (+8..15, +8..15)
+                const int mi = lane >> 3, r = lane & 7;
+                const int tok = np * 16 + ((mi >> 1) << 3) + r;
+                const int dim = ks * 16 + ((mi & 1) << 3);
+                const unsigned char *addr = kt + (dim >> 6) * Lay::kHalfTile + swz128(tok, (dim & 63) * 2);
+                uint32_t b[4];
+                ldmatrix_x4(b, addr);
+                mma_16816(sacc[2 * np], qa[ks], b[0], b[1]);
+                mma_16816(sacc[2 * np + 1], qa[ks], b[2], b[3]);
+            }
+        }
+
+        // ---- online softmax per row (rows g and g+8 of this warp's 16)
+        float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = e >> 1;
+                const int tok = tb + n * 8 + c + (e & 1);
+                if (tok >= Lr[r]) sacc[n][e] = -INFINITY;
+                mx[r] = fmaxf(mx[r], sacc[n][e]);
+            }
+        }
+        float alpha[2], mref[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+            mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+            const float mn = fmaxf(m[r], mx[r]);
+            mref[r] = mn == -INFINITY ? 0.f : mn;  // rows without tokens so far stay at zero
+            alpha[r] = fast_exp2(m[r] - mref[r]);
+            m[r] = mn;
+        }
+        uint32_t pa[NT / 2][4];
+        float rs[2] = {0.f, 0.f};
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            const float p0 = fast_exp2(sacc[n][0] - mref[0]);
+            const float p1 = fast_exp2(sacc[n][1] - mref[0]);
+            const float p2 = fast_exp2(sacc[n][2] - mref[1]);
+            const float p3 = fast_exp2(sacc[n][3] - mref[1]);
+            rs[0] += p0 + p1;
+            rs[1] += p2 + p3;
+            // A operand of P.V for token k-step n/2: a0/a1 from n-tile 2k, a2/a3 from 2k+1
+            pa[n >> 1][(n & 1) * 2 + 0] = pack_half2(p0, p1);
+            pa[n >> 1][(n & 1) * 2 + 1] = pack_half2(p2, p3);
+        }
+#pragma unroll
+        for (int r = 0; r < 2; ++r) l[r] = l[r] * alpha[r] + rs[r];
+#pragma unroll
+        for (int j = 0; j < ON; ++j) {
+            o[j][0] *= alpha[0];
+            o[j][1] *= alpha[0];
+            o[j][2] *= alpha[1];
+            o[j][3] *= alpha[1];
+        }
+
+        // ---- O += P V
+#pragma unroll
+        for (int kt2 = 0; kt2 < NT / 2; ++kt2) {
+#pragma unroll
+            for (int dp = 0; dp < ON / 2; ++dp) {
+                // matrices (transposed): (tokens +0..7, dims +0..7), (+8..15, +0..7), (+0..7, +8..15), (+8..15, +8..15)
+                const int mi = lane >> 3, r = lane & 7;
+                const int tok = kt2 * 16 + ((mi & 1) << 3) + r;
+                const int dim = dp * 16 + ((mi >> 1) << 3);
+                const unsigned char *addr = vt + (dim >> 6) * Lay::kHalfTile + swz128(tok, (dim & 63) * 2);
+                uint32_t b[4];
+                ldmatrix_x4_trans(b, addr);
+                mma_16816(o[2 * dp], pa[kt2], b[0], b[1]);
+                mma_16816(o[2 * dp + 1], pa[kt2], b[2], b[3]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
+    }
+
+    // ---- partials: row sums over the quad, then (lse, o) per sequence
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        l[r] += __shfl_xor_sync(0xffffffffu, l[r], 1);
+        l[r] += __shfl_xor_sync(0xffffffffu, l[r], 2);
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        if (rows[r] >= S) continue;
+        const size_t idx = ((size_t)rows[r] * p.num_heads + h) * p.ws_parts + pp;
+        const bool any = l[r] > 0.f;
+        const float inv = any ? 1.0f / l[r] : 0.f;
+        float *op = p.ws_o + idx * D;
+#pragma unroll
+        for (int j = 0; j < ON; ++j)
+            *reinterpret_cast<float2 *>(op + j * 8 + c) = make_float2(o[j][2 * r] * inv, o[j][2 * r + 1] * inv);
+        if ((lane & 3) == 0) p.ws_lse[idx] = any ? m[r] + fast_log2(l[r]) : -INFINITY;
+    }
+}
+
 }  // namespace pa

@@ -114,6 +114,45 @@ __device__ __forceinline__ uint64_t l2_policy_evict_normal() {
     return p;
 }
 
+// ------------------------------------------------------- tensor cores (mma.sync)
+
+// Four 8x8 b16 matrices from shared memory; lane i gives the address of row
+// i % 8 of matrix i / 8. Lane l receives, of each matrix, the 32-bit word of
+// row l / 4, columns 2 (l % 4) and 2 (l % 4) + 1 (transposed with .trans).
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void *row_addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_u32(row_addr)));
+}
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], const void *row_addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_u32(row_addr)));
+}
+
+// D(16x8, f32) += A(16x16, f16, row) * B(16x8, f16, col).
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                          uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// Byte offset of (row, byte) in a [rows][128 B] tile written by a TMA load
+// with 128-byte swizzle (tile base 1024-byte aligned): the 16-byte chunk
+// index is XORed with row % 8.
+__device__ __forceinline__ uint32_t swz128(int row, int byte) {
+    return (uint32_t)(row * 128 + ((((byte >> 4) ^ row) & 7) << 4) + (byte & 15));
+}
+
 // ----------------------------------------------------------- arithmetic
 
 __device__ __forceinline__ float fast_exp2(float x) {  // ex2.approx: 2^-inf = +0
