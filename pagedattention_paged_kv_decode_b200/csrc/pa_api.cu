@@ -756,11 +756,18 @@ int plan_shared_prefix(const pa_cache_desc &c, int S, int bound, int prefix_bloc
     if (pre->prefix_tokens > bound)
         return fail(PA_ERR_INVALID, "shared prefix (%d tokens) beyond the context bound %d",
                     pre->prefix_tokens, bound);
-    pre->partition = std::max(B, 512 / B * B);
-    pre->parts = (pre->prefix_tokens + pre->partition - 1) / pre->partition;
     pre->heads = 1;
     pre->mma = c.dtype == PA_F16;
     pre->queries = pre->mma ? pa::kPrefixMmaQueries : std::min(S, pa::kMaxConsumerWarps);
+    // prefix partitions of 512 tokens, halved (down to 4 blocks) while the
+    // prefix grid has fewer than two CTAs per SM
+    const int64_t n_qb = (S + pre->queries - 1) / pre->queries;
+    pre->partition = std::max(B, 512 / B * B);
+    while (pre->partition > 4 * B &&
+           (int64_t)c.num_heads * n_qb * ((pre->prefix_tokens + pre->partition - 1) / pre->partition) <
+               2 * kNumSMs)
+        pre->partition /= 2;
+    pre->parts = (pre->prefix_tokens + pre->partition - 1) / pre->partition;
     const size_t sb = pa::SmemLayout(B, 1, c.head_size, elem_bytes(c), 1, 1, 1).stage_bytes;
     pre->stages = (int)std::max<size_t>(2, std::min<size_t>(8, (96 * 1024) / sb));
     pa_decode_config r = cfg ? *cfg : pa_decode_config{0, 0, 0, 0, 0};
