@@ -42,7 +42,14 @@ def build(force: bool = False) -> str:
 def _load():
     global _lib
     if _lib is None:
-        _lib = ctypes.CDLL(build())
+        _lib = _declare(ctypes.CDLL(build()))
+    return _lib
+
+
+def _declare(lib):
+    """Declare the C signatures on a loaded oracle library."""
+    _lib = lib
+    if True:
         P = ctypes.c_void_p
         I = ctypes.c_int
         I64 = ctypes.c_int64
@@ -74,6 +81,25 @@ def _load():
         _lib.oracle_e4m3_array_from_float.restype = None
         _lib.oracle_e4m3_array_from_float.argtypes = [P, P, I64]
     return _lib
+
+
+class using_library:
+    """Context manager: route this module's calls through another build of the
+    oracle's C source (the mutation tests plant mistakes in such builds)."""
+
+    def __init__(self, path: str):
+        self.path = path
+
+    def __enter__(self):
+        global _lib
+        self.saved = _load()
+        _lib = _declare(ctypes.CDLL(self.path))
+        return self
+
+    def __exit__(self, *exc):
+        global _lib
+        _lib = self.saved
+        return False
 
 
 def _ptr(a: np.ndarray | None):

@@ -1,0 +1,233 @@
+"""The oracle's pins must catch plausible mistakes.
+
+Each case below plants one mistake in a copy of oracle/pagedkv_oracle.c (a
+text substitution), builds it, routes the oracle through it and runs the
+pin battery: the worked and growth slot examples, binary16 and E4M3 decoding
+against numpy/torch, E4M3 encoding against torch and the saturation points,
+dense attention on identity tables against torch's SDPA, the closed forms,
+exact-sum brute force, physical-block relabelling, cache-write read-back,
+block copy and swap semantics, and the log-sum-exp identity. Every mutant
+must fail at least one pin; the unmodified source must pass all of them.
+"""
+import math
+import os
+import subprocess
+import tempfile
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "pagedkv_oracle.c")
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+MUTANTS = {
+    "slot offset uses division": ("physical * block_size + pos % block_size", "physical * block_size + pos / block_size"),
+    "slot of position L instead of L-1": ("int pos = L - 1;", "int pos = L;"),
+    "f16 exponent bias": ("v = ldexp((double)(1024 + f), e - 25);", "v = ldexp((double)(1024 + f), e - 24);"),
+    "e4m3 exponent bias": ("v = ldexp((double)(8 + m), e - 10);", "v = ldexp((double)(8 + m), e - 9);"),
+    "e4m3 encode truncates": ("double n = nearbyint(a / quantum);", "double n = floor(a / quantum);"),
+    "e4m3 saturates to NaN": ("        return sign | 0x7e;\n    if (a == 0.0)", "        return sign | 0x7f;\n    if (a == 0.0)"),
+    "softmax scale dropped": ("z[t - t0] = scale * dot;", "z[t - t0] = dot;"),
+    "row offset by block division": ("int64_t base = (((int64_t)blk * block_size + t % block_size) * num_heads + h) * head_size;",
+                                     "int64_t base = (((int64_t)blk * block_size + t / block_size) * num_heads + h) * head_size;"),
+    "logical block by modulo": ("int logical = t / block_size;", "int logical = t % block_size;"),
+    "keys read from the value cache": ("dot += oracle_f16_to_double(q[d]) * cache_value(key_cache, kv_dtype, base + d, k_scale);",
+                                       "dot += oracle_f16_to_double(q[d]) * cache_value(value_cache, kv_dtype, base + d, k_scale);"),
+    "softmax weight sign": ("acc += exp(z[i] - m) * cache_value", "acc += exp(m - z[i]) * cache_value"),
+    "normaliser omitted": ("o[d] = acc / l;", "o[d] = acc;"),
+    "E4M3 V written with k_scale": ("float vq = vf / v_scale;", "float vq = vf / k_scale;"),
+    "copy direction reversed": ("memmove((char *)key_cache + dst * block_bytes,\n                (char *)key_cache + src * block_bytes",
+                                "memmove((char *)key_cache + src * block_bytes,\n                (char *)key_cache + dst * block_bytes"),
+    "swap copies only K": ("memcpy((char *)dst_value + dst * block_bytes", "memcpy((char *)dst_key + dst * block_bytes"),
+    "lse combine weight sign": ("acc += exp(lse[p] - M) * o", "acc += exp(M - lse[p]) * o"),
+    "partial lse without log": ("lse[slot] = m + log(l);", "lse[slot] = m + l;"),
+    "head index ignored": ("const uint16_t *q = query + ((int64_t)s * num_heads + h) * head_size;",
+                           "const uint16_t *q = query + ((int64_t)s * num_heads + 0) * head_size;"),
+}
+
+
+def _build(source: str, path: str):
+    with open(path + ".c", "w") as f:
+        f.write(source)
+    subprocess.check_call(["gcc", "-O1", "-std=c11", "-fno-fast-math", "-ffp-contract=off", "-shared",
+                           "-fPIC", path + ".c", "-o", path, "-lm"])
+
+
+def _rows(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return [ln.split() for ln in f if ln.strip() and not ln.startswith("#")]
+
+
+def _complete(ctx, H=3, D=16, B=8, seed=0, deal="permuted"):
+    ctx = np.asarray(ctx)
+    need = sum(-(-int(L) // B) for L in ctx)
+    w = W.build("m", H, D, B, "f16", ctx, need + 4, max(1, -(-int(ctx.max()) // B)), seed,
+                q_std=1.0, kv_std=1.0, deal_order=deal)
+    kc, vc = w.pool_host()
+    slots = oracle.slot_mapping(w.block_tables, w.context_lens, B)
+    oracle.kv_cache_write(w.new_key, w.new_value, kc, vc, slots)
+    return w, kc, vc
+
+
+def pin_battery():
+    """Returns the names of the pins that fail (each pin is a small check)."""
+    failed = []
+
+    def pin(name, fn):
+        try:
+            ok = fn()
+        except Exception:
+            ok = False
+        if not ok:
+            failed.append(name)
+
+    def worked_example():
+        tables = {"A": [5, 8], "B": [3, -1]}
+        return all(oracle.slot_mapping(np.array([tables[sq]], np.int32), np.array([int(t) + 1], np.int32), 16)[0] == int(sl)
+                   for sq, t, _, _, sl in _rows("slot_mapping_worked_example.txt"))
+
+    def growth_example():
+        bt = np.array([[7, 2, 3, -1]], np.int32)
+        return all(oracle.slot_mapping(bt, np.array([int(ctx)], np.int32), 4)[0] == int(sl)
+                   for _, ctx, _, _, _, sl in _rows("block_growth_example.txt"))
+
+    def f16_decode():
+        bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+        ref = bits.view(np.float16).astype(np.float64)
+        got = oracle.f16_to_double(bits.view(np.float16))
+        fin = np.isfinite(ref)
+        return np.array_equal(got[fin], ref[fin])
+
+    def e4m3_decode():
+        ref = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+        got = oracle.e4m3_to_double(np.arange(256, dtype=np.uint8))
+        fin = ~np.isnan(ref)
+        return np.array_equal(got[fin], ref[fin])
+
+    def e4m3_encode():
+        x = np.random.default_rng(0).standard_normal(20000).astype(np.float32) * 40
+        x = x[np.abs(x) <= 448]
+        ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        sat = oracle.e4m3_from_float(np.float32([449, 1e9, -500]))
+        return np.array_equal(oracle.e4m3_from_float(x), ref) and list(sat) == [0x7E, 0x7E, 0xFE]
+
+    def dense_equivalence():
+        w, kc, vc = _complete([1, 9, 30], H=3, D=16, B=8, deal="identity", seed=1)
+        got = oracle.paged_attention(w.query, kc, vc, w.block_tables, w.context_lens, w.scale)
+        for s in range(3):
+            base = int(w.block_tables[s, 0]) * 8
+            L = int(w.context_lens[s])
+            K = torch.from_numpy(kc.reshape(-1, 3, 16)[base:base + L].astype(np.float64)).permute(1, 0, 2)
+            V = torch.from_numpy(vc.reshape(-1, 3, 16)[base:base + L].astype(np.float64)).permute(1, 0, 2)
+            q = torch.from_numpy(w.query[s].astype(np.float64))[:, None, :]
+            ref = torch.nn.functional.scaled_dot_product_attention(q, K, V, scale=w.scale)[:, 0, :].numpy()
+            if np.abs(got[s] - ref).max() > 1e-12:
+                return False
+        return True
+
+    def context_one():
+        w, kc, vc = _complete([1, 1], seed=3)
+        got = oracle.paged_attention(w.query, kc, vc, w.block_tables, w.context_lens, w.scale)
+        return np.array_equal(got, w.new_value.astype(np.float64))
+
+    def brute_force():
+        rng = np.random.default_rng(5)
+        H, D, B, ctx = 2, 3, 2, np.array([5, 3])
+        nb = 8
+        kc = rng.standard_normal((nb, B, H, D)).astype(np.float16)
+        vc = rng.standard_normal((nb, B, H, D)).astype(np.float16)
+        q = rng.standard_normal((2, H, D)).astype(np.float16)
+        bt = np.array([[6, 1, 4], [0, 7, -1]], np.int32)
+        sc = float(np.float32(0.7))   # the scale crosses the boundary as fp32
+        got = oracle.paged_attention(q, kc, vc, bt, ctx, sc)
+        for s, L in enumerate(ctx):
+            for h in range(H):
+                rows = [(int(bt[s][t // B]), t % B) for t in range(int(L))]
+                z = [sc * math.fsum(float(q[s, h, d]) * float(kc[b, r, h, d]) for d in range(D)) for b, r in rows]
+                p = [math.exp(x) for x in z]
+                for d in range(D):
+                    ref = math.fsum(p[i] * float(vc[b, r, h, d]) for i, (b, r) in enumerate(rows)) / math.fsum(p)
+                    if abs(got[s, h, d] - ref) > 1e-12:
+                        return False
+        return True
+
+    def relabelling():
+        w, kc, vc = _complete([5, 17, 33], seed=2)
+        base = oracle.paged_attention(w.query, kc, vc, w.block_tables, w.context_lens, w.scale)
+        perm = np.random.default_rng(9).permutation(w.num_blocks).astype(np.int32)
+        kc2, vc2 = np.empty_like(kc), np.empty_like(vc)
+        kc2[perm], vc2[perm] = kc, vc
+        bt2 = np.where(w.block_tables >= 0, perm[np.maximum(w.block_tables, 0)], -1).astype(np.int32)
+        return np.array_equal(base, oracle.paged_attention(w.query, kc2, vc2, bt2, w.context_lens, w.scale))
+
+    def cache_write_readback():
+        kc = np.zeros((4, 4, 2, 8), np.float16)
+        vc = np.zeros_like(kc)
+        key = np.random.default_rng(1).standard_normal((2, 2, 8)).astype(np.float16)
+        oracle.kv_cache_write(key, key + 1, kc, vc, np.array([6, 13], np.int32))
+        ek = np.zeros((4, 4, 2, 8), np.uint8)
+        ev = np.zeros_like(ek)
+        oracle.kv_cache_write(key, key, ek, ev, np.array([6, 13], np.int32), 0.5, 2.0)
+        return (np.array_equal(kc[1, 2], key[0]) and np.array_equal(vc[3, 1], key[1] + 1)
+                and np.array_equal(ev[1, 2], oracle.e4m3_from_float(key[0].astype(np.float32) / np.float32(2.0))))
+
+    def copy_semantics():
+        kc = np.random.default_rng(2).standard_normal((4, 2, 1, 8)).astype(np.float16)
+        vc = kc + 1
+        k0 = kc.copy()
+        oracle.copy_blocks(kc, vc, np.array([[1, 3]], np.int32))
+        return np.array_equal(kc[3], k0[1]) and np.array_equal(kc[1], k0[1]) and np.array_equal(vc[3], k0[1] + 1)
+
+    def swap_semantics():
+        src = np.random.default_rng(3).standard_normal((3, 2, 1, 8)).astype(np.float16)
+        dk, dv = np.zeros_like(src), np.zeros_like(src)
+        oracle.swap_blocks(dk, dv, src, src + 1, np.array([[2, 0]], np.int32))
+        return np.array_equal(dk[0], src[2]) and np.array_equal(dv[0], src[2] + 1)
+
+    def lse_identity():
+        w, kc, vc = _complete([15, 40], seed=14)
+        full = oracle.paged_attention(w.query, kc, vc, w.block_tables, w.context_lens, w.scale)
+        o, lse = oracle.attention_partials(w.query, kc, vc, w.block_tables, w.context_lens, w.scale, 16)
+        for s, L in enumerate(w.context_lens):
+            n = -(-int(L) // 16)
+            for h in range(w.num_heads):
+                if np.abs(oracle.lse_combine(o[s, h, :n], lse[s, h, :n]) - full[s, h]).max() > 1e-12:
+                    return False
+        return True
+
+    for name, fn in [("worked example", worked_example), ("growth example", growth_example),
+                     ("f16 decode", f16_decode), ("e4m3 decode", e4m3_decode), ("e4m3 encode", e4m3_encode),
+                     ("dense equivalence", dense_equivalence), ("context one", context_one),
+                     ("brute force", brute_force), ("relabelling", relabelling),
+                     ("cache write", cache_write_readback), ("copy", copy_semantics), ("swap", swap_semantics),
+                     ("lse identity", lse_identity)]:
+        pin(name, fn)
+    return failed
+
+
+@pytest.fixture(scope="module")
+def source():
+    with open(SRC) as f:
+        return f.read()
+
+
+def test_unmodified_source_passes_every_pin(source, tmp_path):
+    path = str(tmp_path / "liborig.so")
+    _build(source, path)
+    with oracle.using_library(path):
+        assert pin_battery() == []
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_fails_a_pin(source, tmp_path, name):
+    old, new = MUTANTS[name]
+    assert source.count(old) == 1, f"mutation anchor not unique: {name}"
+    path = str(tmp_path / "libmutant.so")
+    _build(source.replace(old, new), path)
+    with oracle.using_library(path):
+        failed = pin_battery()
+    assert failed, f"no pin caught: {name}"
