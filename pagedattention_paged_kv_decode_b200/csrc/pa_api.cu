@@ -174,9 +174,8 @@ int fill_config(const pa_cache_desc &c, int num_seqs, int max_ctx, pa_decode_con
     const int C0 = r.units_per_cta;
     // stages must be a multiple of warps_per_head (see the check below).
     if (r.warps_per_head == 0) {
-        // one head per CTA: 2 warps (the ring then holds more stages); 2 heads:
-        // 2 warps each; 4 or more heads: 1 warp each
-        int W = C0 > 1 ? 2 : (G0 >= 4 ? 1 : 2);
+        // one head per CTA: 4 warps; 2 heads: 2 warps each; 4 or more: 1 each
+        int W = C0 > 1 ? 2 : (G0 >= 4 ? 1 : (G0 == 2 ? 2 : 4));
         while (W > 1 && (r.stages != 0 && r.stages % W)) W >>= 1;
         while (W > 1 && C0 * G0 * W > pa::kMaxConsumerWarps) W >>= 1;
         r.warps_per_head = W;
