@@ -72,6 +72,10 @@ def _declare(lib):
         _lib.oracle_paged_attention.argtypes = [P, P, P, P, I, I, I, I, I, P, I, P, I, F, F, F, P, I]
         _lib.oracle_attention_partials.restype = I
         _lib.oracle_attention_partials.argtypes = [P, P, P, P, P, I, I, I, I, I, P, I, P, I, F, F, F, I, I]
+        _lib.oracle_prefill_slot_mapping.restype = I
+        _lib.oracle_prefill_slot_mapping.argtypes = [P, P, P, I, P, I, I]
+        _lib.oracle_paged_prefill.restype = I
+        _lib.oracle_paged_prefill.argtypes = [P, P, P, P, P, I, I, I, I, I, P, I, P, I, F, F, F, P, I]
         _lib.oracle_lse_combine.restype = None
         _lib.oracle_lse_combine.argtypes = [P, P, P, I, I]
         _lib.oracle_f16_array_to_double.restype = None
@@ -156,6 +160,18 @@ def slot_mapping(block_tables: np.ndarray, context_lens: np.ndarray, block_size:
     return out
 
 
+def prefill_slot_mapping(query_start: np.ndarray, block_tables: np.ndarray,
+                         context_lens: np.ndarray, block_size: int) -> np.ndarray:
+    """One slot per new token of a prefill chunk ([total_q] int32)."""
+    qs = np.ascontiguousarray(query_start, dtype=np.int32)
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    ctx = np.ascontiguousarray(context_lens, dtype=np.int32)
+    out = np.full(int(qs[-1]), -1, np.int32)
+    _check(_load().oracle_prefill_slot_mapping(_ptr(out), _ptr(qs), _ptr(bt), bt.shape[1], _ptr(ctx),
+                                               ctx.shape[0], block_size), "prefill_slot_mapping")
+    return out
+
+
 def kv_cache_write(key: np.ndarray, value: np.ndarray, key_cache: np.ndarray,
                    value_cache: np.ndarray, slot_mapping: np.ndarray,
                    k_scale: float = 1.0, v_scale: float = 1.0) -> None:
@@ -214,6 +230,32 @@ def paged_attention(query: np.ndarray, key_cache: np.ndarray, value_cache: np.nd
         _ptr(pairs), 0 if pairs is None else pairs.shape[0])
     _check(rc, "paged_attention")
     return out.reshape(S, nh, hd) if pairs is None else out
+
+
+def paged_prefill(query: np.ndarray, query_start: np.ndarray, key_cache: np.ndarray,
+                  value_cache: np.ndarray, block_tables: np.ndarray, context_lens: np.ndarray,
+                  scale: float, k_scale: float = 1.0, v_scale: float = 1.0,
+                  row_head: np.ndarray | None = None) -> np.ndarray:
+    """Causal attention of packed query rows: float64 [total_q, H, D], or [n, D]
+    for an explicit (row, head) list."""
+    assert query.dtype == np.float16
+    q = np.ascontiguousarray(query)
+    nb, bs, nh, hd = key_cache.shape
+    qs = np.ascontiguousarray(query_start, dtype=np.int32)
+    S = qs.shape[0] - 1
+    assert q.shape[0] == int(qs[-1])
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    ctx = np.ascontiguousarray(context_lens, dtype=np.int32)
+    pairs = None if row_head is None else np.ascontiguousarray(row_head, dtype=np.int32).reshape(-1, 2)
+    n = q.shape[0] * nh if pairs is None else pairs.shape[0]
+    out = np.empty((n, hd), np.float64)
+    rc = _load().oracle_paged_prefill(
+        _ptr(out), _ptr(q.view(np.uint16)), _ptr(qs), _ptr(key_cache), _ptr(value_cache),
+        _dtype_code(key_cache), nb, bs, nh, hd, _ptr(bt), bt.shape[1], _ptr(ctx), S,
+        float(np.float32(scale)), float(np.float32(k_scale)), float(np.float32(v_scale)),
+        _ptr(pairs), 0 if pairs is None else pairs.shape[0])
+    _check(rc, "paged_prefill")
+    return out.reshape(q.shape[0], nh, hd) if pairs is None else out
 
 
 def attention_partials(query, key_cache, value_cache, block_tables, context_lens, scale,

@@ -144,6 +144,36 @@ int oracle_slot_mapping(int32_t *slot_mapping, const int32_t *block_tables,
     return 0;
 }
 
+/* Slots of a prefill chunk. Sequence s brings n_s = query_start[s+1] -
+ * query_start[s] new tokens, the last n_s positions of its context of
+ * L_s = context_lens[s] tokens: token query_start[s] + i sits at position
+ * L_s - n_s + i and gets slot block_tables[s][pos / block_size] * block_size
+ * + pos % block_size, the same rule as above. A full prompt (n_s = L_s)
+ * maps positions 0 .. L_s - 1; a decode step (n_s = 1) maps position L_s - 1.
+ * Returns 0, or -1 if n_s < 0, n_s > L_s, or a table read would fall
+ * outside the table row. */
+int oracle_prefill_slot_mapping(int32_t *slot_mapping, const int32_t *query_start,
+                                const int32_t *block_tables, int max_blocks_per_seq,
+                                const int32_t *context_lens, int num_seqs,
+                                int block_size)
+{
+    for (int s = 0; s < num_seqs; ++s) {
+        int n = query_start[s + 1] - query_start[s];
+        int L = context_lens[s];
+        if (n < 0 || n > L)
+            return -1;
+        for (int i = 0; i < n; ++i) {
+            int pos = L - n + i;
+            int logical = pos / block_size;
+            if (logical >= max_blocks_per_seq)
+                return -1;
+            int physical = block_tables[(int64_t)s * max_blocks_per_seq + logical];
+            slot_mapping[query_start[s] + i] = physical * block_size + pos % block_size;
+        }
+    }
+    return 0;
+}
+
 /* ----------------------------------------------------- cache write (a2) */
 
 /* Store token i's key and value rows (all heads) into the cache slot given
@@ -241,7 +271,8 @@ static double cache_value(const void *cache, int kv_dtype, int64_t idx, double s
     return oracle_e4m3_to_double(((const uint8_t *)cache)[idx]) * scale;
 }
 
-/* Attention of one query row over the tokens [t0, t1) of sequence s, head h,
+/* Attention of the query row q (head_size fp16 values) over the tokens
+ * [t0, t1) of sequence s, head h,
  * walked through the block table ([P1] §2.2, [P2] §2.1): token t lives in
  * physical block block_tables[s][t / block_size] at row t % block_size.
  *   z_t = scale * sum_d q[d] * K_t[d]
@@ -251,7 +282,7 @@ static double cache_value(const void *cache, int kv_dtype, int64_t idx, double s
  * Writes o (head_size doubles), *m_out, *l_out. Returns -1 on a table entry
  * outside [0, num_blocks) or a position beyond the table row. */
 static int attend_range(double *o, double *m_out, double *l_out,
-                        const uint16_t *query, const void *key_cache,
+                        const uint16_t *q, const void *key_cache,
                         const void *value_cache, int kv_dtype, int num_blocks,
                         int block_size, int num_heads, int head_size,
                         const int32_t *block_tables, int max_blocks_per_seq,
@@ -266,7 +297,6 @@ static int attend_range(double *o, double *m_out, double *l_out,
         free(rowbase);
         return -2;
     }
-    const uint16_t *q = query + ((int64_t)s * num_heads + h) * head_size;
     for (int t = t0; t < t1; ++t) {
         int logical = t / block_size;
         if (logical >= max_blocks_per_seq) {
@@ -333,11 +363,65 @@ int oracle_paged_attention(double *out, const uint16_t *query,
                 o[d] = 0.0;
             continue;
         }
+        const uint16_t *q = query + ((int64_t)s * num_heads + h) * head_size;
         double m, l;
-        int rc = attend_range(o, &m, &l, query, key_cache, value_cache, kv_dtype,
+        int rc = attend_range(o, &m, &l, q, key_cache, value_cache, kv_dtype,
                               num_blocks, block_size, num_heads, head_size,
                               block_tables, max_blocks_per_seq, s, h, 0, L,
                               (double)scale, (double)k_scale, (double)v_scale);
+        if (rc)
+            return rc;
+    }
+    return 0;
+}
+
+/* --------------------------------------------------------- paged prefill */
+
+/* Causal multi-query attention over the block table: the prompt (or a chunk
+ * of it) attends its own and all earlier tokens ([P1] §3.2 puts
+ * FlashAttention-style attention on this path; [P3] §4 runs long texts with
+ * block_size 32). Query rows are packed [total_q][num_heads][head_size], the
+ * rows of sequence s being query_start[s] .. query_start[s+1] - 1. With
+ * n_s rows and context length L_s (the cache already holds all L_s tokens),
+ * row query_start[s] + i sits at position L_s - n_s + i and attends the
+ * tokens 0 .. L_s - n_s + i of its sequence, with the same softmax as the
+ * decode above. Computes the (row, head) pairs of row_head ([n_pairs][2]),
+ * or every row x head in (row, head) order when row_head is NULL; out holds
+ * one head_size row of doubles per pair. Returns 0, or -1 on n_s < 0,
+ * n_s > L_s, a pair out of range or a bad table entry. */
+int oracle_paged_prefill(double *out, const uint16_t *query, const int32_t *query_start,
+                         const void *key_cache, const void *value_cache,
+                         int kv_dtype, int num_blocks, int block_size,
+                         int num_heads, int head_size,
+                         const int32_t *block_tables, int max_blocks_per_seq,
+                         const int32_t *context_lens, int num_seqs,
+                         float scale, float k_scale, float v_scale,
+                         const int32_t *row_head, int n_pairs)
+{
+    int total_q = query_start[num_seqs];
+    for (int s = 0; s < num_seqs; ++s) {
+        int n = query_start[s + 1] - query_start[s];
+        if (n < 0 || n > context_lens[s])
+            return -1;
+    }
+    int total = row_head ? n_pairs : total_q * num_heads;
+    for (int i = 0; i < total; ++i) {
+        int row = row_head ? row_head[2 * i] : i / num_heads;
+        int h = row_head ? row_head[2 * i + 1] : i % num_heads;
+        if (row < 0 || row >= total_q || h < 0 || h >= num_heads)
+            return -1;
+        int s = 0;
+        while (query_start[s + 1] <= row)
+            ++s;
+        int n = query_start[s + 1] - query_start[s];
+        int pos = context_lens[s] - n + (row - query_start[s]);
+        const uint16_t *q = query + ((int64_t)row * num_heads + h) * head_size;
+        double m, l;
+        int rc = attend_range(out + (int64_t)i * head_size, &m, &l, q, key_cache,
+                              value_cache, kv_dtype, num_blocks, block_size,
+                              num_heads, head_size, block_tables,
+                              max_blocks_per_seq, s, h, 0, pos + 1, (double)scale,
+                              (double)k_scale, (double)v_scale);
         if (rc)
             return rc;
     }
@@ -378,7 +462,9 @@ int oracle_attention_partials(double *o, double *lse, const uint16_t *query,
                 int t0 = p * partition_size;
                 int t1 = t0 + partition_size < L ? t0 + partition_size : L;
                 double m, l;
-                int rc = attend_range(op, &m, &l, query, key_cache, value_cache,
+                int rc = attend_range(op, &m, &l,
+                                      query + ((int64_t)s * num_heads + h) * head_size,
+                                      key_cache, value_cache,
                                       kv_dtype, num_blocks, block_size, num_heads,
                                       head_size, block_tables, max_blocks_per_seq,
                                       s, h, t0, t1, (double)scale,

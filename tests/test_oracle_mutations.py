@@ -6,7 +6,10 @@ pin battery: the worked and growth slot examples, binary16 and E4M3 decoding
 against numpy/torch, E4M3 encoding against torch and the saturation points,
 dense attention on identity tables against torch's SDPA, the closed forms,
 exact-sum brute force, physical-block relabelling, cache-write read-back,
-block copy and swap semantics, and the log-sum-exp identity. Every mutant
+block copy and swap semantics, the log-sum-exp identity, and for the
+prefill the worked example as a full prompt, one-token chunks against the
+decode slots, and chunks after a cached context against torch's SDPA with a
+position mask. Every mutant
 must fail at least one pin; the unmodified source must pass all of them.
 """
 import math
@@ -25,7 +28,10 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "pagedkv_oracle.c")
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
 MUTANTS = {
-    "slot offset uses division": ("physical * block_size + pos % block_size", "physical * block_size + pos / block_size"),
+    "slot offset uses division": ("slot_mapping[s] = physical * block_size + pos % block_size;",
+                                  "slot_mapping[s] = physical * block_size + pos / block_size;"),
+    "prefill slot offset uses division": ("slot_mapping[query_start[s] + i] = physical * block_size + pos % block_size;",
+                                          "slot_mapping[query_start[s] + i] = physical * block_size + pos / block_size;"),
     "slot of position L instead of L-1": ("int pos = L - 1;", "int pos = L;"),
     "f16 exponent bias": ("v = ldexp((double)(1024 + f), e - 25);", "v = ldexp((double)(1024 + f), e - 24);"),
     "e4m3 exponent bias": ("v = ldexp((double)(8 + m), e - 10);", "v = ldexp((double)(8 + m), e - 9);"),
@@ -45,6 +51,13 @@ MUTANTS = {
     "swap copies only K": ("memcpy((char *)dst_value + dst * block_bytes", "memcpy((char *)dst_key + dst * block_bytes"),
     "lse combine weight sign": ("acc += exp(lse[p] - M) * o", "acc += exp(M - lse[p]) * o"),
     "partial lse without log": ("lse[slot] = m + log(l);", "lse[slot] = m + l;"),
+    "prefill slot position from the chunk start": ("int pos = L - n + i;", "int pos = i;"),
+    "prefill row misses its own token": ("s, h, 0, pos + 1, (double)scale,", "s, h, 0, pos, (double)scale,"),
+    "prefill row sees one token ahead": ("s, h, 0, pos + 1, (double)scale,", "s, h, 0, pos + 2, (double)scale,"),
+    "prefill position ignores the cached context": ("int pos = context_lens[s] - n + (row - query_start[s]);",
+                                                    "int pos = row - query_start[s];"),
+    "prefill query row taken by sequence": ("const uint16_t *q = query + ((int64_t)row * num_heads + h) * head_size;",
+                                            "const uint16_t *q = query + ((int64_t)s * num_heads + h) * head_size;"),
     "head index ignored": ("const uint16_t *q = query + ((int64_t)s * num_heads + h) * head_size;",
                            "const uint16_t *q = query + ((int64_t)s * num_heads + 0) * head_size;"),
 }
@@ -199,12 +212,45 @@ def pin_battery():
                     return False
         return True
 
+    def prefill_worked_example():
+        got = oracle.prefill_slot_mapping(np.array([0, 32, 48], np.int32), np.array([[5, 8], [3, -1]], np.int32),
+                                          np.array([32, 16], np.int32), 16)
+        want = [int(sl) for sq, t, _, _, sl in _rows("slot_mapping_worked_example.txt")]
+        return [int(x) for x in got] == want
+
+    def prefill_one_token_chunks():
+        w = W.build("d", 2, 8, 4, "f16", np.array([1, 4, 5, 13]), 30, 4, 3, 1.0, 1.0)
+        got = oracle.prefill_slot_mapping(np.arange(5, dtype=np.int32), w.block_tables, w.context_lens, 4)
+        return np.array_equal(got, oracle.slot_mapping(w.block_tables, w.context_lens, 4))
+
+    def prefill_dense_causal():
+        ctx, n = [12, 9, 17], [5, 9, 1]
+        need = sum(-(-L // 8) for L in ctx)
+        w = W.build_prefill("p", 2, 16, 8, ctx, n, need + 2, 3, 2, 1.0, 1.0, deal_order="identity")
+        kc, vc = w.pool_host()
+        oracle.kv_cache_write(w.new_key, w.new_value, kc, vc,
+                              oracle.prefill_slot_mapping(w.query_start, w.block_tables, w.context_lens, 8))
+        got = oracle.paged_prefill(w.query, w.query_start, kc, vc, w.block_tables, w.context_lens, w.scale)
+        for s in range(3):
+            r0, r1, L = int(w.query_start[s]), int(w.query_start[s + 1]), ctx[s]
+            base = int(w.block_tables[s, 0]) * 8
+            K = torch.from_numpy(kc.reshape(-1, 2, 16)[base:base + L].astype(np.float64)).permute(1, 0, 2)
+            V = torch.from_numpy(vc.reshape(-1, 2, 16)[base:base + L].astype(np.float64)).permute(1, 0, 2)
+            q = torch.from_numpy(w.query[r0:r1].astype(np.float64)).permute(1, 0, 2)
+            mask = torch.from_numpy(np.arange(L)[None, :] <= np.arange(L - n[s], L)[:, None])
+            ref = torch.nn.functional.scaled_dot_product_attention(q, K, V, attn_mask=mask, scale=w.scale)
+            if not np.abs(got[r0:r1] - ref.permute(1, 0, 2).numpy()).max() <= 1e-12:
+                return False
+        return True
+
     for name, fn in [("worked example", worked_example), ("growth example", growth_example),
                      ("f16 decode", f16_decode), ("e4m3 decode", e4m3_decode), ("e4m3 encode", e4m3_encode),
                      ("dense equivalence", dense_equivalence), ("context one", context_one),
                      ("brute force", brute_force), ("relabelling", relabelling),
                      ("cache write", cache_write_readback), ("copy", copy_semantics), ("swap", swap_semantics),
-                     ("lse identity", lse_identity)]:
+                     ("lse identity", lse_identity), ("prefill worked example", prefill_worked_example),
+                     ("prefill one-token chunks", prefill_one_token_chunks),
+                     ("prefill dense causal", prefill_dense_causal)]:
         pin(name, fn)
     return failed
 

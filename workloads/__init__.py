@@ -32,8 +32,39 @@ POISON_HUGE = "huge"   # +/-60000 in an alternating pattern (finite, dominates a
 POISON_NAN = "nan"     # fp16 NaN: any arithmetic use of an unused slot shows up as NaN
 
 
+class _Pools:
+    """Pool construction shared by the decode and prefill workloads (needs
+    num_blocks, block_size, num_heads, head_size, poison, live_*)."""
+
+    def pool_host(self) -> tuple[np.ndarray, np.ndarray]:
+        """The fp16 pools [NB, B, H, D] before the step (E4M3: the source to encode)."""
+        shape = (self.num_blocks, self.block_size, self.num_heads, self.head_size)
+        pk = _poison_fill(shape, self.poison)
+        pv = _poison_fill(shape, self.poison)
+        pk[self.live_blocks, self.live_offsets] = self.live_key
+        pv[self.live_blocks, self.live_offsets] = self.live_value
+        return pk, pv
+
+    def pool_device(self, device) -> tuple:
+        """The same pools as torch fp16 tensors on ``device`` (filled there)."""
+        import torch
+        shape = (self.num_blocks, self.block_size, self.num_heads, self.head_size)
+        out = []
+        for live in (self.live_key, self.live_value):
+            pool = torch.empty(shape, dtype=torch.float16, device=device)
+            if self.poison == POISON_NAN:
+                pool.fill_(float("nan"))
+            else:
+                pool.view(torch.int32).fill_(_HUGE_PAIR_I32)
+            blk = torch.from_numpy(self.live_blocks.astype(np.int64)).to(device)
+            off = torch.from_numpy(self.live_offsets.astype(np.int64)).to(device)
+            pool[blk, off] = torch.from_numpy(live).to(device)
+            out.append(pool)
+        return out[0], out[1]
+
+
 @dataclass
-class Workload:
+class Workload(_Pools):
     name: str
     num_seqs: int
     num_heads: int
@@ -70,32 +101,6 @@ class Workload:
     @property
     def elem_bytes(self) -> int:
         return 2 if self.kv_dtype == "f16" else 1
-
-    def pool_host(self) -> tuple[np.ndarray, np.ndarray]:
-        """The fp16 pools [NB, B, H, D] before the step (E4M3: the source to encode)."""
-        shape = (self.num_blocks, self.block_size, self.num_heads, self.head_size)
-        pk = _poison_fill(shape, self.poison)
-        pv = _poison_fill(shape, self.poison)
-        pk[self.live_blocks, self.live_offsets] = self.live_key
-        pv[self.live_blocks, self.live_offsets] = self.live_value
-        return pk, pv
-
-    def pool_device(self, device) -> tuple:
-        """The same pools as torch fp16 tensors on ``device`` (filled there)."""
-        import torch
-        shape = (self.num_blocks, self.block_size, self.num_heads, self.head_size)
-        out = []
-        for live in (self.live_key, self.live_value):
-            pool = torch.empty(shape, dtype=torch.float16, device=device)
-            if self.poison == POISON_NAN:
-                pool.fill_(float("nan"))
-            else:
-                pool.view(torch.int32).fill_(_HUGE_PAIR_I32)
-            blk = torch.from_numpy(self.live_blocks.astype(np.int64)).to(device)
-            off = torch.from_numpy(self.live_offsets.astype(np.int64)).to(device)
-            pool[blk, off] = torch.from_numpy(live).to(device)
-            out.append(pool)
-        return out[0], out[1]
 
     def kv_bytes(self) -> int:
         """Logical K+V bytes the decode reads: sum_s L_s * H * D * elem * 2."""
@@ -138,7 +143,7 @@ def _normal_table() -> np.ndarray:
     return _QUANTILES["t"]
 
 
-def _draw_f16(rng: np.random.Generator, shape, std: float, chunk: int = 1 << 25) -> np.ndarray:
+def _draw_f16(rng: np.random.Generator, shape, std: float, chunk: int = 1 << 22) -> np.ndarray:
     """float16 samples of N(0, std^2) by inverse-CDF sampling at 16-bit resolution.
 
     Each value is the N(0,1) quantile at a uniformly drawn 16-bit level, times
@@ -340,3 +345,181 @@ def to_device(w: Workload, device, encode=None) -> DeviceWorkload:
         cow_pairs=up(w.cow_pairs.astype(np.int32)), key_cache=kc, value_cache=vc,
         out=torch.empty((S, H, D), dtype=torch.float16, device=device),
         slots=torch.empty(S, dtype=torch.int32, device=device))
+
+
+# ------------------------------------------------------------ paged prefill
+
+@dataclass
+class PrefillWorkload(_Pools):
+    """One prefill step: sequence s brings n_s new tokens (the last n_s
+    positions of its L_s-token context); tokens 0 .. L_s - n_s - 1 are already
+    in the pool, the chunk's own positions hold poison until its cache write."""
+    name: str
+    num_seqs: int
+    num_heads: int
+    head_size: int
+    block_size: int
+    num_blocks: int
+    scale: float
+    query: np.ndarray              # float16 [total_q, H, D], rows of sequence s at query_start[s] ..
+    new_key: np.ndarray            # float16 [total_q, H, D], the chunk's K rows (same order)
+    new_value: np.ndarray
+    query_start: np.ndarray        # int32 [S + 1], query_start[0] = 0
+    block_tables: np.ndarray       # int32 [S, W], -1 beyond each sequence's blocks
+    context_lens: np.ndarray       # int32 [S], L_s including the chunk
+    live_blocks: np.ndarray
+    live_offsets: np.ndarray
+    live_key: np.ndarray
+    live_value: np.ndarray
+    poison: str = POISON_HUGE
+    seed: int = 0
+    kv_dtype: str = "f16"
+    k_scale: float = 1.0
+    v_scale: float = 1.0
+
+    @property
+    def total_q(self) -> int:
+        return int(self.query_start[-1])
+
+    @property
+    def chunk_lens(self) -> np.ndarray:
+        return np.diff(self.query_start).astype(np.int64)
+
+    @property
+    def max_blocks_per_seq(self) -> int:
+        return int(self.block_tables.shape[1])
+
+    def positions(self) -> np.ndarray:
+        """Position of every query row in its sequence ([total_q] int64)."""
+        n = self.chunk_lens
+        start = self.context_lens.astype(np.int64) - n
+        return np.concatenate([start[s] + np.arange(n[s]) for s in range(self.num_seqs)]) \
+            if self.total_q else np.zeros(0, np.int64)
+
+    def flops(self) -> int:
+        """Algorithmic FLOPs of the attention: each (row, head) at position p
+        does (p + 1) * D multiply-adds for Q.K and as many for P.V."""
+        return 4 * self.num_heads * self.head_size * int((self.positions() + 1).sum())
+
+    def io_bytes(self) -> int:
+        """Bytes the attention must move at least once: every context token's K
+        and V (all heads), the queries and the outputs."""
+        H, D = self.num_heads, self.head_size
+        return int(self.context_lens.astype(np.int64).sum()) * H * D * 2 * 2 + self.total_q * H * D * 2 * 2
+
+
+def build_prefill(name: str, num_heads: int, head_size: int, block_size: int, context_lens,
+                  chunk_lens, num_blocks: int, table_width: int, seed: int, q_std: float,
+                  kv_std: float, poison: str = POISON_HUGE,
+                  rng: np.random.Generator | None = None,
+                  deal_order: str = "permuted") -> PrefillWorkload:
+    """Assemble a prefill step from explicit context and chunk lengths
+    (chunk_lens[s] <= context_lens[s]); blocks are dealt as in ``build``."""
+    rng = rng if rng is not None else np.random.Generator(np.random.PCG64(seed))
+    ctx = np.asarray(context_lens, dtype=np.int32)
+    n = np.asarray(chunk_lens, dtype=np.int32)
+    assert ctx.shape == n.shape and (n >= 0).all() and (n <= ctx).all()
+    S, H, D, B = len(ctx), num_heads, head_size, block_size
+    need = [-(-int(L) // B) for L in ctx]
+    assert sum(need) <= num_blocks, f"pool of {num_blocks} blocks is too small for {sum(need)}"
+    assert max(need, default=0) <= table_width
+    order = rng.permutation(num_blocks).astype(np.int32) if deal_order == "permuted" \
+        else np.arange(num_blocks, dtype=np.int32)
+    tables = np.full((S, table_width), -1, np.int32)
+    cursor = 0
+    for s in range(S):
+        tables[s, :need[s]] = order[cursor:cursor + need[s]]
+        cursor += need[s]
+    blk_list, off_list = [], []
+    for s in range(S):
+        pos = np.arange(0, int(ctx[s]) - int(n[s]))
+        if pos.size:
+            blk_list.append(tables[s, pos // B])
+            off_list.append(pos % B)
+    blk = np.concatenate(blk_list) if blk_list else np.zeros(0, np.int32)
+    off = np.concatenate(off_list) if off_list else np.zeros(0, np.int32)
+    qs = np.zeros(S + 1, np.int32)
+    qs[1:] = np.cumsum(n)
+    T = int(qs[-1])
+    query = _draw_f16(rng, (T, H, D), q_std)
+    new_key = _draw_f16(rng, (T, H, D), kv_std)
+    new_value = _draw_f16(rng, (T, H, D), kv_std)
+    live_k = _draw_f16(rng, (blk.size, H, D), kv_std)
+    live_v = _draw_f16(rng, (blk.size, H, D), kv_std)
+    scale = float(np.float32(1.0) / np.sqrt(np.float32(D)))
+    return PrefillWorkload(name=name, num_seqs=S, num_heads=H, head_size=D, block_size=B,
+                           num_blocks=num_blocks, scale=scale, query=query, new_key=new_key,
+                           new_value=new_value, query_start=qs, block_tables=tables,
+                           context_lens=ctx, live_blocks=blk.astype(np.int32),
+                           live_offsets=off.astype(np.int32), live_key=live_k, live_value=live_v,
+                           poison=poison, seed=seed)
+
+
+PREFILL_NAMES = {
+    1: "prefill_tiny_s4_h4_d128_b32_f16",
+    2: "llama13b_prefill_long_s4_h40_d128_b32_f16",
+    3: "llama7b_chunked_prefill_s8_h32_d128_b16_f16",
+}
+
+
+def prefill_named(config_id: int, seed: int | None = None, poison: str = POISON_HUGE) -> PrefillWorkload:
+    """The prefill workloads (seed defaults to 2000 + config_id):
+
+    1. tiny, for the oracle: 4 sequences (a full 37-token prompt, a 100-token
+       chunk after 200 cached tokens, a single token after 128, a full
+       1-token prompt), 4 heads, head_size 128, 32-token blocks;
+    2. long prompts, the long-text setting of the Llama2-13B comparison: 4
+       full prompts of uniform[2048, 8192] tokens, 40 heads, head_size 128,
+       32-token blocks (the size the pages advise above 4k tokens);
+    3. chunked prefill, LLaMA-7B shapes: 8 sequences each bringing a
+       512-token chunk after uniform[0, 2048] cached tokens, 32 heads,
+       head_size 128, 16-token blocks.
+    K/V are N(0, 0.5^2), queries N(0, 1), blocks dealt from a random permutation.
+    """
+    seed = 2000 + config_id if seed is None else seed
+    rng = np.random.Generator(np.random.PCG64(seed))
+    name = PREFILL_NAMES[config_id]
+    if config_id == 1:
+        ctx, n = [37, 300, 129, 1], [37, 100, 1, 1]
+        return build_prefill(name, 4, 128, 32, ctx, n, 24, 12, seed, 1.0, 0.5, poison, rng=rng)
+    if config_id == 2:
+        ctx = rng.integers(2048, 8193, 4)
+        need = sum(-(-int(L) // 32) for L in ctx)
+        return build_prefill(name, 40, 128, 32, ctx, ctx, need + 64, 256, seed, 1.0, 0.5, poison, rng=rng)
+    if config_id == 3:
+        ctx = 512 + rng.integers(0, 2049, 8)
+        need = sum(-(-int(L) // 16) for L in ctx)
+        return build_prefill(name, 32, 128, 16, ctx, np.full(8, 512), need + 64, 160, seed, 1.0, 0.5,
+                             poison, rng=rng)
+    raise KeyError(config_id)
+
+
+@dataclass
+class DevicePrefill:
+    """A prefill workload's tensors on a CUDA device (torch)."""
+    w: PrefillWorkload
+    query: object
+    new_key: object
+    new_value: object
+    query_start: object
+    block_tables: object
+    context_lens: object
+    key_cache: object
+    value_cache: object
+    out: object
+    slots: object
+
+
+def prefill_to_device(w: PrefillWorkload, device) -> DevicePrefill:
+    import torch
+
+    def up(a):
+        return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+    kc, vc = w.pool_device(device)
+    T, H, D = w.query.shape
+    return DevicePrefill(w=w, query=up(w.query), new_key=up(w.new_key), new_value=up(w.new_value),
+                         query_start=up(w.query_start), block_tables=up(w.block_tables),
+                         context_lens=up(w.context_lens), key_cache=kc, value_cache=vc,
+                         out=torch.empty((T, H, D), dtype=torch.float16, device=device),
+                         slots=torch.empty(T, dtype=torch.int32, device=device))
