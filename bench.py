@@ -11,6 +11,7 @@ leaving dirty lines whose write-back would land in the timed step, so the KV
 bytes come from HBM.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 1..5] [--impl ours|reference]
+    python bench.py --prefill 1..3      (paged prefill: TFLOP/s against the tensor peak)
 
 Under torchrun each rank runs its own independently seeded batch of the same
 shape (sequences are independent; there is no exchange step), and rank 0
@@ -422,6 +423,193 @@ def cpu_baseline(w, seconds: float):
                       f"single-thread fp64"}
 
 
+# ------------------------------------------------------------ paged prefill
+
+PREFILL_METRIC = "paged prefill attention TFLOP/s (causal, over the block table), 1 GPU"
+
+
+def tensor_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            rec = json.load(f)
+        return float(rec["bf16_tflops"]), float(rec["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 1590.0, 1400.0, "fallback"
+
+
+def run_prefill(args, rank, world, local_rank):
+    """One prefill step = slots of the chunk's tokens, their K/V scattered into
+    the cache, causal attention of the chunk over the block table. Same
+    capture, L2 eviction, timing, clock and end-to-end rules as the decode."""
+    import torch
+    import pagedattention_paged_kv_decode_b200 as pk
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    w = W.prefill_named(args.prefill, seed=W.rank_seed(2000 + args.prefill, rank))
+    dp = W.prefill_to_device(w, dev)
+    mql = int(w.chunk_lens.max(initial=0))
+    T = w.total_q
+    n_write = -(-T // 65535)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_sink = torch.zeros((), dtype=torch.int64, device=dev)
+    stream = torch.cuda.Stream(dev)
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
+
+    def step():
+        ev[0].record()
+        pk.prefill_slot_mapping(dp.query_start, dp.block_tables, dp.context_lens, dp.key_cache, mql,
+                                out=dp.slots)
+        for i in range(0, T, 65535):
+            m = min(65535, T - i)
+            pk.kv_cache_write(dp.new_key[i:i + m], dp.new_value[i:i + m], dp.key_cache, dp.value_cache,
+                              dp.slots[i:i + m])
+        ev[1].record()
+        pk.paged_prefill(dp.out, dp.query, dp.query_start, dp.key_cache, dp.value_cache, dp.block_tables,
+                         dp.context_lens, mql, w.scale)
+        ev[2].record()
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            step()
+        stream.synchronize()
+        assert pk.check_status(stream) == 0
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            step()
+        stream.synchronize()
+
+        def evict_l2():
+            flush.fill_(1)
+            flush_sink.copy_(flush.view(torch.int64).sum())
+
+        def timed_step():
+            evict_l2()
+            graph.replay()
+            stream.synchronize()
+            return ev[0].elapsed_time(ev[2]), ev[1].elapsed_time(ev[2])
+
+        for _ in range(max(3, args.warmup)):
+            timed_step()
+        visible = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
+        sampler = ClockSampler(visible[local_rank] if len(visible) > local_rank and visible[local_rank]
+                               else str(local_rank))
+        sampler.start()
+        time.sleep(0.3)
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0 = time.time()
+        step_ms, att_ms = [], []
+        for _ in range(args.steps):
+            a, b = timed_step()
+            step_ms.append(a)
+            att_ms.append(b)
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        t1 = time.time()
+        sampler.stop()
+        assert pk.check_status(stream) == 0
+
+        host_in = {k: getattr(dp, k).cpu().pin_memory()
+                   for k in ("query", "new_key", "new_value", "query_start", "block_tables", "context_lens")}
+        host_out = torch.empty(dp.out.shape, dtype=dp.out.dtype).pin_memory()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+        d2h = host_out.numel() * host_out.element_size()
+        e2e_ms = []
+        for i in range(max(3, args.warmup) + min(args.steps, 200)):
+            evict_l2()
+            e0.record()
+            for k, t in host_in.items():
+                getattr(dp, k).copy_(t, non_blocking=True)
+            graph.replay()
+            host_out.copy_(dp.out, non_blocking=True)
+            e1.record()
+            stream.synchronize()
+            if i >= max(3, args.warmup):
+                e2e_ms.append(e0.elapsed_time(e1))
+
+    step_t, att_t, e2e_t = slowest_rank([statistics.mean(step_ms), statistics.mean(att_ms),
+                                         statistics.mean(e2e_ms)], dist, dev)
+    clocks = sampler.summary(t0, t1)
+    del graph
+    if dist:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    flops = w.flops()
+    peak, peak_sust, kind = tensor_peak()
+    achieved = flops / (att_t * 1e-3) / 1e12
+    line = {
+        "metric": PREFILL_METRIC,
+        "value": round(world * flops / (step_t * 1e-3) / 1e12, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(step_t, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic (seeded numpy PCG64; no dataset)",
+        "config": {
+            "workload": w.name, "num_seqs": w.num_seqs, "num_heads": w.num_heads,
+            "head_size": w.head_size, "block_size": w.block_size, "kv_dtype": "f16",
+            "total_q": T, "context_lens": [int(x) for x in w.context_lens],
+            "chunk_lens": [int(x) for x in w.chunk_lens], "flops_per_step": flops,
+            "parallelism": f"replicas x{world} (independent batches, no collective)",
+            "l2": "before every timed step a 512 MiB buffer is written then read (L2 is 126 MB)",
+            "step": "CUDA graph: prefill_slot_mapping, kv_cache_write, paged_prefill",
+        },
+        "tokens_per_s": round(world * T / (step_t * 1e-3), 1),
+        "prefill_ms": round(att_t, 5),
+        "roofline": {
+            "bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4),
+            "peak_kind": f"{kind} dense bf16 GEMM, burst (fp16 runs at the same nominal rate); "
+                         f"sustained {peak_sust}",
+            "traffic": None, "kernel": "paged_prefill_kernel",
+            "algorithmic_flops_per_launch": flops,
+            "io_bytes_per_launch": w.io_bytes(),
+        },
+        "e2e": {"value": round(world * flops / (e2e_t * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_t, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "path": "pinned host inputs -> device copies -> graph replay -> output to pinned host"},
+        "gpu_launches": (2 + n_write) * args.steps,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_prefill(w, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline_prefill(w, seconds: float):
+    """The oracle, single-threaded, on a seeded sample of (row, head) pairs of
+    the prefill workload (cache write of the chunk outside the timed region);
+    TFLOP/s of the sampled pairs."""
+    import oracle
+    kc, vc = w.pool_host()
+    slots = oracle.prefill_slot_mapping(w.query_start, w.block_tables, w.context_lens, w.block_size)
+    oracle.kv_cache_write(w.new_key, w.new_value, kc, vc, slots)
+    rng = np.random.default_rng(0)
+    pos = w.positions()
+    done, elapsed, n = 0, 0.0, 0
+    while elapsed < seconds and n < 100000:
+        r = int(rng.integers(0, w.total_q))
+        h = int(rng.integers(0, w.num_heads))
+        t = time.perf_counter()
+        oracle.paged_prefill(w.query, w.query_start, kc, vc, w.block_tables, w.context_lens, w.scale,
+                             row_head=np.array([[r, h]], np.int32))
+        elapsed += time.perf_counter() - t
+        done += 4 * w.head_size * (int(pos[r]) + 1)
+        n += 1
+    return {"value": round(done / elapsed / 1e12, 8), "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} random (row, head) pairs of {w.name}: {elapsed:.1f} s, single-thread fp64"}
+
+
 def run_reference(args, rank, world):
     """The CPU oracle as the reference arm: rank 0 only, same metric and unit."""
     if rank != 0:
@@ -464,6 +652,8 @@ def main():
                     help="slot mapping, cache write and decode as three launches")
     ap.add_argument("--launch", default="",
                     help="decode launch shape partition_size,heads_per_cta,warps_per_head,stages")
+    ap.add_argument("--prefill", type=int, default=0, choices=[0, 1, 2, 3],
+                    help="time a paged prefill workload (1 tiny, 2 long prompts, 3 chunked) instead")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -472,6 +662,8 @@ def main():
         print(f"note: --gpus {args.gpus} but WORLD_SIZE {world}; using WORLD_SIZE", file=sys.stderr)
     if args.impl == "reference":
         run_reference(args, rank, world)
+    elif args.prefill:
+        run_prefill(args, rank, world, local_rank)
     else:
         run_ours(args, rank, world, local_rank)
 

@@ -62,6 +62,8 @@ extern "C" {
 #define PA_DEV_BAD_PAIR 16u       /* copy pair index outside [0, num_blocks): pair skipped */
 #define PA_DEV_WAIT_TIMEOUT 32u   /* an on-chip pipeline wait ran out (never expected) */
 #define PA_DEV_PREFIX 64u         /* shared-prefix contract broken (see ..._shared_prefix) */
+#define PA_DEV_BAD_CHUNK 128u     /* prefill chunk longer than its context (or than
+                                     max_query_len given to pa_paged_prefill): skipped */
 
 /* KV cache element type: fp16, or OCP FP8 E4M3 ("fn" variant: no infinities,
  * max 448) with one fp32 scale per cache tensor ([P1] §3.3, [P3] §4). */
@@ -95,7 +97,8 @@ typedef struct {
     int32_t units_per_cta;
 } pa_decode_config;
 
-/* Library version, e.g. 100 for 0.1.0. */
+/* Library version: 100 * minor + patch for 0.minor.patch (200 = 0.2.0, the
+ * release that adds the paged prefill calls). */
 int pa_version(void);
 
 /* Message for the last nonzero status returned on this thread ("" if none). */
@@ -294,6 +297,53 @@ int pa_paged_attention_decode_noalloc(void *out, const void *query,
                                       int max_blocks_per_seq, const int32_t *context_lens,
                                       int num_seqs, int max_context_len, float scale,
                                       float k_scale, float v_scale, void *stream);
+
+/* ------------------------------------------------------- paged prefill
+ * Prompt (or chunked-prompt) attention over the block table. [P1] §3.2 puts
+ * FlashAttention-style attention on the kernel path; [P3] §4 runs long
+ * texts (over 4k tokens) with 32-token blocks. The pages print no formula;
+ * the reading used is causal attention at each row's position:
+ *   sequence s brings n_s = query_start[s+1] - query_start[s] new tokens,
+ *   the last n_s positions of its context of L_s = context_lens[s] tokens
+ *   (0 <= n_s <= L_s); token query_start[s] + i sits at position
+ *   L_s - n_s + i.
+ * query_start: int32 [num_seqs + 1], non-decreasing, query_start[0] = 0
+ * (device). A full prompt has n_s = L_s; a chunk after cached context has
+ * n_s < L_s; n_s = 1 is a decode step. */
+
+/* Slot of every new token of the chunk ([P3] §2.2 slot mapping, at each
+ * token's position):
+ *     slot_mapping[query_start[s] + i] = block_tables[s][pos / block_size]
+ *                                        * block_size + pos % block_size,
+ *     pos = L_s - n_s + i
+ * max_query_len is a sizing hint (any n_s is covered). Device checks: a
+ * chunk with n_s > L_s sets PA_DEV_BAD_CHUNK and gets slots -1; a position
+ * beyond the table row sets PA_DEV_CTX_OVER_TABLE, a block id outside the
+ * pool PA_DEV_BAD_BLOCK; both give slot -1. With pa_kv_cache_write these
+ * slots store the chunk's K/V before pa_paged_prefill reads them. */
+int pa_prefill_slot_mapping(int32_t *slot_mapping, const int32_t *query_start,
+                            const int32_t *block_tables, int max_blocks_per_seq,
+                            const int32_t *context_lens, int num_seqs, int max_query_len,
+                            pa_cache_desc cache, void *stream);
+
+/* Causal attention of packed query rows over the paged cache:
+ *   out[r][h] = sum_{t <= pos(r)} softmax_t(scale * q[r][h] . K_t[h]) V_t[h]
+ * for every row r = query_start[s] + i (pos(r) = L_s - n_s + i) and head h.
+ * query, out: fp16 [total_q][num_heads][head_size], total_q =
+ * query_start[num_seqs]; the cache must already hold all L_s tokens of each
+ * sequence (the chunk's own K/V included). fp16 caches only (PA_ERR_DTYPE
+ * for E4M3). max_query_len: a host-known bound on every n_s (the grid is
+ * sized from it). Computed on tensor cores: Q.K^T and P.V in fp16 x fp16 ->
+ * fp32 (mma.m16n8k16), softmax in fp32 with P rounded to fp16.
+ * Device checks: n_s > L_s or n_s > max_query_len sets PA_DEV_BAD_CHUNK,
+ * L_s beyond the table row PA_DEV_CTX_OVER_TABLE; such a sequence's rows
+ * are not written. Block ids outside the pool read as zeros and set
+ * PA_DEV_BAD_BLOCK. One launch; no workspace. */
+int pa_paged_prefill(void *out, const void *query, const int32_t *query_start,
+                     const void *key_cache, const void *value_cache, pa_cache_desc cache,
+                     const int32_t *block_tables, int max_blocks_per_seq,
+                     const int32_t *context_lens, int num_seqs, int max_query_len, float scale,
+                     void *stream);
 
 #ifdef __cplusplus
 }

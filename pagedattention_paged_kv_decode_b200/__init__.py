@@ -1,4 +1,5 @@
-"""Paged-KV decode attention for NVIDIA B200 (sm_100a).
+"""Paged-KV decode attention for NVIDIA B200 (sm_100a), with the cache
+write, slot derivation, block copy and swap around it and a paged prefill.
 
 The calls below marshal torch tensors into the C ABI of ``libpagedkv.so``
 (``include/pagedkv.h``); every step runs in that library's CUDA kernels.
@@ -18,6 +19,9 @@ from .ops import (  # noqa: F401
     paged_attention_decode,
     paged_attention_decode_append,
     paged_attention_decode_shared_prefix,
+    paged_prefill,
+    prefill_slot_mapping,
+    prefill_step,
     slot_mapping,
     swap_blocks,
     version,

@@ -1,7 +1,8 @@
 // pa_api.cu -- the C ABI of libpagedkv.so (declared in include/pagedkv.h):
 // argument validation, launch-shape choice, TMA descriptors, the split
 // workspace and kernel launches. Every compute step runs in the kernels of
-// pa_decode.cuh and pa_cache_ops.cuh; nothing here touches KV data.
+// pa_decode.cuh, pa_prefill.cuh and pa_cache_ops.cuh; nothing here touches
+// KV data.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -15,6 +16,7 @@
 
 #include "pa_cache_ops.cuh"
 #include "pa_decode.cuh"
+#include "pa_prefill.cuh"
 #include "pagedkv.h"
 
 namespace {
@@ -488,7 +490,7 @@ int current_device(int *dev) {
 
 extern "C" {
 
-int pa_version(void) { return 100; }
+int pa_version(void) { return 200; }
 
 const char *pa_last_error(void) { return g_msg; }
 
@@ -919,4 +921,103 @@ extern "C" int pa_paged_attention_decode_noalloc(
                          max_blocks_per_seq, context_lens, num_seqs, bound, scale, k_scale,
                          v_scale, cfg, need ? scratch : nullptr, static_cast<cudaStream_t>(stream),
                          dev);
+}
+
+// ------------------------------------------------------------ paged prefill
+
+namespace {
+
+using PrefillKernel = void (*)(const CUtensorMap, const CUtensorMap, const pa::PrefillParams);
+
+PrefillKernel pick_prefill(int D, int B) {
+    if (D == 64 && B == 16) return pa::paged_prefill_kernel<64, 16>;
+    if (D == 64 && B == 32) return pa::paged_prefill_kernel<64, 32>;
+    if (D == 128 && B == 16) return pa::paged_prefill_kernel<128, 16>;
+    if (D == 128 && B == 32) return pa::paged_prefill_kernel<128, 32>;
+    return nullptr;
+}
+
+// Ring of the prefill kernel: about 96 KiB of K/V tiles, so that two CTAs
+// (160 threads, under 200 registers each) share an SM.
+int prefill_stages(const pa_cache_desc &c) {
+    const int stage = 4 * c.block_size * c.head_size;  // K + V tiles, fp16
+    return std::max(2, std::min(8, (96 * 1024) / stage));
+}
+
+}  // namespace
+
+extern "C" int pa_prefill_slot_mapping(int32_t *slot_mapping, const int32_t *query_start,
+                                       const int32_t *block_tables, int max_blocks_per_seq,
+                                       const int32_t *context_lens, int num_seqs, int max_query_len,
+                                       pa_cache_desc cache, void *stream) {
+    int rc = check_cache(cache);
+    if (rc) return rc;
+    if (num_seqs < 0 || num_seqs > 65535) return fail(PA_ERR_INVALID, "num_seqs %d not in [0, 65535]", num_seqs);
+    if (max_query_len < 0) return fail(PA_ERR_INVALID, "max_query_len %d < 0", max_query_len);
+    if (num_seqs == 0) return ok();
+    if (!slot_mapping || !query_start || !block_tables || !context_lens)
+        return fail(PA_ERR_INVALID, "null pointer argument");
+    if (max_blocks_per_seq < 1) return fail(PA_ERR_INVALID, "max_blocks_per_seq < 1");
+    const int threads = 256;
+    const int gx = std::max(1, std::min((max_query_len + threads - 1) / threads, 1024));
+    pa::prefill_slot_mapping_kernel<<<dim3(gx, num_seqs), threads, 0, static_cast<cudaStream_t>(stream)>>>(
+        slot_mapping, query_start, block_tables, max_blocks_per_seq, context_lens, cache.block_size,
+        cache.num_blocks);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "prefill_slot_mapping_kernel launch");
+    return ok();
+}
+
+extern "C" int pa_paged_prefill(void *out, const void *query, const int32_t *query_start,
+                                const void *key_cache, const void *value_cache, pa_cache_desc cache,
+                                const int32_t *block_tables, int max_blocks_per_seq,
+                                const int32_t *context_lens, int num_seqs, int max_query_len,
+                                float scale, void *stream) {
+    int rc = check_cache(cache);
+    if (rc) return rc;
+    if (cache.dtype != PA_F16) return fail(PA_ERR_DTYPE, "paged prefill supports fp16 caches only");
+    if (num_seqs < 0 || num_seqs > 65535) return fail(PA_ERR_INVALID, "num_seqs %d not in [0, 65535]", num_seqs);
+    if (max_query_len < 0) return fail(PA_ERR_INVALID, "max_query_len %d < 0", max_query_len);
+    if (num_seqs == 0 || max_query_len == 0) return ok();
+    if (!out || !query || !query_start || !key_cache || !value_cache || !block_tables || !context_lens)
+        return fail(PA_ERR_INVALID, "null pointer argument");
+    if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache))
+        return fail(PA_ERR_INVALID, "out, query and caches must be 16-byte aligned");
+    if (max_blocks_per_seq < 1) return fail(PA_ERR_INVALID, "max_blocks_per_seq %d < 1", max_blocks_per_seq);
+    if ((int64_t)max_blocks_per_seq * cache.block_size >= (int64_t(1) << 31))
+        return fail(PA_ERR_OVERFLOW, "max_blocks_per_seq * block_size overflows int32");
+    if (!std::isfinite(scale)) return fail(PA_ERR_INVALID, "scale is not finite");
+    const int64_t row_tiles = (max_query_len + pa::kPrefillRows - 1) / pa::kPrefillRows;
+    const int64_t n_ctas = row_tiles * num_seqs * cache.num_heads;
+    if (n_ctas > 0x7fffffff) return fail(PA_ERR_INVALID, "too many prefill tiles (%lld)", (long long)n_ctas);
+    int dev = 0;
+    rc = current_device(&dev);
+    if (rc) return rc;
+    PrefillKernel kern = pick_prefill(cache.head_size, cache.block_size);
+    rc = ensure_smem_attr(reinterpret_cast<const void *>(kern), dev);
+    if (rc) return rc;
+    CUtensorMap mk, mv;
+    rc = cache_tensor_map(key_cache, cache, 1, &mk, 1);
+    if (rc) return rc;
+    rc = cache_tensor_map(value_cache, cache, 1, &mv, 1);
+    if (rc) return rc;
+    pa::PrefillParams p{};
+    p.out = static_cast<__half *>(out);
+    p.query = static_cast<const __half *>(query);
+    p.query_start = query_start;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.num_seqs = num_seqs;
+    p.num_heads = cache.num_heads;
+    p.num_blocks = cache.num_blocks;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.max_query_len = max_query_len;
+    p.stages = prefill_stages(cache);
+    p.qk_scale_log2 = scale * pa::kLog2e;
+    // ring + barriers + 1 KiB to align the ring to 1024 bytes in the kernel
+    const size_t smem = (size_t)p.stages * 4 * cache.block_size * cache.head_size + 16 * (size_t)p.stages + 1024;
+    kern<<<dim3((unsigned)n_ctas), dim3(32 * 5), smem, static_cast<cudaStream_t>(stream)>>>(mk, mv, p);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "paged_prefill_kernel launch");
+    return ok();
 }

@@ -838,17 +838,173 @@ paged_prefix_kernel(const __grid_constant__ CUtensorMap tmap_k,
     if (sub == 0) p.ws_lse[idx] = any ? st.m + fast_log2(st.l) : -INFINITY;
 }
 
-// Shared-prefix attention on tensor cores (fp16 caches). One CTA = one head
-// x one prefix partition x up to 64 sequences; consumer warp w takes the 16
-// sequences 16w .. 16w+15 of the CTA's block. The producer streams the
-// shared blocks' K and V tiles (64-dim halves, 128-byte swizzle) through a
-// ring. Per tile and warp:
-//   S (16 x B)  = Q (16 x D) . K^T        mma.m16n8k16, K fragments by ldmatrix
-//   online softmax per row on the S fragments (masked to each row's length)
+// Tensor-core attention of 16 query rows per warp over K/V tiles of B
+// tokens held in shared memory as 64-dim half tiles with 128-byte swizzle
+// (what a TMA load with box {64, 1, B, 1} and CU_TENSOR_MAP_SWIZZLE_128B
+// writes). Fragment layout of mma.m16n8k16: lane l holds rows g = l / 4 and
+// g + 8 and the column pair c = 2 (l % 4), c + 1 of each 8-wide n-tile.
+// Per tile:
+//   S (16 x B)  = Q (16 x D) . K^T        K fragments by ldmatrix
+//   online softmax per row on the S fragments, tokens >= the row's limit masked
 //   O (16 x D) += P (16 x B) . V          P reused from the S registers as the
 //                                         A operand, V fragments by ldmatrix.trans
-// then the partition's partial (lse, o) of each sequence is written. Q and P
-// are f16 (P <= 1: relative rounding <= 2^-11); S and O accumulate in fp32.
+// Q and P are f16 (P <= 1: relative rounding <= 2^-11); S and O accumulate
+// in fp32. Scores are in log2 units: Q is pre-scaled by scale * log2(e).
+template <int D, int B>
+struct MmaRows {
+    static constexpr int KS = D / 16;   // k-steps over dims
+    static constexpr int NT = B / 8;    // score n-tiles (8 tokens each)
+    static constexpr int ON = D / 8;    // output n-tiles (8 dims each)
+    static constexpr int kHalfTile = B * 128;  // bytes of one 64-dim half tile
+
+    uint32_t qa[KS][4];
+    float o[ON][4];
+    float m[2], l[2];
+
+    // q0 / q1: the D query values of fragment rows g and g + 8 (null: zeros).
+    __device__ __forceinline__ void load_q(const __half *q0, const __half *q1, float sc, int lane) {
+        const int c = (lane & 3) * 2;
+        const __half *qr[2] = {q0, q1};
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+#pragma unroll
+                for (int hi = 0; hi < 2; ++hi) {
+                    uint32_t v = 0;
+                    if (qr[r] != nullptr) {
+                        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(qr[r] + ks * 16 + c + 8 * hi));
+                        v = pack_half2(f.x * sc, f.y * sc);
+                    }
+                    qa[ks][r + 2 * hi] = v;  // a0 (row g), a1 (row g+8), a2/a3: +8 columns
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < ON; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+        m[0] = m[1] = -INFINITY;
+        l[0] = l[1] = 0.f;
+    }
+
+    // One tile: kt / vt the K and V tiles, tb the position of its first
+    // token, lim[r] the exclusive token limit of fragment row r, vlim the
+    // end of the sequence: V rows at or after it are unused cache slots
+    // whose contents may be anything (NaN included) and enter P.V as zeros.
+    __device__ __forceinline__ void attend(const unsigned char *kt, const unsigned char *vt, int tb,
+                                           const int (&lim)[2], int vlim, int lane) {
+        const int c = (lane & 3) * 2;
+        // ---- S = Q K^T
+        float sacc[NT][4];
+#pragma unroll
+        for (int n = 0; n < NT; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
+#pragma unroll
+        for (int np = 0; np < NT / 2; ++np) {
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+                // matrices: (tokens +0..7, dims +0..7), (+0..7, +8..15), (+8..15, +0..7), (+8..15, +8..15)
+                const int mi = lane >> 3, r = lane & 7;
+                const int tok = np * 16 + ((mi >> 1) << 3) + r;
+                const int dim = ks * 16 + ((mi & 1) << 3);
+                const unsigned char *addr = kt + (dim >> 6) * kHalfTile + swz128(tok, (dim & 63) * 2);
+                uint32_t b[4];
+                ldmatrix_x4(b, addr);
+                mma_16816(sacc[2 * np], qa[ks], b[0], b[1]);
+                mma_16816(sacc[2 * np + 1], qa[ks], b[2], b[3]);
+            }
+        }
+
+        // ---- online softmax per row (rows g and g+8 of this warp's 16)
+        float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = e >> 1;
+                const int tok = tb + n * 8 + c + (e & 1);
+                if (tok >= lim[r]) sacc[n][e] = -INFINITY;
+                mx[r] = fmaxf(mx[r], sacc[n][e]);
+            }
+        }
+        float alpha[2], mref[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+            mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+            const float mn = fmaxf(m[r], mx[r]);
+            mref[r] = mn == -INFINITY ? 0.f : mn;  // rows without tokens so far stay at zero
+            alpha[r] = fast_exp2(m[r] - mref[r]);
+            m[r] = mn;
+        }
+        uint32_t pa[NT / 2][4];
+        float rs[2] = {0.f, 0.f};
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            const float p0 = fast_exp2(sacc[n][0] - mref[0]);
+            const float p1 = fast_exp2(sacc[n][1] - mref[0]);
+            const float p2 = fast_exp2(sacc[n][2] - mref[1]);
+            const float p3 = fast_exp2(sacc[n][3] - mref[1]);
+            rs[0] += p0 + p1;
+            rs[1] += p2 + p3;
+            // A operand of P.V for token k-step n/2: a0/a1 from n-tile 2k, a2/a3 from 2k+1
+            pa[n >> 1][(n & 1) * 2 + 0] = pack_half2(p0, p1);
+            pa[n >> 1][(n & 1) * 2 + 1] = pack_half2(p2, p3);
+        }
+#pragma unroll
+        for (int r = 0; r < 2; ++r) l[r] = l[r] * alpha[r] + rs[r];
+#pragma unroll
+        for (int j = 0; j < ON; ++j) {
+            o[j][0] *= alpha[0];
+            o[j][1] *= alpha[0];
+            o[j][2] *= alpha[1];
+            o[j][3] *= alpha[1];
+        }
+
+        // ---- O += P V
+        // b[0] and b[2] hold tokens kt2*16 + c, c + 1 (low, high half); b[1]
+        // and b[3] the same + 8. In the sequence's last tile, halves of
+        // tokens >= vlim are cleared.
+        const bool tail = tb + B > vlim;
+#pragma unroll
+        for (int kt2 = 0; kt2 < NT / 2; ++kt2) {
+            uint32_t keep[2] = {0xffffffffu, 0xffffffffu};
+            if (tail) {
+#pragma unroll
+                for (int hi = 0; hi < 2; ++hi) {
+                    const int t = tb + kt2 * 16 + 8 * hi + c;
+                    keep[hi] = (t < vlim ? 0x0000ffffu : 0u) | (t + 1 < vlim ? 0xffff0000u : 0u);
+                }
+            }
+#pragma unroll
+            for (int dp = 0; dp < ON / 2; ++dp) {
+                // matrices (transposed): (tokens +0..7, dims +0..7), (+8..15, +0..7), (+0..7, +8..15), (+8..15, +8..15)
+                const int mi = lane >> 3, r = lane & 7;
+                const int tok = kt2 * 16 + ((mi & 1) << 3) + r;
+                const int dim = dp * 16 + ((mi >> 1) << 3);
+                const unsigned char *addr = vt + (dim >> 6) * kHalfTile + swz128(tok, (dim & 63) * 2);
+                uint32_t b[4];
+                ldmatrix_x4_trans(b, addr);
+                mma_16816(o[2 * dp], pa[kt2], b[0] & keep[0], b[1] & keep[1]);
+                mma_16816(o[2 * dp + 1], pa[kt2], b[2] & keep[0], b[3] & keep[1]);
+            }
+        }
+    }
+
+    // Row sums over the quad that shares each row (after the last tile).
+    __device__ __forceinline__ void reduce_l() {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            l[r] += __shfl_xor_sync(0xffffffffu, l[r], 1);
+            l[r] += __shfl_xor_sync(0xffffffffu, l[r], 2);
+        }
+    }
+};
+
+// Shared-prefix attention on tensor cores (fp16 caches). One CTA = one head
+// x one prefix partition x up to 64 sequences; consumer warp w takes the 16
+// sequences 16w .. 16w+15 of the CTA's block (MmaRows above). The producer
+// streams the shared blocks' K and V tiles (64-dim halves, 128-byte swizzle)
+// through a ring; after the last tile the partition's partial (lse, o) of
+// each sequence is written.
 constexpr int kPrefixMmaQueries = 64;  // sequences per CTA (4 warps x 16)
 
 template <int D, int B>
@@ -864,9 +1020,7 @@ __global__ void __launch_bounds__(32 * 5, 1)
 paged_prefix_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
                         const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
     using Lay = PrefixMmaLayout<D, B>;
-    constexpr int KS = D / 16;   // k-steps over dims
-    constexpr int NT = B / 8;    // score n-tiles (8 tokens each)
-    constexpr int ON = D / 8;    // output n-tiles (8 dims each)
+    constexpr int ON = D / 8;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // 128-byte-swizzled TMA destinations must be 1024-byte aligned: align the
     // ring explicitly (the launch adds 1 KiB of slack).
@@ -939,8 +1093,7 @@ paged_prefix_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int c = (lane & 3) * 2;     // fragment column pair
     const int q0 = q_base + warp * 16;
     const int rows[2] = {q0 + g, q0 + g + 8};
-    int Lr[2];
-    uint32_t qa[KS][4];
+    int lim[2];
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
         int L = 0;
@@ -949,145 +1102,37 @@ paged_prefix_mma_kernel(const __grid_constant__ CUtensorMap tmap_k,
             L = min(L, p.max_blocks_per_seq * B);
             L = max(min(L, p.max_context_len), 0);
         }
-        Lr[r] = min(L, t1);  // this row's tokens end here (within the partition)
+        lim[r] = min(L, t1);  // this row's tokens end here (within the partition)
     }
-    {
-        const float sc = p.qk_scale_log2;
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-#pragma unroll
-                for (int hi = 0; hi < 2; ++hi) {
-                    uint32_t v = 0;
-                    if (rows[r] < S) {
-                        const __half2 x = *reinterpret_cast<const __half2 *>(
-                            p.query + ((size_t)rows[r] * p.num_heads + h) * D + ks * 16 + c + 8 * hi);
-                        const float2 f = __half22float2(x);
-                        v = pack_half2(f.x * sc, f.y * sc);
-                    }
-                    qa[ks][r + 2 * hi] = v;  // a0 (row g), a1 (row g+8), a2/a3: +8 columns
-                }
-            }
-        }
-    }
+    MmaRows<D, B> mr;
+    mr.load_q(rows[0] < S ? p.query + ((size_t)rows[0] * p.num_heads + h) * D : nullptr,
+              rows[1] < S ? p.query + ((size_t)rows[1] * p.num_heads + h) * D : nullptr, p.qk_scale_log2,
+              lane);
     asm volatile("bar.sync 1, %0;" ::"r"((n_consumers + 1) * 32) : "memory");
-
-    float o[ON][4];
-#pragma unroll
-    for (int j = 0; j < ON; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
 
     for (int i = 0; i < nblk; ++i) {
         const int st = i % stages, use = i / stages;
         if (!mbar_wait(&full[st], use & 1)) break;
         const unsigned char *kt = smem + (size_t)st * Lay::kStage;
-        const unsigned char *vt = kt + Lay::kTile;
-        const int tb = t0 + i * B;  // first token of the tile
-
-        // ---- S = Q K^T
-        float sacc[NT][4];
-#pragma unroll
-        for (int n = 0; n < NT; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
-#pragma unroll
-        for (int np = 0; np < NT / 2; ++np) {
-#pragma unroll
-            for (int ks = 0; ks < KS; ++ks) {
-                // matrices: (tokens +0..7, dims +0..7), (+0..7, +8..15), (+8..15, +0..7), (+8..15, +8..15)
-                const int mi = lane >> 3, r = lane & 7;
-                const int tok = np * 16 + ((mi >> 1) << 3) + r;
-                const int dim = ks * 16 + ((mi & 1) << 3);
-                const unsigned char *addr = kt + (dim >> 6) * Lay::kHalfTile + swz128(tok, (dim & 63) * 2);
-                uint32_t b[4];
-                ldmatrix_x4(b, addr);
-                mma_16816(sacc[2 * np], qa[ks], b[0], b[1]);
-                mma_16816(sacc[2 * np + 1], qa[ks], b[2], b[3]);
-            }
-        }
-
-        // ---- online softmax per row (rows g and g+8 of this warp's 16)
-        float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int r = e >> 1;
-                const int tok = tb + n * 8 + c + (e & 1);
-                if (tok >= Lr[r]) sacc[n][e] = -INFINITY;
-                mx[r] = fmaxf(mx[r], sacc[n][e]);
-            }
-        }
-        float alpha[2], mref[2];
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
-            mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
-            const float mn = fmaxf(m[r], mx[r]);
-            mref[r] = mn == -INFINITY ? 0.f : mn;  // rows without tokens so far stay at zero
-            alpha[r] = fast_exp2(m[r] - mref[r]);
-            m[r] = mn;
-        }
-        uint32_t pa[NT / 2][4];
-        float rs[2] = {0.f, 0.f};
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            const float p0 = fast_exp2(sacc[n][0] - mref[0]);
-            const float p1 = fast_exp2(sacc[n][1] - mref[0]);
-            const float p2 = fast_exp2(sacc[n][2] - mref[1]);
-            const float p3 = fast_exp2(sacc[n][3] - mref[1]);
-            rs[0] += p0 + p1;
-            rs[1] += p2 + p3;
-            // A operand of P.V for token k-step n/2: a0/a1 from n-tile 2k, a2/a3 from 2k+1
-            pa[n >> 1][(n & 1) * 2 + 0] = pack_half2(p0, p1);
-            pa[n >> 1][(n & 1) * 2 + 1] = pack_half2(p2, p3);
-        }
-#pragma unroll
-        for (int r = 0; r < 2; ++r) l[r] = l[r] * alpha[r] + rs[r];
-#pragma unroll
-        for (int j = 0; j < ON; ++j) {
-            o[j][0] *= alpha[0];
-            o[j][1] *= alpha[0];
-            o[j][2] *= alpha[1];
-            o[j][3] *= alpha[1];
-        }
-
-        // ---- O += P V
-#pragma unroll
-        for (int kt2 = 0; kt2 < NT / 2; ++kt2) {
-#pragma unroll
-            for (int dp = 0; dp < ON / 2; ++dp) {
-                // matrices (transposed): (tokens +0..7, dims +0..7), (+8..15, +0..7), (+0..7, +8..15), (+8..15, +8..15)
-                const int mi = lane >> 3, r = lane & 7;
-                const int tok = kt2 * 16 + ((mi & 1) << 3) + r;
-                const int dim = dp * 16 + ((mi >> 1) << 3);
-                const unsigned char *addr = vt + (dim >> 6) * Lay::kHalfTile + swz128(tok, (dim & 63) * 2);
-                uint32_t b[4];
-                ldmatrix_x4_trans(b, addr);
-                mma_16816(o[2 * dp], pa[kt2], b[0], b[1]);
-                mma_16816(o[2 * dp + 1], pa[kt2], b[2], b[3]);
-            }
-        }
+        mr.attend(kt, kt + Lay::kTile, t0 + i * B, lim, t1, lane);  // shared blocks are full
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[st]);
     }
 
-    // ---- partials: row sums over the quad, then (lse, o) per sequence
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-        l[r] += __shfl_xor_sync(0xffffffffu, l[r], 1);
-        l[r] += __shfl_xor_sync(0xffffffffu, l[r], 2);
-    }
+    // ---- partials: (lse, o) per sequence
+    mr.reduce_l();
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
         if (rows[r] >= S) continue;
         const size_t idx = ((size_t)rows[r] * p.num_heads + h) * p.ws_parts + pp;
-        const bool any = l[r] > 0.f;
-        const float inv = any ? 1.0f / l[r] : 0.f;
+        const bool any = mr.l[r] > 0.f;
+        const float inv = any ? 1.0f / mr.l[r] : 0.f;
         float *op = p.ws_o + idx * D;
 #pragma unroll
         for (int j = 0; j < ON; ++j)
-            *reinterpret_cast<float2 *>(op + j * 8 + c) = make_float2(o[j][2 * r] * inv, o[j][2 * r + 1] * inv);
-        if ((lane & 3) == 0) p.ws_lse[idx] = any ? m[r] + fast_log2(l[r]) : -INFINITY;
+            *reinterpret_cast<float2 *>(op + j * 8 + c) =
+                make_float2(mr.o[j][2 * r] * inv, mr.o[j][2 * r + 1] * inv);
+        if ((lane & 3) == 0) p.ws_lse[idx] = any ? mr.m[r] + fast_log2(mr.l[r]) : -INFINITY;
     }
 }
 

@@ -342,3 +342,73 @@ def decode_step(out: torch.Tensor, query: torch.Tensor, new_key: torch.Tensor,
     paged_attention_decode(out, query, key_cache, value_cache, block_tables, context_lens, scale,
                            k_scale, v_scale, max_context_len, config, workspace, stream)
     return slots
+
+
+# ------------------------------------------------------------ paged prefill
+
+def prefill_slot_mapping(query_start: torch.Tensor, block_tables: torch.Tensor,
+                         context_lens: torch.Tensor, key_cache: torch.Tensor,
+                         max_query_len: int, out: torch.Tensor | None = None,
+                         total_q: int | None = None, stream=None) -> torch.Tensor:
+    """Slot of every new token of a prefill chunk ([total_q] int32).
+
+    ``total_q`` (= query_start[-1]) must be given when ``out`` is not, since
+    reading it from the device would synchronise."""
+    _i32(query_start, "query_start")
+    _i32(block_tables, "block_tables")
+    _i32(context_lens, "context_lens")
+    S = context_lens.shape[0]
+    if query_start.shape[0] != S + 1 or block_tables.shape[0] != S:
+        raise ValueError("query_start must hold num_seqs + 1 entries and block_tables num_seqs rows")
+    if out is None:
+        if total_q is None:
+            raise ValueError("give out or total_q")
+        out = torch.empty(int(total_q), dtype=torch.int32, device=context_lens.device)
+    _i32(out, "out")
+    check(lib().pa_prefill_slot_mapping(out.data_ptr(), query_start.data_ptr(), block_tables.data_ptr(),
+                                        block_tables.shape[1], context_lens.data_ptr(), S,
+                                        int(max_query_len), cache_desc(key_cache), _stream(stream)))
+    return out
+
+
+def paged_prefill(out: torch.Tensor, query: torch.Tensor, query_start: torch.Tensor,
+                  key_cache: torch.Tensor, value_cache: torch.Tensor, block_tables: torch.Tensor,
+                  context_lens: torch.Tensor, max_query_len: int, scale: float, stream=None) -> None:
+    """Causal attention of packed query rows ([total_q, H, D] fp16) over the
+    paged fp16 cache, which must already hold each sequence's chunk."""
+    _check_pair(key_cache, value_cache)
+    _i32(query_start, "query_start")
+    _i32(block_tables, "block_tables")
+    _i32(context_lens, "context_lens")
+    for t in (out, query):
+        if t.dtype != torch.float16 or not t.is_cuda or not t.is_contiguous() or t.dim() != 3:
+            raise ValueError("out and query must be contiguous float16 CUDA tensors [total_q, H, D]")
+    S = context_lens.shape[0]
+    if out.shape != query.shape or query_start.shape[0] != S + 1 or block_tables.shape[0] != S:
+        raise ValueError("shape mismatch between out, query, query_start, block_tables and context_lens")
+    desc = cache_desc(key_cache)
+    if desc.num_heads != query.shape[1] or desc.head_size != query.shape[2]:
+        raise ValueError("query heads/head_size differ from the cache's")
+    check(lib().pa_paged_prefill(out.data_ptr(), query.data_ptr(), query_start.data_ptr(),
+                                 key_cache.data_ptr(), value_cache.data_ptr(), desc, block_tables.data_ptr(),
+                                 block_tables.shape[1], context_lens.data_ptr(), S, int(max_query_len),
+                                 float(scale), _stream(stream)))
+
+
+def prefill_step(out: torch.Tensor, query: torch.Tensor, new_key: torch.Tensor, new_value: torch.Tensor,
+                 query_start: torch.Tensor, key_cache: torch.Tensor, value_cache: torch.Tensor,
+                 block_tables: torch.Tensor, context_lens: torch.Tensor, max_query_len: int,
+                 scale: float, slots: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """One prefill step on the device, in order: slots of the chunk's tokens,
+    scatter of their K/V rows into the cache, causal attention. Returns the
+    slot tensor."""
+    T = query.shape[0]
+    slots = prefill_slot_mapping(query_start, block_tables, context_lens, key_cache, max_query_len,
+                                 out=slots, total_q=T, stream=stream)
+    for i in range(0, T, 65535):  # the cache write takes at most 65535 tokens a call
+        m = min(65535, T - i)
+        kv_cache_write(new_key[i:i + m], new_value[i:i + m], key_cache, value_cache, slots[i:i + m],
+                       stream=stream)
+    paged_prefill(out, query, query_start, key_cache, value_cache, block_tables, context_lens,
+                  max_query_len, scale, stream)
+    return slots
