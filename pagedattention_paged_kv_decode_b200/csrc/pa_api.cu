@@ -987,13 +987,19 @@ extern "C" int pa_paged_prefill(void *out, const void *query, const int32_t *que
     if ((int64_t)max_blocks_per_seq * cache.block_size >= (int64_t(1) << 31))
         return fail(PA_ERR_OVERFLOW, "max_blocks_per_seq * block_size overflows int32");
     if (!std::isfinite(scale)) return fail(PA_ERR_INVALID, "scale is not finite");
-    const int64_t row_tiles = (max_query_len + pa::kPrefillRows - 1) / pa::kPrefillRows;
+    const int rows_per_cta = (cache.head_size == 128 && scale > 0.f) ? pa::kTcRows : pa::kPrefillRows;
+    const int64_t row_tiles = (max_query_len + rows_per_cta - 1) / rows_per_cta;
     const int64_t n_ctas = row_tiles * num_seqs * cache.num_heads;
     if (n_ctas > 0x7fffffff) return fail(PA_ERR_INVALID, "too many prefill tiles (%lld)", (long long)n_ctas);
     int dev = 0;
     rc = current_device(&dev);
     if (rc) return rc;
-    PrefillKernel kern = pick_prefill(cache.head_size, cache.block_size);
+    // head_size 128 with a positive scale: the tcgen05 kernel (128-row tiles,
+    // S and O in tensor memory); otherwise the mma.sync kernel (64-row tiles).
+    const bool tc = cache.head_size == 128 && scale > 0.f;
+    PrefillKernel kern = tc ? (cache.block_size == 16 ? pa::paged_prefill_tc_kernel<16>
+                                                      : pa::paged_prefill_tc_kernel<32>)
+                            : pick_prefill(cache.head_size, cache.block_size);
     rc = ensure_smem_attr(reinterpret_cast<const void *>(kern), dev);
     if (rc) return rc;
     CUtensorMap mk, mv;
@@ -1014,9 +1020,11 @@ extern "C" int pa_paged_prefill(void *out, const void *query, const int32_t *que
     p.max_query_len = max_query_len;
     p.stages = prefill_stages(cache);
     p.qk_scale_log2 = scale * pa::kLog2e;
-    // ring + barriers + 1 KiB to align the ring to 1024 bytes in the kernel
-    const size_t smem = (size_t)p.stages * 4 * cache.block_size * cache.head_size + 16 * (size_t)p.stages + 1024;
-    kern<<<dim3((unsigned)n_ctas), dim3(32 * 5), smem, static_cast<cudaStream_t>(stream)>>>(mk, mv, p);
+    // ring (or tcgen05 tiles) + barriers + 1 KiB to align to 1024 bytes in the kernel
+    const size_t smem = tc ? (size_t)pa::TcLayout::kBytes + 1024
+                           : (size_t)p.stages * 4 * cache.block_size * cache.head_size + 16 * (size_t)p.stages + 1024;
+    kern<<<dim3((unsigned)n_ctas), dim3(tc ? pa::kTcThreads : 32 * 5), smem, static_cast<cudaStream_t>(stream)>>>(
+        mk, mv, p);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "paged_prefill_kernel launch");
     return ok();

@@ -193,3 +193,377 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
 }
 
 }  // namespace pa
+
+namespace pa {
+
+// ----------------------------------------- prefill on tcgen05 (head_size 128)
+//
+// One CTA = one head x one tile of up to 128 consecutive query rows of one
+// sequence; K/V are consumed 128 tokens at a time. Per K/V tile j:
+//   S_j = Q . K_j^T   128 x 128, eight tcgen05.mma (K = 16 each) into tensor
+//                     memory (two S buffers, so S_{j+1} overlaps the softmax of j)
+//   softmax           thread t of the four softmax warps owns row t (tensor-
+//                     memory lane t): reads its S row, masks tokens after its
+//                     position, keeps a reference maximum that moves only when
+//                     the row maximum exceeds it by more than 2^8 (then O is
+//                     rescaled in tensor memory), writes P = 2^(s - m) as fp16
+//                     into shared memory (128-byte swizzle)
+//   O += P_j . V_j    eight tcgen05.mma into the O columns of tensor memory,
+//                     V read N-contiguous (MN-major)
+// Warps: 0-3 softmax (and Q staging, epilogue), 4 TMA producer, 5 MMA issuer
+// (also allocates the 512 tensor-memory columns). Every wait is bounded; a
+// wait that runs out sets PA_DEV_WAIT_TIMEOUT and an abort flag that ends
+// the other roles' waits, and the CTA still drains its copies and MMAs and
+// frees its tensor memory before it exits.
+constexpr int kTcRows = 128;
+constexpr int kTcKv = 128;
+constexpr int kTcStages = 2;
+constexpr int kTcThreads = 192;
+constexpr int kTcTmemCols = 512;  // S0 [0,128), S1 [128,256), O [256,384)
+
+struct TcLayout {                                       // byte offsets from the 1024-aligned base
+    static constexpr uint32_t kHalf = 128 * 128;         // [128 rows][128 B]: one 64-wide half
+    static constexpr uint32_t kQ = 0;                    // Q: 2 halves (dims 0-63, 64-127)
+    static constexpr uint32_t kStage0 = 2 * kHalf;       // stage s: K (2 halves), then V (2 halves)
+    static constexpr uint32_t kStageBytes = 4 * kHalf;
+    static constexpr uint32_t kP = kStage0 + kTcStages * kStageBytes;  // P: 2 halves (tokens 0-63, 64-127)
+    static constexpr uint32_t kBars = kP + 2 * kHalf;
+    static constexpr uint32_t kBytes = kBars + 128;
+};
+
+// mbarrier indices
+enum : int {
+    kBarQ = 0,                   // Q staged (4 softmax warps)
+    kBarFullK = 1,               // + stage: K tile landed (TMA bytes)
+    kBarFullV = 3,               // + stage: V tile landed
+    kBarEmpty = 5,               // + stage: P.V of the stage's tile done (commit)
+    kBarSFull = 7,               // + buffer: S ready (commit)
+    kBarSFree = 9,               // + buffer: S read by the 4 softmax warps
+    kBarPFull = 11,              // P written, O corrected (4 softmax warps)
+    kBarOReady = 12,             // P.V done (commit)
+    kBarDone = 13,               // every MMA of the CTA done (commit)
+    kNumBars = 14
+};
+
+// Bounded wait that also ends when another role has aborted.
+__device__ __forceinline__ bool tc_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 32; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (*abort) return false;
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            flag_error(PA_DEV_WAIT_TIMEOUT);
+            *abort = 1;
+            return false;
+        }
+    }
+}
+
+// Every lane waits; the warp goes on only if all lanes saw the phase.
+__device__ __forceinline__ bool tc_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    const bool ok = tc_wait(bar, parity, abort);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// 16 bytes at chunk c (0..15) of row r of a [2 halves][128 rows][128 B]
+// swizzled tile.
+__device__ __forceinline__ uint32_t tc_chunk(uint32_t base, int r, int c) {
+    return base + (uint32_t)(c >> 3) * TcLayout::kHalf + (uint32_t)r * 128u +
+           ((uint32_t)(((c & 7) ^ (r & 7))) << 4);
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+template <int B>
+__global__ void __launch_bounds__(kTcThreads, 1)
+paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+                        const PrefillParams p) {
+    constexpr int D = 128;
+    constexpr int BPT = kTcKv / B;  // cache blocks per K/V tile
+    using Lay = TcLayout;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + Lay::kBars);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Lay::kBars + 8 * kNumBars);
+    volatile int *abort = reinterpret_cast<volatile int *>(smem + Lay::kBars + 8 * kNumBars + 4);
+    const uint32_t sbase = smem_u32(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // ---- the CTA's rows (uniform; every early exit precedes any barrier)
+    const int h = blockIdx.x % p.num_heads;
+    const int rest = blockIdx.x / p.num_heads;
+    const int s = rest % p.num_seqs;
+    const int t_rev = rest / p.num_seqs;
+    const int q_begin = __ldg(p.query_start + s);
+    const int n = __ldg(p.query_start + s + 1) - q_begin;
+    const int L = __ldg(p.context_lens + s);
+    if (n <= 0) return;
+    if (n > L || n > p.max_query_len) {
+        if (t_rev == 0 && h == 0 && threadIdx.x == 0) flag_error(PA_DEV_BAD_CHUNK);
+        return;
+    }
+    if (L > p.max_blocks_per_seq * B) {
+        if (t_rev == 0 && h == 0 && threadIdx.x == 0) flag_error(PA_DEV_CTX_OVER_TABLE);
+        return;
+    }
+    const int n_tiles = (n + kTcRows - 1) / kTcRows;
+    if (t_rev >= n_tiles) return;
+    const int r0 = (n_tiles - 1 - t_rev) * kTcRows;
+    const int rows_here = min(kTcRows, n - r0);
+    const int base = L - n;                                  // position of row 0 of the chunk
+    const int kv_end = base + r0 + rows_here;                // tokens the last row sees
+    const int nblk = (kv_end + B - 1) / B;
+    const int n_kv = (kv_end + kTcKv - 1) / kTcKv;
+    const int32_t *table = p.block_tables + (size_t)s * p.max_blocks_per_seq;
+
+    // ---- set-up: tensor memory, barriers
+    if (warp == 5) {
+        tmem_alloc(tmem_slot, kTcTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == 4 && lane == 0) {
+        prefetch_tensor_map(&tmap_k);
+        prefetch_tensor_map(&tmap_v);
+        const uint32_t counts[kNumBars] = {4, 1, 1, 1, 1, 1, 1, 1, 1, 4, 4, 4, 1, 1};
+        for (int i = 0; i < kNumBars; ++i) mbar_init(&bar[i], counts[i]);
+        *abort = 0;
+        fence_mbar_init();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 4) {
+        // ---------------------------------------------------------- producer
+        const uint64_t policy = l2_policy_evict_normal();  // other row tiles re-read these blocks
+        int issued = 0;
+        for (int j = 0; j < n_kv; ++j) {
+            const int st = j % kTcStages, use = j / kTcStages;
+            int blk = p.num_blocks;  // past the sequence: zero filled
+            const int lb = j * BPT + lane;
+            if (lane < BPT && lb < nblk) {
+                const int b = __ldg(table + lb);
+                if (b < 0 || b >= p.num_blocks)
+                    flag_error(PA_DEV_BAD_BLOCK);
+                else
+                    blk = b;
+            }
+            bool ok = true;
+            if (lane == 0 && use > 0) ok = tc_wait(&bar[kBarEmpty + st], (use - 1) & 1, abort);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&bar[kBarFullK + st], (uint32_t)(kTcKv * D * 2));
+                mbar_arrive_expect_tx(&bar[kBarFullV + st], (uint32_t)(kTcKv * D * 2));
+            }
+            __syncwarp();
+            if (lane < BPT) {
+                unsigned char *kdst = smem + Lay::kStage0 + st * Lay::kStageBytes + lane * B * 128;
+                unsigned char *vdst = kdst + 2 * Lay::kHalf;
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    tma_load_4d(kdst + hf * Lay::kHalf, &tmap_k, &bar[kBarFullK + st], 64 * hf, h, 0, blk, policy);
+                    tma_load_4d(vdst + hf * Lay::kHalf, &tmap_v, &bar[kBarFullV + st], 64 * hf, h, 0, blk, policy);
+                }
+            }
+            issued = j + 1;
+        }
+        // let the copies in flight land before the warp retires
+        if (lane == 0) {
+            for (int j = max(0, issued - kTcStages); j < issued; ++j) {
+                const int st = j % kTcStages, use = j / kTcStages;
+                mbar_wait(&bar[kBarFullK + st], use & 1);
+                mbar_wait(&bar[kBarFullV + st], use & 1);
+            }
+        }
+        return;
+    }
+
+    if (warp == 5) {
+        // ---------------------------------------------------------- MMA issuer
+        constexpr uint32_t kIdescS = tc_idesc_f16(kTcRows, kTcKv, false);
+        constexpr uint32_t kIdescPV = tc_idesc_f16(kTcRows, D, true);
+        const uint32_t q_addr = sbase + Lay::kQ, p_addr = sbase + Lay::kP;
+        auto issue_pv = [&](int i) -> bool {
+            if (!tc_wait_warp(&bar[kBarPFull], i & 1, abort)) return false;
+            if (!tc_wait_warp(&bar[kBarFullV + i % kTcStages], (i / kTcStages) & 1, abort)) return false;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t v_addr = sbase + Lay::kStage0 + (i % kTcStages) * Lay::kStageBytes + 2 * Lay::kHalf;
+#pragma unroll
+                for (int kt = 0; kt < kTcKv / 16; ++kt) {
+                    const uint64_t a = sw128_desc(p_addr + (kt >> 2) * Lay::kHalf + (kt & 3) * 32, 16, 1024);
+                    const uint64_t b = sw128_desc(v_addr + kt * 16 * 128, Lay::kHalf, 1024);
+                    tc_mma_f16(tmem + 256, a, b, kIdescPV, (i > 0 || kt > 0) ? 1u : 0u);
+                }
+                tc_commit(&bar[kBarEmpty + i % kTcStages]);
+                tc_commit(&bar[kBarOReady]);
+            }
+            __syncwarp();
+            return true;
+        };
+        bool ok = tc_wait_warp(&bar[kBarQ], 0, abort);
+        int j = 0;
+        for (; ok && j < n_kv; ++j) {
+            const int st = j % kTcStages;
+            ok = tc_wait_warp(&bar[kBarFullK + st], (j / kTcStages) & 1, abort);
+            if (ok && j >= 2) ok = tc_wait_warp(&bar[kBarSFree + (j & 1)], ((j - 2) >> 1) & 1, abort);
+            if (!ok) break;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t k_addr = sbase + Lay::kStage0 + st * Lay::kStageBytes;
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint64_t a = sw128_desc(q_addr + (ks >> 2) * Lay::kHalf + (ks & 3) * 32, 16, 1024);
+                    const uint64_t b = sw128_desc(k_addr + (ks >> 2) * Lay::kHalf + (ks & 3) * 32, 16, 1024);
+                    tc_mma_f16(tmem + (j & 1) * kTcKv, a, b, kIdescS, ks > 0 ? 1u : 0u);
+                }
+                tc_commit(&bar[kBarSFull + (j & 1)]);
+            }
+            __syncwarp();
+            if (j >= 1) ok = issue_pv(j - 1);
+        }
+        if (ok) issue_pv(n_kv - 1);
+        // every MMA issued above completes before the tensor memory is freed
+        if (lane == 0) tc_commit(&bar[kBarDone]);
+        __syncwarp();
+        mbar_wait(&bar[kBarDone], 0);
+        tc_fence_before();
+        asm volatile("bar.sync 2, 160;" ::: "memory");
+        tc_fence_after();
+        tmem_dealloc(tmem, kTcTmemCols);
+        return;
+    }
+
+    // -------------------------------------------------------------- softmax
+    const int t = threadIdx.x;  // row of the tile = tensor-memory lane
+    const int rl = r0 + t;
+    const bool valid = rl < n;
+    const int lim = valid ? base + rl + 1 : 0;  // tokens 0 .. lim-1 are visible
+    {
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.query + ((size_t)(q_begin + (valid ? rl : 0)) * p.num_heads + h) * D);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            const uint4 v = valid ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+            st_shared_v4(tc_chunk(sbase + Lay::kQ, t, c), v);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[kBarQ]);
+    }
+    const float c2 = p.qk_scale_log2;  // > 0 on this path
+    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+        const int st = j % kTcStages;
+        if (!tc_wait_warp(&bar[kBarSFull + (j & 1)], (j >> 1) & 1, abort)) { ok = false; break; }
+        tc_fence_after();
+        float sv[kTcKv];
+#pragma unroll
+        for (int q = 0; q < kTcKv / 32; ++q) {
+            float v32[32];
+            tmem_ld32(tl + (j & 1) * kTcKv + q * 32, v32);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sv[q * 32 + i] = v32[i];
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[kBarSFree + (j & 1)]);
+
+        const int t0 = j * kTcKv;
+        if (t0 + kTcKv > lim) {
+#pragma unroll
+            for (int k = 0; k < kTcKv; ++k)
+                if (t0 + k >= lim) sv[k] = -INFINITY;
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < kTcKv; ++k) mx = fmaxf(mx, sv[k]);
+        mx *= c2;
+        float alpha = 1.f;
+        bool resc = false;
+        if (mx > m_ref + 8.f) {  // the reference maximum moves only by more than 2^8
+            alpha = fast_exp2(m_ref - mx);
+            m_ref = mx;
+            resc = true;
+        }
+        const float mr = m_ref == -INFINITY ? 0.f : m_ref;
+        uint32_t pk[kTcKv / 2];
+        float rs = 0.f;
+#pragma unroll
+        for (int k = 0; k < kTcKv / 2; ++k) {
+            const float p0 = fast_exp2(fmaf(sv[2 * k], c2, -mr));
+            const float p1 = fast_exp2(fmaf(sv[2 * k + 1], c2, -mr));
+            rs += p0 + p1;
+            pk[k] = pack_half2(p0, p1);
+        }
+        l = l * alpha + rs;
+
+        // P.V of tile j-1 done: the P buffer is free and O is current
+        if (j >= 1) {
+            if (!tc_wait_warp(&bar[kBarOReady], (j - 1) & 1, abort)) { ok = false; break; }
+            tc_fence_after();
+            if (__any_sync(0xffffffffu, resc)) {
+#pragma unroll
+                for (int q = 0; q < D / 32; ++q) {
+                    float ov[32];
+                    tmem_ld32(tl + 256 + q * 32, ov);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+                    tmem_st32(tl + 256 + q * 32, ov);
+                }
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+            st_shared_v4(tc_chunk(sbase + Lay::kP, t, c),
+                         make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]));
+        // tokens at or after the sequence end are unused cache slots (any
+        // bits, NaN included): their V rows enter P.V as zeros
+        if (t0 + kTcKv > L) {
+            if (!tc_wait_warp(&bar[kBarFullV + st], (j / kTcStages) & 1, abort)) { ok = false; break; }
+            if (t0 + t >= L) {
+                const uint32_t v_addr = sbase + Lay::kStage0 + st * Lay::kStageBytes + 2 * Lay::kHalf;
+#pragma unroll
+                for (int c = 0; c < 16; ++c) st_shared_v4(tc_chunk(v_addr, t, c), make_uint4(0, 0, 0, 0));
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[kBarPFull]);
+    }
+    if (ok && tc_wait_warp(&bar[kBarOReady], (n_kv - 1) & 1, abort)) {
+        tc_fence_after();
+        const float inv = valid ? 1.0f / l : 0.f;
+        __half *op = p.out + ((size_t)(q_begin + (valid ? rl : 0)) * p.num_heads + h) * D;
+#pragma unroll
+        for (int q = 0; q < D / 32; ++q) {
+            float ov[32];
+            tmem_ld32(tl + 256 + q * 32, ov);
+            if (valid) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint4 v = make_uint4(pack_half2(ov[8 * c] * inv, ov[8 * c + 1] * inv),
+                                               pack_half2(ov[8 * c + 2] * inv, ov[8 * c + 3] * inv),
+                                               pack_half2(ov[8 * c + 4] * inv, ov[8 * c + 5] * inv),
+                                               pack_half2(ov[8 * c + 6] * inv, ov[8 * c + 7] * inv));
+                    *reinterpret_cast<uint4 *>(op + q * 32 + c * 8) = v;
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    asm volatile("bar.sync 2, 160;" ::: "memory");
+}
+
+}  // namespace pa

@@ -1,10 +1,12 @@
 """GPU parity of the paged prefill against the CPU oracle.
 
 Bars: prefill slots and the chunk's cache write bit-exact; attention within
-max-abs 2e-3 (fp16 cache, the decode's bar: Q pre-scaled and P rounded to
-fp16, fp32 accumulation). Full sizes are checked on sampled (row, head)
-pairs that include every sequence's first and last rows and the rows on
-both sides of each 64-row tile edge.
+max-abs 2e-3 (fp16 cache, the decode's bar: fp16 operands with P rounded to
+fp16, fp32 accumulation). head_size 128 runs on the tcgen05 kernel (128-row
+tiles), head_size 64 and scales <= 0 on the mma.sync kernel (64-row tiles).
+Full sizes are checked on sampled (row, head) pairs that include every
+sequence's first and last rows and the rows on both sides of each 64-row
+tile edge.
 """
 import numpy as np
 import pytest
@@ -184,3 +186,13 @@ def test_prefill_is_deterministic(cuda_device):
     pk.paged_prefill(dp.out, dp.query, dp.query_start, dp.key_cache, dp.value_cache, dp.block_tables,
                      dp.context_lens, mql, w.scale)
     assert torch.equal(first, dp.out)
+
+
+def test_non_positive_scale(cuda_device):
+    # a scale <= 0 (a degenerate but valid input) is computed on the warp-MMA path
+    w = ragged_prefill(128, 32, seed=6)
+    for sc in (-w.scale, 0.0):
+        w.scale = sc
+        dp = run_prefill(w, cuda_device)
+        assert pk.check_status() == 0
+        check(w, dp)
