@@ -1018,6 +1018,7 @@ extern "C" int pa_paged_prefill(void *out, const void *query, const int32_t *que
     p.num_blocks = cache.num_blocks;
     p.max_blocks_per_seq = max_blocks_per_seq;
     p.max_query_len = max_query_len;
+    p.row_tiles = (int)row_tiles;
     p.stages = prefill_stages(cache);
     p.qk_scale_log2 = scale * pa::kLog2e;
     // ring (or tcgen05 tiles) + barriers + 1 KiB to align to 1024 bytes in the kernel

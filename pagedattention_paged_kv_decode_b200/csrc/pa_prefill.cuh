@@ -27,6 +27,7 @@ struct PrefillParams {
     int num_blocks;
     int max_blocks_per_seq;
     int max_query_len;
+    int row_tiles;                // ceil(max_query_len / rows per CTA): grid = row_tiles * S * H
     int stages;
     float qk_scale_log2;          // scale * log2(e)
 };
@@ -68,8 +69,9 @@ __global__ void prefill_slot_mapping_kernel(int32_t *__restrict__ slot_mapping,
 // sequence. Consumer warp w takes rows 16w .. 16w+15 of the tile (MmaRows);
 // the producer warp streams the K/V blocks 0 .. (last row's position) / B of
 // the sequence through a ring of TMA half tiles. Tiles are numbered from the
-// end of each sequence, so the CTAs with the longest causal range launch
-// first. A warp whose rows all end before a tile only passes the tile on.
+// end of each sequence, so within a (sequence, head) the CTAs with the
+// longest causal range launch first. A warp whose rows all end before a
+// tile only passes the tile on.
 template <int D, int B>
 __global__ void __launch_bounds__(32 * 5, 1)
 paged_prefill_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
@@ -83,10 +85,12 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
     uint64_t *empty = full + stages;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    const int h = blockIdx.x % p.num_heads;
-    const int rest = blockIdx.x / p.num_heads;
-    const int s = rest % p.num_seqs;
-    const int t_rev = rest / p.num_seqs;
+    // the row tiles of one (sequence, head) are neighbours in the grid, so
+    // they run together and share its K/V blocks through L2
+    const int t_rev = blockIdx.x % p.row_tiles;
+    const int sh = blockIdx.x / p.row_tiles;
+    const int h = sh % p.num_heads;
+    const int s = sh / p.num_heads;
     const int q_begin = __ldg(p.query_start + s);
     const int n = __ldg(p.query_start + s + 1) - q_begin;
     const int L = __ldg(p.context_lens + s);
@@ -298,10 +302,12 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     // ---- the CTA's rows (uniform; every early exit precedes any barrier)
-    const int h = blockIdx.x % p.num_heads;
-    const int rest = blockIdx.x / p.num_heads;
-    const int s = rest % p.num_seqs;
-    const int t_rev = rest / p.num_seqs;
+    // the row tiles of one (sequence, head) are neighbours in the grid, so
+    // they run together and share its K/V blocks through L2
+    const int t_rev = blockIdx.x % p.row_tiles;
+    const int sh = blockIdx.x / p.row_tiles;
+    const int h = sh % p.num_heads;
+    const int s = sh / p.num_heads;
     const int q_begin = __ldg(p.query_start + s);
     const int n = __ldg(p.query_start + s + 1) - q_begin;
     const int L = __ldg(p.context_lens + s);
