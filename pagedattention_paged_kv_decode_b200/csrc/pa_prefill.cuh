@@ -214,39 +214,45 @@ namespace pa {
 //                     into shared memory (128-byte swizzle)
 //   O += P_j . V_j    eight tcgen05.mma into the O columns of tensor memory,
 //                     V read N-contiguous (MN-major)
-// Warps: 0-3 softmax (and Q staging, epilogue), 4 TMA producer, 5 MMA issuer
-// (also allocates the 512 tensor-memory columns). Every wait is bounded; a
-// wait that runs out sets PA_DEV_WAIT_TIMEOUT and an abort flag that ends
-// the other roles' waits, and the CTA still drains its copies and MMAs and
-// frees its tensor memory before it exits.
+// K and V have rings of their own (3 and 2 tiles): a K tile is released as
+// soon as its S is computed, a V tile when its P.V is, so each is reloaded
+// as early as possible. Warps: 0-3 softmax (and Q staging, epilogue), 4 K
+// producer, 5 MMA issuer (also allocates the 512 tensor-memory columns), 6 V
+// producer. Each producer keeps the next 32 block-table entries in flight.
+// Every wait is bounded; a wait that runs out sets PA_DEV_WAIT_TIMEOUT and
+// an abort flag that ends the other roles' waits, and the CTA still drains
+// its copies and MMAs and frees its tensor memory before it exits.
 constexpr int kTcRows = 128;
 constexpr int kTcKv = 128;
-constexpr int kTcStages = 2;
-constexpr int kTcThreads = 192;
+constexpr int kTcKStages = 3;
+constexpr int kTcVStages = 2;
+constexpr int kTcThreads = 224;
 constexpr int kTcTmemCols = 512;  // S0 [0,128), S1 [128,256), O [256,384)
 
 struct TcLayout {                                       // byte offsets from the 1024-aligned base
     static constexpr uint32_t kHalf = 128 * 128;         // [128 rows][128 B]: one 64-wide half
-    static constexpr uint32_t kQ = 0;                    // Q: 2 halves (dims 0-63, 64-127)
-    static constexpr uint32_t kStage0 = 2 * kHalf;       // stage s: K (2 halves), then V (2 halves)
-    static constexpr uint32_t kStageBytes = 4 * kHalf;
-    static constexpr uint32_t kP = kStage0 + kTcStages * kStageBytes;  // P: 2 halves (tokens 0-63, 64-127)
-    static constexpr uint32_t kBars = kP + 2 * kHalf;
-    static constexpr uint32_t kBytes = kBars + 128;
+    static constexpr uint32_t kTile = 2 * kHalf;         // a 128 x 128 fp16 tile in two halves
+    static constexpr uint32_t kQ = 0;                    // Q (dims 0-63, 64-127)
+    static constexpr uint32_t kK = kQ + kTile;           // K ring
+    static constexpr uint32_t kV = kK + kTcKStages * kTile;  // V ring
+    static constexpr uint32_t kP = kV + kTcVStages * kTile;  // P (tokens 0-63, 64-127)
+    static constexpr uint32_t kBars = kP + kTile;
+    static constexpr uint32_t kBytes = kBars + 256;
 };
 
 // mbarrier indices
 enum : int {
-    kBarQ = 0,                   // Q staged (4 softmax warps)
-    kBarFullK = 1,               // + stage: K tile landed (TMA bytes)
-    kBarFullV = 3,               // + stage: V tile landed
-    kBarEmpty = 5,               // + stage: P.V of the stage's tile done (commit)
-    kBarSFull = 7,               // + buffer: S ready (commit)
-    kBarSFree = 9,               // + buffer: S read by the 4 softmax warps
-    kBarPFull = 11,              // P written, O corrected (4 softmax warps)
-    kBarOReady = 12,             // P.V done (commit)
-    kBarDone = 13,               // every MMA of the CTA done (commit)
-    kNumBars = 14
+    kBarQ = 0,                              // Q staged (4 softmax warps)
+    kBarFullK = 1,                          // + stage: K tile landed (TMA bytes)
+    kBarEmptyK = kBarFullK + kTcKStages,    // + stage: S of the stage's tile done (commit)
+    kBarFullV = kBarEmptyK + kTcKStages,    // + stage: V tile landed
+    kBarEmptyV = kBarFullV + kTcVStages,    // + stage: P.V of the stage's tile done (commit)
+    kBarSFull = kBarEmptyV + kTcVStages,    // + buffer: S ready (commit)
+    kBarSFree = kBarSFull + 2,              // + buffer: S read by the 4 softmax warps
+    kBarPFull = kBarSFree + 2,              // P written, O corrected (4 softmax warps)
+    kBarOReady = kBarPFull + 1,             // P.V done (commit)
+    kBarDone = kBarOReady + 1,              // every MMA of the CTA done (commit)
+    kNumBars = kBarDone + 1
 };
 
 // Bounded wait that also ends when another role has aborted.
@@ -286,12 +292,60 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
                  : "memory");
 }
 
+// One producer warp: streams the K (or V) tiles 0 .. n_kv-1 of the CTA
+// through its ring. Lane b < BPT loads cache block b of each tile; lane l
+// holds block-table entry 32c + l of the current chunk c while the next
+// chunk's entries are already being read.
+template <int B, int STAGES>
+__device__ __forceinline__ void tc_produce(const CUtensorMap *tmap, unsigned char *ring, uint64_t *full,
+                                           uint64_t *empty, const int32_t *table, int nblk, int n_kv, int h,
+                                           int num_blocks, volatile int *abort, int lane) {
+    constexpr int BPT = kTcKv / B;
+    const uint64_t policy = l2_policy_evict_normal();  // other row tiles re-read these blocks
+    auto fetch = [&](int chunk) {
+        const int lb = chunk * 32 + lane;
+        return lb < nblk ? __ldg(table + lb) : -1;
+    };
+    int cur = fetch(0), nxt = fetch(1);
+    int issued = 0;
+    for (int j = 0; j < n_kv; ++j) {
+        const int st = j % STAGES, use = j / STAGES;
+        const int lb0 = j * BPT;  // first block of the tile; tiles never straddle a chunk (BPT divides 32)
+        if (lb0 > 0 && (lb0 & 31) == 0) {
+            cur = nxt;
+            nxt = fetch((lb0 >> 5) + 1);
+        }
+        int blk = __shfl_sync(0xffffffffu, cur, (lb0 & 31) + (lane < BPT ? lane : 0));
+        if (lane < BPT) {
+            if (lb0 + lane >= nblk) {
+                blk = num_blocks;  // past the sequence: zero filled
+            } else if (blk < 0 || blk >= num_blocks) {
+                flag_error(PA_DEV_BAD_BLOCK);
+                blk = num_blocks;
+            }
+        }
+        bool ok = true;
+        if (lane == 0 && use > 0) ok = tc_wait(&empty[st], (use - 1) & 1, abort);
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+        if (lane == 0) mbar_arrive_expect_tx(&full[st], (uint32_t)TcLayout::kTile);
+        __syncwarp();
+        if (lane < BPT) {
+            unsigned char *dst = ring + st * TcLayout::kTile + lane * B * 128;
+            tma_load_4d(dst, tmap, &full[st], 0, h, 0, blk, policy);
+            tma_load_4d(dst + TcLayout::kHalf, tmap, &full[st], 64, h, 0, blk, policy);
+        }
+        issued = j + 1;
+    }
+    // let the copies in flight land before the warp retires
+    if (lane == 0)
+        for (int j = max(0, issued - STAGES); j < issued; ++j) mbar_wait(&full[j % STAGES], (j / STAGES) & 1);
+}
+
 template <int B>
 __global__ void __launch_bounds__(kTcThreads, 1)
 paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                         const PrefillParams p) {
     constexpr int D = 128;
-    constexpr int BPT = kTcKv / B;  // cache blocks per K/V tile
     using Lay = TcLayout;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -301,9 +355,9 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
     const uint32_t sbase = smem_u32(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // ---- the CTA's rows (uniform; every early exit precedes any barrier)
-    // the row tiles of one (sequence, head) are neighbours in the grid, so
-    // they run together and share its K/V blocks through L2
+    // ---- the CTA's rows (uniform; every early exit precedes any barrier).
+    // The row tiles of one (sequence, head) are neighbours in the grid, so
+    // they run together and share its K/V blocks through L2.
     const int t_rev = blockIdx.x % p.row_tiles;
     const int sh = blockIdx.x / p.row_tiles;
     const int h = sh % p.num_heads;
@@ -338,8 +392,8 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
     if (warp == 4 && lane == 0) {
         prefetch_tensor_map(&tmap_k);
         prefetch_tensor_map(&tmap_v);
-        const uint32_t counts[kNumBars] = {4, 1, 1, 1, 1, 1, 1, 1, 1, 4, 4, 4, 1, 1};
-        for (int i = 0; i < kNumBars; ++i) mbar_init(&bar[i], counts[i]);
+        for (int i = 0; i < kNumBars; ++i)
+            mbar_init(&bar[i], (i == kBarQ || i == kBarSFree || i == kBarSFree + 1 || i == kBarPFull) ? 4 : 1);
         *abort = 0;
         fence_mbar_init();
     }
@@ -349,47 +403,13 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 4) {
-        // ---------------------------------------------------------- producer
-        const uint64_t policy = l2_policy_evict_normal();  // other row tiles re-read these blocks
-        int issued = 0;
-        for (int j = 0; j < n_kv; ++j) {
-            const int st = j % kTcStages, use = j / kTcStages;
-            int blk = p.num_blocks;  // past the sequence: zero filled
-            const int lb = j * BPT + lane;
-            if (lane < BPT && lb < nblk) {
-                const int b = __ldg(table + lb);
-                if (b < 0 || b >= p.num_blocks)
-                    flag_error(PA_DEV_BAD_BLOCK);
-                else
-                    blk = b;
-            }
-            bool ok = true;
-            if (lane == 0 && use > 0) ok = tc_wait(&bar[kBarEmpty + st], (use - 1) & 1, abort);
-            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&bar[kBarFullK + st], (uint32_t)(kTcKv * D * 2));
-                mbar_arrive_expect_tx(&bar[kBarFullV + st], (uint32_t)(kTcKv * D * 2));
-            }
-            __syncwarp();
-            if (lane < BPT) {
-                unsigned char *kdst = smem + Lay::kStage0 + st * Lay::kStageBytes + lane * B * 128;
-                unsigned char *vdst = kdst + 2 * Lay::kHalf;
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    tma_load_4d(kdst + hf * Lay::kHalf, &tmap_k, &bar[kBarFullK + st], 64 * hf, h, 0, blk, policy);
-                    tma_load_4d(vdst + hf * Lay::kHalf, &tmap_v, &bar[kBarFullV + st], 64 * hf, h, 0, blk, policy);
-                }
-            }
-            issued = j + 1;
-        }
-        // let the copies in flight land before the warp retires
-        if (lane == 0) {
-            for (int j = max(0, issued - kTcStages); j < issued; ++j) {
-                const int st = j % kTcStages, use = j / kTcStages;
-                mbar_wait(&bar[kBarFullK + st], use & 1);
-                mbar_wait(&bar[kBarFullV + st], use & 1);
-            }
-        }
+        tc_produce<B, kTcKStages>(&tmap_k, smem + Lay::kK, &bar[kBarFullK], &bar[kBarEmptyK], table, nblk, n_kv, h,
+                                  p.num_blocks, abort, lane);
+        return;
+    }
+    if (warp == 6) {
+        tc_produce<B, kTcVStages>(&tmap_v, smem + Lay::kV, &bar[kBarFullV], &bar[kBarEmptyV], table, nblk, n_kv, h,
+                                  p.num_blocks, abort, lane);
         return;
     }
 
@@ -399,18 +419,19 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
         constexpr uint32_t kIdescPV = tc_idesc_f16(kTcRows, D, true);
         const uint32_t q_addr = sbase + Lay::kQ, p_addr = sbase + Lay::kP;
         auto issue_pv = [&](int i) -> bool {
+            const int st = i % kTcVStages;
             if (!tc_wait_warp(&bar[kBarPFull], i & 1, abort)) return false;
-            if (!tc_wait_warp(&bar[kBarFullV + i % kTcStages], (i / kTcStages) & 1, abort)) return false;
+            if (!tc_wait_warp(&bar[kBarFullV + st], (i / kTcVStages) & 1, abort)) return false;
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t v_addr = sbase + Lay::kStage0 + (i % kTcStages) * Lay::kStageBytes + 2 * Lay::kHalf;
+                const uint32_t v_addr = sbase + Lay::kV + st * Lay::kTile;
 #pragma unroll
                 for (int kt = 0; kt < kTcKv / 16; ++kt) {
                     const uint64_t a = sw128_desc(p_addr + (kt >> 2) * Lay::kHalf + (kt & 3) * 32, 16, 1024);
                     const uint64_t b = sw128_desc(v_addr + kt * 16 * 128, Lay::kHalf, 1024);
                     tc_mma_f16(tmem + 256, a, b, kIdescPV, (i > 0 || kt > 0) ? 1u : 0u);
                 }
-                tc_commit(&bar[kBarEmpty + i % kTcStages]);
+                tc_commit(&bar[kBarEmptyV + st]);
                 tc_commit(&bar[kBarOReady]);
             }
             __syncwarp();
@@ -419,13 +440,13 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
         bool ok = tc_wait_warp(&bar[kBarQ], 0, abort);
         int j = 0;
         for (; ok && j < n_kv; ++j) {
-            const int st = j % kTcStages;
-            ok = tc_wait_warp(&bar[kBarFullK + st], (j / kTcStages) & 1, abort);
+            const int st = j % kTcKStages;
+            ok = tc_wait_warp(&bar[kBarFullK + st], (j / kTcKStages) & 1, abort);
             if (ok && j >= 2) ok = tc_wait_warp(&bar[kBarSFree + (j & 1)], ((j - 2) >> 1) & 1, abort);
             if (!ok) break;
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t k_addr = sbase + Lay::kStage0 + st * Lay::kStageBytes;
+                const uint32_t k_addr = sbase + Lay::kK + st * Lay::kTile;
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
                     const uint64_t a = sw128_desc(q_addr + (ks >> 2) * Lay::kHalf + (ks & 3) * 32, 16, 1024);
@@ -433,6 +454,7 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
                     tc_mma_f16(tmem + (j & 1) * kTcKv, a, b, kIdescS, ks > 0 ? 1u : 0u);
                 }
                 tc_commit(&bar[kBarSFull + (j & 1)]);
+                tc_commit(&bar[kBarEmptyK + st]);
             }
             __syncwarp();
             if (j >= 1) ok = issue_pv(j - 1);
@@ -470,7 +492,6 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
-        const int st = j % kTcStages;
         if (!tc_wait_warp(&bar[kBarSFull + (j & 1)], (j >> 1) & 1, abort)) { ok = false; break; }
         tc_fence_after();
         float sv[kTcKv];
@@ -536,9 +557,10 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
         // tokens at or after the sequence end are unused cache slots (any
         // bits, NaN included): their V rows enter P.V as zeros
         if (t0 + kTcKv > L) {
-            if (!tc_wait_warp(&bar[kBarFullV + st], (j / kTcStages) & 1, abort)) { ok = false; break; }
+            const int sv_st = j % kTcVStages;
+            if (!tc_wait_warp(&bar[kBarFullV + sv_st], (j / kTcVStages) & 1, abort)) { ok = false; break; }
             if (t0 + t >= L) {
-                const uint32_t v_addr = sbase + Lay::kStage0 + st * Lay::kStageBytes + 2 * Lay::kHalf;
+                const uint32_t v_addr = sbase + Lay::kV + sv_st * Lay::kTile;
 #pragma unroll
                 for (int c = 0; c < 16; ++c) st_shared_v4(tc_chunk(v_addr, t, c), make_uint4(0, 0, 0, 0));
             }
