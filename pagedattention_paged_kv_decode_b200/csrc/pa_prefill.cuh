@@ -255,16 +255,16 @@ enum : int {
     kNumBars = kBarDone + 1
 };
 
-// Bounded wait that also ends when another role has aborted.
+// Bounded wait that also ends when another role has aborted. It spins on
+// the non-blocking test (these waits are short and on the critical path,
+// where a suspended thread would wake up late).
 __device__ __forceinline__ bool tc_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
-#pragma unroll 1
-    for (int i = 0; i < 64; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_test_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
 #pragma unroll 1
-        for (int i = 0; i < 32; ++i)
-            if (mbar_try_wait(bar, parity)) return true;
+        for (int i = 0; i < 64; ++i)
+            if (mbar_test_wait(bar, parity)) return true;
         if (*abort) return false;
         if (global_timer_ns() - t0 > kWaitLimitNs) {
             flag_error(PA_DEV_WAIT_TIMEOUT);
@@ -417,20 +417,25 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
         // ---------------------------------------------------------- MMA issuer
         constexpr uint32_t kIdescS = tc_idesc_f16(kTcRows, kTcKv, false);
         constexpr uint32_t kIdescPV = tc_idesc_f16(kTcRows, D, true);
-        const uint32_t q_addr = sbase + Lay::kQ, p_addr = sbase + Lay::kP;
+        // K-major operands (Q, K, P): 8-row groups 1024 B apart; V: MN-major,
+        // the two 64-dim halves kHalf apart, 8-token groups 1024 B apart. A
+        // k-step moves the start address (descriptor bits 0-13, in 16 B).
+        const uint64_t dq = sw128_desc(sbase + Lay::kQ, 16, 1024);
+        const uint64_t dp = sw128_desc(sbase + Lay::kP, 16, 1024);
+        const uint64_t dk = sw128_desc(sbase + Lay::kK, 16, 1024);
+        const uint64_t dv = sw128_desc(sbase + Lay::kV, Lay::kHalf, 1024);
+        auto kstep = [](int k) { return (uint64_t)(((k >> 2) * Lay::kHalf + (k & 3) * 32) >> 4); };
         auto issue_pv = [&](int i) -> bool {
             const int st = i % kTcVStages;
             if (!tc_wait_warp(&bar[kBarPFull], i & 1, abort)) return false;
             if (!tc_wait_warp(&bar[kBarFullV + st], (i / kTcVStages) & 1, abort)) return false;
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t v_addr = sbase + Lay::kV + st * Lay::kTile;
+                const uint64_t dvs = dv + ((st * Lay::kTile) >> 4);
 #pragma unroll
-                for (int kt = 0; kt < kTcKv / 16; ++kt) {
-                    const uint64_t a = sw128_desc(p_addr + (kt >> 2) * Lay::kHalf + (kt & 3) * 32, 16, 1024);
-                    const uint64_t b = sw128_desc(v_addr + kt * 16 * 128, Lay::kHalf, 1024);
-                    tc_mma_f16(tmem + 256, a, b, kIdescPV, (i > 0 || kt > 0) ? 1u : 0u);
-                }
+                for (int kt = 0; kt < kTcKv / 16; ++kt)
+                    tc_mma_f16(tmem + 256, dp + kstep(kt), dvs + ((kt * 16 * 128) >> 4), kIdescPV,
+                               (i > 0 || kt > 0) ? 1u : 0u);
                 tc_commit(&bar[kBarEmptyV + st]);
                 tc_commit(&bar[kBarOReady]);
             }
@@ -446,13 +451,10 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
             if (!ok) break;
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t k_addr = sbase + Lay::kK + st * Lay::kTile;
+                const uint64_t dks = dk + ((st * Lay::kTile) >> 4);
 #pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint64_t a = sw128_desc(q_addr + (ks >> 2) * Lay::kHalf + (ks & 3) * 32, 16, 1024);
-                    const uint64_t b = sw128_desc(k_addr + (ks >> 2) * Lay::kHalf + (ks & 3) * 32, 16, 1024);
-                    tc_mma_f16(tmem + (j & 1) * kTcKv, a, b, kIdescS, ks > 0 ? 1u : 0u);
-                }
+                for (int ks = 0; ks < D / 16; ++ks)
+                    tc_mma_f16(tmem + (j & 1) * kTcKv, dq + kstep(ks), dks + kstep(ks), kIdescS, ks > 0 ? 1u : 0u);
                 tc_commit(&bar[kBarSFull + (j & 1)]);
                 tc_commit(&bar[kBarEmptyK + st]);
             }
@@ -512,9 +514,15 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
             for (int k = 0; k < kTcKv; ++k)
                 if (t0 + k >= lim) sv[k] = -INFINITY;
         }
-        float mx = -INFINITY;
+        float mx;
+        {  // tree reduction: short dependence chains
+            float m8[8];
 #pragma unroll
-        for (int k = 0; k < kTcKv; ++k) mx = fmaxf(mx, sv[k]);
+            for (int i = 0; i < 8; ++i) m8[i] = sv[i];
+#pragma unroll
+            for (int k = 8; k < kTcKv; ++k) m8[k & 7] = fmaxf(m8[k & 7], sv[k]);
+            mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        }
         mx *= c2;
         float alpha = 1.f;
         bool resc = false;
@@ -525,15 +533,15 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
         }
         const float mr = m_ref == -INFINITY ? 0.f : m_ref;
         uint32_t pk[kTcKv / 2];
-        float rs = 0.f;
+        float rs4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int k = 0; k < kTcKv / 2; ++k) {
             const float p0 = fast_exp2(fmaf(sv[2 * k], c2, -mr));
             const float p1 = fast_exp2(fmaf(sv[2 * k + 1], c2, -mr));
-            rs += p0 + p1;
+            rs4[k & 3] += p0 + p1;
             pk[k] = pack_half2(p0, p1);
         }
-        l = l * alpha + rs;
+        l = l * alpha + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
 
         // P.V of tile j-1 done: the P buffer is free and O is current
         if (j >= 1) {
