@@ -241,6 +241,22 @@ __host__ __device__ constexpr uint32_t tc_idesc_f16(int M, int N, bool b_mn) {
            | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// One fp32 column of this thread's tensor-memory lane (store / load, waited).
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, float v) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};\n\ttcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+                 "r"(__float_as_uint(v))
+                 : "memory");
+}
+
+__device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
+    uint32_t r;
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];\n\ttcgen05.wait::ld.sync.aligned;"
+                 : "=r"(r)
+                 : "r"(taddr)
+                 : "memory");
+    return __uint_as_float(r);
+}
+
 // 32 consecutive fp32 columns of this thread's tensor-memory lane (the warp
 // reads lanes 32 (warp % 4) .. + 31), waited for before returning.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {

@@ -216,9 +216,12 @@ namespace pa {
 //                     V read N-contiguous (MN-major)
 // K and V have rings of their own (3 and 2 tiles): a K tile is released as
 // soon as its S is computed, a V tile when its P.V is, so each is reloaded
-// as early as possible. Warps: 0-3 softmax (and Q staging, epilogue), 4 K
-// producer, 5 MMA issuer (also allocates the 512 tensor-memory columns), 6 V
-// producer. Each producer keeps the next 32 block-table entries in flight.
+// as early as possible. Warps: 0-7 softmax (and Q staging, epilogue): warp
+// w takes rows 32 (w % 4) .. + 31 (its tensor-memory lanes) and columns
+// 64 (w / 4) .. + 63 of S, P and O, the two halves of a row exchanging their
+// maxima and sums through tensor memory; 8 K producer; 9 MMA issuer (also
+// allocates the 512 tensor-memory columns); 10 V producer. Each producer
+// keeps the next 32 block-table entries in flight.
 // Every wait is bounded; a wait that runs out sets PA_DEV_WAIT_TIMEOUT and
 // an abort flag that ends the other roles' waits, and the CTA still drains
 // its copies and MMAs and frees its tensor memory before it exits.
@@ -226,8 +229,11 @@ constexpr int kTcRows = 128;
 constexpr int kTcKv = 128;
 constexpr int kTcKStages = 3;
 constexpr int kTcVStages = 2;
-constexpr int kTcThreads = 224;
-constexpr int kTcTmemCols = 512;  // S0 [0,128), S1 [128,256), O [256,384)
+constexpr int kTcThreads = 352;
+constexpr int kTcSoftmaxWarps = 8;  // two per tensor-memory lane quadrant, one per half row
+constexpr int kTcWarpK = 8, kTcWarpMma = 9, kTcWarpV = 10;
+constexpr int kTcTmemCols = 512;  // S0 [0,128), S1 [128,256), O [256,384), row exchange [384,390)
+constexpr int kTcColX = 384;      // + 2 * tile parity + half: row maxima; + 4 + half: row sums
 
 struct TcLayout {                                       // byte offsets from the 1024-aligned base
     static constexpr uint32_t kHalf = 128 * 128;         // [128 rows][128 B]: one 64-wide half
@@ -242,17 +248,19 @@ struct TcLayout {                                       // byte offsets from the
 
 // mbarrier indices
 enum : int {
-    kBarQ = 0,                              // Q staged (4 softmax warps)
+    kBarQ = 0,                              // Q staged (8 softmax warps)
     kBarFullK = 1,                          // + stage: K tile landed (TMA bytes)
     kBarEmptyK = kBarFullK + kTcKStages,    // + stage: S of the stage's tile done (commit)
     kBarFullV = kBarEmptyK + kTcKStages,    // + stage: V tile landed
     kBarEmptyV = kBarFullV + kTcVStages,    // + stage: P.V of the stage's tile done (commit)
     kBarSFull = kBarEmptyV + kTcVStages,    // + buffer: S ready (commit)
-    kBarSFree = kBarSFull + 2,              // + buffer: S read by the 4 softmax warps
-    kBarPFull = kBarSFree + 2,              // P written, O corrected (4 softmax warps)
+    kBarSFree = kBarSFull + 2,              // + buffer: S read by the 8 softmax warps
+    kBarPFull = kBarSFree + 2,              // P written, O corrected (8 softmax warps)
     kBarOReady = kBarPFull + 1,             // P.V done (commit)
     kBarDone = kBarOReady + 1,              // every MMA of the CTA done (commit)
-    kNumBars = kBarDone + 1
+    kBarPair = kBarDone + 1,                // + 2 * quadrant + tile parity: both halves' row maxima posted
+    kBarPairEnd = kBarPair + 8,             // + quadrant: both halves' row sums posted
+    kNumBars = kBarPairEnd + 4
 };
 
 // Bounded wait that also ends when another role has aborted. It spins on
@@ -385,15 +393,16 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
     const int32_t *table = p.block_tables + (size_t)s * p.max_blocks_per_seq;
 
     // ---- set-up: tensor memory, barriers
-    if (warp == 5) {
+    if (warp == kTcWarpMma) {
         tmem_alloc(tmem_slot, kTcTmemCols);
         tmem_relinquish();
     }
-    if (warp == 4 && lane == 0) {
+    if (warp == kTcWarpK && lane == 0) {
         prefetch_tensor_map(&tmap_k);
         prefetch_tensor_map(&tmap_v);
         for (int i = 0; i < kNumBars; ++i)
-            mbar_init(&bar[i], (i == kBarQ || i == kBarSFree || i == kBarSFree + 1 || i == kBarPFull) ? 4 : 1);
+            mbar_init(&bar[i], (i == kBarQ || i == kBarSFree || i == kBarSFree + 1 || i == kBarPFull)
+                                   ? kTcSoftmaxWarps : (i >= kBarPair ? 2 : 1));
         *abort = 0;
         fence_mbar_init();
     }
@@ -402,18 +411,18 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 4) {
+    if (warp == kTcWarpK) {
         tc_produce<B, kTcKStages>(&tmap_k, smem + Lay::kK, &bar[kBarFullK], &bar[kBarEmptyK], table, nblk, n_kv, h,
                                   p.num_blocks, abort, lane);
         return;
     }
-    if (warp == 6) {
+    if (warp == kTcWarpV) {
         tc_produce<B, kTcVStages>(&tmap_v, smem + Lay::kV, &bar[kBarFullV], &bar[kBarEmptyV], table, nblk, n_kv, h,
                                   p.num_blocks, abort, lane);
         return;
     }
 
-    if (warp == 5) {
+    if (warp == kTcWarpMma) {
         // ---------------------------------------------------------- MMA issuer
         constexpr uint32_t kIdescS = tc_idesc_f16(kTcRows, kTcKv, false);
         constexpr uint32_t kIdescPV = tc_idesc_f16(kTcRows, D, true);
@@ -467,21 +476,23 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
         __syncwarp();
         mbar_wait(&bar[kBarDone], 0);
         tc_fence_before();
-        asm volatile("bar.sync 2, 160;" ::: "memory");
+        asm volatile("bar.sync 2, %0;" ::"r"(32 * (kTcSoftmaxWarps + 1)) : "memory");
         tc_fence_after();
         tmem_dealloc(tmem, kTcTmemCols);
         return;
     }
 
     // -------------------------------------------------------------- softmax
-    const int t = threadIdx.x;  // row of the tile = tensor-memory lane
+    const int t = (warp & 3) * 32 + lane;  // row of the tile = tensor-memory lane
+    const int hh = warp >> 2;              // half of the row: columns 64 hh .. 64 hh + 63
     const int rl = r0 + t;
     const bool valid = rl < n;
     const int lim = valid ? base + rl + 1 : 0;  // tokens 0 .. lim-1 are visible
+    uint64_t *pair = &bar[kBarPair + 2 * (warp & 3)];  // the two warps sharing these rows
     {
         const uint4 *src = reinterpret_cast<const uint4 *>(p.query + ((size_t)(q_begin + (valid ? rl : 0)) * p.num_heads + h) * D);
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
+        for (int c = 8 * hh; c < 8 * hh + 8; ++c) {
             const uint4 v = valid ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
             st_shared_v4(tc_chunk(sbase + Lay::kQ, t, c), v);
         }
@@ -489,18 +500,19 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar[kBarQ]);
     }
+    constexpr int HC = kTcKv / 2;  // columns per thread
     const float c2 = p.qk_scale_log2;  // > 0 on this path
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
         if (!tc_wait_warp(&bar[kBarSFull + (j & 1)], (j >> 1) & 1, abort)) { ok = false; break; }
         tc_fence_after();
-        float sv[kTcKv];
+        float sv[HC];
 #pragma unroll
-        for (int q = 0; q < kTcKv / 32; ++q) {
+        for (int q = 0; q < HC / 32; ++q) {
             float v32[32];
-            tmem_ld32(tl + (j & 1) * kTcKv + q * 32, v32);
+            tmem_ld32(tl + (j & 1) * kTcKv + hh * HC + q * 32, v32);
 #pragma unroll
             for (int i = 0; i < 32; ++i) sv[q * 32 + i] = v32[i];
         }
@@ -508,10 +520,10 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar[kBarSFree + (j & 1)]);
 
-        const int t0 = j * kTcKv;
-        if (t0 + kTcKv > lim) {
+        const int t0 = j * kTcKv + hh * HC;  // position of this thread's first column
+        if (t0 + HC > lim) {
 #pragma unroll
-            for (int k = 0; k < kTcKv; ++k)
+            for (int k = 0; k < HC; ++k)
                 if (t0 + k >= lim) sv[k] = -INFINITY;
         }
         float mx;
@@ -520,10 +532,19 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
 #pragma unroll
             for (int i = 0; i < 8; ++i) m8[i] = sv[i];
 #pragma unroll
-            for (int k = 8; k < kTcKv; ++k) m8[k & 7] = fmaxf(m8[k & 7], sv[k]);
+            for (int k = 8; k < HC; ++k) m8[k & 7] = fmaxf(m8[k & 7], sv[k]);
             mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
         }
-        mx *= c2;
+        // both halves of the row take the same maximum, exchanged through a
+        // tensor-memory column of the row's lane (columns and barriers by
+        // tile parity: a warp runs at most one tile ahead of its partner)
+        tmem_st1(tl + kTcColX + 2 * (j & 1) + hh, mx);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&pair[j & 1]);
+        if (!tc_wait_warp(&pair[j & 1], (j >> 1) & 1, abort)) { ok = false; break; }
+        tc_fence_after();
+        mx = fmaxf(mx, tmem_ld1(tl + kTcColX + 2 * (j & 1) + (hh ^ 1))) * c2;
         float alpha = 1.f;
         bool resc = false;
         if (mx > m_ref + 8.f) {  // the reference maximum moves only by more than 2^8
@@ -532,16 +553,16 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
             resc = true;
         }
         const float mr = m_ref == -INFINITY ? 0.f : m_ref;
-        uint32_t pk[kTcKv / 2];
+        uint32_t pk[HC / 2];
         float rs4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int k = 0; k < kTcKv / 2; ++k) {
+        for (int k = 0; k < HC / 2; ++k) {
             const float p0 = fast_exp2(fmaf(sv[2 * k], c2, -mr));
             const float p1 = fast_exp2(fmaf(sv[2 * k + 1], c2, -mr));
             rs4[k & 3] += p0 + p1;
             pk[k] = pack_half2(p0, p1);
         }
-        l = l * alpha + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
+        l = l * alpha + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));  // this half's share of the row sum
 
         // P.V of tile j-1 done: the P buffer is free and O is current
         if (j >= 1) {
@@ -549,28 +570,29 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
             tc_fence_after();
             if (__any_sync(0xffffffffu, resc)) {
 #pragma unroll
-                for (int q = 0; q < D / 32; ++q) {
+                for (int q = 0; q < HC / 32; ++q) {
                     float ov[32];
-                    tmem_ld32(tl + 256 + q * 32, ov);
+                    tmem_ld32(tl + 256 + hh * HC + q * 32, ov);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) ov[i] *= alpha;
-                    tmem_st32(tl + 256 + q * 32, ov);
+                    tmem_st32(tl + 256 + hh * HC + q * 32, ov);
                 }
             }
         }
 #pragma unroll
-        for (int c = 0; c < 16; ++c)
-            st_shared_v4(tc_chunk(sbase + Lay::kP, t, c),
+        for (int c = 0; c < 8; ++c)
+            st_shared_v4(tc_chunk(sbase + Lay::kP, t, 8 * hh + c),
                          make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]));
         // tokens at or after the sequence end are unused cache slots (any
         // bits, NaN included): their V rows enter P.V as zeros
-        if (t0 + kTcKv > L) {
-            const int sv_st = j % kTcVStages;
-            if (!tc_wait_warp(&bar[kBarFullV + sv_st], (j / kTcVStages) & 1, abort)) { ok = false; break; }
-            if (t0 + t >= L) {
-                const uint32_t v_addr = sbase + Lay::kV + sv_st * Lay::kTile;
+        const int tt = j * kTcKv;
+        if (tt + kTcKv > L) {
+            const int vst = j % kTcVStages;
+            if (!tc_wait_warp(&bar[kBarFullV + vst], (j / kTcVStages) & 1, abort)) { ok = false; break; }
+            if (tt + t >= L) {
+                const uint32_t v_addr = sbase + Lay::kV + vst * Lay::kTile;
 #pragma unroll
-                for (int c = 0; c < 16; ++c) st_shared_v4(tc_chunk(v_addr, t, c), make_uint4(0, 0, 0, 0));
+                for (int c = 8 * hh; c < 8 * hh + 8; ++c) st_shared_v4(tc_chunk(v_addr, t, c), make_uint4(0, 0, 0, 0));
             }
         }
         fence_proxy_async_smem();
@@ -578,14 +600,24 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar[kBarPFull]);
     }
+    // the row sum is the two halves' shares
+    tmem_st1(tl + kTcColX + 4 + hh, l);
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bar[kBarPairEnd + (warp & 3)]);
+    ok = ok && tc_wait_warp(&bar[kBarPairEnd + (warp & 3)], 0, abort);
+    if (ok) {
+        tc_fence_after();
+        l += tmem_ld1(tl + kTcColX + 4 + (hh ^ 1));
+    }
     if (ok && tc_wait_warp(&bar[kBarOReady], (n_kv - 1) & 1, abort)) {
         tc_fence_after();
         const float inv = valid ? 1.0f / l : 0.f;
-        __half *op = p.out + ((size_t)(q_begin + (valid ? rl : 0)) * p.num_heads + h) * D;
+        __half *op = p.out + ((size_t)(q_begin + (valid ? rl : 0)) * p.num_heads + h) * D + hh * HC;
 #pragma unroll
-        for (int q = 0; q < D / 32; ++q) {
+        for (int q = 0; q < HC / 32; ++q) {
             float ov[32];
-            tmem_ld32(tl + 256 + q * 32, ov);
+            tmem_ld32(tl + 256 + hh * HC + q * 32, ov);
             if (valid) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
@@ -599,7 +631,7 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
         }
     }
     tc_fence_before();
-    asm volatile("bar.sync 2, 160;" ::: "memory");
+    asm volatile("bar.sync 2, %0;" ::"r"(32 * (kTcSoftmaxWarps + 1)) : "memory");
 }
 
 }  // namespace pa
