@@ -220,6 +220,18 @@ __device__ __forceinline__ void tc_mma_f16(uint32_t d_tmem, uint64_t a_desc, uin
         : "memory");
 }
 
+// As tc_mma_f16, with A read from tensor memory (a_tmem: lane 0 and the
+// first column of the M x 16 slice; row m in lane m, two fp16 per column).
+__device__ __forceinline__ void tc_mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Shared-memory matrix descriptor for a 128-byte-swizzled operand whose
 // swizzle atoms (8 rows x 128 bytes) start on 1024-byte boundaries.
 // lbo / sbo: leading / stride byte offsets (multiples of 16).

@@ -206,14 +206,14 @@ namespace pa {
 // sequence; K/V are consumed 128 tokens at a time. Per K/V tile j:
 //   S_j = Q . K_j^T   128 x 128, eight tcgen05.mma (K = 16 each) into tensor
 //                     memory (two S buffers, so S_{j+1} overlaps the softmax of j)
-//   softmax           thread t of the four softmax warps owns row t (tensor-
-//                     memory lane t): reads its S row, masks tokens after its
-//                     position, keeps a reference maximum that moves only when
-//                     the row maximum exceeds it by more than 2^8 (then O is
-//                     rescaled in tensor memory), writes P = 2^(s - m) as fp16
-//                     into shared memory (128-byte swizzle)
-//   O += P_j . V_j    eight tcgen05.mma into the O columns of tensor memory,
-//                     V read N-contiguous (MN-major)
+//   softmax           reads S, masks tokens after each row's position, keeps
+//                     a reference maximum that moves only when the row
+//                     maximum exceeds it by more than 2^8 (then O is rescaled
+//                     in tensor memory), and writes P = 2^(s - m) as fp16 back
+//                     into the S buffer it came from (tcgen05.st)
+//   O += P_j . V_j    eight tcgen05.mma with A (P) read from tensor memory and
+//                     V from shared memory, N-contiguous (MN-major)
+// An S buffer takes the next S only once the P.V that reads its P is done.
 // K and V have rings of their own (3 and 2 tiles): a K tile is released as
 // soon as its S is computed, a V tile when its P.V is, so each is reloaded
 // as early as possible. Warps: 0-7 softmax (and Q staging, epilogue): warp
@@ -241,8 +241,7 @@ struct TcLayout {                                       // byte offsets from the
     static constexpr uint32_t kQ = 0;                    // Q (dims 0-63, 64-127)
     static constexpr uint32_t kK = kQ + kTile;           // K ring
     static constexpr uint32_t kV = kK + kTcKStages * kTile;  // V ring
-    static constexpr uint32_t kP = kV + kTcVStages * kTile;  // P (tokens 0-63, 64-127)
-    static constexpr uint32_t kBars = kP + kTile;
+    static constexpr uint32_t kBars = kV + kTcVStages * kTile;
     static constexpr uint32_t kBytes = kBars + 256;
 };
 
@@ -255,7 +254,7 @@ enum : int {
     kBarEmptyV = kBarFullV + kTcVStages,    // + stage: P.V of the stage's tile done (commit)
     kBarSFull = kBarEmptyV + kTcVStages,    // + buffer: S ready (commit)
     kBarSFree = kBarSFull + 2,              // + buffer: S read by the 8 softmax warps
-    kBarPFull = kBarSFree + 2,              // P written, O corrected (8 softmax warps)
+    kBarPFull = kBarSFree + 2,              // P written into tensor memory, O corrected (8 warps)
     kBarOReady = kBarPFull + 1,             // P.V done (commit)
     kBarDone = kBarOReady + 1,              // every MMA of the CTA done (commit)
     kBarPair = kBarDone + 1,                // + 2 * quadrant + tile parity: both halves' row maxima posted
@@ -430,7 +429,6 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
         // the two 64-dim halves kHalf apart, 8-token groups 1024 B apart. A
         // k-step moves the start address (descriptor bits 0-13, in 16 B).
         const uint64_t dq = sw128_desc(sbase + Lay::kQ, 16, 1024);
-        const uint64_t dp = sw128_desc(sbase + Lay::kP, 16, 1024);
         const uint64_t dk = sw128_desc(sbase + Lay::kK, 16, 1024);
         const uint64_t dv = sw128_desc(sbase + Lay::kV, Lay::kHalf, 1024);
         auto kstep = [](int k) { return (uint64_t)(((k >> 2) * Lay::kHalf + (k & 3) * 32) >> 4); };
@@ -443,7 +441,10 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
                 const uint64_t dvs = dv + ((st * Lay::kTile) >> 4);
 #pragma unroll
                 for (int kt = 0; kt < kTcKv / 16; ++kt)
-                    tc_mma_f16(tmem + 256, dp + kstep(kt), dvs + ((kt * 16 * 128) >> 4), kIdescPV,
+                    // P_i in tensor memory, in S buffer i % 2: tokens 64 h .. 64 h + 63
+                    // packed in columns 64 h .. 64 h + 31 (two fp16 per column)
+                    tc_mma_f16_ts(tmem + 256, tmem + (i & 1) * kTcKv + (kt >> 2) * 64 + (kt & 3) * 8,
+                                  dvs + ((kt * 16 * 128) >> 4), kIdescPV,
                                (i > 0 || kt > 0) ? 1u : 0u);
                 tc_commit(&bar[kBarEmptyV + st]);
                 tc_commit(&bar[kBarOReady]);
@@ -457,6 +458,9 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
             const int st = j % kTcKStages;
             ok = tc_wait_warp(&bar[kBarFullK + st], (j / kTcKStages) & 1, abort);
             if (ok && j >= 2) ok = tc_wait_warp(&bar[kBarSFree + (j & 1)], ((j - 2) >> 1) & 1, abort);
+            // S buffer j % 2 holds P_{j-2} until its P.V is done (P.V of j-1
+            // is issued after this S, so the wait names the last completion)
+            if (ok && j >= 2) ok = tc_wait_warp(&bar[kBarOReady], (j - 2) & 1, abort);
             if (!ok) break;
             tc_fence_after();
             if (lane == 0) {
@@ -564,25 +568,25 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
         }
         l = l * alpha + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));  // this half's share of the row sum
 
-        // P.V of tile j-1 done: the P buffer is free and O is current
-        if (j >= 1) {
+        // O must be current before a rescale: wait for P.V of tile j-1
+        if (j >= 1 && __any_sync(0xffffffffu, resc)) {
             if (!tc_wait_warp(&bar[kBarOReady], (j - 1) & 1, abort)) { ok = false; break; }
             tc_fence_after();
-            if (__any_sync(0xffffffffu, resc)) {
 #pragma unroll
-                for (int q = 0; q < HC / 32; ++q) {
-                    float ov[32];
-                    tmem_ld32(tl + 256 + hh * HC + q * 32, ov);
+            for (int q = 0; q < HC / 32; ++q) {
+                float ov[32];
+                tmem_ld32(tl + 256 + hh * HC + q * 32, ov);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) ov[i] *= alpha;
-                    tmem_st32(tl + 256 + hh * HC + q * 32, ov);
-                }
+                for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+                tmem_st32(tl + 256 + hh * HC + q * 32, ov);
             }
         }
+        {  // P into the first half of this warp's S columns (read above)
+            float pf[32];
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-            st_shared_v4(tc_chunk(sbase + Lay::kP, t, 8 * hh + c),
-                         make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]));
+            for (int i = 0; i < 32; ++i) pf[i] = __uint_as_float(pk[i]);
+            tmem_st32(tl + (j & 1) * kTcKv + hh * HC, pf);
+        }
         // tokens at or after the sequence end are unused cache slots (any
         // bits, NaN included): their V rows enter P.V as zeros
         const int tt = j * kTcKv;
@@ -594,8 +598,8 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
 #pragma unroll
                 for (int c = 8 * hh; c < 8 * hh + 8; ++c) st_shared_v4(tc_chunk(v_addr, t, c), make_uint4(0, 0, 0, 0));
             }
+            fence_proxy_async_smem();
         }
-        fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar[kBarPFull]);
