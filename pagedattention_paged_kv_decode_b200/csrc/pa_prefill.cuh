@@ -242,7 +242,7 @@ struct TcLayout {                                       // byte offsets from the
     static constexpr uint32_t kK = kQ + kTile;           // K ring
     static constexpr uint32_t kV = kK + kTcKStages * kTile;  // V ring
     static constexpr uint32_t kBars = kV + kTcVStages * kTile;
-    static constexpr uint32_t kBytes = kBars + 256;
+    static constexpr uint32_t kBytes = kBars + 512;      // barriers, tensor-memory address, abort flag
 };
 
 // mbarrier indices
@@ -261,6 +261,8 @@ enum : int {
     kBarPairEnd = kBarPair + 8,             // + quadrant: both halves' row sums posted
     kNumBars = kBarPairEnd + 4
 };
+static_assert(8 * kNumBars + 8 <= TcLayout::kBytes - TcLayout::kBars, "barrier area too small");
+static_assert(TcLayout::kBytes + 1024 <= 227 * 1024, "shared memory of the tcgen05 prefill kernel");
 
 // Bounded wait that also ends when another role has aborted. It spins on
 // the non-blocking test (these waits are short and on the critical path,
