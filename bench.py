@@ -495,7 +495,7 @@ def run_prefill(args, rank, world, local_rank):
     dp = W.prefill_to_device(w, dev)
     mql = int(w.chunk_lens.max(initial=0))
     T = w.total_q
-    n_write = -(-T // 65535)
+    n_write = -(-T // 65535)  # the library launches the cache write in slices of 65535 tokens
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_sink = torch.zeros((), dtype=torch.int64, device=dev)
     stream = torch.cuda.Stream(dev)
@@ -509,10 +509,7 @@ def run_prefill(args, rank, world, local_rank):
         ev[0].record()
         pk.prefill_slot_mapping(dp.query_start, dp.block_tables, dp.context_lens, dp.key_cache, mql,
                                 out=dp.slots)
-        for i in range(0, T, 65535):
-            m = min(65535, T - i)
-            pk.kv_cache_write(dp.new_key[i:i + m], dp.new_value[i:i + m], dp.key_cache, dp.value_cache,
-                              dp.slots[i:i + m])
+        pk.kv_cache_write(dp.new_key, dp.new_value, dp.key_cache, dp.value_cache, dp.slots)
         ev[1].record()
         pk.paged_prefill(dp.out, dp.query, dp.query_start, dp.key_cache, dp.value_cache, dp.block_tables,
                          dp.context_lens, mql, w.scale)

@@ -36,6 +36,9 @@
  *   - Supported shapes: head_size 64 or 128; block_size 16 or 32;
  *     num_heads >= 1; num_blocks * block_size < 2^31.
  *   - Query, output, new K/V rows and caches must be 16-byte aligned.
+ *   - Counts: num_seqs <= 65535 per decode or prefill call; token and pair
+ *     counts of the cache write, block copy and swap have no such limit (the
+ *     library launches them in slices of 65535, in stream order).
  */
 #ifndef PAGEDKV_H
 #define PAGEDKV_H

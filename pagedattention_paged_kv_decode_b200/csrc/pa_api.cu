@@ -140,6 +140,7 @@ int cache_tensor_map(const void *cache, const pa_cache_desc &c, int G, CUtensorM
 // ----------------------------------------------------- launch shape
 
 constexpr int kNumSMs = 148;
+constexpr int kMaxGridY = 65535;  // grid y extent: token and pair counts are launched in slices of this
 constexpr size_t kMaxSmem = 227 * 1024;
 
 int fill_config(const pa_cache_desc &c, int num_seqs, int max_ctx, pa_decode_config *cfg) {
@@ -534,7 +535,6 @@ int pa_kv_cache_write(const void *key, const void *value, int64_t key_stride, in
     if (rc) return rc;
     if (n_tokens < 0) return fail(PA_ERR_INVALID, "n_tokens %d < 0", n_tokens);
     if (n_tokens == 0) return ok();
-    if (n_tokens > 65535) return fail(PA_ERR_INVALID, "n_tokens %d > 65535 per call", n_tokens);
     if (!key || !value || !key_cache || !value_cache || !slot_mapping)
         return fail(PA_ERR_INVALID, "null pointer argument");
     if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache))
@@ -548,21 +548,25 @@ int pa_kv_cache_write(const void *key, const void *value, int64_t key_stride, in
         !(std::isfinite(k_scale) && std::isfinite(v_scale) && k_scale > 0 && v_scale > 0))
         return fail(PA_ERR_INVALID, "k_scale and v_scale must be finite and > 0");
     const int chunks = row / 8;
-    const dim3 grid((chunks + 127) / 128, n_tokens);
     const int64_t pool_slots = (int64_t)cache.num_blocks * cache.block_size;
     const cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const __half *k = static_cast<const __half *>(key);
-    const __half *v = static_cast<const __half *>(value);
-    if (cache.dtype == PA_F16)
-        pa::kv_cache_write_kernel<false><<<grid, 128, 0, st>>>(
-            k, v, key_stride, value_stride, key_cache, value_cache, slot_mapping, row, pool_slots,
-            1.0f, 1.0f);
-    else
-        pa::kv_cache_write_kernel<true><<<grid, 128, 0, st>>>(
-            k, v, key_stride, value_stride, key_cache, value_cache, slot_mapping, row, pool_slots,
-            k_scale, v_scale);
-    const cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "kv_cache_write_kernel launch");
+    // one launch per 65535 tokens (the grid's y extent), in stream order
+    for (int t0 = 0; t0 < n_tokens; t0 += kMaxGridY) {
+        const int n = std::min(kMaxGridY, n_tokens - t0);
+        const dim3 grid((chunks + 127) / 128, n);
+        const __half *k = static_cast<const __half *>(key) + (size_t)t0 * key_stride;
+        const __half *v = static_cast<const __half *>(value) + (size_t)t0 * value_stride;
+        if (cache.dtype == PA_F16)
+            pa::kv_cache_write_kernel<false><<<grid, 128, 0, st>>>(
+                k, v, key_stride, value_stride, key_cache, value_cache, slot_mapping + t0, row, pool_slots,
+                1.0f, 1.0f);
+        else
+            pa::kv_cache_write_kernel<true><<<grid, 128, 0, st>>>(
+                k, v, key_stride, value_stride, key_cache, value_cache, slot_mapping + t0, row, pool_slots,
+                k_scale, v_scale);
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "kv_cache_write_kernel launch");
+    }
     return ok();
 }
 
@@ -572,7 +576,6 @@ int pa_copy_blocks(void *key_cache, void *value_cache, pa_cache_desc cache,
     if (rc) return rc;
     if (n_pairs < 0) return fail(PA_ERR_INVALID, "n_pairs %d < 0", n_pairs);
     if (n_pairs == 0) return ok();
-    if (n_pairs > 65535) return fail(PA_ERR_INVALID, "n_pairs %d > 65535 per call", n_pairs);
     if (!key_cache || !value_cache || !src_dst_pairs)
         return fail(PA_ERR_INVALID, "null pointer argument");
     if (!aligned16(key_cache) || !aligned16(value_cache))
@@ -580,11 +583,13 @@ int pa_copy_blocks(void *key_cache, void *value_cache, pa_cache_desc cache,
     const int64_t block_vecs =
         (int64_t)cache.block_size * cache.num_heads * cache.head_size * elem_bytes(cache) / 16;
     const int64_t per_cta = (int64_t)pa::kCopyThreads * pa::kCopyVecs;
-    const dim3 grid((unsigned)((block_vecs + per_cta - 1) / per_cta), n_pairs, 2);
-    pa::copy_blocks_kernel<<<grid, pa::kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-        key_cache, value_cache, src_dst_pairs, block_vecs, cache.num_blocks);
-    const cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "copy_blocks_kernel launch");
+    for (int p0 = 0; p0 < n_pairs; p0 += kMaxGridY) {  // one launch per 65535 pairs
+        const dim3 grid((unsigned)((block_vecs + per_cta - 1) / per_cta), std::min(kMaxGridY, n_pairs - p0), 2);
+        pa::copy_blocks_kernel<<<grid, pa::kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+            key_cache, value_cache, src_dst_pairs + 2 * (size_t)p0, block_vecs, cache.num_blocks);
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "copy_blocks_kernel launch");
+    }
     return ok();
 }
 
@@ -600,7 +605,6 @@ int pa_swap_blocks(void *dst_key_cache, void *dst_value_cache, int dst_num_block
                     dst_num_blocks, src_num_blocks);
     if (n_pairs < 0) return fail(PA_ERR_INVALID, "n_pairs %d < 0", n_pairs);
     if (n_pairs == 0) return ok();
-    if (n_pairs > 65535) return fail(PA_ERR_INVALID, "n_pairs %d > 65535 per call", n_pairs);
     if (!dst_key_cache || !dst_value_cache || !src_key_cache || !src_value_cache || !src_dst_pairs)
         return fail(PA_ERR_INVALID, "null pointer argument");
     if (!aligned16(dst_key_cache) || !aligned16(dst_value_cache) || !aligned16(src_key_cache) ||
@@ -609,12 +613,14 @@ int pa_swap_blocks(void *dst_key_cache, void *dst_value_cache, int dst_num_block
     const int64_t block_vecs =
         (int64_t)c.block_size * c.num_heads * c.head_size * elem_bytes(c) / 16;
     const int64_t per_cta = (int64_t)pa::kCopyThreads * pa::kCopyVecs;
-    const dim3 grid((unsigned)((block_vecs + per_cta - 1) / per_cta), n_pairs, 2);
-    pa::swap_blocks_kernel<<<grid, pa::kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-        dst_key_cache, dst_value_cache, src_key_cache, src_value_cache, src_dst_pairs, block_vecs,
-        src_num_blocks, dst_num_blocks);
-    const cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "swap_blocks_kernel launch");
+    for (int p0 = 0; p0 < n_pairs; p0 += kMaxGridY) {  // one launch per 65535 pairs
+        const dim3 grid((unsigned)((block_vecs + per_cta - 1) / per_cta), std::min(kMaxGridY, n_pairs - p0), 2);
+        pa::swap_blocks_kernel<<<grid, pa::kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+            dst_key_cache, dst_value_cache, src_key_cache, src_value_cache, src_dst_pairs + 2 * (size_t)p0,
+            block_vecs, src_num_blocks, dst_num_blocks);
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "swap_blocks_kernel launch");
+    }
     return ok();
 }
 

@@ -287,8 +287,9 @@ def load_cache(key_cache: torch.Tensor, value_cache: torch.Tensor, key_src: torc
                stream=None) -> None:
     """Write whole fp16 pools [NB, B, H, D] into the caches, slot by slot.
 
-    This is ``kv_cache_write`` with the identity slot list, in calls of at
-    most 65535 tokens; for E4M3 caches it quantises with the given scales.
+    This is ``kv_cache_write`` with the identity slot list, in slices of at
+    most 65535 tokens (the slot list stays small); for E4M3 caches it
+    quantises with the given scales.
     """
     _check_pair(key_cache, value_cache)
     nb, bs, nh, hd = key_cache.shape
@@ -405,10 +406,7 @@ def prefill_step(out: torch.Tensor, query: torch.Tensor, new_key: torch.Tensor, 
     T = query.shape[0]
     slots = prefill_slot_mapping(query_start, block_tables, context_lens, key_cache, max_query_len,
                                  out=slots, total_q=T, stream=stream)
-    for i in range(0, T, 65535):  # the cache write takes at most 65535 tokens a call
-        m = min(65535, T - i)
-        kv_cache_write(new_key[i:i + m], new_value[i:i + m], key_cache, value_cache, slots[i:i + m],
-                       stream=stream)
+    kv_cache_write(new_key, new_value, key_cache, value_cache, slots, stream=stream)
     paged_prefill(out, query, query_start, key_cache, value_cache, block_tables, context_lens,
                   max_query_len, scale, stream)
     return slots

@@ -189,3 +189,33 @@ def test_swap_blocks_device_and_pinned_host(cuda_device, kv):
     oracle.swap_blocks(hk, hv, rk, rv, in_pairs)
     assert np.array_equal(gk.cpu().numpy().view(np.uint8), hk.view(np.uint8))
     assert np.array_equal(gv.cpu().numpy().view(np.uint8), hv.view(np.uint8))
+
+
+def test_counts_above_one_grid_slice(cuda_device):
+    # 70000 tokens written and 70000 block pairs copied in one call each: the
+    # library launches slices of 65535; results bit-exact against the oracle
+    rng = np.random.default_rng(11)
+    n = 70000
+    nb, B, H, D = 17500, 16, 1, 64
+    key = rng.standard_normal((n, H, D)).astype(np.float16)
+    val = rng.standard_normal((n, H, D)).astype(np.float16)
+    slots = rng.permutation(nb * B)[:n].astype(np.int32)
+    kc = np.zeros((nb, B, H, D), np.float16)
+    vc = np.zeros_like(kc)
+    gk, gv = torch.from_numpy(kc).to(cuda_device), torch.from_numpy(vc).to(cuda_device)
+    pk.kv_cache_write(torch.from_numpy(key).to(cuda_device), torch.from_numpy(val).to(cuda_device), gk, gv,
+                      torch.from_numpy(slots).to(cuda_device))
+    assert pk.check_status() == 0
+    oracle.kv_cache_write(key, val, kc, vc, slots)
+    assert np.array_equal(gk.cpu().numpy().view(np.uint16), kc.view(np.uint16))
+    assert np.array_equal(gv.cpu().numpy().view(np.uint16), vc.view(np.uint16))
+    # block copy on an E4M3 pool of 2n one-KiB blocks: block i -> block n + i
+    ek = rng.integers(0, 256, (2 * n, B, H, D), dtype=np.uint8)
+    ev = rng.integers(0, 256, (2 * n, B, H, D), dtype=np.uint8)
+    gek, gev = torch.from_numpy(ek).to(cuda_device), torch.from_numpy(ev).to(cuda_device)
+    pairs = np.stack([np.arange(n), np.arange(n) + n], 1).astype(np.int32)
+    pk.copy_blocks(gek, gev, torch.from_numpy(pairs).to(cuda_device))
+    assert pk.check_status() == 0
+    oracle.copy_blocks(ek, ev, pairs)
+    assert np.array_equal(gek.cpu().numpy(), ek)
+    assert np.array_equal(gev.cpu().numpy(), ev)
