@@ -467,7 +467,9 @@ int launch_decode(void *out, const void *query, const void *kc, const void *vc,
     // Packed CTAs are spread over all SMs (some slots of the last ones idle).
     const int64_t n_ctas = std::max<int64_t>((p.num_units + C - 1) / C,
                                              std::min<int64_t>(p.num_units, kNumSMs));
-    if (n_ctas > 0x7fffffff) return fail(PA_ERR_INVALID, "too many work units (%lld)", (long long)p.num_units);
+    // unit ids are 32-bit in the kernels
+    if (n_ctas > 0x7fffffff || p.num_units > 0x7fffffff)
+        return fail(PA_ERR_INVALID, "too many work units (%lld)", (long long)p.num_units);
     const dim3 grid((unsigned)n_ctas);
     const dim3 block(32 * (C * G * W + 1));
     kern<<<grid, block, lay.total, st>>>(mk, mv, p);

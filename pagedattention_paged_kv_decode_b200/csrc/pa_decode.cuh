@@ -327,12 +327,15 @@ struct Unit {
 
 __device__ __forceinline__ Unit unit_of(const DecodeParams &p, int B, int j) {
     Unit u;
-    const int64_t id = (int64_t)blockIdx.x + (int64_t)j * gridDim.x;
-    const int HG = p.num_heads / p.heads_per_cta;
-    const bool exists = id < p.num_units;
-    const int64_t idc = exists ? id : 0;
-    u.part = (int)(idc % p.max_parts);
-    const int64_t rest = idc / p.max_parts;
+    // unit ids fit 32 bits: the host keeps num_units below 2^31, and C * grid
+    // stays below 2^32 for every C
+    const uint32_t id = blockIdx.x + (uint32_t)j * gridDim.x;
+    const uint32_t HG = (uint32_t)(p.num_heads / p.heads_per_cta);
+    const bool exists = (int64_t)id < p.num_units;
+    const uint32_t idc = exists ? id : 0u;
+    const uint32_t mp = (uint32_t)p.max_parts;
+    u.part = (int)(idc % mp);
+    const uint32_t rest = idc / mp;
     u.h0 = (int)(rest % HG) * p.heads_per_cta;
     u.s = (int)(rest / HG);
     u.L_in = exists ? __ldg(p.context_lens + u.s) : 0;
@@ -380,10 +383,10 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
         for (int j = 0; j < kMaxUnitsPerCta; ++j) {
             pre_blk[j] = 0;
             if (j < C) {
-                const int64_t id = (int64_t)blockIdx.x + (int64_t)j * gridDim.x;
-                if (id < p.num_units) {
-                    const int part = (int)(id % p.max_parts);
-                    const int s = (int)(id / p.max_parts / (p.num_heads / G));
+                const uint32_t id = blockIdx.x + (uint32_t)j * gridDim.x;
+                if ((int64_t)id < p.num_units) {
+                    const int part = (int)(id % (uint32_t)p.max_parts);
+                    const int s = (int)(id / (uint32_t)p.max_parts / (uint32_t)(p.num_heads / G));
                     const int e = (p.prefix_tokens + part * p.partition_size) / B + lane;
                     if (e < p.max_blocks_per_seq)
                         pre_blk[j] = __ldg(p.block_tables + (size_t)s * p.max_blocks_per_seq + e);
@@ -504,11 +507,11 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
     // Query row: its address depends on the unit id only.
     uint4 q_raw[EPL / 8], nk_raw[EPL / 8], nv_raw[EPL / 8];
     {
-        const int64_t id = (int64_t)blockIdx.x + (int64_t)slot * gridDim.x;
-        const int64_t idc = id < p.num_units ? id : 0;
-        const int64_t rest = idc / p.max_parts;
-        const int hq = (int)(rest % (p.num_heads / G)) * G + g;
-        const int sq = (int)(rest / (p.num_heads / G));
+        const uint32_t id = blockIdx.x + (uint32_t)slot * gridDim.x;
+        const uint32_t idc = (int64_t)id < p.num_units ? id : 0u;
+        const uint32_t rest = idc / (uint32_t)p.max_parts;
+        const int hq = (int)(rest % (uint32_t)(p.num_heads / G)) * G + g;
+        const int sq = (int)(rest / (uint32_t)(p.num_heads / G));
         const uint4 *qp = reinterpret_cast<const uint4 *>(p.query + ((size_t)sq * p.num_heads + hq) * D);
 #pragma unroll
         for (int c = 0; c < EPL / 8; ++c) q_raw[c] = __ldg(qp + sub * (EPL / 8) + c);
