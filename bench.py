@@ -51,29 +51,33 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash() -> str:
+DECODE_SOURCES = ("pa_decode.cuh", "pa_device.cuh", "pa_cache_ops.cuh")
+PREFILL_SOURCES = ("pa_prefill.cuh", "pa_decode.cuh", "pa_device.cuh")
+
+
+def kernel_source_hash(names=DECODE_SOURCES) -> str:
     """Hash of the device code (kernels and their helpers; not the host-side
     launch logic), so a recorded ncu traffic figure is dropped when a kernel
     changes."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "pagedattention_paged_kv_decode_b200", "csrc")
-    for name in ("pa_decode.cuh", "pa_device.cuh", "pa_cache_ops.cuh"):
+    for name in names:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str):
-    """DRAM bytes per decode launch from the committed ncu summary, if it was
-    taken on the current kernel sources (else None)."""
-    path = os.path.join(ROOT, "profiles", "decode_dram_traffic.json")
+def recorded_traffic(workload: str, record: str = "decode_dram_traffic.json", names=DECODE_SOURCES):
+    """DRAM bytes per launch of the dominant kernel from a committed ncu
+    summary, if it was taken on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", record)
     try:
         with open(path) as f:
             rec = json.load(f)
     except Exception:
         return None
     ent = rec.get(workload)
-    if not ent or ent.get("kernel_source_hash") != kernel_source_hash():
+    if not ent or ent.get("kernel_source_hash") != kernel_source_hash(names):
         return None
     return ent.get("dram_bytes_per_launch")
 
@@ -494,6 +498,7 @@ def run_prefill(args, rank, world, local_rank):
     w = W.prefill_named(args.prefill, seed=W.rank_seed(2000 + args.prefill, rank))
     dp = W.prefill_to_device(w, dev)
     mql = int(w.chunk_lens.max(initial=0))
+    tc = w.head_size in (64, 128) and w.scale > 0  # the library's choice of prefill kernel
     T = w.total_q
     n_write = -(-T // 65535)  # the library launches the cache write in slices of 65535 tokens
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -609,7 +614,8 @@ def run_prefill(args, rank, world, local_rank):
             "frac": round(achieved / peak, 4),
             "peak_kind": f"{kind} dense bf16 GEMM, burst (fp16 runs at the same nominal rate); "
                          f"sustained {peak_sust}",
-            "traffic": None, "kernel": "paged_prefill_kernel",
+            "traffic": recorded_traffic(w.name, "prefill_dram_traffic.json", PREFILL_SOURCES) if tc else None,
+            "kernel": "paged_prefill_tc_kernel" if tc else "paged_prefill_kernel (mma.sync)",
             "algorithmic_flops_per_launch": flops,
             "io_bytes_per_launch": w.io_bytes(),
         },

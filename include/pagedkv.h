@@ -337,7 +337,9 @@ int pa_prefill_slot_mapping(int32_t *slot_mapping, const int32_t *query_start,
  * sequence (the chunk's own K/V included). fp16 caches only (PA_ERR_DTYPE
  * for E4M3). max_query_len: a host-known bound on every n_s (the grid is
  * sized from it). Computed on tensor cores: Q.K^T and P.V in fp16 x fp16 ->
- * fp32 (mma.m16n8k16), softmax in fp32 with P rounded to fp16.
+ * fp32, softmax in fp32 with P rounded to fp16; a positive scale runs
+ * tcgen05.mma over 128-row tiles with S and O in tensor memory, a scale
+ * <= 0 the warp-level mma.m16n8k16 over 64-row tiles.
  * Device checks: n_s > L_s or n_s > max_query_len sets PA_DEV_BAD_CHUNK,
  * L_s beyond the table row PA_DEV_CTX_OVER_TABLE; such a sequence's rows
  * are not written. Block ids outside the pool read as zeros and set

@@ -945,6 +945,14 @@ PrefillKernel pick_prefill(int D, int B) {
     return nullptr;
 }
 
+PrefillKernel pick_prefill_tc(int D, int B) {
+    if (D == 64 && B == 16) return pa::paged_prefill_tc_kernel<64, 16>;
+    if (D == 64 && B == 32) return pa::paged_prefill_tc_kernel<64, 32>;
+    if (D == 128 && B == 16) return pa::paged_prefill_tc_kernel<128, 16>;
+    if (D == 128 && B == 32) return pa::paged_prefill_tc_kernel<128, 32>;
+    return nullptr;
+}
+
 // Ring of the prefill kernel: about 96 KiB of K/V tiles, so that two CTAs
 // (160 threads, under 200 registers each) share an SM.
 int prefill_stages(const pa_cache_desc &c) {
@@ -995,18 +1003,18 @@ extern "C" int pa_paged_prefill(void *out, const void *query, const int32_t *que
     if ((int64_t)max_blocks_per_seq * cache.block_size >= (int64_t(1) << 31))
         return fail(PA_ERR_OVERFLOW, "max_blocks_per_seq * block_size overflows int32");
     if (!std::isfinite(scale)) return fail(PA_ERR_INVALID, "scale is not finite");
-    const int rows_per_cta = (cache.head_size == 128 && scale > 0.f) ? pa::kTcRows : pa::kPrefillRows;
+    // head_size 64 or 128 with a positive scale: the tcgen05 kernel (128-row
+    // tiles, S and O in tensor memory); otherwise the mma.sync kernel (64-row
+    // tiles).
+    const bool tc = (cache.head_size == 64 || cache.head_size == 128) && scale > 0.f;
+    const int rows_per_cta = tc ? pa::kTcRows : pa::kPrefillRows;
     const int64_t row_tiles = (max_query_len + rows_per_cta - 1) / rows_per_cta;
     const int64_t n_ctas = row_tiles * num_seqs * cache.num_heads;
     if (n_ctas > 0x7fffffff) return fail(PA_ERR_INVALID, "too many prefill tiles (%lld)", (long long)n_ctas);
     int dev = 0;
     rc = current_device(&dev);
     if (rc) return rc;
-    // head_size 128 with a positive scale: the tcgen05 kernel (128-row tiles,
-    // S and O in tensor memory); otherwise the mma.sync kernel (64-row tiles).
-    const bool tc = cache.head_size == 128 && scale > 0.f;
-    PrefillKernel kern = tc ? (cache.block_size == 16 ? pa::paged_prefill_tc_kernel<16>
-                                                      : pa::paged_prefill_tc_kernel<32>)
+    PrefillKernel kern = tc ? pick_prefill_tc(cache.head_size, cache.block_size)
                             : pick_prefill(cache.head_size, cache.block_size);
     rc = ensure_smem_attr(reinterpret_cast<const void *>(kern), dev);
     if (rc) return rc;
@@ -1030,7 +1038,7 @@ extern "C" int pa_paged_prefill(void *out, const void *query, const int32_t *que
     p.stages = prefill_stages(cache);
     p.qk_scale_log2 = scale * pa::kLog2e;
     // ring (or tcgen05 tiles) + barriers + 1 KiB to align to 1024 bytes in the kernel
-    const size_t smem = tc ? (size_t)pa::TcLayout::kBytes + 1024
+    const size_t smem = tc ? (size_t)(cache.head_size == 64 ? pa::TcLayout<64>::kBytes : pa::TcLayout<128>::kBytes) + 1024
                            : (size_t)p.stages * 4 * cache.block_size * cache.head_size + 16 * (size_t)p.stages + 1024;
     kern<<<dim3((unsigned)n_ctas), dim3(tc ? pa::kTcThreads : 32 * 5), smem, static_cast<cudaStream_t>(stream)>>>(
         mk, mv, p);

@@ -235,9 +235,10 @@ constexpr int kTcWarpK = 8, kTcWarpMma = 9, kTcWarpV = 10;
 constexpr int kTcTmemCols = 512;  // S0 [0,128), S1 [128,256), O [256,384), row exchange [384,390)
 constexpr int kTcColX = 384;      // + 2 * tile parity + half: row maxima; + 4 + half: row sums
 
+template <int D>
 struct TcLayout {                                       // byte offsets from the 1024-aligned base
     static constexpr uint32_t kHalf = 128 * 128;         // [128 rows][128 B]: one 64-wide half
-    static constexpr uint32_t kTile = 2 * kHalf;         // a 128 x 128 fp16 tile in two halves
+    static constexpr uint32_t kTile = (D / 64) * kHalf;  // a 128 x D fp16 tile in 64-wide halves
     static constexpr uint32_t kQ = 0;                    // Q (dims 0-63, 64-127)
     static constexpr uint32_t kK = kQ + kTile;           // K ring
     static constexpr uint32_t kV = kK + kTcKStages * kTile;  // V ring
@@ -261,8 +262,8 @@ enum : int {
     kBarPairEnd = kBarPair + 8,             // + quadrant: both halves' row sums posted
     kNumBars = kBarPairEnd + 4
 };
-static_assert(8 * kNumBars + 8 <= TcLayout::kBytes - TcLayout::kBars, "barrier area too small");
-static_assert(TcLayout::kBytes + 1024 <= 227 * 1024, "shared memory of the tcgen05 prefill kernel");
+static_assert(8 * kNumBars + 8 <= TcLayout<128>::kBytes - TcLayout<128>::kBars, "barrier area too small");
+static_assert(TcLayout<128>::kBytes + 1024 <= 227 * 1024, "shared memory of the tcgen05 prefill kernel");
 
 // Bounded wait that also ends when another role has aborted. It spins on
 // the non-blocking test (these waits are short and on the critical path,
@@ -289,10 +290,10 @@ __device__ __forceinline__ bool tc_wait_warp(uint64_t *bar, uint32_t parity, vol
     return __all_sync(0xffffffffu, ok);
 }
 
-// 16 bytes at chunk c (0..15) of row r of a [2 halves][128 rows][128 B]
+// 16 bytes at chunk c (0..15) of row r of a [halves][128 rows][128 B]
 // swizzled tile.
 __device__ __forceinline__ uint32_t tc_chunk(uint32_t base, int r, int c) {
-    return base + (uint32_t)(c >> 3) * TcLayout::kHalf + (uint32_t)r * 128u +
+    return base + (uint32_t)(c >> 3) * TcLayout<128>::kHalf + (uint32_t)r * 128u +
            ((uint32_t)(((c & 7) ^ (r & 7))) << 4);
 }
 
@@ -305,7 +306,7 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
 // through its ring. Lane b < BPT loads cache block b of each tile; lane l
 // holds block-table entry 32c + l of the current chunk c while the next
 // chunk's entries are already being read.
-template <int B, int STAGES>
+template <int D, int B, int STAGES>
 __device__ __forceinline__ void tc_produce(const CUtensorMap *tmap, unsigned char *ring, uint64_t *full,
                                            uint64_t *empty, const int32_t *table, int nblk, int n_kv, int h,
                                            int num_blocks, volatile int *abort, int lane) {
@@ -336,12 +337,12 @@ __device__ __forceinline__ void tc_produce(const CUtensorMap *tmap, unsigned cha
         bool ok = true;
         if (lane == 0 && use > 0) ok = tc_wait(&empty[st], (use - 1) & 1, abort);
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-        if (lane == 0) mbar_arrive_expect_tx(&full[st], (uint32_t)TcLayout::kTile);
+        if (lane == 0) mbar_arrive_expect_tx(&full[st], (uint32_t)TcLayout<D>::kTile);
         __syncwarp();
         if (lane < BPT) {
-            unsigned char *dst = ring + st * TcLayout::kTile + lane * B * 128;
+            unsigned char *dst = ring + st * TcLayout<D>::kTile + lane * B * 128;
             tma_load_4d(dst, tmap, &full[st], 0, h, 0, blk, policy);
-            tma_load_4d(dst + TcLayout::kHalf, tmap, &full[st], 64, h, 0, blk, policy);
+            if (D == 128) tma_load_4d(dst + TcLayout<D>::kHalf, tmap, &full[st], 64, h, 0, blk, policy);
         }
         issued = j + 1;
     }
@@ -350,12 +351,12 @@ __device__ __forceinline__ void tc_produce(const CUtensorMap *tmap, unsigned cha
         for (int j = max(0, issued - STAGES); j < issued; ++j) mbar_wait(&full[j % STAGES], (j / STAGES) & 1);
 }
 
-template <int B>
+template <int D, int B>
 __global__ void __launch_bounds__(kTcThreads, 1)
 paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                         const PrefillParams p) {
-    constexpr int D = 128;
-    using Lay = TcLayout;
+    static_assert(D == 64 || D == 128, "head_size 64 or 128");
+    using Lay = TcLayout<D>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bar = reinterpret_cast<uint64_t *>(smem + Lay::kBars);
@@ -413,12 +414,12 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
     const uint32_t tmem = *tmem_slot;
 
     if (warp == kTcWarpK) {
-        tc_produce<B, kTcKStages>(&tmap_k, smem + Lay::kK, &bar[kBarFullK], &bar[kBarEmptyK], table, nblk, n_kv, h,
+        tc_produce<D, B, kTcKStages>(&tmap_k, smem + Lay::kK, &bar[kBarFullK], &bar[kBarEmptyK], table, nblk, n_kv, h,
                                   p.num_blocks, abort, lane);
         return;
     }
     if (warp == kTcWarpV) {
-        tc_produce<B, kTcVStages>(&tmap_v, smem + Lay::kV, &bar[kBarFullV], &bar[kBarEmptyV], table, nblk, n_kv, h,
+        tc_produce<D, B, kTcVStages>(&tmap_v, smem + Lay::kV, &bar[kBarFullV], &bar[kBarEmptyV], table, nblk, n_kv, h,
                                   p.num_blocks, abort, lane);
         return;
     }
@@ -498,7 +499,7 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
     {
         const uint4 *src = reinterpret_cast<const uint4 *>(p.query + ((size_t)(q_begin + (valid ? rl : 0)) * p.num_heads + h) * D);
 #pragma unroll
-        for (int c = 8 * hh; c < 8 * hh + 8; ++c) {
+        for (int c = hh * (D / 16); c < (hh + 1) * (D / 16); ++c) {  // this half's 16-byte chunks
             const uint4 v = valid ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
             st_shared_v4(tc_chunk(sbase + Lay::kQ, t, c), v);
         }
@@ -506,7 +507,8 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar[kBarQ]);
     }
-    constexpr int HC = kTcKv / 2;  // columns per thread
+    constexpr int HC = kTcKv / 2;  // S / P columns per thread
+    constexpr int OC = D / 2;      // O columns per thread
     const float c2 = p.qk_scale_log2;  // > 0 on this path
     const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     float m_ref = -INFINITY, l = 0.f;
@@ -575,12 +577,12 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
             if (!tc_wait_warp(&bar[kBarOReady], (j - 1) & 1, abort)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll
-            for (int q = 0; q < HC / 32; ++q) {
+            for (int q = 0; q < OC / 32; ++q) {
                 float ov[32];
-                tmem_ld32(tl + 256 + hh * HC + q * 32, ov);
+                tmem_ld32(tl + 256 + hh * OC + q * 32, ov);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) ov[i] *= alpha;
-                tmem_st32(tl + 256 + hh * HC + q * 32, ov);
+                tmem_st32(tl + 256 + hh * OC + q * 32, ov);
             }
         }
         {  // P into the first half of this warp's S columns (read above)
@@ -598,7 +600,8 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
             if (tt + t >= L) {
                 const uint32_t v_addr = sbase + Lay::kV + vst * Lay::kTile;
 #pragma unroll
-                for (int c = 8 * hh; c < 8 * hh + 8; ++c) st_shared_v4(tc_chunk(v_addr, t, c), make_uint4(0, 0, 0, 0));
+                for (int c = hh * (D / 16); c < (hh + 1) * (D / 16); ++c)
+                    st_shared_v4(tc_chunk(v_addr, t, c), make_uint4(0, 0, 0, 0));
             }
             fence_proxy_async_smem();
         }
@@ -619,11 +622,11 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
     if (ok && tc_wait_warp(&bar[kBarOReady], (n_kv - 1) & 1, abort)) {
         tc_fence_after();
         const float inv = valid ? 1.0f / l : 0.f;
-        __half *op = p.out + ((size_t)(q_begin + (valid ? rl : 0)) * p.num_heads + h) * D + hh * HC;
+        __half *op = p.out + ((size_t)(q_begin + (valid ? rl : 0)) * p.num_heads + h) * D + hh * OC;
 #pragma unroll
-        for (int q = 0; q < HC / 32; ++q) {
+        for (int q = 0; q < OC / 32; ++q) {
             float ov[32];
-            tmem_ld32(tl + 256 + hh * HC + q * 32, ov);
+            tmem_ld32(tl + 256 + hh * OC + q * 32, ov);
             if (valid) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {

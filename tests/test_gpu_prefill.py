@@ -2,8 +2,9 @@
 
 Bars: prefill slots and the chunk's cache write bit-exact; attention within
 max-abs 2e-3 (fp16 cache, the decode's bar: fp16 operands with P rounded to
-fp16, fp32 accumulation). head_size 128 runs on the tcgen05 kernel (128-row
-tiles), head_size 64 and scales <= 0 on the mma.sync kernel (64-row tiles).
+fp16, fp32 accumulation). head_size 64 and 128 with a positive scale run on the
+tcgen05 kernel (128-row tiles), scales <= 0 on the mma.sync kernel (64-row
+tiles).
 Full sizes are checked on sampled (row, head) pairs that include every
 sequence's first and last rows and the rows on both sides of each 64-row
 tile edge.
@@ -188,9 +189,10 @@ def test_prefill_is_deterministic(cuda_device):
     assert torch.equal(first, dp.out)
 
 
-def test_non_positive_scale(cuda_device):
+@pytest.mark.parametrize("D,B", [(64, 16), (64, 32), (128, 16), (128, 32)])
+def test_non_positive_scale(cuda_device, D, B):
     # a scale <= 0 (a degenerate but valid input) is computed on the warp-MMA path
-    w = ragged_prefill(128, 32, seed=6)
+    w = ragged_prefill(D, B, seed=6 + D + B)
     for sc in (-w.scale, 0.0):
         w.scale = sc
         dp = run_prefill(w, cuda_device)
