@@ -66,7 +66,8 @@ extern "C" {
 #define PA_DEV_WAIT_TIMEOUT 32u   /* an on-chip pipeline wait ran out (never expected) */
 #define PA_DEV_PREFIX 64u         /* shared-prefix contract broken (see ..._shared_prefix) */
 #define PA_DEV_BAD_CHUNK 128u     /* prefill chunk longer than its context (or than
-                                     max_query_len given to pa_paged_prefill): skipped */
+                                     max_query_len given to pa_paged_prefill), or
+                                     rows outside [0, total_q): skipped */
 
 /* KV cache element type: fp16, or OCP FP8 E4M3 ("fn" variant: no infinities,
  * max 448) with one fp32 scale per cache tensor ([P1] §3.3, [P3] §4). */
@@ -100,8 +101,8 @@ typedef struct {
     int32_t units_per_cta;
 } pa_decode_config;
 
-/* Library version: 100 * minor + patch for 0.minor.patch (200 = 0.2.0, the
- * release that adds the paged prefill calls). */
+/* Library version: 100 * minor + patch for 0.minor.patch (201 = 0.2.1: the
+ * paged prefill calls, which take total_q since 0.2.1). */
 int pa_version(void);
 
 /* Message for the last nonzero status returned on this thread ("" if none). */
@@ -312,7 +313,12 @@ int pa_paged_attention_decode_noalloc(void *out, const void *query,
  *   L_s - n_s + i.
  * query_start: int32 [num_seqs + 1], non-decreasing, query_start[0] = 0
  * (device). A full prompt has n_s = L_s; a chunk after cached context has
- * n_s < L_s; n_s = 1 is a decode step. */
+ * n_s < L_s; n_s = 1 is a decode step.
+ * total_q: the rows the caller allocated for the chunk's tokens (query, out,
+ * slot_mapping), normally query_start[num_seqs]. A sequence whose rows do
+ * not lie inside [0, total_q) (query_start negative, decreasing or past
+ * total_q) is touched nowhere and sets PA_DEV_BAD_CHUNK; total_q = 0 is a
+ * no-op. */
 
 /* Slot of every new token of the chunk ([P3] §2.2 slot mapping, at each
  * token's position):
@@ -326,8 +332,8 @@ int pa_paged_attention_decode_noalloc(void *out, const void *query,
  * slots store the chunk's K/V before pa_paged_prefill reads them. */
 int pa_prefill_slot_mapping(int32_t *slot_mapping, const int32_t *query_start,
                             const int32_t *block_tables, int max_blocks_per_seq,
-                            const int32_t *context_lens, int num_seqs, int max_query_len,
-                            pa_cache_desc cache, void *stream);
+                            const int32_t *context_lens, int num_seqs, int total_q,
+                            int max_query_len, pa_cache_desc cache, void *stream);
 
 /* Causal attention of packed query rows over the paged cache:
  *   out[r][h] = sum_{t <= pos(r)} softmax_t(scale * q[r][h] . K_t[h]) V_t[h]
@@ -347,8 +353,8 @@ int pa_prefill_slot_mapping(int32_t *slot_mapping, const int32_t *query_start,
 int pa_paged_prefill(void *out, const void *query, const int32_t *query_start,
                      const void *key_cache, const void *value_cache, pa_cache_desc cache,
                      const int32_t *block_tables, int max_blocks_per_seq,
-                     const int32_t *context_lens, int num_seqs, int max_query_len, float scale,
-                     void *stream);
+                     const int32_t *context_lens, int num_seqs, int total_q, int max_query_len,
+                     float scale, void *stream);
 
 #ifdef __cplusplus
 }

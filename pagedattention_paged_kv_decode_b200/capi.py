@@ -72,8 +72,8 @@ SIGNATURES = {
     "pa_shared_prefix_workspace_size": (ctypes.c_size_t, [CacheDesc, _I, _I, _I, ctypes.POINTER(DecodeConfig)]),
     "pa_paged_attention_decode_noalloc": (_I, [_P, _P, _P, _P, CacheDesc, _P, _I, _P, _I, _I, _F, _F,
                                                _F, _P]),
-    "pa_prefill_slot_mapping": (_I, [_P, _P, _P, _I, _P, _I, _I, CacheDesc, _P]),
-    "pa_paged_prefill": (_I, [_P, _P, _P, _P, _P, CacheDesc, _P, _I, _P, _I, _I, _F, _P]),
+    "pa_prefill_slot_mapping": (_I, [_P, _P, _P, _I, _P, _I, _I, _I, CacheDesc, _P]),
+    "pa_paged_prefill": (_I, [_P, _P, _P, _P, _P, CacheDesc, _P, _I, _P, _I, _I, _I, _F, _P]),
 }
 
 _lib = None

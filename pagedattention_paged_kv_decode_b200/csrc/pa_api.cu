@@ -493,7 +493,7 @@ int current_device(int *dev) {
 
 extern "C" {
 
-int pa_version(void) { return 200; }
+int pa_version(void) { return 201; }
 
 const char *pa_last_error(void) { return g_msg; }
 
@@ -964,20 +964,21 @@ int prefill_stages(const pa_cache_desc &c) {
 
 extern "C" int pa_prefill_slot_mapping(int32_t *slot_mapping, const int32_t *query_start,
                                        const int32_t *block_tables, int max_blocks_per_seq,
-                                       const int32_t *context_lens, int num_seqs, int max_query_len,
-                                       pa_cache_desc cache, void *stream) {
+                                       const int32_t *context_lens, int num_seqs, int total_q,
+                                       int max_query_len, pa_cache_desc cache, void *stream) {
     int rc = check_cache(cache);
     if (rc) return rc;
     if (num_seqs < 0 || num_seqs > 65535) return fail(PA_ERR_INVALID, "num_seqs %d not in [0, 65535]", num_seqs);
+    if (total_q < 0) return fail(PA_ERR_INVALID, "total_q %d < 0", total_q);
     if (max_query_len < 0) return fail(PA_ERR_INVALID, "max_query_len %d < 0", max_query_len);
-    if (num_seqs == 0) return ok();
+    if (num_seqs == 0 || total_q == 0) return ok();
     if (!slot_mapping || !query_start || !block_tables || !context_lens)
         return fail(PA_ERR_INVALID, "null pointer argument");
     if (max_blocks_per_seq < 1) return fail(PA_ERR_INVALID, "max_blocks_per_seq < 1");
     const int threads = 256;
     const int gx = std::max(1, std::min((max_query_len + threads - 1) / threads, 1024));
     pa::prefill_slot_mapping_kernel<<<dim3(gx, num_seqs), threads, 0, static_cast<cudaStream_t>(stream)>>>(
-        slot_mapping, query_start, block_tables, max_blocks_per_seq, context_lens, cache.block_size,
+        slot_mapping, total_q, query_start, block_tables, max_blocks_per_seq, context_lens, cache.block_size,
         cache.num_blocks);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "prefill_slot_mapping_kernel launch");
@@ -987,14 +988,15 @@ extern "C" int pa_prefill_slot_mapping(int32_t *slot_mapping, const int32_t *que
 extern "C" int pa_paged_prefill(void *out, const void *query, const int32_t *query_start,
                                 const void *key_cache, const void *value_cache, pa_cache_desc cache,
                                 const int32_t *block_tables, int max_blocks_per_seq,
-                                const int32_t *context_lens, int num_seqs, int max_query_len,
+                                const int32_t *context_lens, int num_seqs, int total_q, int max_query_len,
                                 float scale, void *stream) {
     int rc = check_cache(cache);
     if (rc) return rc;
     if (cache.dtype != PA_F16) return fail(PA_ERR_DTYPE, "paged prefill supports fp16 caches only");
     if (num_seqs < 0 || num_seqs > 65535) return fail(PA_ERR_INVALID, "num_seqs %d not in [0, 65535]", num_seqs);
+    if (total_q < 0) return fail(PA_ERR_INVALID, "total_q %d < 0", total_q);
     if (max_query_len < 0) return fail(PA_ERR_INVALID, "max_query_len %d < 0", max_query_len);
-    if (num_seqs == 0 || max_query_len == 0) return ok();
+    if (num_seqs == 0 || total_q == 0 || max_query_len == 0) return ok();
     if (!out || !query || !query_start || !key_cache || !value_cache || !block_tables || !context_lens)
         return fail(PA_ERR_INVALID, "null pointer argument");
     if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache))
@@ -1030,6 +1032,7 @@ extern "C" int pa_paged_prefill(void *out, const void *query, const int32_t *que
     p.block_tables = block_tables;
     p.context_lens = context_lens;
     p.num_seqs = num_seqs;
+    p.total_q = total_q;
     p.num_heads = cache.num_heads;
     p.num_blocks = cache.num_blocks;
     p.max_blocks_per_seq = max_blocks_per_seq;

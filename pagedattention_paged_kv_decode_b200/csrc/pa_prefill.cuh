@@ -23,6 +23,7 @@ struct PrefillParams {
     const int32_t *block_tables;  // [S][max_blocks_per_seq]
     const int32_t *context_lens;  // [S]
     int num_seqs;
+    int total_q;                  // rows of query and out
     int num_heads;
     int num_blocks;
     int max_blocks_per_seq;
@@ -32,17 +33,31 @@ struct PrefillParams {
     float qk_scale_log2;          // scale * log2(e)
 };
 
+// Rows [q_begin, q_begin + n) of sequence s. False when they do not lie
+// inside the total_q rows the caller allocated (query_start negative,
+// decreasing or past total_q): such a sequence is touched nowhere.
+__device__ __forceinline__ bool chunk_rows(const int32_t *query_start, int s, int total_q, int &q_begin,
+                                           int &n) {
+    const int64_t a = __ldg(query_start + s), b = __ldg(query_start + s + 1);
+    q_begin = (int)a;
+    n = (int)(b - a);
+    return a >= 0 && b >= a && b <= total_q;
+}
+
 // a1 for a prefill chunk: one thread per new token, grid (row chunks, S);
 // rows beyond the grid are covered by the stride loop.
-__global__ void prefill_slot_mapping_kernel(int32_t *__restrict__ slot_mapping,
+__global__ void prefill_slot_mapping_kernel(int32_t *__restrict__ slot_mapping, int total_q,
                                             const int32_t *__restrict__ query_start,
                                             const int32_t *__restrict__ block_tables,
                                             int max_blocks_per_seq,
                                             const int32_t *__restrict__ context_lens, int block_size,
                                             int num_blocks) {
     const int s = blockIdx.y;
-    const int q0 = query_start[s];
-    const int n = query_start[s + 1] - q0;
+    int q0, n;
+    if (!chunk_rows(query_start, s, total_q, q0, n)) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) flag_error(PA_DEV_BAD_CHUNK);
+        return;
+    }
     const int L = context_lens[s];
     const bool bad_chunk = n > L;
     if (bad_chunk && blockIdx.x == 0 && threadIdx.x == 0) flag_error(PA_DEV_BAD_CHUNK);
@@ -91,10 +106,13 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
     const int sh = blockIdx.x / p.row_tiles;
     const int h = sh % p.num_heads;
     const int s = sh / p.num_heads;
-    const int q_begin = __ldg(p.query_start + s);
-    const int n = __ldg(p.query_start + s + 1) - q_begin;
+    int q_begin, n;
+    if (!chunk_rows(p.query_start, s, p.total_q, q_begin, n)) {
+        if (t_rev == 0 && h == 0 && threadIdx.x == 0) flag_error(PA_DEV_BAD_CHUNK);
+        return;
+    }
     const int L = __ldg(p.context_lens + s);
-    if (n <= 0) return;
+    if (n == 0) return;
     if (n > L || n > p.max_query_len) {  // the whole sequence is skipped
         if (t_rev == 0 && h == 0 && threadIdx.x == 0) flag_error(PA_DEV_BAD_CHUNK);
         return;
@@ -372,10 +390,13 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
     const int sh = blockIdx.x / p.row_tiles;
     const int h = sh % p.num_heads;
     const int s = sh / p.num_heads;
-    const int q_begin = __ldg(p.query_start + s);
-    const int n = __ldg(p.query_start + s + 1) - q_begin;
+    int q_begin, n;
+    if (!chunk_rows(p.query_start, s, p.total_q, q_begin, n)) {
+        if (t_rev == 0 && h == 0 && threadIdx.x == 0) flag_error(PA_DEV_BAD_CHUNK);
+        return;
+    }
     const int L = __ldg(p.context_lens + s);
-    if (n <= 0) return;
+    if (n == 0) return;
     if (n > L || n > p.max_query_len) {
         if (t_rev == 0 && h == 0 && threadIdx.x == 0) flag_error(PA_DEV_BAD_CHUNK);
         return;

@@ -366,8 +366,10 @@ def prefill_slot_mapping(query_start: torch.Tensor, block_tables: torch.Tensor,
             raise ValueError("give out or total_q")
         out = torch.empty(int(total_q), dtype=torch.int32, device=context_lens.device)
     _i32(out, "out")
+    if out.dim() != 1 or (total_q is not None and out.shape[0] != int(total_q)):
+        raise ValueError("out must be a 1-D int32 tensor of total_q entries")
     check(lib().pa_prefill_slot_mapping(out.data_ptr(), query_start.data_ptr(), block_tables.data_ptr(),
-                                        block_tables.shape[1], context_lens.data_ptr(), S,
+                                        block_tables.shape[1], context_lens.data_ptr(), S, out.shape[0],
                                         int(max_query_len), cache_desc(key_cache), _stream(stream)))
     return out
 
@@ -392,8 +394,8 @@ def paged_prefill(out: torch.Tensor, query: torch.Tensor, query_start: torch.Ten
         raise ValueError("query heads/head_size differ from the cache's")
     check(lib().pa_paged_prefill(out.data_ptr(), query.data_ptr(), query_start.data_ptr(),
                                  key_cache.data_ptr(), value_cache.data_ptr(), desc, block_tables.data_ptr(),
-                                 block_tables.shape[1], context_lens.data_ptr(), S, int(max_query_len),
-                                 float(scale), _stream(stream)))
+                                 block_tables.shape[1], context_lens.data_ptr(), S, query.shape[0],
+                                 int(max_query_len), float(scale), _stream(stream)))
 
 
 def prefill_step(out: torch.Tensor, query: torch.Tensor, new_key: torch.Tensor, new_value: torch.Tensor,

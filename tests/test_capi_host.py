@@ -34,7 +34,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_version_and_empty_error():
-    assert capi.lib().pa_version() == 200
+    assert capi.lib().pa_version() == 201
 
 
 F = capi.CacheDesc(64, 16, 8, 128, capi.PA_F16)
@@ -153,23 +153,29 @@ def test_config_validation_and_workspace_size():
 def test_prefill_argument_checks():
     L = capi.lib()
     E = capi.CacheDesc(64, 16, 8, 128, capi.PA_E4M3)
-    # (out, query, query_start, kc, vc, desc, tables, width, ctx, S, max_query_len, scale, stream)
-    assert L.pa_paged_prefill(P, P, P, P, P, E, P, 4, P, 2, 64, 0.1, None) == capi.PA_ERR_DTYPE
+    T = 100  # total_q
+    # (out, query, query_start, kc, vc, desc, tables, width, ctx, S, total_q, max_query_len, scale, stream)
+    assert L.pa_paged_prefill(P, P, P, P, P, E, P, 4, P, 2, T, 64, 0.1, None) == capi.PA_ERR_DTYPE
     assert "fp16" in _last()
-    assert L.pa_paged_prefill(P, P, P, P, P, F, P, 4, P, -1, 64, 0.1, None) == capi.PA_ERR_INVALID
-    assert L.pa_paged_prefill(P, P, P, P, P, F, P, 4, P, 2, -3, 0.1, None) == capi.PA_ERR_INVALID
-    assert L.pa_paged_prefill(P, P, None, P, P, F, P, 4, P, 2, 64, 0.1, None) == capi.PA_ERR_INVALID
-    assert L.pa_paged_prefill(P, P + 4, P, P, P, F, P, 4, P, 2, 64, 0.1, None) == capi.PA_ERR_INVALID
-    assert L.pa_paged_prefill(P, P, P, P, P, F, P, 0, P, 2, 64, 0.1, None) == capi.PA_ERR_INVALID
-    assert L.pa_paged_prefill(P, P, P, P, P, F, P, 4, P, 2, 64, float("nan"), None) == capi.PA_ERR_INVALID
-    assert L.pa_paged_prefill(P, P, P, P, P, capi.CacheDesc(64, 16, 8, 96, 0), P, 4, P, 2, 64, 0.1,
+    assert L.pa_paged_prefill(P, P, P, P, P, F, P, 4, P, -1, T, 64, 0.1, None) == capi.PA_ERR_INVALID
+    assert L.pa_paged_prefill(P, P, P, P, P, F, P, 4, P, 2, -5, 64, 0.1, None) == capi.PA_ERR_INVALID
+    assert "total_q" in _last()
+    assert L.pa_paged_prefill(P, P, P, P, P, F, P, 4, P, 2, T, -3, 0.1, None) == capi.PA_ERR_INVALID
+    assert L.pa_paged_prefill(P, P, None, P, P, F, P, 4, P, 2, T, 64, 0.1, None) == capi.PA_ERR_INVALID
+    assert L.pa_paged_prefill(P, P + 4, P, P, P, F, P, 4, P, 2, T, 64, 0.1, None) == capi.PA_ERR_INVALID
+    assert L.pa_paged_prefill(P, P, P, P, P, F, P, 0, P, 2, T, 64, 0.1, None) == capi.PA_ERR_INVALID
+    assert L.pa_paged_prefill(P, P, P, P, P, F, P, 4, P, 2, T, 64, float("nan"), None) == capi.PA_ERR_INVALID
+    assert L.pa_paged_prefill(P, P, P, P, P, capi.CacheDesc(64, 16, 8, 96, 0), P, 4, P, 2, T, 64, 0.1,
                               None) == capi.PA_ERR_INVALID
     # nothing to do: no launch, no CUDA call
-    assert L.pa_paged_prefill(None, None, None, None, None, F, None, 4, None, 0, 64, 0.1, None) == capi.PA_OK
-    assert L.pa_paged_prefill(None, None, None, None, None, F, None, 4, None, 3, 0, 0.1, None) == capi.PA_OK
-    # (slots, query_start, tables, width, ctx, S, max_query_len, desc, stream)
-    assert L.pa_prefill_slot_mapping(P, None, P, 4, P, 2, 64, F, None) == capi.PA_ERR_INVALID
-    assert L.pa_prefill_slot_mapping(P, P, P, 0, P, 2, 64, F, None) == capi.PA_ERR_INVALID
-    assert L.pa_prefill_slot_mapping(P, P, P, 4, P, 2, -1, F, None) == capi.PA_ERR_INVALID
-    assert L.pa_prefill_slot_mapping(P, P, P, 4, P, 70000, 64, F, None) == capi.PA_ERR_INVALID
-    assert L.pa_prefill_slot_mapping(None, None, None, 4, None, 0, 64, F, None) == capi.PA_OK
+    assert L.pa_paged_prefill(None, None, None, None, None, F, None, 4, None, 0, T, 64, 0.1, None) == capi.PA_OK
+    assert L.pa_paged_prefill(None, None, None, None, None, F, None, 4, None, 3, T, 0, 0.1, None) == capi.PA_OK
+    assert L.pa_paged_prefill(None, None, None, None, None, F, None, 4, None, 3, 0, 64, 0.1, None) == capi.PA_OK
+    # (slots, query_start, tables, width, ctx, S, total_q, max_query_len, desc, stream)
+    assert L.pa_prefill_slot_mapping(P, None, P, 4, P, 2, T, 64, F, None) == capi.PA_ERR_INVALID
+    assert L.pa_prefill_slot_mapping(P, P, P, 0, P, 2, T, 64, F, None) == capi.PA_ERR_INVALID
+    assert L.pa_prefill_slot_mapping(P, P, P, 4, P, 2, T, -1, F, None) == capi.PA_ERR_INVALID
+    assert L.pa_prefill_slot_mapping(P, P, P, 4, P, 2, -1, 64, F, None) == capi.PA_ERR_INVALID
+    assert L.pa_prefill_slot_mapping(P, P, P, 4, P, 70000, T, 64, F, None) == capi.PA_ERR_INVALID
+    assert L.pa_prefill_slot_mapping(None, None, None, 4, None, 0, T, 64, F, None) == capi.PA_OK
+    assert L.pa_prefill_slot_mapping(None, None, None, 4, None, 2, 0, 64, F, None) == capi.PA_OK

@@ -198,3 +198,46 @@ def test_non_positive_scale(cuda_device, D, B):
         dp = run_prefill(w, cuda_device)
         assert pk.check_status() == 0
         check(w, dp)
+
+
+def test_rows_outside_total_q_are_flagged_and_untouched(cuda_device):
+    # query_start past the rows the caller holds, or negative: that sequence
+    # is skipped and flagged; guard rows after the views stay as they were
+    w = ragged_prefill(128, 16, seed=7)
+    dp = run_prefill(w, cuda_device)
+    assert pk.check_status() == 0
+    good = dp.out.clone()
+    T, H, D = dp.out.shape
+    mql = int(w.chunk_lens.max())
+    out_full = torch.full((T + 8, H, D), 7.0, dtype=torch.float16, device=cuda_device)
+    q_full = torch.zeros((T + 8, H, D), dtype=torch.float16, device=cuda_device)
+    q_full[:T] = dp.query
+    slots_full = torch.full((T + 8,), 12345, dtype=torch.int32, device=cuda_device)
+
+    # the last sequence (an empty chunk, context 9) claims 5 rows past total_q
+    qs = dp.query_start.clone()
+    qs[-1] = T + 5
+    pk.paged_prefill(out_full[:T], q_full[:T], qs, dp.key_cache, dp.value_cache, dp.block_tables,
+                     dp.context_lens, mql, w.scale)
+    assert pk.check_status() & capi.PA_DEV_BAD_CHUNK
+    assert torch.equal(out_full[:T], good)
+    assert bool((out_full[T:] == 7.0).all())
+    pk.prefill_slot_mapping(qs, dp.block_tables, dp.context_lens, dp.key_cache, mql, out=slots_full[:T])
+    assert pk.check_status() & capi.PA_DEV_BAD_CHUNK
+    assert torch.equal(slots_full[:T], dp.slots)
+    assert bool((slots_full[T:] == 12345).all())
+
+    # a negative start: sequence 0 (context raised to 4, so that its 4 rows
+    # fit the context and only the row range is wrong) is skipped
+    qs = dp.query_start.clone()
+    qs[0] = -3
+    ctx = dp.context_lens.clone()
+    ctx[0] = 4
+    out_full.fill_(7.0)
+    pk.paged_prefill(out_full[:T], q_full[:T], qs, dp.key_cache, dp.value_cache, dp.block_tables,
+                     ctx, mql, w.scale)
+    assert pk.check_status() & capi.PA_DEV_BAD_CHUNK
+    r1 = int(w.query_start[1])
+    assert bool((out_full[:r1] == 7.0).all())
+    assert torch.equal(out_full[r1:T], good[r1:])
+    assert bool((out_full[T:] == 7.0).all())
