@@ -49,15 +49,69 @@ def _i32(t: torch.Tensor, name: str) -> torch.Tensor:
     return t
 
 
+def _on_current_device(*tensors) -> None:
+    """The library launches on the current CUDA device; a device tensor on
+    another GPU would be a foreign pointer there."""
+    dev = None
+    for t in tensors:
+        if t is None or not t.is_cuda:
+            continue
+        if dev is None:
+            dev = torch.cuda.current_device()
+        if t.device.index != dev:
+            raise ValueError(f"a tensor is on {t.device}, but the current CUDA device is cuda:{dev}")
+
+
+def _table(block_tables: torch.Tensor, S: int) -> None:
+    _i32(block_tables, "block_tables")
+    if block_tables.dim() != 2 or block_tables.shape[0] < S:
+        raise ValueError("block_tables must be int32 [num_seqs, max_blocks_per_seq]")
+
+
+def _f16_3d(t: torch.Tensor, name: str, shape=None, rows_only: bool = False) -> None:
+    """fp16 CUDA [n, H, D]; contiguous, or (rows_only) contiguous within a token."""
+    if t.dtype != torch.float16 or not t.is_cuda or t.dim() != 3:
+        raise ValueError(f"{name} must be a float16 CUDA tensor [n, H, D]")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if rows_only:
+        if t.stride(2) != 1 or t.stride(1) != t.shape[2]:
+            raise ValueError(f"{name} rows must be contiguous within a token")
+    elif not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _slots_out(slot_mapping: torch.Tensor | None, S: int) -> None:
+    if slot_mapping is not None:
+        _i32(slot_mapping, "slot_mapping")
+        if slot_mapping.dim() != 1 or slot_mapping.shape[0] < S:
+            raise ValueError("slot_mapping must be int32 [num_seqs]")
+
+
+def _workspace(workspace: torch.Tensor | None):
+    if workspace is None:
+        return None, 0
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    return workspace.data_ptr(), workspace.numel() * workspace.element_size()
+
+
+def _pairs(src_dst_pairs: torch.Tensor) -> None:
+    _i32(src_dst_pairs, "src_dst_pairs")
+    if src_dst_pairs.dim() != 2 or src_dst_pairs.shape[1] != 2:
+        raise ValueError("src_dst_pairs must be int32 [n_pairs, 2]")
+
+
 def slot_mapping(block_tables: torch.Tensor, context_lens: torch.Tensor, key_cache: torch.Tensor,
                  out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """Slot of each sequence's appended token (position context_len - 1)."""
-    _i32(block_tables, "block_tables")
     _i32(context_lens, "context_lens")
     S = context_lens.shape[0]
+    _table(block_tables, S)
     if out is None:
         out = torch.empty(S, dtype=torch.int32, device=context_lens.device)
-    _i32(out, "out")
+    _slots_out(out, S)
+    _on_current_device(block_tables, context_lens, out)
     check(lib().pa_slot_mapping(out.data_ptr(), block_tables.data_ptr(), block_tables.shape[1],
                                 context_lens.data_ptr(), S, cache_desc(key_cache), _stream(stream)))
     return out
@@ -70,11 +124,10 @@ def kv_cache_write(key: torch.Tensor, value: torch.Tensor, key_cache: torch.Tens
     _check_pair(key_cache, value_cache)
     _i32(slot_mapping, "slot_mapping")
     n = slot_mapping.shape[0]
-    for t in (key, value):
-        if t.dtype != torch.float16 or not t.is_cuda or t.dim() != 3 or t.shape[0] != n:
-            raise ValueError("key/value must be float16 CUDA tensors [n_tokens, H, D]")
-        if t.stride(2) != 1 or t.stride(1) != t.shape[2]:
-            raise ValueError("key/value rows must be contiguous within a token")
+    _, _, H, D = key_cache.shape
+    _f16_3d(key, "key", (n, H, D), rows_only=True)
+    _f16_3d(value, "value", (n, H, D), rows_only=True)
+    _on_current_device(key, value, key_cache, value_cache, slot_mapping)
     check(lib().pa_kv_cache_write(key.data_ptr(), value.data_ptr(), key.stride(0), value.stride(0),
                                   key_cache.data_ptr(), value_cache.data_ptr(), cache_desc(key_cache),
                                   slot_mapping.data_ptr(), n, float(k_scale), float(v_scale),
@@ -85,8 +138,9 @@ def copy_blocks(key_cache: torch.Tensor, value_cache: torch.Tensor, src_dst_pair
                 stream=None) -> None:
     """Copy whole physical blocks (both caches) for each (src, dst) pair."""
     _check_pair(key_cache, value_cache)
-    _i32(src_dst_pairs, "src_dst_pairs")
-    n = src_dst_pairs.numel() // 2
+    _pairs(src_dst_pairs)
+    n = src_dst_pairs.shape[0]
+    _on_current_device(key_cache, value_cache, src_dst_pairs)
     check(lib().pa_copy_blocks(key_cache.data_ptr(), value_cache.data_ptr(), cache_desc(key_cache),
                                src_dst_pairs.data_ptr(), n, _stream(stream)))
 
@@ -106,8 +160,9 @@ def swap_blocks(dst_key_cache: torch.Tensor, dst_value_cache: torch.Tensor,
             raise ValueError("a CPU pool must be pinned (pin_memory())")
     if dst_key_cache.shape[1:] != src_key_cache.shape[1:] or dst_key_cache.dtype != src_key_cache.dtype:
         raise ValueError("source and destination block shapes differ")
-    _i32(src_dst_pairs, "src_dst_pairs")
-    n = src_dst_pairs.numel() // 2
+    _pairs(src_dst_pairs)
+    n = src_dst_pairs.shape[0]
+    _on_current_device(dst_key_cache, dst_value_cache, src_key_cache, src_value_cache, src_dst_pairs)
     check(lib().pa_swap_blocks(dst_key_cache.data_ptr(), dst_value_cache.data_ptr(),
                                dst_key_cache.shape[0], src_key_cache.data_ptr(),
                                src_value_cache.data_ptr(), src_key_cache.shape[0],
@@ -159,11 +214,13 @@ def paged_attention_decode(out: torch.Tensor, query: torch.Tensor, key_cache: to
     S, H, D = query.shape
     if out.shape != query.shape or context_lens.shape[0] != S or block_tables.shape[0] != S:
         raise ValueError("shape mismatch between out, query, block_tables and context_lens")
+    _table(block_tables, S)
     desc = cache_desc(key_cache)
     if desc.num_heads != H or desc.head_size != D:
         raise ValueError("query heads/head_size differ from the cache's")
     if max_context_len is None:
         max_context_len = block_tables.shape[1] * desc.block_size
+    _on_current_device(out, query, key_cache, value_cache, block_tables, context_lens, workspace)
     args = (out.data_ptr(), query.data_ptr(), key_cache.data_ptr(), value_cache.data_ptr(), desc,
             block_tables.data_ptr(), block_tables.shape[1], context_lens.data_ptr(), S,
             int(max_context_len), float(scale), float(k_scale), float(v_scale))
@@ -171,11 +228,7 @@ def paged_attention_decode(out: torch.Tensor, query: torch.Tensor, key_cache: to
         check(lib().pa_paged_attention_decode(*args, _stream(stream)))
         return
     cfg = _config(config)
-    ws_ptr, ws_bytes = None, 0
-    if workspace is not None:
-        if not workspace.is_cuda or not workspace.is_contiguous():
-            raise ValueError("workspace must be a contiguous CUDA tensor")
-        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    ws_ptr, ws_bytes = _workspace(workspace)
     check(lib().pa_paged_attention_decode_ws(*args, ctypes.byref(cfg) if cfg is not None else None,
                                              ws_ptr, ws_bytes, _stream(stream)))
 
@@ -204,17 +257,17 @@ def paged_attention_decode_append(out: torch.Tensor, query: torch.Tensor, new_ke
             raise ValueError("new_key/new_value rows must be contiguous within a token")
     if out.shape != query.shape or context_lens.shape[0] != S or block_tables.shape[0] != S:
         raise ValueError("shape mismatch between out, query, block_tables and context_lens")
+    _table(block_tables, S)
     desc = cache_desc(key_cache)
     if desc.num_heads != H or desc.head_size != D:
         raise ValueError("query heads/head_size differ from the cache's")
     if max_context_len is None:
         max_context_len = block_tables.shape[1] * desc.block_size
-    if slot_mapping is not None:
-        _i32(slot_mapping, "slot_mapping")
+    _slots_out(slot_mapping, S)
     cfg = _config(config)
-    ws_ptr, ws_bytes = None, 0
-    if workspace is not None:
-        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    ws_ptr, ws_bytes = _workspace(workspace)
+    _on_current_device(out, query, new_key, new_value, key_cache, value_cache, block_tables, context_lens,
+                       slot_mapping, workspace)
     check(lib().pa_paged_attention_decode_append(
         out.data_ptr(), query.data_ptr(), new_key.data_ptr(), new_value.data_ptr(),
         new_key.stride(0), new_value.stride(0), key_cache.data_ptr(), value_cache.data_ptr(), desc,
@@ -249,15 +302,19 @@ def paged_attention_decode_shared_prefix(out: torch.Tensor, query: torch.Tensor,
         if t is not None and (t.dtype != torch.float16 or not t.is_cuda or tuple(t.shape) != (S, H, D)
                               or t.stride(2) != 1 or t.stride(1) != D):
             raise ValueError("new_key/new_value must be float16 CUDA tensors [S, H, D] with contiguous rows")
+    if out.shape != query.shape or context_lens.shape[0] != S or block_tables.shape[0] != S:
+        raise ValueError("shape mismatch between out, query, block_tables and context_lens")
+    _table(block_tables, S)
     desc = cache_desc(key_cache)
+    if desc.num_heads != H or desc.head_size != D:
+        raise ValueError("query heads/head_size differ from the cache's")
     if max_context_len is None:
         max_context_len = block_tables.shape[1] * desc.block_size
-    if slot_mapping is not None:
-        _i32(slot_mapping, "slot_mapping")
+    _slots_out(slot_mapping, S)
     cfg = _config(config)
-    ws_ptr, ws_bytes = None, 0
-    if workspace is not None:
-        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    ws_ptr, ws_bytes = _workspace(workspace)
+    _on_current_device(out, query, new_key, new_value, key_cache, value_cache, block_tables, context_lens,
+                       slot_mapping, workspace)
     check(lib().pa_paged_attention_decode_shared_prefix(
         out.data_ptr(), query.data_ptr(),
         new_key.data_ptr() if new_key is not None else None,
@@ -356,10 +413,10 @@ def prefill_slot_mapping(query_start: torch.Tensor, block_tables: torch.Tensor,
     ``total_q`` (= query_start[-1]) must be given when ``out`` is not, since
     reading it from the device would synchronise."""
     _i32(query_start, "query_start")
-    _i32(block_tables, "block_tables")
     _i32(context_lens, "context_lens")
     S = context_lens.shape[0]
-    if query_start.shape[0] != S + 1 or block_tables.shape[0] != S:
+    _table(block_tables, S)
+    if query_start.dim() != 1 or query_start.shape[0] != S + 1 or block_tables.shape[0] != S:
         raise ValueError("query_start must hold num_seqs + 1 entries and block_tables num_seqs rows")
     if out is None:
         if total_q is None:
@@ -368,6 +425,7 @@ def prefill_slot_mapping(query_start: torch.Tensor, block_tables: torch.Tensor,
     _i32(out, "out")
     if out.dim() != 1 or (total_q is not None and out.shape[0] != int(total_q)):
         raise ValueError("out must be a 1-D int32 tensor of total_q entries")
+    _on_current_device(query_start, block_tables, context_lens, out)
     check(lib().pa_prefill_slot_mapping(out.data_ptr(), query_start.data_ptr(), block_tables.data_ptr(),
                                         block_tables.shape[1], context_lens.data_ptr(), S, out.shape[0],
                                         int(max_query_len), cache_desc(key_cache), _stream(stream)))
@@ -381,17 +439,19 @@ def paged_prefill(out: torch.Tensor, query: torch.Tensor, query_start: torch.Ten
     paged fp16 cache, which must already hold each sequence's chunk."""
     _check_pair(key_cache, value_cache)
     _i32(query_start, "query_start")
-    _i32(block_tables, "block_tables")
     _i32(context_lens, "context_lens")
     for t in (out, query):
         if t.dtype != torch.float16 or not t.is_cuda or not t.is_contiguous() or t.dim() != 3:
             raise ValueError("out and query must be contiguous float16 CUDA tensors [total_q, H, D]")
     S = context_lens.shape[0]
-    if out.shape != query.shape or query_start.shape[0] != S + 1 or block_tables.shape[0] != S:
+    _table(block_tables, S)
+    if (out.shape != query.shape or query_start.dim() != 1 or query_start.shape[0] != S + 1
+            or block_tables.shape[0] != S):
         raise ValueError("shape mismatch between out, query, query_start, block_tables and context_lens")
     desc = cache_desc(key_cache)
     if desc.num_heads != query.shape[1] or desc.head_size != query.shape[2]:
         raise ValueError("query heads/head_size differ from the cache's")
+    _on_current_device(out, query, query_start, key_cache, value_cache, block_tables, context_lens)
     check(lib().pa_paged_prefill(out.data_ptr(), query.data_ptr(), query_start.data_ptr(),
                                  key_cache.data_ptr(), value_cache.data_ptr(), desc, block_tables.data_ptr(),
                                  block_tables.shape[1], context_lens.data_ptr(), S, query.shape[0],

@@ -219,3 +219,30 @@ def test_counts_above_one_grid_slice(cuda_device):
     oracle.copy_blocks(ek, ev, pairs)
     assert np.array_equal(gek.cpu().numpy(), ek)
     assert np.array_equal(gev.cpu().numpy(), ev)
+
+
+def test_binding_rejects_mismatched_tensors(cuda_device):
+    # every rejection happens on the host, before any launch
+    w, dw = small(cuda_device)
+    S, H, D = dw.query.shape
+    with pytest.raises(ValueError, match="key"):
+        pk.kv_cache_write(dw.new_key[:, :H - 1], dw.new_value[:, :H - 1], dw.key_cache, dw.value_cache,
+                          dw.slots)
+    with pytest.raises(ValueError, match="slot_mapping"):
+        pk.slot_mapping(dw.block_tables, dw.context_lens, dw.key_cache, out=dw.slots[:S - 1])
+    with pytest.raises(ValueError, match="block_tables"):
+        pk.slot_mapping(dw.block_tables[0], dw.context_lens, dw.key_cache)
+    with pytest.raises(ValueError, match="src_dst_pairs"):
+        pk.copy_blocks(dw.key_cache, dw.value_cache, torch.tensor([0, 1], dtype=torch.int32, device=cuda_device))
+    with pytest.raises(ValueError, match="slot_mapping"):
+        pk.paged_attention_decode_append(dw.out, dw.query, dw.new_key, dw.new_value, dw.key_cache,
+                                         dw.value_cache, dw.block_tables, dw.context_lens, w.scale,
+                                         slot_mapping=dw.slots[:S - 1])
+    with pytest.raises(ValueError, match="workspace"):
+        pk.paged_attention_decode_append(dw.out, dw.query, dw.new_key, dw.new_value, dw.key_cache,
+                                         dw.value_cache, dw.block_tables, dw.context_lens, w.scale,
+                                         workspace=torch.zeros(1 << 20, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="shape mismatch"):
+        pk.paged_attention_decode_shared_prefix(dw.out[:S - 1], dw.query, dw.key_cache, dw.value_cache,
+                                                dw.block_tables, dw.context_lens, 0, w.scale)
+    assert pk.check_status() == 0
