@@ -147,10 +147,11 @@ def test_seq_head_subset_matches_full():
         assert np.array_equal(sub[i], full[s, h])
 
 
-@pytest.mark.parametrize("scale_pow", [0, -3, 2])
-def test_e4m3_cache_equals_f16_cache_of_the_same_values(scale_pow):
+@pytest.mark.parametrize("k_pow,v_pow", [(0, 0), (-3, 2), (2, -1)])
+def test_e4m3_cache_equals_f16_cache_of_the_same_values(k_pow, v_pow):
     """Every E4M3 value times a power of two is exactly an fp16 value, so an E4M3
-    cache and an fp16 cache holding its decoded values must give equal outputs."""
+    cache and an fp16 cache holding its decoded values must give equal outputs.
+    Distinct K and V scales pin which scale goes with which cache."""
     rng = np.random.default_rng(13)
     nb, B, H, D = 6, 4, 2, 8
     codes_k = rng.integers(0, 256, (nb, B, H, D), dtype=np.uint8)
@@ -158,14 +159,15 @@ def test_e4m3_cache_equals_f16_cache_of_the_same_values(scale_pow):
     for c in (codes_k, codes_v):
         c[(c & 0x7F) == 0x7F] = 0x3C           # no NaN codes
         c[(c & 0x78) >= 0x60] &= 0x9F          # keep magnitudes small (exponent field < 12)
-    sc = float(2.0 ** scale_pow)
-    f16_k = (oracle.e4m3_to_double(codes_k) * sc).astype(np.float16)
-    f16_v = (oracle.e4m3_to_double(codes_v) * sc).astype(np.float16)
-    assert np.array_equal(f16_k.astype(np.float64), oracle.e4m3_to_double(codes_k) * sc)
+    sk, sv = float(2.0 ** k_pow), float(2.0 ** v_pow)
+    f16_k = (oracle.e4m3_to_double(codes_k) * sk).astype(np.float16)
+    f16_v = (oracle.e4m3_to_double(codes_v) * sv).astype(np.float16)
+    assert np.array_equal(f16_k.astype(np.float64), oracle.e4m3_to_double(codes_k) * sk)
+    assert np.array_equal(f16_v.astype(np.float64), oracle.e4m3_to_double(codes_v) * sv)
     q = rng.standard_normal((2, H, D)).astype(np.float16)
     bt = np.array([[3, 0, 5], [1, 4, -1]], np.int32)
     ctx = np.array([11, 6], np.int32)
-    a = oracle.paged_attention(q, codes_k, codes_v, bt, ctx, 0.25, k_scale=sc, v_scale=sc)
+    a = oracle.paged_attention(q, codes_k, codes_v, bt, ctx, 0.25, k_scale=sk, v_scale=sv)
     b = oracle.paged_attention(q, f16_k, f16_v, bt, ctx, 0.25)
     assert np.array_equal(a, b)
 

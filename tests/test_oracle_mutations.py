@@ -6,7 +6,8 @@ pin battery: the worked and growth slot examples, binary16 and E4M3 decoding
 against numpy/torch, E4M3 encoding against torch and the saturation points,
 dense attention on identity tables against torch's SDPA, the closed forms,
 exact-sum brute force, physical-block relabelling, cache-write read-back,
-block copy and swap semantics, the log-sum-exp identity, and for the
+block copy and swap semantics, E4M3 attention against fp16 caches holding
+the decoded values at distinct K and V scales, the log-sum-exp identity, and for the
 prefill the worked example as a full prompt, one-token chunks against the
 decode slots, and chunks after a cached context against torch's SDPA with a
 position mask. Every mutant
@@ -58,6 +59,12 @@ MUTANTS = {
                                                     "int pos = row - query_start[s];"),
     "prefill query row taken by sequence": ("const uint16_t *q = query + ((int64_t)row * num_heads + h) * head_size;",
                                             "const uint16_t *q = query + ((int64_t)s * num_heads + h) * head_size;"),
+    "keys dequantised with v_scale": ("cache_value(key_cache, kv_dtype, base + d, k_scale)",
+                                      "cache_value(key_cache, kv_dtype, base + d, v_scale)"),
+    "values dequantised with k_scale": ("cache_value(value_cache, kv_dtype, rowbase[i] + d, v_scale)",
+                                        "cache_value(value_cache, kv_dtype, rowbase[i] + d, k_scale)"),
+    "E4M3 cache scale dropped": ("return oracle_e4m3_to_double(((const uint8_t *)cache)[idx]) * scale;",
+                                 "return oracle_e4m3_to_double(((const uint8_t *)cache)[idx]);"),
     "head index ignored": ("const uint16_t *q = query + ((int64_t)s * num_heads + h) * head_size;",
                            "const uint16_t *q = query + ((int64_t)s * num_heads + 0) * head_size;"),
 }
@@ -201,6 +208,23 @@ def pin_battery():
         oracle.swap_blocks(dk, dv, src, src + 1, np.array([[2, 0]], np.int32))
         return np.array_equal(dk[0], src[2]) and np.array_equal(dv[0], src[2] + 1)
 
+    def e4m3_attention():
+        # an E4M3 cache at scales (1/2, 4) against fp16 caches holding its
+        # decoded values times those scales (exact: small powers of two)
+        rng = np.random.default_rng(21)
+        codes_k = rng.integers(0, 256, (5, 4, 2, 8), dtype=np.uint8)
+        codes_v = rng.integers(0, 256, (5, 4, 2, 8), dtype=np.uint8)
+        for c in (codes_k, codes_v):
+            c[(c & 0x7F) == 0x7F] = 0x3C
+            c[(c & 0x78) >= 0x60] &= 0x9F
+        f16_k = (torch.from_numpy(codes_k).view(torch.float8_e4m3fn).to(torch.float64).numpy() * 0.5).astype(np.float16)
+        f16_v = (torch.from_numpy(codes_v).view(torch.float8_e4m3fn).to(torch.float64).numpy() * 4.0).astype(np.float16)
+        q = rng.standard_normal((2, 2, 8)).astype(np.float16)
+        bt = np.array([[3, 0], [1, 4]], np.int32)
+        ctx = np.array([7, 5], np.int32)
+        a = oracle.paged_attention(q, codes_k, codes_v, bt, ctx, 0.3, k_scale=0.5, v_scale=4.0)
+        return np.array_equal(a, oracle.paged_attention(q, f16_k, f16_v, bt, ctx, 0.3))
+
     def lse_identity():
         w, kc, vc = _complete([15, 40], seed=14)
         full = oracle.paged_attention(w.query, kc, vc, w.block_tables, w.context_lens, w.scale)
@@ -248,6 +272,7 @@ def pin_battery():
                      ("dense equivalence", dense_equivalence), ("context one", context_one),
                      ("brute force", brute_force), ("relabelling", relabelling),
                      ("cache write", cache_write_readback), ("copy", copy_semantics), ("swap", swap_semantics),
+                     ("e4m3 attention", e4m3_attention),
                      ("lse identity", lse_identity), ("prefill worked example", prefill_worked_example),
                      ("prefill one-token chunks", prefill_one_token_chunks),
                      ("prefill dense causal", prefill_dense_causal)]:
