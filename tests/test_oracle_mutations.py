@@ -7,7 +7,8 @@ against numpy/torch, E4M3 encoding against torch and the saturation points,
 dense attention on identity tables against torch's SDPA, the closed forms,
 exact-sum brute force, physical-block relabelling, cache-write read-back,
 block copy and swap semantics, E4M3 attention against fp16 caches holding
-the decoded values at distinct K and V scales, the log-sum-exp identity, and for the
+the decoded values at distinct K and V scales, an empty context (slot -1,
+zero output), the log-sum-exp identity, and for the
 prefill the worked example as a full prompt, one-token chunks against the
 decode slots, and chunks after a cached context against torch's SDPA with a
 position mask. Every mutant
@@ -65,6 +66,10 @@ MUTANTS = {
                                         "cache_value(value_cache, kv_dtype, rowbase[i] + d, k_scale)"),
     "E4M3 cache scale dropped": ("return oracle_e4m3_to_double(((const uint8_t *)cache)[idx]) * scale;",
                                  "return oracle_e4m3_to_double(((const uint8_t *)cache)[idx]);"),
+    "empty context gets a slot": ("if (L <= 0) {\n            slot_mapping[s] = -1;",
+                                  "if (L < 0) {\n            slot_mapping[s] = -1;"),
+    "empty context attends over nothing": ("if (L <= 0) {\n            for (int d = 0; d < head_size; ++d)\n                o[d] = 0.0;",
+                                           "if (L < 0) {\n            for (int d = 0; d < head_size; ++d)\n                o[d] = 0.0;"),
     "head index ignored": ("const uint16_t *q = query + ((int64_t)s * num_heads + h) * head_size;",
                            "const uint16_t *q = query + ((int64_t)s * num_heads + 0) * head_size;"),
 }
@@ -208,6 +213,18 @@ def pin_battery():
         oracle.swap_blocks(dk, dv, src, src + 1, np.array([[2, 0]], np.int32))
         return np.array_equal(dk[0], src[2]) and np.array_equal(dv[0], src[2] + 1)
 
+    def empty_context():
+        # a sequence with no context has no slot and a zero output row
+        rng = np.random.default_rng(22)
+        bt = np.array([[2, -1], [1, 3]], np.int32)
+        ctx = np.array([0, 5], np.int32)
+        slots = oracle.slot_mapping(bt, ctx, 4)
+        kc = rng.standard_normal((4, 4, 1, 8)).astype(np.float16)
+        vc = rng.standard_normal((4, 4, 1, 8)).astype(np.float16)
+        q = rng.standard_normal((2, 1, 8)).astype(np.float16)
+        out = oracle.paged_attention(q, kc, vc, bt, ctx, 0.5)
+        return list(slots) == [-1, 12] and np.array_equal(out[0], np.zeros((1, 8))) and np.isfinite(out).all()
+
     def e4m3_attention():
         # an E4M3 cache at scales (1/2, 4) against fp16 caches holding its
         # decoded values times those scales (exact: small powers of two)
@@ -272,7 +289,7 @@ def pin_battery():
                      ("dense equivalence", dense_equivalence), ("context one", context_one),
                      ("brute force", brute_force), ("relabelling", relabelling),
                      ("cache write", cache_write_readback), ("copy", copy_semantics), ("swap", swap_semantics),
-                     ("e4m3 attention", e4m3_attention),
+                     ("empty context", empty_context), ("e4m3 attention", e4m3_attention),
                      ("lse identity", lse_identity), ("prefill worked example", prefill_worked_example),
                      ("prefill one-token chunks", prefill_one_token_chunks),
                      ("prefill dense causal", prefill_dense_causal)]:
