@@ -3,7 +3,8 @@
 Each case below plants one mistake in a copy of oracle/pagedkv_oracle.c (a
 text substitution), builds it, routes the oracle through it and runs the
 pin battery: the worked and growth slot examples, binary16 and E4M3 decoding
-against numpy/torch, E4M3 encoding against torch and the saturation points,
+against numpy/torch, E4M3 encoding against torch, the saturation points,
+signed zeros and every tie between neighbouring codes (to the even code),
 dense attention on identity tables against torch's SDPA, the closed forms,
 exact-sum brute force, physical-block relabelling, cache-write read-back,
 block copy and swap semantics, E4M3 attention against fp16 caches holding
@@ -38,6 +39,8 @@ MUTANTS = {
     "f16 exponent bias": ("v = ldexp((double)(1024 + f), e - 25);", "v = ldexp((double)(1024 + f), e - 24);"),
     "e4m3 exponent bias": ("v = ldexp((double)(8 + m), e - 10);", "v = ldexp((double)(8 + m), e - 9);"),
     "e4m3 encode truncates": ("double n = nearbyint(a / quantum);", "double n = floor(a / quantum);"),
+    "e4m3 ties away from zero": ("double n = nearbyint(a / quantum);", "double n = round(a / quantum);"),
+    "e4m3 negative zero loses its sign": ("    if (a == 0.0)\n        return sign;", "    if (a == 0.0)\n        return 0;"),
     "e4m3 saturates to NaN": ("        return sign | 0x7e;\n    if (a == 0.0)", "        return sign | 0x7f;\n    if (a == 0.0)"),
     "softmax scale dropped": ("z[t - t0] = scale * dot;", "z[t - t0] = dot;"),
     "row offset by block division": ("int64_t base = (((int64_t)blk * block_size + t % block_size) * num_heads + h) * head_size;",
@@ -137,8 +140,16 @@ def pin_battery():
         x = np.random.default_rng(0).standard_normal(20000).astype(np.float32) * 40
         x = x[np.abs(x) <= 448]
         ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
-        sat = oracle.e4m3_from_float(np.float32([449, 1e9, -500]))
-        return np.array_equal(oracle.e4m3_from_float(x), ref) and list(sat) == [0x7E, 0x7E, 0xFE]
+        sat = oracle.e4m3_from_float(np.float32([449, 1e9, -500, 0.0, -0.0]))
+        # codes 0x00..0x7E ascend in magnitude, so the value halfway between
+        # codes k and k+1 rounds (ties to even) to whichever of them is even
+        codes = np.arange(0x7F, dtype=np.uint8)
+        vals = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+        mids = ((vals[:-1] + vals[1:]) / 2).astype(np.float32)   # exact: five significant bits at most
+        even = np.where(codes[:-1] % 2 == 0, codes[:-1], codes[1:]).astype(np.uint8)
+        return (np.array_equal(oracle.e4m3_from_float(x), ref) and list(sat) == [0x7E, 0x7E, 0xFE, 0x00, 0x80]
+                and np.array_equal(oracle.e4m3_from_float(mids), even)
+                and np.array_equal(oracle.e4m3_from_float(-mids), even | 0x80))
 
     def dense_equivalence():
         w, kc, vc = _complete([1, 9, 30], H=3, D=16, B=8, deal="identity", seed=1)
