@@ -18,10 +18,12 @@ from .ops import (  # noqa: F401
     load_cache,
     paged_attention_decode,
     paged_attention_decode_append,
+    paged_attention_decode_noalloc,
     paged_attention_decode_shared_prefix,
     paged_prefill,
     prefill_slot_mapping,
     prefill_step,
+    shared_prefix_workspace_size,
     slot_mapping,
     swap_blocks,
     version,

@@ -192,19 +192,10 @@ def decode_workspace_size(key_cache: torch.Tensor, num_seqs: int, max_context_le
                                               ctypes.byref(cfg) if cfg is not None else None))
 
 
-def paged_attention_decode(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
-                           value_cache: torch.Tensor, block_tables: torch.Tensor,
-                           context_lens: torch.Tensor, scale: float, k_scale: float = 1.0,
-                           v_scale: float = 1.0, max_context_len: int | None = None,
-                           config=None, workspace: torch.Tensor | None = None, stream=None) -> None:
-    """Decode attention into ``out`` ([S, H, D] fp16).
-
-    ``max_context_len`` is a host-side bound on every context length; by
-    default the table capacity ``block_tables.shape[1] * block_size`` (no
-    device sync). With ``config`` or ``workspace`` given, the caller-workspace
-    entry point is used (``workspace`` a uint8 CUDA tensor of at least
-    ``decode_workspace_size`` bytes).
-    """
+def _decode_args(out, query, key_cache, value_cache, block_tables, context_lens, scale, k_scale, v_scale,
+                 max_context_len, workspace=None) -> tuple:
+    """Checks of a plain decode call; returns its C arguments up to the
+    launch options (the stream, and for the _ws call config and workspace)."""
     _check_pair(key_cache, value_cache)
     _i32(block_tables, "block_tables")
     _i32(context_lens, "context_lens")
@@ -221,9 +212,26 @@ def paged_attention_decode(out: torch.Tensor, query: torch.Tensor, key_cache: to
     if max_context_len is None:
         max_context_len = block_tables.shape[1] * desc.block_size
     _on_current_device(out, query, key_cache, value_cache, block_tables, context_lens, workspace)
-    args = (out.data_ptr(), query.data_ptr(), key_cache.data_ptr(), value_cache.data_ptr(), desc,
+    return (out.data_ptr(), query.data_ptr(), key_cache.data_ptr(), value_cache.data_ptr(), desc,
             block_tables.data_ptr(), block_tables.shape[1], context_lens.data_ptr(), S,
             int(max_context_len), float(scale), float(k_scale), float(v_scale))
+
+
+def paged_attention_decode(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
+                           value_cache: torch.Tensor, block_tables: torch.Tensor,
+                           context_lens: torch.Tensor, scale: float, k_scale: float = 1.0,
+                           v_scale: float = 1.0, max_context_len: int | None = None,
+                           config=None, workspace: torch.Tensor | None = None, stream=None) -> None:
+    """Decode attention into ``out`` ([S, H, D] fp16).
+
+    ``max_context_len`` is a host-side bound on every context length; by
+    default the table capacity ``block_tables.shape[1] * block_size`` (no
+    device sync). With ``config`` or ``workspace`` given, the caller-workspace
+    entry point is used (``workspace`` a uint8 CUDA tensor of at least
+    ``decode_workspace_size`` bytes).
+    """
+    args = _decode_args(out, query, key_cache, value_cache, block_tables, context_lens, scale, k_scale,
+                        v_scale, max_context_len, workspace)
     if config is None and workspace is None:
         check(lib().pa_paged_attention_decode(*args, _stream(stream)))
         return
@@ -231,6 +239,22 @@ def paged_attention_decode(out: torch.Tensor, query: torch.Tensor, key_cache: to
     ws_ptr, ws_bytes = _workspace(workspace)
     check(lib().pa_paged_attention_decode_ws(*args, ctypes.byref(cfg) if cfg is not None else None,
                                              ws_ptr, ws_bytes, _stream(stream)))
+
+
+def paged_attention_decode_noalloc(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
+                                   value_cache: torch.Tensor, block_tables: torch.Tensor,
+                                   context_lens: torch.Tensor, scale: float, k_scale: float = 1.0,
+                                   v_scale: float = 1.0, max_context_len: int | None = None,
+                                   stream=None) -> None:
+    """``paged_attention_decode`` that allocates nothing (library-chosen launch
+    shape). The split partials go to a 16 MiB static array inside the
+    library, one per device: a larger decode is rejected before any launch,
+    calls whose kernels may overlap (other streams or threads) must be
+    serialised, and the first call on a device must precede any stream
+    capture (it looks up the array's address)."""
+    args = _decode_args(out, query, key_cache, value_cache, block_tables, context_lens, scale, k_scale,
+                        v_scale, max_context_len)
+    check(lib().pa_paged_attention_decode_noalloc(*args, _stream(stream)))
 
 
 def paged_attention_decode_append(out: torch.Tensor, query: torch.Tensor, new_key: torch.Tensor,
@@ -275,6 +299,16 @@ def paged_attention_decode_append(out: torch.Tensor, query: torch.Tensor, new_ke
         int(max_context_len), float(scale), float(k_scale), float(v_scale),
         slot_mapping.data_ptr() if slot_mapping is not None else None,
         ctypes.byref(cfg) if cfg is not None else None, ws_ptr, ws_bytes, _stream(stream)))
+
+
+def shared_prefix_workspace_size(key_cache: torch.Tensor, num_seqs: int, max_context_len: int,
+                                 shared_prefix_blocks: int, config=None) -> int:
+    """Workspace bytes of a ``paged_attention_decode_shared_prefix`` call (0 on
+    invalid arguments)."""
+    cfg = _config(config)
+    return int(lib().pa_shared_prefix_workspace_size(cache_desc(key_cache), int(num_seqs), int(max_context_len),
+                                                     int(shared_prefix_blocks),
+                                                     ctypes.byref(cfg) if cfg is not None else None))
 
 
 def paged_attention_decode_shared_prefix(out: torch.Tensor, query: torch.Tensor,

@@ -9,8 +9,9 @@ here must pass both alone in a fresh process and after the rest of the suite.
 The check: through the C ABI, two calls in a row with different batches that
 both need the split path, each compared with the allocating entry point
 pa_paged_attention_decode on the same inputs (max-abs 2e-3, the fp16-KV
-tolerance of the parity tests), plus the clear rejection of a batch whose
-partials exceed the static scratch.
+tolerance of the parity tests), the clear rejection of a batch whose
+partials exceed the static scratch, and the torch binding giving the C
+call's result bit for bit.
 """
 import ctypes
 
@@ -73,3 +74,18 @@ def test_noalloc_rejects_partials_beyond_the_static_scratch(cuda_device):
                                              1.0, None)
     assert rc == capi.PA_ERR_WORKSPACE
     assert b"static scratch" in L.pa_last_error()
+
+
+def test_binding_gives_the_c_call_result(cuda_device):
+    # the torch binding marshals the same arguments (its default bound is the
+    # table capacity, as in _args): bit-identical outputs
+    w, dw = _batch(cuda_device, 23, [600, 40, 1300])
+    assert dw.block_tables.shape[1] == w.max_blocks_per_seq
+    stream = torch.cuda.current_stream().cuda_stream
+    a = torch.full_like(dw.out, float("nan"))
+    b = torch.full_like(dw.out, float("nan"))
+    assert capi.lib().pa_paged_attention_decode_noalloc(*_args(w, dw, a), stream) == 0
+    pk.paged_attention_decode_noalloc(b, dw.query, dw.key_cache, dw.value_cache, dw.block_tables,
+                                      dw.context_lens, w.scale)
+    assert pk.check_status() == 0
+    assert torch.equal(a, b)
