@@ -97,7 +97,8 @@ std::vector<std::pair<MapKey, CUtensorMap>> g_maps;  // small FIFO cache
 // num_blocks}; box {head_size, G, block_size, 1} = one physical block's rows
 // for G heads. Zero fill outside the pool.
 // swz = 1: box {64, 1, block_size, 1} (a 64-dim half of one head's rows)
-// with 128-byte swizzle, for the tensor-core shared-prefix kernel.
+// with 128-byte swizzle, for the tensor-core kernels (shared prefix, both
+// prefills), whose MMA operands take that layout.
 int cache_tensor_map(const void *cache, const pa_cache_desc &c, int G, CUtensorMap *out, int swz = 0) {
     const MapKey key{cache, c.num_blocks, c.block_size, c.num_heads, c.head_size, c.dtype, G, swz};
     {
