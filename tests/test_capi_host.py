@@ -177,5 +177,9 @@ def test_prefill_argument_checks():
     assert L.pa_prefill_slot_mapping(P, P, P, 4, P, 2, T, -1, F, None) == capi.PA_ERR_INVALID
     assert L.pa_prefill_slot_mapping(P, P, P, 4, P, 2, -1, 64, F, None) == capi.PA_ERR_INVALID
     assert L.pa_prefill_slot_mapping(P, P, P, 4, P, 70000, T, 64, F, None) == capi.PA_ERR_INVALID
+    # a grid of more than 2^31 - 1 CTAs is refused before any CUDA call:
+    # 65535 sequences x 8 heads x ceil(2^30 / 128) row tiles
+    assert L.pa_paged_prefill(P, P, P, P, P, F, P, 4, P, 65535, T, 1 << 30, 0.1, None) == capi.PA_ERR_INVALID
+    assert "too many prefill tiles" in _last()
     assert L.pa_prefill_slot_mapping(None, None, None, 4, None, 0, T, 64, F, None) == capi.PA_OK
     assert L.pa_prefill_slot_mapping(None, None, None, 4, None, 2, 0, 64, F, None) == capi.PA_OK
