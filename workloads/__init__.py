@@ -1,4 +1,4 @@
-"""Seeded synthetic inputs for the paged-KV decode path.
+"""Seeded synthetic inputs for the paged-KV decode path and the paged prefill.
 
 This module is shared by the tests, the benchmark and the smoke check, and it
 holds none of the method's arithmetic: it draws context lengths, deals
@@ -16,9 +16,12 @@ Context tokens 0 .. L-2 of each sequence are present in the pool before the
 step; position L-1 (the token the decode step appends) holds poison until the
 step's cache write stores ``new_key``/``new_value`` there.
 
-The five named workloads follow the shapes and value laws of the pages'
-serving setups (LLaMA-7B: 32 heads x 128; Llama2-13B: 40 heads x 128; 16-token
-blocks, 32-token blocks for long shared prompts, FP8 KV cache). No public
+The five named decode workloads follow the shapes and value laws of the
+pages' serving setups (LLaMA-7B: 32 heads x 128; Llama2-13B: 40 heads x 128;
+16-token blocks, 32-token blocks for long shared prompts, FP8 KV cache). The
+three named prefill workloads (``prefill_named``) bring a chunk of new tokens
+per sequence: whole prompts, or chunks after tokens already in the pool,
+whose own positions hold poison until the chunk's cache write. No public
 dataset is involved; every input is drawn from ``numpy.random.PCG64``.
 """
 from __future__ import annotations
