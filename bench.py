@@ -55,15 +55,41 @@ DECODE_SOURCES = ("pa_decode.cuh", "pa_device.cuh", "pa_cache_ops.cuh")
 PREFILL_SOURCES = ("pa_prefill.cuh", "pa_decode.cuh", "pa_device.cuh")
 
 
+def code_tokens(src: str) -> str:
+    """C++ source without its comments, whitespace runs collapsed to one
+    space (string and character literals kept as they are)."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+            out.append(" ")
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_source_hash(names=DECODE_SOURCES) -> str:
     """Hash of the device code (kernels and their helpers; not the host-side
     launch logic), so a recorded ncu traffic figure is dropped when a kernel
-    changes."""
+    changes. Comments and layout do not count."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "pagedattention_paged_kv_decode_b200", "csrc")
     for name in names:
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update(code_tokens(f.read()).encode())
     return h.hexdigest()[:16]
 
 

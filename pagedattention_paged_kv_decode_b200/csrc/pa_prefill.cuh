@@ -218,28 +218,28 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
 
 namespace pa {
 
-// ----------------------------------------- prefill on tcgen05 (head_size 128)
+// -------------------------------- prefill on tcgen05 (head_size 64 or 128)
 //
 // One CTA = one head x one tile of up to 128 consecutive query rows of one
 // sequence; K/V are consumed 128 tokens at a time. Per K/V tile j:
-//   S_j = Q . K_j^T   128 x 128, eight tcgen05.mma (K = 16 each) into tensor
+//   S_j = Q . K_j^T   128 x 128, D / 16 tcgen05.mma (K = 16 each) into tensor
 //                     memory (two S buffers, so S_{j+1} overlaps the softmax of j)
 //   softmax           reads S, masks tokens after each row's position, keeps
 //                     a reference maximum that moves only when the row
 //                     maximum exceeds it by more than 2^8 (then O is rescaled
 //                     in tensor memory), and writes P = 2^(s - m) as fp16 back
 //                     into the S buffer it came from (tcgen05.st)
-//   O += P_j . V_j    eight tcgen05.mma with A (P) read from tensor memory and
-//                     V from shared memory, N-contiguous (MN-major)
+//   O += P_j . V_j    eight tcgen05.mma (N = D) with A (P) read from tensor
+//                     memory and V from shared memory, N-contiguous (MN-major)
 // An S buffer takes the next S only once the P.V that reads its P is done.
 // K and V have rings of their own (3 and 2 tiles): a K tile is released as
 // soon as its S is computed, a V tile when its P.V is, so each is reloaded
 // as early as possible. Warps: 0-7 softmax (and Q staging, epilogue): warp
-// w takes rows 32 (w % 4) .. + 31 (its tensor-memory lanes) and columns
-// 64 (w / 4) .. + 63 of S, P and O, the two halves of a row exchanging their
-// maxima and sums through tensor memory; 8 K producer; 9 MMA issuer (also
-// allocates the 512 tensor-memory columns); 10 V producer. Each producer
-// keeps the next 32 block-table entries in flight.
+// w takes rows 32 (w % 4) .. + 31 (its tensor-memory lanes), columns
+// 64 (w / 4) .. + 63 of S and P and D / 2 columns of O, the two halves of a
+// row exchanging their maxima and sums through tensor memory; 8 K producer;
+// 9 MMA issuer (also allocates the 512 tensor-memory columns); 10 V
+// producer. Each producer keeps the next 32 block-table entries in flight.
 // Every wait is bounded; a wait that runs out sets PA_DEV_WAIT_TIMEOUT and
 // an abort flag that ends the other roles' waits, and the CTA still drains
 // its copies and MMAs and frees its tensor memory before it exits.
@@ -250,7 +250,7 @@ constexpr int kTcVStages = 2;
 constexpr int kTcThreads = 352;
 constexpr int kTcSoftmaxWarps = 8;  // two per tensor-memory lane quadrant, one per half row
 constexpr int kTcWarpK = 8, kTcWarpMma = 9, kTcWarpV = 10;
-constexpr int kTcTmemCols = 512;  // S0 [0,128), S1 [128,256), O [256,384), row exchange [384,390)
+constexpr int kTcTmemCols = 512;  // S0 [0,128), S1 [128,256), O [256,256+D), row exchange [384,390)
 constexpr int kTcColX = 384;      // + 2 * tile parity + half: row maxima; + 4 + half: row sums
 
 template <int D>
