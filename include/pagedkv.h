@@ -1,7 +1,8 @@
 /*
  * pagedkv.h -- C ABI of libpagedkv.so: paged-KV decode attention for NVIDIA
  * B200 (sm_100a), with the cache-write scatter, the slot derivation and the
- * block copy that surround it.
+ * block copy that surround it, block swap to pinned host memory, and the
+ * paged prefill of a prompt or chunk.
  *
  * Sources (each page is cited by its title and section):
  *   [P1] "vLLM-v0.17.1技术解析：PagedAttention内存管理与显存优化技巧",
