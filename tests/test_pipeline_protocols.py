@@ -11,8 +11,10 @@ a tile is read only after it landed, S is overwritten only after it was
 read and its P consumed, and the tail V rows are zeroed before any P.V
 reads them.
 
-The models restate the protocols of pa_decode.cuh (decode ring) and
-pa_prefill.cuh (tcgen05 prefill); they do not run the kernels.
+The models restate the protocols of pa_decode.cuh (decode ring; the
+broadcast ring of the shared-prefix kernels, also used by the mma.sync
+prefill in pa_prefill.cuh) and pa_prefill.cuh (tcgen05 prefill); they do
+not run the kernels.
 """
 import random
 
@@ -84,6 +86,95 @@ def test_decode_ring_false_passes_without_the_rule():
                 if _decode_ring_false_pass(nblk, warps, stages, seed):
                     found.add((warps, stages))
     assert found == {(2, 3), (4, 2), (4, 6)}
+
+
+# ------------------------------------------------------------ broadcast ring
+
+def _broadcast_ring_run(ntiles, consumers, stages, seed, release_count=None):
+    """The ring of the shared-prefix kernels and the mma.sync prefill: one
+    producer puts tile j into stage j % stages once every consumer has
+    released the stage's previous tile (the empty barrier counts
+    `consumers` arrivals); every consumer warp reads every tile in order,
+    waiting on the stage's full barrier by parity. Landings and the order of
+    the roles are random. Returns a description of the first violation, or
+    None. `release_count` replaces the empty barrier's arrival count (to
+    plant a mistake)."""
+    rnd = random.Random(seed)
+    release_count = consumers if release_count is None else release_count
+    full = [0] * stages            # completed phases
+    empty = [0] * stages
+    empty_cnt = [0] * stages
+    content = [None] * stages      # tile held by each stage
+    readers = [set() for _ in range(stages)]   # consumers between their wait and their release
+    inflight = []
+    nxt = 0
+    cons = [0] * consumers         # next tile of each consumer
+    holding = [None] * consumers   # stage a consumer has passed the wait on and not yet released
+    for _ in range(200000):
+        acts = []
+        if nxt < ntiles:
+            st, use = nxt % stages, nxt // stages
+            if use == 0 or (empty[st] & 1) != ((use - 1) & 1):
+                acts.append(("prod",))
+        if inflight:
+            acts.append(("land",))
+        for c in range(consumers):
+            if holding[c] is not None:
+                acts.append(("release", c))
+            elif cons[c] < ntiles:
+                i = cons[c]
+                if (full[i % stages] & 1) != ((i // stages) & 1):
+                    acts.append(("read", c))
+        if not acts:
+            done = nxt == ntiles and not inflight and all(i == ntiles for i in cons)
+            return None if done else "deadlock"
+        a = rnd.choice(acts)
+        if a[0] == "prod":
+            inflight.append(nxt)
+            nxt += 1
+        elif a[0] == "land":
+            j = inflight.pop(rnd.randrange(len(inflight)))
+            st = j % stages
+            if readers[st]:
+                return f"tile {j} overwrote stage {st} while consumers {sorted(readers[st])} read it"
+            content[st] = j
+            full[st] += 1
+        elif a[0] == "read":
+            c = a[1]
+            i = cons[c]
+            st = i % stages
+            if content[st] != i:
+                return f"consumer {c} passed its wait for tile {i} but stage {st} holds {content[st]}"
+            readers[st].add(c)
+            holding[c] = st
+        else:
+            c = a[1]
+            st = holding[c]
+            readers[st].discard(c)
+            holding[c] = None
+            cons[c] += 1
+            empty_cnt[st] += 1
+            if empty_cnt[st] == release_count:
+                empty_cnt[st] = 0
+                empty[st] += 1
+    return "no termination"
+
+
+@pytest.mark.parametrize("consumers", [1, 2, 4])
+def test_broadcast_ring_is_sound(consumers):
+    for stages in (2, 3, 4, 6, 8):
+        for ntiles in (1, 2, 5, 9, 17, 40):
+            for seed in range(20):
+                assert _broadcast_ring_run(ntiles, consumers, stages, seed) is None, \
+                    (consumers, stages, ntiles, seed)
+
+
+def test_broadcast_ring_model_catches_a_missing_release_count():
+    # an empty barrier that completes on every arrival (count 1 instead of
+    # `consumers`) lets the producer overwrite a stage a slower warp is still
+    # reading, or a warp pass a stale phase: the model must report it
+    found = [_broadcast_ring_run(17, 4, 2, seed, release_count=1) or "" for seed in range(40)]
+    assert any(r.startswith("tile") and "overwrote" in r for r in found)
 
 
 # ------------------------------------------------------- tcgen05 prefill
