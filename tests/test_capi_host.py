@@ -14,7 +14,8 @@ HEADER = os.path.join(ROOT, "include", "pagedkv.h")
 
 
 def declared_functions():
-    text = open(HEADER).read()
+    with open(HEADER, encoding="utf-8") as f:
+        text = f.read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", text)))
 
