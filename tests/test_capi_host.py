@@ -184,3 +184,30 @@ def test_prefill_argument_checks():
     assert "too many prefill tiles" in _last()
     assert L.pa_prefill_slot_mapping(None, None, None, 4, None, 0, T, 64, F, None) == capi.PA_OK
     assert L.pa_prefill_slot_mapping(None, None, None, 4, None, 2, 0, 64, F, None) == capi.PA_OK
+
+
+def test_default_config_is_valid_over_a_sweep_of_shapes():
+    # every default choice must satisfy the kernel's constraints (the
+    # library itself refuses a choice over the shared-memory limit)
+    L = capi.lib()
+    n = 0
+    for D in (64, 128):
+        for B in (16, 32):
+            for dt in (capi.PA_F16, capi.PA_E4M3):
+                for H in (1, 2, 3, 4, 8, 12, 32, 40, 64):
+                    desc = capi.CacheDesc(4096, B, H, D, dt)
+                    for S in (1, 2, 7, 16, 64, 256, 1024):
+                        for maxL in (1, 15, 16, 17, 200, 512, 513, 4096, 32768):
+                            rc, c = _choose(desc, S, maxL)
+                            assert rc == capi.PA_OK, (D, B, dt, H, S, maxL, _last())
+                            assert c.partition_size >= B and c.partition_size % B == 0
+                            assert c.heads_per_cta in (1, 2, 4, 8) and H % c.heads_per_cta == 0
+                            assert c.warps_per_head in (1, 2, 4)
+                            assert 2 <= c.stages <= 8 and c.stages % c.warps_per_head == 0
+                            assert 1 <= c.units_per_cta <= 4
+                            assert c.units_per_cta * c.heads_per_cta * c.warps_per_head <= 16
+                            parts = max(1, -(-maxL // c.partition_size))
+                            ws = L.pa_decode_workspace_size(desc, S, maxL, ctypes.byref(c))
+                            assert (ws == 0) == (parts == 1), (D, B, H, S, maxL, ws, parts)
+                            n += 1
+    assert n == 2 * 2 * 2 * 9 * 7 * 9
