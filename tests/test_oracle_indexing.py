@@ -4,7 +4,9 @@ Slot mapping is pinned to the worked example printed on the l189.com/news/180929
 article (section 2.2) and to the growth example of the "在A10G上榨干LLaMA-7B" page
 (section 2.1); both are stored under tests/golden/. Cache write and block copy are
 pinned by reading back through plain numpy indexing of the [block, row, head, dim]
-layout, and by checking that nothing outside the target rows changes.
+layout, and by checking that nothing outside the target rows changes. The block
+copy moves exactly the per-block bytes that the article's section 2.1 prints,
+restated for 2- and 1-byte elements (tests/golden/block_bytes_example.txt).
 """
 import os
 
@@ -180,3 +182,29 @@ def test_swap_blocks_between_pools():
         oracle.swap_blocks(ck, cv, gk, gv, np.array([[6, 0]], np.int32))
     with pytest.raises(ValueError):
         oracle.swap_blocks(ck, cv, gk, gv, np.array([[0, 3]], np.int32))
+
+
+def test_block_bytes_follow_the_printed_block_size():
+    # [P3] §2.1 sizes a 16-token x 32-head x 128-dim K+V block at about 512 KB
+    # with 4-byte elements; the oracle's block copy moves exactly one block
+    # of B*H*D*elem bytes per cache, i.e. the fixture's K+V figure for fp16
+    # and E4M3
+    rows = {}
+    with open(os.path.join(GOLDEN, "block_bytes_example.txt")) as f:
+        for ln in f:
+            if ln.strip() and not ln.startswith("#"):
+                B, H, D, caches, elem, nbytes = map(int, ln.split())
+                assert B * H * D * caches * elem == nbytes
+                rows[elem] = (B, H, D, nbytes)
+    assert rows[4][3] == 512 * 1024
+    rng = np.random.default_rng(17)
+    for elem, dtype in ((2, np.float16), (1, np.uint8)):
+        B, H, D, nbytes = rows[elem]
+        src = rng.integers(1, 256, (3, B, H, D * elem), dtype=np.uint8).view(dtype)
+        kc, vc = src.copy(), src.copy()
+        kc[2] = 0
+        vc[2] = 0
+        k0, v0 = kc.copy(), vc.copy()
+        oracle.copy_blocks(kc, vc, np.array([[0, 2]], np.int32))
+        changed = int((kc.view(np.uint8) != k0.view(np.uint8)).sum() + (vc.view(np.uint8) != v0.view(np.uint8)).sum())
+        assert changed == nbytes
