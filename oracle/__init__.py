@@ -1,4 +1,5 @@
-"""CPU oracle for the paged-KV decode path (test infrastructure only).
+"""CPU oracle for the paged-KV decode path and the paged prefill (test
+infrastructure only).
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package. It wraps ``pagedkv_oracle.c`` -- plain

@@ -1,5 +1,6 @@
 /*
- * pagedkv_oracle.c -- plain, slow, scalar CPU oracle for the paged-KV decode path.
+ * pagedkv_oracle.c -- plain, slow, scalar CPU oracle for the paged-KV decode path
+ * and the paged prefill.
  *
  * TEST INFRASTRUCTURE ONLY. Only the test suite, the smoke check and the CPU
  * baseline leg of the benchmark load this file's shared library. The CUDA
@@ -28,8 +29,12 @@
  * tables against torch's CPU scaled_dot_product_attention, physical-block
  * permutation invariance, L=1 => V, equal keys / scale 0 => mean of V,
  * brute force with exact summation on tiny inputs, convexity bounds, the
- * log-sum-exp identity for partitions, and an independent table-driven
- * E4M3 encoder plus torch's float8_e4m3fn cast.
+ * log-sum-exp identity for partitions, an independent table-driven E4M3
+ * encoder plus torch's float8_e4m3fn cast, E4M3 ties to the even code, E4M3
+ * caches against fp16 caches of their decoded values at distinct K and V
+ * scales, the printed per-block byte size ([P3] §2.1), and for the prefill
+ * the worked slot example as a full prompt, one-token chunks against the
+ * decode slots, and torch's SDPA with a causal / position mask.
  */
 #include <math.h>
 #include <stdint.h>
