@@ -178,6 +178,13 @@ int pa_swap_blocks(void *dst_key_cache, void *dst_value_cache, int dst_num_block
  *     out[s,h,:] = v_scale * sum_t softmax(z)_t * V_t[h,:]       (t < L)
  * (k_scale, v_scale only for E4M3 caches, which hold K/k_scale, V/v_scale).
  * L = 0 gives zeros. query, out: fp16 [num_seqs][num_heads][head_size].
+ * Range of the E4M3 path: the products of q * scale * log2(e) (rounded to
+ * fp16) with the decoded codes (|code| <= 448) are summed in fp16 over 8
+ * elements before k_scale is applied, so |q * scale| per element must stay
+ * below about 12.7 for no partial sum to overflow when every code is +-448
+ * with one sign (queries of trained models are orders of magnitude below;
+ * the P.V sums, with weights <= 1, cannot overflow). fp16 caches compute in
+ * fp32 and have no such limit.
  * max_context_len: a host-known upper bound on every context length (e.g.
  * max_blocks_per_seq*block_size); it sizes the split-context grid. Contexts
  * above it or above the table row are clamped and flagged.
