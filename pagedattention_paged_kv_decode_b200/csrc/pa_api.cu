@@ -762,10 +762,10 @@ int plan_shared_prefix(const pa_cache_desc &c, int S, int bound, int prefix_bloc
                        size_t *ws) {
     const int B = c.block_size;
     if (prefix_blocks < 1) return fail(PA_ERR_INVALID, "shared_prefix_blocks %d < 1", prefix_blocks);
+    if ((int64_t)prefix_blocks * B > bound)  // 64-bit: the size query has no table width to bound it
+        return fail(PA_ERR_INVALID, "shared prefix (%lld tokens) beyond the context bound %d",
+                    (long long)prefix_blocks * B, bound);
     pre->prefix_tokens = prefix_blocks * B;
-    if (pre->prefix_tokens > bound)
-        return fail(PA_ERR_INVALID, "shared prefix (%d tokens) beyond the context bound %d",
-                    pre->prefix_tokens, bound);
     pre->heads = 1;
     pre->mma = c.dtype == PA_F16;
     pre->queries = pre->mma ? pa::kPrefixMmaQueries : std::min(S, pa::kMaxConsumerWarps);

@@ -211,3 +211,37 @@ def test_default_config_is_valid_over_a_sweep_of_shapes():
                             assert (ws == 0) == (parts == 1), (D, B, H, S, maxL, ws, parts)
                             n += 1
     assert n == 2 * 2 * 2 * 9 * 7 * 9
+
+
+def test_swap_append_and_shared_prefix_argument_checks():
+    L = capi.lib()
+    D = capi.CacheDesc(64, 16, 8, 128, capi.PA_F16)
+    # (dst_k, dst_v, dst_nb, src_k, src_v, src_nb, desc, pairs, n, stream)
+    assert L.pa_swap_blocks(P, P, 0, P, P, 8, D, P, 1, None) == capi.PA_ERR_INVALID
+    assert L.pa_swap_blocks(P, P, 8, P, P, 8, D, P, -1, None) == capi.PA_ERR_INVALID
+    assert L.pa_swap_blocks(P, P, 8, P, P, 8, D, None, 1, None) == capi.PA_ERR_INVALID
+    assert L.pa_swap_blocks(P, P + 8, 8, P, P, 8, D, P, 1, None) == capi.PA_ERR_INVALID
+    assert L.pa_swap_blocks(P, P, 8, P, P, 1 << 27, D, P, 1, None) == capi.PA_ERR_OVERFLOW
+    assert L.pa_swap_blocks(None, None, 8, None, None, 8, D, None, 0, None) == capi.PA_OK
+    row = 8 * 128
+    # (out, q, new_k, new_v, k_stride, v_stride, kc, vc, desc, bt, width, ctx, S, max_ctx,
+    #  scale, k_scale, v_scale, slots, cfg, ws, ws_bytes, stream)
+    app = lambda nk, ks, cfg=None: L.pa_paged_attention_decode_append(  # noqa: E731
+        P, P, nk, P, ks, row, P, P, D, P, 4, P, 2, 64, 0.1, 1.0, 1.0, None, cfg, None, 0, None)
+    assert app(None, row) == capi.PA_ERR_INVALID
+    assert app(P + 4, row) == capi.PA_ERR_INVALID
+    assert app(P, row - 8) == capi.PA_ERR_INVALID
+    assert app(P, row + 4) == capi.PA_ERR_INVALID
+    assert "stride" in _last()
+    assert app(P, row, ctypes.byref(capi.DecodeConfig(24, 0, 0, 0, 0))) == capi.PA_ERR_INVALID
+    # (..., S, max_ctx, prefix_blocks, scale, ...)
+    pre = lambda nk, nv, blocks: L.pa_paged_attention_decode_shared_prefix(  # noqa: E731
+        P, P, nk, nv, row, row, P, P, D, P, 4, P, 2, 64, blocks, 0.1, 1.0, 1.0, None, None, None, 0, None)
+    assert pre(P, None, 1) == capi.PA_ERR_INVALID
+    assert pre(None, None, 5) == capi.PA_ERR_INVALID      # more than the 4-entry table
+    assert pre(None, None, 0) == capi.PA_ERR_INVALID
+    assert pre(None, None, -2) == capi.PA_ERR_INVALID
+    # the size query: a prefix past the context bound, however large, gives 0
+    assert L.pa_shared_prefix_workspace_size(D, 2, 64, 5, None) == 0
+    assert L.pa_shared_prefix_workspace_size(D, 2, 64, 1 << 28, None) == 0
+    assert L.pa_shared_prefix_workspace_size(D, 2, 64, 2, None) > 0
