@@ -151,7 +151,7 @@ int fill_config(const pa_cache_desc &c, int num_seqs, int max_ctx, pa_decode_con
         return pa::SmemLayout(B, G, c.head_size, elem_bytes(c), 1, 1, 1).stage_bytes;
     };
     auto units = [&](int G, int P) {  // CTAs of the grid, from the host-side length bound
-        return (int64_t)num_seqs * (H / G) * std::max(1, (max_ctx + P - 1) / P);
+        return (int64_t)num_seqs * (H / G) * std::max<int64_t>(1, ((int64_t)max_ctx + P - 1) / P);
     };
     // Defaults, fitted by launch-shape sweeps on B200 (sequences x heads x
     // contexts of 16x32x<=178, 64x40x<=2048, 32x32x<=4096, 256x32x<=4096):
@@ -228,7 +228,7 @@ int fill_config(const pa_cache_desc &c, int num_seqs, int max_ctx, pa_decode_con
     return PA_OK;
 }
 
-int max_parts_of(int max_ctx, int P) { return std::max(1, (max_ctx + P - 1) / P); }
+int max_parts_of(int max_ctx, int P) { return (int)std::max<int64_t>(1, ((int64_t)max_ctx + P - 1) / P); }
 
 size_t ws_lse_bytes(const pa_cache_desc &c, int S, int parts) {
     return ((size_t)S * c.num_heads * parts * sizeof(float) + 255) / 256 * 256;
@@ -521,7 +521,7 @@ int pa_slot_mapping(int32_t *slot_mapping, const int32_t *block_tables, int max_
         return fail(PA_ERR_INVALID, "null pointer argument");
     if (max_blocks_per_seq < 1) return fail(PA_ERR_INVALID, "max_blocks_per_seq < 1");
     const int threads = 128;
-    pa::slot_mapping_kernel<<<(num_seqs + threads - 1) / threads, threads, 0,
+    pa::slot_mapping_kernel<<<(unsigned)(((int64_t)num_seqs + threads - 1) / threads), threads, 0,
                               static_cast<cudaStream_t>(stream)>>>(
         slot_mapping, block_tables, max_blocks_per_seq, context_lens, num_seqs, cache.block_size,
         cache.num_blocks);
@@ -977,7 +977,7 @@ extern "C" int pa_prefill_slot_mapping(int32_t *slot_mapping, const int32_t *que
         return fail(PA_ERR_INVALID, "null pointer argument");
     if (max_blocks_per_seq < 1) return fail(PA_ERR_INVALID, "max_blocks_per_seq < 1");
     const int threads = 256;
-    const int gx = std::max(1, std::min((max_query_len + threads - 1) / threads, 1024));
+    const int gx = (int)std::max<int64_t>(1, std::min<int64_t>(((int64_t)max_query_len + threads - 1) / threads, 1024));
     pa::prefill_slot_mapping_kernel<<<dim3(gx, num_seqs), threads, 0, static_cast<cudaStream_t>(stream)>>>(
         slot_mapping, total_q, query_start, block_tables, max_blocks_per_seq, context_lens, cache.block_size,
         cache.num_blocks);
@@ -1011,7 +1011,7 @@ extern "C" int pa_paged_prefill(void *out, const void *query, const int32_t *que
     // tiles).
     const bool tc = (cache.head_size == 64 || cache.head_size == 128) && scale > 0.f;
     const int rows_per_cta = tc ? pa::kTcRows : pa::kPrefillRows;
-    const int64_t row_tiles = (max_query_len + rows_per_cta - 1) / rows_per_cta;
+    const int64_t row_tiles = ((int64_t)max_query_len + rows_per_cta - 1) / rows_per_cta;
     const int64_t n_ctas = row_tiles * num_seqs * cache.num_heads;
     if (n_ctas > 0x7fffffff) return fail(PA_ERR_INVALID, "too many prefill tiles (%lld)", (long long)n_ctas);
     int dev = 0;

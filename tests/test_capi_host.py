@@ -245,3 +245,21 @@ def test_swap_append_and_shared_prefix_argument_checks():
     assert L.pa_shared_prefix_workspace_size(D, 2, 64, 5, None) == 0
     assert L.pa_shared_prefix_workspace_size(D, 2, 64, 1 << 28, None) == 0
     assert L.pa_shared_prefix_workspace_size(D, 2, 64, 2, None) > 0
+
+
+def test_bounds_at_the_int32_limit():
+    # ceiling divisions of caller-given bounds are done in 64-bit: a context
+    # or query-length bound of 2^31 - 1 gives a valid plan, or a clean
+    # refusal before any CUDA call
+    L = capi.lib()
+    big = 2**31 - 1
+    desc = capi.CacheDesc(2048, 16, 32, 128, capi.PA_F16)
+    rc, c = _choose(desc, 16, big)
+    assert rc == capi.PA_OK, _last()
+    assert c.partition_size % 16 == 0 and c.stages % c.warps_per_head == 0
+    ws = L.pa_decode_workspace_size(desc, 16, big, None)
+    parts = -(-big // c.partition_size)
+    assert ws >= 16 * 32 * parts * 128 * 4
+    T = 100
+    assert L.pa_paged_prefill(P, P, P, P, P, F, P, 4, P, 65535, T, big, 0.1, None) == capi.PA_ERR_INVALID
+    assert "too many prefill tiles" in _last()
