@@ -35,7 +35,7 @@
  *     num_heads x head_size). Logical token t of a sequence lives in physical
  *     block block_tables[s][t / block_size], row t % block_size.
  *   - Supported shapes: head_size 64 or 128; block_size 16 or 32;
- *     num_heads >= 1; num_blocks * block_size < 2^31.
+ *     1 <= num_heads <= 65535; num_blocks * block_size < 2^31.
  *   - Query, output, new K/V rows and caches must be 16-byte aligned.
  *   - Counts: num_seqs <= 65535 per decode or prefill call; token and pair
  *     counts of the cache write, block copy and swap have no such limit (the

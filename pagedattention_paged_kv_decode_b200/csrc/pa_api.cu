@@ -48,6 +48,8 @@ int check_cache(const pa_cache_desc &c) {
     if (c.num_blocks < 1 || c.num_heads < 1)
         return fail(PA_ERR_INVALID, "num_blocks (%d) and num_heads (%d) must be >= 1",
                     c.num_blocks, c.num_heads);
+    if (c.num_heads > 65535)  // keeps num_heads * head_size and the per-head grids in int
+        return fail(PA_ERR_INVALID, "num_heads %d > 65535", c.num_heads);
     if (c.block_size != 16 && c.block_size != 32)
         return fail(PA_ERR_INVALID, "block_size %d: supported are 16 and 32", c.block_size);
     if (c.head_size != 64 && c.head_size != 128)

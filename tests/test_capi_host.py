@@ -51,6 +51,8 @@ def _last():
     (capi.CacheDesc(64, 8, 8, 128, 0), capi.PA_ERR_INVALID),
     (capi.CacheDesc(64, 16, 8, 96, 0), capi.PA_ERR_INVALID),
     (capi.CacheDesc(0, 16, 8, 128, 0), capi.PA_ERR_INVALID),
+    (capi.CacheDesc(64, 16, 0, 128, 0), capi.PA_ERR_INVALID),
+    (capi.CacheDesc(64, 16, 65536, 128, 0), capi.PA_ERR_INVALID),
     (capi.CacheDesc(1 << 27, 16, 8, 128, 0), capi.PA_ERR_OVERFLOW),
 ])
 def test_bad_cache_descriptors(desc, code):
