@@ -265,3 +265,48 @@ def test_bounds_at_the_int32_limit():
     T = 100
     assert L.pa_paged_prefill(P, P, P, P, P, F, P, 4, P, 65535, T, big, 0.1, None) == capi.PA_ERR_INVALID
     assert "too many prefill tiles" in _last()
+
+
+def _prototypes():
+    """name -> (return type, [parameter types]) of every pa_* prototype in the header."""
+    with open(HEADER, encoding="utf-8") as f:
+        text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+    out = {}
+    for ret, name, params in re.findall(r"([A-Za-z_][\w \*]*?)\s*\b(pa_[a-z0-9_]+)\s*\(([^)]*)\)\s*;", text):
+        types = []
+        for prm in (p.strip() for p in params.split(",")):
+            if prm in ("", "void"):
+                continue
+            types.append(re.sub(r"\s*\b\w+$", "", prm).replace(" *", "*").strip())   # drop the name
+        out[name] = (" ".join(ret.split()).replace(" *", "*"), types)
+    return out
+
+
+_CTYPE_OF = {
+    "int": ctypes.c_int, "int64_t": ctypes.c_int64, "float": ctypes.c_float, "size_t": ctypes.c_size_t,
+    "pa_cache_desc": capi.CacheDesc, "const char*": ctypes.c_char_p,
+}
+
+
+def _expected_ctype(ctype: str):
+    if ctype in _CTYPE_OF:
+        return _CTYPE_OF[ctype]
+    if ctype in ("const pa_decode_config*", "pa_decode_config*"):
+        return ctypes.POINTER(capi.DecodeConfig)
+    if ctype == "uint32_t*":
+        return ctypes.POINTER(ctypes.c_uint32)
+    assert ctype.endswith("*"), ctype
+    return ctypes.c_void_p            # every other pointer crosses as an address
+
+
+def test_ctypes_signatures_match_the_header():
+    protos = _prototypes()
+    assert set(protos) == set(capi.SIGNATURES), set(protos) ^ set(capi.SIGNATURES)
+    for name, (ret, params) in protos.items():
+        res, args = capi.SIGNATURES[name]
+        assert res is _expected_ctype(ret), (name, ret, res)
+        assert len(args) == len(params), (name, params)
+        for i, (ct, a) in enumerate(zip(params, args)):
+            want = _expected_ctype(ct)
+            assert a is want or (isinstance(a, type) and issubclass(want, ctypes._Pointer)
+                                 and a._type_ is want._type_), (name, i, ct, a)
