@@ -11,15 +11,18 @@ from .ops import (  # noqa: F401
     cache_desc,
     check_status,
     choose_config,
+    decode_choose_config,
     copy_blocks,
     decode_step,
     decode_workspace_size,
     kv_cache_write,
+    last_error,
     load_cache,
     paged_attention_decode,
     paged_attention_decode_append,
     paged_attention_decode_noalloc,
     paged_attention_decode_shared_prefix,
+    paged_attention_decode_ws,
     paged_prefill,
     prefill_slot_mapping,
     prefill_step,

@@ -185,6 +185,12 @@ def choose_config(key_cache: torch.Tensor, num_seqs: int, max_context_len: int, 
     return cfg.as_dict()
 
 
+def decode_choose_config(key_cache: torch.Tensor, num_seqs: int, max_context_len: int, config=None) -> dict:
+    """The launch shape the decode would use (``choose_config`` under the C
+    entry point's name)."""
+    return choose_config(key_cache, num_seqs, max_context_len, config)
+
+
 def decode_workspace_size(key_cache: torch.Tensor, num_seqs: int, max_context_len: int,
                           config=None) -> int:
     cfg = _config(config)
@@ -230,11 +236,26 @@ def paged_attention_decode(out: torch.Tensor, query: torch.Tensor, key_cache: to
     entry point is used (``workspace`` a uint8 CUDA tensor of at least
     ``decode_workspace_size`` bytes).
     """
+    if config is not None or workspace is not None:
+        paged_attention_decode_ws(out, query, key_cache, value_cache, block_tables, context_lens, scale,
+                                  k_scale, v_scale, max_context_len, config, workspace, stream)
+        return
+    args = _decode_args(out, query, key_cache, value_cache, block_tables, context_lens, scale, k_scale,
+                        v_scale, max_context_len)
+    check(lib().pa_paged_attention_decode(*args, _stream(stream)))
+
+
+def paged_attention_decode_ws(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
+                              value_cache: torch.Tensor, block_tables: torch.Tensor,
+                              context_lens: torch.Tensor, scale: float, k_scale: float = 1.0,
+                              v_scale: float = 1.0, max_context_len: int | None = None,
+                              config=None, workspace: torch.Tensor | None = None, stream=None) -> None:
+    """Decode with an explicit launch shape (``config``: a dict or DecodeConfig,
+    zero fields = library choice) and/or a caller workspace (a contiguous
+    CUDA tensor of at least ``decode_workspace_size`` bytes, 256-byte
+    aligned); either may be None."""
     args = _decode_args(out, query, key_cache, value_cache, block_tables, context_lens, scale, k_scale,
                         v_scale, max_context_len, workspace)
-    if config is None and workspace is None:
-        check(lib().pa_paged_attention_decode(*args, _stream(stream)))
-        return
     cfg = _config(config)
     ws_ptr, ws_bytes = _workspace(workspace)
     check(lib().pa_paged_attention_decode_ws(*args, ctypes.byref(cfg) if cfg is not None else None,
@@ -371,6 +392,12 @@ def check_status(stream=None) -> int:
 
 def version() -> int:
     return int(lib().pa_version())
+
+
+def last_error() -> str:
+    """Message of the last nonzero status on this thread ("" if none); the
+    binding also raises it as PagedKVError."""
+    return lib().pa_last_error().decode(errors="replace")
 
 
 def load_cache(key_cache: torch.Tensor, value_cache: torch.Tensor, key_src: torch.Tensor,
