@@ -51,6 +51,8 @@ MUTANTS = {
     "softmax weight sign": ("acc += exp(z[i] - m) * cache_value", "acc += exp(m - z[i]) * cache_value"),
     "normaliser omitted": ("o[d] = acc / l;", "o[d] = acc;"),
     "E4M3 V written with k_scale": ("float vq = vf / v_scale;", "float vq = vf / k_scale;"),
+    "E4M3 K written with v_scale": ("float kq = kf / k_scale;", "float kq = kf / v_scale;"),
+    "E4M3 K scale multiplied": ("float kq = kf / k_scale;", "float kq = kf * k_scale;"),
     "copy direction reversed": ("memmove((char *)key_cache + dst * block_bytes,\n                (char *)key_cache + src * block_bytes",
                                 "memmove((char *)key_cache + src * block_bytes,\n                (char *)key_cache + dst * block_bytes"),
     "swap copies only K": ("memcpy((char *)dst_value + dst * block_bytes", "memcpy((char *)dst_key + dst * block_bytes"),
@@ -211,6 +213,7 @@ def pin_battery():
         ev = np.zeros_like(ek)
         oracle.kv_cache_write(key, key, ek, ev, np.array([6, 13], np.int32), 0.5, 2.0)
         return (np.array_equal(kc[1, 2], key[0]) and np.array_equal(vc[3, 1], key[1] + 1)
+                and np.array_equal(ek[1, 2], oracle.e4m3_from_float(key[0].astype(np.float32) / np.float32(0.5)))
                 and np.array_equal(ev[1, 2], oracle.e4m3_from_float(key[0].astype(np.float32) / np.float32(2.0))))
 
     def copy_semantics():
