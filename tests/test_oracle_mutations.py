@@ -153,7 +153,9 @@ def pin_battery():
         even = np.where(codes[:-1] % 2 == 0, codes[:-1], codes[1:]).astype(np.uint8)
         return (np.array_equal(oracle.e4m3_from_float(x), ref) and list(sat) == [0x7E, 0x7E, 0xFE, 0x00, 0x80]
                 and np.array_equal(oracle.e4m3_from_float(mids), even)
-                and np.array_equal(oracle.e4m3_from_float(-mids), even | 0x80))
+                and np.array_equal(oracle.e4m3_from_float(-mids), even | 0x80)
+                and np.array_equal(oracle.e4m3_from_float(vals.astype(np.float32)), codes)       # codes themselves
+                and np.array_equal(oracle.e4m3_from_float(-vals.astype(np.float32)), codes | 0x80))
 
     def dense_equivalence():
         w, kc, vc = _complete([1, 9, 30], H=3, D=16, B=8, deal="identity", seed=1)
@@ -205,41 +207,131 @@ def pin_battery():
         return np.array_equal(base, oracle.paged_attention(w.query, kc2, vc2, bt2, w.context_lens, w.scale))
 
     def cache_write_readback():
+        # slots 0 (the first), 6, 13 and 15 (the last) of a 4 x 4 pool; a
+        # negative slot is padding; every other slot must stay zero
+        slots = np.array([0, 6, -1, 13, 15], np.int32)
+        key = np.random.default_rng(1).standard_normal((5, 2, 8)).astype(np.float16) + np.float16(0.25)
         kc = np.zeros((4, 4, 2, 8), np.float16)
         vc = np.zeros_like(kc)
-        key = np.random.default_rng(1).standard_normal((2, 2, 8)).astype(np.float16)
-        oracle.kv_cache_write(key, key + 1, kc, vc, np.array([6, 13], np.int32))
+        oracle.kv_cache_write(key, key + 1, kc, vc, slots)
         ek = np.zeros((4, 4, 2, 8), np.uint8)
         ev = np.zeros_like(ek)
-        oracle.kv_cache_write(key, key, ek, ev, np.array([6, 13], np.int32), 0.5, 2.0)
-        return (np.array_equal(kc[1, 2], key[0]) and np.array_equal(vc[3, 1], key[1] + 1)
-                and np.array_equal(ek[1, 2], oracle.e4m3_from_float(key[0].astype(np.float32) / np.float32(0.5)))
-                and np.array_equal(ev[1, 2], oracle.e4m3_from_float(key[0].astype(np.float32) / np.float32(2.0))))
+        oracle.kv_cache_write(key, key, ek, ev, slots, 0.5, 2.0)
+        want_k, want_v = np.zeros_like(kc), np.zeros_like(kc)
+        want_ek, want_ev = np.zeros_like(ek), np.zeros_like(ek)
+        for i, sl in enumerate(slots):
+            if sl >= 0:
+                b, r = divmod(int(sl), 4)
+                want_k[b, r], want_v[b, r] = key[i], key[i] + 1
+                want_ek[b, r] = oracle.e4m3_from_float(key[i].astype(np.float32) / np.float32(0.5))
+                want_ev[b, r] = oracle.e4m3_from_float(key[i].astype(np.float32) / np.float32(2.0))
+        return (np.array_equal(kc.view(np.uint16), want_k.view(np.uint16))
+                and np.array_equal(vc.view(np.uint16), want_v.view(np.uint16))
+                and np.array_equal(ek, want_ek) and np.array_equal(ev, want_ev) and want_ek.any())
 
     def copy_semantics():
-        kc = np.random.default_rng(2).standard_normal((4, 2, 1, 8)).astype(np.float16)
+        kc = np.random.default_rng(2).standard_normal((5, 2, 1, 8)).astype(np.float16)
         vc = kc + 1
         k0 = kc.copy()
-        oracle.copy_blocks(kc, vc, np.array([[1, 3]], np.int32))
-        return np.array_equal(kc[3], k0[1]) and np.array_equal(kc[1], k0[1]) and np.array_equal(vc[3], k0[1] + 1)
+        v0 = vc.copy()
+        oracle.copy_blocks(kc, vc, np.array([[1, 3], [2, 0]], np.int32))   # block 0 as a destination
+        oracle.copy_blocks(kc, vc, np.array([[0, 4]], np.int32))           # and then as a source
+        wk, wv = k0.copy(), v0.copy()
+        wk[3], wv[3], wk[0], wv[0], wk[4], wv[4] = k0[1], v0[1], k0[2], v0[2], k0[2], v0[2]
+        return np.array_equal(kc, wk) and np.array_equal(vc, wv)
 
     def swap_semantics():
         src = np.random.default_rng(3).standard_normal((3, 2, 1, 8)).astype(np.float16)
-        dk, dv = np.zeros_like(src), np.zeros_like(src)
-        oracle.swap_blocks(dk, dv, src, src + 1, np.array([[2, 0]], np.int32))
-        return np.array_equal(dk[0], src[2]) and np.array_equal(dv[0], src[2] + 1)
+        dk = np.zeros((4,) + src.shape[1:], np.float16)
+        dv = np.zeros_like(dk)
+        oracle.swap_blocks(dk, dv, src, src + 1, np.array([[2, 1], [0, 3], [1, 0]], np.int32))
+        wk, wv = np.zeros_like(dk), np.zeros_like(dk)
+        wk[1], wv[1], wk[3], wv[3], wk[0], wv[0] = src[2], src[2] + 1, src[0], src[0] + 1, src[1], src[1] + 1
+        return np.array_equal(dk, wk) and np.array_equal(dv, wv)
 
     def empty_context():
-        # a sequence with no context has no slot and a zero output row
+        # a sequence with no context has no slot and a zero output row (the
+        # last row, so that a write past it leaves the array)
         rng = np.random.default_rng(22)
-        bt = np.array([[2, -1], [1, 3]], np.int32)
-        ctx = np.array([0, 5], np.int32)
+        bt = np.array([[1, 3], [2, -1]], np.int32)
+        ctx = np.array([5, 0], np.int32)
         slots = oracle.slot_mapping(bt, ctx, 4)
         kc = rng.standard_normal((4, 4, 1, 8)).astype(np.float16)
         vc = rng.standard_normal((4, 4, 1, 8)).astype(np.float16)
         q = rng.standard_normal((2, 1, 8)).astype(np.float16)
         out = oracle.paged_attention(q, kc, vc, bt, ctx, 0.5)
-        return list(slots) == [-1, 12] and np.array_equal(out[0], np.zeros((1, 8))) and np.isfinite(out).all()
+        return list(slots) == [12, -1] and np.array_equal(out[1], np.zeros((1, 8))) and np.isfinite(out).all()
+
+    def subsets():
+        # selected (sequence, head) / (row, head) pairs equal those rows of the full result
+        w, kc, vc = _complete([5, 17, 33], seed=24)
+        full = oracle.paged_attention(w.query, kc, vc, w.block_tables, w.context_lens, w.scale)
+        pairs = np.array([[2, 1], [0, 2], [1, 0], [2, 2]], np.int32)
+        sub = oracle.paged_attention(w.query, kc, vc, w.block_tables, w.context_lens, w.scale, seq_head=pairs)
+        if not all(np.array_equal(sub[i], full[s, h]) for i, (s, h) in enumerate(pairs)):
+            return False
+        ctx, n = [12, 9], [5, 9]
+        pw = W.build_prefill("sub", 3, 16, 8, ctx, n, 6, 2, 25, 1.0, 1.0)
+        pk_, pv_ = pw.pool_host()
+        oracle.kv_cache_write(pw.new_key, pw.new_value, pk_, pv_,
+                              oracle.prefill_slot_mapping(pw.query_start, pw.block_tables, pw.context_lens, 8))
+        pfull = oracle.paged_prefill(pw.query, pw.query_start, pk_, pv_, pw.block_tables, pw.context_lens, pw.scale)
+        rows = np.array([[13, 2], [0, 1], [6, 0], [4, 2]], np.int32)
+        psub = oracle.paged_prefill(pw.query, pw.query_start, pk_, pv_, pw.block_tables, pw.context_lens, pw.scale,
+                                    row_head=rows)
+        return all(np.array_equal(psub[i], pfull[r, h]) for i, (r, h) in enumerate(rows))
+
+    def input_validation():
+        # each input one step past a bound is rejected; the last valid value
+        # at that bound is accepted
+        def rejects(fn):
+            try:
+                fn()
+            except ValueError:
+                return True
+            return False
+
+        rng = np.random.default_rng(26)
+        pool = rng.standard_normal((4, 4, 1, 8)).astype(np.float16)
+        q = rng.standard_normal((2, 1, 8)).astype(np.float16)
+        bt = np.array([[1, 3], [0, 2]], np.int32)
+        row = np.zeros((1, 1, 8), np.float16)
+        ok = [
+            oracle.slot_mapping(bt, np.array([8, 1], np.int32), 4)[0] == 3 * 4 + 3,            # last table slot
+            rejects(lambda: oracle.slot_mapping(bt, np.array([9, 1], np.int32), 4)),           # one past the table
+            list(oracle.prefill_slot_mapping(np.array([0, 0, 1], np.int32), bt, np.array([3, 1], np.int32), 4))
+            == [0],                                                                             # empty chunk
+            rejects(lambda: oracle.prefill_slot_mapping(np.array([0, 4, 5], np.int32), bt,
+                                                        np.array([3, 1], np.int32), 4)),        # chunk > context
+            rejects(lambda: oracle.prefill_slot_mapping(np.array([0, 9, 10], np.int32), bt,
+                                                        np.array([9, 1], np.int32), 4)),        # past the table
+            rejects(lambda: oracle.kv_cache_write(row, row, pool.copy(), pool.copy(), np.array([16], np.int32))),
+            rejects(lambda: oracle.copy_blocks(pool.copy(), pool.copy(), np.array([[4, 0]], np.int32))),
+            rejects(lambda: oracle.copy_blocks(pool.copy(), pool.copy(), np.array([[0, 4]], np.int32))),
+            rejects(lambda: oracle.copy_blocks(pool.copy(), pool.copy(), np.array([[-1, 0]], np.int32))),
+            rejects(lambda: oracle.swap_blocks(pool[:2].copy(), pool[:2].copy(), pool, pool,
+                                               np.array([[3, 2]], np.int32))),                  # dst past its pool
+            rejects(lambda: oracle.swap_blocks(pool[:2].copy(), pool[:2].copy(), pool, pool,
+                                               np.array([[4, 1]], np.int32))),                  # src past its pool
+            rejects(lambda: oracle.paged_attention(q, pool, pool, np.array([[1, 4], [0, 2]], np.int32),
+                                                   np.array([8, 1], np.int32), 0.5)),           # block id = pool size
+            rejects(lambda: oracle.paged_attention(q, pool, pool, np.array([[1, -1], [0, 2]], np.int32),
+                                                   np.array([8, 1], np.int32), 0.5)),           # hole in the table
+            rejects(lambda: oracle.paged_attention(q, pool, pool, bt, np.array([9, 1], np.int32), 0.5)),
+            rejects(lambda: oracle.paged_attention(q, pool, pool, bt, np.array([8, 1], np.int32), 0.5,
+                                                   seq_head=np.array([[2, 0]], np.int32))),
+            rejects(lambda: oracle.paged_attention(q, pool, pool, bt, np.array([8, 1], np.int32), 0.5,
+                                                   seq_head=np.array([[0, 1]], np.int32))),
+            rejects(lambda: oracle.paged_prefill(q, np.array([0, 2, 2], np.int32), pool, pool, bt,
+                                                 np.array([1, 1], np.int32), 0.5)),             # first chunk > context
+            rejects(lambda: oracle.paged_prefill(q, np.array([0, 1, 2], np.int32), pool, pool, bt,
+                                                 np.array([3, 1], np.int32), 0.5,
+                                                 row_head=np.array([[2, 0]], np.int32))),
+            rejects(lambda: oracle.paged_prefill(q, np.array([0, 1, 2], np.int32), pool, pool, bt,
+                                                 np.array([3, 1], np.int32), 0.5,
+                                                 row_head=np.array([[0, 1]], np.int32))),
+        ]
+        return all(ok)
 
     def e4m3_attention():
         # an E4M3 cache at scales (1/2, 4) against fp16 caches holding its
@@ -259,15 +351,23 @@ def pin_battery():
         return np.array_equal(a, oracle.paged_attention(q, f16_k, f16_v, bt, ctx, 0.3))
 
     def lse_identity():
-        w, kc, vc = _complete([15, 40], seed=14)
+        w, kc, vc = _complete([1, 15, 16, 17, 32, 40], seed=14)
         full = oracle.paged_attention(w.query, kc, vc, w.block_tables, w.context_lens, w.scale)
         o, lse = oracle.attention_partials(w.query, kc, vc, w.block_tables, w.context_lens, w.scale, 16)
         for s, L in enumerate(w.context_lens):
             n = -(-int(L) // 16)
+            if not (np.isnan(lse[s, :, n:]).all() and np.isnan(o[s, :, n:]).all()):
+                return False           # a partition past the context holds nothing
             for h in range(w.num_heads):
                 if not np.abs(oracle.lse_combine(o[s, h, :n], lse[s, h, :n]) - full[s, h]).max() <= 1e-12:
                     return False
-        return True
+        # an empty context has no partition at all (the last sequence, so
+        # that a write past its rows leaves the arrays)
+        bt = np.array([[0, 2], [1, -1]], np.int32)
+        pool = np.random.default_rng(23).standard_normal((3, 16, 1, 8)).astype(np.float16)
+        q = np.ones((2, 1, 8), np.float16)
+        o, lse = oracle.attention_partials(q, pool, pool, bt, np.array([20, 0], np.int32), 0.5, 16)
+        return bool(np.isnan(o[1]).all() and np.isnan(lse[1]).all() and np.isfinite(lse[0]).all())
 
     def prefill_worked_example():
         got = oracle.prefill_slot_mapping(np.array([0, 32, 48], np.int32), np.array([[5, 8], [3, -1]], np.int32),
@@ -281,7 +381,7 @@ def pin_battery():
         return np.array_equal(got, oracle.slot_mapping(w.block_tables, w.context_lens, 4))
 
     def prefill_dense_causal():
-        ctx, n = [12, 9, 17], [5, 9, 1]
+        ctx, n = [12, 9, 17, 6], [5, 9, 1, 0]
         need = sum(-(-L // 8) for L in ctx)
         w = W.build_prefill("p", 2, 16, 8, ctx, n, need + 2, 3, 2, 1.0, 1.0, deal_order="identity")
         kc, vc = w.pool_host()
@@ -306,6 +406,7 @@ def pin_battery():
                      ("brute force", brute_force), ("relabelling", relabelling),
                      ("cache write", cache_write_readback), ("copy", copy_semantics), ("swap", swap_semantics),
                      ("empty context", empty_context), ("e4m3 attention", e4m3_attention),
+                     ("subsets", subsets), ("input validation", input_validation),
                      ("lse identity", lse_identity), ("prefill worked example", prefill_worked_example),
                      ("prefill one-token chunks", prefill_one_token_chunks),
                      ("prefill dense causal", prefill_dense_causal)]:
