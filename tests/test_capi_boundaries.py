@@ -38,6 +38,14 @@ def test_cache_descriptor_bounds(L):
         assert L.pa_kv_cache_write(P, P, ROW, ROW, P, P, d, P, 0, 1.0, 1.0, None) == capi.PA_OK, L.pa_last_error()
 
 
+def test_slot_mapping_checks(L):
+    for i in range(3):
+        args = [P] * 3
+        args[i] = None
+        assert said(L, L.pa_slot_mapping(args[0], args[1], 4, args[2], 2, F, None), "null pointer")
+    assert said(L, L.pa_slot_mapping(P, P, 0, P, 2, F, None), "max_blocks_per_seq")
+
+
 def test_kv_cache_write_checks(L):
     w = lambda k, v, ks, vs, kc, vc, sl, desc=F, kscale=1.0: L.pa_kv_cache_write(  # noqa: E731
         k, v, ks, vs, kc, vc, desc, sl, 4, kscale, 1.0, None)
@@ -109,6 +117,7 @@ def test_append_and_shared_prefix_checks(L):
     assert said(L, pre(None, None, ROW, ROW, 4), "partition_size")             # prefix = the whole table
     assert said(L, pre(None, None, ROW, ROW, 5), "shared_prefix_blocks")
     assert said(L, pre(None, None, ROW, ROW, 1), "partition_size")             # one block is valid
+    assert said(L, pre(P, P, ROW, ROW, 2), "partition_size")                   # row-length strides are valid
     for nk, nv in ((P + 8, P), (P, P + 8)):
         assert said(L, pre(nk, nv, ROW, ROW, 2), "aligned")
     for ks, vs in ((ROW - 8, ROW), (ROW, ROW - 8), (ROW + 4, ROW), (ROW, ROW + 4)):
