@@ -68,17 +68,15 @@ def _table(block_tables: torch.Tensor, S: int) -> None:
         raise ValueError("block_tables must be int32 [num_seqs, max_blocks_per_seq]")
 
 
-def _f16_3d(t: torch.Tensor, name: str, shape=None, rows_only: bool = False) -> None:
-    """fp16 CUDA [n, H, D]; contiguous, or (rows_only) contiguous within a token."""
+def _f16_rows(t: torch.Tensor, name: str, shape) -> None:
+    """fp16 CUDA [n, H, D] of the given shape, each token's row contiguous
+    (the token stride is free)."""
     if t.dtype != torch.float16 or not t.is_cuda or t.dim() != 3:
         raise ValueError(f"{name} must be a float16 CUDA tensor [n, H, D]")
-    if shape is not None and tuple(t.shape) != tuple(shape):
+    if tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
-    if rows_only:
-        if t.stride(2) != 1 or t.stride(1) != t.shape[2]:
-            raise ValueError(f"{name} rows must be contiguous within a token")
-    elif not t.is_contiguous():
-        raise ValueError(f"{name} must be contiguous")
+    if t.stride(2) != 1 or t.stride(1) != t.shape[2]:
+        raise ValueError(f"{name} rows must be contiguous within a token")
 
 
 def _slots_out(slot_mapping: torch.Tensor | None, S: int) -> None:
@@ -125,8 +123,8 @@ def kv_cache_write(key: torch.Tensor, value: torch.Tensor, key_cache: torch.Tens
     _i32(slot_mapping, "slot_mapping")
     n = slot_mapping.shape[0]
     _, _, H, D = key_cache.shape
-    _f16_3d(key, "key", (n, H, D), rows_only=True)
-    _f16_3d(value, "value", (n, H, D), rows_only=True)
+    _f16_rows(key, "key", (n, H, D))
+    _f16_rows(value, "value", (n, H, D))
     _on_current_device(key, value, key_cache, value_cache, slot_mapping)
     check(lib().pa_kv_cache_write(key.data_ptr(), value.data_ptr(), key.stride(0), value.stride(0),
                                   key_cache.data_ptr(), value_cache.data_ptr(), cache_desc(key_cache),

@@ -9,43 +9,12 @@ expected C call, and every argument must convert to the ctypes type that
 the library declares for that position (which a separate test ties to the
 header's prototypes).
 """
-import ctypes
 
 import pytest
 import torch
 
+from _binding_fakes import Recorder as _Recorder, fake as _fake
 from pagedattention_paged_kv_decode_b200 import capi, ops
-
-
-class _FakeCuda(torch.Tensor):
-    @property
-    def is_cuda(self):
-        return True
-
-
-def _fake(t):
-    return torch.Tensor._make_subclass(_FakeCuda, t)
-
-
-class _Recorder:
-    """Stands in for the loaded library: records each pa_* call."""
-
-    def __init__(self):
-        self.calls = []
-
-    def __getattr__(self, name):
-        if name not in capi.SIGNATURES:
-            raise AttributeError(name)
-        res = capi.SIGNATURES[name][0]
-
-        def call(*args):
-            self.calls.append((name, args))
-            if res is ctypes.c_size_t:
-                return 4096
-            if res is ctypes.c_char_p:
-                return b""
-            return 201 if name == "pa_version" else 0
-        return call
 
 
 @pytest.fixture
