@@ -1,6 +1,10 @@
 """Host helpers of bench.py: the code hash that keeps a recorded ncu traffic
-figure tied to the kernel sources it was taken on."""
+figure tied to the kernel sources it was taken on, the clock summary that
+decides whether a run was throttled, the peaks the roofline divides by, and
+the whole-job aggregate."""
 import json
+
+import pytest
 
 import bench
 
@@ -47,3 +51,39 @@ def test_committed_records_are_well_formed():
             assert len(ent["kernel_source_hash"]) == 16 and int(ent["kernel_source_hash"], 16) >= 0
             assert isinstance(ent["dram_bytes_per_launch"], int) and ent["dram_bytes_per_launch"] > 0
             assert ent["source"].startswith("profiles/")
+
+
+def _smi_row(sm, max_sm, reasons):
+    # the ClockSampler field order: timestamp, index, clocks.sm, clocks.max.sm, power.draw,
+    # clocks_event_reasons.active, then hw_slowdown, hw_thermal_slowdown, sw_thermal_slowdown, sw_power_cap
+    return ["2026/01/01 00:00:00.000", "0", str(sm), str(max_sm), "700.0", "0x0"] + reasons
+
+
+def test_clock_summary_reads_the_timed_window():
+    off = ["Not Active"] * 4
+    cs = bench.ClockSampler("0")
+    cs.rows = [(0.0, _smi_row(1200, 1965, off)),
+               (10.0, _smi_row(1965, 1965, off[:3] + ["Active"])),           # sw_power_cap
+               (10.4, _smi_row(1900, 1965, ["Active"] + off[1:])),           # hw_slowdown
+               (60.0, _smi_row(800, 1965, off[:1] + ["Active"] + off[2:]))]  # outside the window
+    s = cs.summary(10.0, 10.4)
+    assert s == {"sm_mhz": 1932.5, "sm_max_mhz": 1965.0, "reasons": ["hw_slowdown", "sw_power_cap"], "samples": 2}
+    # no sample inside the window (a short run): every sample counts
+    s = cs.summary(30.0, 30.1)
+    assert s["samples"] == 4 and s["reasons"] == ["hw_slowdown", "hw_thermal_slowdown", "sw_power_cap"]
+    assert bench.ClockSampler("0").summary(0.0, 1.0)["reasons"] == ["nvidia-smi unavailable"]
+
+
+def test_peaks_come_from_the_measured_file_else_the_fallback(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.hbm_peak() == (bench.FALLBACK_HBM_GBS, "fallback")
+    assert bench.tensor_peak() == (1590.0, 1400.0, "fallback")
+    (tmp_path / "MEASURED_PEAKS.json").write_text(
+        json.dumps({"hbm_gbs": 6000.5, "bf16_tflops": 1600, "bf16_tflops_sustained": 1300}))
+    assert bench.hbm_peak() == (6000.5, "measured")
+    assert bench.tensor_peak() == (1600.0, 1300.0, "measured")
+
+
+def test_aggregate_is_all_ranks_bytes_over_the_slowest_time():
+    assert bench.aggregate_gbs(1, 10**9, 1000.0) == pytest.approx(1.0)
+    assert bench.aggregate_gbs(4, 10**9, 500.0) == pytest.approx(8.0)
