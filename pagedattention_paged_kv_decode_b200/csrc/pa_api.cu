@@ -660,7 +660,7 @@ int pa_paged_attention_decode(void *out, const void *query, const void *key_cach
     if (rc) return rc;
     if (num_seqs == 0) return ok();
     const int bound = (int)std::min<int64_t>(max_context_len, (int64_t)max_blocks_per_seq * cache.block_size);
-    pa_decode_config cfg{0, 0, 0, 0};
+    pa_decode_config cfg{0, 0, 0, 0, 0};
     rc = fill_config(cache, num_seqs, bound, &cfg);
     if (rc) return rc;
     int dev = 0;
@@ -912,7 +912,7 @@ extern "C" int pa_paged_attention_decode_noalloc(
     if (num_seqs == 0) return ok();
     const int bound =
         (int)std::min<int64_t>(max_context_len, (int64_t)max_blocks_per_seq * cache.block_size);
-    pa_decode_config cfg{0, 0, 0, 0};
+    pa_decode_config cfg{0, 0, 0, 0, 0};
     rc = fill_config(cache, num_seqs, bound, &cfg);
     if (rc) return rc;
     const size_t need = ws_bytes(cache, num_seqs, bound, cfg);
