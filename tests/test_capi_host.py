@@ -310,3 +310,11 @@ def test_ctypes_signatures_match_the_header():
             want = _expected_ctype(ct)
             assert a is want or (isinstance(a, type) and issubclass(want, ctypes._Pointer)
                                  and a._type_ is want._type_), (name, i, ct, a)
+
+
+def test_python_constants_match_the_header():
+    with open(HEADER, encoding="utf-8") as f:
+        defines = dict(re.findall(r"^#define (PA_\w+)\s+\(?(-?\d+)u?\)?", f.read(), flags=re.M))
+    assert len(defines) >= 15
+    for name, value in defines.items():
+        assert getattr(capi, name) == int(value), name
