@@ -318,3 +318,15 @@ def test_python_constants_match_the_header():
     assert len(defines) >= 15
     for name, value in defines.items():
         assert getattr(capi, name) == int(value), name
+
+
+def test_ctypes_structs_match_the_header():
+    with open(HEADER, encoding="utf-8") as f:
+        text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+    structs = {name: re.findall(r"(\w+)\s+(\w+);", body)
+               for body, name in re.findall(r"typedef struct \{(.*?)\} (pa_\w+);", text, flags=re.S)}
+    for cname, cls in (("pa_cache_desc", capi.CacheDesc), ("pa_decode_config", capi.DecodeConfig)):
+        fields = structs[cname]
+        assert [n for _, n in fields] == [n for n, _ in cls._fields_], cname
+        assert all(t == "int32_t" for t, _ in fields) and all(ty is ctypes.c_int32 for _, ty in cls._fields_)
+        assert ctypes.sizeof(cls) == 4 * len(fields)
