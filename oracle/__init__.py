@@ -49,43 +49,41 @@ def _load():
 
 def _declare(lib):
     """Declare the C signatures on a loaded oracle library."""
-    _lib = lib
-    if True:
-        P = ctypes.c_void_p
-        I = ctypes.c_int
-        I64 = ctypes.c_int64
-        F = ctypes.c_float
-        _lib.oracle_f16_to_double.restype = ctypes.c_double
-        _lib.oracle_f16_to_double.argtypes = [ctypes.c_uint16]
-        _lib.oracle_e4m3_to_double.restype = ctypes.c_double
-        _lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
-        _lib.oracle_e4m3_from_float.restype = ctypes.c_uint8
-        _lib.oracle_e4m3_from_float.argtypes = [F]
-        _lib.oracle_slot_mapping.restype = I
-        _lib.oracle_slot_mapping.argtypes = [P, P, I, P, I, I]
-        _lib.oracle_kv_cache_write.restype = I
-        _lib.oracle_kv_cache_write.argtypes = [P, P, I64, I64, P, P, I, I, I, I, I, P, I, F, F]
-        _lib.oracle_copy_blocks.restype = I
-        _lib.oracle_copy_blocks.argtypes = [P, P, I64, I, P, I]
-        _lib.oracle_swap_blocks.restype = I
-        _lib.oracle_swap_blocks.argtypes = [P, P, I, P, P, I, I64, P, I]
-        _lib.oracle_paged_attention.restype = I
-        _lib.oracle_paged_attention.argtypes = [P, P, P, P, I, I, I, I, I, P, I, P, I, F, F, F, P, I]
-        _lib.oracle_attention_partials.restype = I
-        _lib.oracle_attention_partials.argtypes = [P, P, P, P, P, I, I, I, I, I, P, I, P, I, F, F, F, I, I]
-        _lib.oracle_prefill_slot_mapping.restype = I
-        _lib.oracle_prefill_slot_mapping.argtypes = [P, P, P, I, P, I, I]
-        _lib.oracle_paged_prefill.restype = I
-        _lib.oracle_paged_prefill.argtypes = [P, P, P, P, P, I, I, I, I, I, P, I, P, I, F, F, F, P, I]
-        _lib.oracle_lse_combine.restype = None
-        _lib.oracle_lse_combine.argtypes = [P, P, P, I, I]
-        _lib.oracle_f16_array_to_double.restype = None
-        _lib.oracle_f16_array_to_double.argtypes = [P, P, I64]
-        _lib.oracle_e4m3_array_to_double.restype = None
-        _lib.oracle_e4m3_array_to_double.argtypes = [P, P, I64]
-        _lib.oracle_e4m3_array_from_float.restype = None
-        _lib.oracle_e4m3_array_from_float.argtypes = [P, P, I64]
-    return _lib
+    P = ctypes.c_void_p
+    I = ctypes.c_int
+    I64 = ctypes.c_int64
+    F = ctypes.c_float
+    lib.oracle_f16_to_double.restype = ctypes.c_double
+    lib.oracle_f16_to_double.argtypes = [ctypes.c_uint16]
+    lib.oracle_e4m3_to_double.restype = ctypes.c_double
+    lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+    lib.oracle_e4m3_from_float.restype = ctypes.c_uint8
+    lib.oracle_e4m3_from_float.argtypes = [F]
+    lib.oracle_slot_mapping.restype = I
+    lib.oracle_slot_mapping.argtypes = [P, P, I, P, I, I]
+    lib.oracle_kv_cache_write.restype = I
+    lib.oracle_kv_cache_write.argtypes = [P, P, I64, I64, P, P, I, I, I, I, I, P, I, F, F]
+    lib.oracle_copy_blocks.restype = I
+    lib.oracle_copy_blocks.argtypes = [P, P, I64, I, P, I]
+    lib.oracle_swap_blocks.restype = I
+    lib.oracle_swap_blocks.argtypes = [P, P, I, P, P, I, I64, P, I]
+    lib.oracle_paged_attention.restype = I
+    lib.oracle_paged_attention.argtypes = [P, P, P, P, I, I, I, I, I, P, I, P, I, F, F, F, P, I]
+    lib.oracle_attention_partials.restype = I
+    lib.oracle_attention_partials.argtypes = [P, P, P, P, P, I, I, I, I, I, P, I, P, I, F, F, F, I, I]
+    lib.oracle_prefill_slot_mapping.restype = I
+    lib.oracle_prefill_slot_mapping.argtypes = [P, P, P, I, P, I, I]
+    lib.oracle_paged_prefill.restype = I
+    lib.oracle_paged_prefill.argtypes = [P, P, P, P, P, I, I, I, I, I, P, I, P, I, F, F, F, P, I]
+    lib.oracle_lse_combine.restype = None
+    lib.oracle_lse_combine.argtypes = [P, P, P, I, I]
+    lib.oracle_f16_array_to_double.restype = None
+    lib.oracle_f16_array_to_double.argtypes = [P, P, I64]
+    lib.oracle_e4m3_array_to_double.restype = None
+    lib.oracle_e4m3_array_to_double.argtypes = [P, P, I64]
+    lib.oracle_e4m3_array_from_float.restype = None
+    lib.oracle_e4m3_array_from_float.argtypes = [P, P, I64]
+    return lib
 
 
 class using_library:
