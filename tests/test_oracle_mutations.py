@@ -18,7 +18,6 @@ must fail at least one pin; the unmodified source must pass all of them.
 import math
 import os
 import subprocess
-import tempfile
 
 import numpy as np
 import pytest

@@ -13,7 +13,6 @@ tolerance of the parity tests), the clear rejection of a batch whose
 partials exceed the static scratch, and the torch binding giving the C
 call's result bit for bit.
 """
-import ctypes
 
 import numpy as np
 import pytest
