@@ -30,11 +30,12 @@ _lib = None
 
 
 def build(force: bool = False) -> str:
-    """Compile the oracle with gcc (no fast-math, no FMA contraction)."""
+    """Compile the oracle with gcc (no fast-math, no FMA contraction; OpenMP
+    only spreads independent (sequence, head) pairs over threads)."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + f".tmp{os.getpid()}"
         subprocess.check_call(
-            ["gcc", "-O2", "-std=c11", "-fno-fast-math", "-ffp-contract=off",
+            ["gcc", "-O2", "-std=c11", "-fno-fast-math", "-ffp-contract=off", "-fopenmp",
              "-Wall", "-shared", "-fPIC", _SRC, "-o", tmp, "-lm"])
         os.replace(tmp, _LIB)
     return _LIB
@@ -69,6 +70,10 @@ def _declare(lib):
     lib.oracle_swap_blocks.argtypes = [P, P, I, P, P, I, I64, P, I]
     lib.oracle_paged_attention.restype = I
     lib.oracle_paged_attention.argtypes = [P, P, P, P, I, I, I, I, I, P, I, P, I, F, F, F, P, I]
+    lib.oracle_paged_attention_threads.restype = I
+    lib.oracle_paged_attention_threads.argtypes = [P, P, P, P, I, I, I, I, I, P, I, P, I, F, F, F, P, I, I]
+    lib.oracle_max_threads.restype = I
+    lib.oracle_max_threads.argtypes = []
     lib.oracle_attention_partials.restype = I
     lib.oracle_attention_partials.argtypes = [P, P, P, P, P, I, I, I, I, I, P, I, P, I, F, F, F, I, I]
     lib.oracle_prefill_slot_mapping.restype = I
@@ -208,11 +213,19 @@ def swap_blocks(dst_key: np.ndarray, dst_value: np.ndarray, src_key: np.ndarray,
                                       src_key[0].nbytes, _ptr(pairs), pairs.shape[0]), "swap_blocks")
 
 
+def max_threads() -> int:
+    """Threads the oracle's threaded calls use by default on this host."""
+    return int(_load().oracle_max_threads())
+
+
 def paged_attention(query: np.ndarray, key_cache: np.ndarray, value_cache: np.ndarray,
                     block_tables: np.ndarray, context_lens: np.ndarray, scale: float,
                     k_scale: float = 1.0, v_scale: float = 1.0,
-                    seq_head: np.ndarray | None = None) -> np.ndarray:
-    """Returns float64 [S, H, D], or [n, D] for an explicit (s, h) list."""
+                    seq_head: np.ndarray | None = None, threads: int | None = None) -> np.ndarray:
+    """Returns float64 [S, H, D], or [n, D] for an explicit (s, h) list.
+    threads=None runs on the calling thread; threads=n (0: the host's
+    default) spreads the (s, h) pairs over n OpenMP threads, each pair
+    computed by the same code, so the result is the same bit for bit."""
     assert query.dtype == np.float16
     q = np.ascontiguousarray(query)
     nb, bs, nh, hd = key_cache.shape
@@ -222,11 +235,14 @@ def paged_attention(query: np.ndarray, key_cache: np.ndarray, value_cache: np.nd
     pairs = None if seq_head is None else np.ascontiguousarray(seq_head, dtype=np.int32).reshape(-1, 2)
     n = S * nh if pairs is None else pairs.shape[0]
     out = np.empty((n, hd), np.float64)
-    rc = _load().oracle_paged_attention(
-        _ptr(out), _ptr(q.view(np.uint16)), _ptr(key_cache), _ptr(value_cache),
-        _dtype_code(key_cache), nb, bs, nh, hd, _ptr(bt), bt.shape[1], _ptr(ctx), S,
-        float(np.float32(scale)), float(np.float32(k_scale)), float(np.float32(v_scale)),
-        _ptr(pairs), 0 if pairs is None else pairs.shape[0])
+    args = (_ptr(out), _ptr(q.view(np.uint16)), _ptr(key_cache), _ptr(value_cache),
+            _dtype_code(key_cache), nb, bs, nh, hd, _ptr(bt), bt.shape[1], _ptr(ctx), S,
+            float(np.float32(scale)), float(np.float32(k_scale)), float(np.float32(v_scale)),
+            _ptr(pairs), 0 if pairs is None else pairs.shape[0])
+    if threads is None:
+        rc = _load().oracle_paged_attention(*args)
+    else:
+        rc = _load().oracle_paged_attention_threads(*args, int(threads))
     _check(rc, "paged_attention")
     return out.reshape(S, nh, hd) if pairs is None else out
 

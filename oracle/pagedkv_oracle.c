@@ -9,6 +9,9 @@
  *
  * Every floating-point result is computed in double precision with no
  * blocking, fusion or reordering beyond what the definitions below state.
+ * The one parallel entry, oracle_paged_attention_threads, only hands whole
+ * (sequence, head) pairs to OpenMP threads; each pair runs the same serial
+ * code, so its results equal the single-thread call's bit for bit.
  * Sources (each page is cited by its title and section):
  *   [P1] "vLLM-v0.17.1技术解析：PagedAttention内存管理与显存优化技巧"
  *        (cnnetsun.cn/a/1550967), §2.2 PagedAttention的创新设计: block table +
@@ -37,6 +40,9 @@
  * decode slots, and torch's SDPA with a causal / position mask.
  */
 #include <math.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -342,10 +348,42 @@ static int attend_range(double *o, double *m_out, double *l_out,
     return 0;
 }
 
+/* Decode attention of pair i: (s, h) = seq_head[i] when seq_head is given,
+ * else (i / num_heads, i % num_heads). Writes head_size doubles at
+ * out + i*head_size. A sequence with context length 0 gives a zero row.
+ * Returns 0, or -1 on a pair out of range or a bad table entry. */
+static int attend_pair(int i, double *out, const uint16_t *query,
+                       const void *key_cache, const void *value_cache,
+                       int kv_dtype, int num_blocks, int block_size,
+                       int num_heads, int head_size,
+                       const int32_t *block_tables, int max_blocks_per_seq,
+                       const int32_t *context_lens, int num_seqs,
+                       float scale, float k_scale, float v_scale,
+                       const int32_t *seq_head)
+{
+    int s = seq_head ? seq_head[2 * i] : i / num_heads;
+    int h = seq_head ? seq_head[2 * i + 1] : i % num_heads;
+    double *o = out + (int64_t)i * head_size;
+    if (s < 0 || s >= num_seqs || h < 0 || h >= num_heads)
+        return -1;
+    int L = context_lens[s];
+    if (L <= 0) {
+        for (int d = 0; d < head_size; ++d)
+            o[d] = 0.0;
+        return 0;
+    }
+    const uint16_t *q = query + ((int64_t)s * num_heads + h) * head_size;
+    double m, l;
+    return attend_range(o, &m, &l, q, key_cache, value_cache, kv_dtype,
+                        num_blocks, block_size, num_heads, head_size,
+                        block_tables, max_blocks_per_seq, s, h, 0, L,
+                        (double)scale, (double)k_scale, (double)v_scale);
+}
+
 /* Decode attention for the (sequence, head) pairs listed in seq_head
  * ([n_pairs][2]), or for every pair in (s, h) order when seq_head is NULL.
- * out holds one head_size row of doubles per computed pair. A sequence with
- * context length 0 gives a zero row. Returns 0, or -1 on a bad table entry. */
+ * out holds one head_size row of doubles per computed pair. Returns 0, or
+ * -1 on a bad pair or table entry. */
 int oracle_paged_attention(double *out, const uint16_t *query,
                            const void *key_cache, const void *value_cache,
                            int kv_dtype, int num_blocks, int block_size,
@@ -357,27 +395,58 @@ int oracle_paged_attention(double *out, const uint16_t *query,
 {
     int total = seq_head ? n_pairs : num_seqs * num_heads;
     for (int i = 0; i < total; ++i) {
-        int s = seq_head ? seq_head[2 * i] : i / num_heads;
-        int h = seq_head ? seq_head[2 * i + 1] : i % num_heads;
-        double *o = out + (int64_t)i * head_size;
-        if (s < 0 || s >= num_seqs || h < 0 || h >= num_heads)
-            return -1;
-        int L = context_lens[s];
-        if (L <= 0) {
-            for (int d = 0; d < head_size; ++d)
-                o[d] = 0.0;
-            continue;
-        }
-        const uint16_t *q = query + ((int64_t)s * num_heads + h) * head_size;
-        double m, l;
-        int rc = attend_range(o, &m, &l, q, key_cache, value_cache, kv_dtype,
-                              num_blocks, block_size, num_heads, head_size,
-                              block_tables, max_blocks_per_seq, s, h, 0, L,
-                              (double)scale, (double)k_scale, (double)v_scale);
+        int rc = attend_pair(i, out, query, key_cache, value_cache, kv_dtype,
+                             num_blocks, block_size, num_heads, head_size,
+                             block_tables, max_blocks_per_seq, context_lens,
+                             num_seqs, scale, k_scale, v_scale, seq_head);
         if (rc)
             return rc;
     }
     return 0;
+}
+
+/* Threads an OpenMP region of this library uses by default (1 in a build
+ * without OpenMP, where the threaded call below runs on the calling thread). */
+int oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* The same computation with the (sequence, head) pairs spread over
+ * n_threads OpenMP threads (n_threads <= 0: the OpenMP default). Pairs are
+ * independent and each is computed by the same attend_pair as above, so the
+ * result is identical, bit for bit, to oracle_paged_attention's. Returns 0,
+ * or the first nonzero status of any pair (a bad pair or table entry). */
+int oracle_paged_attention_threads(double *out, const uint16_t *query,
+                                   const void *key_cache, const void *value_cache,
+                                   int kv_dtype, int num_blocks, int block_size,
+                                   int num_heads, int head_size,
+                                   const int32_t *block_tables, int max_blocks_per_seq,
+                                   const int32_t *context_lens, int num_seqs,
+                                   float scale, float k_scale, float v_scale,
+                                   const int32_t *seq_head, int n_pairs, int n_threads)
+{
+    int total = seq_head ? n_pairs : num_seqs * num_heads;
+    int status = 0;
+    if (n_threads <= 0)
+        n_threads = oracle_max_threads();
+#pragma omp parallel for schedule(dynamic, 1) num_threads(n_threads)
+    for (int i = 0; i < total; ++i) {
+        int rc = attend_pair(i, out, query, key_cache, value_cache, kv_dtype,
+                             num_blocks, block_size, num_heads, head_size,
+                             block_tables, max_blocks_per_seq, context_lens,
+                             num_seqs, scale, k_scale, v_scale, seq_head);
+        if (rc) {
+#pragma omp critical
+            if (status == 0)
+                status = rc;
+        }
+    }
+    return status;
 }
 
 /* --------------------------------------------------------- paged prefill */
