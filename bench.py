@@ -10,7 +10,13 @@ buffer is written and then read back, which evicts the 126 MB L2 without
 leaving dirty lines whose write-back would land in the timed step, so the KV
 bytes come from HBM.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 1..5] [--impl ours|reference]
+By default one run times the decode workloads 3, 2, 4 and 5 in turn. The
+JSON line's top level is the first of them (the Llama2-13B-shaped
+mixed-length batch); the others sit under "workloads", each with its own
+roofline, end-to-end figure, clocks and CPU baseline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 1..5 | --workloads 3,2,4,5]
+                    [--impl ours|reference]
     python bench.py --prefill 1..3      (paged prefill: TFLOP/s against the tensor peak)
 
 Under torchrun each rank runs its own independently seeded batch of the same
@@ -198,20 +204,52 @@ def aggregate_gbs(world: int, bytes_per_rank: int, ms: float) -> float:
     return world * bytes_per_rank / (ms * 1e-3) / 1e9
 
 
-def run_ours(args, rank, world, local_rank):
+HEADLINE_WORKLOAD = 3
+DEFAULT_WORKLOADS = "3,2,4,5"   # headline first; the others are reported beside it
+
+
+def decode_arithmetic(w) -> str:
+    """The arithmetic the decode kernel does for this cache type."""
+    return ("fp32 sums of exact products of the fp16 query with keys decoded exactly from E4M3 "
+            "codes to fp16; softmax weights rounded to fp16 for the exact products with the "
+            "decoded values, summed in fp32" if w.kv_dtype == "e4m3" else
+            "fp32 sums of exact fp16 x fp16 products (query x key); softmax weights rounded to "
+            "fp16 for the exact products with the values, summed in fp32")
+
+
+def empty_graph_ms(torch, stream, steps: int) -> float:
+    """Floor of the event timing: one tiny kernel captured in a graph between
+    two timing events, replayed like a step (mean over `steps` replays)."""
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+    x = torch.zeros(1, dtype=torch.int32, device=stream.device)
+    with torch.cuda.stream(stream):
+        x.add_(1)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            ev[0].record()
+            x.add_(1)
+            ev[1].record()
+        ts = []
+        for i in range(3 + steps):
+            g.replay()
+            stream.synchronize()
+            if i >= 3:
+                ts.append(ev[0].elapsed_time(ev[1]))
+    del g
+    return statistics.mean(ts)
+
+
+def measure_decode(args, wid, rank, world, local_rank, dist, cpu_seconds, with_swap):
+    """One decode workload: build, capture the step in a CUDA graph, time it
+    (and its end-to-end form from pinned host buffers), and return the
+    result dict on rank 0 (None elsewhere). Every rank takes the same
+    collective steps in the same order."""
     import torch
     import pagedattention_paged_kv_decode_b200 as pk
 
     dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
-
-    w = W.named(args.workload, seed=W.rank_seed(1000 + args.workload, rank))
+    w = W.named(wid, seed=W.rank_seed(1000 + wid, rank))
     dw = W.to_device(w, dev, encode=pk.load_cache)
     S = w.num_seqs
     bound = w.max_blocks_per_seq * w.block_size  # host-side bound: table capacity, no sync
@@ -331,36 +369,49 @@ def run_ours(args, rank, world, local_rank):
                 e2e_ms.append(e2e_start.elapsed_time(e2e_end))
 
         # ------------------------------------------------ swap to/from pinned host memory
-        swap = measure_swap(pk, dw, stream, torch)
+        swap = measure_swap(pk, dw, stream, torch) if with_swap else None
+        floor = empty_graph_ms(torch, stream, max(20, args.steps))
 
-    step_t, dec_t, e2e_t = slowest_rank([statistics.mean(step_ms), statistics.mean(dec_ms),
-                                         statistics.mean(e2e_ms)], dist, dev)
+    step_t, dec_t, e2e_t, floor_t = slowest_rank([statistics.mean(step_ms), statistics.mean(dec_ms),
+                                                  statistics.mean(e2e_ms), floor], dist, dev)
     clocks = sampler.summary(t0, t1)
     del graph
-    if dist:
-        dist.destroy_process_group()
+    del dw, flush, packed
+    torch.cuda.empty_cache()
     if rank != 0:
-        return
+        return None
 
     kv = w.kv_bytes()
     peak, peak_kind = hbm_peak()
     dec_bytes = w.decode_bytes() if args.unfused else W.fused_step_bytes(w)
     achieved = dec_bytes / (dec_t * 1e-3) / 1e9
     value = aggregate_gbs(world, kv, step_t)
-    line = {
+    roofline = {
+        "bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+        "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} copy bandwidth",
+        "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
+        "traffic": recorded_traffic(w.name),
+        "kernel": ("paged_prefix_kernel + paged_decode_kernel (fused append) + lse_reduce_kernel"
+                   if shared else "paged_decode_kernel" + ("" if args.unfused else " (fused append)")
+                   + (" + lse_reduce_kernel" if parts > 1 else "")),
+        "algorithmic_bytes_per_launch": dec_bytes,
+    }
+    if w.shared_blocks:
+        uniq = dec_bytes - kv + w.unique_kv_bytes()
+        roofline.update(
+            unique_bytes_per_launch=uniq,
+            unique_achieved=round(uniq / (dec_t * 1e-3) / 1e9, 2),
+            unique_frac=round(uniq / (dec_t * 1e-3) / 1e9 / peak, 4),
+            note="algorithmic bytes count the shared prefix once per sequence (logical); the unique "
+                 "figures count each distinct cache row once")
+    res = {
         "metric": METRIC,
         "value": round(value, 2),
         "unit": "GB/s",
-        "n_gpus": world,
-        "steps": args.steps,
-        "warmup": args.warmup,
         "ms_per_step": round(step_t, 5),
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
         "dtype": "f32",
+        "arithmetic": decode_arithmetic(w),
         "kv_dtype": w.kv_dtype,
-        "data": "synthetic (seeded numpy PCG64; no dataset)",
         "config": {
             "workload": w.name, "num_seqs": S, "num_heads": w.num_heads,
             "head_size": w.head_size, "block_size": w.block_size, "kv_dtype": w.kv_dtype,
@@ -382,25 +433,61 @@ def run_ours(args, rank, world, local_rank):
         "hbm_pct_of_measured": round(100 * value / world / peak, 2),
         "decode_ms": round(dec_t, 5),
         "decode_kv_gbs": round(kv / (dec_t * 1e-3) / 1e9, 2),
-        "roofline": {
-            "bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
-            "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} copy bandwidth",
-            "traffic": recorded_traffic(w.name),
-            "kernel": ("paged_prefix_kernel + paged_decode_kernel (fused append) + lse_reduce_kernel"
-                       if shared else "paged_decode_kernel" + ("" if args.unfused else " (fused append)")
-                       + (" + lse_reduce_kernel" if parts > 1 else "")),
-            "algorithmic_bytes_per_launch": dec_bytes,
-        },
+        "empty_graph_ms": round(floor_t, 5),
+        "roofline": roofline,
         "e2e": {"value": round(aggregate_gbs(world, kv, e2e_t), 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_t, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "path": "pinned host inputs (one packed buffer) -> one copy to the device -> graph replay -> "
                         "output to pinned host"},
         "gpu_launches": launches_per_step * args.steps,
-        "swap_blocks": swap,
         "clocks": clocks,
     }
+    if swap is not None:
+        res["swap_blocks"] = swap
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+        res["cpu_baseline"] = cpu_baseline_both(w, cpu_seconds)
+    return res
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    ids = [args.workload] if args.workload else [int(x) for x in args.workloads.split(",")]
+    results = []
+    for i, wid in enumerate(ids):
+        secs = args.cpu_seconds if i == 0 else max(1.0, args.cpu_seconds / 3)
+        results.append(measure_decode(args, wid, rank, world, local_rank, dist, secs, with_swap=(i == 0)))
+    if dist:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    head = results[0]
+    line = {
+        "metric": METRIC,
+        "value": head["value"],
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "data": "synthetic (seeded numpy PCG64; no dataset)",
+    }
+    line.update({k: v for k, v in head.items() if k not in line})
+    if len(results) > 1:
+        line["workloads"] = {r["config"]["workload"]: {k: v for k, v in r.items() if k != "metric"}
+                             for r in results[1:]}
+        line["gpu_launches_all_workloads"] = sum(r["gpu_launches"] for r in results)
     print(json.dumps(line), flush=True)
 
 
@@ -451,45 +538,80 @@ class OracleState:
             self.encoded = None
 
 
-def cpu_baseline(w, seconds: float, state: "OracleState | None" = None, start: int = 0):
-    """The oracle, single-threaded, on this host: whole decode steps of one
-    sequence at a time (all heads) over a bounded, seeded sample of the
-    workload's sequences (at least one). Building the host pools (and, for
-    E4M3, encoding the sampled sequences' blocks) happens outside the timed
-    region. Returns the same GB/s metric."""
+def _encode_blocks(w, state: "OracleState", seqs) -> None:
+    """E4M3 pools: encode (with the oracle's cache write) the blocks of the
+    given sequences that are not encoded yet. Outside every timed region."""
+    import oracle
+    if w.kv_dtype != "e4m3":
+        return
+    bt = w.block_tables[np.asarray(seqs)]
+    blocks = np.unique(bt[bt >= 0])
+    blocks = blocks[~state.encoded[blocks]].astype(np.int64)
+    if blocks.size:
+        slots = (blocks[:, None] * w.block_size + np.arange(w.block_size)).reshape(-1).astype(np.int32)
+        oracle.kv_cache_write(state.pk[blocks].reshape(-1, w.num_heads, w.head_size),
+                              state.pv[blocks].reshape(-1, w.num_heads, w.head_size), state.kc, state.vc,
+                              slots, w.k_scale, w.v_scale)
+        state.encoded[blocks] = True
+
+
+def _oracle_steps(w, state: "OracleState", seqs, threads) -> None:
+    """The oracle's decode step for the given sequences (all heads each):
+    copy-on-write pairs, slots, cache write, attention."""
+    import oracle
+    seqs = np.asarray(seqs)
+    kc, vc, ctx = state.kc, state.vc, w.context_lens
+    if w.cow_pairs.size:
+        oracle.copy_blocks(kc, vc, w.cow_pairs[seqs])
+    slot = oracle.slot_mapping(w.block_tables[seqs], ctx[seqs], w.block_size)
+    oracle.kv_cache_write(w.new_key[seqs], w.new_value[seqs], kc, vc, slot, w.k_scale, w.v_scale)
+    pairs = np.stack([np.repeat(seqs, w.num_heads), np.tile(np.arange(w.num_heads), seqs.size)],
+                     1).astype(np.int32)
+    oracle.paged_attention(w.query, kc, vc, w.block_tables, ctx, w.scale, w.k_scale, w.v_scale,
+                           seq_head=pairs, threads=threads)
+
+
+def cpu_baseline(w, seconds: float, state: "OracleState | None" = None, start: int = 0,
+                 threads: int | None = None):
+    """The oracle on this host: whole decode steps of a bounded, seeded sample
+    of the workload's sequences (all heads of each; at least one call).
+    threads=None: one sequence per call on one thread. threads=n (0: every
+    core): calls of enough sequences to give each thread two (sequence,
+    head) pairs, spread over n OpenMP threads. Building the host pools (and,
+    for E4M3, encoding the sampled sequences' blocks) happens outside the
+    timed region. Returns the same GB/s metric."""
     import oracle
     order = np.random.default_rng(0).permutation(w.num_seqs)
     state = state or OracleState(w)
-    pk_, pv_, kc, vc, encoded = state.pk, state.pv, state.kc, state.vc, state.encoded
-    ctx = w.context_lens
-    done_bytes, elapsed, n = 0, 0.0, 0
-    while elapsed < seconds and n < 100000:
-        s = int(order[(start + n) % w.num_seqs])
-        if w.kv_dtype == "e4m3":
-            bt = w.block_tables[s]
-            blocks = np.array([b for b in bt[bt >= 0] if not encoded[b]], np.int64)
-            if blocks.size:
-                slots = (blocks[:, None] * w.block_size + np.arange(w.block_size)).reshape(-1).astype(np.int32)
-                oracle.kv_cache_write(pk_[blocks].reshape(-1, w.num_heads, w.head_size),
-                                      pv_[blocks].reshape(-1, w.num_heads, w.head_size), kc, vc,
-                                      slots, w.k_scale, w.v_scale)
-                encoded[blocks] = True
+    cores = 1 if threads is None else (threads or oracle.max_threads())
+    per_call = 1 if threads is None else max(1, -(-2 * cores // w.num_heads))
+    done_bytes, elapsed, n, calls = 0, 0.0, 0, 0
+    while elapsed < seconds and calls < 100000:
+        seqs = [int(order[(start + n + k) % w.num_seqs]) for k in range(per_call)]
+        _encode_blocks(w, state, seqs)
         t = time.perf_counter()
-        if w.cow_pairs.size:
-            oracle.copy_blocks(kc, vc, w.cow_pairs[s:s + 1])
-        slot = oracle.slot_mapping(w.block_tables[s:s + 1], ctx[s:s + 1], w.block_size)
-        oracle.kv_cache_write(w.new_key[s:s + 1], w.new_value[s:s + 1], kc, vc, slot,
-                              w.k_scale, w.v_scale)
-        oracle.paged_attention(w.query[s:s + 1], kc, vc, w.block_tables[s:s + 1], ctx[s:s + 1],
-                               w.scale, w.k_scale, w.v_scale)
+        _oracle_steps(w, state, seqs, threads)
         elapsed += time.perf_counter() - t
-        done_bytes += int(ctx[s]) * w.num_heads * w.head_size * w.elem_bytes * 2
-        n += 1
-    return {"value": round(done_bytes / elapsed / 1e9, 4), "unit": "GB/s", "cores": 1,
+        done_bytes += sum(int(w.context_lens[s]) for s in seqs) * w.num_heads * w.head_size * w.elem_bytes * 2
+        n += per_call
+        calls += 1
+    how = ("single-thread fp64" if threads is None else
+           f"fp64, (sequence, head) pairs over {cores} OpenMP threads, {per_call} sequences per call")
+    return {"value": round(done_bytes / elapsed / 1e9, 4), "unit": "GB/s", "cores": cores,
             "kind": "oracle",
             "sample": f"{n} sequences (all {w.num_heads} heads each) of {w.name}, one decode step "
-                      f"each (copy-on-write, slot, cache write, attention): {elapsed:.1f} s, "
-                      f"single-thread fp64"}
+                      f"each (copy-on-write, slot, cache write, attention): {elapsed:.1f} s, {how}"}
+
+
+def cpu_baseline_both(w, seconds: float) -> dict:
+    """The multi-core oracle (every host core) as the baseline, with the
+    single-thread figure beside it; each leg takes about `seconds`."""
+    state = OracleState(w)
+    single = cpu_baseline(w, seconds, state)
+    multi = cpu_baseline(w, seconds, state, threads=0)
+    multi["single_thread"] = {k: single[k] for k in ("value", "cores", "sample")}
+    multi["host_cpu_count"] = os.cpu_count()
+    return multi
 
 
 # ------------------------------------------------------------ paged prefill
@@ -697,12 +819,13 @@ def run_reference(args, rank, world):
     if args.prefill:
         run_reference_prefill(args, world)
         return
-    w = W.named(args.workload)
+    w = W.named(args.workload or int(args.workloads.split(",")[0]))
     per_step = args.cpu_seconds / max(1, args.steps + args.warmup)
     state = OracleState(w)
-    vals = []
+    vals, cores = [], 1
     for i in range(args.warmup + args.steps):
-        r = cpu_baseline(w, per_step, state, start=i)
+        r = cpu_baseline(w, per_step, state, start=i, threads=0)
+        cores = r["cores"]
         if i >= args.warmup:
             vals.append(r["value"])
     v = statistics.mean(vals)
@@ -714,9 +837,9 @@ def run_reference(args, rank, world):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded numpy PCG64; no dataset)",
         "config": {"workload": w.name, "num_seqs": w.num_seqs, "num_heads": w.num_heads,
                    "head_size": w.head_size, "block_size": w.block_size, "kv_dtype": w.kv_dtype},
-        "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": f"each step: {per_step:.3f} s (at least one sequence) of whole-sequence "
-                                   "oracle steps, single-thread fp64"},
+        "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: {per_step:.3f} s (at least one call) of whole-sequence "
+                                   f"oracle steps, fp64, (sequence, head) pairs over {cores} OpenMP threads"},
         "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -751,7 +874,10 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--workload", type=int, default=0, choices=[0, 1, 2, 3, 4, 5],
+                    help="time one decode workload only (default: the --workloads list)")
+    ap.add_argument("--workloads", default=DEFAULT_WORKLOADS,
+                    help="decode workloads timed in one run; the first is the headline")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

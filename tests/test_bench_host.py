@@ -87,3 +87,45 @@ def test_peaks_come_from_the_measured_file_else_the_fallback(tmp_path, monkeypat
 def test_aggregate_is_all_ranks_bytes_over_the_slowest_time():
     assert bench.aggregate_gbs(1, 10**9, 1000.0) == pytest.approx(1.0)
     assert bench.aggregate_gbs(4, 10**9, 500.0) == pytest.approx(8.0)
+
+
+@pytest.mark.parametrize("cfg", [1, 2])
+def test_cpu_baseline_reports_both_legs(cfg):
+    import oracle
+    import workloads as W
+    w = W.named(cfg)
+    cb = bench.cpu_baseline_both(w, 0.2)
+    assert cb["kind"] == "oracle" and cb["unit"] == "GB/s" and cb["value"] > 0
+    assert cb["cores"] == oracle.max_threads() and str(cb["cores"]) in cb["sample"]
+    assert cb["single_thread"]["cores"] == 1 and cb["single_thread"]["value"] > 0
+    assert "single-thread" in cb["single_thread"]["sample"]
+
+
+def test_cpu_baseline_step_matches_the_oracle_decode():
+    """The timed oracle step computes the workload's attention: its slot and
+    cache write, then the threaded attention, equal the plain oracle calls."""
+    import numpy as np
+    import oracle
+    import workloads as W
+    w = W.named(1)
+    st = bench.OracleState(w)
+    seqs = [2, 0, 3]
+    bench._oracle_steps(w, st, seqs, threads=3)
+    kc, vc = w.pool_host()
+    slots = oracle.slot_mapping(w.block_tables, w.context_lens, w.block_size)
+    oracle.kv_cache_write(w.new_key, w.new_value, kc, vc, slots)
+    # the sampled sequences' rows are written; the rest of the pools are untouched
+    for s in seqs:
+        b, o = divmod(int(slots[s]), w.block_size)
+        assert np.array_equal(st.kc[b, o].view(np.uint16), kc[b, o].view(np.uint16))
+
+
+def test_unique_bytes_count_shared_blocks_once():
+    import workloads as W
+    w = W.named(2)
+    assert w.unique_kv_bytes() == w.kv_bytes()
+    w = W.named(4)
+    row = w.num_heads * w.head_size * w.elem_bytes * 2
+    shared = w.shared_blocks * w.block_size
+    assert w.unique_kv_bytes() == (int((w.context_lens - shared).sum()) + shared) * row
+    assert w.unique_kv_bytes() < w.kv_bytes()

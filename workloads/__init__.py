@@ -109,6 +109,14 @@ class Workload(_Pools):
         """Logical K+V bytes the decode reads: sum_s L_s * H * D * elem * 2."""
         return int(self.context_lens.astype(np.int64).sum()) * self.num_heads * self.head_size * self.elem_bytes * 2
 
+    def unique_kv_bytes(self) -> int:
+        """K+V bytes of distinct cache rows the decode reads: the leading
+        shared_blocks blocks, which every table row points at, count once."""
+        shared = self.shared_blocks * self.block_size
+        L = self.context_lens.astype(np.int64)
+        tokens = int(np.maximum(L - shared, 0).sum()) + (shared if (L > 0).any() else 0)
+        return tokens * self.num_heads * self.head_size * self.elem_bytes * 2
+
     def decode_bytes(self) -> int:
         """Algorithmic bytes of one decode: K/V + query + output + block-table entries + lengths."""
         S, H, D, B = self.num_seqs, self.num_heads, self.head_size, self.block_size
