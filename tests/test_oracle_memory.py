@@ -37,7 +37,7 @@ MEMORY_MUTANTS = {
         "        for (int i = 0; i < n; ++i)\n            acc += exp(z[i] - m) * cache_value",
         "d < head_size", "d <= head_size"),
     "empty-context zero fill one past the row": (
-        "        if (L <= 0) {\n            for (int d = 0; d < head_size; ++d)\n                o[d] = 0.0;",
+        "    if (L <= 0) {\n        for (int d = 0; d < head_size; ++d)\n            o[d] = 0.0;",
         "d < head_size", "d <= head_size"),
     "unused-partition fill one past the row": (
         "                if (p >= nparts) {\n                    for (int d = 0; d < head_size; ++d)",

@@ -74,8 +74,8 @@ MUTANTS = {
                                  "return oracle_e4m3_to_double(((const uint8_t *)cache)[idx]);"),
     "empty context gets a slot": ("if (L <= 0) {\n            slot_mapping[s] = -1;",
                                   "if (L < 0) {\n            slot_mapping[s] = -1;"),
-    "empty context attends over nothing": ("if (L <= 0) {\n            for (int d = 0; d < head_size; ++d)\n                o[d] = 0.0;",
-                                           "if (L < 0) {\n            for (int d = 0; d < head_size; ++d)\n                o[d] = 0.0;"),
+    "empty context attends over nothing": ("if (L <= 0) {\n        for (int d = 0; d < head_size; ++d)\n            o[d] = 0.0;",
+                                           "if (L < 0) {\n        for (int d = 0; d < head_size; ++d)\n            o[d] = 0.0;"),
     "head index ignored": ("const uint16_t *q = query + ((int64_t)s * num_heads + h) * head_size;",
                            "const uint16_t *q = query + ((int64_t)s * num_heads + 0) * head_size;"),
 }
