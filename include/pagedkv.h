@@ -102,8 +102,10 @@ typedef struct {
     int32_t units_per_cta;
 } pa_decode_config;
 
-/* Library version: 100 * minor + patch for 0.minor.patch (201 = 0.2.1: the
- * paged prefill calls, which take total_q since 0.2.1). */
+/* Library version: 100 * minor + patch for 0.minor.patch (202 = 0.2.2: the
+ * paged prefill calls take total_q since 0.2.1; the decode sums exact
+ * fp16 products in fp32 for both cache types, and pa_test_stall_next_decode
+ * exists, since 0.2.2). */
 int pa_version(void);
 
 /* Message for the last nonzero status returned on this thread ("" if none). */
@@ -113,6 +115,21 @@ const char *pa_last_error(void);
  * current device into *code (0 = no device-side error since the last read).
  * Returns PA_OK or PA_ERR_CUDA. */
 int pa_check_status(void *stream, uint32_t *code);
+
+/* Test hook for the bounded on-chip waits (the pages have no counterpart:
+ * it exists so that a test can make one wait run out on purpose). The next
+ * decode this thread launches (pa_paged_attention_decode, _ws, _append,
+ * _shared_prefix or _noalloc) issues no tile loads for its work unit `unit`
+ * and gives each of its pipeline waits wait_limit_ns of wall time instead
+ * of 2 s. Units are numbered with the context partition fastest, then the
+ * head group, then the sequence; unit 0 is partition 0 of heads
+ * 0..heads_per_cta-1 of sequence 0. The consumer warps of that unit give
+ * up at the limit, set PA_DEV_WAIT_TIMEOUT and return; the output rows of
+ * that unit are then undefined, everything else is computed as usual, and
+ * no copy or wait is left pending. Later launches are unaffected.
+ * unit < 0 clears a pending request. Returns PA_OK, or PA_ERR_INVALID for
+ * wait_limit_ns outside [1000, 2000000000]. */
+int pa_test_stall_next_decode(int64_t unit, uint64_t wait_limit_ns);
 
 /* ---------------------------------------------------------------- a1
  * Slot of the token each sequence appends in a decode step ([P3] §2.2 slot
@@ -178,13 +195,12 @@ int pa_swap_blocks(void *dst_key_cache, void *dst_value_cache, int dst_num_block
  *     out[s,h,:] = v_scale * sum_t softmax(z)_t * V_t[h,:]       (t < L)
  * (k_scale, v_scale only for E4M3 caches, which hold K/k_scale, V/v_scale).
  * L = 0 gives zeros. query, out: fp16 [num_seqs][num_heads][head_size].
- * Range of the E4M3 path: the products of q * scale * log2(e) (rounded to
- * fp16) with the decoded codes (|code| <= 448) are summed in fp16 over 8
- * elements before k_scale is applied, so |q * scale| per element must stay
- * below about 12.7 for no partial sum to overflow when every code is +-448
- * with one sign (queries of trained models are orders of magnitude below;
- * the P.V sums, with weights <= 1, cannot overflow). fp16 caches compute in
- * fp32 and have no such limit.
+ * Arithmetic: each product q*K and p*V is formed exactly (fp16 x fp16, the
+ * query as given, K/V as stored: fp16, or E4M3 codes decoded exactly) and
+ * summed in fp32; the scales are applied to the fp32 sums. Softmax weights
+ * are rounded to fp16 (relative error <= 2^-12) and the same rounded
+ * weights form both the numerator and the denominator, so each output row
+ * is a convex combination of V rows. No input range limit beyond fp32's.
  * max_context_len: a host-known upper bound on every context length (e.g.
  * max_blocks_per_seq*block_size); it sizes the split-context grid. Contexts
  * above it or above the table row are clamped and flagged.

@@ -29,5 +29,6 @@ from .ops import (  # noqa: F401
     shared_prefix_workspace_size,
     slot_mapping,
     swap_blocks,
+    test_stall_next_decode,
     version,
 )

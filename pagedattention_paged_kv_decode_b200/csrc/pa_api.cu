@@ -247,9 +247,11 @@ size_t ws_bytes(const pa_cache_desc &c, int S, int max_ctx, const pa_decode_conf
 using DecodeKernel = void (*)(const CUtensorMap, const CUtensorMap, const pa::DecodeParams);
 using ReduceKernel = void (*)(const pa::DecodeParams);
 
-DecodeKernel pick_decode(int D, int B, bool fp8) {
-#define PA_PICK(d, b, f) \
-    if (D == d && B == b && fp8 == f) return pa::paged_decode_kernel<d, b, f>;
+DecodeKernel pick_decode(int D, int B, bool fp8, bool narrow = false) {
+#define PA_PICK(d, b, f)                                                                      \
+    if (D == d && B == b && fp8 == f)                                                         \
+        return narrow ? pa::paged_decode_kernel<d, b, f, pa::kNarrowDecodeThreads, pa::kNarrowDecodeCtas> \
+                      : pa::paged_decode_kernel<d, b, f>;
     PA_PICK(64, 16, false) PA_PICK(64, 32, false) PA_PICK(128, 16, false) PA_PICK(128, 32, false)
     PA_PICK(64, 16, true) PA_PICK(64, 32, true) PA_PICK(128, 16, true) PA_PICK(128, 32, true)
 #undef PA_PICK
@@ -288,6 +290,32 @@ int ensure_smem_attr(const void *fn, int device) {
         cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxSmem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
     g_attr_done.emplace_back(fn, device);
+    return PA_OK;
+}
+
+// Resident CTAs per SM of a kernel at a block size and dynamic shared
+// memory, cached per (kernel, block, smem) (the answer depends on no state).
+struct OccEntry {
+    const void *fn;
+    int threads;
+    size_t smem;
+    int ctas;
+};
+std::mutex g_occ_mu;
+std::vector<OccEntry> g_occ;
+
+int ctas_per_sm(const void *fn, int threads, size_t smem, int *out) {
+    std::lock_guard<std::mutex> lk(g_occ_mu);
+    for (const auto &e : g_occ)
+        if (e.fn == fn && e.threads == threads && e.smem == smem) {
+            *out = e.ctas;
+            return PA_OK;
+        }
+    int n = 0;
+    const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, threads, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    g_occ.push_back({fn, threads, smem, n});
+    *out = n;
     return PA_OK;
 }
 
@@ -369,6 +397,14 @@ struct PrefixPlan {
     bool mma;           // fp16 caches: the tensor-core kernel
 };
 
+// pa_test_stall_next_decode: consumed (and cleared) by the next decode
+// launch of this thread.
+struct StallRequest {
+    int64_t unit = -1;
+    uint64_t wait_limit_ns = 0;
+};
+thread_local StallRequest g_stall;
+
 int launch_decode(void *out, const void *query, const void *kc, const void *vc,
                   const pa_cache_desc &c, const int32_t *bt, int maxblk, const int32_t *ctx, int S,
                   int max_ctx, float scale, float k_scale, float v_scale,
@@ -434,10 +470,31 @@ int launch_decode(void *out, const void *query, const void *kc, const void *vc,
         p.v_scale = fp8 ? v_scale : 1.0f;
     }
 
+    if (g_stall.unit >= 0) {
+        p.stall_unit_plus1 = g_stall.unit + 1;
+        p.wait_limit_ns = g_stall.wait_limit_ns;
+        g_stall = StallRequest{};
+    }
+
+    const int C = cfg.units_per_cta;
+    const pa::SmemLayout lay(B, G, D, elem_bytes(c), W, cfg.stages, C);
+    const int threads = 32 * (C * G * W + 1);
     DecodeKernel kern = pick_decode(D, B, fp8);
     if (!kern) return fail(PA_ERR_INVALID, "no kernel for head_size %d block_size %d", D, B);
     rc = ensure_smem_attr(reinterpret_cast<const void *>(kern), device);
     if (rc) return rc;
+    if (threads <= pa::kNarrowDecodeThreads) {
+        // the register-capped instantiation, where it fits more CTAs on an SM
+        DecodeKernel narrow = pick_decode(D, B, fp8, true);
+        rc = ensure_smem_attr(reinterpret_cast<const void *>(narrow), device);
+        if (rc) return rc;
+        int wide_ctas = 0, narrow_ctas = 0;
+        rc = ctas_per_sm(reinterpret_cast<const void *>(kern), threads, lay.total, &wide_ctas);
+        if (rc) return rc;
+        rc = ctas_per_sm(reinterpret_cast<const void *>(narrow), threads, lay.total, &narrow_ctas);
+        if (rc) return rc;
+        if (narrow_ctas > wide_ctas) kern = narrow;
+    }
     cudaError_t e;
     if (pre) {
         DecodeKernel pkern = pre->mma ? pick_prefix_mma(D, B) : pick_prefix(D, B, fp8);
@@ -464,8 +521,6 @@ int launch_decode(void *out, const void *query, const void *kc, const void *vc,
         e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "paged_prefix_kernel launch");
     }
-    const int C = cfg.units_per_cta;
-    const pa::SmemLayout lay(B, G, D, elem_bytes(c), W, cfg.stages, C);
     // Every unit u is served by CTA u % grid, slot u / grid: grid * C >= units.
     // Packed CTAs are spread over all SMs (some slots of the last ones idle).
     const int64_t n_ctas = std::max<int64_t>((p.num_units + C - 1) / C,
@@ -474,7 +529,7 @@ int launch_decode(void *out, const void *query, const void *kc, const void *vc,
     if (n_ctas > 0x7fffffff || p.num_units > 0x7fffffff)
         return fail(PA_ERR_INVALID, "too many work units (%lld)", (long long)p.num_units);
     const dim3 grid((unsigned)n_ctas);
-    const dim3 block(32 * (C * G * W + 1));
+    const dim3 block(threads);
     kern<<<grid, block, lay.total, st>>>(mk, mv, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "paged_decode_kernel launch");
@@ -496,9 +551,22 @@ int current_device(int *dev) {
 
 extern "C" {
 
-int pa_version(void) { return 201; }
+int pa_version(void) { return 202; }
 
 const char *pa_last_error(void) { return g_msg; }
+
+int pa_test_stall_next_decode(int64_t unit, uint64_t wait_limit_ns) {
+    if (unit < 0) {
+        g_stall = StallRequest{};
+        return ok();
+    }
+    if (wait_limit_ns < 1000 || wait_limit_ns > pa::kWaitLimitNs)
+        return fail(PA_ERR_INVALID, "wait_limit_ns %llu outside [1000, %llu]",
+                    (unsigned long long)wait_limit_ns, (unsigned long long)pa::kWaitLimitNs);
+    g_stall.unit = unit;
+    g_stall.wait_limit_ns = wait_limit_ns;
+    return ok();
+}
 
 int pa_check_status(void *stream, uint32_t *code) {
     if (!code) return fail(PA_ERR_INVALID, "code is null");

@@ -82,6 +82,13 @@ struct DecodeParams {
     int32_t *slot_out;
     float k_scale;               // E4M3 encode scales (1 for fp16 caches)
     float v_scale;
+    // Bounded waits of the decode kernel: the wall-time limit of each
+    // mbarrier wait (0, the default: kWaitLimitNs; a test may shorten it),
+    // and a test hook: with stall_unit_plus1 = u + 1 the producer issues no
+    // tile loads for work unit u, so that unit's consumers must give up at
+    // the limit (0, the default: no unit is stalled).
+    uint64_t wait_limit_ns;
+    int64_t stall_unit_plus1;
 };
 
 
@@ -162,31 +169,34 @@ __device__ __forceinline__ void unpack16<true>(const uint4 &raw, float *f) {
 // Lane layout (Geometry): lane group `grp` takes TPG tokens of each tile,
 // lane `sub` of the group holds EPL elements of the query, K/V rows and
 // output accumulator.
+//
+// Arithmetic: every product is formed exactly (fp16 x fp16 into fp32, one
+// FMA-pipe instruction per element, fma.rn.f32.f16) and summed in fp32:
+//   logits  z_t = (scale * log2 e * k_scale) * sum_d q[d] k_t[d]   (q as given, k
+//           as stored: fp16, or the E4M3 code decoded exactly to fp16);
+//   weights p_t = 2^(z_t - m), rounded to fp16 once, and that same fp16
+//           value enters both l = sum_t p_t and acc[d] = sum_t p_t v_t[d],
+//           so acc / l is an exact convex combination of the rows.
+// The reference maximum m moves lazily: only when a tile holds a logit more
+// than kLazyMax above it (then m becomes the running maximum and l, acc are
+// rescaled). Weights therefore stay at most 2^kLazyMax, and most tiles of a
+// long context cost no warp-wide maximum and no rescale.
 template <int D, int B, bool kFp8>
 struct HeadAttn {
     using Geo = Geometry<D, B, kFp8>;
     static constexpr int EPL = Geo::EPL, LPR = Geo::LPR, TPG = Geo::TPG, DUP = Geo::DUP;
-    // fp16 caches: query in fp32, pre-scaled by scale*log2(e). E4M3 caches:
-    // the pre-scaled query rounded to f16 pairs for packed f16x2 products
-    // with the decoded keys (k_scale goes on each logit).
-    float q[kFp8 ? 1 : EPL];
-    uint32_t q2[kFp8 ? EPL / 2 : 1];
+    static constexpr float kLazyMax = 8.0f;
+    uint32_t q2[EPL / 2];  // this lane's query elements as fp16 pairs (bits as given)
     float m, l;
     float acc[EPL];
 
-    __device__ __forceinline__ void init(const uint4 (&q_raw)[EPL / 8], float qk_scale_log2) {
-        float qf[EPL];
+    __device__ __forceinline__ void init(const uint4 (&q_raw)[EPL / 8]) {
 #pragma unroll
-        for (int c = 0; c < EPL / 8; ++c) unpack16<false>(q_raw[c], qf + 8 * c);
-        if constexpr (kFp8) {
-#pragma unroll
-            for (int e = 0; e < EPL / 2; ++e) {
-                const __half2 h = __floats2half2_rn(qf[2 * e] * qk_scale_log2, qf[2 * e + 1] * qk_scale_log2);
-                q2[e] = *reinterpret_cast<const uint32_t *>(&h);
-            }
-        } else {
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) q[e] = qf[e] * qk_scale_log2;
+        for (int c = 0; c < EPL / 8; ++c) {
+            q2[4 * c + 0] = q_raw[c].x;
+            q2[4 * c + 1] = q_raw[c].y;
+            q2[4 * c + 2] = q_raw[c].z;
+            q2[4 * c + 3] = q_raw[c].w;
         }
         m = -INFINITY;
         l = 0.f;
@@ -194,91 +204,88 @@ struct HeadAttn {
         for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
     }
 
+    // sum over this lane's EPL dims of q * k (16 bytes of one K row)
+    __device__ __forceinline__ float dot16(const uint4 &raw) const {
+        float c0 = 0.f, c1 = 0.f;
+        const uint32_t *w = reinterpret_cast<const uint32_t *>(&raw);
+        if constexpr (kFp8) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                uint32_t k01, k23;
+                e4m3x4_to_half2x2(w[i], k01, k23);
+                fma2_f16_f32(q2[2 * i], k01, c0, c1);
+                fma2_f16_f32(q2[2 * i + 1], k23, c0, c1);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) fma2_f16_f32(q2[i], w[i], c0, c1);
+        }
+        return c0 + c1;
+    }
+
+    // acc += p * v over this lane's EPL dims (p: fp16 in the low half of p1)
+    __device__ __forceinline__ void axpy16(uint32_t p1, const uint4 &raw) {
+        const uint32_t *w = reinterpret_cast<const uint32_t *>(&raw);
+        if constexpr (kFp8) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                uint32_t v01, v23;
+                e4m3x4_to_half2x2(w[i], v01, v23);
+                fma1x2_f16_f32(p1, v01, acc[4 * i], acc[4 * i + 1]);
+                fma1x2_f16_f32(p1, v23, acc[4 * i + 2], acc[4 * i + 3]);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) fma1x2_f16_f32(p1, w[i], acc[2 * i], acc[2 * i + 1]);
+        }
+    }
+
     // One tile: rows t < valid of the tile (row t at `ktile + t*row_stride +
-    // head_off`, V likewise) take part; row t_new (if >= 0) is taken from
-    // k_new/v_new instead (the appended token, already in cache format).
-    __device__ __forceinline__ void consume(const unsigned char *ktile, const unsigned char *vtile,
-                                            size_t row_stride, size_t head_off, int valid, int t_new,
-                                            const uint4 &k_new, const uint4 &v_new,
-                                            float logit_k_scale, int lane) {
+    // head_off`, V likewise) take part; rows at or past `valid` are never
+    // multiplied into acc (they may hold anything, NaN included).
+    template <bool kFull>
+    __device__ __forceinline__ void tile(const unsigned char *ktile, const unsigned char *vtile,
+                                         size_t row_stride, size_t head_off, int valid, float qk_mul,
+                                         int lane) {
         const int grp = lane / LPR, sub = lane % LPR;
         // ---- logits of this lane group's TPG tokens
         float part_dot[TPG];
 #pragma unroll
         for (int j = 0; j < TPG; ++j) {
             const int t = grp * TPG + j;
-            uint4 raw;
-            if (t == t_new) raw = k_new;
-            else raw = *reinterpret_cast<const uint4 *>(ktile + t * row_stride + head_off);
-            float d = 0.f;
-            if constexpr (kFp8) {
-                // packed f16x2 products of the f16 query and the decoded keys,
-                // summed in f16x2 over this lane's 16 elements, then in fp32
-                const uint16_t *c = reinterpret_cast<const uint16_t *>(&raw);
-                __half2 s2 = __float2half2_rn(0.f);
-#pragma unroll
-                for (int e = 0; e < EPL / 2; ++e)
-                    s2 = __hfma2(*reinterpret_cast<const __half2 *>(&q2[e]), e4m3x2_to_half2(c[e]), s2);
-                const float2 sf = __half22float2(s2);
-                d = sf.x + sf.y;
-            } else {
-                float k[EPL];
-                unpack16<false>(raw, k);
-#pragma unroll
-                for (int e = 0; e < EPL; ++e) d = fmaf(q[e], k[e], d);
-            }
-            part_dot[j] = d;
+            part_dot[j] = dot16(*reinterpret_cast<const uint4 *>(ktile + t * row_stride + head_off));
         }
         const int my_t = grp * TPG + sub / DUP;
-        float z = butterfly_reduce<TPG, LPR>(part_dot, lane);
-        if constexpr (kFp8) z *= logit_k_scale;
-        z = (my_t < valid) ? z : -INFINITY;
+        float z = butterfly_reduce<TPG, LPR>(part_dot, lane) * qk_mul;
+        if (!kFull) z = (my_t < valid) ? z : -INFINITY;
 
-        // ---- online softmax (base 2)
-        const float m_new = fmaxf(m, warp_max(z));
-        const float alpha = fast_exp2(m - m_new);
-        const float pz = fast_exp2(z - m_new);
-        l = l * alpha + pz;
+        // ---- online softmax (base 2) with a lazily moved reference maximum
+        if (__any_sync(0xffffffffu, z > m + kLazyMax)) {
+            const float m_new = fmaxf(m, warp_max(z));
+            const float alpha = fast_exp2(m - m_new);  // m = -inf on the first tile: 0
+            l *= alpha;
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) acc[e] *= alpha;
-        m = m_new;
-
-        // ---- P.V for this lane group's tokens (E4M3: the tile's tokens are
-        //      accumulated in f16x2, then added to the fp32 accumulators)
-        __half2 pv2[kFp8 ? EPL / 2 : 1];
-        if constexpr (kFp8) {
-#pragma unroll
-            for (int e = 0; e < EPL / 2; ++e) pv2[e] = __float2half2_rn(0.f);
+            for (int e = 0; e < EPL; ++e) acc[e] *= alpha;
+            m = m_new;
         }
+        const uint32_t p1 = f32_to_f16_bits(fast_exp2(z - m));  // <= 2^kLazyMax
+        l = add_f16_f32(p1, l);
+
+        // ---- P.V for this lane group's tokens
 #pragma unroll
         for (int j = 0; j < TPG; ++j) {
             const int t = grp * TPG + j;
-            const float pj = __shfl_sync(0xffffffffu, pz, grp * LPR + j * DUP);
-            if (t < valid) {
-                uint4 raw;
-                if (t == t_new) raw = v_new;
-                else raw = *reinterpret_cast<const uint4 *>(vtile + t * row_stride + head_off);
-                if constexpr (kFp8) {
-                    const __half2 p2 = __float2half2_rn(pj);  // weight <= 1 in f16
-                    const uint16_t *c = reinterpret_cast<const uint16_t *>(&raw);
-#pragma unroll
-                    for (int e = 0; e < EPL / 2; ++e) pv2[e] = __hfma2(p2, e4m3x2_to_half2(c[e]), pv2[e]);
-                } else {
-                    float v[EPL];
-                    unpack16<false>(raw, v);
-#pragma unroll
-                    for (int e = 0; e < EPL; ++e) acc[e] = fmaf(pj, v[e], acc[e]);
-                }
-            }
+            const uint32_t pj = __shfl_sync(0xffffffffu, p1, grp * LPR + j * DUP);
+            if (kFull || t < valid)
+                axpy16(pj, *reinterpret_cast<const uint4 *>(vtile + t * row_stride + head_off));
         }
-        if constexpr (kFp8) {
-#pragma unroll
-            for (int e = 0; e < EPL / 2; ++e) {
-                const float2 f = __half22float2(pv2[e]);
-                acc[2 * e] += f.x;
-                acc[2 * e + 1] += f.y;
-            }
-        }
+    }
+
+    __device__ __forceinline__ void consume(const unsigned char *ktile, const unsigned char *vtile,
+                                            size_t row_stride, size_t head_off, int valid, float qk_mul,
+                                            int lane) {
+        if (valid >= B) tile<true>(ktile, vtile, row_stride, head_off, valid, qk_mul, lane);
+        else tile<false>(ktile, vtile, row_stride, head_off, valid, qk_mul, lane);
     }
 
     // Sums l over all lanes and acc over the lane groups (group 0 then holds
@@ -357,8 +364,15 @@ __device__ __forceinline__ Unit unit_of(const DecodeParams &p, int B, int j) {
     return u;
 }
 
-template <int D, int B, bool kFp8>
-__global__ void __launch_bounds__(kMaxDecodeThreads, 1)
+// Launch bounds: the default instantiation takes any launch shape (up to
+// kMaxDecodeThreads threads); the "narrow" one (at most kNarrowDecodeThreads
+// threads, registers capped so that kNarrowDecodeCtas CTAs fit an SM) is
+// used when the cap lets more CTAs share an SM (two warps per head).
+constexpr int kNarrowDecodeThreads = 288;
+constexpr int kNarrowDecodeCtas = 3;
+
+template <int D, int B, bool kFp8, int kThreads = kMaxDecodeThreads, int kMinCtas = 1>
+__global__ void __launch_bounds__(kThreads, kMinCtas)
 paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
     using Geo = Geometry<D, B, kFp8>;
@@ -376,6 +390,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int lane = threadIdx.x & 31;
     const int per_slot = G * W;
     const int n_consumers = C * per_slot;
+    const uint64_t wait_limit = p.wait_limit_ns ? p.wait_limit_ns : kWaitLimitNs;
 
     if (warp == n_consumers) {
         // ================================================================ producer
@@ -415,6 +430,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
         for (int j = 0; j < kMaxUnitsPerCta; ++j) {  // independent loads: all in flight together
             if (j < C) u[j] = unit_of(p, B, j);
             else u[j].live = u[j].append = false, u[j].nblk = 0;
+            if (j < C && (int64_t)blockIdx.x + (int64_t)j * gridDim.x + 1 == p.stall_unit_plus1) u[j].nblk = 0;
             issued[j] = 0;
             cur_blk[j] = pre_blk[j];
         }
@@ -465,7 +481,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
             const int st = i % stages, use = i / stages;
             if (lane == 0) {
                 if (bad) flag_error(PA_DEV_BAD_BLOCK);
-                if (use > 0) ok = mbar_wait(&empty_all[j * stages + st], (use - 1) & 1);
+                if (use > 0) ok = mbar_wait(&empty_all[j * stages + st], (use - 1) & 1, wait_limit);
                 if (ok) {
                     unsigned char *kdst = smem + (size_t)j * lay.slot_bytes + (size_t)st * lay.stage_bytes;
                     uint64_t *fb = &full_all[j * stages + st];
@@ -547,21 +563,27 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
     }
 
     HeadAttn<D, B, kFp8> st;
-    st.init(q_raw, p.qk_scale_log2);
+    st.init(q_raw);
+    const float qk_mul = p.qk_scale_log2 * p.logit_k_scale;
 
     const size_t row_stride = (size_t)G * D * EB;  // bytes between tokens in a tile
     const size_t head_off = (size_t)g * D * EB + (size_t)sub * 16;
     // Fused append (a1 + a2): the unit holding position L-1 takes the new
-    // token from registers, in cache format (E4M3 codes for an fp8 cache, so
-    // that it is used exactly as a later step will read it back), and the
-    // first warp of each head stores the head's row into the token's slot.
-    // That row of the tile is never read, so no tile load waits for the store.
+    // token in cache format (E4M3 codes for an fp8 cache, so that it is used
+    // exactly as a later step will read it back). The lanes of group 0 park
+    // their part of the row in this warp's merge area (unused until the
+    // merge) instead of keeping it in registers through the loop; once the
+    // block holding the token has landed, the lanes that read that row copy
+    // it over their head's part of the row in shared memory. The first warp
+    // of each head stores the head's row into the token's slot in the cache.
+    // The loaded row itself is never used, so no tile load waits for the store.
     int t_new_block = -1, t_new_row = -1;
-    uint4 k_new = make_uint4(0, 0, 0, 0), v_new = make_uint4(0, 0, 0, 0);
+    uint2 *stash = reinterpret_cast<uint2 *>(merge + (size_t)(w * G + g) * (D + 2)) + sub * 4;
     if (x.append) {
         const int pos = x.L - 1;
         t_new_block = (pos - x.t0) / B;
         t_new_row = pos % B;
+        uint4 k_new, v_new;
         if constexpr (!kFp8) {
             k_new = nk_raw[0];
             v_new = nv_raw[0];
@@ -570,6 +592,12 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
             const uint2 v0 = encode8_e4m3(nv_raw[0], p.v_scale), v1 = encode8_e4m3(nv_raw[1], p.v_scale);
             k_new = make_uint4(k0.x, k0.y, k1.x, k1.y);
             v_new = make_uint4(v0.x, v0.y, v1.x, v1.y);
+        }
+        if (grp == 0) {
+            stash[0] = make_uint2(k_new.x, k_new.y);
+            stash[1] = make_uint2(k_new.z, k_new.w);
+            stash[2] = make_uint2(v_new.x, v_new.y);
+            stash[3] = make_uint2(v_new.z, v_new.w);
         }
         if (w == 0 && grp == 0) {
             const int blk = __ldg(p.block_tables + (size_t)x.s * p.max_blocks_per_seq + pos / B);
@@ -581,19 +609,28 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
             if (p.slot_out && h == 0 && sub == 0) p.slot_out[x.s] = bad ? -1 : blk * B + pos % B;
         }
+        __syncwarp();
     }
     int stage = w % stages, use = w / stages;
     for (int i = w; i < x.nblk; i += W) {
-        if (!mbar_wait(&full[stage], use & 1)) break;
-        const unsigned char *ktile = slot_base + (size_t)stage * lay.stage_bytes;
-        const unsigned char *vtile = ktile + lay.tile_bytes;
+        if (!mbar_wait(&full[stage], use & 1, wait_limit)) break;
+        unsigned char *ktile = slot_base + (size_t)stage * lay.stage_bytes;
+        unsigned char *vtile = ktile + lay.tile_bytes;
         const int valid = min(B, x.t1 - (x.t0 + i * B));  // tokens of this block inside the context
-        const int t_new = (i == t_new_block) ? t_new_row : -1;
-        st.consume(ktile, vtile, row_stride, head_off, valid, t_new, k_new, v_new, p.logit_k_scale, lane);
+        if (i == t_new_block) {
+            if (grp == t_new_row / Geo::TPG) {
+                const uint2 k0 = stash[0], k1 = stash[1], v0 = stash[2], v1 = stash[3];
+                *reinterpret_cast<uint4 *>(ktile + t_new_row * row_stride + head_off) = make_uint4(k0.x, k0.y, k1.x, k1.y);
+                *reinterpret_cast<uint4 *>(vtile + t_new_row * row_stride + head_off) = make_uint4(v0.x, v0.y, v1.x, v1.y);
+                fence_proxy_async_smem();  // before the stage is refilled by the next TMA
+            }
+            __syncwarp();
+        }
+        st.consume(ktile, vtile, row_stride, head_off, valid, qk_mul, lane);
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[stage]);
         stage += W;
-        while (stage >= stages) {
+        if (stage >= stages) {  // W <= stages
             stage -= stages;
             ++use;
         }
@@ -813,19 +850,18 @@ paged_prefix_kernel(const __grid_constant__ CUtensorMap tmap_k,
     }
     asm volatile("bar.sync 1, %0;" ::"r"((n_consumers + 1) * 32) : "memory");
     HeadAttn<D, B, kFp8> st;
-    st.init(q_raw, p.qk_scale_log2);
+    st.init(q_raw);
+    const float qk_mul = p.qk_scale_log2 * p.logit_k_scale;
     const int end = min(t1, L);  // this sequence's tokens in the partition
     const size_t row_stride = (size_t)G * D * EB;
     const size_t head_off = (size_t)g * D * EB + (size_t)sub * 16;
-    const uint4 none = make_uint4(0, 0, 0, 0);
     for (int i = 0; i < nblk; ++i) {
         const int stg = i % stages, use = i / stages;
         if (!mbar_wait(&full[stg], use & 1)) break;
         const int valid = min(B, end - (t0 + i * B));
         if (valid > 0) {
             const unsigned char *ktile = smem + (size_t)stg * lay.stage_bytes;
-            st.consume(ktile, ktile + lay.tile_bytes, row_stride, head_off, valid, -1, none, none,
-                       p.logit_k_scale, lane);
+            st.consume(ktile, ktile + lay.tile_bytes, row_stride, head_off, valid, qk_mul, lane);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[stg]);

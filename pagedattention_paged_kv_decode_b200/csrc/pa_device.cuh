@@ -75,12 +75,13 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
     return done != 0;
 }
 
-// A wait that gives up after kWaitLimitNs of wall time (2 s), sets
-// PA_DEV_WAIT_TIMEOUT and returns false. In a correct launch every wait ends
-// within microseconds; the limit only keeps a broken one from hanging the GPU.
+// A wait that gives up after limit_ns of wall time (by default kWaitLimitNs,
+// 2 s), sets PA_DEV_WAIT_TIMEOUT and returns false. In a correct launch every
+// wait ends within microseconds; the limit only keeps a broken one from
+// hanging the GPU.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
 #pragma unroll 1
     for (int i = 0; i < 64; ++i)  // the common case: no timer read at all
         if (mbar_try_wait(bar, parity)) return true;
@@ -89,7 +90,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
 #pragma unroll 1
         for (int i = 0; i < 32; ++i)
             if (mbar_try_wait(bar, parity)) return true;
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
+        if (global_timer_ns() - t0 > limit_ns) {
             flag_error(PA_DEV_WAIT_TIMEOUT);
             return false;
         }
@@ -332,6 +333,60 @@ __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int m = 16; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
     return v;
+}
+
+// Mixed-precision multiply-add on the FMA pipe: the product of two fp16
+// values is exact in fp32 (11 x 11 significant bits), so each call adds the
+// exact products to fp32 accumulators with one rounding per add.
+// c0 += lo(a2) * lo(b2), c1 += hi(a2) * hi(b2) (a2, b2: packed fp16 pairs).
+__device__ __forceinline__ void fma2_f16_f32(uint32_t a2, uint32_t b2, float &c0, float &c1) {
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
+        "mov.b32 {al, ah}, %2;\n\t"
+        "mov.b32 {bl, bh}, %3;\n\t"
+        "fma.rn.f32.f16 %0, al, bl, %0;\n\t"
+        "fma.rn.f32.f16 %1, ah, bh, %1;\n\t}"
+        : "+f"(c0), "+f"(c1)
+        : "r"(a2), "r"(b2));
+}
+
+// c0 += p * lo(v2), c1 += p * hi(v2) with p one fp16 value (low half of p1).
+__device__ __forceinline__ void fma1x2_f16_f32(uint32_t p1, uint32_t v2, float &c0, float &c1) {
+    asm("{\n\t.reg .b16 pl, ph, vl, vh;\n\t"
+        "mov.b32 {pl, ph}, %2;\n\t"
+        "mov.b32 {vl, vh}, %3;\n\t"
+        "fma.rn.f32.f16 %0, pl, vl, %0;\n\t"
+        "fma.rn.f32.f16 %1, pl, vh, %1;\n\t}"
+        : "+f"(c0), "+f"(c1)
+        : "r"(p1), "r"(v2));
+}
+
+// fp32 -> fp16 (round to nearest even) in the low half of a 32-bit word, and
+// c + that fp16 value (exact conversion, one fp32 rounding).
+__device__ __forceinline__ uint32_t f32_to_f16_bits(float x) {
+    uint16_t h;
+    asm("cvt.rn.f16.f32 %0, %1;" : "=h"(h) : "f"(x));
+    return h;
+}
+
+__device__ __forceinline__ float add_f16_f32(uint32_t h1, float c) {
+    float d;
+    asm("{\n\t.reg .b16 hl, hh;\n\t"
+        "mov.b32 {hl, hh}, %1;\n\t"
+        "add.rn.f32.f16 %0, hl, %2;\n\t}"
+        : "=f"(d)
+        : "r"(h1), "f"(c));
+    return d;
+}
+
+// Four E4M3 codes (one 32-bit word, first element in the low byte) -> two
+// packed fp16 pairs, exact: lo gets codes 0-1, hi codes 2-3.
+__device__ __forceinline__ void e4m3x4_to_half2x2(uint32_t codes, uint32_t &lo, uint32_t &hi) {
+    asm("{\n\t.reg .b16 cl, ch;\n\t"
+        "mov.b32 {cl, ch}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, cl;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %1, ch;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(codes));
 }
 
 // Two E4M3 codes (low byte = first element) -> two halves, exact.

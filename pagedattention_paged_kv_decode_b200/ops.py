@@ -392,6 +392,16 @@ def version() -> int:
     return int(lib().pa_version())
 
 
+def test_stall_next_decode(unit: int, wait_limit_ns: int) -> None:
+    """Test hook of the bounded waits: the next decode launched on this
+    thread issues no tile loads for work unit `unit` and limits each wait to
+    wait_limit_ns (that unit then reports PA_DEV_WAIT_TIMEOUT; its output
+    rows are undefined). unit < 0 clears a pending request."""
+    if int(unit) >= 0 and not 1000 <= int(wait_limit_ns) <= 2_000_000_000:
+        raise ValueError(f"wait_limit_ns {wait_limit_ns} outside [1000, 2e9]")
+    check(lib().pa_test_stall_next_decode(int(unit), int(wait_limit_ns)))
+
+
 def last_error() -> str:
     """Message of the last nonzero status on this thread ("" if none); the
     binding also raises it as PagedKVError."""

@@ -49,5 +49,5 @@ class Recorder:
                 return 4096
             if res is ctypes.c_char_p:
                 return b""
-            return 201 if name == "pa_version" else 0
+            return 202 if name == "pa_version" else 0
         return call

@@ -118,7 +118,7 @@ def test_size_and_status_calls(rec):
     _check(rec, "pa_decode_choose_config")
     assert ops.check_status(stream=0) == 0
     _check(rec, "pa_check_status")
-    assert ops.version() == 201
+    assert ops.version() == 202
     _check(rec, "pa_version")
     assert ops.last_error() == ""
     _check(rec, "pa_last_error")

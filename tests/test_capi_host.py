@@ -35,7 +35,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_version_and_empty_error():
-    assert capi.lib().pa_version() == 201
+    assert capi.lib().pa_version() == 202
 
 
 F = capi.CacheDesc(64, 16, 8, 128, capi.PA_F16)
@@ -283,7 +283,8 @@ def _prototypes():
 
 
 _CTYPE_OF = {
-    "int": ctypes.c_int, "int64_t": ctypes.c_int64, "float": ctypes.c_float, "size_t": ctypes.c_size_t,
+    "int": ctypes.c_int, "int64_t": ctypes.c_int64, "uint64_t": ctypes.c_uint64, "float": ctypes.c_float,
+    "size_t": ctypes.c_size_t,
     "pa_cache_desc": capi.CacheDesc, "const char*": ctypes.c_char_p,
 }
 

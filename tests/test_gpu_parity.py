@@ -39,13 +39,36 @@ def host(t):
     return t.cpu().numpy()
 
 
-def compare_step(w, dw, seqs, check_all_blocks):
-    slots, kc, vc, out_ref, blocks = oracle_step(w, seqs)
+def same_cache(a: np.ndarray, b: np.ndarray) -> bool:
+    """Bitwise equality of two caches, with every NaN code of E4M3 counted
+    as the same NaN (the encoders agree on values; NaN poison may differ in
+    its sign)."""
+    if a.dtype == np.uint8:
+        nan_a = (a & 0x7F) == 0x7F
+        nan_b = (b & 0x7F) == 0x7F
+        return bool(np.array_equal(nan_a, nan_b) and np.array_equal(np.where(nan_a, 0, a), np.where(nan_b, 0, b)))
+    return bool(np.array_equal(a.view(np.uint16), b.view(np.uint16)))
+
+
+_ORACLE_STEPS = {}
+
+
+def oracle_full_step(w):
+    """Oracle step of a named workload over every sequence and the whole pool
+    (cached: the fused and separate GPU runs check against the same result)."""
+    if w.name not in _ORACLE_STEPS:
+        _ORACLE_STEPS.clear()
+        _ORACLE_STEPS[w.name] = oracle_step(w, whole_pool=True)
+    return _ORACLE_STEPS[w.name]
+
+
+def compare_step(w, dw, seqs, check_all_blocks, ref=None):
+    slots, kc, vc, out_ref, blocks = ref if ref is not None else oracle_step(w, seqs)
     assert np.array_equal(host(dw.slots), slots)
     gk, gv = dw.key_cache, dw.value_cache
-    if check_all_blocks and w.kv_dtype == "f16":
-        assert np.array_equal(host(gk).view(np.uint16), kc.view(np.uint16))
-        assert np.array_equal(host(gv).view(np.uint16), vc.view(np.uint16))
+    if check_all_blocks and (w.kv_dtype == "f16" or ref is not None):
+        assert same_cache(host(gk), kc)
+        assert same_cache(host(gv), vc)
     else:
         idx = torch.from_numpy(blocks).to(gk.device)
         a, b = host(gk[idx]), kc[blocks]
@@ -66,10 +89,11 @@ def compare_step(w, dw, seqs, check_all_blocks):
 @pytest.mark.parametrize("fused", [True, False], ids=["fused", "separate"])
 @pytest.mark.parametrize("cfg", [1, 2, 3, 4, 5])
 def test_named_workload_step(cuda_device, cfg, fused):
+    """Every sequence and head of the workload, and the whole pool after the
+    step (E4M3 pools encoded in full by the oracle)."""
     w = W.named(cfg)
     dw = run_step(w, cuda_device, fused=fused)
-    seqs = list(range(w.num_seqs)) if cfg <= 2 else sample_seqs(w, 8, seed=cfg)
-    compare_step(w, dw, seqs, check_all_blocks=cfg <= 2)
+    compare_step(w, dw, list(range(w.num_seqs)), check_all_blocks=True, ref=oracle_full_step(w))
 
 
 def ragged_case(D, B, kv, seed, ctx=None, poison=W.POISON_HUGE, H=4):
@@ -103,6 +127,10 @@ LAUNCH = [
     dict(partition_size=32, heads_per_cta=2, warps_per_head=1, stages=3, units_per_cta=3),
     dict(partition_size=512, heads_per_cta=1, warps_per_head=1, stages=2, units_per_cta=2),
     dict(partition_size=128, heads_per_cta=4, warps_per_head=2, stages=2, units_per_cta=2),
+    # nine-warp CTAs whose ring leaves room for three per SM: the register-capped
+    # instantiation of the decode kernel is the one launched
+    dict(partition_size=512, heads_per_cta=4, warps_per_head=2, stages=2),
+    dict(partition_size=256, heads_per_cta=4, warps_per_head=2, stages=4),
 ]
 
 
@@ -133,7 +161,16 @@ def test_nan_poison_is_never_touched(cuda_device, kv):
 
 
 def test_split_partials_match_oracle_partitions(cuda_device):
-    """Row by row check of the partition kernel's workspace (lse, o)."""
+    """Row by row check of the partition kernel's workspace (lse, o).
+
+    Tolerances follow from the kernel's arithmetic: each softmax weight p_t
+    is rounded to fp16 once (p'_t = p_t (1 + e_t), |e_t| <= 2^-12) and the
+    same p'_t enters the numerator and the denominator. A normalised partial
+    o = sum p'_t v_t / sum p'_t then differs from the exact one by at most
+    2^-12 / (1 - 2^-12) * max_t |v_t[d] - o[d]| per element (the exact
+    weights sum p_t (v_t - o) to zero), and its log-sum-exp by at most
+    ln(1 + 2^-12) in natural-log units; 2e-5 covers the fp32 sums and the
+    hardware exp2/log2."""
     w = ragged_case(128, 16, "f16", seed=5, ctx=[600, 1100, 40, 1024])
     cfg = dict(partition_size=256, heads_per_cta=2, warps_per_head=2, stages=4)
     dw = W.to_device(w, cuda_device)
@@ -157,12 +194,21 @@ def test_split_partials_match_oracle_partitions(cuda_device):
     o = raw[lse_bytes:lse_bytes + S * H * P * D * 4].view(np.float32).reshape(S, H, P, D)
     _, kc, vc, _, _ = oracle_step(w)
     ro, rlse = oracle.attention_partials(w.query, kc, vc, w.block_tables, w.context_lens, w.scale, 256)
+    eps = 2.0 ** -12
+    B = w.block_size
     for s, L in enumerate(w.context_lens):
         n = -(-int(L) // 256)
         if n <= 1:
             continue                              # single partitions write the output directly
-        np.testing.assert_allclose(lse2[s, :, :n] * np.log(2.0), rlse[s, :, :n], rtol=0, atol=2e-4)
-        np.testing.assert_allclose(o[s, :, :n], ro[s, :, :n], rtol=0, atol=1e-4)
+        np.testing.assert_allclose(lse2[s, :, :n] * np.log(2.0), rlse[s, :, :n], rtol=0,
+                                   atol=np.log1p(eps) + 2e-5)
+        for p in range(n):
+            t = np.arange(p * 256, min(int(L), (p + 1) * 256))
+            rows = vc[w.block_tables[s, t // B], t % B].astype(np.float64)    # [tokens, H, D]
+            spread = np.abs(rows - ro[s, :, p][None]).max(axis=0)           # [H, D]
+            bound = eps / (1 - eps) * spread + 2e-5
+            assert (np.abs(o[s, :, p] - ro[s, :, p]) <= bound).all(), \
+                float((np.abs(o[s, :, p] - ro[s, :, p]) - bound).max())
 
 
 def test_e4m3_encode_every_f16_value(cuda_device):
@@ -256,3 +302,18 @@ def test_shared_prefix_contract_is_checked(cuda_device):
                                             slot_mapping=dw.slots)
     assert pk.check_status() == capi.PA_DEV_PREFIX
     assert dw.slots.cpu().tolist()[0] == -1
+
+
+@pytest.mark.parametrize("q_std", [30.0, 300.0])
+@pytest.mark.parametrize("kv", ["f16", "e4m3"])
+def test_large_queries(cuda_device, kv, q_std):
+    """Queries far above a trained model's scale (|q * scale| per element up
+    to ~100): the logits' products are exact and summed in fp32, so neither
+    cache type overflows and the result stays within the parity bar."""
+    ctx = [1, 17, 300, 1100, 64]
+    B, H, D = 16, 4, 128
+    need = sum(-(-L // B) for L in ctx)
+    w = W.build(f"large_q_{kv}", H, D, B, kv, ctx, need + 6, -(-max(ctx) // B), 41,
+                q_std=q_std, kv_std=1.0)
+    dw = run_step(w, cuda_device)
+    compare_step(w, dw, list(range(w.num_seqs)), check_all_blocks=True)

@@ -62,3 +62,39 @@ def test_threaded_reports_a_bad_table_entry():
 
 def test_max_threads_is_positive():
     assert oracle.max_threads() >= 1
+
+
+@pytest.mark.parametrize("kv", ["f16", "e4m3"])
+def test_threaded_cache_write_equals_single_thread(kv):
+    """Duplicate slots (the later token wins), padding slots and a strided
+    source row, on both cache types."""
+    rng = np.random.default_rng(11)
+    NB, B, H, D = 9, 16, 3, 32
+    n = 40
+    src = (rng.standard_normal((n, H, D + 8)) * 3).astype(np.float16)[:, :, :D]  # strided rows
+    key = np.ascontiguousarray(src)
+    val = (rng.standard_normal((n, H, D)) * 200).astype(np.float16)
+    slots = rng.integers(-2, NB * B, n).astype(np.int32)
+    slots[5] = slots[17] = slots[30]          # duplicates
+    dt = np.float16 if kv == "f16" else np.uint8
+    a = [np.zeros((NB, B, H, D), dt) for _ in range(2)]
+    b = [np.zeros((NB, B, H, D), dt) for _ in range(2)]
+    oracle.kv_cache_write(key, val, a[0], a[1], slots, 0.05, 0.7)
+    oracle.kv_cache_write(key, val, b[0], b[1], slots, 0.05, 0.7, threads=4)
+    for x, y in zip(a, b):
+        assert np.array_equal(x.view(np.uint8), y.view(np.uint8))
+
+
+def test_threaded_cache_write_stops_at_the_same_bad_slot():
+    NB, B, H, D = 4, 16, 2, 16
+    key = np.ones((6, H, D), np.float16)
+    slots = np.array([0, 5, NB * B, 7, 8, 9], np.int32)   # the third is beyond the pool
+    a = [np.zeros((NB, B, H, D), np.float16) for _ in range(2)]
+    b = [np.zeros((NB, B, H, D), np.float16) for _ in range(2)]
+    with pytest.raises(ValueError):
+        oracle.kv_cache_write(key, key, a[0], a[1], slots)
+    with pytest.raises(ValueError):
+        oracle.kv_cache_write(key, key, b[0], b[1], slots, threads=3)
+    assert np.array_equal(a[0].view(np.uint16), b[0].view(np.uint16))
+    assert np.array_equal(a[0].reshape(-1, H, D)[[0, 5]], key[:2])
+    assert not a[0].reshape(-1, H, D)[[7, 8, 9]].any()

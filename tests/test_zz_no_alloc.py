@@ -7,17 +7,18 @@ inside the library. This file is collected last on purpose, and every test
 here must pass both alone in a fresh process and after the rest of the suite.
 
 The check: through the C ABI, two calls in a row with different batches that
-both need the split path, each compared with the allocating entry point
-pa_paged_attention_decode on the same inputs (max-abs 2e-3, the fp16-KV
-tolerance of the parity tests), the clear rejection of a batch whose
-partials exceed the static scratch, and the torch binding giving the C
-call's result bit for bit.
+both need the split path, each compared with the CPU oracle and with the
+allocating entry point pa_paged_attention_decode on the same inputs
+(max-abs 2e-3, the fp16-KV tolerance of the parity tests), the clear
+rejection of a batch whose partials exceed the static scratch, and the torch
+binding giving the C call's result bit for bit.
 """
 
 import numpy as np
 import pytest
 import torch
 
+import oracle
 import pagedattention_paged_kv_decode_b200 as pk
 from pagedattention_paged_kv_decode_b200 import capi
 import workloads as W
@@ -61,6 +62,15 @@ def test_noalloc_matches_allocating_entry_point_two_calls(cuda_device):
         b = ref.cpu().numpy().astype(np.float64)
         assert np.isfinite(a).all()
         assert np.abs(a - b).max() <= 2e-3
+        assert np.abs(a - _oracle_out(w)).max() <= 2e-3
+
+
+def _oracle_out(w):
+    """The oracle's own slots, cache write and attention on the batch's inputs."""
+    kc, vc = w.pool_host()
+    slots = oracle.slot_mapping(w.block_tables, w.context_lens, w.block_size)
+    oracle.kv_cache_write(w.new_key, w.new_value, kc, vc, slots)
+    return oracle.paged_attention(w.query, kc, vc, w.block_tables, w.context_lens, w.scale, threads=0)
 
 
 def test_noalloc_rejects_partials_beyond_the_static_scratch(cuda_device):
