@@ -240,6 +240,34 @@ def empty_graph_ms(torch, stream, steps: int) -> float:
     return statistics.mean(ts)
 
 
+def read_floor_ms(torch, stream, nbytes: int, evict, steps: int) -> float:
+    """Reference for the decode's byte rate: a plain reduction (torch's
+    sum) over nbytes of fp16 in one contiguous buffer, captured in a graph
+    between two timing events and replayed after the same L2 eviction as a
+    step (mean over `steps` replays). It reads the same number of bytes as
+    the decode's K/V stream with no gather, no block table and no softmax."""
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+    buf = torch.ones(max(nbytes // 2, 1), dtype=torch.float16, device=stream.device)
+    res = torch.zeros((), dtype=torch.float32, device=stream.device)
+    with torch.cuda.stream(stream):
+        res.copy_(buf.sum(dtype=torch.float32))
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            ev[0].record()
+            res.copy_(buf.sum(dtype=torch.float32))
+            ev[1].record()
+        ts = []
+        for i in range(3 + steps):
+            evict()
+            g.replay()
+            stream.synchronize()
+            if i >= 3:
+                ts.append(ev[0].elapsed_time(ev[1]))
+    del g, buf
+    return statistics.mean(ts)
+
+
 def measure_decode(args, wid, rank, world, local_rank, dist, cpu_seconds, with_swap):
     """One decode workload: build, capture the step in a CUDA graph, time it
     (and its end-to-end form from pinned host buffers), and return the
@@ -249,7 +277,7 @@ def measure_decode(args, wid, rank, world, local_rank, dist, cpu_seconds, with_s
     import pagedattention_paged_kv_decode_b200 as pk
 
     dev = torch.device("cuda", local_rank)
-    w = W.named(wid, seed=W.rank_seed(1000 + wid, rank))
+    w = W.named(wid, seed=W.rank_seed(1000 + wid, rank), num_seqs=args.num_seqs or None)
     dw = W.to_device(w, dev, encode=pk.load_cache)
     S = w.num_seqs
     bound = w.max_blocks_per_seq * w.block_size  # host-side bound: table capacity, no sync
@@ -371,9 +399,10 @@ def measure_decode(args, wid, rank, world, local_rank, dist, cpu_seconds, with_s
         # ------------------------------------------------ swap to/from pinned host memory
         swap = measure_swap(pk, dw, stream, torch) if with_swap else None
         floor = empty_graph_ms(torch, stream, max(20, args.steps))
+        read_ms = read_floor_ms(torch, stream, w.unique_kv_bytes(), evict_l2, max(20, args.steps))
 
-    step_t, dec_t, e2e_t, floor_t = slowest_rank([statistics.mean(step_ms), statistics.mean(dec_ms),
-                                                  statistics.mean(e2e_ms), floor], dist, dev)
+    step_t, dec_t, e2e_t, floor_t, read_t = slowest_rank(
+        [statistics.mean(step_ms), statistics.mean(dec_ms), statistics.mean(e2e_ms), floor, read_ms], dist, dev)
     clocks = sampler.summary(t0, t1)
     del graph
     del dw, flush, packed
@@ -434,6 +463,10 @@ def measure_decode(args, wid, rank, world, local_rank, dist, cpu_seconds, with_s
         "decode_ms": round(dec_t, 5),
         "decode_kv_gbs": round(kv / (dec_t * 1e-3) / 1e9, 2),
         "empty_graph_ms": round(floor_t, 5),
+        "plain_read": {"ms": round(read_t, 5), "bytes": w.unique_kv_bytes(),
+                       "gbs": round(w.unique_kv_bytes() / (read_t * 1e-3) / 1e9, 2),
+                       "what": "torch sum over one contiguous fp16 buffer of the step's distinct K/V bytes, "
+                               "same graph, events and L2 eviction (a reference rate for this size, not our kernel)"},
         "roofline": roofline,
         "e2e": {"value": round(aggregate_gbs(world, kv, e2e_t), 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_t, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -878,6 +911,9 @@ def main():
                     help="time one decode workload only (default: the --workloads list)")
     ap.add_argument("--workloads", default=DEFAULT_WORKLOADS,
                     help="decode workloads timed in one run; the first is the headline")
+    ap.add_argument("--num-seqs", type=int, default=0,
+                    help="batch size of the decode workloads (default: each workload's own); a smaller "
+                         "batch of the same recipe keeps a profiler capture small")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -279,29 +279,39 @@ NAMES = {
 }
 
 
-def named(config_id: int, seed: int | None = None, poison: str = POISON_HUGE) -> Workload:
-    """The five workloads (seed defaults to 1000 + config_id)."""
+def named(config_id: int, seed: int | None = None, poison: str = POISON_HUGE,
+          num_seqs: int | None = None) -> Workload:
+    """The five workloads (seed defaults to 1000 + config_id). num_seqs gives
+    a smaller (or larger) batch drawn by the same recipe -- the same length
+    law, head count, head size, block size and pool rule -- for profiler
+    captures that must stay small; its name carries its own batch size."""
     seed = 1000 + config_id if seed is None else seed
     rng = np.random.Generator(np.random.PCG64(seed))
     name = NAMES[config_id]
+    S0 = {1: 4, 2: 16, 3: 64, 4: 32, 5: 256}[config_id]
+    S = S0 if num_seqs is None else int(num_seqs)
+    if S != S0:
+        if config_id == 3 and S % 2:
+            raise ValueError("the mixed-length batch needs an even number of sequences")
+        name = name.replace(f"_s{S0}_", f"_s{S}_")
     if config_id == 1:
-        ctx = rng.integers(1, 65, 4)
-        return build(name, 4, 64, 16, "f16", ctx, 32, 4, seed, 1.0, 1.0, poison, rng=rng)
+        ctx = rng.integers(1, 65, S)
+        return build(name, 4, 64, 16, "f16", ctx, 32 * S // 4, 4, seed, 1.0, 1.0, poison, rng=rng)
     if config_id == 2:
-        ctx = 50 + rng.integers(0, 129, 16)
-        return build(name, 32, 128, 16, "f16", ctx, 2048, 12, seed, 0.5, 0.5, poison, rng=rng)
+        ctx = 50 + rng.integers(0, 129, S)
+        return build(name, 32, 128, 16, "f16", ctx, 2048 * S // 16, 12, seed, 0.5, 0.5, poison, rng=rng)
     if config_id == 3:
-        ctx = np.concatenate([rng.integers(64, 129, 32), rng.integers(1024, 2049, 32)])
-        ctx = ctx[rng.permutation(64)]
-        return build(name, 40, 128, 16, "f16", ctx, 16384, 128, seed, 0.5, 0.5, poison, rng=rng)
+        ctx = np.concatenate([rng.integers(64, 129, S // 2), rng.integers(1024, 2049, S // 2)])
+        ctx = ctx[rng.permutation(S)]
+        return build(name, 40, 128, 16, "f16", ctx, 16384 * S // 64, 128, seed, 0.5, 0.5, poison, rng=rng)
     if config_id == 4:
-        ctx = 3072 + rng.integers(1, 1025, 32)
+        ctx = 3072 + rng.integers(1, 1025, S)
         private = sum(-(-(int(L) - 3072) // 32) for L in ctx)
-        nb = 96 + private + 32
+        nb = 96 + private + S
         return build(name, 32, 128, 32, "f16", ctx, nb, 128, seed, 0.5, 0.5, poison,
                      shared_prefix=3072, cow=True, rng=rng)
     if config_id == 5:
-        ctx = np.floor(np.exp(rng.uniform(math.log(16), math.log(4096), 256))).astype(np.int64)
+        ctx = np.floor(np.exp(rng.uniform(math.log(16), math.log(4096), S))).astype(np.int64)
         nb = int(math.ceil(1.1 * sum(-(-int(L) // 16) for L in ctx)))
         return build(name, 32, 128, 16, "e4m3", ctx, nb, 256, seed, 1.0, 1.0, poison, rng=rng)
     raise KeyError(config_id)
