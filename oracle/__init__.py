@@ -64,6 +64,8 @@ def _declare(lib):
     lib.oracle_slot_mapping.argtypes = [P, P, I, P, I, I]
     lib.oracle_kv_cache_write.restype = I
     lib.oracle_kv_cache_write.argtypes = [P, P, I64, I64, P, P, I, I, I, I, I, P, I, F, F]
+    lib.oracle_kv_cache_write_threads.restype = I
+    lib.oracle_kv_cache_write_threads.argtypes = [P, P, I64, I64, P, P, I, I, I, I, I, P, I, F, F, I]
     lib.oracle_copy_blocks.restype = I
     lib.oracle_copy_blocks.argtypes = [P, P, I64, I, P, I]
     lib.oracle_swap_blocks.restype = I
@@ -178,8 +180,11 @@ def prefill_slot_mapping(query_start: np.ndarray, block_tables: np.ndarray,
 
 def kv_cache_write(key: np.ndarray, value: np.ndarray, key_cache: np.ndarray,
                    value_cache: np.ndarray, slot_mapping: np.ndarray,
-                   k_scale: float = 1.0, v_scale: float = 1.0) -> None:
-    """In place on key_cache/value_cache ([NB, B, H, D], float16 or uint8 codes)."""
+                   k_scale: float = 1.0, v_scale: float = 1.0, threads: int | None = None) -> None:
+    """In place on key_cache/value_cache ([NB, B, H, D], float16 or uint8 codes).
+    threads=None runs on the calling thread; threads=n (0: the host's
+    default) spreads each token's row over n OpenMP threads, tokens still in
+    order, with the same result bit for bit."""
     assert key.dtype == np.float16 and value.dtype == np.float16
     nb, bs, nh, hd = key_cache.shape
     n = slot_mapping.shape[0]
@@ -188,10 +193,13 @@ def kv_cache_write(key: np.ndarray, value: np.ndarray, key_cache: np.ndarray,
     assert k2.shape[1] == nh * hd and k2.strides[1] == 2 and v2.strides[1] == 2
     slots = np.ascontiguousarray(slot_mapping, dtype=np.int32)
     lib = _load()
-    rc = lib.oracle_kv_cache_write(
-        k2.ctypes.data, v2.ctypes.data, k2.strides[0] // 2, v2.strides[0] // 2,
-        _ptr(key_cache), _ptr(value_cache), _dtype_code(key_cache), nb, bs, nh, hd,
-        _ptr(slots), n, float(np.float32(k_scale)), float(np.float32(v_scale)))
+    args = (k2.ctypes.data, v2.ctypes.data, k2.strides[0] // 2, v2.strides[0] // 2,
+            _ptr(key_cache), _ptr(value_cache), _dtype_code(key_cache), nb, bs, nh, hd,
+            _ptr(slots), n, float(np.float32(k_scale)), float(np.float32(v_scale)))
+    if threads is None:
+        rc = lib.oracle_kv_cache_write(*args)
+    else:
+        rc = lib.oracle_kv_cache_write_threads(*args, int(threads))
     _check(rc, "kv_cache_write")
 
 

@@ -9,9 +9,11 @@
  *
  * Every floating-point result is computed in double precision with no
  * blocking, fusion or reordering beyond what the definitions below state.
- * The one parallel entry, oracle_paged_attention_threads, only hands whole
- * (sequence, head) pairs to OpenMP threads; each pair runs the same serial
- * code, so its results equal the single-thread call's bit for bit.
+ * The two parallel entries only hand independent work to OpenMP threads:
+ * oracle_paged_attention_threads whole (sequence, head) pairs, and
+ * oracle_kv_cache_write_threads the elements of one token row at a time
+ * (tokens in order). Each item runs the same serial code, so their results
+ * equal the single-thread calls' bit for bit.
  * Sources (each page is cited by its title and section):
  *   [P1] "vLLM-v0.17.1技术解析：PagedAttention内存管理与显存优化技巧"
  *        (cnnetsun.cn/a/1550967), §2.2 PagedAttention的创新设计: block table +
@@ -49,6 +51,17 @@
 
 #define ORACLE_F16 0
 #define ORACLE_E4M3 1
+
+/* Threads an OpenMP region of this library uses by default (1 in a build
+ * without OpenMP, where the threaded calls run on the calling thread). */
+int oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
 
 /* ---------------------------------------------------------------- numbers */
 
@@ -194,6 +207,27 @@ int oracle_prefill_slot_mapping(int32_t *slot_mapping, const int32_t *query_star
  * E4M3 caches take e4m3(fp32(x) / scale), with an IEEE fp32 divide.
  * key/value are fp16 bits, row i at key + i*key_stride (elements).
  * Returns 0, or -1 if a slot is beyond the pool (nothing after it is written). */
+/* Element j of token i's key and value rows into cache row `base`. */
+static void write_element(const uint16_t *key, const uint16_t *value,
+                          int64_t key_stride, int64_t value_stride,
+                          void *key_cache, void *value_cache, int kv_dtype,
+                          int i, int64_t base, int64_t j, float k_scale, float v_scale)
+{
+    uint16_t kb = key[(int64_t)i * key_stride + j];
+    uint16_t vb = value[(int64_t)i * value_stride + j];
+    if (kv_dtype == ORACLE_F16) {
+        ((uint16_t *)key_cache)[base + j] = kb;
+        ((uint16_t *)value_cache)[base + j] = vb;
+    } else {
+        float kf = (float)oracle_f16_to_double(kb);
+        float vf = (float)oracle_f16_to_double(vb);
+        float kq = kf / k_scale;
+        float vq = vf / v_scale;
+        ((uint8_t *)key_cache)[base + j] = oracle_e4m3_from_float(kq);
+        ((uint8_t *)value_cache)[base + j] = oracle_e4m3_from_float(vq);
+    }
+}
+
 int oracle_kv_cache_write(const uint16_t *key, const uint16_t *value,
                           int64_t key_stride, int64_t value_stride,
                           void *key_cache, void *value_cache, int kv_dtype,
@@ -211,23 +245,48 @@ int oracle_kv_cache_write(const uint16_t *key, const uint16_t *value,
         int64_t blk = slot / block_size;
         int64_t off = slot % block_size;
         int64_t base = (blk * block_size + off) * row;
-        for (int64_t j = 0; j < row; ++j) {
-            uint16_t kb = key[(int64_t)i * key_stride + j];
-            uint16_t vb = value[(int64_t)i * value_stride + j];
-            if (kv_dtype == ORACLE_F16) {
-                ((uint16_t *)key_cache)[base + j] = kb;
-                ((uint16_t *)value_cache)[base + j] = vb;
-            } else {
-                float kf = (float)oracle_f16_to_double(kb);
-                float vf = (float)oracle_f16_to_double(vb);
-                float kq = kf / k_scale;
-                float vq = vf / v_scale;
-                ((uint8_t *)key_cache)[base + j] = oracle_e4m3_from_float(kq);
-                ((uint8_t *)value_cache)[base + j] = oracle_e4m3_from_float(vq);
-            }
-        }
+        for (int64_t j = 0; j < row; ++j)
+            write_element(key, value, key_stride, value_stride, key_cache, value_cache,
+                          kv_dtype, i, base, j, k_scale, v_scale);
     }
     return 0;
+}
+
+/* The same cache write with each token's row spread over n_threads OpenMP
+ * threads (n_threads <= 0: the OpenMP default). Tokens are still taken in
+ * order, one after the other, so duplicate slots end as in the serial call
+ * (the later token wins) and the pools are identical to its result, bit for
+ * bit; a slot beyond the pool stops the write at the same token, with the
+ * same status. */
+int oracle_kv_cache_write_threads(const uint16_t *key, const uint16_t *value,
+                                  int64_t key_stride, int64_t value_stride,
+                                  void *key_cache, void *value_cache, int kv_dtype,
+                                  int num_blocks, int block_size, int num_heads,
+                                  int head_size, const int32_t *slot_mapping,
+                                  int n_tokens, float k_scale, float v_scale, int n_threads)
+{
+    int64_t row = (int64_t)num_heads * head_size;
+    int n_ok = n_tokens, status = 0;
+    for (int i = 0; i < n_tokens; ++i)
+        if (slot_mapping[i] >= 0 && (int64_t)slot_mapping[i] >= (int64_t)num_blocks * block_size) {
+            n_ok = i;
+            status = -1;
+            break;
+        }
+    if (n_threads <= 0)
+        n_threads = oracle_max_threads();
+#pragma omp parallel num_threads(n_threads)
+    for (int i = 0; i < n_ok; ++i) {
+        int32_t slot = slot_mapping[i];
+        if (slot < 0)
+            continue;
+        int64_t base = ((int64_t)(slot / block_size) * block_size + slot % block_size) * row;
+#pragma omp for schedule(static)
+        for (int64_t j = 0; j < row; ++j)
+            write_element(key, value, key_stride, value_stride, key_cache, value_cache,
+                          kv_dtype, i, base, j, k_scale, v_scale);
+    }
+    return status;
 }
 
 /* ----------------------------------------------------- block copy (a3) */
@@ -403,17 +462,6 @@ int oracle_paged_attention(double *out, const uint16_t *query,
             return rc;
     }
     return 0;
-}
-
-/* Threads an OpenMP region of this library uses by default (1 in a build
- * without OpenMP, where the threaded call below runs on the calling thread). */
-int oracle_max_threads(void)
-{
-#ifdef _OPENMP
-    return omp_get_max_threads();
-#else
-    return 1;
-#endif
 }
 
 /* The same computation with the (sequence, head) pairs spread over
