@@ -119,17 +119,19 @@ int pa_check_status(void *stream, uint32_t *code);
 /* Test hook for the bounded on-chip waits (the pages have no counterpart:
  * it exists so that a test can make one wait run out on purpose). The next
  * decode this thread launches (pa_paged_attention_decode, _ws, _append,
- * _shared_prefix or _noalloc) issues no tile loads for its work unit `unit`
- * and gives each of its pipeline waits wait_limit_ns of wall time instead
- * of 2 s. Units are numbered with the context partition fastest, then the
- * head group, then the sequence; unit 0 is partition 0 of heads
- * 0..heads_per_cta-1 of sequence 0. The consumer warps of that unit give
- * up at the limit, set PA_DEV_WAIT_TIMEOUT and return; the output rows of
- * that unit are then undefined, everything else is computed as usual, and
- * no copy or wait is left pending. Later launches are unaffected.
- * unit < 0 clears a pending request. Returns PA_OK, or PA_ERR_INVALID for
- * wait_limit_ns outside [1000, 2000000000]. */
-int pa_test_stall_next_decode(int64_t unit, uint64_t wait_limit_ns);
+ * _shared_prefix or _noalloc) issues no tile loads for the work unit that
+ * holds head `head` of sequence `seq` in context partition `partition`
+ * (partition p covers the tokens from p * partition_size, counted after a
+ * shared prefix; see pa_decode_choose_config), and gives each of its
+ * pipeline waits wait_limit_ns of wall time instead of 2 s. If that unit
+ * has tokens, its consumer warps give up at the limit, set
+ * PA_DEV_WAIT_TIMEOUT and return; its output rows are then undefined,
+ * everything else is computed as usual, and no copy or wait is left
+ * pending. A unit without tokens, or a (seq, head, partition) outside the
+ * launch, stalls nothing. The request is consumed by the next decode
+ * launch; seq < 0 clears it. Returns PA_OK, or PA_ERR_INVALID for a
+ * negative head or partition or wait_limit_ns outside [1000, 2000000000]. */
+int pa_test_stall_next_decode(int seq, int head, int partition, uint64_t wait_limit_ns);
 
 /* ---------------------------------------------------------------- a1
  * Slot of the token each sequence appends in a decode step ([P3] §2.2 slot
@@ -208,7 +210,8 @@ int pa_swap_blocks(void *dst_key_cache, void *dst_value_cache, int dst_num_block
  * a normalised partial output and its log-sum-exp, and a second kernel
  * combines them. The workspace for those partials is owned by the library:
  * one buffer per (device, stream), grown with cudaMallocAsync on `stream`
- * and never shrunk. It is not allocated when no sequence can span more than
+ * and never shrunk; an outgrown buffer is kept (not freed), so a CUDA graph
+ * captured before the growth still replays into valid memory. It is not allocated when no sequence can span more than
  * one partition. Issue a first call with the largest shapes before
  * capturing a CUDA graph so that capture does not need to grow it. */
 int pa_paged_attention_decode(void *out, const void *query,
@@ -279,7 +282,13 @@ int pa_paged_attention_decode_append(void *out, const void *query, const void *n
  * that differs sets PA_DEV_PREFIX. Each shared tile is read once per head
  * and applied to up to 16 sequences' queries; the private rest of every
  * context is decoded as in pa_paged_attention_decode; a log-sum-exp
- * reduction merges both (three launches). Results equal
+ * reduction merges both (three launches). The prefix kernel runs on a
+ * second stream of the library's (one per device and caller stream, made
+ * on the first call: make that call before any stream capture), forked
+ * from `stream` after everything already queued there and joined back
+ * before the reduce, so it overlaps the private-part decode while the call
+ * keeps its place in the order of `stream` (a graph captured on `stream`
+ * holds both branches). Results equal
  * pa_paged_attention_decode (or _append when new_key is given) on the same
  * tables. With new_key/new_value (both or neither), each sequence's new
  * token must lie after the prefix (L > n * block_size), else it is not

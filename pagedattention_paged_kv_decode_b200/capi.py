@@ -54,7 +54,7 @@ SIGNATURES = {
     "pa_version": (_I, []),
     "pa_last_error": (ctypes.c_char_p, []),
     "pa_check_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
-    "pa_test_stall_next_decode": (_I, [_I64, ctypes.c_uint64]),
+    "pa_test_stall_next_decode": (_I, [_I, _I, _I, ctypes.c_uint64]),
     "pa_slot_mapping": (_I, [_P, _P, _I, _P, _I, CacheDesc, _P]),
     "pa_kv_cache_write": (_I, [_P, _P, _I64, _I64, _P, _P, CacheDesc, _P, _I, _F, _F, _P]),
     "pa_copy_blocks": (_I, [_P, _P, CacheDesc, _P, _I, _P]),

@@ -319,6 +319,36 @@ int ctas_per_sm(const void *fn, int threads, size_t smem, int *out) {
     return PA_OK;
 }
 
+// ---------------------------------------------- second stream (shared prefix)
+
+// One non-blocking stream and two events per (device, caller stream), made
+// on first use and kept for the life of the process.
+struct SideStream {
+    int device;
+    cudaStream_t caller;
+    cudaStream_t stream;
+    cudaEvent_t fork, join;
+};
+std::mutex g_side_mu;
+std::vector<SideStream> g_side;
+
+int side_stream(cudaStream_t st, int device, SideStream *out) {
+    std::lock_guard<std::mutex> lk(g_side_mu);
+    for (const auto &e : g_side)
+        if (e.device == device && e.caller == st) {
+            *out = e;
+            return PA_OK;
+        }
+    SideStream s{device, st, nullptr, nullptr, nullptr};
+    cudaError_t e = cudaStreamCreateWithFlags(&s.stream, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming);
+    if (e != cudaSuccess) return cuda_fail(e, "second stream for the shared prefix");
+    g_side.push_back(s);
+    *out = s;
+    return PA_OK;
+}
+
 // ---------------------------------------------- internal split workspace
 
 struct WsEntry {
@@ -329,6 +359,11 @@ struct WsEntry {
 };
 std::mutex g_ws_mu;
 std::vector<WsEntry> g_ws;
+// Outgrown workspaces are kept, not freed: a CUDA graph captured before a
+// workspace grew still holds the old address, and replaying it must not
+// touch freed memory. Growth is by at least 1.25x, so the kept buffers add
+// up to at most about four times the current one.
+std::vector<void *> g_ws_retired;
 
 int internal_workspace(size_t need, cudaStream_t st, int device, void **out) {
     std::lock_guard<std::mutex> lk(g_ws_mu);
@@ -344,8 +379,7 @@ int internal_workspace(size_t need, cudaStream_t st, int device, void **out) {
     cudaError_t e = cudaMallocAsync(&p, bytes, st);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync (split workspace)");
     if (ent) {
-        e = cudaFreeAsync(ent->ptr, st);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync (split workspace)");
+        g_ws_retired.push_back(ent->ptr);
         ent->ptr = p;
         ent->bytes = bytes;
     } else {
@@ -400,7 +434,7 @@ struct PrefixPlan {
 // pa_test_stall_next_decode: consumed (and cleared) by the next decode
 // launch of this thread.
 struct StallRequest {
-    int64_t unit = -1;
+    int seq = -1, head = 0, partition = 0;
     uint64_t wait_limit_ns = 0;
 };
 thread_local StallRequest g_stall;
@@ -470,10 +504,18 @@ int launch_decode(void *out, const void *query, const void *kc, const void *vc,
         p.v_scale = fp8 ? v_scale : 1.0f;
     }
 
-    if (g_stall.unit >= 0) {
-        p.stall_unit_plus1 = g_stall.unit + 1;
-        p.wait_limit_ns = g_stall.wait_limit_ns;
+    if (g_stall.seq >= 0) {
+        // the unit holding (seq, head, partition), numbered as unit_coord does
+        // in the kernel: partition slowest (highest first), then sequence,
+        // then head group
+        const StallRequest r = g_stall;
         g_stall = StallRequest{};
+        if (r.seq < S && r.head < c.num_heads && r.partition < parts) {
+            const int64_t hg_count = c.num_heads / G;
+            const int64_t unit = ((int64_t)(parts - 1 - r.partition) * S + r.seq) * hg_count + r.head / G;
+            p.stall_unit_plus1 = unit + 1;
+            p.wait_limit_ns = r.wait_limit_ns;
+        }
     }
 
     const int C = cfg.units_per_cta;
@@ -496,30 +538,44 @@ int launch_decode(void *out, const void *query, const void *kc, const void *vc,
         if (narrow_ctas > wide_ctas) kern = narrow;
     }
     cudaError_t e;
+    // Shared prefix: the prefix kernel runs on a second stream beside the
+    // decode of the private parts (the two write disjoint partials; the
+    // prefix kernel reads only the shared blocks). The second stream waits
+    // for everything before this call on `st`, and `st` waits for it before
+    // the reduce, so the call keeps its place in the caller's stream order
+    // (and a CUDA graph captured on `st` takes both branches).
+    DecodeKernel pkern = nullptr;
+    CUtensorMap pk_, pv_;
+    pa::DecodeParams pp = p;
+    int64_t pn = 0;
+    size_t psmem = 0;
+    int pthreads = 0;
+    SideStream side{};
     if (pre) {
-        DecodeKernel pkern = pre->mma ? pick_prefix_mma(D, B) : pick_prefix(D, B, fp8);
+        pkern = pre->mma ? pick_prefix_mma(D, B) : pick_prefix(D, B, fp8);
         rc = ensure_smem_attr(reinterpret_cast<const void *>(pkern), device);
         if (rc) return rc;
-        CUtensorMap pk_, pv_;
         rc = cache_tensor_map(kc, c, pre->heads, &pk_, pre->mma ? 1 : 0);
         if (rc) return rc;
         rc = cache_tensor_map(vc, c, pre->heads, &pv_, pre->mma ? 1 : 0);
         if (rc) return rc;
-        pa::DecodeParams pp = p;
         pp.heads_per_cta = pre->heads;
         pp.stages = pre->stages;
         const int64_t n_qb = (S + pre->queries - 1) / pre->queries;
-        const int64_t n = (int64_t)(c.num_heads / pre->heads) * pre->parts * n_qb;
+        pn = (int64_t)(c.num_heads / pre->heads) * pre->parts * n_qb;
         if (pre->mma) {
             // ring + barriers + 1 KiB to align the ring to 1024 bytes in the kernel
-            const size_t smem_bytes = (size_t)pre->stages * 4 * B * D + 16 * (size_t)pre->stages + 1024;
-            pkern<<<dim3((unsigned)n), dim3(32 * 5), smem_bytes, st>>>(pk_, pv_, pp);
+            psmem = (size_t)pre->stages * 4 * B * D + 16 * (size_t)pre->stages + 1024;
+            pthreads = 32 * 5;
         } else {
-            const pa::SmemLayout play(B, pre->heads, D, elem_bytes(c), 1, pre->stages, 1);
-            pkern<<<dim3((unsigned)n), dim3(32 * (pre->heads * pre->queries + 1)), play.total, st>>>(pk_, pv_, pp);
+            psmem = pa::SmemLayout(B, pre->heads, D, elem_bytes(c), 1, pre->stages, 1).total;
+            pthreads = 32 * (pre->heads * pre->queries + 1);
         }
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return cuda_fail(e, "paged_prefix_kernel launch");
+        rc = side_stream(st, device, &side);
+        if (rc) return rc;
+        e = cudaEventRecord(side.fork, st);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(side.stream, side.fork, 0);
+        if (e != cudaSuccess) return cuda_fail(e, "shared-prefix stream fork");
     }
     // Every unit u is served by CTA u % grid, slot u / grid: grid * C >= units.
     // Packed CTAs are spread over all SMs (some slots of the last ones idle).
@@ -533,6 +589,14 @@ int launch_decode(void *out, const void *query, const void *kc, const void *vc,
     kern<<<grid, block, lay.total, st>>>(mk, mv, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "paged_decode_kernel launch");
+    if (pre) {
+        pkern<<<dim3((unsigned)pn), dim3(pthreads), psmem, side.stream>>>(pk_, pv_, pp);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "paged_prefix_kernel launch");
+        e = cudaEventRecord(side.join, side.stream);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(st, side.join, 0);
+        if (e != cudaSuccess) return cuda_fail(e, "shared-prefix stream join");
+    }
     if (ws_parts > 1 || pre) {
         pick_reduce(D)<<<dim3((c.num_heads + 3) / 4, S), 128, 0, st>>>(p);
         e = cudaGetLastError();
@@ -555,15 +619,19 @@ int pa_version(void) { return 202; }
 
 const char *pa_last_error(void) { return g_msg; }
 
-int pa_test_stall_next_decode(int64_t unit, uint64_t wait_limit_ns) {
-    if (unit < 0) {
+int pa_test_stall_next_decode(int seq, int head, int partition, uint64_t wait_limit_ns) {
+    if (seq < 0) {
         g_stall = StallRequest{};
         return ok();
     }
+    if (head < 0 || partition < 0)
+        return fail(PA_ERR_INVALID, "head %d and partition %d must be >= 0", head, partition);
     if (wait_limit_ns < 1000 || wait_limit_ns > pa::kWaitLimitNs)
         return fail(PA_ERR_INVALID, "wait_limit_ns %llu outside [1000, %llu]",
                     (unsigned long long)wait_limit_ns, (unsigned long long)pa::kWaitLimitNs);
-    g_stall.unit = unit;
+    g_stall.seq = seq;
+    g_stall.head = head;
+    g_stall.partition = partition;
     g_stall.wait_limit_ns = wait_limit_ns;
     return ok();
 }

@@ -323,9 +323,31 @@ struct SmemLayout {
 
 // One work unit: sequence s, heads h0 .. h0+G-1, partition `part` of the
 // context (tokens t0 .. t1-1 in physical blocks blk0 .. blk0+nblk-1 of the
-// table row). Units are numbered with the partition fastest, then the head
-// group, then the sequence; CTA c serves units c, c + gridDim.x, ... (one per
-// slot), so neighbouring units land on different CTAs.
+// table row). CTA c serves units c, c + gridDim.x, ... (one per slot).
+//
+// Units are numbered with the partition slowest and the highest partition
+// first, then the sequence, then the head group. The highest partitions
+// exist only for the longest contexts, so the grid starts with their (full)
+// partitions and ends with partition 0 of every sequence, the short
+// contexts' only work: long work first, short work last, without knowing
+// the lengths on the host. Units of a partition beyond a context's length
+// exit at once. Neighbouring CTAs take the head groups of one sequence, so
+// together they read whole token rows of its blocks.
+struct UnitCoord {
+    int s, hg, part;
+};
+
+__device__ __forceinline__ UnitCoord unit_coord(const DecodeParams &p, uint32_t id) {
+    // unit ids fit 32 bits: the host keeps num_units below 2^31
+    const uint32_t HG = (uint32_t)(p.num_heads / p.heads_per_cta);
+    const uint32_t per_part = (uint32_t)p.num_seqs * HG;
+    UnitCoord c;
+    c.part = p.max_parts - 1 - (int)(id / per_part);
+    const uint32_t r = id % per_part;
+    c.s = (int)(r / HG);
+    c.hg = (int)(r % HG);
+    return c;
+}
 struct Unit {
     int s, h0, part;
     int L_in, L;       // context length as given and as clamped to the table and bound
@@ -340,14 +362,11 @@ __device__ __forceinline__ Unit unit_of(const DecodeParams &p, int B, int j) {
     // unit ids fit 32 bits: the host keeps num_units below 2^31, and C * grid
     // stays below 2^32 for every C
     const uint32_t id = blockIdx.x + (uint32_t)j * gridDim.x;
-    const uint32_t HG = (uint32_t)(p.num_heads / p.heads_per_cta);
     const bool exists = (int64_t)id < p.num_units;
-    const uint32_t idc = exists ? id : 0u;
-    const uint32_t mp = (uint32_t)p.max_parts;
-    u.part = (int)(idc % mp);
-    const uint32_t rest = idc / mp;
-    u.h0 = (int)(rest % HG) * p.heads_per_cta;
-    u.s = (int)(rest / HG);
+    const UnitCoord c = unit_coord(p, exists ? id : 0u);
+    u.part = c.part;
+    u.h0 = c.hg * p.heads_per_cta;
+    u.s = c.s;
     u.L_in = exists ? __ldg(p.context_lens + u.s) : 0;
     int L = min(u.L_in, p.max_blocks_per_seq * B);
     L = min(L, p.max_context_len);
@@ -403,11 +422,10 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
             if (j < C) {
                 const uint32_t id = blockIdx.x + (uint32_t)j * gridDim.x;
                 if ((int64_t)id < p.num_units) {
-                    const int part = (int)(id % (uint32_t)p.max_parts);
-                    const int s = (int)(id / (uint32_t)p.max_parts / (uint32_t)(p.num_heads / G));
-                    const int e = (p.prefix_tokens + part * p.partition_size) / B + lane;
+                    const UnitCoord c = unit_coord(p, id);
+                    const int e = (p.prefix_tokens + c.part * p.partition_size) / B + lane;
                     if (e < p.max_blocks_per_seq)
-                        pre_blk[j] = __ldg(p.block_tables + (size_t)s * p.max_blocks_per_seq + e);
+                        pre_blk[j] = __ldg(p.block_tables + (size_t)c.s * p.max_blocks_per_seq + e);
                 }
             }
         }
@@ -527,10 +545,9 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
     uint4 q_raw[EPL / 8], nk_raw[EPL / 8], nv_raw[EPL / 8];
     {
         const uint32_t id = blockIdx.x + (uint32_t)slot * gridDim.x;
-        const uint32_t idc = (int64_t)id < p.num_units ? id : 0u;
-        const uint32_t rest = idc / (uint32_t)p.max_parts;
-        const int hq = (int)(rest % (uint32_t)(p.num_heads / G)) * G + g;
-        const int sq = (int)(rest / (uint32_t)(p.num_heads / G));
+        const UnitCoord c = unit_coord(p, (int64_t)id < p.num_units ? id : 0u);
+        const int hq = c.hg * G + g;
+        const int sq = c.s;
         const uint4 *qp = reinterpret_cast<const uint4 *>(p.query + ((size_t)sq * p.num_heads + hq) * D);
 #pragma unroll
         for (int c = 0; c < EPL / 8; ++c) q_raw[c] = __ldg(qp + sub * (EPL / 8) + c);
@@ -732,7 +749,8 @@ lse_reduce_kernel(const DecodeParams p) {
 #pragma unroll
     for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
     float wsum = 0.f;
-    for (int i = 0; i < n_parts; ++i) {
+#pragma unroll 4
+    for (int i = 0; i < n_parts; ++i) {  // unrolled: several partials' loads in flight at once
         const float wgt = fast_exp2(p.ws_lse[base + i] - M);
         wsum += wgt;
         const float *o = p.ws_o + (base + i) * D + lane * DPL;

@@ -392,14 +392,18 @@ def version() -> int:
     return int(lib().pa_version())
 
 
-def test_stall_next_decode(unit: int, wait_limit_ns: int) -> None:
+def test_stall_next_decode(seq: int, head: int = 0, partition: int = 0, wait_limit_ns: int = 1_000_000) -> None:
     """Test hook of the bounded waits: the next decode launched on this
-    thread issues no tile loads for work unit `unit` and limits each wait to
-    wait_limit_ns (that unit then reports PA_DEV_WAIT_TIMEOUT; its output
-    rows are undefined). unit < 0 clears a pending request."""
-    if int(unit) >= 0 and not 1000 <= int(wait_limit_ns) <= 2_000_000_000:
-        raise ValueError(f"wait_limit_ns {wait_limit_ns} outside [1000, 2e9]")
-    check(lib().pa_test_stall_next_decode(int(unit), int(wait_limit_ns)))
+    thread issues no tile loads for the work unit holding (seq, head,
+    partition) and limits each wait to wait_limit_ns; that unit then reports
+    PA_DEV_WAIT_TIMEOUT and its output rows are undefined. seq < 0 clears a
+    pending request."""
+    if int(seq) >= 0:
+        if int(head) < 0 or int(partition) < 0:
+            raise ValueError(f"head {head} and partition {partition} must be >= 0")
+        if not 1000 <= int(wait_limit_ns) <= 2_000_000_000:
+            raise ValueError(f"wait_limit_ns {wait_limit_ns} outside [1000, 2e9]")
+    check(lib().pa_test_stall_next_decode(int(seq), int(head), int(partition), int(wait_limit_ns)))
 
 
 def last_error() -> str:

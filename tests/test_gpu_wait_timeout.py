@@ -2,9 +2,9 @@
 
 Every mbarrier wait of the decode kernel has a wall-time limit. Here the
 test hook pa_test_stall_next_decode makes the next decode's producer issue
-no tile loads for one work unit and shortens the limit to 1 ms: that unit's
-consumer warps must give up, set PA_DEV_WAIT_TIMEOUT in the device error
-word and return. The call must end well inside a second (not the default
+no tile loads for the work unit holding one (sequence, head, partition) and
+shortens the limit to 1 ms: that unit's consumer warps must give up, set
+PA_DEV_WAIT_TIMEOUT in the device error word and return. The call must end well inside a second (not the default
 2 s limit, and never hang), and the very next decode on the same device
 must match the oracle with a clean error word.
 """
@@ -48,8 +48,9 @@ def test_stalled_unit_times_out_and_the_next_decode_is_clean(cuda_device, kv, la
 
     step()  # loads the kernels and sizes the workspace outside the timed calls
     assert pk.check_status() == 0
-    for unit in (0, 2):   # sequence 0, first partition / a later unit of the grid
-        pk.test_stall_next_decode(unit, 1_000_000)
+    # sequence 0 (200 tokens): its first partition, and a later one of another head
+    for seq, head, part in ((0, 0, 0), (0, 1, 2)):
+        pk.test_stall_next_decode(seq, head, part, 1_000_000)
         t0 = time.perf_counter()
         step()
         code = pk.check_status()
@@ -66,12 +67,20 @@ def test_stalled_unit_times_out_and_the_next_decode_is_clean(cuda_device, kv, la
     assert np.abs(got - out_ref).max() <= (2e-3 if kv == "f16" else 1e-2)
 
 
-def test_cleared_request_stalls_nothing(cuda_device):
+@pytest.mark.parametrize("request_", ["cleared", "empty unit", "outside the launch"])
+def test_requests_that_stall_nothing(cuda_device, request_):
     w = _case("f16", seed=32)
     dw = W.to_device(w, cuda_device)
-    pk.test_stall_next_decode(0, 1_000_000)
-    pk.test_stall_next_decode(-1, 0)
+    if request_ == "cleared":
+        pk.test_stall_next_decode(0, 0, 0, 1_000_000)
+        pk.test_stall_next_decode(-1)
+    elif request_ == "empty unit":
+        pk.test_stall_next_decode(4, 0, 0, 1_000_000)      # sequence 4 has no tokens
+    else:
+        pk.test_stall_next_decode(0, 0, 1000, 1_000_000)   # no such partition
     pk.decode_step(dw.out, dw.query, dw.new_key, dw.new_value, dw.key_cache, dw.value_cache,
                    dw.block_tables, dw.context_lens, w.scale, slots=dw.slots,
                    max_context_len=w.max_context_len)
     assert pk.check_status() == 0
+    _, _, _, out_ref, _ = oracle_step(w)
+    assert np.abs(dw.out.cpu().numpy().astype(np.float64) - out_ref).max() <= 2e-3
