@@ -281,6 +281,39 @@ struct HeadAttn {
         }
     }
 
+    // One tile whose V rows at or past `valid` hold zeros (the caller wrote
+    // them): the logits are masked, the P.V loop runs over every row.
+    __device__ __forceinline__ void consume_v_zeroed(const unsigned char *ktile, const unsigned char *vtile,
+                                                     size_t row_stride, size_t head_off, int valid,
+                                                     float qk_mul, int lane) {
+        const int grp = lane / LPR, sub = lane % LPR;
+        float part_dot[TPG];
+#pragma unroll
+        for (int j = 0; j < TPG; ++j) {
+            const int t = grp * TPG + j;
+            part_dot[j] = dot16(*reinterpret_cast<const uint4 *>(ktile + t * row_stride + head_off));
+        }
+        const int my_t = grp * TPG + sub / DUP;
+        float z = butterfly_reduce<TPG, LPR>(part_dot, lane) * qk_mul;
+        z = (my_t < valid) ? z : -INFINITY;
+        if (__any_sync(0xffffffffu, z > m + kLazyMax)) {
+            const float m_new = fmaxf(m, warp_max(z));
+            const float alpha = fast_exp2(m - m_new);
+            l *= alpha;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) acc[e] *= alpha;
+            m = m_new;
+        }
+        const uint32_t p1 = f32_to_f16_bits(fast_exp2(z - m));
+        l = add_f16_f32(p1, l);
+#pragma unroll
+        for (int j = 0; j < TPG; ++j) {
+            const int t = grp * TPG + j;
+            const uint32_t pj = __shfl_sync(0xffffffffu, p1, grp * LPR + j * DUP);
+            axpy16(pj, *reinterpret_cast<const uint4 *>(vtile + t * row_stride + head_off));
+        }
+    }
+
     __device__ __forceinline__ void consume(const unsigned char *ktile, const unsigned char *vtile,
                                             size_t row_stride, size_t head_off, int valid, float qk_mul,
                                             int lane) {
@@ -643,7 +676,19 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
             __syncwarp();
         }
-        st.consume(ktile, vtile, row_stride, head_off, valid, qk_mul, lane);
+        // The context ends inside this block: zero this head's V rows past it
+        // (they may hold anything, NaN included), so that one P.V loop serves
+        // every tile; the logits of those rows are masked.
+        if (valid < B) {
+#pragma unroll
+            for (int j = 0; j < Geo::TPG; ++j) {
+                const int t = grp * Geo::TPG + j;
+                if (t >= valid) *reinterpret_cast<uint4 *>(vtile + t * row_stride + head_off) = make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+        }
+        st.consume_v_zeroed(ktile, vtile, row_stride, head_off, valid, qk_mul, lane);
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[stage]);
         stage += W;
