@@ -502,6 +502,12 @@ def run_ours(args, rank, world, local_rank):
         dist.destroy_process_group()
     if rank != 0:
         return
+    print(json.dumps(assemble_line(results, args, world)), flush=True)
+
+
+def assemble_line(results, args, world):
+    """The JSON line: the first workload's result at the top level (the
+    contract's keys first), the others under "workloads" by name."""
     head = results[0]
     line = {
         "metric": METRIC,
@@ -521,7 +527,7 @@ def run_ours(args, rank, world, local_rank):
         line["workloads"] = {r["config"]["workload"]: {k: v for k, v in r.items() if k != "metric"}
                              for r in results[1:]}
         line["gpu_launches_all_workloads"] = sum(r["gpu_launches"] for r in results)
-    print(json.dumps(line), flush=True)
+    return line
 
 
 def measure_swap(pk, dw, stream, torch, n_blocks: int = 256, reps: int = 5):

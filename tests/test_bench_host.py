@@ -129,3 +129,26 @@ def test_unique_bytes_count_shared_blocks_once():
     shared = w.shared_blocks * w.block_size
     assert w.unique_kv_bytes() == (int((w.context_lens - shared).sum()) + shared) * row
     assert w.unique_kv_bytes() < w.kv_bytes()
+
+
+def test_line_puts_the_first_workload_on_top_and_the_rest_beside_it():
+    import argparse
+    args = argparse.Namespace(steps=20, warmup=5)
+
+    def result(name, value, launches):
+        return {"metric": bench.METRIC, "value": value, "unit": "GB/s", "ms_per_step": 0.1, "dtype": "f32",
+                "config": {"workload": name}, "roofline": {"frac": 0.9}, "e2e": {"value": 1.0},
+                "gpu_launches": launches, "clocks": {}, "cpu_baseline": {"cores": 16}}
+
+    line = bench.assemble_line([result("w3", 6000.0, 40), result("w2", 1500.0, 20), result("w5", 5500.0, 40)],
+                               args, 1)
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches",
+                "clocks", "cpu_baseline"):
+        assert key in line, key
+    assert line["config"]["workload"] == "w3" and line["value"] == 6000.0 and line["n_gpus"] == 1
+    assert list(line["workloads"]) == ["w2", "w5"]
+    assert line["workloads"]["w5"]["value"] == 5500.0 and "metric" not in line["workloads"]["w5"]
+    assert line["gpu_launches"] == 40 and line["gpu_launches_all_workloads"] == 100
+    one = bench.assemble_line([result("w3", 6000.0, 40)], args, 2)
+    assert "workloads" not in one and one["n_gpus"] == 2
