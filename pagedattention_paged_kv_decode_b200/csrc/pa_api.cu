@@ -598,8 +598,19 @@ int launch_decode(void *out, const void *query, const void *kc, const void *vc,
         if (e != cudaSuccess) return cuda_fail(e, "shared-prefix stream join");
     }
     if (ws_parts > 1 || pre) {
-        pick_reduce(D)<<<dim3((c.num_heads + 3) / 4, S), 128, 0, st>>>(p);
-        e = cudaGetLastError();
+        // programmatic dependent launch: the reduce is scheduled while the
+        // partition kernel drains and waits for it on the device
+        cudaLaunchConfig_t lc = {};
+        lc.gridDim = dim3((c.num_heads + 3) / 4, S);
+        lc.blockDim = dim3(128);
+        lc.dynamicSmemBytes = 0;
+        lc.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        lc.attrs = attr;
+        lc.numAttrs = 1;
+        e = cudaLaunchKernelEx(&lc, pick_reduce(D), p);
         if (e != cudaSuccess) return cuda_fail(e, "lse_reduce_kernel launch");
     }
     return ok();

@@ -443,6 +443,9 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int per_slot = G * W;
     const int n_consumers = C * per_slot;
     const uint64_t wait_limit = p.wait_limit_ns ? p.wait_limit_ns : kWaitLimitNs;
+    // A dependent reduce may be scheduled once every CTA of this grid runs
+    // (it waits for this grid's completion before touching its partials).
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     if (warp == n_consumers) {
         // ================================================================ producer
@@ -781,6 +784,9 @@ lse_reduce_kernel(const DecodeParams p) {
     constexpr int DPL = D / 32;  // dims per lane
     __half *op = p.out + ((size_t)s * p.num_heads + h) * D + lane * DPL;
     if (p.prefix_tokens == 0 && n_parts <= 1) return;  // written by the partition kernel
+    // Launched as a programmatic dependent of the partition kernel: wait for
+    // it (and its memory) before reading partials or writing the output.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     if (L == 0) {
 #pragma unroll
         for (int e = 0; e < DPL; e += 2) *reinterpret_cast<__half2 *>(op + e) = __floats2half2_rn(0.f, 0.f);
