@@ -15,13 +15,15 @@
 //     full/empty mbarriers, a ring-full per slot first, then in turn;
 //   * G x W consumer warps: warp (g, w) owns head g and every W-th block of
 //     the partition. Per block it forms the logits with 16-byte shared loads
-//     (fp16 caches: fp32 FMAs; E4M3: decoded pairs in packed f16x2 products,
-//     summed into fp32), reduces them with a transposing butterfly (one
-//     shuffle per token per lane), runs the online-softmax update and
-//     accumulates P.V in fp32 registers;
+//     (exact fp16 x fp16 products summed in fp32; E4M3 codes are first
+//     decoded exactly to fp16 pairs), reduces them with a transposing
+//     butterfly (one shuffle per token per lane), runs the online-softmax
+//     update with a lazily moved maximum and accumulates P.V in fp32;
+//   * units are numbered long partitions first (see unit_coord);
 //   * the W warps of a head merge (m, l, acc) through shared memory; a
 //     sequence that fits one partition writes fp16 output directly, longer
-//     ones write (lse, normalised o) for the log-sum-exp reduce kernel.
+//     ones write (lse, normalised o) for the log-sum-exp reduce kernel, which
+//     is launched as a programmatic dependent of this one.
 // The plain decode is not a dense contraction (one query row per head), so
 // it runs on the CUDA cores and is bound by HBM bandwidth. The shared-prefix
 // kernels further down are where one K/V tile meets many query rows (every
