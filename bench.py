@@ -395,13 +395,14 @@ def measure_decode(args, wid, rank, world, local_rank, dist, cpu_seconds, with_s
             host_out.copy_(dw.out, non_blocking=True)
         stream.synchronize()
         e2e_ms = []
-        for i in range(max(3, args.warmup) + args.steps):
+        e2e_warm = max(20, args.warmup)  # untimed: the first replays of a new graph with host copies run slow
+        for i in range(e2e_warm + args.steps):
             evict_l2()
             e2e_start.record()
             e2e_graph.replay()
             e2e_end.record()
             stream.synchronize()
-            if i >= max(3, args.warmup):
+            if i >= e2e_warm:
                 e2e_ms.append(e2e_start.elapsed_time(e2e_end))
 
         # ------------------------------------------------ swap to/from pinned host memory
@@ -769,13 +770,14 @@ def run_prefill(args, rank, world, local_rank):
             host_out.copy_(dp.out, non_blocking=True)
         stream.synchronize()
         e2e_ms = []
-        for i in range(max(3, args.warmup) + min(args.steps, 200)):
+        e2e_warm = max(20, args.warmup)  # untimed: the first replays of a new graph with host copies run slow
+        for i in range(e2e_warm + min(args.steps, 200)):
             evict_l2()
             e0.record()
             e2e_graph.replay()
             e1.record()
             stream.synchronize()
-            if i >= max(3, args.warmup):
+            if i >= e2e_warm:
                 e2e_ms.append(e0.elapsed_time(e1))
 
     step_t, att_t, e2e_t = slowest_rank([statistics.mean(step_ms), statistics.mean(att_ms),
