@@ -30,6 +30,8 @@
 // sequence of the batch); the fp16 one computes that on tensor cores.
 #pragma once
 
+#include <type_traits>
+
 #include "pa_device.cuh"
 
 namespace pa {
@@ -795,30 +797,48 @@ lse_reduce_kernel(const DecodeParams p) {
         return;
     }
     const size_t base = ((size_t)s * p.num_heads + h) * p.ws_parts;
-    float M = -INFINITY;
-    for (int i = lane; i < n_parts; i += 32) M = fmaxf(M, p.ws_lse[base + i]);
+    // The partials' loads go out together, in chunks of kChunk, the first
+    // chunk with the log-sum-exps: lane i of the warp holds the weight of
+    // partial c0 + i of each 32-wide group, the others take it by shuffle.
+    using Vec = typename std::conditional<DPL == 4, float4, float2>::type;
+    constexpr int kChunk = 16;
+    Vec v[kChunk];
+    auto load_chunk = [&](int c0) {
+#pragma unroll
+        for (int k = 0; k < kChunk; ++k) {
+            const int i = c0 + k;
+            if (i < n_parts) v[k] = *reinterpret_cast<const Vec *>(p.ws_o + (base + i) * D + lane * DPL);
+            else v[k] = Vec{};
+        }
+    };
+    load_chunk(0);
+    const float lse0 = lane < n_parts ? p.ws_lse[base + lane] : -INFINITY;
+    float M = lse0;
+    for (int i = lane + 32; i < n_parts; i += 32) M = fmaxf(M, p.ws_lse[base + i]);
     M = warp_max(M);
+    float wl = fast_exp2(lse0 - M);  // lanes past the partials: 0
+    float wsum = wl;
     float acc[DPL];
 #pragma unroll
     for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-    float wsum = 0.f;
-#pragma unroll 4
-    for (int i = 0; i < n_parts; ++i) {  // unrolled: several partials' loads in flight at once
-        const float wgt = fast_exp2(p.ws_lse[base + i] - M);
-        wsum += wgt;
-        const float *o = p.ws_o + (base + i) * D + lane * DPL;
-        if constexpr (DPL == 4) {
-            const float4 v = *reinterpret_cast<const float4 *>(o);
-            acc[0] = fmaf(wgt, v.x, acc[0]);
-            acc[1] = fmaf(wgt, v.y, acc[1]);
-            acc[2] = fmaf(wgt, v.z, acc[2]);
-            acc[3] = fmaf(wgt, v.w, acc[3]);
-        } else {
-            const float2 v = *reinterpret_cast<const float2 *>(o);
-            acc[0] = fmaf(wgt, v.x, acc[0]);
-            acc[1] = fmaf(wgt, v.y, acc[1]);
+    for (int c0 = 0; c0 < n_parts; c0 += kChunk) {
+        if (c0 > 0) {
+            load_chunk(c0);
+            if ((c0 & 31) == 0) {
+                const int i = c0 + lane;
+                wl = fast_exp2((i < n_parts ? p.ws_lse[base + i] : -INFINITY) - M);
+                wsum += wl;
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < kChunk; ++k) {
+            const float wgt = __shfl_sync(0xffffffffu, wl, (c0 + k) & 31);  // 0 past the partials
+            const float *x = reinterpret_cast<const float *>(&v[k]);
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) acc[e] = fmaf(wgt, x[e], acc[e]);
         }
     }
+    wsum = warp_sum(wsum);
     const float f = p.out_scale / wsum;
 #pragma unroll
     for (int e = 0; e < DPL; e += 2)
