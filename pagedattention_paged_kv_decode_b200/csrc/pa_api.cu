@@ -146,7 +146,11 @@ constexpr int kNumSMs = 148;
 constexpr int kMaxGridY = 65535;  // grid y extent: token and pair counts are launched in slices of this
 constexpr size_t kMaxSmem = 227 * 1024;
 
-int fill_config(const pa_cache_desc &c, int num_seqs, int max_ctx, pa_decode_config *cfg) {
+// `beside`: CTAs of a kernel that runs next to this decode (the shared-prefix
+// kernel on its second stream). They keep SMs busy too, so the decode needs
+// fewer, longer units of its own.
+int fill_config(const pa_cache_desc &c, int num_seqs, int max_ctx, pa_decode_config *cfg,
+                int64_t beside = 0) {
     const int H = c.num_heads, B = c.block_size;
     pa_decode_config r = *cfg;
     auto stage_bytes = [&](int G) {
@@ -159,18 +163,23 @@ int fill_config(const pa_cache_desc &c, int num_seqs, int max_ctx, pa_decode_con
     // contexts of 16x32x<=178, 64x40x<=2048, 32x32x<=4096, 256x32x<=4096):
     // about four consumer warps per CTA, a ring of about 64 KiB so that three
     // or more CTAs share an SM, enough CTAs for every SM, and long partitions
-    // only when the grid stays large with them.
+    // only when the grid stays large with them. Beside the shared-prefix
+    // kernel (sweeps of 8-128 sequences sharing a 3072-token prefix, 1-1024
+    // private tokens each) partitions of 1024 tokens already paid off from
+    // 4 CTAs per SM in both grids together.
     if (r.heads_per_cta == 0) {
         int G = 4;
         while (G > 1 && (H % G || stage_bytes(G) * 2 > 96 * 1024)) G >>= 1;
         const int P0 = r.partition_size ? r.partition_size : 512;
-        while (G > 1 && units(G, P0) < 3 * kNumSMs) G >>= 1;
+        while (G > 1 && units(G, P0) + beside < 3 * kNumSMs) G >>= 1;
         r.heads_per_cta = G;
     }
     const int G0 = r.heads_per_cta;
     if (r.partition_size == 0) {
-        int P = units(G0, 1024) >= 12 * kNumSMs ? 1024 : 512;
-        while (P > 4 * B && units(G0, P) < 3 * kNumSMs) P >>= 1;
+        const bool long_parts = beside > 0 ? units(G0, 1024) + beside >= 4 * kNumSMs
+                                           : units(G0, 1024) >= 12 * kNumSMs;
+        int P = long_parts ? 1024 : 512;
+        while (P > 4 * B && units(G0, P) + beside < 3 * kNumSMs) P >>= 1;
         r.partition_size = P;
     }
     // One unit per CTA by default: measured on B200, packing 2-4 units of a
@@ -931,7 +940,8 @@ int plan_shared_prefix(const pa_cache_desc &c, int S, int bound, int prefix_bloc
     pre->stages = (int)std::max<size_t>(2, std::min<size_t>(8, (96 * 1024) / sb));
     pa_decode_config r = cfg ? *cfg : pa_decode_config{0, 0, 0, 0, 0};
     const int suffix_bound = std::max(bound - pre->prefix_tokens, B);
-    int rc = fill_config(c, S, suffix_bound, &r);
+    const int64_t prefix_ctas = (int64_t)(c.num_heads / pre->heads) * n_qb * pre->parts;
+    int rc = fill_config(c, S, suffix_bound, &r, prefix_ctas);
     if (rc) return rc;
     *suffix = r;
     const int ws_parts = max_parts_of(suffix_bound, r.partition_size) + pre->parts;
