@@ -223,7 +223,8 @@ namespace pa {
 // One CTA = one head x one tile of up to 128 consecutive query rows of one
 // sequence; K/V are consumed 128 tokens at a time. Per K/V tile j:
 //   S_j = Q . K_j^T   128 x 128, D / 16 tcgen05.mma (K = 16 each) into tensor
-//                     memory (two S buffers, so S_{j+1} overlaps the softmax of j)
+//                     memory (three S buffers: S_{j+2} is computed while the
+//                     softmax works on j, so the softmax never waits for S)
 //   softmax           reads S, masks tokens after each row's position, keeps
 //                     a reference maximum that moves only when the row
 //                     maximum exceeds it by more than 2^8 (then O is rescaled
@@ -232,12 +233,14 @@ namespace pa {
 //   O += P_j . V_j    eight tcgen05.mma (N = D) with A (P) read from tensor
 //                     memory and V from shared memory, N-contiguous (MN-major)
 // An S buffer takes the next S only once the P.V that reads its P is done.
+// One thread issues the MMAs: S_0, S_1, then per tile j, S_{j+2} (as soon
+// as its buffer is free) before P.V of j (once P_j is written).
 // K and V have rings of their own (3 and 2 tiles): a K tile is released as
 // soon as its S is computed, a V tile when its P.V is, so each is reloaded
 // as early as possible. Warps: 0-7 softmax (and Q staging, epilogue): warp
 // w takes rows 32 (w % 4) .. + 31 (its tensor-memory lanes), columns
 // 64 (w / 4) .. + 63 of S and P and D / 2 columns of O, the two halves of a
-// row exchanging their maxima and sums through tensor memory; 8 K producer;
+// row exchanging their maxima and sums through shared memory; 8 K producer;
 // 9 MMA issuer (also allocates the 512 tensor-memory columns); 10 V
 // producer. Each producer keeps the next 32 block-table entries in flight.
 // Every wait is bounded; a wait that runs out sets PA_DEV_WAIT_TIMEOUT and
@@ -250,8 +253,9 @@ constexpr int kTcVStages = 2;
 constexpr int kTcThreads = 352;
 constexpr int kTcSoftmaxWarps = 8;  // two per tensor-memory lane quadrant, one per half row
 constexpr int kTcWarpK = 8, kTcWarpMma = 9, kTcWarpV = 10;
-constexpr int kTcTmemCols = 512;  // S0 [0,128), S1 [128,256), O [256,256+D), row exchange [384,390)
-constexpr int kTcColX = 384;      // + 2 * tile parity + half: row maxima; + 4 + half: row sums
+constexpr int kTcSBufs = 3;        // S buffers (P of a tile is written over its S)
+constexpr int kTcTmemCols = 512;   // S0 [0,128), S1 [128,256), S2 [256,384), O [384,384+D)
+constexpr int kTcColO = kTcSBufs * kTcKv;
 
 template <int D>
 struct TcLayout {                                       // byte offsets from the 1024-aligned base
@@ -261,7 +265,9 @@ struct TcLayout {                                       // byte offsets from the
     static constexpr uint32_t kK = kQ + kTile;           // K ring
     static constexpr uint32_t kV = kK + kTcKStages * kTile;  // V ring
     static constexpr uint32_t kBars = kV + kTcVStages * kTile;
-    static constexpr uint32_t kBytes = kBars + 512;      // barriers, tensor-memory address, abort flag
+    static constexpr uint32_t kX = kBars + 512;          // barriers, tensor-memory address, abort flag
+    static constexpr uint32_t kXSum = kX + 2 * 2 * kTcRows * 4;  // row maxima [tile parity][half][row]
+    static constexpr uint32_t kBytes = kXSum + 2 * kTcRows * 4;  // row sums [half][row]
 };
 
 // mbarrier indices
@@ -272,10 +278,12 @@ enum : int {
     kBarFullV = kBarEmptyK + kTcKStages,    // + stage: V tile landed
     kBarEmptyV = kBarFullV + kTcVStages,    // + stage: P.V of the stage's tile done (commit)
     kBarSFull = kBarEmptyV + kTcVStages,    // + buffer: S ready (commit)
-    kBarSFree = kBarSFull + 2,              // + buffer: S read by the 8 softmax warps
-    kBarPFull = kBarSFree + 2,              // P written into tensor memory, O corrected (8 warps)
-    kBarOReady = kBarPFull + 1,             // P.V done (commit)
-    kBarDone = kBarOReady + 1,              // every MMA of the CTA done (commit)
+    kBarSFree = kBarSFull + kTcSBufs,       // + buffer: S read by the 8 softmax warps
+    kBarPFull = kBarSFree + kTcSBufs,       // + buffer: P written into tensor memory, O corrected (8 warps)
+    kBarOReady = kBarPFull + kTcSBufs,      // + buffer: P.V of the buffer's tile done (commit); one
+                                            // per buffer, as a warp may reach tile j before P.V of
+                                            // j-2 is done, and a wait must stay within two phases
+    kBarDone = kBarOReady + kTcSBufs,       // every MMA of the CTA done (commit)
     kBarPair = kBarDone + 1,                // + 2 * quadrant + tile parity: both halves' row maxima posted
     kBarPairEnd = kBarPair + 8,             // + quadrant: both halves' row sums posted
     kNumBars = kBarPairEnd + 4
@@ -300,6 +308,16 @@ __device__ __forceinline__ bool tc_wait(uint64_t *bar, uint32_t parity, volatile
             return false;
         }
     }
+}
+
+// Lane 0 waits; the warp goes on (all lanes, ordered after the wait) if it
+// saw the phase.
+__device__ __forceinline__ bool tc_wait_lane0(uint64_t *bar, uint32_t parity, volatile int *abort, int lane) {
+    bool ok = true;
+    if (lane == 0) ok = tc_wait(bar, parity, abort);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok;
 }
 
 // Every lane waits; the warp goes on only if all lanes saw the phase.
@@ -424,7 +442,8 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
         prefetch_tensor_map(&tmap_k);
         prefetch_tensor_map(&tmap_v);
         for (int i = 0; i < kNumBars; ++i)
-            mbar_init(&bar[i], (i == kBarQ || i == kBarSFree || i == kBarSFree + 1 || i == kBarPFull)
+            mbar_init(&bar[i], (i == kBarQ || (i >= kBarSFree && i < kBarSFree + kTcSBufs) ||
+                                (i >= kBarPFull && i < kBarPFull + kTcSBufs))
                                    ? kTcSoftmaxWarps : (i >= kBarPair ? 2 : 1));
         *abort = 0;
         fence_mbar_init();
@@ -456,53 +475,55 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
         const uint64_t dk = sw128_desc(sbase + Lay::kK, 16, 1024);
         const uint64_t dv = sw128_desc(sbase + Lay::kV, Lay::kHalf, 1024);
         auto kstep = [](int k) { return (uint64_t)(((k >> 2) * Lay::kHalf + (k & 3) * 32) >> 4); };
-        auto issue_pv = [&](int i) -> bool {
-            const int st = i % kTcVStages;
-            if (!tc_wait_warp(&bar[kBarPFull], i & 1, abort)) return false;
-            if (!tc_wait_warp(&bar[kBarFullV + st], (i / kTcVStages) & 1, abort)) return false;
-            tc_fence_after();
-            if (lane == 0) {
-                const uint64_t dvs = dv + ((st * Lay::kTile) >> 4);
-#pragma unroll
-                for (int kt = 0; kt < kTcKv / 16; ++kt)
-                    // P_i in tensor memory, in S buffer i % 2: tokens 64 h .. 64 h + 63
-                    // packed in columns 64 h .. 64 h + 31 (two fp16 per column)
-                    tc_mma_f16_ts(tmem + 256, tmem + (i & 1) * kTcKv + (kt >> 2) * 64 + (kt & 3) * 8,
-                                  dvs + ((kt * 16 * 128) >> 4), kIdescPV,
-                               (i > 0 || kt > 0) ? 1u : 0u);
-                tc_commit(&bar[kBarEmptyV + st]);
-                tc_commit(&bar[kBarOReady]);
+        // One thread issues every MMA and takes every wait of this role
+        // (a waiting lane costs the softmax warps of its sub-partition issue
+        // slots); the other lanes wait for it at the end.
+        auto issue_s = [&](int j) -> bool {
+            const int st = j % kTcKStages, b = j % kTcSBufs;
+            if (!tc_wait(&bar[kBarFullK + st], (j / kTcKStages) & 1, abort)) return false;
+            if (j >= kTcSBufs) {
+                // buffer b holds S_{j-3} until every softmax warp has read it,
+                // then P_{j-3} until its P.V is done (the last P.V issued)
+                if (!tc_wait(&bar[kBarSFree + b], (j / kTcSBufs - 1) & 1, abort)) return false;
+                if (!tc_wait(&bar[kBarOReady + b], (j / kTcSBufs - 1) & 1, abort)) return false;
             }
-            __syncwarp();
+            tc_fence_after();
+            const uint64_t dks = dk + ((st * Lay::kTile) >> 4);
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks)
+                tc_mma_f16(tmem + b * kTcKv, dq + kstep(ks), dks + kstep(ks), kIdescS, ks > 0 ? 1u : 0u);
+            tc_commit(&bar[kBarSFull + b]);
+            tc_commit(&bar[kBarEmptyK + st]);
             return true;
         };
-        bool ok = tc_wait_warp(&bar[kBarQ], 0, abort);
-        int j = 0;
-        for (; ok && j < n_kv; ++j) {
-            const int st = j % kTcKStages;
-            ok = tc_wait_warp(&bar[kBarFullK + st], (j / kTcKStages) & 1, abort);
-            if (ok && j >= 2) ok = tc_wait_warp(&bar[kBarSFree + (j & 1)], ((j - 2) >> 1) & 1, abort);
-            // S buffer j % 2 holds P_{j-2} until its P.V is done (P.V of j-1
-            // is issued after this S, so the wait names the last completion)
-            if (ok && j >= 2) ok = tc_wait_warp(&bar[kBarOReady], (j - 2) & 1, abort);
-            if (!ok) break;
+        auto issue_pv = [&](int i) -> bool {
+            const int st = i % kTcVStages, b = i % kTcSBufs;
+            if (!tc_wait(&bar[kBarPFull + b], (i / kTcSBufs) & 1, abort)) return false;
+            if (!tc_wait(&bar[kBarFullV + st], (i / kTcVStages) & 1, abort)) return false;
             tc_fence_after();
-            if (lane == 0) {
-                const uint64_t dks = dk + ((st * Lay::kTile) >> 4);
+            const uint64_t dvs = dv + ((st * Lay::kTile) >> 4);
 #pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks)
-                    tc_mma_f16(tmem + (j & 1) * kTcKv, dq + kstep(ks), dks + kstep(ks), kIdescS, ks > 0 ? 1u : 0u);
-                tc_commit(&bar[kBarSFull + (j & 1)]);
-                tc_commit(&bar[kBarEmptyK + st]);
+            for (int kt = 0; kt < kTcKv / 16; ++kt)
+                // P_i in tensor memory, in S buffer i % 3: tokens 64 h .. 64 h + 63
+                // packed in columns 64 h .. 64 h + 31 (two fp16 per column)
+                tc_mma_f16_ts(tmem + kTcColO, tmem + b * kTcKv + (kt >> 2) * 64 + (kt & 3) * 8,
+                              dvs + ((kt * 16 * 128) >> 4), kIdescPV, (i > 0 || kt > 0) ? 1u : 0u);
+            tc_commit(&bar[kBarEmptyV + st]);
+            tc_commit(&bar[kBarOReady + b]);
+            return true;
+        };
+        if (lane == 0) {
+            bool ok = tc_wait(&bar[kBarQ], 0, abort);
+            for (int j = 0; ok && j < min(kTcSBufs - 1, n_kv); ++j) ok = issue_s(j);
+            for (int j = 0; ok && j < n_kv; ++j) {
+                if (j + kTcSBufs - 1 < n_kv) ok = issue_s(j + kTcSBufs - 1);
+                if (ok) ok = issue_pv(j);
             }
-            __syncwarp();
-            if (j >= 1) ok = issue_pv(j - 1);
+            // every MMA issued above completes before the tensor memory is freed
+            tc_commit(&bar[kBarDone]);
+            mbar_wait(&bar[kBarDone], 0);
         }
-        if (ok) issue_pv(n_kv - 1);
-        // every MMA issued above completes before the tensor memory is freed
-        if (lane == 0) tc_commit(&bar[kBarDone]);
         __syncwarp();
-        mbar_wait(&bar[kBarDone], 0);
         tc_fence_before();
         asm volatile("bar.sync 2, %0;" ::"r"(32 * (kTcSoftmaxWarps + 1)) : "memory");
         tc_fence_after();
@@ -517,6 +538,7 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
     const bool valid = rl < n;
     const int lim = valid ? base + rl + 1 : 0;  // tokens 0 .. lim-1 are visible
     uint64_t *pair = &bar[kBarPair + 2 * (warp & 3)];  // the two warps sharing these rows
+    float *xmax = reinterpret_cast<float *>(smem + Lay::kX);  // [tile parity][half][row]
     {
         const uint4 *src = reinterpret_cast<const uint4 *>(p.query + ((size_t)(q_begin + (valid ? rl : 0)) * p.num_heads + h) * D);
 #pragma unroll
@@ -535,19 +557,20 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
-        if (!tc_wait_warp(&bar[kBarSFull + (j & 1)], (j >> 1) & 1, abort)) { ok = false; break; }
+        const int sb = j % kTcSBufs;  // S / P buffer of this tile
+        if (!tc_wait_warp(&bar[kBarSFull + sb], (j / kTcSBufs) & 1, abort)) { ok = false; break; }
         tc_fence_after();
         float sv[HC];
 #pragma unroll
         for (int q = 0; q < HC / 32; ++q) {
             float v32[32];
-            tmem_ld32(tl + (j & 1) * kTcKv + hh * HC + q * 32, v32);
+            tmem_ld32(tl + sb * kTcKv + hh * HC + q * 32, v32);
 #pragma unroll
             for (int i = 0; i < 32; ++i) sv[q * 32 + i] = v32[i];
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[kBarSFree + (j & 1)]);
+        if (lane == 0) mbar_arrive(&bar[kBarSFree + sb]);
 
         const int t0 = j * kTcKv + hh * HC;  // position of this thread's first column
         if (t0 + HC > lim) {
@@ -564,16 +587,14 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
             for (int k = 8; k < HC; ++k) m8[k & 7] = fmaxf(m8[k & 7], sv[k]);
             mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
         }
-        // both halves of the row take the same maximum, exchanged through a
-        // tensor-memory column of the row's lane (columns and barriers by
-        // tile parity: a warp runs at most one tile ahead of its partner)
-        tmem_st1(tl + kTcColX + 2 * (j & 1) + hh, mx);
-        tc_fence_before();
+        // both halves of the row take the same maximum, exchanged through
+        // shared memory (slots and barriers by tile parity: a warp runs at
+        // most one tile ahead of its partner); one lane waits, bounded
+        xmax[((j & 1) * 2 + hh) * kTcRows + t] = mx;
         __syncwarp();
         if (lane == 0) mbar_arrive(&pair[j & 1]);
-        if (!tc_wait_warp(&pair[j & 1], (j >> 1) & 1, abort)) { ok = false; break; }
-        tc_fence_after();
-        mx = fmaxf(mx, tmem_ld1(tl + kTcColX + 2 * (j & 1) + (hh ^ 1))) * c2;
+        if (!tc_wait_lane0(&pair[j & 1], (j >> 1) & 1, abort, lane)) { ok = false; break; }
+        mx = fmaxf(mx, xmax[((j & 1) * 2 + (hh ^ 1)) * kTcRows + t]) * c2;
         float alpha = 1.f;
         bool resc = false;
         if (mx > m_ref + 8.f) {  // the reference maximum moves only by more than 2^8
@@ -595,28 +616,39 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
 
         // O must be current before a rescale: wait for P.V of tile j-1
         if (j >= 1 && __any_sync(0xffffffffu, resc)) {
-            if (!tc_wait_warp(&bar[kBarOReady], (j - 1) & 1, abort)) { ok = false; break; }
+            if (!tc_wait_warp(&bar[kBarOReady + (j - 1) % kTcSBufs], ((j - 1) / kTcSBufs) & 1, abort)) {
+                ok = false;
+                break;
+            }
             tc_fence_after();
 #pragma unroll
             for (int q = 0; q < OC / 32; ++q) {
                 float ov[32];
-                tmem_ld32(tl + 256 + hh * OC + q * 32, ov);
+                tmem_ld32(tl + kTcColO + hh * OC + q * 32, ov);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) ov[i] *= alpha;
-                tmem_st32(tl + 256 + hh * OC + q * 32, ov);
+                tmem_st32(tl + kTcColO + hh * OC + q * 32, ov);
             }
         }
         {  // P into the first half of this warp's S columns (read above)
             float pf[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) pf[i] = __uint_as_float(pk[i]);
-            tmem_st32(tl + (j & 1) * kTcKv + hh * HC, pf);
+            tmem_st32(tl + sb * kTcKv + hh * HC, pf);
         }
         // tokens at or after the sequence end are unused cache slots (any
         // bits, NaN included): their V rows enter P.V as zeros
         const int tt = j * kTcKv;
         if (tt + kTcKv > L) {
             const int vst = j % kTcVStages;
+            // V_{j-2} shares the stage and may not have landed yet (this warp
+            // can be two tiles ahead of P.V): wait for its P.V first, so that
+            // the stage's wait below names its last phase or the one before
+            if (j >= kTcVStages &&
+                !tc_wait_warp(&bar[kBarOReady + (j - kTcVStages) % kTcSBufs], ((j - kTcVStages) / kTcSBufs) & 1, abort)) {
+                ok = false;
+                break;
+            }
             if (!tc_wait_warp(&bar[kBarFullV + vst], (j / kTcVStages) & 1, abort)) { ok = false; break; }
             if (tt + t >= L) {
                 const uint32_t v_addr = sbase + Lay::kV + vst * Lay::kTile;
@@ -628,26 +660,23 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[kBarPFull]);
+        if (lane == 0) mbar_arrive(&bar[kBarPFull + sb]);
     }
-    // the row sum is the two halves' shares
-    tmem_st1(tl + kTcColX + 4 + hh, l);
-    tc_fence_before();
+    // the row sum is the two halves' shares (exchanged through shared memory)
+    float *xsum = reinterpret_cast<float *>(smem + Lay::kXSum);  // [half][row]
+    xsum[hh * kTcRows + t] = l;
     __syncwarp();
     if (lane == 0) mbar_arrive(&bar[kBarPairEnd + (warp & 3)]);
-    ok = ok && tc_wait_warp(&bar[kBarPairEnd + (warp & 3)], 0, abort);
-    if (ok) {
-        tc_fence_after();
-        l += tmem_ld1(tl + kTcColX + 4 + (hh ^ 1));
-    }
-    if (ok && tc_wait_warp(&bar[kBarOReady], (n_kv - 1) & 1, abort)) {
+    ok = ok && tc_wait_lane0(&bar[kBarPairEnd + (warp & 3)], 0, abort, lane);
+    if (ok) l += xsum[(hh ^ 1) * kTcRows + t];
+    if (ok && tc_wait_warp(&bar[kBarOReady + (n_kv - 1) % kTcSBufs], ((n_kv - 1) / kTcSBufs) & 1, abort)) {
         tc_fence_after();
         const float inv = valid ? 1.0f / l : 0.f;
         __half *op = p.out + ((size_t)(q_begin + (valid ? rl : 0)) * p.num_heads + h) * D + hh * OC;
 #pragma unroll
         for (int q = 0; q < OC / 32; ++q) {
             float ov[32];
-            tmem_ld32(tl + 256 + hh * OC + q * 32, ov);
+            tmem_ld32(tl + kTcColO + hh * OC + q * 32, ov);
             if (valid) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {

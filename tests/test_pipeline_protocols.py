@@ -180,6 +180,8 @@ def test_broadcast_ring_model_catches_a_missing_release_count():
 # ------------------------------------------------------- tcgen05 prefill
 
 K_STAGES, V_STAGES = 3, 2
+ROW_SPLIT = 2                  # softmax warps sharing a row (halves of its S columns)
+N_SOFTMAX = 4 * ROW_SPLIT      # softmax warps: ROW_SPLIT per tensor-memory lane quadrant
 
 
 class _Bar:
@@ -194,34 +196,48 @@ class _Bar:
             self.pending = self.count
 
 
-def _prefill_run(n_kv, tail, seed):
+S_BUFS = 3                     # S buffers in tensor memory (P of a tile overwrites its S)
+
+
+def _prefill_run(n_kv, tail, seed, p_bars=S_BUFS, o_bars=S_BUFS):
     """One CTA of paged_prefill_tc_kernel: K and V producers, the MMA issuer
-    and the eight softmax warps (pairs exchange their maxima every tile)."""
+    and the eight softmax warps (the two halves of a row exchange their
+    maxima every tile through shared-memory slots chosen by tile parity).
+    The MMA issuer computes S one buffer ahead of need: S_0 .. S_{B-2} first,
+    then per tile j, S_{j+B-1} (once its buffer is free) before P.V of j.
+    P barriers are indexed by tile % p_bars, P.V-done barriers by
+    tile % o_bars."""
     rnd = random.Random(seed)
     bars = {}
+    SB = S_BUFS
 
     def mk(name, count):
         bars[name] = _Bar(name, count)
 
-    mk("q", 8)
+    mk("q", N_SOFTMAX)
     for s in range(K_STAGES):
         mk(f"fk{s}", 1)
         mk(f"ek{s}", 1)
     for s in range(V_STAGES):
         mk(f"fv{s}", 1)
         mk(f"ev{s}", 1)
-    for b in range(2):
+    for b in range(SB):
         mk(f"sf{b}", 1)
-        mk(f"sr{b}", 8)
-    mk("pf", 8)
-    mk("or", 1)
+        mk(f"sr{b}", N_SOFTMAX)
+    for b in range(p_bars):
+        mk(f"pf{b}", N_SOFTMAX)
+    for b in range(o_bars):
+        mk(f"or{b}", 1)                       # P.V of a tile of this index done
     for q in range(4):
         for par in range(2):
-            mk(f"pair{q}{par}", 2)
-        mk(f"pend{q}", 2)
-    st = {"k": [None] * K_STAGES, "v": [None] * V_STAGES, "S": [None, None], "Sread": [set(), set()],
-          "pv": set(), "zeroed": set()}
-    pending = []
+            mk(f"pair{q}{par}", ROW_SPLIT)
+        mk(f"pend{q}", ROW_SPLIT)
+    st = {"k": [None] * K_STAGES, "v": [None] * V_STAGES, "S": [None] * SB, "Sread": [set() for _ in range(SB)],
+          "pv": set(), "zeroed": set(), "P": [0] * n_kv,
+          # exchange slots: [lane quadrant][tile parity][half] -> tile whose maximum it holds
+          "x": [[[None] * ROW_SPLIT for _ in range(2)] for _ in range(4)]}
+    pending = []   # tile loads in flight: they land in any order
+    mma_q = []     # MMAs of the one issuing thread: they complete in issue order
 
     def wait(b, k):
         return ("wait", b, k)
@@ -237,58 +253,80 @@ def _prefill_run(n_kv, tail, seed):
     def mma():
         yield wait("q", 0)
 
-        def pv(i):
-            yield wait("pf", i)
-            yield wait(f"fv{i % V_STAGES}", i // V_STAGES)
-            assert st["v"][i % V_STAGES] == i
-            pending.append(("pv", i))
-            yield ("nop",)
-
-        for j in range(n_kv):
+        def issue_s(j):
             yield wait(f"fk{j % K_STAGES}", j // K_STAGES)
             assert st["k"][j % K_STAGES] == j
-            if j >= 2:
-                yield wait(f"sr{j & 1}", (j - 2) // 2)
-                yield wait("or", j - 2)          # P_{j-2} in this S buffer consumed
-                assert (j - 2) in st["pv"]
-            pending.append(("s", j))
+            if j >= SB:
+                yield wait(f"sr{j % SB}", j // SB - 1)
+                yield wait(f"or{(j - SB) % o_bars}", (j - SB) // o_bars)   # P_{j-SB} in this S buffer consumed
+                assert (j - SB) in st["pv"]
+            mma_q.append(("s", j))
             yield ("nop",)
-            if j >= 1:
-                yield from pv(j - 1)
-        yield from pv(n_kv - 1)
+
+        def pv(i):
+            yield wait(f"pf{i % p_bars}", i // p_bars)
+            assert st["P"][i] == N_SOFTMAX, "P.V issued before every warp wrote its part of P"
+            yield wait(f"fv{i % V_STAGES}", i // V_STAGES)
+            assert st["v"][i % V_STAGES] == i
+            mma_q.append(("pv", i))
+            yield ("nop",)
+
+        for j in range(min(SB - 1, n_kv)):
+            yield from issue_s(j)
+        for j in range(n_kv):
+            if j + SB - 1 < n_kv:
+                yield from issue_s(j + SB - 1)
+            yield from pv(j)
 
     rescale = {j: rnd.random() < 0.3 for j in range(n_kv)}
 
     def softmax(w):
-        q = w & 3
+        q, half = w & 3, w // 4
         yield ("arrive", "q")
         for j in range(n_kv):
-            yield wait(f"sf{j & 1}", j // 2)
-            assert st["S"][j & 1] == j
-            yield ("arrive", f"sr{j & 1}", w)
+            yield wait(f"sf{j % SB}", j // SB)
+            assert st["S"][j % SB] == j
+            yield ("arrive", f"sr{j % SB}", w)
+            st["x"][q][j & 1][half] = j         # this half's maximum of tile j
             yield ("arrive", f"pair{q}{j & 1}")
             yield wait(f"pair{q}{j & 1}", j // 2)
+            yield ("nop",)                       # the read may lag the wait
+            assert st["x"][q][j & 1] == [j] * ROW_SPLIT, "a row maximum read before it was posted or after it was overwritten"
             if j >= 1 and rescale[j]:
-                yield wait("or", j - 1)
-                assert (j - 1) in st["pv"]
+                yield wait(f"or{(j - 1) % o_bars}", (j - 1) // o_bars)
+                assert all(i in st["pv"] for i in range(j)), "O rescaled before every earlier P.V was done"
             if tail and j == n_kv - 1:
+                if j >= V_STAGES:   # V_{j-2} (same stage) consumed, so landed: the wait below stays in window
+                    yield wait(f"or{(j - V_STAGES) % o_bars}", (j - V_STAGES) // o_bars)
                 yield wait(f"fv{j % V_STAGES}", j // V_STAGES)
                 st["zeroed"].add((j, w))
-            yield ("arrive", "pf")
+            st["P"][j] += 1
+            yield ("arrive", f"pf{j % p_bars}")
         yield ("arrive", f"pend{q}")
         yield wait(f"pend{q}", 0)
-        yield wait("or", n_kv - 1)
+        yield wait(f"or{(n_kv - 1) % o_bars}", (n_kv - 1) // o_bars)
+        assert all(i in st["pv"] for i in range(n_kv)), "O read before every P.V was done"
 
     roles = {"pk": producer("k", K_STAGES), "pv": producer("v", V_STAGES), "mma": mma(),
-             **{f"w{w}": softmax(w) for w in range(8)}}
+             **{f"w{w}": softmax(w) for w in range(N_SOFTMAX)}}
     cur = {k: None for k in roles}
     alive = set(roles)
+    # each role runs at its own speed, so warps drift apart by many steps
+    speed = {r: rnd.choice([1.0, 0.5, 0.1]) for r in roles}
+    # in some runs the tile loads of one kind are slow to land
+    slow = rnd.choice([None, "k", "v"])
     for _ in range(400000):
-        if not alive and not pending:
+        if not alive and not pending and not mma_q:
             return
         progressed = False
-        if pending and rnd.random() < 0.4:
-            op = pending.pop(rnd.randrange(len(pending)))
+        op = None
+        if (pending or mma_q) and rnd.random() < 0.4:
+            k = rnd.randrange(len(pending) + (1 if mma_q else 0))
+            if k < len(pending) and pending[k][0] == slow and rnd.random() < 0.9:
+                k = None                       # this load stays in flight a while longer
+            if k is not None:
+                op = pending.pop(k) if k < len(pending) else mma_q.pop(0)
+        if op is not None:
             if op[0] == "k":
                 st["k"][op[2]] = op[1]
                 bars[f"fk{op[2]}"].arrive()
@@ -297,26 +335,32 @@ def _prefill_run(n_kv, tail, seed):
                 bars[f"fv{op[2]}"].arrive()
             elif op[0] == "s":
                 j = op[1]
-                prev = st["S"][j & 1]
+                prev = st["S"][j % SB]
                 if prev is not None:
-                    assert len(st["Sread"][j & 1]) == 8, "S overwritten before all warps read it"
+                    assert len(st["Sread"][j % SB]) == N_SOFTMAX, "S overwritten before all warps read it"
                     assert prev in st["pv"], "S overwritten while its P was still to be read by P.V"
-                st["S"][j & 1] = j
-                st["Sread"][j & 1] = set()
-                bars[f"sf{j & 1}"].arrive()
+                st["S"][j % SB] = j
+                st["Sread"][j % SB] = set()
+                bars[f"sf{j % SB}"].arrive()
                 bars[f"ek{j % K_STAGES}"].arrive()
             else:
                 i = op[1]
                 if tail and i == n_kv - 1:
-                    assert len([1 for (jj, _) in st["zeroed"] if jj == i]) == 8, "P.V read the V tail before zeroing"
+                    assert len([1 for (jj, _) in st["zeroed"] if jj == i]) == N_SOFTMAX, \
+                        "P.V read the V tail before zeroing"
+                assert all(k in st["pv"] for k in range(i)), "P.V completed out of order"
                 st["pv"].add(i)
                 bars[f"ev{i % V_STAGES}"].arrive()
-                bars["or"].arrive()
+                bars[f"or{i % o_bars}"].arrive()
             progressed = True
         order = list(alive)
         rnd.shuffle(order)
         for r in order:
             ev = cur[r]
+            if rnd.random() > speed[r]:  # this role sits out the step
+                if ev is None or ev[0] != "wait" or bars[ev[1]].done >= ev[2] + 1:
+                    progressed = True    # (it could have moved)
+                continue
             if ev is None:
                 try:
                     ev = next(roles[r])
@@ -328,24 +372,55 @@ def _prefill_run(n_kv, tail, seed):
             if ev[0] == "wait":
                 b = bars[ev[1]]
                 assert b.done <= ev[2] + 1, f"{r} waits {ev[1]} phase {ev[2]} with {b.done} phases done"
+                # a parity wait two phases ahead would pass at once
+                assert b.done >= ev[2], f"{r} waits {ev[1]} phase {ev[2]} with only {b.done} phases done"
                 if b.done >= ev[2] + 1:
                     cur[r] = None
                     progressed = True
             elif ev[0] == "arrive":
                 bars[ev[1]].arrive()
                 if ev[1].startswith("sr"):
-                    st["Sread"][int(ev[1][2])].add(ev[2])
+                    st["Sread"][int(ev[1][2:])].add(ev[2])
                 cur[r] = None
                 progressed = True
             else:
                 cur[r] = None
                 progressed = True
-        assert progressed or pending, f"deadlock: {cur}"
+        assert progressed or pending or mma_q, f"deadlock: {cur}"
     raise AssertionError("no termination")
 
 
 @pytest.mark.parametrize("n_kv", [1, 2, 3, 4, 7])
 @pytest.mark.parametrize("tail", [False, True])
 def test_prefill_protocol(n_kv, tail):
-    for seed in range(60):
+    for seed in range(150):
         _prefill_run(n_kv, tail, seed)
+
+
+@pytest.mark.parametrize("p_bars", [1, 2])
+def test_prefill_protocol_catches_too_few_p_barriers(p_bars):
+    # With fewer P barriers than S buffers, warps of another lane quadrant
+    # that run ahead (their S is computed S_BUFS - 1 tiles early) can complete
+    # a phase in place of a slow warp, and P.V would read that warp's columns
+    # before its P is written. The model (warps at their own speeds) must find
+    # that interleaving.
+    failures = 0
+    for seed in range(200):
+        try:
+            _prefill_run(5, False, seed, p_bars=p_bars)
+        except AssertionError:
+            failures += 1
+    assert failures > 0
+
+
+def test_prefill_protocol_catches_one_pv_barrier_for_all_buffers():
+    # With three S buffers a warp can reach tile j before P.V of j-2 is done;
+    # one P.V-done barrier for every tile then puts the rescale's wait for
+    # P.V of j-1 two phases ahead, where a parity wait passes at once.
+    failures = 0
+    for seed in range(100):
+        try:
+            _prefill_run(5, False, seed, o_bars=1)
+        except AssertionError:
+            failures += 1
+    assert failures > 0
