@@ -237,12 +237,13 @@ namespace pa {
 // as its buffer is free) before P.V of j (once P_j is written).
 // K and V have rings of their own (3 and 2 tiles): a K tile is released as
 // soon as its S is computed, a V tile when its P.V is, so each is reloaded
-// as early as possible. Warps: 0-7 softmax (and Q staging, epilogue): warp
-// w takes rows 32 (w % 4) .. + 31 (its tensor-memory lanes), columns
-// 64 (w / 4) .. + 63 of S and P and D / 2 columns of O, the two halves of a
-// row exchanging their maxima and sums through shared memory; 8 K producer;
-// 9 MMA issuer (also allocates the 512 tensor-memory columns); 10 V
-// producer. Each producer keeps the next 32 block-table entries in flight.
+// as early as possible. Warps: 0-3 softmax (and Q staging, epilogue): warp
+// w takes rows 32 w .. + 31 (its tensor-memory lanes), each thread a whole
+// row of S, P and O, so no row is shared and no warp waits for another
+// within a tile; the sub-partition's MUFU serves the row's exponentials
+// alone. 4 K producer; 5 MMA issuer (also allocates the 512 tensor-memory
+// columns); 6 V producer. Each producer keeps the next 32 block-table
+// entries in flight.
 // Every wait is bounded; a wait that runs out sets PA_DEV_WAIT_TIMEOUT and
 // an abort flag that ends the other roles' waits, and the CTA still drains
 // its copies and MMAs and frees its tensor memory before it exits.
@@ -250,9 +251,9 @@ constexpr int kTcRows = 128;
 constexpr int kTcKv = 128;
 constexpr int kTcKStages = 3;
 constexpr int kTcVStages = 2;
-constexpr int kTcThreads = 352;
-constexpr int kTcSoftmaxWarps = 8;  // two per tensor-memory lane quadrant, one per half row
-constexpr int kTcWarpK = 8, kTcWarpMma = 9, kTcWarpV = 10;
+constexpr int kTcSoftmaxWarps = 4;  // one per tensor-memory lane quadrant, one thread per row
+constexpr int kTcWarpK = 4, kTcWarpMma = 5, kTcWarpV = 6;
+constexpr int kTcThreads = 32 * (kTcSoftmaxWarps + 3);
 constexpr int kTcSBufs = 3;        // S buffers (P of a tile is written over its S)
 constexpr int kTcTmemCols = 512;   // S0 [0,128), S1 [128,256), S2 [256,384), O [384,384+D)
 constexpr int kTcColO = kTcSBufs * kTcKv;
@@ -265,28 +266,25 @@ struct TcLayout {                                       // byte offsets from the
     static constexpr uint32_t kK = kQ + kTile;           // K ring
     static constexpr uint32_t kV = kK + kTcKStages * kTile;  // V ring
     static constexpr uint32_t kBars = kV + kTcVStages * kTile;
-    static constexpr uint32_t kX = kBars + 512;          // barriers, tensor-memory address, abort flag
-    static constexpr uint32_t kXSum = kX + 2 * 2 * kTcRows * 4;  // row maxima [tile parity][half][row]
-    static constexpr uint32_t kBytes = kXSum + 2 * kTcRows * 4;  // row sums [half][row]
+    static constexpr uint32_t kBytes = kBars + 512;      // barriers, tensor-memory address, abort flag
 };
 
 // mbarrier indices
 enum : int {
-    kBarQ = 0,                              // Q staged (8 softmax warps)
+    kBarQ = 0,                              // Q staged (every softmax warp)
     kBarFullK = 1,                          // + stage: K tile landed (TMA bytes)
     kBarEmptyK = kBarFullK + kTcKStages,    // + stage: S of the stage's tile done (commit)
     kBarFullV = kBarEmptyK + kTcKStages,    // + stage: V tile landed
     kBarEmptyV = kBarFullV + kTcVStages,    // + stage: P.V of the stage's tile done (commit)
     kBarSFull = kBarEmptyV + kTcVStages,    // + buffer: S ready (commit)
-    kBarSFree = kBarSFull + kTcSBufs,       // + buffer: S read by the 8 softmax warps
-    kBarPFull = kBarSFree + kTcSBufs,       // + buffer: P written into tensor memory, O corrected (8 warps)
+    kBarSFree = kBarSFull + kTcSBufs,       // + buffer: S read by every softmax warp
+    kBarPFull = kBarSFree + kTcSBufs,       // + buffer: P written into tensor memory, O corrected (every
+                                            // softmax warp)
     kBarOReady = kBarPFull + kTcSBufs,      // + buffer: P.V of the buffer's tile done (commit); one
                                             // per buffer, as a warp may reach tile j before P.V of
                                             // j-2 is done, and a wait must stay within two phases
     kBarDone = kBarOReady + kTcSBufs,       // every MMA of the CTA done (commit)
-    kBarPair = kBarDone + 1,                // + 2 * quadrant + tile parity: both halves' row maxima posted
-    kBarPairEnd = kBarPair + 8,             // + quadrant: both halves' row sums posted
-    kNumBars = kBarPairEnd + 4
+    kNumBars = kBarDone + 1
 };
 static_assert(8 * kNumBars + 8 <= TcLayout<128>::kBytes - TcLayout<128>::kBars, "barrier area too small");
 static_assert(TcLayout<128>::kBytes + 1024 <= 227 * 1024, "shared memory of the tcgen05 prefill kernel");
@@ -318,12 +316,6 @@ __device__ __forceinline__ bool tc_wait_lane0(uint64_t *bar, uint32_t parity, vo
     ok = __shfl_sync(0xffffffffu, ok, 0);
     __syncwarp();
     return ok;
-}
-
-// Every lane waits; the warp goes on only if all lanes saw the phase.
-__device__ __forceinline__ bool tc_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort) {
-    const bool ok = tc_wait(bar, parity, abort);
-    return __all_sync(0xffffffffu, ok);
 }
 
 // 16 bytes at chunk c (0..15) of row r of a [halves][128 rows][128 B]
@@ -444,7 +436,7 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
         for (int i = 0; i < kNumBars; ++i)
             mbar_init(&bar[i], (i == kBarQ || (i >= kBarSFree && i < kBarSFree + kTcSBufs) ||
                                 (i >= kBarPFull && i < kBarPFull + kTcSBufs))
-                                   ? kTcSoftmaxWarps : (i >= kBarPair ? 2 : 1));
+                                   ? kTcSoftmaxWarps : 1);
         *abort = 0;
         fence_mbar_init();
     }
@@ -532,17 +524,14 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
     }
 
     // -------------------------------------------------------------- softmax
-    const int t = (warp & 3) * 32 + lane;  // row of the tile = tensor-memory lane
-    const int hh = warp >> 2;              // half of the row: columns 64 hh .. 64 hh + 63
+    const int t = warp * 32 + lane;  // row of the tile = tensor-memory lane
     const int rl = r0 + t;
     const bool valid = rl < n;
     const int lim = valid ? base + rl + 1 : 0;  // tokens 0 .. lim-1 are visible
-    uint64_t *pair = &bar[kBarPair + 2 * (warp & 3)];  // the two warps sharing these rows
-    float *xmax = reinterpret_cast<float *>(smem + Lay::kX);  // [tile parity][half][row]
     {
         const uint4 *src = reinterpret_cast<const uint4 *>(p.query + ((size_t)(q_begin + (valid ? rl : 0)) * p.num_heads + h) * D);
 #pragma unroll
-        for (int c = hh * (D / 16); c < (hh + 1) * (D / 16); ++c) {  // this half's 16-byte chunks
+        for (int c = 0; c < D / 8; ++c) {  // the row's 16-byte chunks
             const uint4 v = valid ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
             st_shared_v4(tc_chunk(sbase + Lay::kQ, t, c), v);
         }
@@ -550,21 +539,19 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar[kBarQ]);
     }
-    constexpr int HC = kTcKv / 2;  // S / P columns per thread
-    constexpr int OC = D / 2;      // O columns per thread
     const float c2 = p.qk_scale_log2;  // > 0 on this path
-    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
         const int sb = j % kTcSBufs;  // S / P buffer of this tile
-        if (!tc_wait_warp(&bar[kBarSFull + sb], (j / kTcSBufs) & 1, abort)) { ok = false; break; }
+        if (!tc_wait_lane0(&bar[kBarSFull + sb], (j / kTcSBufs) & 1, abort, lane)) { ok = false; break; }
         tc_fence_after();
-        float sv[HC];
+        float sv[kTcKv];
 #pragma unroll
-        for (int q = 0; q < HC / 32; ++q) {
+        for (int q = 0; q < kTcKv / 32; ++q) {
             float v32[32];
-            tmem_ld32(tl + sb * kTcKv + hh * HC + q * 32, v32);
+            tmem_ld32(tl + sb * kTcKv + q * 32, v32);
 #pragma unroll
             for (int i = 0; i < 32; ++i) sv[q * 32 + i] = v32[i];
         }
@@ -572,10 +559,10 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar[kBarSFree + sb]);
 
-        const int t0 = j * kTcKv + hh * HC;  // position of this thread's first column
-        if (t0 + HC > lim) {
+        const int t0 = j * kTcKv;  // position of the tile's first column
+        if (t0 + kTcKv > lim) {
 #pragma unroll
-            for (int k = 0; k < HC; ++k)
+            for (int k = 0; k < kTcKv; ++k)
                 if (t0 + k >= lim) sv[k] = -INFINITY;
         }
         float mx;
@@ -584,17 +571,10 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
 #pragma unroll
             for (int i = 0; i < 8; ++i) m8[i] = sv[i];
 #pragma unroll
-            for (int k = 8; k < HC; ++k) m8[k & 7] = fmaxf(m8[k & 7], sv[k]);
+            for (int k = 8; k < kTcKv; ++k) m8[k & 7] = fmaxf(m8[k & 7], sv[k]);
             mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
         }
-        // both halves of the row take the same maximum, exchanged through
-        // shared memory (slots and barriers by tile parity: a warp runs at
-        // most one tile ahead of its partner); one lane waits, bounded
-        xmax[((j & 1) * 2 + hh) * kTcRows + t] = mx;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&pair[j & 1]);
-        if (!tc_wait_lane0(&pair[j & 1], (j >> 1) & 1, abort, lane)) { ok = false; break; }
-        mx = fmaxf(mx, xmax[((j & 1) * 2 + (hh ^ 1)) * kTcRows + t]) * c2;
+        mx *= c2;
         float alpha = 1.f;
         bool resc = false;
         if (mx > m_ref + 8.f) {  // the reference maximum moves only by more than 2^8
@@ -603,38 +583,39 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
             resc = true;
         }
         const float mr = m_ref == -INFINITY ? 0.f : m_ref;
-        uint32_t pk[HC / 2];
+        // P = 2^(s - m) as fp16 pairs: tokens 64 h .. 64 h + 63 of the tile go
+        // to columns 64 h .. 64 h + 31 of the buffer (all S columns are in
+        // registers by now)
         float rs4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int k = 0; k < HC / 2; ++k) {
-            const float p0 = fast_exp2(fmaf(sv[2 * k], c2, -mr));
-            const float p1 = fast_exp2(fmaf(sv[2 * k + 1], c2, -mr));
-            rs4[k & 3] += p0 + p1;
-            pk[k] = pack_half2(p0, p1);
+        for (int hh = 0; hh < 2; ++hh) {
+            float pf[32];
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                const float p0 = fast_exp2(fmaf(sv[64 * hh + 2 * k], c2, -mr));
+                const float p1 = fast_exp2(fmaf(sv[64 * hh + 2 * k + 1], c2, -mr));
+                rs4[k & 3] += p0 + p1;
+                pf[k] = __uint_as_float(pack_half2(p0, p1));
+            }
+            tmem_st32(tl + sb * kTcKv + 64 * hh, pf);
         }
-        l = l * alpha + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));  // this half's share of the row sum
+        l = l * alpha + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
 
         // O must be current before a rescale: wait for P.V of tile j-1
         if (j >= 1 && __any_sync(0xffffffffu, resc)) {
-            if (!tc_wait_warp(&bar[kBarOReady + (j - 1) % kTcSBufs], ((j - 1) / kTcSBufs) & 1, abort)) {
+            if (!tc_wait_lane0(&bar[kBarOReady + (j - 1) % kTcSBufs], ((j - 1) / kTcSBufs) & 1, abort, lane)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
 #pragma unroll
-            for (int q = 0; q < OC / 32; ++q) {
+            for (int q = 0; q < D / 32; ++q) {
                 float ov[32];
-                tmem_ld32(tl + kTcColO + hh * OC + q * 32, ov);
+                tmem_ld32(tl + kTcColO + q * 32, ov);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) ov[i] *= alpha;
-                tmem_st32(tl + kTcColO + hh * OC + q * 32, ov);
+                tmem_st32(tl + kTcColO + q * 32, ov);
             }
-        }
-        {  // P into the first half of this warp's S columns (read above)
-            float pf[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) pf[i] = __uint_as_float(pk[i]);
-            tmem_st32(tl + sb * kTcKv + hh * HC, pf);
         }
         // tokens at or after the sequence end are unused cache slots (any
         // bits, NaN included): their V rows enter P.V as zeros
@@ -645,16 +626,16 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
             // can be two tiles ahead of P.V): wait for its P.V first, so that
             // the stage's wait below names its last phase or the one before
             if (j >= kTcVStages &&
-                !tc_wait_warp(&bar[kBarOReady + (j - kTcVStages) % kTcSBufs], ((j - kTcVStages) / kTcSBufs) & 1, abort)) {
+                !tc_wait_lane0(&bar[kBarOReady + (j - kTcVStages) % kTcSBufs], ((j - kTcVStages) / kTcSBufs) & 1, abort,
+                               lane)) {
                 ok = false;
                 break;
             }
-            if (!tc_wait_warp(&bar[kBarFullV + vst], (j / kTcVStages) & 1, abort)) { ok = false; break; }
+            if (!tc_wait_lane0(&bar[kBarFullV + vst], (j / kTcVStages) & 1, abort, lane)) { ok = false; break; }
             if (tt + t >= L) {
                 const uint32_t v_addr = sbase + Lay::kV + vst * Lay::kTile;
 #pragma unroll
-                for (int c = hh * (D / 16); c < (hh + 1) * (D / 16); ++c)
-                    st_shared_v4(tc_chunk(v_addr, t, c), make_uint4(0, 0, 0, 0));
+                for (int c = 0; c < D / 8; ++c) st_shared_v4(tc_chunk(v_addr, t, c), make_uint4(0, 0, 0, 0));
             }
             fence_proxy_async_smem();
         }
@@ -662,21 +643,14 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar[kBarPFull + sb]);
     }
-    // the row sum is the two halves' shares (exchanged through shared memory)
-    float *xsum = reinterpret_cast<float *>(smem + Lay::kXSum);  // [half][row]
-    xsum[hh * kTcRows + t] = l;
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&bar[kBarPairEnd + (warp & 3)]);
-    ok = ok && tc_wait_lane0(&bar[kBarPairEnd + (warp & 3)], 0, abort, lane);
-    if (ok) l += xsum[(hh ^ 1) * kTcRows + t];
-    if (ok && tc_wait_warp(&bar[kBarOReady + (n_kv - 1) % kTcSBufs], ((n_kv - 1) / kTcSBufs) & 1, abort)) {
+    if (ok && tc_wait_lane0(&bar[kBarOReady + (n_kv - 1) % kTcSBufs], ((n_kv - 1) / kTcSBufs) & 1, abort, lane)) {
         tc_fence_after();
         const float inv = valid ? 1.0f / l : 0.f;
-        __half *op = p.out + ((size_t)(q_begin + (valid ? rl : 0)) * p.num_heads + h) * D + hh * OC;
+        __half *op = p.out + ((size_t)(q_begin + (valid ? rl : 0)) * p.num_heads + h) * D;
 #pragma unroll
-        for (int q = 0; q < OC / 32; ++q) {
+        for (int q = 0; q < D / 32; ++q) {
             float ov[32];
-            tmem_ld32(tl + kTcColO + hh * OC + q * 32, ov);
+            tmem_ld32(tl + kTcColO + q * 32, ov);
             if (valid) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {

@@ -180,8 +180,7 @@ def test_broadcast_ring_model_catches_a_missing_release_count():
 # ------------------------------------------------------- tcgen05 prefill
 
 K_STAGES, V_STAGES = 3, 2
-ROW_SPLIT = 2                  # softmax warps sharing a row (halves of its S columns)
-N_SOFTMAX = 4 * ROW_SPLIT      # softmax warps: ROW_SPLIT per tensor-memory lane quadrant
+ROW_SPLIT = 1                  # softmax warps sharing a row (1: a thread owns its whole row)
 
 
 class _Bar:
@@ -199,10 +198,11 @@ class _Bar:
 S_BUFS = 3                     # S buffers in tensor memory (P of a tile overwrites its S)
 
 
-def _prefill_run(n_kv, tail, seed, p_bars=S_BUFS, o_bars=S_BUFS):
+def _prefill_run(n_kv, tail, seed, p_bars=S_BUFS, o_bars=S_BUFS, row_split=ROW_SPLIT):
     """One CTA of paged_prefill_tc_kernel: K and V producers, the MMA issuer
-    and the eight softmax warps (the two halves of a row exchange their
-    maxima every tile through shared-memory slots chosen by tile parity).
+    and the softmax warps: row_split per tensor-memory lane quadrant (with
+    more than one, the parts of a row exchange their maxima every tile
+    through shared-memory slots chosen by tile parity).
     The MMA issuer computes S one buffer ahead of need: S_0 .. S_{B-2} first,
     then per tile j, S_{j+B-1} (once its buffer is free) before P.V of j.
     P barriers are indexed by tile % p_bars, P.V-done barriers by
@@ -210,6 +210,7 @@ def _prefill_run(n_kv, tail, seed, p_bars=S_BUFS, o_bars=S_BUFS):
     rnd = random.Random(seed)
     bars = {}
     SB = S_BUFS
+    N_SOFTMAX = 4 * row_split
 
     def mk(name, count):
         bars[name] = _Bar(name, count)
@@ -230,12 +231,12 @@ def _prefill_run(n_kv, tail, seed, p_bars=S_BUFS, o_bars=S_BUFS):
         mk(f"or{b}", 1)                       # P.V of a tile of this index done
     for q in range(4):
         for par in range(2):
-            mk(f"pair{q}{par}", ROW_SPLIT)
-        mk(f"pend{q}", ROW_SPLIT)
+            mk(f"pair{q}{par}", row_split)
+        mk(f"pend{q}", row_split)
     st = {"k": [None] * K_STAGES, "v": [None] * V_STAGES, "S": [None] * SB, "Sread": [set() for _ in range(SB)],
           "pv": set(), "zeroed": set(), "P": [0] * n_kv,
           # exchange slots: [lane quadrant][tile parity][half] -> tile whose maximum it holds
-          "x": [[[None] * ROW_SPLIT for _ in range(2)] for _ in range(4)]}
+          "x": [[[None] * row_split for _ in range(2)] for _ in range(4)]}
     pending = []   # tile loads in flight: they land in any order
     mma_q = []     # MMAs of the one issuing thread: they complete in issue order
 
@@ -287,11 +288,13 @@ def _prefill_run(n_kv, tail, seed, p_bars=S_BUFS, o_bars=S_BUFS):
             yield wait(f"sf{j % SB}", j // SB)
             assert st["S"][j % SB] == j
             yield ("arrive", f"sr{j % SB}", w)
-            st["x"][q][j & 1][half] = j         # this half's maximum of tile j
-            yield ("arrive", f"pair{q}{j & 1}")
-            yield wait(f"pair{q}{j & 1}", j // 2)
-            yield ("nop",)                       # the read may lag the wait
-            assert st["x"][q][j & 1] == [j] * ROW_SPLIT, "a row maximum read before it was posted or after it was overwritten"
+            if row_split > 1:
+                st["x"][q][j & 1][half] = j         # this part's maximum of tile j
+                yield ("arrive", f"pair{q}{j & 1}")
+                yield wait(f"pair{q}{j & 1}", j // 2)
+                yield ("nop",)                       # the read may lag the wait
+                assert st["x"][q][j & 1] == [j] * row_split, \
+                    "a row maximum read before it was posted or after it was overwritten"
             if j >= 1 and rescale[j]:
                 yield wait(f"or{(j - 1) % o_bars}", (j - 1) // o_bars)
                 assert all(i in st["pv"] for i in range(j)), "O rescaled before every earlier P.V was done"
@@ -302,8 +305,9 @@ def _prefill_run(n_kv, tail, seed, p_bars=S_BUFS, o_bars=S_BUFS):
                 st["zeroed"].add((j, w))
             st["P"][j] += 1
             yield ("arrive", f"pf{j % p_bars}")
-        yield ("arrive", f"pend{q}")
-        yield wait(f"pend{q}", 0)
+        if row_split > 1:
+            yield ("arrive", f"pend{q}")
+            yield wait(f"pend{q}", 0)
         yield wait(f"or{(n_kv - 1) % o_bars}", (n_kv - 1) // o_bars)
         assert all(i in st["pv"] for i in range(n_kv)), "O read before every P.V was done"
 
@@ -395,6 +399,14 @@ def _prefill_run(n_kv, tail, seed, p_bars=S_BUFS, o_bars=S_BUFS):
 def test_prefill_protocol(n_kv, tail):
     for seed in range(150):
         _prefill_run(n_kv, tail, seed)
+
+
+@pytest.mark.parametrize("n_kv", [2, 5])
+def test_prefill_protocol_with_rows_split_over_two_warps(n_kv):
+    # the exchange of row maxima by tile parity, for a kernel that splits
+    # each row over two warps of a lane quadrant
+    for seed in range(100):
+        _prefill_run(n_kv, True, seed, row_split=2)
 
 
 @pytest.mark.parametrize("p_bars", [1, 2])
