@@ -114,7 +114,9 @@ def recorded_traffic(workload: str, record: str = "decode_dram_traffic.json", na
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle samples (200 ms) while the timed region runs."""
+    """Clock and throttle-reason samples while the timed region runs: NVML
+    read about every millisecond (queries only; nothing is set), else
+    nvidia-smi every 200 ms. Rows keep nvidia-smi's field order."""
 
     FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -124,8 +126,48 @@ class ClockSampler:
         self.gpu = gpu_index
         self.rows = []
         self.proc = None
+        self.thread = None
+        self.source = "nvidia-smi"
+        self._stop = threading.Event()
+
+    def _start_nvml(self) -> bool:
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            h = (nv.nvmlDeviceGetHandleByUUID(self.gpu) if self.gpu.startswith(("GPU-", "MIG-"))
+                 else nv.nvmlDeviceGetHandleByIndex(int(self.gpu)))
+            max_sm = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            bits = (nv.nvmlClocksThrottleReasonHwSlowdown, nv.nvmlClocksThrottleReasonHwThermalSlowdown,
+                    nv.nvmlClocksThrottleReasonSwThermalSlowdown, nv.nvmlClocksThrottleReasonSwPowerCap)
+            reasons(h)
+        except Exception:
+            return False
+
+        def loop():
+            while not self._stop.is_set():
+                try:
+                    sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                    r = reasons(h)
+                except Exception:
+                    break
+                self.rows.append((time.time(), ["", str(self.gpu), str(sm), str(max_sm), "", hex(r)] +
+                                  ["Active" if r & bit else "Not Active" for bit in bits]))
+                self._stop.wait(0.001)
+            try:
+                nv.nvmlShutdown()
+            except Exception:
+                pass
+
+        self.source = "nvml"
+        self.thread = threading.Thread(target=loop, daemon=True)
+        self.thread.start()
+        return True
 
     def start(self):
+        if self._start_nvml():
+            return
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -141,15 +183,25 @@ class ClockSampler:
             self.rows.append((time.time(), [x.strip() for x in line.split(",")]))
 
     def stop(self):
+        self._stop.set()
         if self.proc:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
 
     def summary(self, t0: float, t1: float):
-        rows = [r for t, r in self.rows if t0 - 0.25 <= t <= t1 + 0.25] or [r for _, r in self.rows]
+        # nvidia-smi's 200 ms period may put no sample inside a short timed
+        # region, so it takes a quarter second on either side; NVML samples
+        # are taken inside the region only (the nearest one if none is)
+        slack = 0.25 if self.source == "nvidia-smi" else 0.0
+        rows = [r for t, r in self.rows if t0 - slack <= t <= t1 + slack]
+        if not rows and self.rows:
+            rows = ([r for _, r in self.rows] if self.source == "nvidia-smi" else
+                    [min(self.rows, key=lambda tr: min(abs(tr[0] - t0), abs(tr[0] - t1)))[1]])
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
@@ -157,7 +209,8 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if len(r) > 6 + i and r[6 + i] == "Active"})
         return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows),
+                "source": self.source}
 
 
 # ----------------------------------------------------------------- our arm

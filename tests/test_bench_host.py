@@ -67,11 +67,30 @@ def test_clock_summary_reads_the_timed_window():
                (10.4, _smi_row(1900, 1965, ["Active"] + off[1:])),           # hw_slowdown
                (60.0, _smi_row(800, 1965, off[:1] + ["Active"] + off[2:]))]  # outside the window
     s = cs.summary(10.0, 10.4)
-    assert s == {"sm_mhz": 1932.5, "sm_max_mhz": 1965.0, "reasons": ["hw_slowdown", "sw_power_cap"], "samples": 2}
+    assert s == {"sm_mhz": 1932.5, "sm_max_mhz": 1965.0, "reasons": ["hw_slowdown", "sw_power_cap"], "samples": 2,
+                 "source": "nvidia-smi"}
     # no sample inside the window (a short run): every sample counts
     s = cs.summary(30.0, 30.1)
     assert s["samples"] == 4 and s["reasons"] == ["hw_slowdown", "hw_thermal_slowdown", "sw_power_cap"]
     assert bench.ClockSampler("0").summary(0.0, 1.0)["reasons"] == ["nvidia-smi unavailable"]
+
+
+def test_clock_summary_of_nvml_samples_keeps_to_the_timed_window():
+    # NVML rows come about every millisecond: only those inside the timed
+    # region count (idle samples before and after it would lower the median)
+    off = ["Not Active"] * 4
+    cs = bench.ClockSampler("0")
+    cs.source = "nvml"
+    cs.rows = [(9.9, _smi_row(600, 1965, off)),                       # idle, before the region
+               (10.001, _smi_row(1965, 1965, off)),
+               (10.002, _smi_row(1950, 1965, off[:3] + ["Active"])),   # sw_power_cap
+               (10.003, _smi_row(1965, 1965, off)),
+               (10.2, _smi_row(600, 1965, ["Active"] + off[1:]))]      # after the region
+    s = cs.summary(10.0, 10.0035)
+    assert s == {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3, "source": "nvml"}
+    # a region shorter than the period: the nearest sample alone
+    s = cs.summary(10.0015, 10.0016)
+    assert s["samples"] == 1 and s["sm_mhz"] == 1950.0     # the sample at 10.002
 
 
 def test_peaks_come_from_the_measured_file_else_the_fallback(tmp_path, monkeypatch):
