@@ -198,13 +198,19 @@ class _Bar:
 S_BUFS = 3                     # S buffers in tensor memory (P of a tile overwrites its S)
 
 
-def _prefill_run(n_kv, tail, seed, p_bars=S_BUFS, o_bars=S_BUFS, row_split=ROW_SPLIT):
+MMA_ISSUERS = 1               # threads issuing the MMAs (2: one for S, one for P.V)
+
+
+def _prefill_run(n_kv, tail, seed, p_bars=S_BUFS, o_bars=S_BUFS, row_split=ROW_SPLIT, issuers=MMA_ISSUERS):
     """One CTA of paged_prefill_tc_kernel: K and V producers, the MMA issuer
     and the softmax warps: row_split per tensor-memory lane quadrant (with
     more than one, the parts of a row exchange their maxima every tile
     through shared-memory slots chosen by tile parity).
-    The MMA issuer computes S one buffer ahead of need: S_0 .. S_{B-2} first,
-    then per tile j, S_{j+B-1} (once its buffer is free) before P.V of j.
+    With one MMA issuer, S is computed one buffer ahead of need: S_0 ..
+    S_{B-2} first, then per tile j, S_{j+B-1} (once its buffer is free)
+    before P.V of j. With two, one thread issues every S (each once its
+    buffer is free) and another every P.V; a thread's MMAs complete in its
+    issue order, the two threads' in any interleaving.
     P barriers are indexed by tile % p_bars, P.V-done barriers by
     tile % o_bars."""
     rnd = random.Random(seed)
@@ -238,7 +244,8 @@ def _prefill_run(n_kv, tail, seed, p_bars=S_BUFS, o_bars=S_BUFS, row_split=ROW_S
           # exchange slots: [lane quadrant][tile parity][half] -> tile whose maximum it holds
           "x": [[[None] * row_split for _ in range(2)] for _ in range(4)]}
     pending = []   # tile loads in flight: they land in any order
-    mma_q = []     # MMAs of the one issuing thread: they complete in issue order
+    mma_qs = {"s": [], "pv": []} if issuers == 2 else {"all": []}   # per issuing thread, in order
+    q_s, q_pv = (mma_qs["s"], mma_qs["pv"]) if issuers == 2 else (mma_qs["all"], mma_qs["all"])
 
     def wait(b, k):
         return ("wait", b, k)
@@ -251,33 +258,41 @@ def _prefill_run(n_kv, tail, seed, p_bars=S_BUFS, o_bars=S_BUFS, row_split=ROW_S
             pending.append((kind, j, s))
             yield ("nop",)
 
+    def issue_s(j):
+        yield wait(f"fk{j % K_STAGES}", j // K_STAGES)
+        assert st["k"][j % K_STAGES] == j
+        if j >= SB:
+            yield wait(f"sr{j % SB}", j // SB - 1)
+            yield wait(f"or{(j - SB) % o_bars}", (j - SB) // o_bars)   # P_{j-SB} in this S buffer consumed
+            assert (j - SB) in st["pv"]
+        q_s.append(("s", j))
+        yield ("nop",)
+
+    def pv(i):
+        yield wait(f"pf{i % p_bars}", i // p_bars)
+        assert st["P"][i] == N_SOFTMAX, "P.V issued before every warp wrote its part of P"
+        yield wait(f"fv{i % V_STAGES}", i // V_STAGES)
+        assert st["v"][i % V_STAGES] == i
+        q_pv.append(("pv", i))
+        yield ("nop",)
+
     def mma():
         yield wait("q", 0)
-
-        def issue_s(j):
-            yield wait(f"fk{j % K_STAGES}", j // K_STAGES)
-            assert st["k"][j % K_STAGES] == j
-            if j >= SB:
-                yield wait(f"sr{j % SB}", j // SB - 1)
-                yield wait(f"or{(j - SB) % o_bars}", (j - SB) // o_bars)   # P_{j-SB} in this S buffer consumed
-                assert (j - SB) in st["pv"]
-            mma_q.append(("s", j))
-            yield ("nop",)
-
-        def pv(i):
-            yield wait(f"pf{i % p_bars}", i // p_bars)
-            assert st["P"][i] == N_SOFTMAX, "P.V issued before every warp wrote its part of P"
-            yield wait(f"fv{i % V_STAGES}", i // V_STAGES)
-            assert st["v"][i % V_STAGES] == i
-            mma_q.append(("pv", i))
-            yield ("nop",)
-
         for j in range(min(SB - 1, n_kv)):
             yield from issue_s(j)
         for j in range(n_kv):
             if j + SB - 1 < n_kv:
                 yield from issue_s(j + SB - 1)
             yield from pv(j)
+
+    def mma_s():
+        yield wait("q", 0)
+        for j in range(n_kv):
+            yield from issue_s(j)
+
+    def mma_pv():
+        for i in range(n_kv):
+            yield from pv(i)
 
     rescale = {j: rnd.random() < 0.3 for j in range(n_kv)}
 
@@ -311,7 +326,8 @@ def _prefill_run(n_kv, tail, seed, p_bars=S_BUFS, o_bars=S_BUFS, row_split=ROW_S
         yield wait(f"or{(n_kv - 1) % o_bars}", (n_kv - 1) // o_bars)
         assert all(i in st["pv"] for i in range(n_kv)), "O read before every P.V was done"
 
-    roles = {"pk": producer("k", K_STAGES), "pv": producer("v", V_STAGES), "mma": mma(),
+    mma_roles = {"mma_s": mma_s(), "mma_pv": mma_pv()} if issuers == 2 else {"mma": mma()}
+    roles = {"pk": producer("k", K_STAGES), "pv": producer("v", V_STAGES), **mma_roles,
              **{f"w{w}": softmax(w) for w in range(N_SOFTMAX)}}
     cur = {k: None for k in roles}
     alive = set(roles)
@@ -320,16 +336,17 @@ def _prefill_run(n_kv, tail, seed, p_bars=S_BUFS, o_bars=S_BUFS, row_split=ROW_S
     # in some runs the tile loads of one kind are slow to land
     slow = rnd.choice([None, "k", "v"])
     for _ in range(400000):
-        if not alive and not pending and not mma_q:
+        heads = [q for q in mma_qs.values() if q]
+        if not alive and not pending and not heads:
             return
         progressed = False
         op = None
-        if (pending or mma_q) and rnd.random() < 0.4:
-            k = rnd.randrange(len(pending) + (1 if mma_q else 0))
+        if (pending or heads) and rnd.random() < 0.4:
+            k = rnd.randrange(len(pending) + len(heads))
             if k < len(pending) and pending[k][0] == slow and rnd.random() < 0.9:
                 k = None                       # this load stays in flight a while longer
             if k is not None:
-                op = pending.pop(k) if k < len(pending) else mma_q.pop(0)
+                op = pending.pop(k) if k < len(pending) else heads[k - len(pending)].pop(0)
         if op is not None:
             if op[0] == "k":
                 st["k"][op[2]] = op[1]
@@ -390,7 +407,7 @@ def _prefill_run(n_kv, tail, seed, p_bars=S_BUFS, o_bars=S_BUFS, row_split=ROW_S
             else:
                 cur[r] = None
                 progressed = True
-        assert progressed or pending or mma_q, f"deadlock: {cur}"
+        assert progressed or pending or any(mma_qs.values()), f"deadlock: {cur}"
     raise AssertionError("no termination")
 
 
@@ -399,6 +416,14 @@ def _prefill_run(n_kv, tail, seed, p_bars=S_BUFS, o_bars=S_BUFS, row_split=ROW_S
 def test_prefill_protocol(n_kv, tail):
     for seed in range(150):
         _prefill_run(n_kv, tail, seed)
+
+
+@pytest.mark.parametrize("n_kv", [1, 3, 7])
+def test_prefill_protocol_with_two_mma_issuers(n_kv):
+    # the same barriers with S and P.V issued by two threads, each chain
+    # completing in its own order (a variant that measured slower on B200)
+    for seed in range(100):
+        _prefill_run(n_kv, True, seed, issuers=2)
 
 
 @pytest.mark.parametrize("n_kv", [2, 5])
