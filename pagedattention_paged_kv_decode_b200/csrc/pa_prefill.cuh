@@ -277,8 +277,7 @@ enum : int {
     kBarFullV = kBarEmptyK + kTcKStages,    // + stage: V tile landed
     kBarEmptyV = kBarFullV + kTcVStages,    // + stage: P.V of the stage's tile done (commit)
     kBarSFull = kBarEmptyV + kTcVStages,    // + buffer: S ready (commit)
-    kBarSFree = kBarSFull + kTcSBufs,       // + buffer: S read by every softmax warp
-    kBarPFull = kBarSFree + kTcSBufs,       // + buffer: P written into tensor memory, O corrected (every
+    kBarPFull = kBarSFull + kTcSBufs,       // + buffer: P written into tensor memory, O corrected (every
                                             // softmax warp)
     kBarOReady = kBarPFull + kTcSBufs,      // + buffer: P.V of the buffer's tile done (commit); one
                                             // per buffer, as a warp may reach tile j before P.V of
@@ -434,8 +433,7 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
         prefetch_tensor_map(&tmap_k);
         prefetch_tensor_map(&tmap_v);
         for (int i = 0; i < kNumBars; ++i)
-            mbar_init(&bar[i], (i == kBarQ || (i >= kBarSFree && i < kBarSFree + kTcSBufs) ||
-                                (i >= kBarPFull && i < kBarPFull + kTcSBufs))
+            mbar_init(&bar[i], (i == kBarQ || (i >= kBarPFull && i < kBarPFull + kTcSBufs))
                                    ? kTcSoftmaxWarps : 1);
         *abort = 0;
         fence_mbar_init();
@@ -473,12 +471,11 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
         auto issue_s = [&](int j) -> bool {
             const int st = j % kTcKStages, b = j % kTcSBufs;
             if (!tc_wait(&bar[kBarFullK + st], (j / kTcKStages) & 1, abort)) return false;
-            if (j >= kTcSBufs) {
-                // buffer b holds S_{j-3} until every softmax warp has read it,
-                // then P_{j-3} until its P.V is done (the last P.V issued)
-                if (!tc_wait(&bar[kBarSFree + b], (j / kTcSBufs - 1) & 1, abort)) return false;
-                if (!tc_wait(&bar[kBarOReady + b], (j / kTcSBufs - 1) & 1, abort)) return false;
-            }
+            // buffer b holds S_{j-3}, then P_{j-3}, until the P.V of tile j-3
+            // is done (the last P.V issued). That P.V follows every softmax
+            // warp's P of the tile, and each warp writes its P only after its
+            // loads of S have completed, so the one wait covers both.
+            if (j >= kTcSBufs && !tc_wait(&bar[kBarOReady + b], (j / kTcSBufs - 1) & 1, abort)) return false;
             tc_fence_after();
             const uint64_t dks = dk + ((st * Lay::kTile) >> 4);
 #pragma unroll
@@ -555,9 +552,6 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
 #pragma unroll
             for (int i = 0; i < 32; ++i) sv[q * 32 + i] = v32[i];
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[kBarSFree + sb]);
 
         const int t0 = j * kTcKv;  // position of the tile's first column
         if (t0 + kTcKv > lim) {

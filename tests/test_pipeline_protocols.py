@@ -201,7 +201,11 @@ S_BUFS = 3                     # S buffers in tensor memory (P of a tile overwri
 MMA_ISSUERS = 1               # threads issuing the MMAs (2: one for S, one for P.V)
 
 
-def _prefill_run(n_kv, tail, seed, p_bars=S_BUFS, o_bars=S_BUFS, row_split=ROW_SPLIT, issuers=MMA_ISSUERS):
+S_READ_BARRIER = False        # True: the S issuer also waits for "S read by every softmax warp"
+
+
+def _prefill_run(n_kv, tail, seed, p_bars=S_BUFS, o_bars=S_BUFS, row_split=ROW_SPLIT, issuers=MMA_ISSUERS,
+                 s_read_barrier=S_READ_BARRIER, skip_pv_wait=False, release_barriers=True):
     """One CTA of paged_prefill_tc_kernel: K and V producers, the MMA issuer
     and the softmax warps: row_split per tensor-memory lane quadrant (with
     more than one, the parts of a row exchange their maxima every tile
@@ -212,7 +216,14 @@ def _prefill_run(n_kv, tail, seed, p_bars=S_BUFS, o_bars=S_BUFS, row_split=ROW_S
     buffer is free) and another every P.V; a thread's MMAs complete in its
     issue order, the two threads' in any interleaving.
     P barriers are indexed by tile % p_bars, P.V-done barriers by
-    tile % o_bars."""
+    tile % o_bars. Without s_read_barrier, an S buffer is reused on the P.V
+    of its previous tile alone (that P.V follows every warp's P, which each
+    warp writes after reading S). skip_pv_wait plants a mistake: S reuses a
+    buffer without waiting for that P.V. Without release_barriers the
+    producers reuse a K stage on "S ready" of its previous tile (K stages
+    and S buffers are both three) and a V stage on "P.V done" of its
+    previous tile, instead of barriers of their own (a variant that measured
+    slower on B200; the kernel has release barriers)."""
     rnd = random.Random(seed)
     bars = {}
     SB = S_BUFS
@@ -254,7 +265,13 @@ def _prefill_run(n_kv, tail, seed, p_bars=S_BUFS, o_bars=S_BUFS, row_split=ROW_S
         for j in range(n_kv):
             s, use = j % stages, j // stages
             if use > 0:
-                yield wait(f"e{kind}{s}", use - 1)
+                if release_barriers:
+                    yield wait(f"e{kind}{s}", use - 1)
+                elif kind == "k":
+                    assert stages == SB
+                    yield wait(f"sf{s}", use - 1)                                   # S of tile j-3 done
+                else:
+                    yield wait(f"or{(j - stages) % o_bars}", (j - stages) // o_bars)  # P.V of tile j-2 done
             pending.append((kind, j, s))
             yield ("nop",)
 
@@ -262,9 +279,11 @@ def _prefill_run(n_kv, tail, seed, p_bars=S_BUFS, o_bars=S_BUFS, row_split=ROW_S
         yield wait(f"fk{j % K_STAGES}", j // K_STAGES)
         assert st["k"][j % K_STAGES] == j
         if j >= SB:
-            yield wait(f"sr{j % SB}", j // SB - 1)
-            yield wait(f"or{(j - SB) % o_bars}", (j - SB) // o_bars)   # P_{j-SB} in this S buffer consumed
-            assert (j - SB) in st["pv"]
+            if s_read_barrier:
+                yield wait(f"sr{j % SB}", j // SB - 1)
+            if not skip_pv_wait:
+                yield wait(f"or{(j - SB) % o_bars}", (j - SB) // o_bars)   # P_{j-SB} in this S buffer consumed
+                assert (j - SB) in st["pv"]
         q_s.append(("s", j))
         yield ("nop",)
 
@@ -302,7 +321,11 @@ def _prefill_run(n_kv, tail, seed, p_bars=S_BUFS, o_bars=S_BUFS, row_split=ROW_S
         for j in range(n_kv):
             yield wait(f"sf{j % SB}", j // SB)
             assert st["S"][j % SB] == j
-            yield ("arrive", f"sr{j % SB}", w)
+            if s_read_barrier:
+                yield ("arrive", f"sr{j % SB}", w)
+            else:
+                st["Sread"][j % SB].add(w)           # the read completes before this warp's P
+                yield ("nop",)
             if row_split > 1:
                 st["x"][q][j & 1][half] = j         # this part's maximum of tile j
                 yield ("arrive", f"pair{q}{j & 1}")
@@ -418,6 +441,12 @@ def test_prefill_protocol(n_kv, tail):
         _prefill_run(n_kv, tail, seed)
 
 
+@pytest.mark.parametrize("n_kv", [2, 7])
+def test_prefill_protocol_with_stages_released_by_s_and_pv_barriers(n_kv):
+    for seed in range(100):
+        _prefill_run(n_kv, True, seed, release_barriers=False)
+
+
 @pytest.mark.parametrize("n_kv", [1, 3, 7])
 def test_prefill_protocol_with_two_mma_issuers(n_kv):
     # the same barriers with S and P.V issued by two threads, each chain
@@ -458,6 +487,21 @@ def test_prefill_protocol_catches_one_pv_barrier_for_all_buffers():
     for seed in range(100):
         try:
             _prefill_run(5, False, seed, o_bars=1)
+        except AssertionError:
+            failures += 1
+    assert failures > 0
+
+
+def test_prefill_protocol_catches_s_reuse_without_the_pv_wait():
+    # without the "S read" barrier the P.V-done wait is what keeps S_{j+3}
+    # off a buffer still being read or holding P_j: dropping it must fail.
+    # (With one issuer the model's in-order completion would hide the
+    # mistake; the kernel does not rely on that order between different
+    # MMAs, so the check runs with S and P.V on two issuers.)
+    failures = 0
+    for seed in range(100):
+        try:
+            _prefill_run(6, False, seed, skip_pv_wait=True, issuers=2)
         except AssertionError:
             failures += 1
     assert failures > 0
