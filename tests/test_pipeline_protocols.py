@@ -505,3 +505,4 @@ def test_prefill_protocol_catches_s_reuse_without_the_pv_wait():
         except AssertionError:
             failures += 1
     assert failures > 0
+
