@@ -332,18 +332,18 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
 // One producer warp: streams the K (or V) tiles 0 .. n_kv-1 of the CTA
 // through its ring. Lane b < BPT loads cache block b of each tile; lane l
 // holds block-table entry 32c + l of the current chunk c while the next
-// chunk's entries are already being read.
+// chunk's entries are already being read (the first two chunks, cur and
+// nxt, are read by the caller before the CTA's set-up).
 template <int D, int B, int STAGES>
 __device__ __forceinline__ void tc_produce(const CUtensorMap *tmap, unsigned char *ring, uint64_t *full,
                                            uint64_t *empty, const int32_t *table, int nblk, int n_kv, int h,
-                                           int num_blocks, volatile int *abort, int lane) {
+                                           int num_blocks, volatile int *abort, int lane, int cur, int nxt) {
     constexpr int BPT = kTcKv / B;
     const uint64_t policy = l2_policy_evict_normal();  // other row tiles re-read these blocks
     auto fetch = [&](int chunk) {
         const int lb = chunk * 32 + lane;
         return lb < nblk ? __ldg(table + lb) : -1;
     };
-    int cur = fetch(0), nxt = fetch(1);
     int issued = 0;
     for (int j = 0; j < n_kv; ++j) {
         const int st = j % STAGES, use = j / STAGES;
@@ -424,6 +424,23 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
     const int n_kv = (kv_end + kTcKv - 1) / kTcKv;
     const int32_t *table = p.block_tables + (size_t)s * p.max_blocks_per_seq;
 
+    // ---- reads that depend on nothing set up below go out first: the
+    // producers' first 64 block-table entries and each softmax thread's Q row
+    int tab0 = -1, tab1 = -1;
+    if (warp == kTcWarpK || warp == kTcWarpV) {
+        tab0 = lane < nblk ? __ldg(table + lane) : -1;
+        tab1 = 32 + lane < nblk ? __ldg(table + 32 + lane) : -1;
+    }
+    const int t = warp * 32 + lane;  // softmax warps: row of the tile = tensor-memory lane
+    const int rl = r0 + t;
+    const bool valid = warp < kTcSoftmaxWarps && rl < n;
+    uint4 q_row[D / 8];
+    if (warp < kTcSoftmaxWarps) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.query + ((size_t)(q_begin + (valid ? rl : 0)) * p.num_heads + h) * D);
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) q_row[c] = valid ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+    }
+
     // ---- set-up: tensor memory, barriers
     if (warp == kTcWarpMma) {
         tmem_alloc(tmem_slot, kTcTmemCols);
@@ -445,12 +462,12 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
 
     if (warp == kTcWarpK) {
         tc_produce<D, B, kTcKStages>(&tmap_k, smem + Lay::kK, &bar[kBarFullK], &bar[kBarEmptyK], table, nblk, n_kv, h,
-                                  p.num_blocks, abort, lane);
+                                  p.num_blocks, abort, lane, tab0, tab1);
         return;
     }
     if (warp == kTcWarpV) {
         tc_produce<D, B, kTcVStages>(&tmap_v, smem + Lay::kV, &bar[kBarFullV], &bar[kBarEmptyV], table, nblk, n_kv, h,
-                                  p.num_blocks, abort, lane);
+                                  p.num_blocks, abort, lane, tab0, tab1);
         return;
     }
 
@@ -521,17 +538,10 @@ paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid
     }
 
     // -------------------------------------------------------------- softmax
-    const int t = warp * 32 + lane;  // row of the tile = tensor-memory lane
-    const int rl = r0 + t;
-    const bool valid = rl < n;
     const int lim = valid ? base + rl + 1 : 0;  // tokens 0 .. lim-1 are visible
     {
-        const uint4 *src = reinterpret_cast<const uint4 *>(p.query + ((size_t)(q_begin + (valid ? rl : 0)) * p.num_heads + h) * D);
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c) {  // the row's 16-byte chunks
-            const uint4 v = valid ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
-            st_shared_v4(tc_chunk(sbase + Lay::kQ, t, c), v);
-        }
+        for (int c = 0; c < D / 8; ++c) st_shared_v4(tc_chunk(sbase + Lay::kQ, t, c), q_row[c]);  // the row's 16-byte chunks
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar[kBarQ]);
