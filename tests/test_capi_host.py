@@ -331,3 +331,30 @@ def test_ctypes_structs_match_the_header():
         assert [n for _, n in fields] == [n for n, _ in cls._fields_], cname
         assert all(t == "int32_t" for t, _ in fields) and all(ty is ctypes.c_int32 for _, ty in cls._fields_)
         assert ctypes.sizeof(cls) == 4 * len(fields)
+
+
+def _partials_bytes(S, H, D, parts):
+    lse = (S * H * parts * 4 + 255) // 256 * 256
+    return lse + S * H * parts * D * 4
+
+
+def test_shared_prefix_suffix_shape_counts_the_prefix_kernel():
+    # 32 sequences x 32 heads, head_size 128, 32-token blocks, a 96-block
+    # (3072-token) shared prefix under a 4096-token bound: the prefix kernel
+    # runs 32 heads x 12 partitions of 256 tokens = 384 CTAs beside the
+    # decode of the private parts. Counting them, the private parts' grid
+    # (2 heads per CTA: 512 units with 1024-token partitions) plus the prefix
+    # grid reaches 4 CTAs per SM, so the suffix takes one 1024-token partition:
+    # 12 + 1 partials per (sequence, head). Without the prefix kernel's CTAs the
+    # rule would have split the suffix in two (12 + 2).
+    L = capi.lib()
+    desc = capi.CacheDesc(4096, 32, 32, 128, capi.PA_F16)
+    got = L.pa_shared_prefix_workspace_size(desc, 32, 4096, 96, None)
+    assert got == _partials_bytes(32, 32, 128, 12 + 1)
+    # an explicit 512-token suffix partition gives the two-partition layout
+    cfg = capi.DecodeConfig(512, 0, 0, 0, 0)
+    assert L.pa_shared_prefix_workspace_size(desc, 32, 4096, 96, ctypes.byref(cfg)) == \
+        _partials_bytes(32, 32, 128, 12 + 2)
+    # a small batch (8 sequences) stays at two heads per CTA and 512-token partitions:
+    # 8 x 16 x 2 = 256 units + 384 prefix CTAs are below 4 per SM at 1024 tokens
+    assert L.pa_shared_prefix_workspace_size(desc, 8, 4096, 96, None) == _partials_bytes(8, 32, 128, 12 + 2)
